@@ -1,0 +1,190 @@
+/*
+ * mobi.h — C ABI of libmobi: the token-routed mixed-bit linear layer of
+ * MoBiQuant on NVIDIA B200 (sm_100a).
+ *
+ * Sources (the two explainer pages of "MoBiQuant: Mixture-of-Bits Quantization
+ * for Token-Adaptive Elastic LLMs"):
+ *   [ja]  gist.science/ja/paper/2602.20191 — §2.1 MoBiSlice, §2.2 MoBiRoute
+ *   [en]  gist.science/paper/2602.20191 — §2.A MoBiSlice, §2.B MoBiRoute,
+ *         §3 Key Contributions (specialised kernels)
+ *
+ * The layer has three steps and one entry point per step:
+ *   mobi_pack   MoBiSlice: W[N,K] -> S residual slices of 2-bit codes with a
+ *               per-(slice,row,group) fp16 scale and fp16 zero.
+ *               [ja] §2.1 (R_1 = W, W_e = Q(R_e), R_{e+1} = R_e - W_e);
+ *               [en] §2.A "Recursive Decomposition" / "Process".
+ *   mobi_route  MoBiRoute: k_t = 1 + argmax_j (x_t . Wr[:,j] + b_j), then a
+ *               stable bucketing of the tokens by k_t.
+ *               [ja] §2.2; [en] §2.B "Routing Mechanism", "Dynamic Adjustment".
+ *   mobi_gemm   y_t = x_t . (sum_{s <= k_t} deq(slice_s))^T, fp32 accumulation.
+ *               [ja] §2.1 (W^(b) = sum W_e); [en] §2.A "Elasticity".
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is a DEVICE pointer (allocated by the caller, e.g.
+ *     through PyTorch), unless stated otherwise. The library never allocates or
+ *     frees device memory; all scratch memory comes from the caller's `ws`.
+ *   - Every pointer must be 16-byte aligned (128-bit vector accesses).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls enqueue work and return without synchronising.
+ *   - Arguments are validated on the host before anything is launched; on an
+ *     error nothing is enqueued and the status says why.
+ *   - Supported shapes: S in {1,2,3} slices of b = 2 bits, group G = 128 along
+ *     K, K % 128 == 0, N % 16 == 0, T >= 0. K, N, T up to 2^30 elements per
+ *     dimension and N*K, T*K, T*N below 2^40.
+ *   - A device-side bounded wait that runs out sets a per-device error word;
+ *     the next call on that device (or mobi_sync_check) reports
+ *     MOBI_ERR_TIMEOUT and clears it.
+ *   - The library keeps no per-call host state and is reentrant.
+ *
+ * Packed format (one checkpoint serves every precision: [ja] §3 "Many-in-One";
+ * [en] §3 "MoBiSlice Architecture"). Slices are stored one after another, so a
+ * token that needs k slices reads only the first k slices' bytes ([en] §3:
+ * bit-major packing avoids the all-or-nothing fetch).
+ *
+ *   codes  uint32 [S][N][K/16]   word w of (slice s, row n) holds the codes of
+ *          k = 16w .. 16w+15; code q(s,n,16w+i) sits in bits [2i+1 : 2i]
+ *          (little-endian 2-bit fields). mobi_codes_bytes() gives the size.
+ *   sz     uint32 [S][N][K/G]    element (s,n,g): bits [15:0] = fp16 scale,
+ *          bits [31:16] = fp16 zero (an integer 0..3). mobi_sz_bytes().
+ *   The dequantised slice is deq_s[n,k] = (q(s,n,k) - zero(s,n,k/G)) *
+ *   scale(s,n,k/G), and the k-slice weight is W^(k) = sum_{s<k} deq_s.
+ *
+ * Quantiser (the pages name Q(.) but do not define it; this is the reading
+ * the library implements, in IEEE fp32 with round-to-nearest-even):
+ *   for each (row n, group g):  R <- (float)W[n, group g]
+ *   for s = 0..S-1:
+ *     mn = min R, mx = max R
+ *     sc = max((mx - mn) / 3, 2^-14);  scale = fp16_rne(sc);  s = (float)scale
+ *     z  = clamp(rint(-mn / s), 0, 3)
+ *     q  = clamp(rint(R / s) + z, 0, 3)          (per element)
+ *     R  = R - (q - z) * s                      (the product is exact)
+ */
+#ifndef MOBI_H_
+#define MOBI_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOBI_OK = 0,
+  MOBI_ERR_INVALID_ARG = 1,       /* null pointer, negative size, S/G out of range */
+  MOBI_ERR_UNSUPPORTED_SHAPE = 2, /* K % 128, N % 16, or sizes beyond the limits */
+  MOBI_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
+  MOBI_ERR_WORKSPACE = 4,         /* ws == NULL or ws_bytes below the required size */
+  MOBI_ERR_CUDA = 5,              /* a CUDA launch or query failed (error cleared) */
+  MOBI_ERR_TIMEOUT = 6            /* a device-side bounded wait ran out */
+} mobi_status;
+
+/* Human-readable name of a status (static storage, never NULL). */
+const char* mobi_status_string(mobi_status st);
+
+/* Library version as an integer MAJOR*10000 + MINOR*100 + PATCH. */
+int mobi_version(void);
+
+/* Bytes of the packed code array for S slices of an N x K matrix:
+ * S * N * (K/16) * 4. Returns 0 for invalid sizes. */
+size_t mobi_codes_bytes(int64_t N, int64_t K, int S);
+
+/* Bytes of the scale/zero array: S * N * (K/G) * 4. Returns 0 for invalid sizes. */
+size_t mobi_sz_bytes(int64_t N, int64_t K, int S, int G);
+
+/* Scratch bytes that mobi_route needs for T tokens (may be 0). */
+size_t mobi_route_workspace_bytes(int64_t T, int64_t K, int S);
+
+/* Scratch bytes that mobi_gemm needs (covers both the decode and the prefill
+ * kernels, so one buffer serves every T up to the given one). */
+size_t mobi_gemm_workspace_bytes(int64_t T, int64_t N, int64_t K, int S);
+
+/*
+ * mobi_pack — MoBiSlice recursive residual quantisation of W.
+ *   [ja] §2.1, [en] §2.A; quantiser as stated at the top of this header.
+ *   W        fp16 [N][K] row-major (device). Values must be finite.
+ *   N, K     rows and columns; K % G == 0, N % 16 == 0.
+ *   G        group size along K; must be 128.
+ *   S        number of slices, 1..3.
+ *   codes    out, uint32 [S][N][K/16] (layout above).
+ *   sz       out, uint32 [S][N][K/G]  (fp16 scale | fp16 zero << 16).
+ * Bit-exact with the quantiser above (IEEE division, RNE, no flush-to-zero).
+ */
+mobi_status mobi_pack(const void* W, int64_t N, int64_t K, int G, int S,
+                      uint32_t* codes, uint32_t* sz, void* stream);
+
+/*
+ * mobi_route — MoBiRoute slice count per token and token bucketing.
+ *   [ja] §2.2 (a router scores each token; the score fixes how many residual
+ *   slices are active); [en] §2.B. The router here is linear:
+ *   logit_j(t) = sum_k x[t,k] * Wr[k,j] + bias[j] (fp32 values; the kernel
+ *   accumulates in fp32 chunks and fp64 across chunks), and
+ *   k_t = 1 + argmax_j logit_j(t), the lowest j winning an exact tie.
+ *   X        bf16 [T][K] row-major.
+ *   Wr       fp32 [K][S] row-major.  bias  fp32 [S], or NULL for zeros.
+ *   k_t      out, int32 [T], values 1..S.
+ *   perm     out, int32 [T]: tokens sorted by k_t ascending, stable
+ *            (ties keep the original order); perm[i] = original index.
+ *   offsets  out, int32 [S+1]: tokens with k_t = j+1 are
+ *            perm[offsets[j] .. offsets[j+1]); offsets[0] = 0, offsets[S] = T.
+ *   ws       scratch of mobi_route_workspace_bytes(T, K, S) bytes (may be
+ *            NULL when that size is 0).
+ */
+mobi_status mobi_route(const void* X, int64_t T, int64_t K, const float* Wr,
+                       const float* bias, int S, int32_t* k_t, int32_t* perm,
+                       int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * mobi_gemm — token-routed mixed-bit GEMM.
+ *   y[t,n] = sum_k x[t,k] * W^(k_t)[n,k],  W^(k) = sum_{s<k} deq_s,
+ *   [ja] §2.1 (W^(b) = sum W_e), [en] §2.A "Elasticity". fp32 accumulation of
+ *   exact products: the codes enter the tensor cores as exact small integers
+ *   and each slice's fp16 scale is applied in fp32 once per 128-wide group.
+ *   X        bf16 [T][K]; k_t, perm, offsets as produced by mobi_route
+ *            (k_t values 1..S; perm a permutation sorted by k_t).
+ *   codes, sz as produced by mobi_pack for the same N, K, G and >= S slices.
+ *   Y        out, fp32 [T][N], original token order.
+ *   ws       scratch of mobi_gemm_workspace_bytes(T, N, K, S) bytes.
+ * T <= 16 runs the decode kernel (streams only the slices up to the batch's
+ * largest k_t), larger T the tcgen05 prefill kernel.
+ */
+mobi_status mobi_gemm(const void* X, int64_t T, int64_t K, const int32_t* k_t,
+                      const int32_t* perm, const int32_t* offsets,
+                      const uint32_t* codes, const uint32_t* sz, int64_t N, int G,
+                      int S, float* Y, void* ws, size_t ws_bytes, void* stream);
+
+/* Kernel selection for mobi_gemm_path. */
+typedef enum {
+  MOBI_PATH_AUTO = 0,    /* decode for T <= 16, prefill otherwise */
+  MOBI_PATH_DECODE = 1,  /* decode kernel; requires T <= 16 */
+  MOBI_PATH_PREFILL = 2  /* tcgen05 prefill kernel, any T */
+} mobi_path;
+
+/* mobi_gemm with an explicit kernel choice (same arguments and result). */
+mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const int32_t* k_t,
+                           const int32_t* perm, const int32_t* offsets,
+                           const uint32_t* codes, const uint32_t* sz, int64_t N,
+                           int G, int S, float* Y, void* ws, size_t ws_bytes,
+                           void* stream, int path);
+
+/*
+ * mobi_sync_check — synchronise `stream`, then report and clear the
+ * device-side error word of the current device. Returns MOBI_ERR_TIMEOUT if a
+ * bounded wait ran out since the last check, MOBI_ERR_CUDA on a CUDA error.
+ */
+mobi_status mobi_sync_check(void* stream);
+
+/*
+ * mobi_debug_set_wait_limit — set the iteration limit of the device-side
+ * bounded waits of the current device (0 restores the default). A tiny limit
+ * makes the prefill kernel's waits run out, which exercises the timeout path
+ * without faulting anything: the kernel records the error, drains its own
+ * copies in flight, frees its tensor memory and returns. Test use only.
+ */
+mobi_status mobi_debug_set_wait_limit(int64_t limit);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOBI_H_ */

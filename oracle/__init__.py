@@ -1,0 +1,157 @@
+"""CPU oracle of the MoBiQuant token-routed mixed-bit linear layer.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke()``
+and by the CPU-baseline leg of ``bench.py``; never by the product package.
+
+The arithmetic lives in ``mobi_oracle.c`` (plain C, fp32 quantiser, fp64
+routing and GEMM); this module compiles it with gcc on first use and wraps it
+with numpy arrays. See the C file's header for the sources it follows
+(the MoBiQuant explainer pages, §2.1/§2.A MoBiSlice and §2.2/§2.B MoBiRoute)
+and for the readings taken where the pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mobi_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+# -ffp-contract=off: no fused multiply-add, so every fp32 operation of the
+# quantiser rounds exactly once, as IEEE arithmetic written out.
+CFLAGS = ["-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-std=c11"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/_build/liboracle.so`` (if stale) and return its path."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            p = ctypes.c_void_p
+            i64 = ctypes.c_int64
+            ci = ctypes.c_int
+            lib.oracle_pack.argtypes = [p, i64, i64, ci, ci, p, p, p, ci]
+            lib.oracle_pack.restype = ci
+            lib.oracle_unpack.argtypes = [p, i64, i64, ci, p]
+            lib.oracle_unpack.restype = None
+            lib.oracle_reconstruct.argtypes = [p, p, i64, i64, ci, ci, ci, p]
+            lib.oracle_reconstruct.restype = None
+            lib.oracle_route.argtypes = [p, i64, i64, p, p, ci, p, p, p, ci]
+            lib.oracle_route.restype = None
+            lib.oracle_bucket.argtypes = [p, i64, ci, p, p]
+            lib.oracle_bucket.restype = ci
+            lib.oracle_gemm.argtypes = [p, i64, i64, p, p, p, i64, ci, ci, p, i64, p, ci]
+            lib.oracle_gemm.restype = None
+            lib.oracle_max_threads.argtypes = []
+            lib.oracle_max_threads.restype = ci
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a) -> np.ndarray:
+    """fp16 / bf16 arrays (numpy, or CPU torch tensors) travel as their uint16 bit patterns."""
+    if hasattr(a, "element_size") and hasattr(a, "view"):  # a torch tensor
+        import torch
+        a = a.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    a = np.ascontiguousarray(a)
+    return a.view(np.uint16) if a.dtype != np.uint16 else a
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def pack(W_f16: np.ndarray, G: int = 128, S: int = 3, nthreads: int = 0):
+    """MoBiSlice packing. Returns (codes uint32 [S,N,K/16], sz uint32 [S,N,K/G], q uint8 [S,N,K])."""
+    lib = _load()
+    W = _u16(W_f16)
+    N, K = W.shape
+    codes = np.zeros((S, N, K // 16), np.uint32)
+    sz = np.zeros((S, N, K // G), np.uint32)
+    q = np.zeros((S, N, K), np.uint8)
+    rc = lib.oracle_pack(_ptr(W), N, K, G, S, _ptr(codes), _ptr(sz), _ptr(q), nthreads)
+    if rc != 0:
+        raise ValueError("oracle_pack: unsupported arguments")
+    return codes, sz, q
+
+
+def unpack(codes: np.ndarray, N: int, K: int, S: int) -> np.ndarray:
+    """Packed words -> codes uint8 [S,N,K] by the documented layout."""
+    lib = _load()
+    codes = np.ascontiguousarray(codes, np.uint32)
+    q = np.zeros((S, N, K), np.uint8)
+    lib.oracle_unpack(_ptr(codes), N, K, S, _ptr(q))
+    return q
+
+
+def reconstruct(codes: np.ndarray, sz: np.ndarray, N: int, K: int, k: int, G: int = 128, S: int = 3) -> np.ndarray:
+    """W^(k) = sum of the first k dequantised slices, fp64 [N,K]."""
+    lib = _load()
+    out = np.zeros((N, K), np.float64)
+    lib.oracle_reconstruct(_ptr(np.ascontiguousarray(codes, np.uint32)), _ptr(np.ascontiguousarray(sz, np.uint32)),
+                           N, K, G, S, k, _ptr(out))
+    return out
+
+
+def route(X_bf16: np.ndarray, Wr: np.ndarray, bias: np.ndarray | None = None, nthreads: int = 0):
+    """Returns (k_t int32 [T], gap fp64 [T], logits fp64 [T,S])."""
+    lib = _load()
+    X = _u16(X_bf16)
+    T, K = X.shape
+    Wr = np.ascontiguousarray(Wr, np.float32)
+    S = Wr.shape[1]
+    b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    k = np.zeros(T, np.int32)
+    gap = np.zeros(T, np.float64)
+    logits = np.zeros((T, S), np.float64)
+    lib.oracle_route(_ptr(X), T, K, _ptr(Wr), _ptr(b), S, _ptr(k), _ptr(gap), _ptr(logits), nthreads)
+    return k, gap, logits
+
+
+def bucket(k_t: np.ndarray, S: int = 3):
+    """Returns (perm int32 [T], offsets int32 [S+1])."""
+    lib = _load()
+    k_t = np.ascontiguousarray(k_t, np.int32)
+    T = k_t.shape[0]
+    perm = np.zeros(T, np.int32)
+    offsets = np.zeros(S + 1, np.int32)
+    if lib.oracle_bucket(_ptr(k_t), T, S, _ptr(perm), _ptr(offsets)) != 0:
+        raise ValueError("oracle_bucket: k_t outside 1..S")
+    return perm, offsets
+
+
+def gemm(X_bf16: np.ndarray, k_t: np.ndarray, codes: np.ndarray, sz: np.ndarray, N: int,
+         G: int = 128, S: int = 3, tokens: np.ndarray | None = None, nthreads: int = 0) -> np.ndarray:
+    """Y fp64 [len(tokens) or T, N] = x_t . W^(k_t)^T for the listed tokens."""
+    lib = _load()
+    X = _u16(X_bf16)
+    T, K = X.shape
+    k_t = np.ascontiguousarray(k_t, np.int32)
+    tok = None if tokens is None else np.ascontiguousarray(tokens, np.int32)
+    n_tok = T if tok is None else tok.shape[0]
+    Y = np.zeros((n_tok, N), np.float64)
+    lib.oracle_gemm(_ptr(X), T, K, _ptr(k_t), _ptr(np.ascontiguousarray(codes, np.uint32)),
+                    _ptr(np.ascontiguousarray(sz, np.uint32)), N, G, S, _ptr(tok), n_tok, _ptr(Y), nthreads)
+    return Y

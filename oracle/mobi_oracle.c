@@ -1,0 +1,292 @@
+/*
+ * mobi_oracle.c — TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT.
+ *
+ * A plain, slow, obviously correct CPU implementation of the MoBiQuant
+ * token-routed mixed-bit linear layer, used only by the tests, by the smoke
+ * check and by the benchmark's CPU-baseline leg. The CUDA library never links,
+ * loads or calls this file, and this file shares no code with it.
+ *
+ * Sources (explainer pages of "MoBiQuant: Mixture-of-Bits Quantization for
+ * Token-Adaptive Elastic LLMs"):
+ *   [ja] gist.science/ja/paper/2602.20191 — §2.1 MoBiSlice (recursive residual
+ *        quantisation R_1 = W, W_e = Q(R_e), R_{e+1} = R_e - W_e; W^(b) = sum W_e),
+ *        §2.2 MoBiRoute (per-token score decides how many residual slices are
+ *        active).
+ *   [en] gist.science/paper/2602.20191 — §2.A MoBiSlice ("Recursive
+ *        Decomposition", "Process", "Elasticity": a 6-bit weight is the 2-bit
+ *        base plus two 2-bit residuals), §2.B MoBiRoute ("Routing Mechanism",
+ *        "Dynamic Adjustment").
+ *
+ * Precision: the quantiser runs in IEEE fp32 with round-to-nearest-even
+ * (compiled with -ffp-contract=off, no fast-math); routing logits and the GEMM
+ * run in fp64 on exact operands.
+ *
+ * Readings where the pages are silent (the quantiser Q is named, not defined):
+ *   asymmetric min-max round-to-nearest over groups of G = 128 along K, with an
+ *   integer zero-point z = clamp(rint(-min/s), 0, 3), the scale s = (max-min)/3
+ *   floored at 2^-14 and rounded to fp16 BEFORE it is used, deq = (q - z) * s,
+ *   and the reconstruction W^(k) = sum_{s<k} deq_s kept exact (no rounding to
+ *   a 16-bit type). Routing: a linear router, k_t = 1 + argmax (lowest index on
+ *   an exact tie). Bucketing: stable ascending sort by k_t.
+ *
+ * Parity pins: every function here is pinned by tests/test_oracle.py against
+ * closed-form groups, hand-derived packed words, invariants (non-increasing
+ * reconstruction error, half-step rounding bound), brute force (numpy fp64
+ * matmul on tiny shapes, one-hot inputs) and special cases; see that file.
+ * Whether the quantiser reading matches the MoBiQuant authors' own Q cannot be
+ * pinned from the pages ("parity unpinned" for that reading, not for the code).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ---- scalar conversions (IEEE, round-to-nearest-even) ------------------- */
+
+static float half_bits_to_float(uint16_t h) {
+  _Float16 v;
+  memcpy(&v, &h, sizeof v);
+  return (float)v;
+}
+
+static uint16_t float_to_half_bits(float f) {
+  _Float16 v = (_Float16)f; /* IEEE conversion, round to nearest even */
+  uint16_t h;
+  memcpy(&h, &v, sizeof h);
+  return h;
+}
+
+static double bf16_bits_to_double(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+static void set_threads(int nthreads) {
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+}
+
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* ---- MoBiSlice ---------------------------------------------------------- */
+
+/*
+ * One group of G weights of one row through S rounds of the recursion
+ * R_1 = W, W_s = Q(R_s), R_{s+1} = R_s - W_s   ([ja] §2.1, [en] §2.A).
+ * q_out[s*G + i] receives the code of element i in slice s; scale_out[s] and
+ * zero_out[s] the fp16 bit patterns of that slice's scale and zero.
+ */
+static void quantise_group(const uint16_t* w, int G, int S, uint8_t* q_out,
+                           uint16_t* scale_out, uint16_t* zero_out) {
+  float R[1024];
+  for (int i = 0; i < G; ++i) R[i] = half_bits_to_float(w[i]);
+  for (int s = 0; s < S; ++s) {
+    float mn = R[0], mx = R[0];
+    for (int i = 1; i < G; ++i) {
+      if (R[i] < mn) mn = R[i];
+      if (R[i] > mx) mx = R[i];
+    }
+    float sc = (mx - mn) / 3.0f;           /* 2 bits: 4 levels, 3 steps */
+    if (sc < 0x1p-14f) sc = 0x1p-14f;      /* degenerate group: smallest normal fp16 */
+    uint16_t scale_bits = float_to_half_bits(sc);
+    float step = half_bits_to_float(scale_bits); /* the stored scale is the one used */
+    float zf = rintf(-mn / step);
+    if (zf < 0.0f) zf = 0.0f;
+    if (zf > 3.0f) zf = 3.0f;
+    int z = (int)zf;
+    for (int i = 0; i < G; ++i) {
+      float qf = rintf(R[i] / step) + (float)z;
+      if (qf < 0.0f) qf = 0.0f;
+      if (qf > 3.0f) qf = 3.0f;
+      int q = (int)qf;
+      q_out[s * G + i] = (uint8_t)q;
+      float deq = (float)(q - z) * step; /* exact: |q-z| <= 3 times an fp16 */
+      R[i] = R[i] - deq;                 /* the residual of the next round */
+    }
+    scale_out[s] = scale_bits;
+    zero_out[s] = float_to_half_bits((float)z);
+  }
+}
+
+/*
+ * oracle_pack: W fp16 [N][K] -> codes (the documented 2-bit word layout:
+ * word (s, n, w) holds q(s, n, 16w + i) in bits [2i+1:2i]) and sz
+ * (fp16 scale in bits [15:0], fp16 zero in bits [31:16]), plus, if q_out is
+ * not NULL, the unpacked codes uint8 [S][N][K].
+ * Returns 0, or -1 on an unsupported argument.
+ */
+int oracle_pack(const uint16_t* W, int64_t N, int64_t K, int G, int S,
+                uint32_t* codes, uint32_t* sz, uint8_t* q_out, int nthreads) {
+  if (G <= 0 || G > 1024 || K % G != 0 || K % 16 != 0 || S < 1 || S > 8) return -1;
+  set_threads(nthreads);
+  const int64_t ngroups = K / G;
+  const int64_t nwords = K / 16;
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t n = 0; n < N; ++n) {
+    uint8_t q[8 * 1024];
+    uint16_t sc[8], zr[8];
+    uint8_t* row_codes = (uint8_t*)malloc((size_t)S * (size_t)K);
+    for (int64_t g = 0; g < ngroups; ++g) {
+      quantise_group(W + n * K + g * G, G, S, q, sc, zr);
+      for (int s = 0; s < S; ++s) {
+        sz[((int64_t)s * N + n) * ngroups + g] = (uint32_t)sc[s] | ((uint32_t)zr[s] << 16);
+        for (int i = 0; i < G; ++i) row_codes[(int64_t)s * K + g * G + i] = q[s * G + i];
+      }
+    }
+    for (int s = 0; s < S; ++s) {
+      for (int64_t w = 0; w < nwords; ++w) {
+        uint32_t word = 0;
+        for (int i = 0; i < 16; ++i)
+          word |= (uint32_t)row_codes[(int64_t)s * K + 16 * w + i] << (2 * i);
+        codes[((int64_t)s * N + n) * nwords + w] = word;
+      }
+      if (q_out)
+        memcpy(q_out + ((int64_t)s * N + n) * K, row_codes + (int64_t)s * K, (size_t)K);
+    }
+    free(row_codes);
+  }
+  return 0;
+}
+
+/* oracle_unpack: the documented word layout back to codes uint8 [S][N][K]. */
+void oracle_unpack(const uint32_t* codes, int64_t N, int64_t K, int S, uint8_t* q_out) {
+  const int64_t nwords = K / 16;
+  for (int64_t s = 0; s < S; ++s)
+    for (int64_t n = 0; n < N; ++n)
+      for (int64_t k = 0; k < K; ++k) {
+        uint32_t word = codes[(s * N + n) * nwords + k / 16];
+        q_out[(s * N + n) * K + k] = (uint8_t)((word >> (2 * (k % 16))) & 3u);
+      }
+}
+
+/*
+ * oracle_reconstruct: the k-slice weight W^(k)[n][j] = sum_{s<k} (q - z) * scale
+ * in fp64 (exact: every term is a small integer times an fp16 value)
+ * ([ja] §2.1 W^(b) = sum W_e; [en] §2.A "Elasticity").
+ */
+void oracle_reconstruct(const uint32_t* codes, const uint32_t* sz, int64_t N, int64_t K,
+                        int G, int S, int k, double* W_hat) {
+  const int64_t nwords = K / 16, ngroups = K / G;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t j = 0; j < K; ++j) {
+      double acc = 0.0;
+      for (int s = 0; s < k && s < S; ++s) {
+        uint32_t word = codes[((int64_t)s * N + n) * nwords + j / 16];
+        int q = (int)((word >> (2 * (j % 16))) & 3u);
+        uint32_t e = sz[((int64_t)s * N + n) * ngroups + j / G];
+        double scale = (double)half_bits_to_float((uint16_t)(e & 0xffffu));
+        double zero = (double)half_bits_to_float((uint16_t)(e >> 16));
+        acc += ((double)q - zero) * scale;
+      }
+      W_hat[n * K + j] = acc;
+    }
+}
+
+/* ---- MoBiRoute ---------------------------------------------------------- */
+
+/*
+ * oracle_route: logit_j(t) = sum_k x[t,k] Wr[k,j] + bias_j in fp64 and
+ * k_t = 1 + argmax_j (the first maximum wins) ([ja] §2.2, [en] §2.B).
+ * gap[t] = best logit minus the runner-up (+inf when S == 1), so that callers
+ * can tell near-ties apart. logits (fp64 [T][S]) may be NULL.
+ */
+void oracle_route(const uint16_t* X, int64_t T, int64_t K, const float* Wr, const float* bias,
+                  int S, int32_t* k_out, double* gap, double* logits, int nthreads) {
+  set_threads(nthreads);
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    double l[8];
+    for (int j = 0; j < S; ++j) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += bf16_bits_to_double(X[t * K + k]) * (double)Wr[k * S + j];
+      l[j] = acc + (bias ? (double)bias[j] : 0.0);
+    }
+    int best = 0;
+    for (int j = 1; j < S; ++j)
+      if (l[j] > l[best]) best = j;
+    double second = -INFINITY;
+    for (int j = 0; j < S; ++j)
+      if (j != best && l[j] > second) second = l[j];
+    k_out[t] = best + 1;
+    if (gap) gap[t] = l[best] - second;
+    if (logits)
+      for (int j = 0; j < S; ++j) logits[t * S + j] = l[j];
+  }
+}
+
+/*
+ * oracle_bucket: stable counting sort of the tokens by k_t ascending.
+ * perm[i] = original index of the i-th token; bucket j (k_t = j+1) is
+ * perm[offsets[j] .. offsets[j+1]). Returns -1 if a k_t is outside 1..S.
+ */
+int oracle_bucket(const int32_t* k_t, int64_t T, int S, int32_t* perm, int32_t* offsets) {
+  int64_t count[9] = {0};
+  for (int64_t t = 0; t < T; ++t) {
+    if (k_t[t] < 1 || k_t[t] > S) return -1;
+    count[k_t[t] - 1]++;
+  }
+  int64_t next[9];
+  offsets[0] = 0;
+  for (int j = 0; j < S; ++j) {
+    next[j] = offsets[j];
+    offsets[j + 1] = (int32_t)(offsets[j] + count[j]);
+  }
+  for (int64_t t = 0; t < T; ++t) perm[next[k_t[t] - 1]++] = (int32_t)t;
+  return 0;
+}
+
+/* ---- mixed-bit GEMM ----------------------------------------------------- */
+
+/*
+ * oracle_gemm: for each listed token t = tokens[i] (all tokens when tokens is
+ * NULL, i = t), Y[i][n] = sum_k x[t,k] * W^(k_t)[n,k] in fp64, with
+ * W^(k) = sum_{s<k} (q - z) * scale built exactly ([ja] §2.1; [en] §2.A).
+ * Y is fp64 [n_tokens][N]. The sum over k runs in index order.
+ */
+void oracle_gemm(const uint16_t* X, int64_t T, int64_t K, const int32_t* k_t,
+                 const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S,
+                 const int32_t* tokens, int64_t n_tokens, double* Y, int nthreads) {
+  (void)T;
+  set_threads(nthreads);
+  const int64_t nwords = K / 16, ngroups = K / G;
+  if (!tokens) n_tokens = T;
+#pragma omp parallel for schedule(dynamic, 8)
+  for (int64_t n = 0; n < N; ++n) {
+    /* the S reconstructions of row n: W^(1), ..., W^(S) */
+    double* wk = (double*)malloc(sizeof(double) * (size_t)S * (size_t)K);
+    for (int64_t j = 0; j < K; ++j) {
+      double acc = 0.0;
+      for (int s = 0; s < S; ++s) {
+        uint32_t word = codes[((int64_t)s * N + n) * nwords + j / 16];
+        int q = (int)((word >> (2 * (j % 16))) & 3u);
+        uint32_t e = sz[((int64_t)s * N + n) * ngroups + j / G];
+        double scale = (double)half_bits_to_float((uint16_t)(e & 0xffffu));
+        double zero = (double)half_bits_to_float((uint16_t)(e >> 16));
+        acc += ((double)q - zero) * scale;
+        wk[(int64_t)s * K + j] = acc;
+      }
+    }
+    for (int64_t i = 0; i < n_tokens; ++i) {
+      int64_t t = tokens ? tokens[i] : i;
+      const double* w = wk + (int64_t)(k_t[t] - 1) * K;
+      double acc = 0.0;
+      for (int64_t j = 0; j < K; ++j) acc += bf16_bits_to_double(X[t * K + j]) * w[j];
+      Y[i * N + n] = acc;
+    }
+    free(wk);
+  }
+}

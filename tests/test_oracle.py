@@ -1,0 +1,307 @@
+"""Pins of the CPU oracle against things other than itself.
+
+The MoBiQuant explainer pages print no worked numeric example, so each oracle
+function is pinned by (a) groups whose quantisation is derived by hand below
+(closed forms), (b) library routines for special cases (torch's fake-quantise
+and MinMax observer for one round of asymmetric min-max RTN, numpy fp64 matmul
+and argmax, numpy stable argsort), (c) invariants of the recursion of
+[ja] §2.1 / [en] §2.A (R_{s+1} = R_s - Q(R_s): the residual never grows, a
+rounding error stays within half a step) and (d) brute force on tiny shapes.
+"""
+import numpy as np
+import pytest
+import torch
+
+from token_adaptive_mixed_b200 import workloads as wl
+
+F16 = np.float16
+
+
+def f16_bits(x: float) -> int:
+    return int(np.array([x], F16).view(np.uint16)[0])
+
+
+def group_row(pattern, G=128):
+    """One fp16 row of G weights repeating `pattern`."""
+    vals = np.array([pattern[i % len(pattern)] for i in range(G)], np.float64)
+    W = vals.astype(F16)
+    assert np.all(W.astype(np.float64) == vals), "pattern must be fp16-exact"
+    return W.reshape(1, G)
+
+
+# ---- (a) closed-form groups --------------------------------------------------
+
+def test_exact_grid_group(oracle):
+    """Values {-1,0,1,2} * 2^-5: range 3*2^-5, so the step is exactly 2^-5 and
+    zero = rint(1) = 1; codes are 0,1,2,3 repeated and slice 1 is exact. The
+    residual is 0, so slices 2 and 3 see a degenerate group: step floored to
+    2^-14 (fp16 0x0400), zero 0, all codes 0."""
+    s = 2.0 ** -5
+    W = group_row([-s, 0.0, s, 2 * s])
+    codes, sz, q = oracle.pack(W, S=3)
+    assert np.all(codes[0] == 0xE4E4E4E4)        # fields 0,1,2,3 -> 0b11100100 per byte
+    assert np.all(sz[0] == (f16_bits(s) | (f16_bits(1.0) << 16)))
+    assert np.all(codes[1:] == 0)
+    assert np.all(sz[1:] == 0x0400)              # scale 2^-14, zero +0
+    W1 = oracle.reconstruct(codes, sz, 1, 128, k=1)
+    assert np.array_equal(W1, W.astype(np.float64))
+
+
+def test_rounding_ties_and_clamps(oracle):
+    """Values {-1.5,-0.5,0.5,1.5}/16, derived by hand:
+    slice 1: step 1/16 (0x2C00), zero rint(1.5)=2 (ties to even), R/step rounds
+      to {-2,-0,0,2} -> codes {0,2,2,3} (4 clamps to 3) -> byte 0xE8;
+      residual {1,-1,1,1}/32.
+    slice 2: (2/32)/3 = 1/48 rounds in fp16 to 1365/65536 (0x2555); zero
+      rint(2048/1365)=2; R/step = +-1.50037 -> +-2 -> codes {3,0,3,3} -> 0xF3;
+      residual {683,682,683,683}/65536.
+    slice 3: range 1/65536 -> step floored to 2^-14; zero rint(-170.5) = -170
+      clamps to 0; R/step = 170.75 / 170.5 -> codes all 3 (clamped) -> 0xFF."""
+    W = group_row([-1.5 / 16, -0.5 / 16, 0.5 / 16, 1.5 / 16])
+    codes, sz, q = oracle.pack(W, S=3)
+    assert np.all(codes[0] == 0xE8E8E8E8)
+    assert np.all(sz[0] == (0x2C00 | (f16_bits(2.0) << 16)))
+    assert np.all(codes[1] == 0xF3F3F3F3)
+    assert np.all(sz[1] == (0x2555 | (f16_bits(2.0) << 16)))
+    assert np.all(codes[2] == 0xFFFFFFFF)
+    assert np.all(sz[2] == 0x0400)
+    W2 = oracle.reconstruct(codes, sz, 1, 128, k=2)
+    resid = W.astype(np.float64) - W2
+    expect = np.array([683, 682, 683, 683] * 32, np.float64) / 65536
+    assert np.array_equal(resid.ravel(), expect)
+    W3 = oracle.reconstruct(codes, sz, 1, 128, k=3)
+    expect3 = np.array([671, 670, 671, 671] * 32, np.float64) / 65536
+    assert np.array_equal((W.astype(np.float64) - W3).ravel(), expect3)
+
+
+def test_all_negative_group(oracle):
+    """Values {-4,-3,-2,-1}/64: step 1/64 (0x2400), zero rint(4) = 4 -> clamps
+    to 3 (0x4200); codes {0,0,1,2} (byte 0x90); residual {-1,0,0,0}/64.
+    slice 2: step fp16(1/192) = 1365/262144, zero rint(3.0007) = 3, codes
+    {0,3,3,3} (byte 0xFC); residual {-1,0,0,0}/262144.
+    slice 3: step 2^-14, zero rint(1/16) = 0, codes all 0."""
+    W = group_row([-4 / 64, -3 / 64, -2 / 64, -1 / 64])
+    codes, sz, _ = oracle.pack(W, S=3)
+    assert np.all(codes[0] == 0x90909090)
+    assert np.all(sz[0] == (0x2400 | (0x4200 << 16)))
+    assert np.all(codes[1] == 0xFCFCFCFC)
+    assert np.all(sz[1] == (f16_bits(1365 / 262144) | (0x4200 << 16)))
+    assert f16_bits(1365 / 262144) == 0x1D55
+    assert np.all(codes[2] == 0)
+    assert np.all(sz[2] == 0x0400)
+    W3 = oracle.reconstruct(codes, sz, 1, 128, k=3)
+    expect = np.array([-1, 0, 0, 0] * 32, np.float64) / 262144
+    assert np.array_equal((W.astype(np.float64) - W3).ravel(), expect)
+
+
+def test_constant_positive_group(oracle):
+    """A constant group c = 1: range 0 -> step 2^-14, zero clamps to 0, every
+    code clamps to 3, so each slice removes exactly 3 * 2^-14."""
+    W = group_row([1.0])
+    codes, sz, _ = oracle.pack(W, S=3)
+    assert np.all(codes == 0xFFFFFFFF)
+    assert np.all(sz == 0x0400)
+    for k in (1, 2, 3):
+        Wk = oracle.reconstruct(codes, sz, 1, 128, k=k)
+        assert np.all(Wk == 3 * k * 2.0 ** -14)
+
+
+def test_packed_word_bit_order(oracle):
+    """Code of k = 16w + i sits in bits [2i+1:2i] of word w: a row whose slice-1
+    codes are 3 only at k = 5 and k = 16+15 gives words 0x00000C00 and 0xC0000000."""
+    s = 2.0 ** -4
+    vals = np.zeros(128)
+    vals[:] = 0.0
+    vals[5] = 3 * s
+    vals[31] = 3 * s
+    # min 0, max 3s -> step s, zero 0: codes are 3 at k=5, 31 and 0 elsewhere.
+    W = vals.astype(F16).reshape(1, 128)
+    codes, sz, q = oracle.pack(W, S=1)
+    assert codes[0, 0, 0] == 0x00000C00
+    assert codes[0, 0, 1] == 0xC0000000
+    assert np.all(codes[0, 0, 2:] == 0)
+    assert np.array_equal(oracle.unpack(codes, 1, 128, 1), q)
+
+
+# ---- (b) library special cases -----------------------------------------------
+
+def _random_W(N, K, seed, outliers=4):
+    return wl.draw_weights(np.random.default_rng(seed), N, K, 0.02, outliers)
+
+
+def test_slice1_matches_torch_fake_quantize(oracle):
+    """Slice 1 is one round of asymmetric RTN: given the oracle's per-group
+    scale and zero, torch.fake_quantize_per_channel_affine (round half to even,
+    clamp to [0,3]) must give the oracle's dequantised slice bit for bit."""
+    N, K = 64, 512
+    W = _random_W(N, K, 11)
+    codes, sz, q = oracle.pack(W, S=1)
+    scale = (sz[0] & 0xFFFF).astype(np.uint16).view(F16).astype(np.float32).ravel()
+    zero = (sz[0] >> 16).astype(np.uint16).view(F16).astype(np.float32).ravel().astype(np.int32)
+    x = torch.from_numpy(W.astype(np.float32).reshape(N * K // 128, 128))
+    fq = torch.fake_quantize_per_channel_affine(x, torch.from_numpy(scale), torch.from_numpy(zero), 0, 0, 3)
+    W1 = oracle.reconstruct(codes, sz, N, K, k=1, S=1)
+    assert np.array_equal(fq.numpy().astype(np.float64).reshape(N, K), W1)
+
+
+def test_scale_matches_torch_minmax_observer(oracle):
+    """For a group holding both signs, torch's MinMax observer (quint8 with
+    quant range [0,3]) computes the step (max - min)/3 in fp32; rounded to fp16
+    it is the oracle's stored slice-1 scale."""
+    from torch.ao.quantization.observer import MinMaxObserver
+    N, K = 8, 256
+    W = _random_W(N, K, 12)
+    codes, sz, _ = oracle.pack(W, S=1)
+    for n in range(N):
+        for g in range(K // 128):
+            grp = torch.from_numpy(W[n, g * 128:(g + 1) * 128].astype(np.float32))
+            assert grp.min() < 0 < grp.max()
+            obs = MinMaxObserver(dtype=torch.quint8, quant_min=0, quant_max=3)
+            obs(grp)
+            sc, _ = obs.calculate_qparams()
+            assert f16_bits(float(sc.to(torch.float16))) == int(sz[0, n, g] & 0xFFFF)
+
+
+# ---- (c) invariants ------------------------------------------------------------
+
+def test_residual_never_grows(oracle):
+    """0 is always on the grid (integer zero in [0,3]) and clamping moves toward
+    it, so |W - W^(k+1)| <= |W - W^(k)| element by element (up to the fp32
+    rounding of the residual), and the Frobenius error falls with k."""
+    N, K = 128, 1024
+    W = _random_W(N, K, 13, outliers=8)
+    codes, sz, _ = oracle.pack(W, S=3)
+    Wd = W.astype(np.float64)
+    errs = [np.abs(Wd)]
+    fro = [np.linalg.norm(Wd)]
+    for k in (1, 2, 3):
+        e = np.abs(Wd - oracle.reconstruct(codes, sz, N, K, k=k))
+        errs.append(e)
+        fro.append(np.linalg.norm(e))
+    for a, b in zip(errs[:-1], errs[1:]):
+        assert np.all(b <= a + 1e-6 * np.abs(Wd) + 1e-9)
+    assert fro[1] < fro[0] and fro[2] < fro[1] and fro[3] < fro[2]
+    rel = [f / fro[0] for f in fro[1:]]
+    assert rel[2] < 0.2 * rel[0]
+
+
+def test_half_step_bound(oracle):
+    """Where a group holds both signs and no code clamps, slice s leaves each
+    element within half a step (plus the gap left when the fp16 step times 3
+    falls short of the range)."""
+    N, K = 64, 512
+    W = _random_W(N, K, 14)
+    codes, sz, q = oracle.pack(W, S=1)
+    Wd = W.astype(np.float64).reshape(N, K // 128, 128)
+    W1 = oracle.reconstruct(codes, sz, N, K, k=1, S=1).reshape(N, K // 128, 128)
+    step = (sz[0] & 0xFFFF).astype(np.uint16).view(F16).astype(np.float64)
+    rng_ = Wd.max(-1) - Wd.min(-1)
+    slack = np.maximum(rng_ - 3 * step, 0.0)
+    err = np.abs(Wd - W1).max(-1)
+    assert np.all(err <= step / 2 * (1 + 1e-6) + slack)
+
+
+# ---- (d) routing, bucketing and GEMM -------------------------------------------
+
+def test_route_brute_force(oracle):
+    L = wl.layer("t", 16, 256, 64, seed=21)
+    k, gap, logits = oracle.route(L.X, L.Wr)
+    ref = L.X.to(torch.float64).numpy() @ L.Wr.astype(np.float64)
+    assert np.allclose(logits, ref, rtol=0, atol=1e-12)
+    assert np.array_equal(k, np.argmax(ref, axis=1) + 1)
+
+
+def test_route_ties_and_dominant_column(oracle):
+    T, K = 8, 128
+    X = wl.to_bf16(np.ones((T, K), np.float32))
+    Wr = np.zeros((K, 3), np.float32)
+    k, gap, _ = oracle.route(X, Wr)                       # all logits equal: lowest index
+    assert np.all(k == 1) and np.all(gap == 0)
+    k, _, _ = oracle.route(X, Wr, np.array([0, 1, 1], np.float32))   # tie between 2 and 3
+    assert np.all(k == 2)
+    Wr[:, 2] = 1.0                                        # column 3 dominates a positive x
+    k, gap, _ = oracle.route(X, Wr)
+    assert np.all(k == 3) and np.allclose(gap, K)
+
+
+def test_bucket_is_stable_sort(oracle):
+    rng = np.random.default_rng(5)
+    for T in (0, 1, 7, 1000):
+        k = rng.integers(1, 4, T).astype(np.int32)
+        perm, off = oracle.bucket(k)
+        assert np.array_equal(perm, np.argsort(k, kind="stable"))
+        assert off[0] == 0 and off[3] == T
+        for j in range(3):
+            assert np.all(k[perm[off[j]:off[j + 1]]] == j + 1)
+
+
+def test_gemm_brute_force(oracle):
+    """Y = x_t . W^(k_t)^T: against numpy fp64 matmul of the per-k reconstructions."""
+    N, K, T = 48, 384, 24
+    W = _random_W(N, K, 31)
+    rng = np.random.default_rng(32)
+    X = wl.draw_activations(rng, T, K)
+    k = rng.integers(1, 4, T).astype(np.int32)
+    codes, sz, _ = oracle.pack(W, S=3)
+    Y = oracle.gemm(X, k, codes, sz, N)
+    Xd = X.to(torch.float64).numpy()
+    for t in range(T):
+        Wk = oracle.reconstruct(codes, sz, N, K, k=int(k[t]))
+        ref = Wk @ Xd[t]
+        assert np.allclose(Y[t], ref, rtol=1e-13, atol=1e-13)
+    sub = np.array([3, 0, 17], np.int32)
+    Ys = oracle.gemm(X, k, codes, sz, N, tokens=sub)
+    assert np.array_equal(Ys, Y[sub])
+
+
+def test_gemm_one_hot(oracle):
+    """x = e_j picks column j of W^(k_t): checks the orientation of the product."""
+    N, K = 32, 256
+    W = _random_W(N, K, 41)
+    codes, sz, _ = oracle.pack(W, S=3)
+    cols = [0, 1, 127, 128, 255]
+    X = np.zeros((len(cols), K), np.float32)
+    for i, j in enumerate(cols):
+        X[i, j] = 1.0
+    k = np.array([1, 2, 3, 2, 1], np.int32)
+    Y = oracle.gemm(wl.to_bf16(X), k, codes, sz, N)
+    for i, j in enumerate(cols):
+        assert np.array_equal(Y[i], oracle.reconstruct(codes, sz, N, K, k=int(k[i]))[:, j])
+
+
+def test_tiny_workload_fractions_and_error(oracle):
+    """The tiny workload: relative reconstruction error falls with each slice
+    and the 2-slice error is well under the 1-slice one."""
+    L = wl.tiny()
+    codes, sz, _ = oracle.pack(L.W, S=3)
+    Wd = L.W.astype(np.float64)
+    rel = [np.linalg.norm(Wd - oracle.reconstruct(codes, sz, L.N, L.K, k=k)) / np.linalg.norm(Wd)
+           for k in (1, 2, 3)]
+    assert rel[0] > rel[1] > rel[2]
+    assert rel[2] < 0.15
+
+
+def test_golden_tiny_fixture(oracle):
+    """The oracle reproduces its committed outputs on the tiny workload."""
+    import os
+    g = np.load(os.path.join(os.path.dirname(__file__), "golden", "tiny_oracle.npz"))
+    L = wl.tiny()
+    codes, sz, _ = oracle.pack(L.W, S=3)
+    k, gap, _ = oracle.route(L.X, L.Wr, L.bias)
+    perm, off = oracle.bucket(k)
+    assert np.array_equal(codes, g["codes"]) and np.array_equal(sz, g["sz"])
+    assert np.array_equal(k, g["k_t"]) and np.array_equal(perm, g["perm"]) and np.array_equal(off, g["offsets"])
+    assert np.array_equal(oracle.gemm(L.X, k, codes, sz, L.N), g["Y"])
+
+
+@pytest.mark.slow
+def test_workload_mixes(oracle):
+    """The bias solver gives the stated slice-count mixes on the prefill workloads."""
+    L = wl.prefill()
+    k, _, _ = oracle.route(L.X, L.Wr, L.bias)
+    frac = np.bincount(k, minlength=4)[1:] / L.T
+    assert np.all(np.abs(frac - 1 / 3) < 0.05), frac
+    L = wl.skewed_prefill()
+    k, _, _ = oracle.route(L.X, L.Wr, L.bias)
+    frac = np.bincount(k, minlength=4)[1:] / L.T
+    assert np.all(np.abs(frac - np.array([0.7, 0.2, 0.1])) < 0.04), frac
