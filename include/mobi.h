@@ -44,8 +44,10 @@
  *   codes  uint32 [S][N][K/16]   word w of (slice s, row n) holds the codes of
  *          k = 16w .. 16w+15; code q(s,n,16w+i) sits in bits [2i+1 : 2i]
  *          (little-endian 2-bit fields). mobi_codes_bytes() gives the size.
- *   sz     uint32 [S][N][K/G]    element (s,n,g): bits [15:0] = fp16 scale,
+ *   sz     uint32 [S][K/G][N]    element (s,g,n): bits [15:0] = fp16 scale,
  *          bits [31:16] = fp16 zero (an integer 0..3). mobi_sz_bytes().
+ *          Group-major so that the scales of one group for consecutive rows
+ *          are contiguous (N*4-byte rows, which tensor copies can stage).
  *   The dequantised slice is deq_s[n,k] = (q(s,n,k) - zero(s,n,k/G)) *
  *   scale(s,n,k/G), and the k-slice weight is W^(k) = sum_{s<k} deq_s.
  *
@@ -65,6 +67,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define MOBI_API __attribute__((visibility("default")))
+#else
+#define MOBI_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -80,24 +88,24 @@ typedef enum {
 } mobi_status;
 
 /* Human-readable name of a status (static storage, never NULL). */
-const char* mobi_status_string(mobi_status st);
+MOBI_API const char* mobi_status_string(mobi_status st);
 
 /* Library version as an integer MAJOR*10000 + MINOR*100 + PATCH. */
-int mobi_version(void);
+MOBI_API int mobi_version(void);
 
 /* Bytes of the packed code array for S slices of an N x K matrix:
  * S * N * (K/16) * 4. Returns 0 for invalid sizes. */
-size_t mobi_codes_bytes(int64_t N, int64_t K, int S);
+MOBI_API size_t mobi_codes_bytes(int64_t N, int64_t K, int S);
 
 /* Bytes of the scale/zero array: S * N * (K/G) * 4. Returns 0 for invalid sizes. */
-size_t mobi_sz_bytes(int64_t N, int64_t K, int S, int G);
+MOBI_API size_t mobi_sz_bytes(int64_t N, int64_t K, int S, int G);
 
 /* Scratch bytes that mobi_route needs for T tokens (may be 0). */
-size_t mobi_route_workspace_bytes(int64_t T, int64_t K, int S);
+MOBI_API size_t mobi_route_workspace_bytes(int64_t T, int64_t K, int S);
 
 /* Scratch bytes that mobi_gemm needs (covers both the decode and the prefill
  * kernels, so one buffer serves every T up to the given one). */
-size_t mobi_gemm_workspace_bytes(int64_t T, int64_t N, int64_t K, int S);
+MOBI_API size_t mobi_gemm_workspace_bytes(int64_t T, int64_t N, int64_t K, int S);
 
 /*
  * mobi_pack — MoBiSlice recursive residual quantisation of W.
@@ -107,10 +115,10 @@ size_t mobi_gemm_workspace_bytes(int64_t T, int64_t N, int64_t K, int S);
  *   G        group size along K; must be 128.
  *   S        number of slices, 1..3.
  *   codes    out, uint32 [S][N][K/16] (layout above).
- *   sz       out, uint32 [S][N][K/G]  (fp16 scale | fp16 zero << 16).
+ *   sz       out, uint32 [S][K/G][N]  (fp16 scale | fp16 zero << 16).
  * Bit-exact with the quantiser above (IEEE division, RNE, no flush-to-zero).
  */
-mobi_status mobi_pack(const void* W, int64_t N, int64_t K, int G, int S,
+MOBI_API mobi_status mobi_pack(const void* W, int64_t N, int64_t K, int G, int S,
                       uint32_t* codes, uint32_t* sz, void* stream);
 
 /*
@@ -130,7 +138,7 @@ mobi_status mobi_pack(const void* W, int64_t N, int64_t K, int G, int S,
  *   ws       scratch of mobi_route_workspace_bytes(T, K, S) bytes (may be
  *            NULL when that size is 0).
  */
-mobi_status mobi_route(const void* X, int64_t T, int64_t K, const float* Wr,
+MOBI_API mobi_status mobi_route(const void* X, int64_t T, int64_t K, const float* Wr,
                        const float* bias, int S, int32_t* k_t, int32_t* perm,
                        int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
 
@@ -148,7 +156,7 @@ mobi_status mobi_route(const void* X, int64_t T, int64_t K, const float* Wr,
  * T <= 16 runs the decode kernel (streams only the slices up to the batch's
  * largest k_t), larger T the tcgen05 prefill kernel.
  */
-mobi_status mobi_gemm(const void* X, int64_t T, int64_t K, const int32_t* k_t,
+MOBI_API mobi_status mobi_gemm(const void* X, int64_t T, int64_t K, const int32_t* k_t,
                       const int32_t* perm, const int32_t* offsets,
                       const uint32_t* codes, const uint32_t* sz, int64_t N, int G,
                       int S, float* Y, void* ws, size_t ws_bytes, void* stream);
@@ -161,7 +169,7 @@ typedef enum {
 } mobi_path;
 
 /* mobi_gemm with an explicit kernel choice (same arguments and result). */
-mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const int32_t* k_t,
+MOBI_API mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const int32_t* k_t,
                            const int32_t* perm, const int32_t* offsets,
                            const uint32_t* codes, const uint32_t* sz, int64_t N,
                            int G, int S, float* Y, void* ws, size_t ws_bytes,
@@ -172,7 +180,7 @@ mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const int32_t* k
  * device-side error word of the current device. Returns MOBI_ERR_TIMEOUT if a
  * bounded wait ran out since the last check, MOBI_ERR_CUDA on a CUDA error.
  */
-mobi_status mobi_sync_check(void* stream);
+MOBI_API mobi_status mobi_sync_check(void* stream);
 
 /*
  * mobi_debug_set_wait_limit — set the iteration limit of the device-side
@@ -181,7 +189,7 @@ mobi_status mobi_sync_check(void* stream);
  * without faulting anything: the kernel records the error, drains its own
  * copies in flight, frees its tensor memory and returns. Test use only.
  */
-mobi_status mobi_debug_set_wait_limit(int64_t limit);
+MOBI_API mobi_status mobi_debug_set_wait_limit(int64_t limit);
 
 #ifdef __cplusplus
 }

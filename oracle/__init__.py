@@ -84,12 +84,12 @@ def max_threads() -> int:
 
 
 def pack(W_f16: np.ndarray, G: int = 128, S: int = 3, nthreads: int = 0):
-    """MoBiSlice packing. Returns (codes uint32 [S,N,K/16], sz uint32 [S,N,K/G], q uint8 [S,N,K])."""
+    """MoBiSlice packing. Returns (codes uint32 [S,N,K/16], sz uint32 [S,K/G,N], q uint8 [S,N,K])."""
     lib = _load()
     W = _u16(W_f16)
     N, K = W.shape
     codes = np.zeros((S, N, K // 16), np.uint32)
-    sz = np.zeros((S, N, K // G), np.uint32)
+    sz = np.zeros((S, K // G, N), np.uint32)
     q = np.zeros((S, N, K), np.uint8)
     rc = lib.oracle_pack(_ptr(W), N, K, G, S, _ptr(codes), _ptr(sz), _ptr(q), nthreads)
     if rc != 0:

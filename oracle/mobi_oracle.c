@@ -124,7 +124,7 @@ static void quantise_group(const uint16_t* w, int G, int S, uint8_t* q_out,
 
 /*
  * oracle_pack: W fp16 [N][K] -> codes (the documented 2-bit word layout:
- * word (s, n, w) holds q(s, n, 16w + i) in bits [2i+1:2i]) and sz
+ * word (s, n, w) holds q(s, n, 16w + i) in bits [2i+1:2i]) and sz [S][K/G][N]
  * (fp16 scale in bits [15:0], fp16 zero in bits [31:16]), plus, if q_out is
  * not NULL, the unpacked codes uint8 [S][N][K].
  * Returns 0, or -1 on an unsupported argument.
@@ -143,7 +143,7 @@ int oracle_pack(const uint16_t* W, int64_t N, int64_t K, int G, int S,
     for (int64_t g = 0; g < ngroups; ++g) {
       quantise_group(W + n * K + g * G, G, S, q, sc, zr);
       for (int s = 0; s < S; ++s) {
-        sz[((int64_t)s * N + n) * ngroups + g] = (uint32_t)sc[s] | ((uint32_t)zr[s] << 16);
+        sz[((int64_t)s * ngroups + g) * N + n] = (uint32_t)sc[s] | ((uint32_t)zr[s] << 16);
         for (int i = 0; i < G; ++i) row_codes[(int64_t)s * K + g * G + i] = q[s * G + i];
       }
     }
@@ -187,7 +187,7 @@ void oracle_reconstruct(const uint32_t* codes, const uint32_t* sz, int64_t N, in
       for (int s = 0; s < k && s < S; ++s) {
         uint32_t word = codes[((int64_t)s * N + n) * nwords + j / 16];
         int q = (int)((word >> (2 * (j % 16))) & 3u);
-        uint32_t e = sz[((int64_t)s * N + n) * ngroups + j / G];
+        uint32_t e = sz[((int64_t)s * ngroups + j / G) * N + n];
         double scale = (double)half_bits_to_float((uint16_t)(e & 0xffffu));
         double zero = (double)half_bits_to_float((uint16_t)(e >> 16));
         acc += ((double)q - zero) * scale;
@@ -273,7 +273,7 @@ void oracle_gemm(const uint16_t* X, int64_t T, int64_t K, const int32_t* k_t,
       for (int s = 0; s < S; ++s) {
         uint32_t word = codes[((int64_t)s * N + n) * nwords + j / 16];
         int q = (int)((word >> (2 * (j % 16))) & 3u);
-        uint32_t e = sz[((int64_t)s * N + n) * ngroups + j / G];
+        uint32_t e = sz[((int64_t)s * ngroups + j / G) * N + n];
         double scale = (double)half_bits_to_float((uint16_t)(e & 0xffffu));
         double zero = (double)half_bits_to_float((uint16_t)(e >> 16));
         acc += ((double)q - zero) * scale;

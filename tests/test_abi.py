@@ -1,0 +1,97 @@
+"""The C ABI loads and exports every function include/mobi.h declares; host-side
+validation returns the documented status before anything reaches CUDA.
+
+These tests run without a GPU: the calls below fail validation (bad shape,
+null or misaligned pointer, short workspace) and return before any CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import token_adaptive_mixed_b200 as mobi
+from token_adaptive_mixed_b200 import build as mobi_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    mobi_build.build()
+    return mobi.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "mobi.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mobi_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(mobi.EXPORTED_SYMBOLS) == names
+
+
+def test_status_strings_and_sizes(L):
+    assert mobi.mobi_status_string(0) == "MOBI_OK"
+    assert mobi.mobi_status_string(6) == "MOBI_ERR_TIMEOUT"
+    assert mobi.mobi_version() >= 100
+    assert mobi.mobi_codes_bytes(4096, 4096, 3) == 3 * 4096 * 256 * 4
+    assert mobi.mobi_sz_bytes(4096, 4096, 3, 128) == 3 * 4096 * 32 * 4
+    assert mobi.mobi_codes_bytes(16, 100, 3) == 0  # K % 16 != 0
+    assert mobi.mobi_gemm_workspace_bytes(16, 4096, 4096, 3) > 0
+
+
+FAKE = 1 << 20  # a 16-byte-aligned non-null address; never dereferenced: validation fails first
+
+
+def test_pack_validation(L):
+    p = ctypes.c_void_p
+    assert L.mobi_pack(p(FAKE), 16, 100, 128, 3, p(FAKE), p(FAKE), None) == 2   # K % 128
+    assert L.mobi_pack(p(FAKE), 24, 128, 128, 3, p(FAKE), p(FAKE), None) == 2   # N % 16
+    assert L.mobi_pack(p(FAKE), 16, 128, 64, 3, p(FAKE), p(FAKE), None) == 2    # G != 128
+    assert L.mobi_pack(p(FAKE), 16, 128, 128, 4, p(FAKE), p(FAKE), None) == 1   # S > 3
+    assert L.mobi_pack(None, 16, 128, 128, 3, p(FAKE), p(FAKE), None) == 1      # null W
+    assert L.mobi_pack(p(FAKE + 2), 16, 128, 128, 3, p(FAKE), p(FAKE), None) == 3  # misaligned
+    assert L.mobi_pack(p(FAKE), 0, 128, 128, 3, p(FAKE), p(FAKE), None) == 0    # empty: no-op
+
+
+def test_route_validation(L):
+    p = ctypes.c_void_p
+    args = lambda X=p(FAKE), T=16, K=256, S=3, ws=None, wsb=0: (X, T, K, p(FAKE), None, S, p(FAKE), p(FAKE),
+                                                                 p(FAKE), ws, wsb, None)
+    assert L.mobi_route(*args(K=100)) == 2
+    assert L.mobi_route(*args(S=0)) == 1
+    assert L.mobi_route(*args(X=None)) == 1
+    assert L.mobi_route(*args(X=p(FAKE + 8))) == 3
+    T, K = 1, 4096  # small T splits K and needs a workspace
+    assert mobi.mobi_route_workspace_bytes(T, K, 3) > 0
+    assert L.mobi_route(*args(T=T, K=K)) == 4
+
+
+def test_gemm_validation(L):
+    p = ctypes.c_void_p
+
+    def call(T=16, K=256, N=64, S=3, G=128, ws=p(FAKE), wsb=1 << 30, path=0, X=p(FAKE), Y=p(FAKE)):
+        return L.mobi_gemm_path(X, T, K, p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE), N, G, S, Y, ws, wsb,
+                                None, path)
+    assert call(K=200) == 2
+    assert call(N=24) == 2
+    assert call(G=32) == 2
+    assert call(S=0) == 1
+    assert call(path=7) == 1
+    assert call(T=17, path=1) == 2        # decode kernel takes at most 16 tokens
+    assert call(X=None) == 1
+    assert call(Y=p(FAKE + 4)) == 3
+    assert call(wsb=16) == 4
+    assert call(T=0) == 0                 # nothing to do
+
+
+def test_workspace_sizes_edge_cases(L):
+    assert mobi.mobi_route_workspace_bytes(0, 256, 3) == 0
+    assert mobi.mobi_route_workspace_bytes(2048, 4096, 3) == 0   # many token tiles: no split
+    assert mobi.mobi_gemm_workspace_bytes(0, 0, 0, 3) >= 0

@@ -136,8 +136,8 @@ def test_slice1_matches_torch_fake_quantize(oracle):
     N, K = 64, 512
     W = _random_W(N, K, 11)
     codes, sz, q = oracle.pack(W, S=1)
-    scale = (sz[0] & 0xFFFF).astype(np.uint16).view(F16).astype(np.float32).ravel()
-    zero = (sz[0] >> 16).astype(np.uint16).view(F16).astype(np.float32).ravel().astype(np.int32)
+    scale = (sz[0].T & 0xFFFF).astype(np.uint16).view(F16).astype(np.float32).ravel()
+    zero = (sz[0].T >> 16).astype(np.uint16).view(F16).astype(np.float32).ravel().astype(np.int32)
     x = torch.from_numpy(W.astype(np.float32).reshape(N * K // 128, 128))
     fq = torch.fake_quantize_per_channel_affine(x, torch.from_numpy(scale), torch.from_numpy(zero), 0, 0, 3)
     W1 = oracle.reconstruct(codes, sz, N, K, k=1, S=1)
@@ -159,7 +159,7 @@ def test_scale_matches_torch_minmax_observer(oracle):
             obs = MinMaxObserver(dtype=torch.quint8, quant_min=0, quant_max=3)
             obs(grp)
             sc, _ = obs.calculate_qparams()
-            assert f16_bits(float(sc.to(torch.float16))) == int(sz[0, n, g] & 0xFFFF)
+            assert f16_bits(float(sc.to(torch.float16))) == int(sz[0, g, n] & 0xFFFF)
 
 
 # ---- (c) invariants ------------------------------------------------------------
@@ -194,7 +194,7 @@ def test_half_step_bound(oracle):
     codes, sz, q = oracle.pack(W, S=1)
     Wd = W.astype(np.float64).reshape(N, K // 128, 128)
     W1 = oracle.reconstruct(codes, sz, N, K, k=1, S=1).reshape(N, K // 128, 128)
-    step = (sz[0] & 0xFFFF).astype(np.uint16).view(F16).astype(np.float64)
+    step = (sz[0].T & 0xFFFF).astype(np.uint16).view(F16).astype(np.float64)
     rng_ = Wd.max(-1) - Wd.min(-1)
     slack = np.maximum(rng_ - 3 * step, 0.0)
     err = np.abs(Wd - W1).max(-1)

@@ -1,0 +1,201 @@
+"""token_adaptive_mixed_b200 — the MoBiQuant token-routed mixed-bit linear layer on B200.
+
+A thin ctypes binding over ``libmobi.so`` (the C ABI declared in
+``include/mobi.h``). Every function here only marshals torch tensors into
+pointers, sizes and the current CUDA stream; all arithmetic runs in the
+library's sm_100a kernels. There is no CPU fallback: if the library is missing
+or a tensor is not on a CUDA device, the call raises.
+
+Entry points (same names as the C ABI):
+  mobi_pack(W)                      MoBiSlice packing   -> (codes, sz)
+  mobi_route(X, Wr, bias)           MoBiRoute routing   -> (k_t, perm, offsets)
+  mobi_gemm(X, k_t, perm, offsets, codes, sz, N)         -> Y  (fp32)
+  mobi_gemm_path(..., path)         the same with a forced kernel
+  mobi_sync_check()                 sync + device-side error word
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "MobiError", "lib", "mobi_version", "mobi_status_string", "mobi_codes_bytes", "mobi_sz_bytes",
+    "mobi_route_workspace_bytes", "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm",
+    "mobi_gemm_path", "mobi_sync_check", "mobi_debug_set_wait_limit", "PATH_AUTO", "PATH_DECODE",
+    "PATH_PREFILL", "EXPORTED_SYMBOLS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.environ.get("MOBI_LIB", os.path.join(_HERE, "libmobi.so"))
+
+PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
+STATUS_NAMES = ["MOBI_OK", "MOBI_ERR_INVALID_ARG", "MOBI_ERR_UNSUPPORTED_SHAPE", "MOBI_ERR_MISALIGNED",
+                "MOBI_ERR_WORKSPACE", "MOBI_ERR_CUDA", "MOBI_ERR_TIMEOUT"]
+
+# Every symbol include/mobi.h declares.
+EXPORTED_SYMBOLS = (
+    "mobi_status_string", "mobi_version", "mobi_codes_bytes", "mobi_sz_bytes", "mobi_route_workspace_bytes",
+    "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm", "mobi_gemm_path", "mobi_sync_check",
+    "mobi_debug_set_wait_limit",
+)
+
+
+class MobiError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        name = STATUS_NAMES[status] if 0 <= status < len(STATUS_NAMES) else f"status {status}"
+        super().__init__(f"{fn}: {name}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmobi.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libmobi.so not found at {LIB_PATH}; build it with "
+                              f"`python -m token_adaptive_mixed_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        p, i64, ci, sz_t = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.mobi_status_string.argtypes = [ci]
+        L.mobi_status_string.restype = ctypes.c_char_p
+        L.mobi_version.argtypes = []
+        L.mobi_version.restype = ci
+        L.mobi_codes_bytes.argtypes = [i64, i64, ci]
+        L.mobi_codes_bytes.restype = sz_t
+        L.mobi_sz_bytes.argtypes = [i64, i64, ci, ci]
+        L.mobi_sz_bytes.restype = sz_t
+        L.mobi_route_workspace_bytes.argtypes = [i64, i64, ci]
+        L.mobi_route_workspace_bytes.restype = sz_t
+        L.mobi_gemm_workspace_bytes.argtypes = [i64, i64, i64, ci]
+        L.mobi_gemm_workspace_bytes.restype = sz_t
+        L.mobi_pack.argtypes = [p, i64, i64, ci, ci, p, p, p]
+        L.mobi_pack.restype = ci
+        L.mobi_route.argtypes = [p, i64, i64, p, p, ci, p, p, p, p, sz_t, p]
+        L.mobi_route.restype = ci
+        L.mobi_gemm.argtypes = [p, i64, i64, p, p, p, p, p, i64, ci, ci, p, p, sz_t, p]
+        L.mobi_gemm.restype = ci
+        L.mobi_gemm_path.argtypes = [p, i64, i64, p, p, p, p, p, i64, ci, ci, p, p, sz_t, p, ci]
+        L.mobi_gemm_path.restype = ci
+        L.mobi_sync_check.argtypes = [p]
+        L.mobi_sync_check.restype = ci
+        L.mobi_debug_set_wait_limit.argtypes = [i64]
+        L.mobi_debug_set_wait_limit.restype = ci
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise MobiError(fn, status)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libmobi takes CUDA tensors only (no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError("libmobi takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def mobi_version() -> int:
+    return lib().mobi_version()
+
+
+def mobi_status_string(status: int) -> str:
+    return lib().mobi_status_string(status).decode()
+
+
+def mobi_codes_bytes(N: int, K: int, S: int = 3) -> int:
+    return lib().mobi_codes_bytes(N, K, S)
+
+
+def mobi_sz_bytes(N: int, K: int, S: int = 3, G: int = 128) -> int:
+    return lib().mobi_sz_bytes(N, K, S, G)
+
+
+def mobi_route_workspace_bytes(T: int, K: int, S: int = 3) -> int:
+    return lib().mobi_route_workspace_bytes(T, K, S)
+
+
+def mobi_gemm_workspace_bytes(T: int, N: int, K: int, S: int = 3) -> int:
+    return lib().mobi_gemm_workspace_bytes(T, N, K, S)
+
+
+def _workspace(nbytes: int, device, ws: torch.Tensor | None) -> torch.Tensor:
+    if ws is not None:
+        return ws
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
+def mobi_pack(W: torch.Tensor, S: int = 3, G: int = 128, codes: torch.Tensor | None = None,
+              sz: torch.Tensor | None = None, stream=None):
+    """MoBiSlice packing of fp16 W[N,K] -> (codes int32 [S,N,K/16], sz int32 [S,K/G,N])."""
+    if W.dtype != torch.float16 or W.dim() != 2:
+        raise ValueError("W must be a 2-D fp16 tensor")
+    N, K = W.shape
+    if codes is None:
+        codes = torch.empty((S, N, K // 16), dtype=torch.int32, device=W.device)
+    if sz is None:
+        sz = torch.empty((S, K // G, N), dtype=torch.int32, device=W.device)
+    _check("mobi_pack", lib().mobi_pack(_ptr(W), N, K, G, S, _ptr(codes), _ptr(sz), _stream(stream)))
+    return codes, sz
+
+
+def mobi_route(X: torch.Tensor, Wr: torch.Tensor, bias: torch.Tensor | None = None, k_t=None, perm=None,
+               offsets=None, ws: torch.Tensor | None = None, stream=None):
+    """MoBiRoute: k_t = 1 + argmax(x.Wr + b) and the stable bucketing -> (k_t, perm, offsets)."""
+    if X.dtype != torch.bfloat16 or Wr.dtype != torch.float32:
+        raise ValueError("X must be bf16 and Wr fp32")
+    T, K = X.shape
+    S = Wr.shape[1]
+    dev = X.device
+    k_t = torch.empty(T, dtype=torch.int32, device=dev) if k_t is None else k_t
+    perm = torch.empty(T, dtype=torch.int32, device=dev) if perm is None else perm
+    offsets = torch.empty(S + 1, dtype=torch.int32, device=dev) if offsets is None else offsets
+    need = mobi_route_workspace_bytes(T, K, S)
+    ws = _workspace(need, dev, ws) if need > 0 else ws
+    _check("mobi_route", lib().mobi_route(_ptr(X), T, K, _ptr(Wr), _ptr(bias), S, _ptr(k_t), _ptr(perm),
+                                          _ptr(offsets), _ptr(ws), 0 if ws is None else ws.numel(),
+                                          _stream(stream)))
+    return k_t, perm, offsets
+
+
+def mobi_gemm_path(X: torch.Tensor, k_t: torch.Tensor, perm: torch.Tensor, offsets: torch.Tensor,
+                   codes: torch.Tensor, sz: torch.Tensor, N: int, path: int = PATH_AUTO, S: int | None = None,
+                   G: int = 128, Y: torch.Tensor | None = None, ws: torch.Tensor | None = None, stream=None):
+    """Token-routed mixed-bit GEMM y_t = x_t . W^(k_t)^T (fp32) with an explicit kernel choice."""
+    T, K = X.shape
+    S = codes.shape[0] if S is None else S
+    Y = torch.empty((T, N), dtype=torch.float32, device=X.device) if Y is None else Y
+    ws = _workspace(mobi_gemm_workspace_bytes(T, N, K, S), X.device, ws)
+    _check("mobi_gemm", lib().mobi_gemm_path(_ptr(X), T, K, _ptr(k_t), _ptr(perm), _ptr(offsets), _ptr(codes),
+                                             _ptr(sz), N, G, S, _ptr(Y), _ptr(ws), ws.numel(), _stream(stream),
+                                             path))
+    return Y
+
+
+def mobi_gemm(X, k_t, perm, offsets, codes, sz, N, S=None, G=128, Y=None, ws=None, stream=None):
+    """Token-routed mixed-bit GEMM (decode kernel for T <= 16, tcgen05 prefill kernel above)."""
+    return mobi_gemm_path(X, k_t, perm, offsets, codes, sz, N, PATH_AUTO, S, G, Y, ws, stream)
+
+
+def mobi_sync_check(stream=None) -> None:
+    """Synchronise the stream and raise MobiError if a kernel recorded a device-side error."""
+    _check("mobi_sync_check", lib().mobi_sync_check(_stream(stream)))
+
+
+def mobi_debug_set_wait_limit(limit: int) -> None:
+    _check("mobi_debug_set_wait_limit", lib().mobi_debug_set_wait_limit(limit))

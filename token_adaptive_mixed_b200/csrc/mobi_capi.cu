@@ -1,0 +1,273 @@
+// mobi_capi.cu — the C ABI of libmobi (declared in include/mobi.h): argument
+// validation, kernel dispatch, the per-device status word and host helpers.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mobi.h"
+#include "mobi_device.cuh"
+#include "mobi_host.h"
+
+namespace mobi {
+
+// Launchers defined in the kernel files.
+cudaError_t launch_pack(const void* W, int64_t N, int64_t K, int S, uint32_t* codes, uint32_t* sz,
+                        cudaStream_t stream, int num_sms);
+cudaError_t launch_route(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias, int S,
+                         int32_t* k_t, int32_t* perm, int32_t* offsets, void* ws, cudaStream_t stream);
+size_t route_ws_bytes(int64_t T, int64_t K, int S);
+cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
+                          const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
+                          DeviceStatus* st);
+size_t decode_ws_bytes(int64_t N, int64_t K);
+cudaError_t launch_prefill(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
+                           const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int S,
+                           float* Y, void* ws, cudaStream_t stream, DeviceStatus* st);
+size_t prefill_ws_bytes(int64_t T, int64_t N, int64_t K);
+
+// One status block per device, in the module's device memory.
+__device__ DeviceStatus g_device_status;
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_mu;
+static DeviceStatus* g_status_ptr[kMaxDevices];
+static int g_sms[kMaxDevices];
+static std::atomic<uint64_t> g_wait_limit[kMaxDevices];
+
+static int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) return -1;
+  return (d >= 0 && d < kMaxDevices) ? d : -1;
+}
+
+DeviceStatus* device_status(cudaError_t* err) {
+  const int d = current_device();
+  *err = cudaSuccess;
+  if (d < 0) {
+    *err = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_status_ptr[d]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_device_status);
+    if (e != cudaSuccess) {
+      *err = e;
+      return nullptr;
+    }
+    g_status_ptr[d] = static_cast<DeviceStatus*>(p);
+  }
+  return g_status_ptr[d];
+}
+
+uint64_t wait_limit() {
+  const int d = current_device();
+  if (d < 0) return kDefaultWaitLimit;
+  const uint64_t v = g_wait_limit[d].load();
+  return v ? v : kDefaultWaitLimit;
+}
+
+int num_sms() {
+  const int d = current_device();
+  if (d < 0) return 148;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_sms[d]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || v <= 0) v = 148;
+    g_sms[d] = v;
+  }
+  return g_sms[d];
+}
+
+cudaError_t set_smem(const void* func, int bytes) {
+  return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t cols, uint64_t rows,
+                  uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace mobi
+
+using namespace mobi;
+
+namespace {
+
+constexpr int64_t kMaxDim = int64_t(1) << 28;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+mobi_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MOBI_OK;
+  (void)cudaGetLastError();  // clear a sticky launch error
+  return MOBI_ERR_CUDA;
+}
+
+mobi_status check_matrix(int64_t N, int64_t K, int G, int S) {
+  if (N < 0 || K < 0 || S < 1 || S > 3) return MOBI_ERR_INVALID_ARG;
+  if (G != 128) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  if (K % 128 != 0 || N % 16 != 0 || N > kMaxDim || K > kMaxDim) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  return MOBI_OK;
+}
+
+size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+
+}  // namespace
+
+extern "C" {
+
+const char* mobi_status_string(mobi_status st) {
+  switch (st) {
+    case MOBI_OK: return "MOBI_OK";
+    case MOBI_ERR_INVALID_ARG: return "MOBI_ERR_INVALID_ARG";
+    case MOBI_ERR_UNSUPPORTED_SHAPE: return "MOBI_ERR_UNSUPPORTED_SHAPE";
+    case MOBI_ERR_MISALIGNED: return "MOBI_ERR_MISALIGNED";
+    case MOBI_ERR_WORKSPACE: return "MOBI_ERR_WORKSPACE";
+    case MOBI_ERR_CUDA: return "MOBI_ERR_CUDA";
+    case MOBI_ERR_TIMEOUT: return "MOBI_ERR_TIMEOUT";
+  }
+  return "MOBI_ERR_UNKNOWN";
+}
+
+int mobi_version(void) { return 100; }
+
+size_t mobi_codes_bytes(int64_t N, int64_t K, int S) {
+  if (N < 0 || K < 0 || K % 16 != 0 || S < 1 || S > 3) return 0;
+  return (size_t)S * (size_t)N * (size_t)(K / 16) * 4;
+}
+
+size_t mobi_sz_bytes(int64_t N, int64_t K, int S, int G) {
+  if (N < 0 || K < 0 || G <= 0 || K % G != 0 || S < 1 || S > 3) return 0;
+  return (size_t)S * (size_t)N * (size_t)(K / G) * 4;
+}
+
+size_t mobi_route_workspace_bytes(int64_t T, int64_t K, int S) {
+  if (T < 0 || K < 0 || S < 1 || S > 3) return 0;
+  return route_ws_bytes(T, K, S);
+}
+
+size_t mobi_gemm_workspace_bytes(int64_t T, int64_t N, int64_t K, int S) {
+  if (T < 0 || N < 0 || K < 0 || S < 1 || S > 3) return 0;
+  size_t b = decode_ws_bytes(N, K);
+  if (T > 16) {
+    const size_t p = prefill_ws_bytes(T, N, K);
+    if (p > b) b = p;
+  }
+  return align256(b);
+}
+
+mobi_status mobi_pack(const void* W, int64_t N, int64_t K, int G, int S, uint32_t* codes, uint32_t* sz,
+                      void* stream) {
+  mobi_status st = check_matrix(N, K, G, S);
+  if (st != MOBI_OK) return st;
+  if (N == 0 || K == 0) return MOBI_OK;
+  if (!W || !codes || !sz) return MOBI_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(codes) || !aligned16(sz)) return MOBI_ERR_MISALIGNED;
+  return cuda_status(launch_pack(W, N, K, S, codes, sz, static_cast<cudaStream_t>(stream), num_sms()));
+}
+
+mobi_status mobi_route(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias, int S,
+                       int32_t* k_t, int32_t* perm, int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
+  if (T < 0 || K < 0 || S < 1 || S > 3) return MOBI_ERR_INVALID_ARG;
+  if (K % 128 != 0 || K > kMaxDim || T > kMaxDim) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  if (!offsets || (T > 0 && (!X || !Wr || !k_t || !perm))) return MOBI_ERR_INVALID_ARG;
+  if (T > 0 && K == 0) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  if ((X && !aligned16(X)) || (Wr && !aligned16(Wr)) || (bias && !aligned4(bias)) || (k_t && !aligned4(k_t)) ||
+      (perm && !aligned4(perm)) || !aligned4(offsets))
+    return MOBI_ERR_MISALIGNED;
+  const size_t need = route_ws_bytes(T, K, S);
+  if (need > 0 && (!ws || ws_bytes < need)) return MOBI_ERR_WORKSPACE;
+  if (ws && !aligned16(ws)) return MOBI_ERR_MISALIGNED;
+  return cuda_status(
+      launch_route(X, T, K, Wr, bias, S, k_t, perm, offsets, ws, static_cast<cudaStream_t>(stream)));
+}
+
+mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
+                           const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int G,
+                           int S, float* Y, void* ws, size_t ws_bytes, void* stream, int path) {
+  mobi_status st = check_matrix(N, K, G, S);
+  if (st != MOBI_OK) return st;
+  if (T < 0) return MOBI_ERR_INVALID_ARG;
+  if (T > kMaxDim) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  if (path < MOBI_PATH_AUTO || path > MOBI_PATH_PREFILL) return MOBI_ERR_INVALID_ARG;
+  if (T == 0 || N == 0) return MOBI_OK;
+  if (K == 0) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  if (!X || !k_t || !perm || !offsets || !codes || !sz || !Y || !ws) return MOBI_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(codes) || !aligned16(sz) || !aligned16(Y) || !aligned16(ws) ||
+      !aligned4(k_t) || !aligned4(perm) || !aligned4(offsets))
+    return MOBI_ERR_MISALIGNED;
+  const bool decode = path == MOBI_PATH_DECODE || (path == MOBI_PATH_AUTO && T <= 16);
+  if (decode && T > 16) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  const size_t need = decode ? decode_ws_bytes(N, K) : prefill_ws_bytes(T, N, K);
+  if (ws_bytes < need) return MOBI_ERR_WORKSPACE;
+  cudaError_t e;
+  DeviceStatus* dst = device_status(&e);
+  if (!dst) return cuda_status(e);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (decode) return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, ws, s, dst));
+  return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, ws, s, dst));
+}
+
+mobi_status mobi_gemm(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
+                      const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S,
+                      float* Y, void* ws, size_t ws_bytes, void* stream) {
+  return mobi_gemm_path(X, T, K, k_t, perm, offsets, codes, sz, N, G, S, Y, ws, ws_bytes, stream,
+                        MOBI_PATH_AUTO);
+}
+
+mobi_status mobi_sync_check(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_status(e);
+  DeviceStatus* dst = device_status(&e);
+  if (!dst) return cuda_status(e);
+  DeviceStatus h;
+  e = cudaMemcpy(&h, dst, sizeof h, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (h.error == 0) return MOBI_OK;
+  const DeviceStatus zero = {};
+  e = cudaMemcpy(dst, &zero, sizeof zero, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (h.error & kErrTimeout) return MOBI_ERR_TIMEOUT;
+  return MOBI_ERR_INVALID_ARG;  // kErrInputRange: an activation outside the supported range
+}
+
+mobi_status mobi_debug_set_wait_limit(int64_t limit) {
+  if (limit < 0) return MOBI_ERR_INVALID_ARG;
+  const int d = current_device();
+  if (d < 0) return MOBI_ERR_CUDA;
+  g_wait_limit[d].store((uint64_t)limit);
+  return MOBI_OK;
+}
+
+}  // extern "C"

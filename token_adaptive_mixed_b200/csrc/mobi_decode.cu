@@ -1,0 +1,375 @@
+// mobi_decode.cu — decode GEMM (T <= 16 tokens) of the token-routed mixed-bit
+// linear layer on sm_100a.
+//
+// y[t,n] = sum_{s < k_t} sum_g scale[s,g,n] * sum_{k in g} x[t,k] (q[s,n,k] - z[s,g,n])
+// (MoBiQuant explainer [ja] §2.1 W^(b) = sum W_e; [en] §2.A "Elasticity").
+// Only the slices up to the batch's largest k_t are read ([en] §3: fetch only
+// the slices that are needed).
+//
+// Exact operands on the tensor cores. A 2-bit code q sitting at bit 2f of a
+// byte is, read as a bf16 bit pattern, the subnormal value q * 4^f * 2^-133
+// (bf16 values with exponent field 0 or 1 are linear in their bit pattern).
+// So `word & (0x00030003 << 2f)` (after an optional 8-bit shift) is a pair of
+// exact A-operand values, one AND per two weights. The activations are staged
+// once per call as x * 2^96 / 4^f (exact in bf16 for |x| < 2^31), so every
+// product is q * x * 2^-37 exactly and every field carries the same weight.
+// The zero point is folded in once per (row, group): sum_k x (q - z) =
+// sum_k x q - z * sum_k x, with sum_k x prepared in fp64 and rounded once.
+// fp32 accumulation happens in the tensor core (mma.sync m16n8k16) and in the
+// per-group promotion y += scale * 2^37 * acc - scale * z * xsum.
+//
+// Work split: CTA = 64 rows x 8 groups (1024 columns), 4 warps; warp w handles
+// groups 2w, 2w+1 for all four 16-row tiles, so each activation fragment is
+// read from shared memory once and used for 4 tiles x k slices. Codes, scales
+// and the staged activations arrive by TMA, one mbarrier per slice, so slice 0
+// is computed while slices 1..k-1 are still in flight. Column splits are
+// combined deterministically: every CTA writes its partial to the workspace
+// and the last CTA of a row block (atomic ticket) sums them in order.
+#include <cstdint>
+
+#include "mobi_device.cuh"
+#include "mobi_host.h"
+
+namespace mobi {
+
+constexpr int kDecRows = 64;      // rows per CTA
+constexpr int kDecGroups = 8;     // 128-wide groups per CTA
+constexpr int kDecThreads = 128;  // 4 warps
+constexpr float kTwo96 = 79228162514264337593543950336.0f;  // 2^96
+constexpr float kTwo37 = 137438953472.0f;                   // 2^37
+
+// ---- staging of the activations ------------------------------------------------
+//
+// Xd[g][j][lane][nb][2] (uint32 = bf16 pair) is the B fragment of k16 step j
+// (j = 4h + f) of group g for lane (gid = lane/4, t4 = lane%4) and token
+// gid + 8nb. Register ih in {0,1} holds the pair e in {0,1} at physical column
+//   k = 128g + 32 t4 + 16 ih + 4h + f + 8e,
+// scaled by 2^(96 - 2f). xs[g][t] = sum of x[t, group g] (fp64, stored fp32).
+// meta[0] = max k_t; meta[1..] are the per-row-block tickets (zeroed here).
+__global__ void __launch_bounds__(256) decode_prep_kernel(const __nv_bfloat16* __restrict__ X, int T,
+                                                          int64_t K, int NB, const int32_t* __restrict__ k_t,
+                                                          uint32_t* __restrict__ Xd, float* __restrict__ xs,
+                                                          int32_t* __restrict__ meta, int64_t n_tickets,
+                                                          DeviceStatus* st) {
+  const int64_t g = blockIdx.x;
+  const int tid = threadIdx.x;
+  {
+    const int j = tid >> 5, lane = tid & 31;
+    const int gid = lane >> 2, t4 = lane & 3, h = j >> 2, f = j & 3;
+    const float mult = kTwo96 / (float)(1 << (2 * f));
+    bool bad = false;
+    for (int nb = 0; nb < NB; ++nb) {
+      const int tok = gid + 8 * nb;
+      uint32_t reg[2];
+#pragma unroll
+      for (int ih = 0; ih < 2; ++ih) {
+        uint32_t pair = 0;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int64_t k = 128 * g + 32 * t4 + 16 * ih + 4 * h + f + 8 * e;
+          float x = 0.0f;
+          if (tok < T) x = __bfloat162float(X[(int64_t)tok * K + k]);
+          bad |= !(fabsf(x) < 0x1p31f);
+          const __nv_bfloat16 b = __float2bfloat16_rn(x * mult);  // exact: power-of-two scaling
+          pair |= (uint32_t)__bfloat16_as_ushort(b) << (16 * e);
+        }
+        reg[ih] = pair;
+      }
+      uint32_t* dst = Xd + (((g * 8 + j) * 32 + lane) * NB + nb) * 2;
+      dst[0] = reg[0];
+      dst[1] = reg[1];
+    }
+    if (bad) report_error(st, kErrInputRange, 0x100);
+  }
+  {
+    // Group sums: thread (tok = tid/16, part = tid%16) adds 8 columns in fp64,
+    // then a fixed xor tree over the 16 parts.
+    const int tok = tid >> 4, part = tid & 15;
+    double s = 0.0;
+    if (tok < T) {
+      const __nv_bfloat16* p = X + (int64_t)tok * K + 128 * g + 8 * part;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s += (double)__bfloat162float(p[i]);
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (part == 0) xs[g * 16 + tok] = (float)s;
+  }
+  if (g == 0 && tid == 0) {
+    int km = 1;
+    for (int t = 0; t < T; ++t) km = max(km, (int)k_t[t]);
+    meta[0] = km;
+  }
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + tid; i < n_tickets; i += (int64_t)gridDim.x * blockDim.x)
+    meta[1 + i] = 0;
+}
+
+// ---- the decode kernel ------------------------------------------------------------
+
+struct DecSmem {
+  uint32_t codes[3][kDecRows][kDecGroups * 8];   // [slice][row][word]          48 KB
+  uint32_t sz[3][kDecGroups][kDecRows];          // [slice][group][row]          6 KB
+  float xs[kDecGroups][16];                      // group sums                 512 B
+  int32_t kt[16];
+  int32_t is_last;
+  uint64_t bar[3];
+};
+
+__device__ __forceinline__ void mma_bf16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int NB>
+__global__ void __launch_bounds__(kDecThreads) decode_kernel(
+    const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_sz,
+    const uint32_t* __restrict__ Xd, const float* __restrict__ xs_g, const int32_t* __restrict__ k_t,
+    int32_t* __restrict__ meta, int T, int64_t N, int64_t ngroups, int S, float* __restrict__ partial,
+    float* __restrict__ Y, DeviceStatus* st, uint64_t limit) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
+  uint32_t* xd_s = reinterpret_cast<uint32_t*>(smem_raw + sizeof(DecSmem) + (128 - sizeof(DecSmem) % 128) % 128);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gid = lane >> 2, t4 = lane & 3;
+  const int64_t rb = blockIdx.x;                  // row block
+  const int64_t ch = blockIdx.y;                  // column chunk (8 groups)
+  const int nch = gridDim.y;
+  const int64_t g0 = ch * kDecGroups;
+  const int ngc = (int)(ngroups - g0 < kDecGroups ? ngroups - g0 : kDecGroups);
+  const int kmax = min(S, max(1, (int)__ldg(meta)));
+
+  if (tid == 0) {
+    for (int s = 0; s < 3; ++s) mbar_init(&sm.bar[s], 1);
+    fence_barrier_init();
+  }
+  if (tid < 16) sm.kt[tid] = tid < T ? k_t[tid] : 0;
+  __syncthreads();
+
+  if (tid == 0) {
+    const uint32_t xd_bytes = (uint32_t)ngc * 2048u * NB;
+    const uint32_t xs_bytes = (uint32_t)ngc * 64u;
+    for (int s = 0; s < kmax; ++s) {
+      const uint32_t bytes = sizeof(sm.codes[0]) + sizeof(sm.sz[0]) + (s == 0 ? xd_bytes + xs_bytes : 0u);
+      mbar_arrive_expect_tx(&sm.bar[s], bytes);
+      tma_load_2d(&sm.codes[s][0][0], &tm_codes, (int)(g0 * 8), (int)(s * N + rb * kDecRows), &sm.bar[s]);
+      tma_load_2d(&sm.sz[s][0][0], &tm_sz, (int)(rb * kDecRows), (int)(s * ngroups + g0), &sm.bar[s]);
+      if (s == 0) {
+        bulk_g2s(xd_s, Xd + g0 * 2048 / 4 * NB, xd_bytes, &sm.bar[0]);
+        bulk_g2s(&sm.xs[0][0], xs_g + g0 * 16, xs_bytes, &sm.bar[0]);
+      }
+    }
+  }
+
+  float yt[4][4 * NB];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int i = 0; i < 4 * NB; ++i) yt[r][i] = 0.0f;
+
+  bool ok = true;
+  for (int s = 0; s < kmax; ++s) {
+    if (!mbar_wait(&sm.bar[s], 0, limit, st, 0x200 + s)) {
+      ok = false;
+      mbar_wait(&sm.bar[s], 0, kDefaultWaitLimit, st, 0x210 + s);  // drain the copies in flight
+      continue;
+    }
+    if (!ok) continue;
+    float ys[4][4 * NB];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int i = 0; i < 4 * NB; ++i) ys[r][i] = 0.0f;
+
+#pragma unroll
+    for (int gg = 0; gg < 2; ++gg) {
+      const int gi = 2 * warp + gg;
+      if (gi < ngc) {
+        // B fragments of the 8 k16 steps of this group.
+        uint32_t b[8][2 * NB];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t* src = xd_s + ((gi * 8 + j) * 32 + lane) * NB * 2;
+          if constexpr (NB == 2) {
+            const uint4 v = *reinterpret_cast<const uint4*>(src);
+            b[j][0] = v.x; b[j][1] = v.y; b[j][2] = v.z; b[j][3] = v.w;
+          } else {
+            const uint2 v = *reinterpret_cast<const uint2*>(src);
+            b[j][0] = v.x; b[j][1] = v.y;
+          }
+        }
+        float xsv[2 * NB];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          xsv[2 * nb] = sm.xs[gi][2 * t4 + 8 * nb];
+          xsv[2 * nb + 1] = sm.xs[gi][2 * t4 + 1 + 8 * nb];
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int rowA = 16 * r + gid, rowB = rowA + 8;
+          const uint2 wa = *reinterpret_cast<const uint2*>(&sm.codes[s][rowA][gi * 8 + 2 * t4]);
+          const uint2 wb = *reinterpret_cast<const uint2*>(&sm.codes[s][rowB][gi * 8 + 2 * t4]);
+          float d[NB][4];
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) d[nb][0] = d[nb][1] = d[nb][2] = d[nb][3] = 0.0f;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t a0w = wa.x >> (8 * h), a2w = wa.y >> (8 * h);
+            const uint32_t a1w = wb.x >> (8 * h), a3w = wb.y >> (8 * h);
+#pragma unroll
+            for (int f = 0; f < 4; ++f) {
+              const uint32_t m = 0x00030003u << (2 * f);
+              const int j = 4 * h + f;
+#pragma unroll
+              for (int nb = 0; nb < NB; ++nb)
+                mma_bf16_16816(d[nb], a0w & m, a1w & m, a2w & m, a3w & m, b[j][2 * nb], b[j][2 * nb + 1]);
+            }
+          }
+          const uint32_t szA = sm.sz[s][gi][rowA], szB = sm.sz[s][gi][rowB];
+          const float scA = __half2float(__ushort_as_half((unsigned short)(szA & 0xffffu)));
+          const float zA = __half2float(__ushort_as_half((unsigned short)(szA >> 16)));
+          const float scB = __half2float(__ushort_as_half((unsigned short)(szB & 0xffffu)));
+          const float zB = __half2float(__ushort_as_half((unsigned short)(szB >> 16)));
+          const float aA = scA * kTwo37, cA = scA * zA;  // both exact
+          const float aB = scB * kTwo37, cB = scB * zB;
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            ys[r][4 * nb + 0] = fmaf(-cA, xsv[2 * nb], fmaf(aA, d[nb][0], ys[r][4 * nb + 0]));
+            ys[r][4 * nb + 1] = fmaf(-cA, xsv[2 * nb + 1], fmaf(aA, d[nb][1], ys[r][4 * nb + 1]));
+            ys[r][4 * nb + 2] = fmaf(-cB, xsv[2 * nb], fmaf(aB, d[nb][2], ys[r][4 * nb + 2]));
+            ys[r][4 * nb + 3] = fmaf(-cB, xsv[2 * nb + 1], fmaf(aB, d[nb][3], ys[r][4 * nb + 3]));
+          }
+        }
+      }
+    }
+    // Tokens with k_t <= s do not take slice s.
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      const bool m0 = sm.kt[2 * t4 + 8 * nb] > s, m1 = sm.kt[2 * t4 + 1 + 8 * nb] > s;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        if (m0) { yt[r][4 * nb + 0] += ys[r][4 * nb + 0]; yt[r][4 * nb + 2] += ys[r][4 * nb + 2]; }
+        if (m1) { yt[r][4 * nb + 1] += ys[r][4 * nb + 1]; yt[r][4 * nb + 3] += ys[r][4 * nb + 3]; }
+      }
+    }
+  }
+
+  // Cross-warp reduction through shared memory (reuses the code buffer).
+  __syncthreads();
+  float* red = reinterpret_cast<float*>(&sm.codes[0][0][0]);  // [warp][token][row], 16 KB
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int rowA = 16 * r + gid, tk0 = 2 * t4 + 8 * nb;
+      red[(warp * 16 + tk0) * 64 + rowA] = yt[r][4 * nb + 0];
+      red[(warp * 16 + tk0 + 1) * 64 + rowA] = yt[r][4 * nb + 1];
+      red[(warp * 16 + tk0) * 64 + rowA + 8] = yt[r][4 * nb + 2];
+      red[(warp * 16 + tk0 + 1) * 64 + rowA + 8] = yt[r][4 * nb + 3];
+    }
+  __syncthreads();
+  const int ntk = 8 * NB;
+  for (int o = tid; o < ntk * 64; o += kDecThreads) {
+    const int tk = o >> 6, row = o & 63;
+    const int64_t n = rb * kDecRows + row;
+    if (tk < T && n < N) {
+      const float v = red[(0 * 16 + tk) * 64 + row] + red[(1 * 16 + tk) * 64 + row] +
+                      red[(2 * 16 + tk) * 64 + row] + red[(3 * 16 + tk) * 64 + row];
+      if (nch == 1) Y[(int64_t)tk * N + n] = v;
+      else partial[((int64_t)ch * 16 + tk) * N + n] = v;
+    }
+  }
+  if (nch == 1) return;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int ticket = atomicAdd(&meta[1 + rb], 1);
+    sm.is_last = (ticket == nch - 1);
+  }
+  __syncthreads();
+  if (!sm.is_last) return;
+  __threadfence();
+  for (int o = tid; o < ntk * 64; o += kDecThreads) {
+    const int tk = o >> 6, row = o & 63;
+    const int64_t n = rb * kDecRows + row;
+    if (tk < T && n < N) {
+      float v = 0.0f;
+      for (int c = 0; c < nch; ++c) v += __ldcg(&partial[((int64_t)c * 16 + tk) * N + n]);
+      Y[(int64_t)tk * N + n] = v;
+    }
+  }
+  if (tid == 0) meta[1 + rb] = 0;
+}
+
+// ---- host side -----------------------------------------------------------------------
+
+size_t decode_ws_bytes(int64_t N, int64_t K) {
+  const int64_t ngroups = K / 128;
+  const int64_t nch = (ngroups + kDecGroups - 1) / kDecGroups;
+  const int64_t nrb = (N + kDecRows - 1) / kDecRows;
+  size_t b = 0;
+  b += (size_t)ngroups * 2048 * 2;                             // Xd: 2048 * NB bytes per group, NB <= 2
+  b = (b + 255) / 256 * 256;
+  b += (size_t)ngroups * 16 * sizeof(float);                   // xs
+  b = (b + 255) / 256 * 256;
+  b += (size_t)(1 + nrb) * sizeof(int32_t);                    // meta
+  b = (b + 255) / 256 * 256;
+  b += (size_t)nch * 16 * (size_t)N * sizeof(float);           // partials
+  return (b + 255) / 256 * 256;
+}
+
+static size_t dec_smem_bytes(int NB) {
+  size_t b = sizeof(DecSmem);
+  b = (b + 127) / 128 * 128;
+  return b + (size_t)kDecGroups * 2048 * NB;
+}
+
+cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
+                          const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
+                          DeviceStatus* st) {
+  const int64_t ngroups = K / 128;
+  const int64_t nch = (ngroups + kDecGroups - 1) / kDecGroups;
+  const int64_t nrb = (N + kDecRows - 1) / kDecRows;
+  const int NB = T > 8 ? 2 : 1;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  size_t off = 0;
+  uint32_t* Xd = reinterpret_cast<uint32_t*>(p + off);
+  off += (size_t)ngroups * 2048 * 2;
+  off = (off + 255) / 256 * 256;
+  float* xs = reinterpret_cast<float*>(p + off);
+  off += (size_t)ngroups * 16 * sizeof(float);
+  off = (off + 255) / 256 * 256;
+  int32_t* meta = reinterpret_cast<int32_t*>(p + off);
+  off += (size_t)(1 + nrb) * sizeof(int32_t);
+  off = (off + 255) / 256 * 256;
+  float* partial = reinterpret_cast<float*>(p + off);
+
+  CUtensorMap tm_codes, tm_sz;
+  if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4, 64, 64,
+                    false))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, 64, 8, false))
+    return cudaErrorInvalidValue;
+
+  decode_prep_kernel<<<(unsigned)ngroups, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T, K, NB, k_t,
+                                                             Xd, xs, meta, nrb, st);
+  const size_t smem = dec_smem_bytes(NB);
+  dim3 grid((unsigned)nrb, (unsigned)nch);
+  cudaError_t e;
+  if (NB == 2) {
+    if ((e = set_smem((const void*)decode_kernel<2>, (int)smem)) != cudaSuccess) return e;
+    decode_kernel<2><<<grid, kDecThreads, smem, stream>>>(tm_codes, tm_sz, Xd, xs, k_t, meta, T, N, ngroups,
+                                                          S, partial, Y, st, wait_limit());
+  } else {
+    if ((e = set_smem((const void*)decode_kernel<1>, (int)smem)) != cudaSuccess) return e;
+    decode_kernel<1><<<grid, kDecThreads, smem, stream>>>(tm_codes, tm_sz, Xd, xs, k_t, meta, T, N, ngroups,
+                                                          S, partial, Y, st, wait_limit());
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace mobi

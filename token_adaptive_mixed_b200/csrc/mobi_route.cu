@@ -1,0 +1,238 @@
+// mobi_route.cu — MoBiRoute token routing and stable token bucketing on sm_100a.
+//
+// MoBiQuant explainer [ja] §2.2 / [en] §2.B: a router scores every token and
+// the score decides how many residual slices it activates. Here the router is
+// linear: logit_j(t) = sum_k x[t,k] Wr[k,j] + b_j and k_t = 1 + argmax_j
+// (lowest j on an exact tie). Tokens are then stably sorted by k_t.
+//
+// route_partial_kernel: grid (token tiles of 16, K splits), 256 threads. Each
+//   thread owns 8 consecutive columns per 2048-wide pass and accumulates the
+//   x.Wr products of its columns in fp32; the warp reduces in fp32 and the
+//   warps (and K splits) combine in fp64 in a fixed order, so the result is
+//   deterministic and far more accurate than the 1e-5 near-tie band.
+//   Bound: HBM read of X (T*K*2 bytes).
+// bucket_kernel: one CTA. Finishes the K-split logits (if any), takes the
+//   argmax, then counts and scatters the tokens in index order with warp
+//   ballots, which keeps the sort stable.
+#include <cstdint>
+
+#include "mobi_device.cuh"
+
+namespace mobi {
+
+constexpr int kRouteTB = 16;       // tokens per CTA
+constexpr int kRouteThreads = 256;
+constexpr int kRoutePass = 2048;   // columns covered per pass (256 threads x 8)
+
+__device__ __forceinline__ int argmax_lowest(const double* l, int S) {
+  int best = 0;
+  for (int j = 1; j < S; ++j)
+    if (l[j] > l[best]) best = j;
+  return best;
+}
+
+// partial[ks][t][j] (fp64) when ksplit > 1, otherwise k_t directly.
+template <int S>
+__global__ void __launch_bounds__(kRouteThreads) route_partial_kernel(
+    const __nv_bfloat16* __restrict__ X, int64_t T, int64_t K, const float* __restrict__ Wr,
+    const float* __restrict__ bias, int64_t k_per_split, int32_t* __restrict__ k_t,
+    double* __restrict__ partial) {
+  __shared__ float red[kRouteThreads / 32][kRouteTB * S];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t t0 = (int64_t)blockIdx.x * kRouteTB;
+  const int ntok = (int)(T - t0 < kRouteTB ? T - t0 : kRouteTB);
+  const int64_t kbeg = (int64_t)blockIdx.y * k_per_split;
+  const int64_t kend = (K < kbeg + k_per_split) ? K : kbeg + k_per_split;
+
+  float acc[kRouteTB][S];
+#pragma unroll
+  for (int i = 0; i < kRouteTB; ++i)
+#pragma unroll
+    for (int j = 0; j < S; ++j) acc[i][j] = 0.0f;
+
+  for (int64_t k = kbeg + 8 * tid; k < kend; k += kRoutePass) {
+    float w[8][S];
+    const float* wp = Wr + k * S;
+#pragma unroll
+    for (int e = 0; e < 8 * S; ++e) w[e / S][e % S] = __ldg(wp + e);
+#pragma unroll
+    for (int i = 0; i < kRouteTB; ++i) {
+      if (i < ntok) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(X + (t0 + i) * K + k));
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float x0 = bf16lo(u[p]), x1 = bf16hi(u[p]);
+#pragma unroll
+          for (int j = 0; j < S; ++j) {
+            acc[i][j] = fmaf(x0, w[2 * p][j], acc[i][j]);
+            acc[i][j] = fmaf(x1, w[2 * p + 1][j], acc[i][j]);
+          }
+        }
+      }
+    }
+  }
+
+  // Warp reduction (fp32, fixed xor tree), then warps in fp64 in order.
+#pragma unroll
+  for (int i = 0; i < kRouteTB; ++i)
+#pragma unroll
+    for (int j = 0; j < S; ++j) {
+      float v = acc[i][j];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) red[warp][i * S + j] = v;
+    }
+  __syncthreads();
+  if (tid < kRouteTB) {
+    const int i = tid;
+    if (i < ntok) {
+      double l[S];
+#pragma unroll
+      for (int j = 0; j < S; ++j) {
+        double s = 0.0;
+        for (int w8 = 0; w8 < kRouteThreads / 32; ++w8) s += (double)red[w8][i * S + j];
+        l[j] = s;
+      }
+      if (partial != nullptr) {
+#pragma unroll
+        for (int j = 0; j < S; ++j) partial[((int64_t)blockIdx.y * T + t0 + i) * S + j] = l[j];
+      } else {
+#pragma unroll
+        for (int j = 0; j < S; ++j) l[j] += bias ? (double)__ldg(bias + j) : 0.0;
+        k_t[t0 + i] = 1 + argmax_lowest(l, S);
+      }
+    }
+  }
+}
+
+constexpr int kBucketThreads = 1024;
+
+// Single CTA: optional finish of split logits, then the stable counting sort.
+template <int S>
+__global__ void __launch_bounds__(kBucketThreads) bucket_kernel(int64_t T, int ksplit,
+                                                                const double* __restrict__ partial,
+                                                                const float* __restrict__ bias,
+                                                                int32_t* __restrict__ k_t,
+                                                                int32_t* __restrict__ perm,
+                                                                int32_t* __restrict__ offsets) {
+  __shared__ int cnt[S];
+  __shared__ int base[S];
+  __shared__ int warp_cnt[kBucketThreads / 32][S];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  if (ksplit > 1) {
+    for (int64_t t = tid; t < T; t += kBucketThreads) {
+      double l[S];
+#pragma unroll
+      for (int j = 0; j < S; ++j) {
+        double s = 0.0;
+        for (int ks = 0; ks < ksplit; ++ks) s += partial[((int64_t)ks * T + t) * S + j];
+        l[j] = s + (bias ? (double)bias[j] : 0.0);
+      }
+      k_t[t] = 1 + argmax_lowest(l, S);
+    }
+    __syncthreads();
+    __threadfence_block();
+  }
+
+  if (tid < S) cnt[tid] = 0;
+  __syncthreads();
+  int local[S];
+#pragma unroll
+  for (int j = 0; j < S; ++j) local[j] = 0;
+  for (int64_t t = tid; t < T; t += kBucketThreads) {
+    const int k = k_t[t];
+#pragma unroll
+    for (int j = 0; j < S; ++j) local[j] += (k == j + 1);
+  }
+#pragma unroll
+  for (int j = 0; j < S; ++j) {
+    int v = local[j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) atomicAdd(&cnt[j], v);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int j = 0; j < S; ++j) {
+      offsets[j] = run;
+      base[j] = run;
+      run += cnt[j];
+    }
+    offsets[S] = run;
+  }
+  __syncthreads();
+
+  // Stable scatter, one chunk of 1024 tokens at a time, in token order.
+  for (int64_t c0 = 0; c0 < T; c0 += kBucketThreads) {
+    const int64_t t = c0 + tid;
+    const int k = t < T ? k_t[t] : 0;
+    unsigned my_rank = 0;
+#pragma unroll
+    for (int j = 0; j < S; ++j) {
+      const unsigned m = __ballot_sync(0xffffffffu, k == j + 1);
+      if (k == j + 1) my_rank = __popc(m & ((1u << lane) - 1u));
+      if (lane == 0) warp_cnt[warp][j] = __popc(m);
+    }
+    __syncthreads();
+    if (tid < S) {  // exclusive scan over warps for value tid+1
+      int run = 0;
+      for (int w = 0; w < kBucketThreads / 32; ++w) {
+        const int c = warp_cnt[w][tid];
+        warp_cnt[w][tid] = run;
+        run += c;
+      }
+      cnt[tid] = run;  // chunk total
+    }
+    __syncthreads();
+    if (t < T) perm[base[k - 1] + warp_cnt[warp][k - 1] + (int)my_rank] = (int32_t)t;
+    __syncthreads();
+    if (tid < S) base[tid] += cnt[tid];
+    __syncthreads();
+  }
+}
+
+int route_ksplit(int64_t T, int64_t K) {
+  const int64_t tiles = (T + kRouteTB - 1) / kRouteTB;
+  if (tiles == 0 || tiles >= 64) return 1;
+  int64_t ks = (K + 1023) / 1024;
+  const int64_t want = (128 + tiles - 1) / tiles;
+  if (ks > want) ks = want;
+  if (ks < 1) ks = 1;
+  return (int)ks;
+}
+
+size_t route_ws_bytes(int64_t T, int64_t K, int S) {
+  const int ks = route_ksplit(T, K);
+  return ks > 1 ? (size_t)ks * (size_t)T * (size_t)S * sizeof(double) : 0;
+}
+
+template <int S>
+static cudaError_t launch_route_s(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
+                                  int32_t* k_t, int32_t* perm, int32_t* offsets, void* ws,
+                                  cudaStream_t stream) {
+  const int ks = route_ksplit(T, K);
+  int64_t kps = (K + ks - 1) / ks;
+  kps = (kps + 7) / 8 * 8;  // whole 8-column octets per split
+  double* partial = ks > 1 ? static_cast<double*>(ws) : nullptr;
+  if (T > 0) {
+    dim3 grid((unsigned)((T + kRouteTB - 1) / kRouteTB), (unsigned)ks);
+    route_partial_kernel<S><<<grid, kRouteThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(X), T, K, Wr, bias, kps, k_t, partial);
+  }
+  bucket_kernel<S><<<1, kBucketThreads, 0, stream>>>(T, ks, partial, bias, k_t, perm, offsets);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias, int S,
+                         int32_t* k_t, int32_t* perm, int32_t* offsets, void* ws, cudaStream_t stream) {
+  switch (S) {
+    case 1: return launch_route_s<1>(X, T, K, Wr, bias, k_t, perm, offsets, ws, stream);
+    case 2: return launch_route_s<2>(X, T, K, Wr, bias, k_t, perm, offsets, ws, stream);
+    default: return launch_route_s<3>(X, T, K, Wr, bias, k_t, perm, offsets, ws, stream);
+  }
+}
+
+}  // namespace mobi
