@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the MoBiQuant token-routed mixed-bit linear layer on B200.
+
+Metric: "mixed-bit GEMM: decode HBM GB/s & prefill TFLOP/s, % of B200 roofline".
+Workload of the headline line: the decode GEMV workload — Llama-7B-shaped
+projections (N, K) = (4096, 4096), (11008, 4096), (4096, 11008), each for
+T = 1, 4 and 16 tokens (bf16 X ~ N(0,1), fp16 W ~ N(0, 0.02^2) with 0.5%
+outlier input columns x10, 3 x 2-bit slices, group 128, router N(0, 1/K)).
+
+One step = the per-token hot path over all nine (shape, T) cases: MoBiRoute
+(routing + stable bucketing) and the mixed-bit GEMM that streams only the
+slices the batch needs. Packing (MoBiSlice) is the one-time conversion of a
+checkpoint; it is timed in the same run and reported under "pack".
+value = decode algorithmic bytes of all ranks / max-over-ranks step time, with
+decode bytes per GEMV = sum_{s <= k_max} (N*K/4 + N*(K/128)*4) + T*K*2.
+Every call of a step reads its own packed copy, and a copy is reused only
+after ~270 MB of other traffic, which exceeds twice the 126 MB L2.
+
+--impl reference times the CPU oracle on the machine's host cores on a bounded
+sample of the same workload (the only other place this file runs the oracle).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "mixed-bit GEMM: decode HBM GB/s & prefill TFLOP/s, % of B200 roofline"
+WORKLOAD = ("decode GEMV, Llama-7B projections (N,K) in {(4096,4096),(11008,4096),(4096,11008)} "
+            "x T in {1,4,16}, 3x2-bit slices, group 128, route+bucket+GEMM per call")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0)), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def decode_bytes(N, K, T, kmax):
+    return kmax * (N * K // 4 + N * (K // 128) * 4) + T * K * 2
+
+
+class ClockSampler:
+    """NVML samples of SM clock and throttle reasons while the timed region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self._stop = period_s, threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML unavailable: report no clocks rather than guess
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            r = self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+            for name, bit in self.REASONS.items():
+                if r & bit:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def __enter__(self):
+        if self.nv:
+            self._sample()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv:
+            self._stop.set()
+            self.t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---- the decode workload on the GPU ----------------------------------------------------
+
+class DecodeCase:
+    def __init__(self, mobi, wl, N, K, T, codes, sz, dev):
+        L = wl.decode(N, K, T)
+        self.N, self.K, self.T = N, K, T
+        self.X = L.X.to(dev)
+        self.X_host = L.X.pin_memory()
+        self.Wr = torch.from_numpy(L.Wr).to(dev)
+        self.codes, self.sz = codes, sz
+        self.k_t = torch.empty(T, dtype=torch.int32, device=dev)
+        self.perm = torch.empty(T, dtype=torch.int32, device=dev)
+        self.off = torch.empty(4, dtype=torch.int32, device=dev)
+        self.Y = torch.empty((T, N), dtype=torch.float32, device=dev)
+        self.Y_host = torch.empty((T, N), dtype=torch.float32).pin_memory()
+        self.ws_r = torch.empty(max(mobi.mobi_route_workspace_bytes(T, K, 3), 16), dtype=torch.uint8, device=dev)
+        self.ws_g = torch.empty(mobi.mobi_gemm_workspace_bytes(T, N, K, 3), dtype=torch.uint8, device=dev)
+        self.mobi = mobi
+
+    def route(self):
+        self.mobi.mobi_route(self.X, self.Wr, None, self.k_t, self.perm, self.off, self.ws_r)
+
+    def gemm(self):
+        self.mobi.mobi_gemm(self.X, self.k_t, self.perm, self.off, self.codes, self.sz, self.N, Y=self.Y, ws=self.ws_g)
+
+    def step(self):
+        self.route()
+        self.gemm()
+
+    def kmax(self):
+        return int(self.k_t.max().item())
+
+
+def build_decode_cases(mobi, wl, dev):
+    cases = []
+    for (N, K) in wl.DECODE_SHAPES:
+        L = wl.decode(N, K, 1)
+        W = torch.from_numpy(L.W).to(dev)
+        for T in wl.DECODE_TOKENS:  # one packed copy per call: rotation beyond L2
+            codes, sz = mobi.mobi_pack(W, S=3)
+            cases.append(DecodeCase(mobi, wl, N, K, T, codes, sz, dev))
+        del W
+    torch.cuda.synchronize()
+    return cases
+
+
+def time_pack(mobi, wl, dev, reps=10):
+    N, K = 11008, 4096
+    W = torch.from_numpy(wl.decode(N, K, 1).W).to(dev)
+    codes = torch.empty((3, N, K // 16), dtype=torch.int32, device=dev)
+    sz = torch.empty((3, K // 128, N), dtype=torch.int32, device=dev)
+    for _ in range(3):
+        mobi.mobi_pack(W, 3, codes=codes, sz=sz)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        mobi.mobi_pack(W, 3, codes=codes, sz=sz)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    nbytes = N * K * 2 + codes.numel() * 4 + sz.numel() * 4
+    return {"shape": [N, K], "ms": ms, "GB/s": nbytes / ms / 1e6, "bytes": nbytes,
+            "weights_per_s": N * K / ms * 1e3}
+
+
+def run_gpu(args, world, rank):
+    import token_adaptive_mixed_b200 as mobi
+    from token_adaptive_mixed_b200 import build as mobi_build
+    from token_adaptive_mixed_b200 import workloads as wl
+
+    if rank == 0:
+        mobi_build.build()
+    barrier(world)
+    mobi.lib()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    hbm_peak, tf_peak, tf_sust, peak_kind = peaks()
+
+    cases = build_decode_cases(mobi, wl, dev)
+    for c in cases:
+        c.step()
+    mobi.mobi_sync_check()
+    kmax = [c.kmax() for c in cases]
+    bytes_step = sum(decode_bytes(c.N, c.K, c.T, km) for c, km in zip(cases, kmax))
+
+    # Capture one step (9 x (route + GEMM) = 36 kernel launches) in a CUDA graph.
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            for c in cases:
+                c.step()
+    torch.cuda.current_stream().wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for c in cases:
+            c.step()
+    launches_per_step = 4 * len(cases)
+
+    for _ in range(max(args.warmup, 3)):
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record()
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ms_local = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    value = world * bytes_step / (ms * 1e-3) / 1e9
+
+    # Roofline of the dominant kernel pair (staging + decode GEMM kernels): events
+    # around each mobi_gemm on the launching stream, rotating through the cases.
+    per_case_ms = []
+    reps = 20
+    for c in cases:
+        c.gemm()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps * len(cases))]
+    i = 0
+    for r in range(reps):
+        for c in cases:
+            ev[i][0].record()
+            c.gemm()
+            ev[i][1].record()
+            i += 1
+    torch.cuda.synchronize()
+    for ci, c in enumerate(cases):
+        per_case_ms.append(statistics.mean(ev[r * len(cases) + ci][0].elapsed_time(ev[r * len(cases) + ci][1])
+                                           for r in range(reps)))
+    gemm_ms = sum(per_case_ms)
+    achieved = bytes_step / (gemm_ms * 1e-3) / 1e9
+
+    # End to end through the public API with host buffers (pinned), copies inside.
+    h2d = sum(c.T * c.K * 2 for c in cases)
+    d2h = sum(c.T * c.N * 4 for c in cases)
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step():
+        for c in cases:
+            c.X.copy_(c.X_host, non_blocking=True)
+            c.step()
+            c.Y_host.copy_(c.Y, non_blocking=True)
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e_value = world * bytes_step / (e2e_ms * 1e-3) / 1e9
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "bytes_per_step": bytes_step, "kmax_per_call": kmax,
+                   "l2": "rotating packed copies, ~270 MB between reuses (> 2x L2)",
+                   "timing": "CUDA graph of one step, CUDA events, max over ranks", "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "kernel": "decode GEMM (staging + mma.sync decode kernels)",
+                     "achieved": round(achieved, 2), "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "frac_of_8TBs_nominal": round(achieved / 8000.0, 4),
+                     "traffic": None, "per_call_us": [round(1e3 * x, 2) for x in per_case_ms]},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        out["pack"] = time_pack(mobi, wl, dev)
+    return out
+
+
+# ---- the oracle on the host cores ------------------------------------------------------
+
+def oracle_decode_sample(budget_s: float, cases_spec, rows_cap=None):
+    """Time the CPU oracle (route + GEMM) on a bounded sample of the decode workload.
+    Returns (bytes credited, seconds, threads, description)."""
+    import oracle
+    from token_adaptive_mixed_b200 import workloads as wl
+    threads = oracle.max_threads()
+    credited, spent, done = 0, 0.0, []
+    for (N, K, T) in cases_spec:
+        if spent >= budget_s:
+            break
+        L = wl.decode(N, K, T)
+        rows = N if rows_cap is None else min(N, rows_cap)
+        c_sub, s_sub, _ = oracle.pack(np.ascontiguousarray(L.W[:rows]), S=3)
+        t0 = time.perf_counter()
+        k, _, _ = oracle.route(L.X, L.Wr)
+        oracle.gemm(L.X, k, c_sub, s_sub, rows)
+        dt = time.perf_counter() - t0
+        km = int(k.max())
+        credited += km * (rows * K // 4 + rows * (K // 128) * 4) + T * K * 2
+        spent += dt
+        done.append(f"{rows}/{N}x{K} T={T}")
+    return credited, spent, threads, "; ".join(done)
+
+
+def cpu_baseline(budget_s=20.0):
+    from token_adaptive_mixed_b200 import workloads as wl
+    spec = [(N, K, T) for (N, K) in wl.DECODE_SHAPES for T in wl.DECODE_TOKENS]
+    credited, spent, threads, desc = oracle_decode_sample(budget_s, spec, rows_cap=1024)
+    return {"value": round(credited / spent / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"oracle route + fp64 GEMM on the first 1024 rows of each decode case until ~{budget_s:.0f}s: "
+                      f"{desc}; {spent:.1f}s"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    from token_adaptive_mixed_b200 import workloads as wl
+    import oracle
+    oracle.build()
+    spec = [(N, K, T) for (N, K) in wl.DECODE_SHAPES for T in wl.DECODE_TOKENS]
+    per_step_budget = max(0.2, 150.0 / max(1, args.steps + args.warmup))
+    # rows per step sized so one sampled case fits the per-step budget (4096x4096 T=16 ~ 1 s per 1024 rows)
+    rows = int(max(16, min(4096, 1024 * per_step_budget)))
+    rows -= rows % 16
+    for i in range(args.warmup):
+        oracle_decode_sample(1e9, [spec[i % len(spec)]], rows_cap=rows)
+    tot_b, tot_s = 0, 0.0
+    for i in range(args.steps):
+        b, s, threads, desc = oracle_decode_sample(1e9, [spec[i % len(spec)]], rows_cap=rows)
+        tot_b += b
+        tot_s += s
+    value = tot_b / tot_s / 1e9
+    return {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.max_threads(),
+                             "kind": "oracle",
+                             "sample": f"per step: oracle route + fp64 GEMM on the first {rows} rows of one decode case, "
+                                       f"cycling through the nine cases"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="mobi", choices=["mobi", "reference"])
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out))
+        return
+
+    world, rank, _ = dist_setup(args.gpus)
+    out = run_gpu(args, world, rank)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(args.cpu_baseline_seconds)
+        print(json.dumps(out))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -90,6 +90,11 @@ typedef enum {
 /* Human-readable name of a status (static storage, never NULL). */
 MOBI_API const char* mobi_status_string(mobi_status st);
 
+/* Description of the most recent failure seen by a libmobi call on the
+ * calling thread (the failing CUDA call or check, and the CUDA error name);
+ * empty when none. Static thread-local storage, never NULL. */
+MOBI_API const char* mobi_last_error(void);
+
 /* Library version as an integer MAJOR*10000 + MINOR*100 + PATCH. */
 MOBI_API int mobi_version(void);
 

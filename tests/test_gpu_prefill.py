@@ -1,0 +1,130 @@
+"""GPU parity of the tcgen05 prefill GEMM against the CPU oracle.
+
+Sizes span several weight tiles (128 rows) and token tiles (192 tokens) with
+ragged tails, every mix of slice counts, tokens unsorted (the routing order is
+applied inside), and the full prefill workloads on sampled tokens. The bar is
+max |y - y_ref| <= 1e-2 (|y_ref| + 1e-3) element-wise and a relative
+Frobenius error <= 2e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+from parity import check_gemm, check_route
+from token_adaptive_mixed_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def mobi():
+    import token_adaptive_mixed_b200 as m
+    from token_adaptive_mixed_b200 import build
+    build.build()
+    m.lib()
+    return m
+
+
+def u32(a):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int32)).to(DEV)
+
+
+def bucket_host(k):
+    perm = np.argsort(k, kind="stable").astype(np.int32)
+    off = np.concatenate([[0], np.cumsum(np.bincount(k, minlength=4)[1:])]).astype(np.int32)
+    return perm, off
+
+
+def gemm(mobi, X, k, codes, sz, N, path):
+    perm, off = bucket_host(k)
+    Y = mobi.mobi_gemm_path(X.to(DEV), torch.from_numpy(k).to(DEV), torch.from_numpy(perm).to(DEV),
+                            torch.from_numpy(off).to(DEV), u32(codes), u32(sz), N, path=path)
+    mobi.mobi_sync_check()
+    return Y.cpu().numpy()
+
+
+@pytest.mark.parametrize("N,K,T", [(128, 128, 17), (256, 384, 100), (272, 1152, 191), (128, 256, 192),
+                                   (384, 640, 193), (144, 2048, 500), (512, 512, 1000)])
+def test_prefill_shapes(mobi, oracle, N, K, T):
+    L = wl.layer("p", N, K, T, seed=N * 7 + K + T, outlier_frac_cols=0.005)
+    codes, sz, _ = oracle.pack(L.W, S=3)
+    k = np.random.default_rng(T).integers(1, 4, T).astype(np.int32)
+    Y = gemm(mobi, L.X, k, codes, sz, N, path=2)
+    check_gemm(Y, oracle.gemm(L.X, k, codes, sz, N), f"prefill N={N} K={K} T={T}")
+
+
+@pytest.mark.parametrize("mix", [(1, 0, 0), (0, 0, 1), (0, 1, 0), (0.7, 0.2, 0.1), (0.1, 0.1, 0.8)])
+def test_prefill_bucket_mixes(mobi, oracle, mix):
+    """Empty buckets, single-bucket batches and skewed mixes."""
+    N, K, T = 256, 512, 400
+    L = wl.layer("m", N, K, T, seed=55, outlier_frac_cols=0.01)
+    codes, sz, _ = oracle.pack(L.W, S=3)
+    rng = np.random.default_rng(3)
+    k = (rng.choice(3, T, p=np.array(mix) / sum(mix)) + 1).astype(np.int32)
+    Y = gemm(mobi, L.X, k, codes, sz, N, path=2)
+    check_gemm(Y, oracle.gemm(L.X, k, codes, sz, N), f"mix {mix}")
+
+
+@pytest.mark.parametrize("T", [1, 7, 16])
+def test_prefill_matches_decode_small_T(mobi, oracle, T):
+    """Both kernels on the same small batch: each within the bar of the oracle."""
+    L = wl.tiny(T)
+    codes, sz, _ = oracle.pack(L.W, S=3)
+    k, _, _ = oracle.route(L.X, L.Wr)
+    ref = oracle.gemm(L.X, k, codes, sz, L.N)
+    check_gemm(gemm(mobi, L.X, k, codes, sz, L.N, path=2), ref, "prefill")
+    check_gemm(gemm(mobi, L.X, k, codes, sz, L.N, path=1), ref, "decode")
+
+
+def test_prefill_one_slice(mobi, oracle):
+    """S = 1 packing: a plain 2-bit RTN GEMM."""
+    N, K, T = 128, 256, 64
+    L = wl.layer("s1", N, K, T, seed=8)
+    codes, sz, _ = oracle.pack(L.W, S=1)
+    k = np.ones(T, np.int32)
+    perm, off = np.arange(T, dtype=np.int32), np.array([0, T], np.int32)
+    Y = mobi.mobi_gemm_path(L.X.to(DEV), torch.from_numpy(k).to(DEV), torch.from_numpy(perm).to(DEV),
+                            torch.from_numpy(off).to(DEV), u32(codes), u32(sz), N, path=2, S=1)
+    mobi.mobi_sync_check()
+    check_gemm(Y.cpu().numpy(), oracle.gemm(L.X, k, codes, sz, N, S=1), "S=1")
+
+
+def _full_workload(mobi, oracle, L, n_sample):
+    W = torch.from_numpy(L.W).to(DEV)
+    codes_t, sz_t = mobi.mobi_pack(W, S=3)
+    X = L.X.to(DEV)
+    b = None if L.bias is None else torch.from_numpy(L.bias).to(DEV)
+    k_t, perm, off = mobi.mobi_route(X, torch.from_numpy(L.Wr).to(DEV), b)
+    Y = mobi.mobi_gemm(X, k_t, perm, off, codes_t, sz_t, L.N)
+    mobi.mobi_sync_check()
+    codes = codes_t.cpu().numpy().view(np.uint32)
+    sz = sz_t.cpu().numpy().view(np.uint32)
+    rows = np.random.default_rng(1).choice(L.N, 48, replace=False)
+    c_ref, s_ref, _ = oracle.pack(L.W[rows], S=3)
+    assert np.array_equal(codes[:, rows], c_ref) and np.array_equal(sz[:, :, rows], s_ref)
+    k_ref, gap, _ = oracle.route(L.X, L.Wr, L.bias)
+    k_gpu = k_t.cpu().numpy()
+    check_route(k_gpu, k_ref, gap)
+    # sampled tokens: some from every bucket, plus the first and last
+    rng = np.random.default_rng(2)
+    toks = [0, L.T - 1]
+    for j in (1, 2, 3):
+        idx = np.nonzero(k_gpu == j)[0]
+        if idx.size:
+            toks += list(rng.choice(idx, min(n_sample // 3, idx.size), replace=False))
+    toks = np.array(sorted(set(int(t) for t in toks)), np.int32)
+    ref = oracle.gemm(L.X, k_gpu, codes, sz, L.N, tokens=toks)
+    return check_gemm(Y.cpu().numpy()[toks], ref, L.name)
+
+
+@pytest.mark.slow
+def test_prefill_workload_full_size(mobi, oracle):
+    """T=2048, N=11008, K=4096, thirds: sampled tokens against the oracle (all N)."""
+    _full_workload(mobi, oracle, wl.prefill(), 24)
+
+
+@pytest.mark.slow
+def test_skewed_prefill_workload_full_size(mobi, oracle):
+    """T=4096, N=28672, K=8192, 70/20/10 with 2% tokens x8: sampled tokens."""
+    _full_workload(mobi, oracle, wl.skewed_prefill(), 12)

@@ -22,7 +22,7 @@ import torch
 
 __all__ = [
     "MobiError", "lib", "mobi_version", "mobi_status_string", "mobi_codes_bytes", "mobi_sz_bytes",
-    "mobi_route_workspace_bytes", "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm",
+    "mobi_route_workspace_bytes", "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm", "mobi_last_error",
     "mobi_gemm_path", "mobi_sync_check", "mobi_debug_set_wait_limit", "PATH_AUTO", "PATH_DECODE",
     "PATH_PREFILL", "EXPORTED_SYMBOLS",
 ]
@@ -36,17 +36,17 @@ STATUS_NAMES = ["MOBI_OK", "MOBI_ERR_INVALID_ARG", "MOBI_ERR_UNSUPPORTED_SHAPE",
 
 # Every symbol include/mobi.h declares.
 EXPORTED_SYMBOLS = (
-    "mobi_status_string", "mobi_version", "mobi_codes_bytes", "mobi_sz_bytes", "mobi_route_workspace_bytes",
+    "mobi_status_string", "mobi_last_error", "mobi_version", "mobi_codes_bytes", "mobi_sz_bytes", "mobi_route_workspace_bytes",
     "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm", "mobi_gemm_path", "mobi_sync_check",
     "mobi_debug_set_wait_limit",
 )
 
 
 class MobiError(RuntimeError):
-    def __init__(self, fn: str, status: int):
+    def __init__(self, fn: str, status: int, detail: str = ""):
         self.status = status
         name = STATUS_NAMES[status] if 0 <= status < len(STATUS_NAMES) else f"status {status}"
-        super().__init__(f"{fn}: {name}")
+        super().__init__(f"{fn}: {name}" + (f" [{detail}]" if detail else ""))
 
 
 _lib = None
@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         p, i64, ci, sz_t = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
         L.mobi_status_string.argtypes = [ci]
         L.mobi_status_string.restype = ctypes.c_char_p
+        L.mobi_last_error.argtypes = []
+        L.mobi_last_error.restype = ctypes.c_char_p
         L.mobi_version.argtypes = []
         L.mobi_version.restype = ci
         L.mobi_codes_bytes.argtypes = [i64, i64, ci]
@@ -91,7 +93,7 @@ def lib() -> ctypes.CDLL:
 
 def _check(fn: str, status: int) -> None:
     if status != 0:
-        raise MobiError(fn, status)
+        raise MobiError(fn, status, lib().mobi_last_error().decode(errors="replace"))
 
 
 def _ptr(t: torch.Tensor | None):
@@ -116,6 +118,10 @@ def mobi_version() -> int:
 
 def mobi_status_string(status: int) -> str:
     return lib().mobi_status_string(status).decode()
+
+
+def mobi_last_error() -> str:
+    return lib().mobi_last_error().decode(errors="replace")
 
 
 def mobi_codes_bytes(N: int, K: int, S: int = 3) -> int:

@@ -6,6 +6,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -29,6 +30,14 @@ cudaError_t launch_prefill(const void* X, int64_t T, int64_t K, const int32_t* k
                            const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int S,
                            float* Y, void* ws, cudaStream_t stream, DeviceStatus* st);
 size_t prefill_ws_bytes(int64_t T, int64_t N, int64_t K);
+
+static thread_local char g_last_error[256];
+
+cudaError_t note_error(const char* where, cudaError_t e) {
+  if (e != cudaSuccess) snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", where, cudaGetErrorName(e),
+                                 cudaGetErrorString(e));
+  return e;
+}
 
 // One status block per device, in the module's device memory.
 __device__ DeviceStatus g_device_status;
@@ -85,7 +94,8 @@ int num_sms() {
 }
 
 cudaError_t set_smem(const void* func, int bytes) {
-  return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  return note_error("cudaFuncSetAttribute(max dynamic shared memory)",
+                    cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -114,6 +124,11 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t c
   CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    snprintf(g_last_error, sizeof g_last_error,
+             "cuTensorMapEncodeTiled: CUresult %d (dims %llu x %llu, stride %llu, box %u x %u, swizzle %d)", (int)r,
+             (unsigned long long)cols, (unsigned long long)rows, (unsigned long long)row_stride_bytes, box_cols,
+             box_rows, (int)swizzle128);
   return r == CUDA_SUCCESS;
 }
 
@@ -130,6 +145,7 @@ bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0
 
 mobi_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return MOBI_OK;
+  if (!g_last_error[0]) note_error("CUDA", e);
   (void)cudaGetLastError();  // clear a sticky launch error
   return MOBI_ERR_CUDA;
 }
@@ -160,6 +176,8 @@ const char* mobi_status_string(mobi_status st) {
   return "MOBI_ERR_UNKNOWN";
 }
 
+const char* mobi_last_error(void) { return g_last_error; }
+
 int mobi_version(void) { return 100; }
 
 size_t mobi_codes_bytes(int64_t N, int64_t K, int S) {
@@ -189,6 +207,7 @@ size_t mobi_gemm_workspace_bytes(int64_t T, int64_t N, int64_t K, int S) {
 
 mobi_status mobi_pack(const void* W, int64_t N, int64_t K, int G, int S, uint32_t* codes, uint32_t* sz,
                       void* stream) {
+  g_last_error[0] = 0;
   mobi_status st = check_matrix(N, K, G, S);
   if (st != MOBI_OK) return st;
   if (N == 0 || K == 0) return MOBI_OK;
@@ -199,6 +218,7 @@ mobi_status mobi_pack(const void* W, int64_t N, int64_t K, int G, int S, uint32_
 
 mobi_status mobi_route(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias, int S,
                        int32_t* k_t, int32_t* perm, int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
   if (T < 0 || K < 0 || S < 1 || S > 3) return MOBI_ERR_INVALID_ARG;
   if (K % 128 != 0 || K > kMaxDim || T > kMaxDim) return MOBI_ERR_UNSUPPORTED_SHAPE;
   if (!offsets || (T > 0 && (!X || !Wr || !k_t || !perm))) return MOBI_ERR_INVALID_ARG;
@@ -216,6 +236,7 @@ mobi_status mobi_route(const void* X, int64_t T, int64_t K, const float* Wr, con
 mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
                            const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int G,
                            int S, float* Y, void* ws, size_t ws_bytes, void* stream, int path) {
+  g_last_error[0] = 0;
   mobi_status st = check_matrix(N, K, G, S);
   if (st != MOBI_OK) return st;
   if (T < 0) return MOBI_ERR_INVALID_ARG;

@@ -369,7 +369,7 @@ cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, c
     decode_kernel<1><<<grid, kDecThreads, smem, stream>>>(tm_codes, tm_sz, Xd, xs, k_t, meta, T, N, ngroups,
                                                           S, partial, Y, st, wait_limit());
   }
-  return cudaGetLastError();
+  return note_error("kernel launch", cudaGetLastError());
 }
 
 }  // namespace mobi

@@ -24,7 +24,7 @@ struct DeviceStatus {
   uint64_t wait_limit;
 };
 
-constexpr uint64_t kDefaultWaitLimit = 1ull << 26;  // ~ seconds of polling: far above any real wait
+constexpr uint64_t kDefaultWaitLimit = 1ull << 24;  // seconds of polling: far above any real wait
 
 __device__ __forceinline__ void report_error(DeviceStatus* st, uint32_t bit, uint32_t where) {
   if ((atomicOr(&st->error, bit) & bit) == 0) st->where = where;

@@ -15,6 +15,8 @@ namespace mobi {
 DeviceStatus* device_status(cudaError_t* err);
 // Wait limit for bounded device waits on the current device.
 uint64_t wait_limit();
+// Record a failure description for mobi_last_error (thread-local) and return e.
+cudaError_t note_error(const char* where, cudaError_t e);
 // Multiprocessor count of the current device (cached).
 int num_sms();
 // Opt a kernel into `bytes` of dynamic shared memory (idempotent).

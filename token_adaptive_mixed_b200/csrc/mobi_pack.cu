@@ -16,6 +16,7 @@
 #include <cstdint>
 
 #include "mobi_device.cuh"
+#include "mobi_host.h"
 
 namespace mobi {
 
@@ -110,7 +111,7 @@ cudaError_t launch_pack(const void* W, int64_t N, int64_t K, int S, uint32_t* co
   if (blocks < 1) blocks = 1;
   pack_kernel<<<(unsigned)blocks, 32 * warps_per_block, 0, stream>>>(
       static_cast<const __half*>(W), N, K, S, codes, sz);
-  return cudaGetLastError();
+  return note_error("kernel launch", cudaGetLastError());
 }
 
 }  // namespace mobi

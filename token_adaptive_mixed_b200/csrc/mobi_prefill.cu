@@ -1,18 +1,487 @@
-// mobi_prefill.cu — prefill GEMM (T > 16) of the token-routed mixed-bit layer.
-// The tcgen05 kernel is not in this file yet; the launcher reports "not supported".
+// mobi_prefill.cu — prefill GEMM (any T, used for T > 16) of the token-routed
+// mixed-bit linear layer on sm_100a: tcgen05 tensor cores, TMEM accumulators,
+// TMA-staged tiles.
+//
+// y[t,n] = sum_{s < k_t} sum_g scale[s,g,n] * sum_{k in g} x[t,k] (q[s,n,k] - z[s,g,n])
+// (MoBiQuant explainer [ja] §2.1 W^(b) = sum W_e; [en] §2.A "Elasticity"),
+// fp32 accumulation, exact operands.
+//
+// Tokens are taken in bucket order (perm from the routing step, ascending
+// k_t). A tile is 128 weight rows x 192 consecutive bucket-ordered tokens; for
+// group g and slice s < kmax(tile) one "unit" computes
+//   D[n, t] = sum_{k in g} (q - z)[s, n, k] * x[t, k]
+// with 8 tcgen05.mma (M=128, N=192, K=16, bf16 in, fp32 in TMEM), and the
+// epilogue promotes acc[n, t] += scale[s,g,n] * D[n, t] for the tokens that take
+// slice s (a suffix of the tile's columns, since tokens are sorted by k_t).
+//
+// Operands:
+//   A (weights) lives in tensor memory: four dequant warps turn the 2-bit codes
+//     of their rows into exact bf16 (q - z) pairs — (word >> 2c) & 0x00030003
+//     | 0x43004300 is the pair (128 + q) as bf16, and one bf16x2 subtraction of
+//     (128 + z) gives q - z exactly — and write them with tcgen05.st, so the
+//     dequantised operand never touches shared memory.
+//   B (tokens) comes from shared memory: x tiles staged by TMA with 128-byte
+//     swizzle from a gathered copy Xb of the activations, rows in bucket order
+//     and, within each 16-column block, columns interleaved as (c, c+8) to
+//     match the pair order of the packed words.
+// Warp roles (16 warps): 0 TMA producer, 1 MMA issuer (also owns TMEM),
+// 4-7 dequant (one per TMEM lane quadrant), 8-15 epilogue (two per quadrant,
+// 96 token columns each); warps 2-3 only take part in set-up and teardown. TMEM: D double-buffered (2 x 192 columns) and
+// A double-buffered (2 x 64 columns) = 512 columns. All mbarrier waits are
+// bounded; on a timeout the kernel records the error, stops issuing, drains
+// its copies and MMAs in flight, frees TMEM and returns.
 #include <cstdint>
+#include <cstdio>
 
 #include "mobi_device.cuh"
 #include "mobi_host.h"
 
 namespace mobi {
 
-size_t prefill_ws_bytes(int64_t T, int64_t N, int64_t K) { return 0; }
+namespace pf {
+constexpr int BM = 128;          // weight rows per tile (tcgen05 M)
+constexpr int BN = 192;          // tokens per tile (tcgen05 N)
+constexpr int GK = 128;          // group width along K
+constexpr int XST = 3;           // x-tile stages (one group each)
+constexpr int CST = 4;           // code/scale stages (one unit each)
+// Registers are budgeted per group of four warps, so the block is 16 warps of
+// at most 128 registers: 0 producer, 1 MMA, 2-3 idle, 4-7 dequant, 8-15 epilogue.
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kDeqWarp0 = 4;
+constexpr int kEpiWarp0 = 8;
+constexpr int kEpiWarps = 8;                   // two per TMEM lane quadrant
+constexpr int kColsPerEpi = BN / 2;            // 96 token columns per epilogue warp
+constexpr uint32_t kXHalfBytes = BN * 128;     // 192 rows x 64 bf16 = 24576
+constexpr uint32_t kXStageBytes = 2 * kXHalfBytes;
+constexpr uint32_t kCodeBytes = BM * 32;       // 128 rows x 8 words
+constexpr uint32_t kSzBytes = BM * 4;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemD0 = 0, kTmemD1 = BN, kTmemA0 = 2 * BN, kTmemA1 = 2 * BN + 64;
+}  // namespace pf
 
-cudaError_t launch_prefill(const void*, int64_t, int64_t, const int32_t*, const int32_t*, const int32_t*,
-                           const uint32_t*, const uint32_t*, int64_t, int, float*, void*, cudaStream_t,
-                           DeviceStatus*) {
-  return cudaErrorNotSupported;
+struct PfSmem {
+  uint8_t x[pf::XST][pf::kXStageBytes];     // 1024-byte aligned (offset 0)
+  uint32_t codes[pf::CST][pf::BM * 8];      // [row][word]
+  uint32_t sz[pf::CST][pf::BM];
+  uint64_t x_full[pf::XST], x_empty[pf::XST];
+  uint64_t c_full[pf::CST], c_empty[pf::CST];
+  uint64_t a_full[2], a_empty[2];
+  uint64_t d_full[2], d_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int32_t abort_flag;
+};
+
+// ---- tcgen05 wrappers ----------------------------------------------------------------
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16 (bf16 in, fp32 accumulate).
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+// 32 lanes x 32 bits, 16 consecutive columns per thread.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 32 bits, 16 consecutive columns per thread.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms of
+// 1024 bytes (stride byte offset), version 1 (sm_100).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;                   // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024u >> 4) << 32;         // stride byte offset
+  d |= (uint64_t)1u << 46;                   // descriptor version
+  d |= (uint64_t)2u << 61;                   // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, N = BN, M = BM.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// ---- tile bookkeeping ------------------------------------------------------------------
+
+struct TileInfo {
+  int64_t n0;      // first weight row
+  int64_t t0;      // first bucket-ordered token
+  int nvalid;      // tokens in the tile
+  int kmax;        // slices needed by the tile (k of its last token)
+  int lo[3];       // first tile column whose token takes slice s
+};
+
+__device__ __forceinline__ TileInfo tile_info(int64_t tile, int64_t n_tt, int64_t T, const int32_t* off, int S) {
+  TileInfo ti;
+  const int64_t wt = tile / n_tt, tt = tile % n_tt;
+  ti.n0 = wt * pf::BM;
+  ti.t0 = tt * pf::BN;
+  ti.nvalid = (int)(T - ti.t0 < pf::BN ? T - ti.t0 : pf::BN);
+  const int64_t last = ti.t0 + ti.nvalid - 1;
+  int km = 1;
+#pragma unroll
+  for (int j = 1; j < 3; ++j)
+    if (j < S && (int64_t)off[j] <= last) km = j + 1;
+  ti.kmax = km;
+#pragma unroll
+  for (int s = 0; s < 3; ++s) {
+    int64_t l = s < S ? (int64_t)off[s] - ti.t0 : 0;
+    l = l < 0 ? 0 : (l > ti.nvalid ? ti.nvalid : l);
+    ti.lo[s] = (int)l;
+  }
+  return ti;
+}
+
+// Bounded wait that also gives up when another role has aborted.
+__device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, uint64_t limit, DeviceStatus* st,
+                                        uint32_t where, volatile int32_t* abort_flag) {
+  for (uint64_t i = 0; i < limit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255) == 255 && *abort_flag) return false;
+  }
+  report_error(st, kErrTimeout, where);
+  *abort_flag = 1;
+  return false;
+}
+
+__global__ void __maxnreg__(128) prefill_kernel(
+    const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
+    const __grid_constant__ CUtensorMap tm_sz, const uint32_t* __restrict__ sz, const int32_t* __restrict__ perm,
+    const int32_t* __restrict__ offsets, int64_t T, int64_t N, int64_t ngroups, int S, float* __restrict__ Y,
+    DeviceStatus* st, uint64_t limit) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // Dynamic shared memory is rounded up to a 1024-byte boundary for the swizzled tiles.
+  PfSmem& sm = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int32_t* abort_flag = &sm.abort_flag;
+
+  const int64_t n_wt = (N + pf::BM - 1) / pf::BM;
+  const int64_t n_tt = (T + pf::BN - 1) / pf::BN;
+  const int64_t ntiles = n_wt * n_tt;
+  int32_t off[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) off[j] = j <= S ? __ldg(offsets + j) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < pf::XST; ++i) { mbar_init(&sm.x_full[i], 1); mbar_init(&sm.x_empty[i], 1); }
+    for (int i = 0; i < pf::CST; ++i) { mbar_init(&sm.c_full[i], 1); mbar_init(&sm.c_empty[i], 4); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.a_full[i], 4); mbar_init(&sm.a_empty[i], 1);
+      mbar_init(&sm.d_full[i], 1); mbar_init(&sm.d_empty[i], pf::kEpiWarps);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&sm.tmem_base, pf::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      prefetch_tmap(&tm_x); prefetch_tmap(&tm_codes); prefetch_tmap(&tm_sz);
+      uint32_t xi = 0, ci = 0;  // running stage counters
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const TileInfo ti = tile_info(tile, n_tt, T, off, S);
+        for (int64_t g = 0; g < ngroups && ok; ++g) {
+          const uint32_t xs = xi % pf::XST, xph = (xi / pf::XST) & 1;
+          if (!(ok = pf_wait(&sm.x_empty[xs], xph ^ 1, limit, st, 0x301, abort_flag))) break;
+          mbar_arrive_expect_tx(&sm.x_full[xs], pf::kXStageBytes);
+          tma_load_2d(&sm.x[xs][0], &tm_x, (int)(g * pf::GK), (int)ti.t0, &sm.x_full[xs]);
+          tma_load_2d(&sm.x[xs][pf::kXHalfBytes], &tm_x, (int)(g * pf::GK + 64), (int)ti.t0, &sm.x_full[xs]);
+          ++xi;
+          for (int s = 0; s < ti.kmax; ++s) {
+            const uint32_t cs = ci % pf::CST, cph = (ci / pf::CST) & 1;
+            if (!(ok = pf_wait(&sm.c_empty[cs], cph ^ 1, limit, st, 0x302, abort_flag))) break;
+            mbar_arrive_expect_tx(&sm.c_full[cs], pf::kCodeBytes + pf::kSzBytes);
+            tma_load_2d(&sm.codes[cs][0], &tm_codes, (int)(g * 8), (int)(s * N + ti.n0), &sm.c_full[cs]);
+            tma_load_2d(&sm.sz[cs][0], &tm_sz, (int)ti.n0, (int)(s * ngroups + g), &sm.c_full[cs]);
+            ++ci;
+          }
+        }
+      }
+      // Drain: every copy issued lands before the CTA may exit.
+      for (uint32_t i = (xi > pf::XST ? xi - pf::XST : 0); i < xi; ++i)
+        mbar_wait(&sm.x_full[i % pf::XST], (i / pf::XST) & 1, kDefaultWaitLimit, st, 0x3F1);
+      for (uint32_t i = (ci > pf::CST ? ci - pf::CST : 0); i < ci; ++i)
+        mbar_wait(&sm.c_full[i % pf::CST], (i / pf::CST) & 1, kDefaultWaitLimit, st, 0x3F2);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(pf::BM, pf::BN);
+      uint32_t xi = 0, u = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const TileInfo ti = tile_info(tile, n_tt, T, off, S);
+        for (int64_t g = 0; g < ngroups && ok; ++g) {
+          const uint32_t xs = xi % pf::XST, xph = (xi / pf::XST) & 1;
+          if (!(ok = pf_wait(&sm.x_full[xs], xph, limit, st, 0x311, abort_flag))) break;
+          const uint32_t xbase = smem_addr(&sm.x[xs][0]);
+          for (int s = 0; s < ti.kmax; ++s, ++u) {
+            const uint32_t b = u & 1, ph = (u >> 1) & 1;
+            if (!(ok = pf_wait(&sm.a_full[b], ph, limit, st, 0x312, abort_flag))) break;
+            if (!(ok = pf_wait(&sm.d_empty[b], ph ^ 1, limit, st, 0x313, abort_flag))) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem + (b ? pf::kTmemD1 : pf::kTmemD0);
+            const uint32_t a_tmem = tmem + (b ? pf::kTmemA1 : pf::kTmemA0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t saddr = xbase + (i >> 2) * pf::kXHalfBytes + (i & 3) * 32;
+              mma_ts(d_tmem, a_tmem + 8 * i, desc_sw128(saddr), idesc, i > 0 ? 1u : 0u);
+            }
+            mma_commit(&sm.a_empty[b]);
+            mma_commit(&sm.d_full[b]);
+            if (s == ti.kmax - 1) mma_commit(&sm.x_empty[xs]);
+          }
+          ++xi;
+        }
+      }
+      // Drain: wait for every MMA issued so far before TMEM is released.
+      mma_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, kDefaultWaitLimit, st, 0x3F3);
+    }
+  } else if (warp >= pf::kDeqWarp0 && warp < pf::kDeqWarp0 + 4) {
+    // ---------------- dequant: codes -> exact (q - z) bf16 pairs in TMEM ----------------
+    const int q = warp & 3;               // TMEM lane quadrant of this warp
+    const int r = 32 * q + lane;          // row within the tile
+    const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
+    uint32_t ci = 0, u = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      const TileInfo ti = tile_info(tile, n_tt, T, off, S);
+      for (int64_t g = 0; g < ngroups && ok; ++g) {
+        for (int s = 0; s < ti.kmax; ++s, ++u, ++ci) {
+          const uint32_t cs = ci % pf::CST, cph = (ci / pf::CST) & 1;
+          if (!(ok = pf_wait(&sm.c_full[cs], cph, limit, st, 0x321, abort_flag))) break;
+          const uint4 w0 = *reinterpret_cast<const uint4*>(&sm.codes[cs][r * 8]);
+          const uint4 w1 = *reinterpret_cast<const uint4*>(&sm.codes[cs][r * 8 + 4]);
+          const uint32_t zsz = sm.sz[cs][r];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.c_empty[cs]);
+          const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+          // bf16 (128 + z) in both halves; zero is an integer 0..3 stored as fp16.
+          const float zf = __half2float(__ushort_as_half((unsigned short)(zsz >> 16)));
+          const uint32_t zb = 0x4300u + (uint32_t)(int)zf;  // bf16 of 128 + z (exact)
+          const uint32_t zz2 = zb | (zb << 16);
+          const __nv_bfloat162 zz = *reinterpret_cast<const __nv_bfloat162*>(&zz2);
+          const uint32_t b = u & 1, ph = (u >> 1) & 1;
+          if (!(ok = pf_wait(&sm.a_empty[b], ph ^ 1, limit, st, 0x322, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t a_tmem = tmem + lane_addr + (b ? pf::kTmemA1 : pf::kTmemA0);
+#pragma unroll
+          for (int half = 0; half < 4; ++half) {  // 16 columns (two words) per store
+            uint32_t regs[16];
+#pragma unroll
+            for (int ww = 0; ww < 2; ++ww) {
+              const uint32_t w = words[2 * half + ww];
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const uint32_t v = ((w >> (2 * c)) & 0x00030003u) | 0x43004300u;
+                __nv_bfloat162 p = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&v), zz);
+                regs[8 * ww + c] = *reinterpret_cast<uint32_t*>(&p);
+              }
+            }
+            tmem_st16(a_tmem + 16 * half, regs);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.a_full[b]);
+        }
+      }
+    }
+  } else if (warp >= pf::kEpiWarp0) {
+    // ---------------- epilogue: per-group fp32 scale promotion ----------------
+    const int e = warp - pf::kEpiWarp0;   // 0..7
+    const int q = warp & 3;               // TMEM lane quadrant
+    const int cbase = (e >> 2) * pf::kColsPerEpi;  // 0 or 96
+    const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
+    uint32_t u = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      const TileInfo ti = tile_info(tile, n_tt, T, off, S);
+      const int64_t n = ti.n0 + 32 * q + lane;
+      float acc[pf::kColsPerEpi];
+#pragma unroll
+      for (int c = 0; c < pf::kColsPerEpi; ++c) acc[c] = 0.0f;
+      for (int64_t g = 0; g < ngroups && ok; ++g) {
+        for (int s = 0; s < ti.kmax; ++s, ++u) {
+          const uint32_t b = u & 1, ph = (u >> 1) & 1;
+          // Scale of (slice s, group g, row n): one coalesced load per warp, issued
+          // before the wait so that its latency hides behind the MMA.
+          const uint32_t szw = n < N ? __ldg(sz + ((int64_t)s * ngroups + g) * N + n) : 0u;
+          if (!(ok = pf_wait(&sm.d_full[b], ph, limit, st, 0x331, abort_flag))) break;
+          tc_fence_after();
+          const float sc = __half2float(__ushort_as_half((unsigned short)(szw & 0xffffu)));
+          const uint32_t d_tmem = tmem + lane_addr + (b ? pf::kTmemD1 : pf::kTmemD0) + cbase;
+          const int lo = (s == 0 ? ti.lo[0] : (s == 1 ? ti.lo[1] : ti.lo[2])) - cbase;  // first active column
+#pragma unroll
+          for (int ch = 0; ch < pf::kColsPerEpi / 16; ++ch) {
+            if (16 * ch + 16 <= lo) continue;  // whole chunk inactive (warp-uniform)
+            uint32_t r[16];
+            tmem_ld16(d_tmem + 16 * ch, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int c = 16 * ch + j;
+              if (c >= lo) acc[c] = fmaf(sc, __uint_as_float(r[j]), acc[c]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.d_empty[b]);
+        }
+      }
+      if (!ok) break;
+      if (n < N) {
+#pragma unroll
+        for (int c = 0; c < pf::kColsPerEpi; ++c) {
+          const int col = cbase + c;
+          if (col < ti.nvalid) {
+            const int32_t t = __ldg(perm + ti.t0 + col);
+            if (t >= 0 && t < T) Y[(int64_t)t * N + n] = acc[c];
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, pf::kTmemCols);
+  }
+}
+
+// ---- gather: bucket-ordered, pair-interleaved copy of the activations --------------------
+//
+// Xb[i][16w + 2c + e] = X[perm[i]][16w + c + 8e]: row i is the i-th token in
+// bucket order, and within each 16-column block the columns are interleaved so
+// that column pair (2c, 2c+1) holds the activations of the packed pair
+// (c, c+8). One thread per 16-column block.
+__global__ void __launch_bounds__(256) prefill_gather_kernel(const __nv_bfloat16* __restrict__ X, int64_t T,
+                                                             int64_t K, const int32_t* __restrict__ perm,
+                                                             __nv_bfloat16* __restrict__ Xb) {
+  const int64_t nblk = K / 16;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= T * nblk) return;
+  const int64_t i = idx / nblk, w = idx % nblk;
+  int32_t src = __ldg(perm + i);
+  uint4 a = make_uint4(0, 0, 0, 0), b = a;
+  if (src >= 0 && src < T) {
+    const uint4* p = reinterpret_cast<const uint4*>(X + (int64_t)src * K + 16 * w);
+    a = __ldg(p);
+    b = __ldg(p + 1);
+  }
+  const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};  // x[0..15] as bf16 pairs
+  uint32_t out[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t lo = (in[c >> 1] >> (16 * (c & 1))) & 0xffffu;              // x[c]
+    const uint32_t hi = (in[(c + 8) >> 1] >> (16 * ((c + 8) & 1))) & 0xffffu;  // x[c + 8]
+    out[c] = lo | (hi << 16);
+  }
+  uint4* q = reinterpret_cast<uint4*>(Xb + i * K + 16 * w);
+  q[0] = make_uint4(out[0], out[1], out[2], out[3]);
+  q[1] = make_uint4(out[4], out[5], out[6], out[7]);
+}
+
+// ---- host side -------------------------------------------------------------------------
+
+size_t prefill_ws_bytes(int64_t T, int64_t N, int64_t K) {
+  (void)N;
+  return ((size_t)T * (size_t)K * 2 + 255) / 256 * 256;
+}
+
+static size_t pf_smem_bytes() { return sizeof(PfSmem) + 1024; }
+
+cudaError_t launch_prefill(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
+                           const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int S,
+                           float* Y, void* ws, cudaStream_t stream, DeviceStatus* st) {
+  (void)k_t;
+  const int64_t ngroups = K / 128;
+  __nv_bfloat16* Xb = static_cast<__nv_bfloat16*>(ws);
+  CUtensorMap tm_x, tm_codes, tm_sz;
+  if (!make_tmap_2d(&tm_x, Xb, 2, (uint64_t)K, (uint64_t)T, (uint64_t)K * 2, 64, pf::BN, true))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4, 8, pf::BM,
+                    false))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, pf::BM, 1, false))
+    return cudaErrorInvalidValue;
+
+  const int64_t blocks_g = (T * (K / 16) + 255) / 256;
+  prefill_gather_kernel<<<(unsigned)blocks_g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T, K, perm, Xb);
+
+  const int64_t ntiles = ((N + pf::BM - 1) / pf::BM) * ((T + pf::BN - 1) / pf::BN);
+  const int grid = (int)(ntiles < num_sms() ? ntiles : num_sms());
+  const size_t smem = pf_smem_bytes();
+  cudaError_t e = set_smem((const void*)prefill_kernel, (int)smem);
+  if (e != cudaSuccess) return e;
+  prefill_kernel<<<grid, pf::kThreads, smem, stream>>>(tm_x, tm_codes, tm_sz, sz, perm, offsets, T, N, ngroups, S, Y,
+                                                       st, wait_limit());
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    cudaFuncAttributes fa{};
+    cudaFuncGetAttributes(&fa, (const void*)prefill_kernel);
+    char where[160];
+    snprintf(where, sizeof where, "prefill launch (%d threads, %d regs/thread, max %d threads, %zu B smem)",
+             pf::kThreads, fa.numRegs, fa.maxThreadsPerBlock, smem);
+    return note_error(where, e);
+  }
+  return cudaSuccess;
 }
 
 }  // namespace mobi

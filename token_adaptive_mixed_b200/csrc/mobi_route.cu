@@ -17,6 +17,7 @@
 #include <cstdint>
 
 #include "mobi_device.cuh"
+#include "mobi_host.h"
 
 namespace mobi {
 
@@ -223,7 +224,7 @@ static cudaError_t launch_route_s(const void* X, int64_t T, int64_t K, const flo
         static_cast<const __nv_bfloat16*>(X), T, K, Wr, bias, kps, k_t, partial);
   }
   bucket_kernel<S><<<1, kBucketThreads, 0, stream>>>(T, ks, partial, bias, k_t, perm, offsets);
-  return cudaGetLastError();
+  return note_error("kernel launch", cudaGetLastError());
 }
 
 cudaError_t launch_route(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias, int S,
