@@ -201,6 +201,65 @@ def time_pack(mobi, wl, dev, reps=10):
             "weights_per_s": N * K / ms * 1e3}
 
 
+def l2_flush_buffer(dev):
+    return torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+
+def time_prefill(mobi, L, dev, reps, tf_peak, flush):
+    """Route + bucket + tcgen05 prefill GEMM on one prefill workload; CUDA events
+    per repetition with the L2 flushed (256 MB write) before each one."""
+    W = torch.from_numpy(L.W).to(dev)
+    codes, sz = mobi.mobi_pack(W, S=3)
+    del W
+    X = L.X.to(dev)
+    Wr = torch.from_numpy(L.Wr).to(dev)
+    b = None if L.bias is None else torch.from_numpy(L.bias).to(dev)
+    T, N, K = L.T, L.N, L.K
+    k_t = torch.empty(T, dtype=torch.int32, device=dev)
+    perm = torch.empty(T, dtype=torch.int32, device=dev)
+    off = torch.empty(4, dtype=torch.int32, device=dev)
+    Y = torch.empty((T, N), dtype=torch.float32, device=dev)
+    ws_r = torch.empty(max(mobi.mobi_route_workspace_bytes(T, K, 3), 16), dtype=torch.uint8, device=dev)
+    ws_g = torch.empty(mobi.mobi_gemm_workspace_bytes(T, N, K, 3), dtype=torch.uint8, device=dev)
+
+    def route():
+        mobi.mobi_route(X, Wr, b, k_t, perm, off, ws_r)
+
+    def gemm():
+        mobi.mobi_gemm(X, k_t, perm, off, codes, sz, N, Y=Y, ws=ws_g)
+    for _ in range(3):
+        route()
+        gemm()
+    mobi.mobi_sync_check()
+    sumk = int(k_t.sum().item())
+    counts = torch.bincount(k_t, minlength=4)[1:].tolist()
+    t_route, t_gemm = [], []
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for _ in range(reps):
+        flush.fill_(1.0)
+        e[0].record()
+        route()
+        e[1].record()
+        gemm()
+        e[2].record()
+        torch.cuda.synchronize()
+        t_route.append(e[0].elapsed_time(e[1]))
+        t_gemm.append(e[1].elapsed_time(e[2]))
+    mobi.mobi_sync_check()
+    ms_gemm = statistics.median(t_gemm)
+    ms_step = statistics.median([a + b2 for a, b2 in zip(t_route, t_gemm)])
+    issued = 2.0 * N * K * sumk
+    eff = 2.0 * T * N * K
+    return {"workload": L.name, "T": T, "N": N, "K": K, "k_counts": counts, "sum_k": sumk,
+            "ms_step": round(ms_step, 4), "ms_gemm": round(ms_gemm, 4), "ms_route": round(statistics.median(t_route), 4),
+            "tflops_issued": round(issued / ms_gemm / 1e9, 2), "tflops_effective": round(eff / ms_gemm / 1e9, 2),
+            "tflops_issued_step": round(issued / ms_step / 1e9, 2),
+            "roofline": {"bound": "tensor", "kernel": "prefill GEMM (gather + tcgen05 prefill kernels)",
+                         "achieved": round(issued / ms_gemm / 1e9, 2), "peak": tf_peak, "unit": "TFLOP/s",
+                         "frac": round(issued / ms_gemm / 1e9 / tf_peak, 4), "traffic": None},
+            "reps": reps, "l2": "256 MB flush before each repetition"}
+
+
 def run_gpu(args, world, rank):
     import token_adaptive_mixed_b200 as mobi
     from token_adaptive_mixed_b200 import build as mobi_build
@@ -213,6 +272,12 @@ def run_gpu(args, world, rank):
     dev = torch.device("cuda", torch.cuda.current_device())
     hbm_peak, tf_peak, tf_sust, peak_kind = peaks()
 
+    if args.only == "prefill":
+        flush = l2_flush_buffer(dev)
+        out = {"prefill": time_prefill(mobi, wl.prefill(), dev, args.prefill_reps, tf_peak, flush)}
+        if not args.skip_skewed:
+            out["skewed_prefill"] = time_prefill(mobi, wl.skewed_prefill(), dev, args.prefill_reps, tf_peak, flush)
+        return out
     cases = build_decode_cases(mobi, wl, dev)
     for c in cases:
         c.step()
@@ -313,27 +378,49 @@ def run_gpu(args, world, rank):
     }
     if rank == 0:
         out["pack"] = time_pack(mobi, wl, dev)
+    if args.only != "decode":
+        del cases, graph
+        torch.cuda.empty_cache()
+        flush = l2_flush_buffer(dev)
+        out["prefill"] = time_prefill(mobi, wl.prefill(), dev, args.prefill_reps, tf_peak, flush)
+        if not args.skip_skewed:
+            out["skewed_prefill"] = time_prefill(mobi, wl.skewed_prefill(), dev, args.prefill_reps, tf_peak, flush)
     return out
 
 
 # ---- the oracle on the host cores ------------------------------------------------------
 
-def oracle_decode_sample(budget_s: float, cases_spec, rows_cap=None):
-    """Time the CPU oracle (route + GEMM) on a bounded sample of the decode workload.
-    Returns (bytes credited, seconds, threads, description)."""
+_ORACLE_CASES = {}
+
+
+def _oracle_case(N, K, T, rows):
+    """Inputs of one decode case for the oracle (cached: drawing W is not timed)."""
     import oracle
     from token_adaptive_mixed_b200 import workloads as wl
+    key = (N, K, T, rows)
+    if key not in _ORACLE_CASES:
+        L = wl.decode(N, K, T)
+        c_sub, s_sub, _ = oracle.pack(np.ascontiguousarray(L.W[:rows]), S=3)
+        _ORACLE_CASES[key] = (L.X, L.Wr, c_sub, s_sub)
+    return _ORACLE_CASES[key]
+
+
+def oracle_decode_sample(budget_s: float, cases_spec, rows_cap=None):
+    """Time the CPU oracle (route + GEMM) on a bounded sample of the decode workload:
+    every listed case once, then further passes until `budget_s` of CPU time.
+    Returns (bytes credited, seconds, threads, description)."""
+    import oracle
     threads = oracle.max_threads()
     credited, spent, done = 0, 0.0, []
-    for (N, K, T) in cases_spec:
-        if spent >= budget_s:
-            break
-        L = wl.decode(N, K, T)
+    i = 0
+    while i < len(cases_spec) or spent < budget_s:
+        N, K, T = cases_spec[i % len(cases_spec)]
+        i += 1
         rows = N if rows_cap is None else min(N, rows_cap)
-        c_sub, s_sub, _ = oracle.pack(np.ascontiguousarray(L.W[:rows]), S=3)
+        X, Wr, c_sub, s_sub = _oracle_case(N, K, T, rows)
         t0 = time.perf_counter()
-        k, _, _ = oracle.route(L.X, L.Wr)
-        oracle.gemm(L.X, k, c_sub, s_sub, rows)
+        k, _, _ = oracle.route(X, Wr)
+        oracle.gemm(X, k, c_sub, s_sub, rows)
         dt = time.perf_counter() - t0
         km = int(k.max())
         credited += km * (rows * K // 4 + rows * (K // 128) * 4) + T * K * 2
@@ -345,10 +432,10 @@ def oracle_decode_sample(budget_s: float, cases_spec, rows_cap=None):
 def cpu_baseline(budget_s=20.0):
     from token_adaptive_mixed_b200 import workloads as wl
     spec = [(N, K, T) for (N, K) in wl.DECODE_SHAPES for T in wl.DECODE_TOKENS]
-    credited, spent, threads, desc = oracle_decode_sample(budget_s, spec, rows_cap=1024)
+    credited, spent, threads, desc = oracle_decode_sample(budget_s, spec, rows_cap=4096)
     return {"value": round(credited / spent / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"oracle route + fp64 GEMM on the first 1024 rows of each decode case until ~{budget_s:.0f}s: "
-                      f"{desc}; {spent:.1f}s"}
+            "sample": f"oracle route + fp64 GEMM on the first 4096 rows of the decode cases, cycling through the "
+                      f"nine cases until ~{budget_s:.0f}s of CPU time ({len(desc.split(';'))} GEMVs, {spent:.1f}s)"}
 
 
 def run_reference(args, world, rank):
@@ -363,10 +450,10 @@ def run_reference(args, world, rank):
     rows = int(max(16, min(4096, 1024 * per_step_budget)))
     rows -= rows % 16
     for i in range(args.warmup):
-        oracle_decode_sample(1e9, [spec[i % len(spec)]], rows_cap=rows)
+        oracle_decode_sample(0.0, [spec[i % len(spec)]], rows_cap=rows)
     tot_b, tot_s = 0, 0.0
     for i in range(args.steps):
-        b, s, threads, desc = oracle_decode_sample(1e9, [spec[i % len(spec)]], rows_cap=rows)
+        b, s, threads, desc = oracle_decode_sample(0.0, [spec[i % len(spec)]], rows_cap=rows)
         tot_b += b
         tot_s += s
     value = tot_b / tot_s / 1e9
@@ -389,6 +476,10 @@ def main():
     ap.add_argument("--impl", default="mobi", choices=["mobi", "reference"])
     ap.add_argument("--cpu-baseline-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill"],
+                    help="run a subset (profiling); the default runs everything")
+    ap.add_argument("--prefill-reps", type=int, default=10)
+    ap.add_argument("--skip-skewed", action="store_true")
     args = ap.parse_args()
 
     if args.impl == "reference":
@@ -402,7 +493,7 @@ def main():
     world, rank, _ = dist_setup(args.gpus)
     out = run_gpu(args, world, rank)
     if rank == 0:
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and args.only == "all":
             out["cpu_baseline"] = cpu_baseline(args.cpu_baseline_seconds)
         print(json.dumps(out))
     if world > 1:
