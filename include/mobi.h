@@ -181,6 +181,30 @@ MOBI_API mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const i
                            void* stream, int path);
 
 /*
+ * mobi_gemm_decode_noalloc — the decode GEMM (T <= 16) without a workspace.
+ *   Not part of the method: the MoBiQuant pages have no counterpart of this
+ *   call. It exists for callers that cannot allocate device memory at launch
+ *   time: an engine plugin whose enqueue step must not allocate, a real-time
+ *   loop that runs under a fixed memory budget, or a host whose device memory
+ *   belongs to another runtime that only hands out input and output buffers.
+ *   Such callers cannot provide the workspace that mobi_gemm needs.
+ *   Same arguments and result as mobi_gemm for T <= 16, minus perm, offsets
+ *   and the workspace: the scratch lives in one 8 MiB array of static device
+ *   memory that every GPU loading this library holds until the process exits.
+ *   Shapes whose decode scratch exceeds 8 MiB (mobi_gemm_workspace_bytes
+ *   larger than 8 MiB, e.g. N * ceil(K/1024) * 64 bytes beyond it) are
+ *   rejected with MOBI_ERR_WORKSPACE before anything is launched.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   All calls on a device share the one array and it keeps the last call's
+ *   contents, so calls that overlap on the GPU (other streams, other host
+ *   threads) race: serialise them. The call itself allocates nothing.
+ */
+MOBI_API mobi_status mobi_gemm_decode_noalloc(const void* X, int64_t T, int64_t K, const int32_t* k_t,
+                                              const uint32_t* codes, const uint32_t* sz, int64_t N, int G,
+                                              int S, float* Y, void* stream);
+
+/*
  * mobi_sync_check — synchronise `stream`, then report and clear the
  * device-side error word of the current device. Returns MOBI_ERR_TIMEOUT if a
  * bounded wait ran out since the last check, MOBI_ERR_CUDA on a CUDA error.

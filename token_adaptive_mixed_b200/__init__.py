@@ -23,7 +23,8 @@ import torch
 __all__ = [
     "MobiError", "lib", "mobi_version", "mobi_status_string", "mobi_codes_bytes", "mobi_sz_bytes",
     "mobi_route_workspace_bytes", "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm", "mobi_last_error",
-    "mobi_gemm_path", "mobi_sync_check", "mobi_debug_set_wait_limit", "PATH_AUTO", "PATH_DECODE",
+    "mobi_gemm_path", "mobi_sync_check", "mobi_debug_set_wait_limit", "mobi_gemm_decode_noalloc", "PATH_AUTO",
+    "PATH_DECODE",
     "PATH_PREFILL", "EXPORTED_SYMBOLS",
 ]
 
@@ -38,7 +39,7 @@ STATUS_NAMES = ["MOBI_OK", "MOBI_ERR_INVALID_ARG", "MOBI_ERR_UNSUPPORTED_SHAPE",
 EXPORTED_SYMBOLS = (
     "mobi_status_string", "mobi_last_error", "mobi_version", "mobi_codes_bytes", "mobi_sz_bytes", "mobi_route_workspace_bytes",
     "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm", "mobi_gemm_path", "mobi_sync_check",
-    "mobi_debug_set_wait_limit",
+    "mobi_debug_set_wait_limit", "mobi_gemm_decode_noalloc",
 )
 
 
@@ -83,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.mobi_gemm.restype = ci
         L.mobi_gemm_path.argtypes = [p, i64, i64, p, p, p, p, p, i64, ci, ci, p, p, sz_t, p, ci]
         L.mobi_gemm_path.restype = ci
+        L.mobi_gemm_decode_noalloc.argtypes = [p, i64, i64, p, p, p, i64, ci, ci, p, p]
+        L.mobi_gemm_decode_noalloc.restype = ci
         L.mobi_sync_check.argtypes = [p]
         L.mobi_sync_check.restype = ci
         L.mobi_debug_set_wait_limit.argtypes = [i64]
@@ -196,6 +199,16 @@ def mobi_gemm_path(X: torch.Tensor, k_t: torch.Tensor, perm: torch.Tensor, offse
 def mobi_gemm(X, k_t, perm, offsets, codes, sz, N, S=None, G=128, Y=None, ws=None, stream=None):
     """Token-routed mixed-bit GEMM (decode kernel for T <= 16, tcgen05 prefill kernel above)."""
     return mobi_gemm_path(X, k_t, perm, offsets, codes, sz, N, PATH_AUTO, S, G, Y, ws, stream)
+
+
+def mobi_gemm_decode_noalloc(X, k_t, codes, sz, N, S=None, G=128, Y=None, stream=None):
+    """Decode GEMM (T <= 16) whose scratch is the library's static device array (no workspace)."""
+    T, K = X.shape
+    S = codes.shape[0] if S is None else S
+    Y = torch.empty((T, N), dtype=torch.float32, device=X.device) if Y is None else Y
+    _check("mobi_gemm_decode_noalloc", lib().mobi_gemm_decode_noalloc(_ptr(X), T, K, _ptr(k_t), _ptr(codes),
+                                                                      _ptr(sz), N, G, S, _ptr(Y), _stream(stream)))
+    return Y
 
 
 def mobi_sync_check(stream=None) -> None:

@@ -26,7 +26,10 @@
 // combined deterministically: every CTA writes its partial to the workspace
 // and the last CTA of a row block (atomic ticket) sums them in order.
 #include <cstdint>
+#include <cstdio>
+#include <mutex>
 
+#include "../../include/mobi.h"
 #include "mobi_device.cuh"
 #include "mobi_host.h"
 
@@ -373,3 +376,75 @@ cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, c
 }
 
 }  // namespace mobi
+
+// ---- the decode GEMM with static scratch (mobi_gemm_decode_noalloc) -------------------
+//
+// For callers that cannot allocate: the decode scratch (staged activations,
+// group sums, split-K tickets and partials) lives in one file-scope array of
+// static device memory instead of a caller workspace. The kernels are the ones
+// above; only the scratch pointer differs.
+
+namespace mobi {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+static std::mutex g_scratch_mu;
+static void* g_scratch_dev[64];
+
+// Device address of g_decode_scratch on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+static void* noalloc_scratch(cudaError_t* err) {
+  int d = 0;
+  *err = cudaGetDevice(&d);
+  if (*err != cudaSuccess) return nullptr;
+  if (d < 0 || d >= 64) {
+    *err = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_dev[d]) {
+    void* p = nullptr;
+    *err = note_error("cudaGetSymbolAddress(decode scratch)", cudaGetSymbolAddress((void**)&p, g_decode_scratch));
+    if (*err != cudaSuccess) return nullptr;
+    g_scratch_dev[d] = p;
+  }
+  return g_scratch_dev[d];
+}
+
+}  // namespace mobi
+
+extern "C" mobi_status mobi_gemm_decode_noalloc(const void* X, int64_t T, int64_t K, const int32_t* k_t,
+                                                const uint32_t* codes, const uint32_t* sz, int64_t N, int G,
+                                                int S, float* Y, void* stream) {
+  using namespace mobi;
+  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (N < 0 || K < 0 || T < 0 || S < 1 || S > 3) return MOBI_ERR_INVALID_ARG;
+  if (G != 128 || K % 128 != 0 || N % 16 != 0 || T > 16 || N > (int64_t(1) << 28) || K > (int64_t(1) << 28))
+    return MOBI_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0 || N == 0) return MOBI_OK;
+  if (K == 0) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  if (!X || !k_t || !codes || !sz || !Y) return MOBI_ERR_INVALID_ARG;
+  if (!a16(X) || !a16(codes) || !a16(sz) || !a16(Y) || (reinterpret_cast<uintptr_t>(k_t) & 3u))
+    return MOBI_ERR_MISALIGNED;
+  const size_t need = decode_ws_bytes(N, K);
+  if (need > kNoAllocScratchBytes) {
+    char msg[128];
+    snprintf(msg, sizeof msg, "decode scratch of %zu bytes exceeds the %zu-byte static array", need,
+             kNoAllocScratchBytes);
+    note_error(msg, cudaErrorInvalidValue);
+    return MOBI_ERR_WORKSPACE;
+  }
+  cudaError_t e;
+  DeviceStatus* st = device_status(&e);
+  if (!st) return MOBI_ERR_CUDA;
+  void* scratch = noalloc_scratch(&e);
+  if (!scratch) return MOBI_ERR_CUDA;
+  e = launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, scratch, static_cast<cudaStream_t>(stream), st);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOBI_ERR_CUDA;
+  }
+  return MOBI_OK;
+}
