@@ -198,10 +198,8 @@ size_t mobi_route_workspace_bytes(int64_t T, int64_t K, int S) {
 size_t mobi_gemm_workspace_bytes(int64_t T, int64_t N, int64_t K, int S) {
   if (T < 0 || N < 0 || K < 0 || S < 1 || S > 3) return 0;
   size_t b = decode_ws_bytes(N, K);
-  if (T > 16) {
-    const size_t p = prefill_ws_bytes(T, N, K);
-    if (p > b) b = p;
-  }
+  const size_t p = prefill_ws_bytes(T, N, K);  // either kernel may be chosen (mobi_gemm_path)
+  if (p > b) b = p;
   return align256(b);
 }
 

@@ -37,7 +37,7 @@ namespace mobi {
 
 constexpr int kDecRows = 64;      // rows per CTA
 constexpr int kDecGroups = 8;     // 128-wide groups per CTA
-constexpr int kDecThreads = 128;  // 4 warps
+constexpr int kDecThreads = 256;  // 8 warps, one 128-wide group each
 constexpr float kTwo96 = 79228162514264337593543950336.0f;  // 2^96
 constexpr float kTwo37 = 137438953472.0f;                   // 2^37
 
@@ -56,6 +56,9 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __nv_bfloat16* _
                                                           DeviceStatus* st) {
   const int64_t g = blockIdx.x;
   const int tid = threadIdx.x;
+  // The decode kernel may start now: it only reads these outputs after its
+  // grid-dependency wait.
+  asm volatile("griddepcontrol.launch_dependents;");
   {
     const int j = tid >> 5, lane = tid & 31;
     const int gid = lane >> 2, t4 = lane & 3, h = j >> 2, f = j & 3;
@@ -110,10 +113,14 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const __nv_bfloat16* _
 // ---- the decode kernel ------------------------------------------------------------
 
 struct DecSmem {
-  uint32_t codes[3][kDecRows][kDecGroups * 8];   // [slice][row][word]          48 KB
+  // Codes of one slice: two TMA boxes of [64 rows][32 words] with 128-byte
+  // swizzle (16-byte chunk j of row r sits at chunk j ^ (r & 7)), so the eight
+  // rows a warp reads in one instruction fall on different banks.
+  uint32_t codes[3][2][kDecRows][32];            // 48 KB, 1024-byte aligned
   uint32_t sz[3][kDecGroups][kDecRows];          // [slice][group][row]          6 KB
   float xs[kDecGroups][16];                      // group sums                 512 B
   int32_t kt[16];
+  int32_t kmax;
   int32_t is_last;
   uint64_t bar[3];
 };
@@ -127,15 +134,25 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Words 2*t4 and 2*t4+1 of group gi of `row` from the swizzled code tile.
+__device__ __forceinline__ uint2 code_pair(const uint32_t (*tile)[kDecRows][32], int row, int gi, int t4) {
+  const int half = gi >> 2;
+  const int chunk = ((gi & 3) << 1) + (t4 >> 1);
+  const int phys = chunk ^ (row & 7);
+  return *reinterpret_cast<const uint2*>(&tile[half][row][phys * 4 + ((t4 & 1) << 1)]);
+}
+
+constexpr size_t kDecSmemXd = (sizeof(DecSmem) + 127) / 128 * 128;
+
 template <int NB>
 __global__ void __launch_bounds__(kDecThreads) decode_kernel(
     const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_sz,
     const uint32_t* __restrict__ Xd, const float* __restrict__ xs_g, const int32_t* __restrict__ k_t,
     int32_t* __restrict__ meta, int T, int64_t N, int64_t ngroups, int S, float* __restrict__ partial,
     float* __restrict__ Y, DeviceStatus* st, uint64_t limit) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
-  uint32_t* xd_s = reinterpret_cast<uint32_t*>(smem_raw + sizeof(DecSmem) + (128 - sizeof(DecSmem) % 128) % 128);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  DecSmem& sm = *reinterpret_cast<DecSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* xd_s = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(&sm) + kDecSmemXd);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, t4 = lane & 3;
@@ -144,29 +161,40 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(
   const int nch = gridDim.y;
   const int64_t g0 = ch * kDecGroups;
   const int ngc = (int)(ngroups - g0 < kDecGroups ? ngroups - g0 : kDecGroups);
-  const int kmax = min(S, max(1, (int)__ldg(meta)));
 
+  // k_t was written before this call's staging kernel started, so it can be
+  // read before the grid dependency is resolved.
+  if (tid < 16) sm.kt[tid] = tid < T ? k_t[tid] : 0;
   if (tid == 0) {
     for (int s = 0; s < 3; ++s) mbar_init(&sm.bar[s], 1);
     fence_barrier_init();
   }
-  if (tid < 16) sm.kt[tid] = tid < T ? k_t[tid] : 0;
   __syncthreads();
-
   if (tid == 0) {
+    int km = 1;
+    for (int t = 0; t < T; ++t) km = max(km, (int)sm.kt[t]);
+    km = min(km, S);
+    sm.kmax = km;
     const uint32_t xd_bytes = (uint32_t)ngc * 2048u * NB;
     const uint32_t xs_bytes = (uint32_t)ngc * 64u;
-    for (int s = 0; s < kmax; ++s) {
+    for (int s = 0; s < km; ++s) {
       const uint32_t bytes = sizeof(sm.codes[0]) + sizeof(sm.sz[0]) + (s == 0 ? xd_bytes + xs_bytes : 0u);
       mbar_arrive_expect_tx(&sm.bar[s], bytes);
-      tma_load_2d(&sm.codes[s][0][0], &tm_codes, (int)(g0 * 8), (int)(s * N + rb * kDecRows), &sm.bar[s]);
+      const int y = (int)(s * N + rb * kDecRows);
+      tma_load_2d(&sm.codes[s][0][0][0], &tm_codes, (int)(g0 * 8), y, &sm.bar[s]);
+      tma_load_2d(&sm.codes[s][1][0][0], &tm_codes, (int)(g0 * 8 + 32), y, &sm.bar[s]);
       tma_load_2d(&sm.sz[s][0][0], &tm_sz, (int)(rb * kDecRows), (int)(s * ngroups + g0), &sm.bar[s]);
-      if (s == 0) {
-        bulk_g2s(xd_s, Xd + g0 * 2048 / 4 * NB, xd_bytes, &sm.bar[0]);
-        bulk_g2s(&sm.xs[0][0], xs_g + g0 * 16, xs_bytes, &sm.bar[0]);
-      }
     }
   }
+  // The staged activations, group sums and tickets come from the staging
+  // kernel launched just before (programmatic dependent launch).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (tid == 0) {
+    bulk_g2s(xd_s, Xd + g0 * 512 * NB, (uint32_t)ngc * 2048u * NB, &sm.bar[0]);
+    bulk_g2s(&sm.xs[0][0], xs_g + g0 * 16, (uint32_t)ngc * 64u, &sm.bar[0]);
+  }
+  __syncthreads();
+  const int kmax = sm.kmax;
 
   float yt[4][4 * NB];
 #pragma unroll
@@ -174,96 +202,83 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(
 #pragma unroll
     for (int i = 0; i < 4 * NB; ++i) yt[r][i] = 0.0f;
 
+  const int gi = warp;  // this warp's group within the chunk
   bool ok = true;
-  for (int s = 0; s < kmax; ++s) {
-    if (!mbar_wait(&sm.bar[s], 0, limit, st, 0x200 + s)) {
-      ok = false;
-      mbar_wait(&sm.bar[s], 0, kDefaultWaitLimit, st, 0x210 + s);  // drain the copies in flight
-      continue;
-    }
-    if (!ok) continue;
-    float ys[4][4 * NB];
+  if (gi < ngc || warp == 0) {
+    for (int s = 0; s < kmax; ++s) {
+      if (!mbar_wait(&sm.bar[s], 0, limit, st, 0x200 + s)) {
+        ok = false;
+        mbar_wait(&sm.bar[s], 0, kDefaultWaitLimit, st, 0x210 + s);  // drain the copies in flight
+        continue;
+      }
+      if (!ok || gi >= ngc) continue;
+      // B fragments of the 8 k16 steps, zeroed for tokens that do not take slice s.
+      uint32_t b[8][2 * NB];
+      bool on[NB];
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+      for (int nb = 0; nb < NB; ++nb) on[nb] = sm.kt[gid + 8 * nb] > s;
 #pragma unroll
-      for (int i = 0; i < 4 * NB; ++i) ys[r][i] = 0.0f;
-
-#pragma unroll
-    for (int gg = 0; gg < 2; ++gg) {
-      const int gi = 2 * warp + gg;
-      if (gi < ngc) {
-        // B fragments of the 8 k16 steps of this group.
-        uint32_t b[8][2 * NB];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t* src = xd_s + ((gi * 8 + j) * 32 + lane) * NB * 2;
-          if constexpr (NB == 2) {
-            const uint4 v = *reinterpret_cast<const uint4*>(src);
-            b[j][0] = v.x; b[j][1] = v.y; b[j][2] = v.z; b[j][3] = v.w;
-          } else {
-            const uint2 v = *reinterpret_cast<const uint2*>(src);
-            b[j][0] = v.x; b[j][1] = v.y;
-          }
-        }
-        float xsv[2 * NB];
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-          xsv[2 * nb] = sm.xs[gi][2 * t4 + 8 * nb];
-          xsv[2 * nb + 1] = sm.xs[gi][2 * t4 + 1 + 8 * nb];
-        }
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int rowA = 16 * r + gid, rowB = rowA + 8;
-          const uint2 wa = *reinterpret_cast<const uint2*>(&sm.codes[s][rowA][gi * 8 + 2 * t4]);
-          const uint2 wb = *reinterpret_cast<const uint2*>(&sm.codes[s][rowB][gi * 8 + 2 * t4]);
-          float d[NB][4];
-#pragma unroll
-          for (int nb = 0; nb < NB; ++nb) d[nb][0] = d[nb][1] = d[nb][2] = d[nb][3] = 0.0f;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t a0w = wa.x >> (8 * h), a2w = wa.y >> (8 * h);
-            const uint32_t a1w = wb.x >> (8 * h), a3w = wb.y >> (8 * h);
-#pragma unroll
-            for (int f = 0; f < 4; ++f) {
-              const uint32_t m = 0x00030003u << (2 * f);
-              const int j = 4 * h + f;
-#pragma unroll
-              for (int nb = 0; nb < NB; ++nb)
-                mma_bf16_16816(d[nb], a0w & m, a1w & m, a2w & m, a3w & m, b[j][2 * nb], b[j][2 * nb + 1]);
-            }
-          }
-          const uint32_t szA = sm.sz[s][gi][rowA], szB = sm.sz[s][gi][rowB];
-          const float scA = __half2float(__ushort_as_half((unsigned short)(szA & 0xffffu)));
-          const float zA = __half2float(__ushort_as_half((unsigned short)(szA >> 16)));
-          const float scB = __half2float(__ushort_as_half((unsigned short)(szB & 0xffffu)));
-          const float zB = __half2float(__ushort_as_half((unsigned short)(szB >> 16)));
-          const float aA = scA * kTwo37, cA = scA * zA;  // both exact
-          const float aB = scB * kTwo37, cB = scB * zB;
-#pragma unroll
-          for (int nb = 0; nb < NB; ++nb) {
-            ys[r][4 * nb + 0] = fmaf(-cA, xsv[2 * nb], fmaf(aA, d[nb][0], ys[r][4 * nb + 0]));
-            ys[r][4 * nb + 1] = fmaf(-cA, xsv[2 * nb + 1], fmaf(aA, d[nb][1], ys[r][4 * nb + 1]));
-            ys[r][4 * nb + 2] = fmaf(-cB, xsv[2 * nb], fmaf(aB, d[nb][2], ys[r][4 * nb + 2]));
-            ys[r][4 * nb + 3] = fmaf(-cB, xsv[2 * nb + 1], fmaf(aB, d[nb][3], ys[r][4 * nb + 3]));
-          }
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t* src = xd_s + ((gi * 8 + j) * 32 + lane) * NB * 2;
+        if constexpr (NB == 2) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src);
+          b[j][0] = on[0] ? v.x : 0u; b[j][1] = on[0] ? v.y : 0u;
+          b[j][2] = on[1] ? v.z : 0u; b[j][3] = on[1] ? v.w : 0u;
+        } else {
+          const uint2 v = *reinterpret_cast<const uint2*>(src);
+          b[j][0] = on[0] ? v.x : 0u; b[j][1] = on[0] ? v.y : 0u;
         }
       }
-    }
-    // Tokens with k_t <= s do not take slice s.
+      float xsv[2 * NB];
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      const bool m0 = sm.kt[2 * t4 + 8 * nb] > s, m1 = sm.kt[2 * t4 + 1 + 8 * nb] > s;
+      for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int tk = 2 * t4 + e + 8 * nb;
+          xsv[2 * nb + e] = sm.kt[tk] > s ? sm.xs[gi][tk] : 0.0f;
+        }
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
-        if (m0) { yt[r][4 * nb + 0] += ys[r][4 * nb + 0]; yt[r][4 * nb + 2] += ys[r][4 * nb + 2]; }
-        if (m1) { yt[r][4 * nb + 1] += ys[r][4 * nb + 1]; yt[r][4 * nb + 3] += ys[r][4 * nb + 3]; }
+        const int rowA = 16 * r + gid, rowB = rowA + 8;
+        const uint2 wa = code_pair(sm.codes[s], rowA, gi, t4);
+        const uint2 wb = code_pair(sm.codes[s], rowB, gi, t4);
+        float d[NB][4];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) d[nb][0] = d[nb][1] = d[nb][2] = d[nb][3] = 0.0f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t a0w = wa.x >> (8 * h), a2w = wa.y >> (8 * h);
+          const uint32_t a1w = wb.x >> (8 * h), a3w = wb.y >> (8 * h);
+#pragma unroll
+          for (int f = 0; f < 4; ++f) {
+            const uint32_t m = 0x00030003u << (2 * f);
+            const int j = 4 * h + f;
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+              mma_bf16_16816(d[nb], a0w & m, a1w & m, a2w & m, a3w & m, b[j][2 * nb], b[j][2 * nb + 1]);
+          }
+        }
+        const uint32_t szA = sm.sz[s][gi][rowA], szB = sm.sz[s][gi][rowB];
+        const float scA = __half2float(__ushort_as_half((unsigned short)(szA & 0xffffu)));
+        const float zA = __half2float(__ushort_as_half((unsigned short)(szA >> 16)));
+        const float scB = __half2float(__ushort_as_half((unsigned short)(szB & 0xffffu)));
+        const float zB = __half2float(__ushort_as_half((unsigned short)(szB >> 16)));
+        const float aA = scA * kTwo37, cA = scA * zA;  // both exact
+        const float aB = scB * kTwo37, cB = scB * zB;
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          yt[r][4 * nb + 0] = fmaf(-cA, xsv[2 * nb], fmaf(aA, d[nb][0], yt[r][4 * nb + 0]));
+          yt[r][4 * nb + 1] = fmaf(-cA, xsv[2 * nb + 1], fmaf(aA, d[nb][1], yt[r][4 * nb + 1]));
+          yt[r][4 * nb + 2] = fmaf(-cB, xsv[2 * nb], fmaf(aB, d[nb][2], yt[r][4 * nb + 2]));
+          yt[r][4 * nb + 3] = fmaf(-cB, xsv[2 * nb + 1], fmaf(aB, d[nb][3], yt[r][4 * nb + 3]));
+        }
       }
     }
   }
 
   // Cross-warp reduction through shared memory (reuses the code buffer).
   __syncthreads();
-  float* red = reinterpret_cast<float*>(&sm.codes[0][0][0]);  // [warp][token][row], 16 KB
+  float* red = reinterpret_cast<float*>(&sm.codes[0][0][0][0]);  // [warp][token][row], 32 KB
 #pragma unroll
   for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
@@ -280,8 +295,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(
     const int tk = o >> 6, row = o & 63;
     const int64_t n = rb * kDecRows + row;
     if (tk < T && n < N) {
-      const float v = red[(0 * 16 + tk) * 64 + row] + red[(1 * 16 + tk) * 64 + row] +
-                      red[(2 * 16 + tk) * 64 + row] + red[(3 * 16 + tk) * 64 + row];
+      float v = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kDecThreads / 32; ++w) v += red[(w * 16 + tk) * 64 + row];
       if (nch == 1) Y[(int64_t)tk * N + n] = v;
       else partial[((int64_t)ch * 16 + tk) * N + n] = v;
     }
@@ -326,9 +342,7 @@ size_t decode_ws_bytes(int64_t N, int64_t K) {
 }
 
 static size_t dec_smem_bytes(int NB) {
-  size_t b = sizeof(DecSmem);
-  b = (b + 127) / 128 * 128;
-  return b + (size_t)kDecGroups * 2048 * NB;
+  return kDecSmemXd + (size_t)kDecGroups * 2048 * NB + 1024;  // + 1024 for the manual alignment
 }
 
 cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
@@ -352,8 +366,8 @@ cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, c
   float* partial = reinterpret_cast<float*>(p + off);
 
   CUtensorMap tm_codes, tm_sz;
-  if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4, 64, 64,
-                    false))
+  if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4, 32, 64,
+                    true))
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, 64, 8, false))
     return cudaErrorInvalidValue;
@@ -361,17 +375,28 @@ cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, c
   decode_prep_kernel<<<(unsigned)ngroups, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T, K, NB, k_t,
                                                              Xd, xs, meta, nrb, st);
   const size_t smem = dec_smem_bytes(NB);
-  dim3 grid((unsigned)nrb, (unsigned)nch);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)nrb, (unsigned)nch);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap with the staging kernel
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   cudaError_t e;
+  const uint64_t lim = wait_limit();
   if (NB == 2) {
     if ((e = set_smem((const void*)decode_kernel<2>, (int)smem)) != cudaSuccess) return e;
-    decode_kernel<2><<<grid, kDecThreads, smem, stream>>>(tm_codes, tm_sz, Xd, xs, k_t, meta, T, N, ngroups,
-                                                          S, partial, Y, st, wait_limit());
+    e = cudaLaunchKernelEx(&cfg, decode_kernel<2>, tm_codes, tm_sz, (const uint32_t*)Xd, (const float*)xs, k_t, meta,
+                           T, N, ngroups, S, partial, Y, st, lim);
   } else {
     if ((e = set_smem((const void*)decode_kernel<1>, (int)smem)) != cudaSuccess) return e;
-    decode_kernel<1><<<grid, kDecThreads, smem, stream>>>(tm_codes, tm_sz, Xd, xs, k_t, meta, T, N, ngroups,
-                                                          S, partial, Y, st, wait_limit());
+    e = cudaLaunchKernelEx(&cfg, decode_kernel<1>, tm_codes, tm_sz, (const uint32_t*)Xd, (const float*)xs, k_t, meta,
+                           T, N, ngroups, S, partial, Y, st, lim);
   }
+  if (e != cudaSuccess) return note_error("decode launch", e);
   return note_error("kernel launch", cudaGetLastError());
 }
 

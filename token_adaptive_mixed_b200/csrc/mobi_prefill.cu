@@ -16,20 +16,28 @@
 //
 // Operands:
 //   A (weights) lives in tensor memory: four dequant warps turn the 2-bit codes
-//     of their rows into exact bf16 (q - z) pairs — (word >> 2c) & 0x00030003
-//     | 0x43004300 is the pair (128 + q) as bf16, and one bf16x2 subtraction of
-//     (128 + z) gives q - z exactly — and write them with tcgen05.st, so the
-//     dequantised operand never touches shared memory.
-//   B (tokens) comes from shared memory: x tiles staged by TMA with 128-byte
-//     swizzle from a gathered copy Xb of the activations, rows in bucket order
-//     and, within each 16-column block, columns interleaved as (c, c+8) to
-//     match the pair order of the packed words.
-// Warp roles (16 warps): 0 TMA producer, 1 MMA issuer (also owns TMEM),
-// 4-7 dequant (one per TMEM lane quadrant), 8-15 epilogue (two per quadrant,
-// 96 token columns each); warps 2-3 only take part in set-up and teardown. TMEM: D double-buffered (2 x 192 columns) and
-// A double-buffered (2 x 64 columns) = 512 columns. All mbarrier waits are
-// bounded; on a timeout the kernel records the error, stops issuing, drains
-// its copies and MMAs in flight, frees TMEM and returns.
+//     of their rows into exact bf16 (q - z) pairs and write them with
+//     tcgen05.st, so the dequantised operand never touches shared memory.
+//     With w the packed word, ((w >> sh) & (0x00030003 << 2f)) | 0x43004300 is
+//     the bf16 pair (128 + 4^f q); one bf16x2 FMA by 4^-f minus (128 / 4^f + z)
+//     gives q - z exactly, so each pair costs one logic op and one FMA (plus a
+//     shift shared by three pairs).
+//   B (tokens) comes from shared memory: one bulk copy per group brings a
+//     192-token x tile that the gather kernel has already laid out as the
+//     128-byte-swizzled shared-memory image (rows in bucket order and, within
+//     each 16-column block, columns interleaved as (c, c+8) to match the pair
+//     order of the packed words).
+// Pipeline: units flow through two accumulator buffers in TMEM (D, 2 x 192
+// columns) and the A operand through four half-group slots (4 x 32 columns), so
+// the MMA of a unit overlaps both the epilogue of the one before and the
+// dequantisation of the next; the MMA can start on the first half of a group
+// while its second half is still being dequantised.
+// Warp roles (16 warps): 0 TMA producer, 1 and 2 MMA issuers (even and odd
+// units; warp 1 also owns TMEM), 4-7 dequant (one per TMEM lane quadrant),
+// 8-15 epilogue (two per quadrant, 96 token columns each); warp 3 only takes
+// part in set-up and teardown.
+// All mbarrier waits are bounded; on a timeout the kernel records the error,
+// stops issuing, drains its copies and MMAs in flight, frees TMEM and returns.
 #include <cstdint>
 #include <cstdio>
 
@@ -43,9 +51,11 @@ constexpr int BM = 128;          // weight rows per tile (tcgen05 M)
 constexpr int BN = 192;          // tokens per tile (tcgen05 N)
 constexpr int GK = 128;          // group width along K
 constexpr int XST = 3;           // x-tile stages (one group each)
-constexpr int CST = 4;           // code/scale stages (one unit each)
-// Registers are budgeted per group of four warps, so the block is 16 warps of
-// at most 128 registers: 0 producer, 1 MMA, 2-3 idle, 4-7 dequant, 8-15 epilogue.
+constexpr int CST = 6;           // code/scale stages (one unit each)
+constexpr int DST = 2;           // accumulator buffers in TMEM (one unit each)
+constexpr int AST = 4;           // A-operand slots in TMEM (one half group each)
+// 16 warps launched with 128 registers each; the warpgroups then rebalance
+// registers (setmaxnreg): producer/MMA 40, dequant 80, epilogue 168.
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kDeqWarp0 = 4;
@@ -57,7 +67,9 @@ constexpr uint32_t kXStageBytes = 2 * kXHalfBytes;
 constexpr uint32_t kCodeBytes = BM * 32;       // 128 rows x 8 words
 constexpr uint32_t kSzBytes = BM * 4;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemD0 = 0, kTmemD1 = BN, kTmemA0 = 2 * BN, kTmemA1 = 2 * BN + 64;
+constexpr uint32_t kTmemD = 0;                 // D slot j at columns j * BN
+constexpr uint32_t kTmemA = DST * BN;          // A slot j at columns kTmemA + 32 j
+static_assert(DST * BN + AST * 32 <= kTmemCols, "TMEM budget");
 }  // namespace pf
 
 struct PfSmem {
@@ -66,8 +78,8 @@ struct PfSmem {
   uint32_t sz[pf::CST][pf::BM];
   uint64_t x_full[pf::XST], x_empty[pf::XST];
   uint64_t c_full[pf::CST], c_empty[pf::CST];
-  uint64_t a_full[2], a_empty[2];
-  uint64_t d_full[2], d_empty[2];
+  uint64_t a_full[pf::AST], a_empty[pf::AST];
+  uint64_t d_full[pf::DST], d_empty[pf::DST];
   uint64_t drain;
   uint32_t tmem_base;
   int32_t abort_flag;
@@ -189,8 +201,8 @@ __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, uint64_t
   return false;
 }
 
-__global__ void __maxnreg__(128) prefill_kernel(
-    const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
+__global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
+    const uint8_t* __restrict__ Xt, const __grid_constant__ CUtensorMap tm_codes,
     const __grid_constant__ CUtensorMap tm_sz, const uint32_t* __restrict__ sz, const int32_t* __restrict__ perm,
     const int32_t* __restrict__ offsets, int64_t T, int64_t N, int64_t ngroups, int S, float* __restrict__ Y,
     DeviceStatus* st, uint64_t limit) {
@@ -199,6 +211,7 @@ __global__ void __maxnreg__(128) prefill_kernel(
   PfSmem& sm = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int32_t* abort_flag = &sm.abort_flag;
+  (void)sz;
 
   const int64_t n_wt = (N + pf::BM - 1) / pf::BM;
   const int64_t n_tt = (T + pf::BN - 1) / pf::BN;
@@ -208,13 +221,14 @@ __global__ void __maxnreg__(128) prefill_kernel(
   for (int j = 0; j < 4; ++j) off[j] = j <= S ? __ldg(offsets + j) : 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < pf::XST; ++i) { mbar_init(&sm.x_full[i], 1); mbar_init(&sm.x_empty[i], 1); }
-    for (int i = 0; i < pf::CST; ++i) { mbar_init(&sm.c_full[i], 1); mbar_init(&sm.c_empty[i], 4); }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.a_full[i], 4); mbar_init(&sm.a_empty[i], 1);
-      mbar_init(&sm.d_full[i], 1); mbar_init(&sm.d_empty[i], pf::kEpiWarps);
-    }
-    mbar_init(&sm.drain, 1);
+    // An x stage is released by both MMA issuers (each commits after its own MMAs).
+    for (int i = 0; i < pf::XST; ++i) { mbar_init(&sm.x_full[i], 1); mbar_init(&sm.x_empty[i], 2); }
+    // A code/scale stage is released by the 4 dequant warps and the 8 epilogue
+    // warps (which read the scales from it).
+    for (int i = 0; i < pf::CST; ++i) { mbar_init(&sm.c_full[i], 1); mbar_init(&sm.c_empty[i], 4 + pf::kEpiWarps); }
+    for (int i = 0; i < pf::AST; ++i) { mbar_init(&sm.a_full[i], 4); mbar_init(&sm.a_empty[i], 1); }
+    for (int i = 0; i < pf::DST; ++i) { mbar_init(&sm.d_full[i], 1); mbar_init(&sm.d_empty[i], pf::kEpiWarps); }
+    mbar_init(&sm.drain, 2);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
@@ -224,10 +238,13 @@ __global__ void __maxnreg__(128) prefill_kernel(
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp == 0) {
+  // Each warpgroup rebalances its registers (setmaxnreg) at the top of its role.
+  if (warp < 4) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      prefetch_tmap(&tm_x); prefetch_tmap(&tm_codes); prefetch_tmap(&tm_sz);
+      prefetch_tmap(&tm_codes); prefetch_tmap(&tm_sz);
       uint32_t xi = 0, ci = 0;  // running stage counters
       bool ok = true;
       for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
@@ -236,8 +253,10 @@ __global__ void __maxnreg__(128) prefill_kernel(
           const uint32_t xs = xi % pf::XST, xph = (xi / pf::XST) & 1;
           if (!(ok = pf_wait(&sm.x_empty[xs], xph ^ 1, limit, st, 0x301, abort_flag))) break;
           mbar_arrive_expect_tx(&sm.x_full[xs], pf::kXStageBytes);
-          tma_load_2d(&sm.x[xs][0], &tm_x, (int)(g * pf::GK), (int)ti.t0, &sm.x_full[xs]);
-          tma_load_2d(&sm.x[xs][pf::kXHalfBytes], &tm_x, (int)(g * pf::GK + 64), (int)ti.t0, &sm.x_full[xs]);
+          // Pre-swizzled tile (token tile, group g): one contiguous bulk copy.
+          const int64_t tt = ti.t0 / pf::BN;
+          bulk_g2s(&sm.x[xs][0], Xt + (tt * ngroups + g) * (int64_t)pf::kXStageBytes, pf::kXStageBytes,
+                   &sm.x_full[xs]);
           ++xi;
           for (int s = 0; s < ti.kmax; ++s) {
             const uint32_t cs = ci % pf::CST, cph = (ci / pf::CST) & 1;
@@ -255,34 +274,53 @@ __global__ void __maxnreg__(128) prefill_kernel(
       for (uint32_t i = (ci > pf::CST ? ci - pf::CST : 0); i < ci; ++i)
         mbar_wait(&sm.c_full[i % pf::CST], (i / pf::CST) & 1, kDefaultWaitLimit, st, 0x3F2);
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+   } else if (warp == 1 || warp == 2) {
+    // ---------------- MMA issuers ----------------
+    // Two issuing threads in separate warps: warp 1 takes the even units and
+    // owns D buffer 0 and A half-slots 0-1, warp 2 the odd units with D buffer 1
+    // and A slots 2-3. A barrier check costs a few hundred cycles, so while one
+    // thread checks the prerequisites of its next unit the other keeps the
+    // tensor pipe fed. tcgen05.commit tracks the issuing thread's own MMAs, so
+    // both threads release every x stage (count 2).
     if (lane == 0) {
+      const uint32_t par = (uint32_t)(warp - 1);
       const uint32_t idesc = idesc_bf16(pf::BM, pf::BN);
-      uint32_t xi = 0, u = 0;
+      uint32_t xi = 0, u = 0;  // x stages, units (all units are counted by both threads)
       bool ok = true;
       for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
         const TileInfo ti = tile_info(tile, n_tt, T, off, S);
         for (int64_t g = 0; g < ngroups && ok; ++g) {
           const uint32_t xs = xi % pf::XST, xph = (xi / pf::XST) & 1;
-          if (!(ok = pf_wait(&sm.x_full[xs], xph, limit, st, 0x311, abort_flag))) break;
           const uint32_t xbase = smem_addr(&sm.x[xs][0]);
-          for (int s = 0; s < ti.kmax; ++s, ++u) {
-            const uint32_t b = u & 1, ph = (u >> 1) & 1;
-            if (!(ok = pf_wait(&sm.a_full[b], ph, limit, st, 0x312, abort_flag))) break;
-            if (!(ok = pf_wait(&sm.d_empty[b], ph ^ 1, limit, st, 0x313, abort_flag))) break;
-            tc_fence_after();
-            const uint32_t d_tmem = tmem + (b ? pf::kTmemD1 : pf::kTmemD0);
-            const uint32_t a_tmem = tmem + (b ? pf::kTmemA1 : pf::kTmemA0);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const uint32_t saddr = xbase + (i >> 2) * pf::kXHalfBytes + (i & 3) * 32;
-              mma_ts(d_tmem, a_tmem + 8 * i, desc_sw128(saddr), idesc, i > 0 ? 1u : 0u);
+          bool have_x = false;
+          for (int s = 0; s < ti.kmax && ok; ++s, ++u) {
+            if ((u & 1) != par) continue;
+            if (!have_x) {
+              if (!(ok = pf_wait(&sm.x_full[xs], xph, limit, st, 0x311, abort_flag))) break;
+              have_x = true;
             }
-            mma_commit(&sm.a_empty[b]);
-            mma_commit(&sm.d_full[b]);
-            if (s == ti.kmax - 1) mma_commit(&sm.x_empty[xs]);
+            const uint32_t db = par, dph = (u >> 1) & 1;  // this thread's D buffer, its (u/2)-th use
+            if (!(ok = pf_wait(&sm.d_empty[db], dph ^ 1, limit, st, 0x313, abort_flag))) break;
+            // The dequant warps fill half 0 before half 1, so half 1 being full
+            // covers both halves.
+            const uint32_t hh1 = 2 * u + 1;
+            if (!(ok = pf_wait(&sm.a_full[hh1 % pf::AST], (hh1 / pf::AST) & 1, limit, st, 0x312, abort_flag))) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem + pf::kTmemD + db * pf::BN;
+            for (int half = 0; half < 2; ++half) {
+              const uint32_t ab = (2 * u + half) % pf::AST;
+              const uint32_t a_tmem = tmem + pf::kTmemA + ab * 32;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {  // k16 steps 4*half .. 4*half+3: one x half tile
+                const uint32_t saddr = xbase + half * pf::kXHalfBytes + i * 32;
+                mma_ts(d_tmem, a_tmem + 8 * i, desc_sw128(saddr), idesc, (half > 0 || i > 0) ? 1u : 0u);
+              }
+              mma_commit(&sm.a_empty[ab]);
+            }
+            mma_commit(&sm.d_full[db]);
           }
+          if (!ok) break;
+          mma_commit(&sm.x_empty[xs]);
           ++xi;
         }
       }
@@ -290,18 +328,20 @@ __global__ void __maxnreg__(128) prefill_kernel(
       mma_commit(&sm.drain);
       mbar_wait(&sm.drain, 0, kDefaultWaitLimit, st, 0x3F3);
     }
+   }
   } else if (warp >= pf::kDeqWarp0 && warp < pf::kDeqWarp0 + 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
     // ---------------- dequant: codes -> exact (q - z) bf16 pairs in TMEM ----------------
     const int q = warp & 3;               // TMEM lane quadrant of this warp
     const int r = 32 * q + lane;          // row within the tile
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
-    uint32_t ci = 0, u = 0;
+    uint32_t u = 0, hh = 0;
     bool ok = true;
     for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       const TileInfo ti = tile_info(tile, n_tt, T, off, S);
       for (int64_t g = 0; g < ngroups && ok; ++g) {
-        for (int s = 0; s < ti.kmax; ++s, ++u, ++ci) {
-          const uint32_t cs = ci % pf::CST, cph = (ci / pf::CST) & 1;
+        for (int s = 0; s < ti.kmax && ok; ++s, ++u) {
+          const uint32_t cs = u % pf::CST, cph = (u / pf::CST) & 1;
           if (!(ok = pf_wait(&sm.c_full[cs], cph, limit, st, 0x321, abort_flag))) break;
           const uint4 w0 = *reinterpret_cast<const uint4*>(&sm.codes[cs][r * 8]);
           const uint4 w1 = *reinterpret_cast<const uint4*>(&sm.codes[cs][r * 8 + 4]);
@@ -309,77 +349,101 @@ __global__ void __maxnreg__(128) prefill_kernel(
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.c_empty[cs]);
           const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-          // bf16 (128 + z) in both halves; zero is an integer 0..3 stored as fp16.
+          // FMA constants: v * 4^-f - (128 / 4^f + z) = q - z for the field at bit 2f.
           const float zf = __half2float(__ushort_as_half((unsigned short)(zsz >> 16)));
-          const uint32_t zb = 0x4300u + (uint32_t)(int)zf;  // bf16 of 128 + z (exact)
-          const uint32_t zz2 = zb | (zb << 16);
-          const __nv_bfloat162 zz = *reinterpret_cast<const __nv_bfloat162*>(&zz2);
-          const uint32_t b = u & 1, ph = (u >> 1) & 1;
-          if (!(ok = pf_wait(&sm.a_empty[b], ph ^ 1, limit, st, 0x322, abort_flag))) break;
-          tc_fence_after();
-          const uint32_t a_tmem = tmem + lane_addr + (b ? pf::kTmemA1 : pf::kTmemA0);
+          __nv_bfloat162 mul[3], add[3];
 #pragma unroll
-          for (int half = 0; half < 4; ++half) {  // 16 columns (two words) per store
-            uint32_t regs[16];
-#pragma unroll
-            for (int ww = 0; ww < 2; ++ww) {
-              const uint32_t w = words[2 * half + ww];
-#pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                const uint32_t v = ((w >> (2 * c)) & 0x00030003u) | 0x43004300u;
-                __nv_bfloat162 p = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&v), zz);
-                regs[8 * ww + c] = *reinterpret_cast<uint32_t*>(&p);
-              }
-            }
-            tmem_st16(a_tmem + 16 * half, regs);
+          for (int f = 0; f < 3; ++f) {
+            const float m = 1.0f / (float)(1 << (2 * f));
+            mul[f] = __floats2bfloat162_rn(m, m);
+            const float a = -(128.0f * m + zf);  // exact in bf16: 128 + z, 32 + z or 8 + z
+            add[f] = __floats2bfloat162_rn(a, a);
           }
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.a_full[b]);
+          for (int half = 0; half < 2 && ok; ++half, ++hh) {
+            const uint32_t ab = hh % pf::AST, aph = (hh / pf::AST) & 1;
+            if (!(ok = pf_wait(&sm.a_empty[ab], aph ^ 1, limit, st, 0x322, abort_flag))) break;
+            tc_fence_after();
+            const uint32_t a_tmem = tmem + lane_addr + pf::kTmemA + ab * 32;
+#pragma unroll
+            for (int wp = 0; wp < 2; ++wp) {  // 16 columns (two words) per store
+              uint32_t regs[16];
+#pragma unroll
+              for (int ww = 0; ww < 2; ++ww) {
+                const uint32_t w = words[4 * half + 2 * wp + ww];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  // pair (c, c+8): field f = c % 3 of the word shifted by 6 * (c / 3)
+                  const int f = c % 3, sh = 6 * (c / 3);
+                  const uint32_t v = ((w >> sh) & (0x00030003u << (2 * f))) | 0x43004300u;
+                  __nv_bfloat162 p = __hfma2(*reinterpret_cast<const __nv_bfloat162*>(&v), mul[f], add[f]);
+                  regs[8 * ww + c] = *reinterpret_cast<uint32_t*>(&p);
+                }
+              }
+              tmem_st16(a_tmem + 16 * wp, regs);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.a_full[ab]);
+          }
         }
       }
     }
   } else if (warp >= pf::kEpiWarp0) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 168;");
     // ---------------- epilogue: per-group fp32 scale promotion ----------------
     const int e = warp - pf::kEpiWarp0;   // 0..7
     const int q = warp & 3;               // TMEM lane quadrant
-    const int cbase = (e >> 2) * pf::kColsPerEpi;  // 0 or 96
+    const int cbase = (e >> 2) * pf::kColsPerEpi;  // 0 or 64
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     uint32_t u = 0;
     bool ok = true;
     for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       const TileInfo ti = tile_info(tile, n_tt, T, off, S);
       const int64_t n = ti.n0 + 32 * q + lane;
-      float acc[pf::kColsPerEpi];
+      float2 acc[pf::kColsPerEpi / 2];
 #pragma unroll
-      for (int c = 0; c < pf::kColsPerEpi; ++c) acc[c] = 0.0f;
+      for (int c = 0; c < pf::kColsPerEpi / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
       for (int64_t g = 0; g < ngroups && ok; ++g) {
         for (int s = 0; s < ti.kmax; ++s, ++u) {
-          const uint32_t b = u & 1, ph = (u >> 1) & 1;
-          // Scale of (slice s, group g, row n): one coalesced load per warp, issued
-          // before the wait so that its latency hides behind the MMA.
-          const uint32_t szw = n < N ? __ldg(sz + ((int64_t)s * ngroups + g) * N + n) : 0u;
-          if (!(ok = pf_wait(&sm.d_full[b], ph, limit, st, 0x331, abort_flag))) break;
-          tc_fence_after();
+          // Scale of (slice s, group g, row r) from the staged copy of this unit.
+          const uint32_t cs = u % pf::CST, cph = (u / pf::CST) & 1;
+          if (!(ok = pf_wait(&sm.c_full[cs], cph, limit, st, 0x332, abort_flag))) break;
+          const uint32_t szw = sm.sz[cs][32 * q + lane];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.c_empty[cs]);
           const float sc = __half2float(__ushort_as_half((unsigned short)(szw & 0xffffu)));
-          const uint32_t d_tmem = tmem + lane_addr + (b ? pf::kTmemD1 : pf::kTmemD0) + cbase;
+          const float2 sc2 = make_float2(sc, sc);
+          const uint32_t db = u % pf::DST, dph = (u / pf::DST) & 1;
+          if (!(ok = pf_wait(&sm.d_full[db], dph, limit, st, 0x331, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + lane_addr + pf::kTmemD + db * pf::BN + cbase;
           const int lo = (s == 0 ? ti.lo[0] : (s == 1 ? ti.lo[1] : ti.lo[2])) - cbase;  // first active column
 #pragma unroll
-          for (int ch = 0; ch < pf::kColsPerEpi / 16; ++ch) {
-            if (16 * ch + 16 <= lo) continue;  // whole chunk inactive (warp-uniform)
-            uint32_t r[16];
-            tmem_ld16(d_tmem + 16 * ch, r);
+          for (int cp = 0; cp < pf::kColsPerEpi / 48; ++cp) {  // three 16-column loads per wait
+            if (48 * cp + 48 <= lo) continue;  // all three chunks inactive (warp-uniform)
+            uint32_t r[48];
+            tmem_ld16(d_tmem + 48 * cp, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+            tmem_ld16(d_tmem + 48 * cp + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+            tmem_ld16(d_tmem + 48 * cp + 32, *reinterpret_cast<uint32_t(*)[16]>(&r[32]));
             tmem_ld_wait();
+            if (48 * cp >= lo) {  // all 48 columns active: packed fp32x2 FMAs
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int c = 16 * ch + j;
-              if (c >= lo) acc[c] = fmaf(sc, __uint_as_float(r[j]), acc[c]);
+              for (int j = 0; j < 24; ++j)
+                acc[24 * cp + j] = __ffma2_rn(sc2, make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])),
+                                              acc[24 * cp + j]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 24; ++j) {
+                const int c = 48 * cp + 2 * j;
+                if (c >= lo) acc[24 * cp + j].x = fmaf(sc, __uint_as_float(r[2 * j]), acc[24 * cp + j].x);
+                if (c + 1 >= lo) acc[24 * cp + j].y = fmaf(sc, __uint_as_float(r[2 * j + 1]), acc[24 * cp + j].y);
+              }
             }
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.d_empty[b]);
+          if (lane == 0) mbar_arrive(&sm.d_empty[db]);
         }
       }
       if (!ok) break;
@@ -389,7 +453,7 @@ __global__ void __maxnreg__(128) prefill_kernel(
           const int col = cbase + c;
           if (col < ti.nvalid) {
             const int32_t t = __ldg(perm + ti.t0 + col);
-            if (t >= 0 && t < T) Y[(int64_t)t * N + n] = acc[c];
+            if (t >= 0 && t < T) Y[(int64_t)t * N + n] = (c & 1) ? acc[c >> 1].y : acc[c >> 1].x;
           }
         }
       }
@@ -405,25 +469,29 @@ __global__ void __maxnreg__(128) prefill_kernel(
   }
 }
 
-// ---- gather: bucket-ordered, pair-interleaved copy of the activations --------------------
+// ---- gather: bucket-ordered, swizzled copy of the activations --------------------------
 //
-// Xb[i][16w + 2c + e] = X[perm[i]][16w + c + 8e]: row i is the i-th token in
-// bucket order, and within each 16-column block the columns are interleaved so
-// that column pair (2c, 2c+1) holds the activations of the packed pair
-// (c, c+8). One thread per 16-column block.
+// Xt holds, for every (token tile tt, group g), the 48 KB shared-memory image of
+// the x tile that the MMA reads: two halves (64 columns each) of 192 rows x 128
+// bytes, 16-byte chunk j of row r stored at chunk j ^ (r & 7) (128-byte
+// swizzle). Row r of tile tt is the token perm[192 tt + r] (zeros beyond T);
+// its permuted column 16w + 2c + e holds x[16w + c + 8e], matching the pair
+// order (c, c+8) of a packed word. One thread per 16-column block of a row.
 __global__ void __launch_bounds__(256) prefill_gather_kernel(const __nv_bfloat16* __restrict__ X, int64_t T,
                                                              int64_t K, const int32_t* __restrict__ perm,
-                                                             __nv_bfloat16* __restrict__ Xb) {
+                                                             int64_t T_pad, uint8_t* __restrict__ Xt) {
   const int64_t nblk = K / 16;
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= T * nblk) return;
+  if (idx >= T_pad * nblk) return;
   const int64_t i = idx / nblk, w = idx % nblk;
-  int32_t src = __ldg(perm + i);
   uint4 a = make_uint4(0, 0, 0, 0), b = a;
-  if (src >= 0 && src < T) {
-    const uint4* p = reinterpret_cast<const uint4*>(X + (int64_t)src * K + 16 * w);
-    a = __ldg(p);
-    b = __ldg(p + 1);
+  if (i < T) {
+    const int32_t src = __ldg(perm + i);
+    if (src >= 0 && src < T) {
+      const uint4* p = reinterpret_cast<const uint4*>(X + (int64_t)src * K + 16 * w);
+      a = __ldg(p);
+      b = __ldg(p + 1);
+    }
   }
   const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};  // x[0..15] as bf16 pairs
   uint32_t out[8];
@@ -433,16 +501,20 @@ __global__ void __launch_bounds__(256) prefill_gather_kernel(const __nv_bfloat16
     const uint32_t hi = (in[(c + 8) >> 1] >> (16 * ((c + 8) & 1))) & 0xffffu;  // x[c + 8]
     out[c] = lo | (hi << 16);
   }
-  uint4* q = reinterpret_cast<uint4*>(Xb + i * K + 16 * w);
-  q[0] = make_uint4(out[0], out[1], out[2], out[3]);
-  q[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  const int64_t ngroups = K / 128;
+  const int64_t tt = i / pf::BN, r = i % pf::BN;
+  const int64_t g = w / 8, h = (w % 8) / 4, j0 = 2 * (w % 4);  // chunks j0, j0+1 of half h
+  uint8_t* tile = Xt + ((tt * ngroups + g) * 2 + h) * (int64_t)pf::kXHalfBytes + r * 128;
+  *reinterpret_cast<uint4*>(tile + 16 * ((j0) ^ (r & 7))) = make_uint4(out[0], out[1], out[2], out[3]);
+  *reinterpret_cast<uint4*>(tile + 16 * ((j0 + 1) ^ (r & 7))) = make_uint4(out[4], out[5], out[6], out[7]);
 }
 
 // ---- host side -------------------------------------------------------------------------
 
 size_t prefill_ws_bytes(int64_t T, int64_t N, int64_t K) {
   (void)N;
-  return ((size_t)T * (size_t)K * 2 + 255) / 256 * 256;
+  const int64_t T_pad = (T + pf::BN - 1) / pf::BN * pf::BN;
+  return ((size_t)T_pad * (size_t)K * 2 + 255) / 256 * 256;
 }
 
 static size_t pf_smem_bytes() { return sizeof(PfSmem) + 1024; }
@@ -452,25 +524,25 @@ cudaError_t launch_prefill(const void* X, int64_t T, int64_t K, const int32_t* k
                            float* Y, void* ws, cudaStream_t stream, DeviceStatus* st) {
   (void)k_t;
   const int64_t ngroups = K / 128;
-  __nv_bfloat16* Xb = static_cast<__nv_bfloat16*>(ws);
-  CUtensorMap tm_x, tm_codes, tm_sz;
-  if (!make_tmap_2d(&tm_x, Xb, 2, (uint64_t)K, (uint64_t)T, (uint64_t)K * 2, 64, pf::BN, true))
-    return cudaErrorInvalidValue;
+  const int64_t T_pad = (T + pf::BN - 1) / pf::BN * pf::BN;
+  uint8_t* Xt = static_cast<uint8_t*>(ws);
+  CUtensorMap tm_codes, tm_sz;
   if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4, 8, pf::BM,
                     false))
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, pf::BM, 1, false))
     return cudaErrorInvalidValue;
 
-  const int64_t blocks_g = (T * (K / 16) + 255) / 256;
-  prefill_gather_kernel<<<(unsigned)blocks_g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T, K, perm, Xb);
+  const int64_t blocks_g = (T_pad * (K / 16) + 255) / 256;
+  prefill_gather_kernel<<<(unsigned)blocks_g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T, K, perm,
+                                                               T_pad, Xt);
 
   const int64_t ntiles = ((N + pf::BM - 1) / pf::BM) * ((T + pf::BN - 1) / pf::BN);
   const int grid = (int)(ntiles < num_sms() ? ntiles : num_sms());
   const size_t smem = pf_smem_bytes();
   cudaError_t e = set_smem((const void*)prefill_kernel, (int)smem);
   if (e != cudaSuccess) return e;
-  prefill_kernel<<<grid, pf::kThreads, smem, stream>>>(tm_x, tm_codes, tm_sz, sz, perm, offsets, T, N, ngroups, S, Y,
+  prefill_kernel<<<grid, pf::kThreads, smem, stream>>>(Xt, tm_codes, tm_sz, sz, perm, offsets, T, N, ngroups, S, Y,
                                                        st, wait_limit());
   e = cudaGetLastError();
   if (e != cudaSuccess) {
