@@ -54,6 +54,20 @@ def test_prefill_shapes(mobi, oracle, N, K, T):
     check_gemm(Y, oracle.gemm(L.X, k, codes, sz, N), f"prefill N={N} K={K} T={T}")
 
 
+@pytest.mark.parametrize("N,K,T", [(1664, 256, 2304), (2048, 128, 4000)])
+def test_prefill_persistent_multi_tile(mobi, oracle, N, K, T):
+    """More tiles (128 rows x 192 tokens) than SMs, so CTAs walk several tiles
+    and the pipeline state carries across tile boundaries; sampled tokens from
+    every bucket and every token tile against the oracle (all N)."""
+    L = wl.layer("mt", N, K, T, seed=T + 3, outlier_frac_cols=0.005)
+    codes, sz, _ = oracle.pack(L.W, S=3)
+    k = np.random.default_rng(T).integers(1, 4, T).astype(np.int32)
+    Y = gemm(mobi, L.X, k, codes, sz, N, path=2)
+    perm = np.argsort(k, kind="stable")
+    toks = np.unique(np.concatenate([perm[::97], perm[191::192], perm[:3], perm[-3:]])).astype(np.int32)
+    check_gemm(Y[toks], oracle.gemm(L.X, k, codes, sz, N, tokens=toks), f"multi-tile N={N} K={K} T={T}")
+
+
 @pytest.mark.parametrize("mix", [(1, 0, 0), (0, 0, 1), (0, 1, 0), (0.7, 0.2, 0.1), (0.1, 0.1, 0.8)])
 def test_prefill_bucket_mixes(mobi, oracle, mix):
     """Empty buckets, single-bucket batches and skewed mixes."""
