@@ -196,11 +196,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(
   __syncthreads();
   const int kmax = sm.kmax;
 
-  float yt[4][4 * NB];
+  // yt[r][2 nb + 0] = row 16r+gid, tokens (2t4, 2t4+1) + 8nb; [2 nb + 1] = row +8.
+  float2 yt[4][2 * NB];
 #pragma unroll
   for (int r = 0; r < 4; ++r)
 #pragma unroll
-    for (int i = 0; i < 4 * NB; ++i) yt[r][i] = 0.0f;
+    for (int i = 0; i < 2 * NB; ++i) yt[r][i] = make_float2(0.0f, 0.0f);
 
   const int gi = warp;  // this warp's group within the chunk
   bool ok = true;
@@ -229,14 +230,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(
           b[j][0] = on[0] ? v.x : 0u; b[j][1] = on[0] ? v.y : 0u;
         }
       }
-      float xsv[2 * NB];
+      float2 xsv[NB];
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int tk = 2 * t4 + e + 8 * nb;
-          xsv[2 * nb + e] = sm.kt[tk] > s ? sm.xs[gi][tk] : 0.0f;
-        }
+      for (int nb = 0; nb < NB; ++nb) {
+        const int tk = 2 * t4 + 8 * nb;
+        xsv[nb] = make_float2(sm.kt[tk] > s ? sm.xs[gi][tk] : 0.0f, sm.kt[tk + 1] > s ? sm.xs[gi][tk + 1] : 0.0f);
+      }
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int rowA = 16 * r + gid, rowB = rowA + 8;
@@ -263,14 +262,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(
         const float zA = __half2float(__ushort_as_half((unsigned short)(szA >> 16)));
         const float scB = __half2float(__ushort_as_half((unsigned short)(szB & 0xffffu)));
         const float zB = __half2float(__ushort_as_half((unsigned short)(szB >> 16)));
-        const float aA = scA * kTwo37, cA = scA * zA;  // both exact
-        const float aB = scB * kTwo37, cB = scB * zB;
+        // Packed fp32x2 FMAs: y += scale 2^37 * acc - scale z * xsum (both constants exact).
+        const float2 aA = make_float2(scA * kTwo37, scA * kTwo37), cA = make_float2(-scA * zA, -scA * zA);
+        const float2 aB = make_float2(scB * kTwo37, scB * kTwo37), cB = make_float2(-scB * zB, -scB * zB);
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
-          yt[r][4 * nb + 0] = fmaf(-cA, xsv[2 * nb], fmaf(aA, d[nb][0], yt[r][4 * nb + 0]));
-          yt[r][4 * nb + 1] = fmaf(-cA, xsv[2 * nb + 1], fmaf(aA, d[nb][1], yt[r][4 * nb + 1]));
-          yt[r][4 * nb + 2] = fmaf(-cB, xsv[2 * nb], fmaf(aB, d[nb][2], yt[r][4 * nb + 2]));
-          yt[r][4 * nb + 3] = fmaf(-cB, xsv[2 * nb + 1], fmaf(aB, d[nb][3], yt[r][4 * nb + 3]));
+          yt[r][2 * nb] = __ffma2_rn(cA, xsv[nb], __ffma2_rn(aA, make_float2(d[nb][0], d[nb][1]), yt[r][2 * nb]));
+          yt[r][2 * nb + 1] = __ffma2_rn(cB, xsv[nb], __ffma2_rn(aB, make_float2(d[nb][2], d[nb][3]), yt[r][2 * nb + 1]));
         }
       }
     }
@@ -284,10 +282,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int rowA = 16 * r + gid, tk0 = 2 * t4 + 8 * nb;
-      red[(warp * 16 + tk0) * 64 + rowA] = yt[r][4 * nb + 0];
-      red[(warp * 16 + tk0 + 1) * 64 + rowA] = yt[r][4 * nb + 1];
-      red[(warp * 16 + tk0) * 64 + rowA + 8] = yt[r][4 * nb + 2];
-      red[(warp * 16 + tk0 + 1) * 64 + rowA + 8] = yt[r][4 * nb + 3];
+      red[(warp * 16 + tk0) * 64 + rowA] = yt[r][2 * nb].x;
+      red[(warp * 16 + tk0 + 1) * 64 + rowA] = yt[r][2 * nb].y;
+      red[(warp * 16 + tk0) * 64 + rowA + 8] = yt[r][2 * nb + 1].x;
+      red[(warp * 16 + tk0 + 1) * 64 + rowA + 8] = yt[r][2 * nb + 1].y;
     }
   __syncthreads();
   const int ntk = 8 * NB;
