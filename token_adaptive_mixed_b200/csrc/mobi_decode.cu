@@ -10,21 +10,27 @@
 // byte is, read as a bf16 bit pattern, the subnormal value q * 4^f * 2^-133
 // (bf16 values with exponent field 0 or 1 are linear in their bit pattern).
 // So `word & (0x00030003 << 2f)` (after an optional 8-bit shift) is a pair of
-// exact A-operand values, one AND per two weights. The activations are staged
-// once per call as x * 2^96 / 4^f (exact in bf16 for |x| < 2^31), so every
-// product is q * x * 2^-37 exactly and every field carries the same weight.
-// The zero point is folded in once per (row, group): sum_k x (q - z) =
-// sum_k x q - z * sum_k x, with sum_k x prepared in fp64 and rounded once.
-// fp32 accumulation happens in the tensor core (mma.sync m16n8k16) and in the
-// per-group promotion y += scale * 2^37 * acc - scale * z * xsum.
+// exact A-operand values, one AND per two weights. The activations enter as
+// x * 2^96 / 4^f (exact in bf16 for |x| < 2^31), so every product is
+// q * x * 2^-37 exactly and every field carries the same weight. The zero
+// point is folded in once per (row, group): sum_k x (q - z) = sum_k x q -
+// z * sum_k x, where sum_k x comes from the same tensor-core pass with an
+// all-ones code operand. fp32 accumulation happens in the tensor core
+// (mma.sync m16n8k16) and in the per-group promotion
+// y += scale * 2^37 * acc - scale * z * xsum.
 //
-// Work split: CTA = 64 rows x 8 groups (1024 columns), 4 warps; warp w handles
-// groups 2w, 2w+1 for all four 16-row tiles, so each activation fragment is
-// read from shared memory once and used for 4 tiles x k slices. Codes, scales
-// and the staged activations arrive by TMA, one mbarrier per slice, so slice 0
-// is computed while slices 1..k-1 are still in flight. Column splits are
-// combined deterministically: every CTA writes its partial to the workspace
-// and the last CTA of a row block (atomic ticket) sums them in order.
+// Work split (persistent, one CTA per SM). K is cut into chunks of 8 groups
+// (1024 columns); a CTA owns one chunk and a contiguous range of 32-row
+// blocks (two 16-row MMA tiles each). Its warps form teams of two: both warps
+// of a team work on the same block, each on 4 of the chunk's 8 groups, and the
+// odd warp hands its sums to the even one through shared memory. A warp keeps
+// the activation fragments of its 4 groups in registers for the whole kernel
+// (built once from X) and runs its own TMA ring of (block, slice) stages, so
+// code bytes stream in while earlier stages are multiplied. A stage carries
+// 64 MMAs, enough to cover the fixed cost of its barrier wait and refill.
+// Chunks are combined by a second,
+// programmatically dependent kernel that adds the per-chunk partials in chunk
+// order (deterministic).
 #include <cstdint>
 #include <cstdio>
 #include <mutex>
@@ -35,95 +41,41 @@
 
 namespace mobi {
 
-constexpr int kDecRows = 64;      // rows per CTA
-constexpr int kDecGroups = 8;     // 128-wide groups per CTA
-constexpr int kDecThreads = 256;  // 8 warps, one 128-wide group each
-constexpr float kTwo96 = 79228162514264337593543950336.0f;  // 2^96
-constexpr float kTwo37 = 137438953472.0f;                   // 2^37
+constexpr int kDecGW = 4;                    // groups per warp (128 bytes of a code row)
+constexpr int kDecChunk = 2 * kDecGW;        // groups per CTA chunk (two warps per tile)
+constexpr int kDecRows = 32;                 // rows per stage: two 16-row MMA tiles
+constexpr uint32_t kDecSlotCodes = kDecRows * 128;     // one stage: 32 rows x 128 bytes of codes
+constexpr uint32_t kDecSlotSz = kDecGW * kDecRows * 4;  // and [4 groups][32 rows] scale/zero words
 
-// ---- staging of the activations ------------------------------------------------
-//
-// Xd[g][j][lane][nb][2] (uint32 = bf16 pair) is the B fragment of k16 step j
-// (j = 4h + f) of group g for lane (gid = lane/4, t4 = lane%4) and token
-// gid + 8nb. Register ih in {0,1} holds the pair e in {0,1} at physical column
-//   k = 128g + 32 t4 + 16 ih + 4h + f + 8e,
-// scaled by 2^(96 - 2f). xs[g][t] = sum of x[t, group g] (fp64, stored fp32).
-// meta[0] = max k_t; meta[1..] are the per-row-block tickets (zeroed here).
-__global__ void __launch_bounds__(256) decode_prep_kernel(const __nv_bfloat16* __restrict__ X, int T,
-                                                          int64_t K, int NB, const int32_t* __restrict__ k_t,
-                                                          uint32_t* __restrict__ Xd, float* __restrict__ xs,
-                                                          int32_t* __restrict__ meta, int64_t n_tickets,
-                                                          DeviceStatus* st) {
-  const int64_t g = blockIdx.x;
-  const int tid = threadIdx.x;
-  // The decode kernel may start now: it only reads these outputs after its
-  // grid-dependency wait.
-  asm volatile("griddepcontrol.launch_dependents;");
-  {
-    const int j = tid >> 5, lane = tid & 31;
-    const int gid = lane >> 2, t4 = lane & 3, h = j >> 2, f = j & 3;
-    const float mult = kTwo96 / (float)(1 << (2 * f));
-    bool bad = false;
-    for (int nb = 0; nb < NB; ++nb) {
-      const int tok = gid + 8 * nb;
-      uint32_t reg[2];
-#pragma unroll
-      for (int ih = 0; ih < 2; ++ih) {
-        uint32_t pair = 0;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int64_t k = 128 * g + 32 * t4 + 16 * ih + 4 * h + f + 8 * e;
-          float x = 0.0f;
-          if (tok < T) x = __bfloat162float(X[(int64_t)tok * K + k]);
-          bad |= !(fabsf(x) < 0x1p31f);
-          const __nv_bfloat16 b = __float2bfloat16_rn(x * mult);  // exact: power-of-two scaling
-          pair |= (uint32_t)__bfloat16_as_ushort(b) << (16 * e);
-        }
-        reg[ih] = pair;
-      }
-      uint32_t* dst = Xd + (((g * 8 + j) * 32 + lane) * NB + nb) * 2;
-      dst[0] = reg[0];
-      dst[1] = reg[1];
-    }
-    if (bad) report_error(st, kErrInputRange, 0x100);
-  }
-  {
-    // Group sums: thread (tok = tid/16, part = tid%16) adds 8 columns in fp64,
-    // then a fixed xor tree over the 16 parts.
-    const int tok = tid >> 4, part = tid & 15;
-    double s = 0.0;
-    if (tok < T) {
-      const __nv_bfloat16* p = X + (int64_t)tok * K + 128 * g + 8 * part;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) s += (double)__bfloat162float(p[i]);
-    }
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (part == 0) xs[g * 16 + tok] = (float)s;
-  }
-  if (g == 0 && tid == 0) {
-    int km = 1;
-    for (int t = 0; t < T; ++t) km = max(km, (int)k_t[t]);
-    meta[0] = km;
-  }
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + tid; i < n_tickets; i += (int64_t)gridDim.x * blockDim.x)
-    meta[1 + i] = 0;
-}
-
-// ---- the decode kernel ------------------------------------------------------------
-
-struct DecSmem {
-  // Codes of one slice: two TMA boxes of [64 rows][32 words] with 128-byte
-  // swizzle (16-byte chunk j of row r sits at chunk j ^ (r & 7)), so the eight
-  // rows a warp reads in one instruction fall on different banks.
-  uint32_t codes[3][2][kDecRows][32];            // 48 KB, 1024-byte aligned
-  uint32_t sz[3][kDecGroups][kDecRows];          // [slice][group][row]          6 KB
-  float xs[kDecGroups][16];                      // group sums                 512 B
-  int32_t kt[16];
-  int32_t kmax;
-  int32_t is_last;
-  uint64_t bar[3];
+template <int NB>
+struct DecCfg;
+template <>
+struct DecCfg<1> {  // T <= 8: 16 B-fragment registers per group
+  static constexpr int kTeams = 5;
+  static constexpr int kDepth = 4;
 };
+template <>
+struct DecCfg<2> {  // T <= 16: 32 per group
+  static constexpr int kTeams = 3;
+  static constexpr int kDepth = 5;
+};
+
+template <int NB>
+struct DecLayout {
+  static constexpr int kWarps = 2 * DecCfg<NB>::kTeams;  // consumer warps; one producer warp follows
+  static constexpr int kThreads = 32 * (kWarps + 1);
+  static constexpr int kDepth = DecCfg<NB>::kDepth;
+  static constexpr uint32_t kCodes = 0;                                              // [warp][slot] 4 KB, 1 KB aligned
+  static constexpr uint32_t kSz = kCodes + kWarps * kDepth * kDecSlotCodes;          // [warp][slot][4][32]
+  static constexpr uint32_t kXchg = kSz + kWarps * kDepth * kDecSlotSz;              // [team][2][32][8 NB] floats
+  static constexpr uint32_t kBar = kXchg + DecCfg<NB>::kTeams * 2 * 32 * 8 * NB * 4;  // full, empty [warp][slot]
+  static constexpr uint32_t kReady = kBar + 2 * kWarps * kDepth * 8;  // consumers' fragments built
+  static constexpr uint32_t kAbort = kReady + 8;
+  static constexpr uint32_t kBytes = kAbort + 8;
+  static constexpr size_t kDynamic = kBytes + 1024;  // + manual 1 KB alignment
+};
+
+constexpr float kTwo37 = 137438953472.0f;  // 2^37
 
 __device__ __forceinline__ void mma_bf16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
@@ -134,267 +86,501 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Words 2*t4 and 2*t4+1 of group gi of `row` from the swizzled code tile.
-__device__ __forceinline__ uint2 code_pair(const uint32_t (*tile)[kDecRows][32], int row, int gi, int t4) {
-  const int half = gi >> 2;
-  const int chunk = ((gi & 3) << 1) + (t4 >> 1);
-  const int phys = chunk ^ (row & 7);
-  return *reinterpret_cast<const uint2*>(&tile[half][row][phys * 4 + ((t4 & 1) << 1)]);
+// Exact for a power-of-two multiplier as long as nothing overflows.
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
-constexpr size_t kDecSmemXd = (sizeof(DecSmem) + 127) / 128 * 128;
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Issue one stage of a warp into ring slot `slot`: the warp's 128-byte slice
+// of 32 code rows (x = word column, y = s*N + row) and the matching
+// [4 groups][32 rows] scale/zero words.
+// Weights are read once per call, so they go in with L2 evict-first.
+__device__ __forceinline__ void dec_issue(const CUtensorMap* tm_codes, const CUtensorMap* tm_sz, uint8_t* codes_slot,
+                                          uint32_t* sz_slot, uint64_t* bar, int block, int s, int N, int ngroups,
+                                          int gbase, uint64_t policy) {
+  mbar_arrive_expect_tx(bar, kDecSlotCodes + kDecSlotSz);
+  tma_load_2d_hint(codes_slot, tm_codes, gbase * 8, s * N + block * kDecRows, bar, policy);
+  tma_load_2d_hint(sz_slot, tm_sz, block * kDecRows, s * ngroups + gbase, bar, policy);
+}
+
+// Groups g0, g0 + 1 of one stage for TT tiles: four MMA chains in flight.
+template <int NB, int TT>
+__device__ __forceinline__ void dec_group_pair(int g0, const uint8_t* cs, const uint32_t* ss,
+                                               const uint32_t (&coff)[kDecGW], const uint32_t (&B)[kDecGW][8][2 * NB],
+                                               const float2 (&xs)[kDecGW][NB], const float2 (&m37)[NB],
+                                               const float2 (&m1)[NB], int gid, float2 (&yA)[2][NB],
+                                               float2 (&yB)[2][NB]) {
+  uint2 wa[2][TT], wb[2][TT];
+#pragma unroll
+  for (int gg = 0; gg < 2; ++gg)
+#pragma unroll
+    for (int tt = 0; tt < TT; ++tt) {
+      wa[gg][tt] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + tt * 16 * 128);
+      wb[gg][tt] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + tt * 16 * 128 + 8 * 128);
+    }
+  float d[2][TT][NB][4];
+#pragma unroll
+  for (int gg = 0; gg < 2; ++gg)
+#pragma unroll
+    for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) d[gg][tt][nb][0] = d[gg][tt][nb][1] = d[gg][tt][nb][2] = d[gg][tt][nb][3] = 0.0f;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int f = 0; f < 4; ++f) {
+      const uint32_t m = 0x00030003u << (2 * f);
+#pragma unroll
+      for (int gg = 0; gg < 2; ++gg)
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt) {
+          const uint32_t a0 = (wa[gg][tt].x >> (8 * h)) & m, a2 = (wa[gg][tt].y >> (8 * h)) & m;
+          const uint32_t a1 = (wb[gg][tt].x >> (8 * h)) & m, a3 = (wb[gg][tt].y >> (8 * h)) & m;
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb)
+            mma_bf16_16816(d[gg][tt][nb], a0, a1, a2, a3, B[g0 + gg][4 * h + f][2 * nb],
+                           B[g0 + gg][4 * h + f][2 * nb + 1]);
+        }
+    }
+#pragma unroll
+  for (int gg = 0; gg < 2; ++gg) {
+    const int g = g0 + gg;
+    float2 xm[NB];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) xm[nb] = __fmul2_rn(xs[g][nb], m1[nb]);
+#pragma unroll
+    for (int tt = 0; tt < TT; ++tt) {
+      const uint32_t szA = ss[g * kDecRows + tt * 16 + gid], szB = ss[g * kDecRows + tt * 16 + gid + 8];
+      const float scA = __half2float(__ushort_as_half((unsigned short)(szA & 0xffffu)));
+      const float zA = __half2float(__ushort_as_half((unsigned short)(szA >> 16)));
+      const float scB = __half2float(__ushort_as_half((unsigned short)(szB & 0xffffu)));
+      const float zB = __half2float(__ushort_as_half((unsigned short)(szB >> 16)));
+      const float cA = -scA * zA, cB = -scB * zB;
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        // y += m * (scale 2^37 acc - scale z xsum), as packed fp32x2 FMAs.
+        yA[tt][nb] = __ffma2_rn(make_float2(cA, cA), xm[nb],
+                                __ffma2_rn(__fmul2_rn(make_float2(scA, scA), m37[nb]),
+                                           make_float2(d[gg][tt][nb][0], d[gg][tt][nb][1]), yA[tt][nb]));
+        yB[tt][nb] = __ffma2_rn(make_float2(cB, cB), xm[nb],
+                                __ffma2_rn(__fmul2_rn(make_float2(scB, scB), m37[nb]),
+                                           make_float2(d[gg][tt][nb][2], d[gg][tt][nb][3]), yB[tt][nb]));
+      }
+    }
+  }
+}
+
+// One stage: the warp's ngv valid groups (warp-uniform) for TT tiles.
+template <int NB, int TT>
+__device__ __forceinline__ void dec_stage(int ngv, const uint8_t* cs, const uint32_t* ss,
+                                          const uint32_t (&coff)[kDecGW], const uint32_t (&B)[kDecGW][8][2 * NB],
+                                          const float2 (&xs)[kDecGW][NB], const float2 (&m37)[NB],
+                                          const float2 (&m1)[NB], int gid, float2 (&yA)[2][NB], float2 (&yB)[2][NB]) {
+  // A group beyond K has zero activations and zero-filled codes, so it only
+  // costs time; the pair loop skips whole pairs past the last valid group.
+  dec_group_pair<NB, TT>(0, cs, ss, coff, B, xs, m37, m1, gid, yA, yB);
+  if (ngv > 2) dec_group_pair<NB, TT>(2, cs, ss, coff, B, xs, m37, m1, gid, yA, yB);
+}
+
+// Bounded wait that also gives up once another warp has aborted.
+__device__ __forceinline__ bool dec_wait(uint64_t* bar, uint32_t parity, uint64_t limit, DeviceStatus* st,
+                                         uint32_t where, volatile int32_t* abort_flag) {
+  for (uint64_t i = 0; i < limit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255) == 255 && *abort_flag) return false;
+  }
+  report_error(st, kErrTimeout, where);
+  *abort_flag = 1;
+  return false;
+}
+
+// grid = (CTAs per chunk, chunks). out = Y when there is one chunk, else the
+// per-chunk partials [chunk][T][N]. All loop bookkeeping is incremental
+// 32-bit arithmetic (sizes are validated to N, K < 2^28).
+// Warps 0 .. kWarps-1 consume (teams of two), warp kWarps issues the copies.
 template <int NB>
-__global__ void __launch_bounds__(kDecThreads) decode_kernel(
+__global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
     const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_sz,
-    const uint32_t* __restrict__ Xd, const float* __restrict__ xs_g, const int32_t* __restrict__ k_t,
-    int32_t* __restrict__ meta, int T, int64_t N, int64_t ngroups, int S, float* __restrict__ partial,
-    float* __restrict__ Y, DeviceStatus* st, uint64_t limit) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  DecSmem& sm = *reinterpret_cast<DecSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint32_t* xd_s = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(&sm) + kDecSmemXd);
+    const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ k_t, int T, int N, int K, int ngroups, int S,
+    int nblocks, float* __restrict__ out, DeviceStatus* st, uint64_t limit) {
+  using L = DecLayout<NB>;
+  constexpr int kTeams = DecCfg<NB>::kTeams;
+  constexpr int kW = L::kWarps;
+  constexpr int D = L::kDepth;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gid = lane >> 2, t4 = lane & 3;
-  const int64_t rb = blockIdx.x;                  // row block
-  const int64_t ch = blockIdx.y;                  // column chunk (8 groups)
-  const int nch = gridDim.y;
-  const int64_t g0 = ch * kDecGroups;
-  const int ngc = (int)(ngroups - g0 < kDecGroups ? ngroups - g0 : kDecGroups);
+  // The reduction kernel behind this one may be scheduled now; it waits for
+  // this grid's completion before reading anything.
+  asm volatile("griddepcontrol.launch_dependents;");
 
-  // k_t was written before this call's staging kernel started, so it can be
-  // read before the grid dependency is resolved.
-  if (tid < 16) sm.kt[tid] = tid < T ? k_t[tid] : 0;
-  if (tid == 0) {
-    for (int s = 0; s < 3; ++s) mbar_init(&sm.bar[s], 1);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ch = blockIdx.y;
+  // This CTA's 32-row blocks [b_begin, b_end); team t takes every kTeams-th
+  // of them, starting with block b_begin + t.
+  const int b_begin = (int)((int64_t)blockIdx.x * nblocks / gridDim.x);
+  const int b_end = (int)((int64_t)(blockIdx.x + 1) * nblocks / gridDim.x);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::kBar);  // [warp][slot]
+  uint64_t* empty = full + kW * D;
+  uint64_t* ready = reinterpret_cast<uint64_t*>(sm + L::kReady);
+  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(sm + L::kAbort);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kW * D; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(ready, kW);
+    *abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
-  if (tid == 0) {
-    int km = 1;
-    for (int t = 0; t < T; ++t) km = max(km, (int)sm.kt[t]);
-    km = min(km, S);
-    sm.kmax = km;
-    const uint32_t xd_bytes = (uint32_t)ngc * 2048u * NB;
-    const uint32_t xs_bytes = (uint32_t)ngc * 64u;
-    for (int s = 0; s < km; ++s) {
-      const uint32_t bytes = sizeof(sm.codes[0]) + sizeof(sm.sz[0]) + (s == 0 ? xd_bytes + xs_bytes : 0u);
-      mbar_arrive_expect_tx(&sm.bar[s], bytes);
-      const int y = (int)(s * N + rb * kDecRows);
-      tma_load_2d(&sm.codes[s][0][0][0], &tm_codes, (int)(g0 * 8), y, &sm.bar[s]);
-      tma_load_2d(&sm.codes[s][1][0][0], &tm_codes, (int)(g0 * 8 + 32), y, &sm.bar[s]);
-      tma_load_2d(&sm.sz[s][0][0], &tm_sz, (int)(rb * kDecRows), (int)(s * ngroups + g0), &sm.bar[s]);
-    }
-  }
-  // The staged activations, group sums and tickets come from the staging
-  // kernel launched just before (programmatic dependent launch).
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (tid == 0) {
-    bulk_g2s(xd_s, Xd + g0 * 512 * NB, (uint32_t)ngc * 2048u * NB, &sm.bar[0]);
-    bulk_g2s(&sm.xs[0][0], xs_g + g0 * 16, (uint32_t)ngc * 64u, &sm.bar[0]);
-  }
-  __syncthreads();
-  const int kmax = sm.kmax;
 
-  // yt[r][2 nb + 0] = row 16r+gid, tokens (2t4, 2t4+1) + 8nb; [2 nb + 1] = row +8.
-  float2 yt[4][2 * NB];
+  if (warp == kW) {
+    // ---------------- producer: one thread feeds every consumer's ring ----------------
+    int niss[kW];  // items issued per consumer warp
 #pragma unroll
-  for (int r = 0; r < 4; ++r)
+    for (int w = 0; w < kW; ++w) niss[w] = 0;
+    // The consumers' activation loads go out before the first weight copy.
+    named_bar_sync(15, 32 * (kW + 1));
+    if (lane == 0) {
+      prefetch_tmap(&tm_codes);
+      prefetch_tmap(&tm_sz);
+      const uint64_t policy = l2_evict_first_policy();
+      int kmax = 1;
+      for (int t = 0; t < T; ++t) kmax = max(kmax, (int)__ldg(k_t + t));
+      kmax = kmax > S ? S : kmax;
+      int nit[kW];  // items of each consumer warp: its blocks x kmax (0 past the last group)
+      int maxit = 0;
 #pragma unroll
-    for (int i = 0; i < 2 * NB; ++i) yt[r][i] = make_float2(0.0f, 0.0f);
-
-  const int gi = warp;  // this warp's group within the chunk
-  bool ok = true;
-  if (gi < ngc || warp == 0) {
-    for (int s = 0; s < kmax; ++s) {
-      if (!mbar_wait(&sm.bar[s], 0, limit, st, 0x200 + s)) {
-        ok = false;
-        mbar_wait(&sm.bar[s], 0, kDefaultWaitLimit, st, 0x210 + s);  // drain the copies in flight
-        continue;
+      for (int w = 0; w < kW; ++w) {
+        const int team = w >> 1, gb = ch * kDecChunk + (w & 1) * kDecGW;
+        const int myb = b_end - b_begin > team ? (b_end - b_begin - team + kTeams - 1) / kTeams : 0;
+        nit[w] = gb < ngroups ? myb * kmax : 0;
+        maxit = max(maxit, nit[w]);
       }
-      if (!ok || gi >= ngc) continue;
-      // B fragments of the 8 k16 steps, zeroed for tokens that do not take slice s.
-      uint32_t b[8][2 * NB];
-      bool on[NB];
+      bool ok = true;
+      int slot = 0, bo = 0, s = 0;  // round r: slot r % D, block offset r / kmax, slice r % kmax
+      uint32_t eph = 1;             // parity of the empty phase that frees `slot` in round r (r >= D)
+      for (int r = 0; r < maxit && ok; ++r) {
+        // Two stages per consumer first; the rest once every consumer has its
+        // activations, so that those small loads do not queue behind the ring.
+        if (r == 2 && !(ok = dec_wait(ready, 0, limit, st, 0x2e1, abort_flag))) break;
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb) on[nb] = sm.kt[gid + 8 * nb] > s;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t* src = xd_s + ((gi * 8 + j) * 32 + lane) * NB * 2;
-        if constexpr (NB == 2) {
-          const uint4 v = *reinterpret_cast<const uint4*>(src);
-          b[j][0] = on[0] ? v.x : 0u; b[j][1] = on[0] ? v.y : 0u;
-          b[j][2] = on[1] ? v.z : 0u; b[j][3] = on[1] ? v.w : 0u;
-        } else {
-          const uint2 v = *reinterpret_cast<const uint2*>(src);
-          b[j][0] = on[0] ? v.x : 0u; b[j][1] = on[0] ? v.y : 0u;
-        }
-      }
-      float2 xsv[NB];
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        const int tk = 2 * t4 + 8 * nb;
-        xsv[nb] = make_float2(sm.kt[tk] > s ? sm.xs[gi][tk] : 0.0f, sm.kt[tk + 1] > s ? sm.xs[gi][tk + 1] : 0.0f);
-      }
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int rowA = 16 * r + gid, rowB = rowA + 8;
-        const uint2 wa = code_pair(sm.codes[s], rowA, gi, t4);
-        const uint2 wb = code_pair(sm.codes[s], rowB, gi, t4);
-        float d[NB][4];
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) d[nb][0] = d[nb][1] = d[nb][2] = d[nb][3] = 0.0f;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t a0w = wa.x >> (8 * h), a2w = wa.y >> (8 * h);
-          const uint32_t a1w = wb.x >> (8 * h), a3w = wb.y >> (8 * h);
-#pragma unroll
-          for (int f = 0; f < 4; ++f) {
-            const uint32_t m = 0x00030003u << (2 * f);
-            const int j = 4 * h + f;
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb)
-              mma_bf16_16816(d[nb], a0w & m, a1w & m, a2w & m, a3w & m, b[j][2 * nb], b[j][2 * nb + 1]);
+        for (int w = 0; w < kW; ++w) {
+          if (r < nit[w] && ok) {
+            if (r >= D && !(ok = dec_wait(&empty[w * D + slot], eph, limit, st, 0x2e0, abort_flag))) break;
+            const int team = w >> 1, gb = ch * kDecChunk + (w & 1) * kDecGW;
+            dec_issue(&tm_codes, &tm_sz, sm + L::kCodes + (uint32_t)(w * D + slot) * kDecSlotCodes,
+                      reinterpret_cast<uint32_t*>(sm + L::kSz + (uint32_t)(w * D + slot) * kDecSlotSz),
+                      &full[w * D + slot], b_begin + team + bo * kTeams, s, N, ngroups, gb, policy);
+            ++niss[w];
           }
         }
-        const uint32_t szA = sm.sz[s][gi][rowA], szB = sm.sz[s][gi][rowB];
-        const float scA = __half2float(__ushort_as_half((unsigned short)(szA & 0xffffu)));
-        const float zA = __half2float(__ushort_as_half((unsigned short)(szA >> 16)));
-        const float scB = __half2float(__ushort_as_half((unsigned short)(szB & 0xffffu)));
-        const float zB = __half2float(__ushort_as_half((unsigned short)(szB >> 16)));
-        // Packed fp32x2 FMAs: y += scale 2^37 * acc - scale z * xsum (both constants exact).
-        const float2 aA = make_float2(scA * kTwo37, scA * kTwo37), cA = make_float2(-scA * zA, -scA * zA);
-        const float2 aB = make_float2(scB * kTwo37, scB * kTwo37), cB = make_float2(-scB * zB, -scB * zB);
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-          yt[r][2 * nb] = __ffma2_rn(cA, xsv[nb], __ffma2_rn(aA, make_float2(d[nb][0], d[nb][1]), yt[r][2 * nb]));
-          yt[r][2 * nb + 1] = __ffma2_rn(cB, xsv[nb], __ffma2_rn(aB, make_float2(d[nb][2], d[nb][3]), yt[r][2 * nb + 1]));
-        }
+        if (++s == kmax) { s = 0; ++bo; }
+        if (++slot == D) { slot = 0; eph = r + 1 >= D ? eph ^ 1u : 0u; }
       }
     }
+    // Normally the consumers have waited for every copy. If any warp gave up,
+    // every copy issued must still land before the CTA can exit (the last
+    // copy into a slot completes after the earlier ones).
+    __syncwarp();
+    __syncthreads();  // all consumers are done
+    if (lane == 0 && *abort_flag) {
+#pragma unroll
+      for (int w = 0; w < kW; ++w)
+        for (int sl = 0; sl < D && sl < niss[w]; ++sl) {
+          const int last = sl + (niss[w] - 1 - sl) / D * D;
+          mbar_wait(&full[w * D + sl], (uint32_t)((last / D) & 1), kDefaultWaitLimit, st, 0x2f0);
+        }
+    }
+    return;
   }
 
-  // Cross-warp reduction through shared memory (reuses the code buffer).
-  __syncthreads();
-  float* red = reinterpret_cast<float*>(&sm.codes[0][0][0][0]);  // [warp][token][row], 32 KB
+  // ---------------- consumers ----------------
+  const int gid = lane >> 2, t4 = lane & 3;
+  const int team = warp >> 1, q = warp & 1;
+  const int gbase = ch * kDecChunk + q * kDecGW;  // first group of this warp
+  const int ngv = ngroups - gbase < 0 ? 0 : (ngroups - gbase > kDecGW ? kDecGW : ngroups - gbase);
+  const int my_blocks = b_end - b_begin > team ? (b_end - b_begin - team + kTeams - 1) / kTeams : 0;
+  const uint8_t* codes_w = sm + L::kCodes + (uint32_t)warp * D * kDecSlotCodes;
+  const uint32_t* sz_w = reinterpret_cast<const uint32_t*>(sm + L::kSz + (uint32_t)warp * D * kDecSlotSz);
+  float* xchg = reinterpret_cast<float*>(sm + L::kXchg) + team * 2 * 32 * 8 * NB;
+  uint64_t* full_w = full + warp * D;
+  uint64_t* empty_w = empty + warp * D;
+
+  // This lane's activations (token gid + 8 nb, columns 32 t4 .. +31 of each
+  // group) and k_t[lane].
+  uint4 raw[kDecGW][NB][4];
 #pragma unroll
-  for (int nb = 0; nb < NB; ++nb)
+  for (int g = 0; g < kDecGW; ++g)
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int rowA = 16 * r + gid, tk0 = 2 * t4 + 8 * nb;
-      red[(warp * 16 + tk0) * 64 + rowA] = yt[r][2 * nb].x;
-      red[(warp * 16 + tk0 + 1) * 64 + rowA] = yt[r][2 * nb].y;
-      red[(warp * 16 + tk0) * 64 + rowA + 8] = yt[r][2 * nb + 1].x;
-      red[(warp * 16 + tk0 + 1) * 64 + rowA + 8] = yt[r][2 * nb + 1].y;
+    for (int nb = 0; nb < NB; ++nb) {
+      const int tok = gid + 8 * nb;
+      if (g < ngv && tok < T) {
+        const uint4* src = reinterpret_cast<const uint4*>(X + (int64_t)tok * K + (gbase + g) * 128 + 32 * t4);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) raw[g][nb][v] = __ldg(src + v);
+      } else {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) raw[g][nb][v] = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
-  __syncthreads();
-  const int ntk = 8 * NB;
-  for (int o = tid; o < ntk * 64; o += kDecThreads) {
-    const int tk = o >> 6, row = o & 63;
-    const int64_t n = rb * kDecRows + row;
-    if (tk < T && n < N) {
-      float v = 0.0f;
+  const int my_kt = lane < T ? k_t[lane] : 0;
+  asm volatile("bar.arrive 15, %0;" ::"r"(32 * (kW + 1)) : "memory");
+  int kmax = __reduce_max_sync(0xffffffffu, my_kt);
+  kmax = kmax < 1 ? 1 : (kmax > S ? S : kmax);
+
+  // Activation fragments of the warp's groups, in registers for the whole
+  // kernel. B[g][j][2 nb + ih] is the B fragment of k16 step j = 4h + f for
+  // token gid + 8 nb: register ih holds columns 32 t4 + 16 ih + 4h + f + 8e
+  // (e = 0 low half, 1 high half) of group g, scaled by 2^(96 - 2f). The
+  // matching A fragment of the codes is (word 2 t4 + ih >> 8h) & (3 << 2f).
+  uint32_t B[kDecGW][8][2 * NB];
+  float2 xs[kDecGW][NB];  // sum_k x of tokens (2 t4, 2 t4 + 1) + 8 nb, group g
+  {
+    bool bad = false;
 #pragma unroll
-      for (int w = 0; w < kDecThreads / 32; ++w) v += red[(w * 16 + tk) * 64 + row];
-      if (nch == 1) Y[(int64_t)tk * N + n] = v;
-      else partial[((int64_t)ch * 16 + tk) * N + n] = v;
+    for (int g = 0; g < kDecGW; ++g) {
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        const uint32_t u[16] = {raw[g][nb][0].x, raw[g][nb][0].y, raw[g][nb][0].z, raw[g][nb][0].w,
+                                raw[g][nb][1].x, raw[g][nb][1].y, raw[g][nb][1].z, raw[g][nb][1].w,
+                                raw[g][nb][2].x, raw[g][nb][2].y, raw[g][nb][2].z, raw[g][nb][2].w,
+                                raw[g][nb][3].x, raw[g][nb][3].y, raw[g][nb][3].z, raw[g][nb][3].w};
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          bad |= ((u[i] & 0x7F80u) >= (158u << 7)) || ((u[i] & 0x7F800000u) >= (158u << 23));
+#pragma unroll
+        for (int ih = 0; ih < 2; ++ih)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int f = 0; f < 4; ++f) {
+              const int w0 = 8 * ih + 2 * h + (f >> 1);
+              const uint32_t pair = __byte_perm(u[w0], u[w0 + 4], (f & 1) ? 0x7632u : 0x5410u);
+              const uint32_t e = (uint32_t)(223 - 2 * f) << 7;  // bf16 bits of 2^(96 - 2f)
+              B[g][4 * h + f][2 * nb + ih] = bf16x2_mul(pair, e | (e << 16));
+            }
+      }
+    }
+    // Group sums on the tensor core: codes all 1 -> every D row is sum_k x * 2^-37.
+    float d[kDecGW][NB][4];
+#pragma unroll
+    for (int g = 0; g < kDecGW; ++g)
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) d[g][nb][0] = d[g][nb][1] = d[g][nb][2] = d[g][nb][3] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t one = 0x00010001u << (2 * (j & 3));
+#pragma unroll
+      for (int g = 0; g < kDecGW; ++g)
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+          mma_bf16_16816(d[g][nb], one, one, one, one, B[g][j][2 * nb], B[g][j][2 * nb + 1]);
+    }
+#pragma unroll
+    for (int g = 0; g < kDecGW; ++g)
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) xs[g][nb] = make_float2(d[g][nb][0] * kTwo37, d[g][nb][1] * kTwo37);
+    if (__any_sync(0xffffffffu, bad) && lane == 0) report_error(st, kErrInputRange, 0x100);
+  }
+  if (lane == 0) mbar_arrive(ready);
+
+  // k_t of the two tokens whose D columns this lane holds.
+  int ktl[NB][2];
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    ktl[nb][0] = __shfl_sync(0xffffffffu, my_kt, 2 * t4 + 8 * nb);
+    ktl[nb][1] = __shfl_sync(0xffffffffu, my_kt, 2 * t4 + 1 + 8 * nb);
+  }
+
+  // Code words 2 t4, 2 t4 + 1 of group g of row gid in the 128-byte-swizzled
+  // stage (16-byte chunk c of row r sits at c ^ (r & 7)); rows gid + 8, +16,
+  // +24 share the swizzle and sit 1, 2, 3 KB further on.
+  uint32_t coff[kDecGW];
+#pragma unroll
+  for (int g = 0; g < kDecGW; ++g)
+    coff[g] = (uint32_t)gid * 128u + (uint32_t)(((2 * g + (t4 >> 1)) ^ gid) * 16) + (t4 & 1) * 8u;
+
+  // y[tt][nb]: tile tt of the block, rows gid (A) and gid + 8 (B) of it,
+  // tokens (2 t4, 2 t4 + 1) + 8 nb.
+  float2 yA[2][NB], yB[2][NB];
+#pragma unroll
+  for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) yA[tt][nb] = yB[tt][nb] = make_float2(0.0f, 0.0f);
+
+  bool ok = true;
+  int slot = 0;
+  uint32_t parity = 0;
+  int s = 0, blk = b_begin + team, blk_i = 0;
+  const int total_iters = my_blocks * kmax;  // both warps of a team walk the same sequence
+  for (int it = 0; it < total_iters; ++it) {
+    const bool two = blk * kDecRows + 16 < N;  // the block's second tile exists (N % 16 == 0)
+    if (ok && ngv > 0) {
+      const bool got = __all_sync(0xffffffffu, dec_wait(&full_w[slot], parity, limit, st, 0x200 + s, abort_flag));
+      if (!got) {
+        ok = false;
+      } else {
+        const uint8_t* cs = codes_w + (uint32_t)slot * kDecSlotCodes;
+        const uint32_t* ss = sz_w + (uint32_t)slot * (kDecSlotSz / 4);
+        float2 m37[NB], m1[NB];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          m37[nb] = make_float2(ktl[nb][0] > s ? kTwo37 : 0.0f, ktl[nb][1] > s ? kTwo37 : 0.0f);
+          m1[nb] = make_float2(ktl[nb][0] > s ? 1.0f : 0.0f, ktl[nb][1] > s ? 1.0f : 0.0f);
+        }
+        // Past N the second tile holds zero-filled or neighbouring rows; its
+        // sums are computed like the first tile's and never written.
+        dec_stage<NB, 2>(ngv, cs, ss, coff, B, xs, m37, m1, gid, yA, yB);
+        // Slot free again for the producer.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_w[slot]);
+      }
+    }
+    if (++slot == D) { slot = 0; parity ^= 1u; }
+    if (s == kmax - 1) {
+      // Team hand-off: the odd warp's 4 groups join the even warp's.
+      float* xb = xchg + ((blk_i & 1) * 32 + lane) * 8 * NB;
+      if (q == 1) {
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb)
+            *reinterpret_cast<float4*>(xb + 8 * nb + 4 * tt) =
+                make_float4(yA[tt][nb].x, yA[tt][nb].y, yB[tt][nb].x, yB[tt][nb].y);
+      }
+      named_bar_sync(1 + team, 64);
+      if (q == 0) {
+        float* o = out + (int64_t)ch * T * N + blk * kDecRows;
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+          if (tt == 1 && !two) break;
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            const float4 p = *reinterpret_cast<const float4*>(xb + 8 * nb + 4 * tt);
+            const float v[4] = {yA[tt][nb].x + p.x, yA[tt][nb].y + p.y, yB[tt][nb].x + p.z, yB[tt][nb].y + p.w};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int tk = 2 * t4 + 8 * nb + e;
+              if (tk < T) {
+                o[(int64_t)tk * N + tt * 16 + gid] = v[e];
+                o[(int64_t)tk * N + tt * 16 + gid + 8] = v[2 + e];
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) yA[tt][nb] = yB[tt][nb] = make_float2(0.0f, 0.0f);
+      s = 0;
+      blk += kTeams;
+      ++blk_i;
+    } else {
+      ++s;
     }
   }
-  if (nch == 1) return;
-  __threadfence();
+  // Final CTA barrier: the producer then drains its copies if a warp gave up.
+  __syncwarp();
   __syncthreads();
-  if (tid == 0) {
-    const int ticket = atomicAdd(&meta[1 + rb], 1);
-    sm.is_last = (ticket == nch - 1);
-  }
-  __syncthreads();
-  if (!sm.is_last) return;
-  __threadfence();
-  for (int o = tid; o < ntk * 64; o += kDecThreads) {
-    const int tk = o >> 6, row = o & 63;
-    const int64_t n = rb * kDecRows + row;
-    if (tk < T && n < N) {
-      float v = 0.0f;
-      for (int c = 0; c < nch; ++c) v += __ldcg(&partial[((int64_t)c * 16 + tk) * N + n]);
-      Y[(int64_t)tk * N + n] = v;
+}
+
+// Y[t][n] = sum over chunks c (in order) of partial[c][t][n]; n4 = T*N/4.
+__global__ void __launch_bounds__(256) decode_reduce_kernel(const float4* __restrict__ partial, int64_t n4, int nch,
+                                                            float4* __restrict__ Y) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    float4 a = partial[i];
+    for (int c = 1; c < nch; ++c) {
+      const float4 b = partial[(int64_t)c * n4 + i];
+      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
     }
+    Y[i] = a;
   }
-  if (tid == 0) meta[1 + rb] = 0;
 }
 
 // ---- host side -----------------------------------------------------------------------
 
+static int64_t dec_chunks(int64_t K) { return (K / 128 + kDecChunk - 1) / kDecChunk; }
+
 size_t decode_ws_bytes(int64_t N, int64_t K) {
-  const int64_t ngroups = K / 128;
-  const int64_t nch = (ngroups + kDecGroups - 1) / kDecGroups;
-  const int64_t nrb = (N + kDecRows - 1) / kDecRows;
-  size_t b = 0;
-  b += (size_t)ngroups * 2048 * 2;                             // Xd: 2048 * NB bytes per group, NB <= 2
-  b = (b + 255) / 256 * 256;
-  b += (size_t)ngroups * 16 * sizeof(float);                   // xs
-  b = (b + 255) / 256 * 256;
-  b += (size_t)(1 + nrb) * sizeof(int32_t);                    // meta
-  b = (b + 255) / 256 * 256;
-  b += (size_t)nch * 16 * (size_t)N * sizeof(float);           // partials
-  return (b + 255) / 256 * 256;
+  const int64_t nch = dec_chunks(K);
+  if (nch <= 1) return 256;
+  return ((size_t)nch * 16 * (size_t)N * sizeof(float) + 255) / 256 * 256;  // partials for up to 16 tokens
 }
 
-static size_t dec_smem_bytes(int NB) {
-  return kDecSmemXd + (size_t)kDecGroups * 2048 * NB + 1024;  // + 1024 for the manual alignment
+// Grid of the decode kernel: (CTAs per chunk, chunks), one CTA per SM.
+void decode_grid(int64_t N, int64_t K, int sms, int64_t* cpc, int64_t* nch) {
+  *nch = dec_chunks(K);
+  const int64_t nblocks = (N + kDecRows - 1) / kDecRows;
+  int64_t c = sms / *nch;
+  if (c < 1) c = 1;
+  if (c > nblocks) c = nblocks;
+  *cpc = c;
+}
+
+template <int NB>
+static cudaError_t launch_decode_nb(const CUtensorMap& tm_codes, const CUtensorMap& tm_sz, const void* X, int T,
+                                    int64_t K, const int32_t* k_t, int64_t N, int S, float* out, int64_t cpc,
+                                    int64_t nch, cudaStream_t stream, DeviceStatus* st) {
+  using L = DecLayout<NB>;
+  cudaError_t e = set_smem((const void*)decode_kernel<NB>, (int)L::kDynamic);
+  if (e != cudaSuccess) return e;
+  decode_kernel<NB><<<dim3((unsigned)cpc, (unsigned)nch), L::kThreads, L::kDynamic, stream>>>(
+      tm_codes, tm_sz, static_cast<const __nv_bfloat16*>(X), k_t, T, (int)N, (int)K, (int)(K / 128), S,
+      (int)((N + kDecRows - 1) / kDecRows), out, st, wait_limit());
+  return note_error("decode launch", cudaGetLastError());
 }
 
 cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
                           const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
                           DeviceStatus* st) {
   const int64_t ngroups = K / 128;
-  const int64_t nch = (ngroups + kDecGroups - 1) / kDecGroups;
-  const int64_t nrb = (N + kDecRows - 1) / kDecRows;
-  const int NB = T > 8 ? 2 : 1;
-  uint8_t* p = static_cast<uint8_t*>(ws);
-  size_t off = 0;
-  uint32_t* Xd = reinterpret_cast<uint32_t*>(p + off);
-  off += (size_t)ngroups * 2048 * 2;
-  off = (off + 255) / 256 * 256;
-  float* xs = reinterpret_cast<float*>(p + off);
-  off += (size_t)ngroups * 16 * sizeof(float);
-  off = (off + 255) / 256 * 256;
-  int32_t* meta = reinterpret_cast<int32_t*>(p + off);
-  off += (size_t)(1 + nrb) * sizeof(int32_t);
-  off = (off + 255) / 256 * 256;
-  float* partial = reinterpret_cast<float*>(p + off);
+  int64_t cpc, nch;
+  decode_grid(N, K, num_sms(), &cpc, &nch);
+  float* partial = static_cast<float*>(ws);
+  float* out = nch > 1 ? partial : Y;
 
   CUtensorMap tm_codes, tm_sz;
-  if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4, 32, 64,
-                    true))
-    return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, 64, 8, false))
-    return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4, 32,
+                    kDecRows, true))
+    return note_error("decode tensor map (codes)", cudaErrorInvalidValue);
+  if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, kDecRows, kDecGW, false))
+    return note_error("decode tensor map (scale/zero)", cudaErrorInvalidValue);
 
-  decode_prep_kernel<<<(unsigned)ngroups, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T, K, NB, k_t,
-                                                             Xd, xs, meta, nrb, st);
-  const size_t smem = dec_smem_bytes(NB);
+  cudaError_t e = T > 8 ? launch_decode_nb<2>(tm_codes, tm_sz, X, T, K, k_t, N, S, out, cpc, nch, stream, st)
+                        : launch_decode_nb<1>(tm_codes, tm_sz, X, T, K, k_t, N, S, out, cpc, nch, stream, st);
+  if (e != cudaSuccess || nch <= 1) return e;
+
+  // Chunk reduction, launched as a programmatic dependent of the decode kernel.
+  const int64_t n4 = (int64_t)T * N / 4;
+  int64_t blocks = (n4 + 255) / 256;
+  const int64_t cap = (int64_t)num_sms() * 4;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)nrb, (unsigned)nch);
-  cfg.blockDim = dim3(kDecThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap with the staging kernel
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e;
-  const uint64_t lim = wait_limit();
-  if (NB == 2) {
-    if ((e = set_smem((const void*)decode_kernel<2>, (int)smem)) != cudaSuccess) return e;
-    e = cudaLaunchKernelEx(&cfg, decode_kernel<2>, tm_codes, tm_sz, (const uint32_t*)Xd, (const float*)xs, k_t, meta,
-                           T, N, ngroups, S, partial, Y, st, lim);
-  } else {
-    if ((e = set_smem((const void*)decode_kernel<1>, (int)smem)) != cudaSuccess) return e;
-    e = cudaLaunchKernelEx(&cfg, decode_kernel<1>, tm_codes, tm_sz, (const uint32_t*)Xd, (const float*)xs, k_t, meta,
-                           T, N, ngroups, S, partial, Y, st, lim);
-  }
-  if (e != cudaSuccess) return note_error("decode launch", e);
+  e = cudaLaunchKernelEx(&cfg, decode_reduce_kernel, (const float4*)partial, n4, (int)nch,
+                         reinterpret_cast<float4*>(Y));
+  if (e != cudaSuccess) return note_error("decode reduce launch", e);
   return note_error("kernel launch", cudaGetLastError());
 }
 
