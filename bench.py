@@ -168,6 +168,13 @@ class DecodeCase:
         return int(self.k_t.max().item())
 
 
+def launches_per_call(T, K):
+    """Library kernels one route + GEMM call launches (T <= 16): the one-cluster
+    route kernel, the decode kernel and, when K spans more than one 1024-column
+    chunk, the chunk-reduce kernel."""
+    return 1 + 1 + (1 if K > 1024 else 0)
+
+
 def build_decode_cases(mobi, wl, dev):
     cases = []
     for (N, K) in wl.DECODE_SHAPES:
@@ -285,7 +292,7 @@ def run_gpu(args, world, rank):
     kmax = [c.kmax() for c in cases]
     bytes_step = sum(decode_bytes(c.N, c.K, c.T, km) for c, km in zip(cases, kmax))
 
-    # Capture one step (9 x (route + GEMM) = 36 kernel launches) in a CUDA graph.
+    # Capture one step (9 x (route + GEMM), 27 kernel launches) in a CUDA graph.
     stream = torch.cuda.Stream()
     stream.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(stream):
@@ -297,7 +304,7 @@ def run_gpu(args, world, rank):
     with torch.cuda.graph(graph):
         for c in cases:
             c.step()
-    launches_per_step = 4 * len(cases)
+    launches_per_step = sum(launches_per_call(c.T, c.K) for c in cases)
 
     for _ in range(max(args.warmup, 3)):
         graph.replay()

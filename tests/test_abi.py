@@ -68,9 +68,10 @@ def test_route_validation(L):
     assert L.mobi_route(*args(S=0)) == 1
     assert L.mobi_route(*args(X=None)) == 1
     assert L.mobi_route(*args(X=p(FAKE + 8))) == 3
-    T, K = 1, 4096  # small T splits K and needs a workspace
+    T, K = 32, 4096  # two token tiles: K is split, which needs a workspace
     assert mobi.mobi_route_workspace_bytes(T, K, 3) > 0
     assert L.mobi_route(*args(T=T, K=K)) == 4
+    assert mobi.mobi_route_workspace_bytes(16, K, 3) == 0  # up to 16 tokens: one cluster launch, no workspace
 
 
 def test_gemm_validation(L):

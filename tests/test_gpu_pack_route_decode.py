@@ -76,6 +76,7 @@ def test_pack_slices_1_and_2(mobi, oracle):
 # ---- route -------------------------------------------------------------------------
 
 @pytest.mark.parametrize("T,K,mix", [(16, 512, None), (1, 4096, None), (3, 11008, None), (17, 256, None),
+                                     (16, 128, None), (16, 11008, (0.5, 0.3, 0.2)), (9, 4096, (0.1, 0.1, 0.8)),
                                      (100, 1024, (0.2, 0.3, 0.5)), (2048, 4096, (1 / 3, 1 / 3, 1 / 3)),
                                      (1500, 2048, (0.7, 0.2, 0.1))])
 def test_route_and_bucket(mobi, oracle, T, K, mix):
@@ -89,6 +90,22 @@ def test_route_and_bucket(mobi, oracle, T, K, mix):
     k_gpu = k_t.cpu().numpy()
     check_route(k_gpu, k_ref, gap, f"T={T}")
     perm_ref, off_ref = oracle.bucket(k_gpu)
+    assert np.array_equal(perm.cpu().numpy(), perm_ref)
+    assert np.array_equal(off.cpu().numpy(), off_ref)
+
+
+@pytest.mark.parametrize("S", [1, 2])
+@pytest.mark.parametrize("T", [1, 13])
+def test_route_small_fewer_slices(mobi, oracle, T, S):
+    """Up to 16 tokens (one cluster launch) with one or two slices."""
+    L = wl.layer("r", 16, 1024, T, seed=300 + T + S)
+    Wr = np.ascontiguousarray(L.Wr[:, :S])
+    k_ref, gap, _ = oracle.route(L.X, Wr, None)
+    k_t, perm, off = mobi.mobi_route(L.X.to(DEV), torch.from_numpy(Wr).to(DEV))
+    mobi.mobi_sync_check()
+    k_gpu = k_t.cpu().numpy()
+    check_route(k_gpu, k_ref, gap, f"T={T} S={S}")
+    perm_ref, off_ref = oracle.bucket(k_gpu, S)
     assert np.array_equal(perm.cpu().numpy(), perm_ref)
     assert np.array_equal(off.cpu().numpy(), off_ref)
 

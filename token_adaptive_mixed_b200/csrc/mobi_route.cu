@@ -14,6 +14,8 @@
 // bucket_kernel: one CTA. Finishes the K-split logits (if any), takes the
 //   argmax, then counts and scatters the tokens in index order with warp
 //   ballots, which keeps the sort stable.
+// route_small_kernel (T <= 16, the decode case): both steps in one launch of
+//   one thread-block cluster; see below.
 #include <cstdint>
 
 #include "mobi_device.cuh"
@@ -195,6 +197,141 @@ __global__ void __launch_bounds__(kBucketThreads) bucket_kernel(int64_t T, int k
   }
 }
 
+// ---- small batches (T <= 16): one launch of one 8-CTA cluster ------------------------
+//
+// CTA r of the cluster sums the logits of every token over its share of the
+// 8-column octets of K (fp32 within a thread, fp32 xor tree within a warp,
+// fp64 across warps), keeps them in its shared memory, and after a cluster
+// barrier CTA 0 adds the eight partials in rank order through distributed
+// shared memory (fp64), takes the argmax and writes the stable bucketing
+// (warp ballots over the at most 16 tokens). A second cluster barrier keeps
+// the other CTAs alive until CTA 0 has read their partials.
+constexpr int kRouteSmallT = 16;
+constexpr int kRouteCluster = 8;
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of `p` (this CTA's shared memory) in the shared memory of cluster CTA `rank`.
+__device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ double ld_dsmem_f64(uint32_t addr) {
+  double v;
+  asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+template <int S>
+__global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
+    const __nv_bfloat16* __restrict__ X, int T, int64_t K, const float* __restrict__ Wr,
+    const float* __restrict__ bias, int32_t* __restrict__ k_t, int32_t* __restrict__ perm,
+    int32_t* __restrict__ offsets) {
+  __shared__ float red[kRouteThreads / 32][kRouteSmallT * S];
+  __shared__ double part[kRouteSmallT * S];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t rank;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+  const int64_t noct = K / 8;
+  const int64_t o_beg = rank * noct / kRouteCluster, o_end = (rank + 1) * noct / kRouteCluster;
+
+  float acc[kRouteSmallT][S];
+#pragma unroll
+  for (int i = 0; i < kRouteSmallT; ++i)
+#pragma unroll
+    for (int j = 0; j < S; ++j) acc[i][j] = 0.0f;
+  for (int64_t o = o_beg + tid; o < o_end; o += kRouteThreads) {
+    const int64_t k = 8 * o;
+    float w[8][S];
+#pragma unroll
+    for (int e = 0; e < 8 * S; ++e) w[e / S][e % S] = __ldg(Wr + k * S + e);
+#pragma unroll
+    for (int i = 0; i < kRouteSmallT; ++i) {
+      if (i < T) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(X + (int64_t)i * K + k));
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float x0 = bf16lo(u[p]), x1 = bf16hi(u[p]);
+#pragma unroll
+          for (int j = 0; j < S; ++j) {
+            acc[i][j] = fmaf(x0, w[2 * p][j], acc[i][j]);
+            acc[i][j] = fmaf(x1, w[2 * p + 1][j], acc[i][j]);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kRouteSmallT; ++i)
+#pragma unroll
+    for (int j = 0; j < S; ++j) {
+      float v = acc[i][j];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) red[warp][i * S + j] = v;
+    }
+  __syncthreads();
+  if (tid < kRouteSmallT * S) {
+    double s = 0.0;
+    for (int w8 = 0; w8 < kRouteThreads / 32; ++w8) s += (double)red[w8][tid];
+    part[tid] = s;
+  }
+  cluster_sync_all();  // every CTA's partial logits are in its shared memory
+
+  if (rank == 0 && warp == 0) {
+    // Lane t < T: the logits of token t, partials added in rank order.
+    int k = 0;
+    if (lane < T) {
+      double l[S];
+#pragma unroll
+      for (int j = 0; j < S; ++j) {
+        double s = 0.0;
+        for (uint32_t r = 0; r < kRouteCluster; ++r) s += ld_dsmem_f64(dsmem_addr(&part[lane * S + j], r));
+        l[j] = s + (bias ? (double)__ldg(bias + j) : 0.0);
+      }
+      k = 1 + argmax_lowest(l, S);
+      k_t[lane] = k;
+    }
+    // Stable bucketing: tokens of value v keep their index order.
+    int run = 0;
+#pragma unroll
+    for (int j = 0; j < S; ++j) {
+      const unsigned m = __ballot_sync(0xffffffffu, k == j + 1);
+      if (lane == 0) offsets[j] = run;
+      if (k == j + 1) perm[run + __popc(m & ((1u << lane) - 1u))] = lane;
+      run += __popc(m);
+    }
+    if (lane == 0) offsets[S] = run;
+  }
+  cluster_sync_all();  // CTA 0 is done reading the others' shared memory
+}
+
+template <int S>
+static cudaError_t launch_route_small(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
+                                      int32_t* k_t, int32_t* perm, int32_t* offsets, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kRouteCluster);
+  cfg.blockDim = dim3(kRouteThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kRouteCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, route_small_kernel<S>, static_cast<const __nv_bfloat16*>(X), (int)T, K,
+                                           Wr, bias, k_t, perm, offsets);
+  if (e != cudaSuccess) return note_error("route launch", e);
+  return note_error("kernel launch", cudaGetLastError());
+}
+
 int route_ksplit(int64_t T, int64_t K) {
   const int64_t tiles = (T + kRouteTB - 1) / kRouteTB;
   if (tiles == 0 || tiles >= 64) return 1;
@@ -206,6 +343,7 @@ int route_ksplit(int64_t T, int64_t K) {
 }
 
 size_t route_ws_bytes(int64_t T, int64_t K, int S) {
+  if (T >= 1 && T <= kRouteSmallT) return 0;  // one cluster launch, no workspace
   const int ks = route_ksplit(T, K);
   return ks > 1 ? (size_t)ks * (size_t)T * (size_t)S * sizeof(double) : 0;
 }
@@ -214,6 +352,7 @@ template <int S>
 static cudaError_t launch_route_s(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
                                   int32_t* k_t, int32_t* perm, int32_t* offsets, void* ws,
                                   cudaStream_t stream) {
+  if (T >= 1 && T <= kRouteSmallT) return launch_route_small<S>(X, T, K, Wr, bias, k_t, perm, offsets, stream);
   const int ks = route_ksplit(T, K);
   int64_t kps = (K + ks - 1) / ks;
   kps = (kps + 7) / 8 * 8;  // whole 8-column octets per split
