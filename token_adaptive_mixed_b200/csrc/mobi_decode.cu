@@ -21,14 +21,14 @@
 //
 // Work split (persistent, one CTA per SM). K is cut into chunks of 8 groups
 // (1024 columns); a CTA owns one chunk and a contiguous range of 32-row
-// blocks (two 16-row MMA tiles each). Its warps form teams of two: both warps
-// of a team work on the same block, each on 4 of the chunk's 8 groups, and the
-// odd warp hands its sums to the even one through shared memory. A warp keeps
-// the activation fragments of its 4 groups in registers for the whole kernel
-// (built once from X) and runs its own TMA ring of (block, slice) stages, so
-// code bytes stream in while earlier stages are multiplied. A stage carries
-// 64 MMAs, enough to cover the fixed cost of its barrier wait and refill.
-// Chunks are combined by a second,
+// blocks (two 16-row MMA tiles each). Its consumer warps form teams of four:
+// the warps of a team work on the same block, each on 2 of the chunk's 8
+// groups, and hand their sums to the team's first warp through shared
+// memory. A warp keeps the activation fragments of its 2 groups in registers
+// for the whole kernel (built once from X), which keeps its unrolled stage
+// code small enough for the instruction cache. One producer warp feeds a
+// TMA ring per consumer warp with (block, slice) stages, so code bytes stream
+// in while earlier stages are multiplied. Chunks are combined by a second,
 // programmatically dependent kernel that adds the per-chunk partials in chunk
 // order (deterministic).
 #include <cstdint>
@@ -41,34 +41,41 @@
 
 namespace mobi {
 
-constexpr int kDecGW = 4;                    // groups per warp (128 bytes of a code row)
-constexpr int kDecChunk = 2 * kDecGW;        // groups per CTA chunk (two warps per tile)
+constexpr int kDecGW = 2;                    // groups per warp (64 bytes of a code row)
+constexpr int kDecQ = 4;                     // warps per team (one team per 32-row block)
+constexpr int kDecChunk = kDecQ * kDecGW;    // groups per CTA chunk
 constexpr int kDecRows = 32;                 // rows per stage: two 16-row MMA tiles
-constexpr uint32_t kDecSlotCodes = kDecRows * 128;     // one stage: 32 rows x 128 bytes of codes
-constexpr uint32_t kDecSlotSz = kDecGW * kDecRows * 4;  // and [4 groups][32 rows] scale/zero words
+constexpr uint32_t kDecRowBytes = kDecGW * 32;               // code bytes of one row in a stage
+constexpr uint32_t kDecSlotCodes = kDecRows * kDecRowBytes;  // one stage: 32 rows x 64 bytes of codes
+constexpr uint32_t kDecSlotSz = kDecGW * kDecRows * 4;       // and [2 groups][32 rows] scale/zero words
 
 template <int NB>
 struct DecCfg;
 template <>
 struct DecCfg<1> {  // T <= 8: 16 B-fragment registers per group
-  static constexpr int kTeams = 5;
+  static constexpr int kTeams = 4;
   static constexpr int kDepth = 4;
 };
 template <>
 struct DecCfg<2> {  // T <= 16: 32 per group
-  static constexpr int kTeams = 3;
-  static constexpr int kDepth = 5;
+  static constexpr int kTeams = 2;
+  static constexpr int kDepth = 8;
 };
 
 template <int NB>
 struct DecLayout {
-  static constexpr int kWarps = 2 * DecCfg<NB>::kTeams;  // consumer warps; one producer warp follows
+  static constexpr int kWarps = kDecQ * DecCfg<NB>::kTeams;  // consumer warps; one producer warp follows
   static constexpr int kThreads = 32 * (kWarps + 1);
+  // Registers per thread for one CTA: the warps are spread over the SM's four
+  // 16K-register sub-partitions, so the fullest one decides.
+  static constexpr int kMaxRegs = (16384 / (32 * ((kWarps + 4) / 4))) / 8 * 8 > 248
+                                      ? 248
+                                      : (16384 / (32 * ((kWarps + 4) / 4))) / 8 * 8;
   static constexpr int kDepth = DecCfg<NB>::kDepth;
-  static constexpr uint32_t kCodes = 0;                                              // [warp][slot] 4 KB, 1 KB aligned
-  static constexpr uint32_t kSz = kCodes + kWarps * kDepth * kDecSlotCodes;          // [warp][slot][4][32]
-  static constexpr uint32_t kXchg = kSz + kWarps * kDepth * kDecSlotSz;              // [team][2][32][8 NB] floats
-  static constexpr uint32_t kBar = kXchg + DecCfg<NB>::kTeams * 2 * 32 * 8 * NB * 4;  // full, empty [warp][slot]
+  static constexpr uint32_t kCodes = 0;                                      // [warp][slot] 2 KB, 1 KB aligned
+  static constexpr uint32_t kSz = kCodes + kWarps * kDepth * kDecSlotCodes;  // [warp][slot][2][32]
+  static constexpr uint32_t kXchg = kSz + kWarps * kDepth * kDecSlotSz;      // [team][2][kDecQ-1][32][8 NB] floats
+  static constexpr uint32_t kBar = kXchg + DecCfg<NB>::kTeams * 2 * (kDecQ - 1) * 32 * 8 * NB * 4;  // full, empty
   static constexpr uint32_t kReady = kBar + 2 * kWarps * kDepth * 8;  // consumers' fragments built
   static constexpr uint32_t kAbort = kReady + 8;
   static constexpr uint32_t kBytes = kAbort + 8;
@@ -101,9 +108,9 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// Issue one stage of a warp into ring slot `slot`: the warp's 128-byte slice
-// of 32 code rows (x = word column, y = s*N + row) and the matching
-// [4 groups][32 rows] scale/zero words.
+// Issue one stage of a warp into ring slot `slot`: the warp's 64-byte slice
+// of 32 code rows (x = word column, y = s*N + row; 64-byte swizzle) and the
+// matching [2 groups][32 rows] scale/zero words.
 // Weights are read once per call, so they go in with L2 evict-first.
 __device__ __forceinline__ void dec_issue(const CUtensorMap* tm_codes, const CUtensorMap* tm_sz, uint8_t* codes_slot,
                                           uint32_t* sz_slot, uint64_t* bar, int block, int s, int N, int ngroups,
@@ -125,8 +132,8 @@ __device__ __forceinline__ void dec_group_pair(int g0, const uint8_t* cs, const 
   for (int gg = 0; gg < 2; ++gg)
 #pragma unroll
     for (int tt = 0; tt < TT; ++tt) {
-      wa[gg][tt] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + tt * 16 * 128);
-      wb[gg][tt] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + tt * 16 * 128 + 8 * 128);
+      wa[gg][tt] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + tt * 16 * kDecRowBytes);
+      wb[gg][tt] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + tt * 16 * kDecRowBytes + 8 * kDecRowBytes);
     }
   float d[2][TT][NB][4];
 #pragma unroll
@@ -180,16 +187,15 @@ __device__ __forceinline__ void dec_group_pair(int g0, const uint8_t* cs, const 
   }
 }
 
-// One stage: the warp's ngv valid groups (warp-uniform) for TT tiles.
+// One stage: the warp's groups for TT tiles.
 template <int NB, int TT>
 __device__ __forceinline__ void dec_stage(int ngv, const uint8_t* cs, const uint32_t* ss,
                                           const uint32_t (&coff)[kDecGW], const uint32_t (&B)[kDecGW][8][2 * NB],
                                           const float2 (&xs)[kDecGW][NB], const float2 (&m37)[NB],
                                           const float2 (&m1)[NB], int gid, float2 (&yA)[2][NB], float2 (&yB)[2][NB]) {
-  // A group beyond K has zero activations and zero-filled codes, so it only
-  // costs time; the pair loop skips whole pairs past the last valid group.
+  // A group beyond K has zero activations and zero-filled codes: it adds 0.
+  (void)ngv;
   dec_group_pair<NB, TT>(0, cs, ss, coff, B, xs, m37, m1, gid, yA, yB);
-  if (ngv > 2) dec_group_pair<NB, TT>(2, cs, ss, coff, B, xs, m37, m1, gid, yA, yB);
 }
 
 // Bounded wait that also gives up once another warp has aborted.
@@ -207,9 +213,9 @@ __device__ __forceinline__ bool dec_wait(uint64_t* bar, uint32_t parity, uint64_
 // grid = (CTAs per chunk, chunks). out = Y when there is one chunk, else the
 // per-chunk partials [chunk][T][N]. All loop bookkeeping is incremental
 // 32-bit arithmetic (sizes are validated to N, K < 2^28).
-// Warps 0 .. kWarps-1 consume (teams of two), warp kWarps issues the copies.
+// Warps 0 .. kWarps-1 consume (teams of four), warp kWarps issues the copies.
 template <int NB>
-__global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
+__global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLayout<NB>::kMaxRegs) decode_kernel(
     const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_sz,
     const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ k_t, int T, int N, int K, int ngroups, int S,
     int nblocks, float* __restrict__ out, DeviceStatus* st, uint64_t limit) {
@@ -235,57 +241,61 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
   uint64_t* ready = reinterpret_cast<uint64_t*>(sm + L::kReady);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(sm + L::kAbort);
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kW * D; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    mbar_init(ready, kW);
-    *abort_flag = 0;
-    fence_barrier_init();
+  // One barrier per thread (about 130 in all), then one fence per warp.
+  for (int i = threadIdx.x; i < 2 * kW * D + 1; i += blockDim.x) {
+    if (i < kW * D) mbar_init(&full[i], 1);
+    else if (i < 2 * kW * D) mbar_init(&empty[i - kW * D], 1);
+    else mbar_init(ready, kW);
   }
+  if (threadIdx.x == 0) *abort_flag = 0;
+  if (lane == 0) fence_barrier_init();
   __syncthreads();
 
   if (warp == kW) {
-    // ---------------- producer: one thread feeds every consumer's ring ----------------
-    int niss[kW];  // items issued per consumer warp
-#pragma unroll
-    for (int w = 0; w < kW; ++w) niss[w] = 0;
-    // The consumers' activation loads go out before the first weight copy.
-    named_bar_sync(15, 32 * (kW + 1));
+    // ---------------- producer: lane w feeds consumer warp w's ring ----------------
+    // All lanes poll their ring's empty barrier in one non-blocking test and
+    // issue their copies together, so one poll serves every consumer warp.
+    named_bar_sync(15, 32 * (kW + 1));  // the consumers' activation loads go out first
     if (lane == 0) {
       prefetch_tmap(&tm_codes);
       prefetch_tmap(&tm_sz);
-      const uint64_t policy = l2_evict_first_policy();
-      int kmax = 1;
-      for (int t = 0; t < T; ++t) kmax = max(kmax, (int)__ldg(k_t + t));
-      kmax = kmax > S ? S : kmax;
-      int nit[kW];  // items of each consumer warp: its blocks x kmax (0 past the last group)
-      int maxit = 0;
-#pragma unroll
-      for (int w = 0; w < kW; ++w) {
-        const int team = w >> 1, gb = ch * kDecChunk + (w & 1) * kDecGW;
-        const int myb = b_end - b_begin > team ? (b_end - b_begin - team + kTeams - 1) / kTeams : 0;
-        nit[w] = gb < ngroups ? myb * kmax : 0;
-        maxit = max(maxit, nit[w]);
-      }
-      bool ok = true;
-      int slot = 0, bo = 0, s = 0;  // round r: slot r % D, block offset r / kmax, slice r % kmax
-      uint32_t eph = 1;             // parity of the empty phase that frees `slot` in round r (r >= D)
-      for (int r = 0; r < maxit && ok; ++r) {
-        // Two stages per consumer first; the rest once every consumer has its
-        // activations, so that those small loads do not queue behind the ring.
-        if (r == 2 && !(ok = dec_wait(ready, 0, limit, st, 0x2e1, abort_flag))) break;
-#pragma unroll
-        for (int w = 0; w < kW; ++w) {
-          if (r < nit[w] && ok) {
-            if (r >= D && !(ok = dec_wait(&empty[w * D + slot], eph, limit, st, 0x2e0, abort_flag))) break;
-            const int team = w >> 1, gb = ch * kDecChunk + (w & 1) * kDecGW;
-            dec_issue(&tm_codes, &tm_sz, sm + L::kCodes + (uint32_t)(w * D + slot) * kDecSlotCodes,
-                      reinterpret_cast<uint32_t*>(sm + L::kSz + (uint32_t)(w * D + slot) * kDecSlotSz),
-                      &full[w * D + slot], b_begin + team + bo * kTeams, s, N, ngroups, gb, policy);
-            ++niss[w];
-          }
+    }
+    const uint64_t policy = l2_evict_first_policy();
+    int kmax = __reduce_max_sync(0xffffffffu, lane < T ? (int)__ldg(k_t + lane) : 1);
+    kmax = kmax < 1 ? 1 : (kmax > S ? S : kmax);
+    const int w = lane;
+    const int team = w / kDecQ, gb = ch * kDecChunk + (w % kDecQ) * kDecGW;
+    const int myb = (w < kW && b_end - b_begin > team) ? (b_end - b_begin - team + kTeams - 1) / kTeams : 0;
+    const int nit = (w < kW && gb < ngroups) ? myb * kmax : 0;  // items of warp w: blocks x slices
+    int r = 0, bo = 0, s = 0;  // next item of warp w: its index, block offset and slice
+    bool gate = false;         // every consumer has built its activations
+    bool ok = true;
+    uint64_t idle = 0;         // polls in a row without a copy issued
+    while (true) {
+      // Two stages per consumer first; the rest once every consumer has its
+      // activations, so that those small loads do not queue behind the rings.
+      if (!gate) gate = __shfl_sync(0xffffffffu, lane == 0 ? (int)mbar_test_wait(ready, 0) : 0, 0) != 0;
+      bool issued = false;
+      if (ok && r < nit && (r < 2 || gate)) {
+        const int slot = r % D;
+        if (r < D || mbar_test_wait(&empty[w * D + slot], (uint32_t)(((r / D) & 1) ^ 1))) {
+          dec_issue(&tm_codes, &tm_sz, sm + L::kCodes + (uint32_t)(w * D + slot) * kDecSlotCodes,
+                    reinterpret_cast<uint32_t*>(sm + L::kSz + (uint32_t)(w * D + slot) * kDecSlotSz),
+                    &full[w * D + slot], b_begin + team + bo * kTeams, s, N, ngroups, gb, policy);
+          ++r;
+          if (++s == kmax) { s = 0; ++bo; }
+          issued = true;
         }
-        if (++s == kmax) { s = 0; ++bo; }
-        if (++slot == D) { slot = 0; eph = r + 1 >= D ? eph ^ 1u : 0u; }
+      }
+      if (!__any_sync(0xffffffffu, ok && r < nit)) break;
+      if (__any_sync(0xffffffffu, issued)) {
+        idle = 0;
+      } else if (++idle >= limit || ((idle & 255) == 0 && *abort_flag)) {
+        if (idle >= limit && lane == 0) {
+          report_error(st, kErrTimeout, 0x2e0);
+          *abort_flag = 1;
+        }
+        ok = false;
       }
     }
     // Normally the consumers have waited for every copy. If any warp gave up,
@@ -293,26 +303,24 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
     // copy into a slot completes after the earlier ones).
     __syncwarp();
     __syncthreads();  // all consumers are done
-    if (lane == 0 && *abort_flag) {
-#pragma unroll
-      for (int w = 0; w < kW; ++w)
-        for (int sl = 0; sl < D && sl < niss[w]; ++sl) {
-          const int last = sl + (niss[w] - 1 - sl) / D * D;
-          mbar_wait(&full[w * D + sl], (uint32_t)((last / D) & 1), kDefaultWaitLimit, st, 0x2f0);
-        }
+    if (*abort_flag) {
+      for (int sl = 0; sl < D && sl < r; ++sl) {
+        const int last = sl + (r - 1 - sl) / D * D;
+        mbar_wait(&full[w * D + sl], (uint32_t)((last / D) & 1), kDefaultWaitLimit, st, 0x2f0);
+      }
     }
     return;
   }
 
   // ---------------- consumers ----------------
   const int gid = lane >> 2, t4 = lane & 3;
-  const int team = warp >> 1, q = warp & 1;
+  const int team = warp / kDecQ, q = warp % kDecQ;
   const int gbase = ch * kDecChunk + q * kDecGW;  // first group of this warp
   const int ngv = ngroups - gbase < 0 ? 0 : (ngroups - gbase > kDecGW ? kDecGW : ngroups - gbase);
   const int my_blocks = b_end - b_begin > team ? (b_end - b_begin - team + kTeams - 1) / kTeams : 0;
   const uint8_t* codes_w = sm + L::kCodes + (uint32_t)warp * D * kDecSlotCodes;
   const uint32_t* sz_w = reinterpret_cast<const uint32_t*>(sm + L::kSz + (uint32_t)warp * D * kDecSlotSz);
-  float* xchg = reinterpret_cast<float*>(sm + L::kXchg) + team * 2 * 32 * 8 * NB;
+  float* xchg = reinterpret_cast<float*>(sm + L::kXchg) + team * 2 * (kDecQ - 1) * 32 * 8 * NB;
   uint64_t* full_w = full + warp * D;
   uint64_t* empty_w = empty + warp * D;
 
@@ -402,13 +410,14 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
     ktl[nb][1] = __shfl_sync(0xffffffffu, my_kt, 2 * t4 + 1 + 8 * nb);
   }
 
-  // Code words 2 t4, 2 t4 + 1 of group g of row gid in the 128-byte-swizzled
-  // stage (16-byte chunk c of row r sits at c ^ (r & 7)); rows gid + 8, +16,
-  // +24 share the swizzle and sit 1, 2, 3 KB further on.
+  // Code words 2 t4, 2 t4 + 1 of group g of row gid in the 64-byte-swizzled
+  // stage (16-byte chunk c of row r sits at c ^ ((r >> 1) & 3)); rows gid + 8,
+  // +16, +24 share the swizzle and sit 512 bytes apart.
   uint32_t coff[kDecGW];
 #pragma unroll
   for (int g = 0; g < kDecGW; ++g)
-    coff[g] = (uint32_t)gid * 128u + (uint32_t)(((2 * g + (t4 >> 1)) ^ gid) * 16) + (t4 & 1) * 8u;
+    coff[g] = (uint32_t)gid * kDecRowBytes + (uint32_t)(((2 * g + (t4 >> 1)) ^ ((gid >> 1) & 3)) * 16) +
+              (t4 & 1) * 8u;
 
   // y[tt][nb]: tile tt of the block, rows gid (A) and gid + 8 (B) of it,
   // tokens (2 t4, 2 t4 + 1) + 8 nb.
@@ -448,17 +457,19 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
     }
     if (++slot == D) { slot = 0; parity ^= 1u; }
     if (s == kmax - 1) {
-      // Team hand-off: the odd warp's 4 groups join the even warp's.
-      float* xb = xchg + ((blk_i & 1) * 32 + lane) * 8 * NB;
-      if (q == 1) {
+      // Team hand-off: warps 1..3 of the team pass their groups' sums to
+      // warp 0, which adds them in warp order.
+      float* xb = xchg + (blk_i & 1) * (kDecQ - 1) * 32 * 8 * NB;
+      if (q > 0) {
+        float* mine = xb + ((q - 1) * 32 + lane) * 8 * NB;
 #pragma unroll
         for (int tt = 0; tt < 2; ++tt)
 #pragma unroll
           for (int nb = 0; nb < NB; ++nb)
-            *reinterpret_cast<float4*>(xb + 8 * nb + 4 * tt) =
+            *reinterpret_cast<float4*>(mine + 8 * nb + 4 * tt) =
                 make_float4(yA[tt][nb].x, yA[tt][nb].y, yB[tt][nb].x, yB[tt][nb].y);
       }
-      named_bar_sync(1 + team, 64);
+      named_bar_sync(1 + team, 32 * kDecQ);
       if (q == 0) {
         float* o = out + (int64_t)ch * T * N + blk * kDecRows;
 #pragma unroll
@@ -466,8 +477,12 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
           if (tt == 1 && !two) break;
 #pragma unroll
           for (int nb = 0; nb < NB; ++nb) {
-            const float4 p = *reinterpret_cast<const float4*>(xb + 8 * nb + 4 * tt);
-            const float v[4] = {yA[tt][nb].x + p.x, yA[tt][nb].y + p.y, yB[tt][nb].x + p.z, yB[tt][nb].y + p.w};
+            float v[4] = {yA[tt][nb].x, yA[tt][nb].y, yB[tt][nb].x, yB[tt][nb].y};
+#pragma unroll
+            for (int w = 0; w < kDecQ - 1; ++w) {
+              const float4 p = *reinterpret_cast<const float4*>(xb + (w * 32 + lane) * 8 * NB + 8 * nb + 4 * tt);
+              v[0] += p.x; v[1] += p.y; v[2] += p.z; v[3] += p.w;
+            }
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int tk = 2 * t4 + 8 * nb + e;
@@ -552,10 +567,10 @@ cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, c
   float* out = nch > 1 ? partial : Y;
 
   CUtensorMap tm_codes, tm_sz;
-  if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4, 32,
-                    kDecRows, true))
+  if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4,
+                    kDecGW * 8, kDecRows, 64))
     return note_error("decode tensor map (codes)", cudaErrorInvalidValue);
-  if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, kDecRows, kDecGW, false))
+  if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, kDecRows, kDecGW, 0))
     return note_error("decode tensor map (scale/zero)", cudaErrorInvalidValue);
 
   cudaError_t e = T > 8 ? launch_decode_nb<2>(tm_codes, tm_sz, X, T, K, k_t, N, S, out, cpc, nch, stream, st)

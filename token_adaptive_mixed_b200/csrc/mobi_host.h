@@ -23,8 +23,9 @@ int num_sms();
 cudaError_t set_smem(const void* func, int bytes);
 
 // 2-D tiled tensor map over a row-major [rows][cols] array of `elem_bytes`
-// elements (cols innermost), box [box_rows][box_cols], optional 128-byte swizzle.
+// elements (cols innermost), box [box_rows][box_cols]; swizzle_bytes is 0 (none),
+// 32, 64 or 128 (the shared-memory swizzle span of the copied tile).
 bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t cols, uint64_t rows,
-                  uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128);
+                  uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes);
 
 }  // namespace mobi

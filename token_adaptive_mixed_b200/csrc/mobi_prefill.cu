@@ -528,9 +528,9 @@ cudaError_t launch_prefill(const void* X, int64_t T, int64_t K, const int32_t* k
   uint8_t* Xt = static_cast<uint8_t*>(ws);
   CUtensorMap tm_codes, tm_sz;
   if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4, 8, pf::BM,
-                    false))
+                    0))
     return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, pf::BM, 1, false))
+  if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, pf::BM, 1, 0))
     return cudaErrorInvalidValue;
 
   const int64_t blocks_g = (T_pad * (K / 16) + 255) / 256;
