@@ -37,7 +37,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "mixed-bit GEMM: decode HBM GB/s & prefill TFLOP/s, % of B200 roofline"
 WORKLOAD = ("decode GEMV, Llama-7B projections (N,K) in {(4096,4096),(11008,4096),(4096,11008)} "
-            "x T in {1,4,16}, 3x2-bit slices, group 128, route+bucket+GEMM per call")
+            "x T in {1,4,16}, 3x2-bit slices, group 128, route+bucket+GEMM per call (mobi_linear)")
 
 
 def peaks():
@@ -152,6 +152,7 @@ class DecodeCase:
         self.Y_host = torch.empty((T, N), dtype=torch.float32).pin_memory()
         self.ws_r = torch.empty(max(mobi.mobi_route_workspace_bytes(T, K, 3), 16), dtype=torch.uint8, device=dev)
         self.ws_g = torch.empty(mobi.mobi_gemm_workspace_bytes(T, N, K, 3), dtype=torch.uint8, device=dev)
+        self.ws_l = torch.empty(max(mobi.mobi_linear_workspace_bytes(T, N, K, 3), 16), dtype=torch.uint8, device=dev)
         self.mobi = mobi
 
     def route(self):
@@ -161,8 +162,9 @@ class DecodeCase:
         self.mobi.mobi_gemm(self.X, self.k_t, self.perm, self.off, self.codes, self.sz, self.N, Y=self.Y, ws=self.ws_g)
 
     def step(self):
-        self.route()
-        self.gemm()
+        """One layer call through the public API: routing + GEMM (mobi_linear)."""
+        self.mobi.mobi_linear(self.X, self.Wr, None, self.codes, self.sz, self.N, Y=self.Y, k_t=self.k_t,
+                              perm=self.perm, offsets=self.off, ws=self.ws_l)
 
     def kmax(self):
         return int(self.k_t.max().item())

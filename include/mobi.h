@@ -180,6 +180,33 @@ MOBI_API mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const i
                            int G, int S, float* Y, void* ws, size_t ws_bytes,
                            void* stream, int path);
 
+/* Scratch bytes of mobi_linear: the routing workspace (rounded up to 256
+ * bytes) followed by the GEMM workspace. */
+MOBI_API size_t mobi_linear_workspace_bytes(int64_t T, int64_t N, int64_t K, int S);
+
+/*
+ * mobi_linear — the token-routed mixed-bit linear layer in one call:
+ *   mobi_route followed by mobi_gemm on the same stream, with the same
+ *   arguments, outputs and results ([ja] §2.2 then §2.1; [en] §2.B then §2.A).
+ *   X, Wr, bias, k_t, perm, offsets as for mobi_route; codes, sz, N, G, S, Y
+ *   as for mobi_gemm (S is the router's column count as well).
+ *   ws       scratch of mobi_linear_workspace_bytes(T, N, K, S) bytes (may be
+ *            NULL when that size is 0); the first
+ *            align256(mobi_route_workspace_bytes) bytes serve the routing step.
+ * What the single call adds: for T <= 16 the decode kernel is launched as a
+ * programmatic dependent of the routing kernel and, knowing that kernel
+ * writes only k_t, perm and offsets, loads X and its first weight stages
+ * before waiting on it, so the routing time is hidden behind the GEMM's
+ * start. Nothing in X, Wr, bias, codes or sz may be written by other work
+ * while the call runs. Errors as for mobi_route and mobi_gemm; nothing is
+ * launched when an argument is rejected.
+ */
+MOBI_API mobi_status mobi_linear(const void* X, int64_t T, int64_t K, const float* Wr,
+                                 const float* bias, const uint32_t* codes, const uint32_t* sz,
+                                 int64_t N, int G, int S, int32_t* k_t, int32_t* perm,
+                                 int32_t* offsets, float* Y, void* ws, size_t ws_bytes,
+                                 void* stream);
+
 /*
  * mobi_gemm_decode_noalloc — the decode GEMM (T <= 16) without a workspace.
  *   Not part of the method: the MoBiQuant pages have no counterpart of this

@@ -92,6 +92,26 @@ def test_gemm_validation(L):
     assert call(T=0) == 0                 # nothing to do
 
 
+def test_linear_validation(L):
+    p = ctypes.c_void_p
+
+    def call(T=16, K=256, N=64, S=3, G=128, ws=p(FAKE), wsb=1 << 30, X=p(FAKE), Y=p(FAKE), codes=p(FAKE)):
+        return L.mobi_linear(X, T, K, p(FAKE), None, codes, p(FAKE), N, G, S, p(FAKE), p(FAKE), p(FAKE), Y, ws,
+                             wsb, None)
+    assert call(K=200) == 2
+    assert call(N=24) == 2
+    assert call(G=64) == 2
+    assert call(S=4) == 1
+    assert call(X=None) == 1
+    assert call(codes=None) == 1
+    assert call(Y=p(FAKE + 4)) == 3
+    assert call(wsb=16) == 4
+    T, N, K = 16, 4096, 4096
+    assert mobi.mobi_linear_workspace_bytes(T, N, K, 3) >= mobi.mobi_gemm_workspace_bytes(T, N, K, 3)
+    assert mobi.mobi_linear_workspace_bytes(64, N, K, 3) >= (mobi.mobi_route_workspace_bytes(64, K, 3)
+                                                             + mobi.mobi_gemm_workspace_bytes(64, N, K, 3))
+
+
 def test_workspace_sizes_edge_cases(L):
     assert mobi.mobi_route_workspace_bytes(0, 256, 3) == 0
     assert mobi.mobi_route_workspace_bytes(2048, 4096, 3) == 0   # many token tiles: no split

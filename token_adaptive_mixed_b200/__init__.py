@@ -11,6 +11,7 @@ Entry points (same names as the C ABI):
   mobi_route(X, Wr, bias)           MoBiRoute routing   -> (k_t, perm, offsets)
   mobi_gemm(X, k_t, perm, offsets, codes, sz, N)         -> Y  (fp32)
   mobi_gemm_path(..., path)         the same with a forced kernel
+  mobi_linear(X, Wr, bias, codes, sz, N)  route + GEMM in one call -> (Y, k_t, perm, offsets)
   mobi_sync_check()                 sync + device-side error word
 """
 from __future__ import annotations
@@ -23,7 +24,8 @@ import torch
 __all__ = [
     "MobiError", "lib", "mobi_version", "mobi_status_string", "mobi_codes_bytes", "mobi_sz_bytes",
     "mobi_route_workspace_bytes", "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm", "mobi_last_error",
-    "mobi_gemm_path", "mobi_sync_check", "mobi_debug_set_wait_limit", "mobi_gemm_decode_noalloc", "PATH_AUTO",
+    "mobi_gemm_path", "mobi_sync_check", "mobi_debug_set_wait_limit", "mobi_gemm_decode_noalloc", "mobi_linear",
+    "mobi_linear_workspace_bytes", "PATH_AUTO",
     "PATH_DECODE",
     "PATH_PREFILL", "EXPORTED_SYMBOLS",
 ]
@@ -39,7 +41,7 @@ STATUS_NAMES = ["MOBI_OK", "MOBI_ERR_INVALID_ARG", "MOBI_ERR_UNSUPPORTED_SHAPE",
 EXPORTED_SYMBOLS = (
     "mobi_status_string", "mobi_last_error", "mobi_version", "mobi_codes_bytes", "mobi_sz_bytes", "mobi_route_workspace_bytes",
     "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm", "mobi_gemm_path", "mobi_sync_check",
-    "mobi_debug_set_wait_limit", "mobi_gemm_decode_noalloc",
+    "mobi_debug_set_wait_limit", "mobi_gemm_decode_noalloc", "mobi_linear", "mobi_linear_workspace_bytes",
 )
 
 
@@ -86,6 +88,10 @@ def lib() -> ctypes.CDLL:
         L.mobi_gemm_path.restype = ci
         L.mobi_gemm_decode_noalloc.argtypes = [p, i64, i64, p, p, p, i64, ci, ci, p, p]
         L.mobi_gemm_decode_noalloc.restype = ci
+        L.mobi_linear_workspace_bytes.argtypes = [i64, i64, i64, ci]
+        L.mobi_linear_workspace_bytes.restype = sz_t
+        L.mobi_linear.argtypes = [p, i64, i64, p, p, p, p, i64, ci, ci, p, p, p, p, p, sz_t, p]
+        L.mobi_linear.restype = ci
         L.mobi_sync_check.argtypes = [p]
         L.mobi_sync_check.restype = ci
         L.mobi_debug_set_wait_limit.argtypes = [i64]
@@ -209,6 +215,28 @@ def mobi_gemm_decode_noalloc(X, k_t, codes, sz, N, S=None, G=128, Y=None, stream
     _check("mobi_gemm_decode_noalloc", lib().mobi_gemm_decode_noalloc(_ptr(X), T, K, _ptr(k_t), _ptr(codes),
                                                                       _ptr(sz), N, G, S, _ptr(Y), _stream(stream)))
     return Y
+
+
+def mobi_linear_workspace_bytes(T: int, N: int, K: int, S: int = 3) -> int:
+    return lib().mobi_linear_workspace_bytes(T, N, K, S)
+
+
+def mobi_linear(X, Wr, bias, codes, sz, N, G=128, Y=None, k_t=None, perm=None, offsets=None, ws=None, stream=None):
+    """Route + mixed-bit GEMM in one call (S = Wr.shape[1]) -> (Y fp32 [T,N], k_t, perm, offsets)."""
+    if X.dtype != torch.bfloat16 or Wr.dtype != torch.float32:
+        raise ValueError("X must be bf16 and Wr fp32")
+    T, K = X.shape
+    S = Wr.shape[1]
+    dev = X.device
+    Y = torch.empty((T, N), dtype=torch.float32, device=dev) if Y is None else Y
+    k_t = torch.empty(T, dtype=torch.int32, device=dev) if k_t is None else k_t
+    perm = torch.empty(T, dtype=torch.int32, device=dev) if perm is None else perm
+    offsets = torch.empty(S + 1, dtype=torch.int32, device=dev) if offsets is None else offsets
+    ws = _workspace(mobi_linear_workspace_bytes(T, N, K, S), dev, ws)
+    _check("mobi_linear", lib().mobi_linear(_ptr(X), T, K, _ptr(Wr), _ptr(bias), _ptr(codes), _ptr(sz), N, G, S,
+                                            _ptr(k_t), _ptr(perm), _ptr(offsets), _ptr(Y), _ptr(ws), ws.numel(),
+                                            _stream(stream)))
+    return Y, k_t, perm, offsets
 
 
 def mobi_sync_check(stream=None) -> None:

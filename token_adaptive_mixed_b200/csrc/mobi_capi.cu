@@ -24,7 +24,7 @@ cudaError_t launch_route(const void* X, int64_t T, int64_t K, const float* Wr, c
 size_t route_ws_bytes(int64_t T, int64_t K, int S);
 cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
                           const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
-                          DeviceStatus* st);
+                          DeviceStatus* st, bool early);
 size_t decode_ws_bytes(int64_t N, int64_t K);
 cudaError_t launch_prefill(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
                            const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int S,
@@ -257,8 +257,46 @@ mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const int32_t* k
   DeviceStatus* dst = device_status(&e);
   if (!dst) return cuda_status(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (decode) return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, ws, s, dst));
+  if (decode) return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, ws, s, dst, false));
   return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, ws, s, dst));
+}
+
+size_t mobi_linear_workspace_bytes(int64_t T, int64_t N, int64_t K, int S) {
+  if (T < 0 || N < 0 || K < 0 || S < 1 || S > 3) return 0;
+  return align256(route_ws_bytes(T, K, S)) + mobi_gemm_workspace_bytes(T, N, K, S);
+}
+
+mobi_status mobi_linear(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
+                        const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S, int32_t* k_t,
+                        int32_t* perm, int32_t* offsets, float* Y, void* ws, size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  mobi_status st = check_matrix(N, K, G, S);
+  if (st != MOBI_OK) return st;
+  if (T < 0) return MOBI_ERR_INVALID_ARG;
+  if (T > kMaxDim) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  if (!offsets || (T > 0 && (!X || !Wr || !k_t || !perm))) return MOBI_ERR_INVALID_ARG;
+  if (T > 0 && K == 0) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  if (T > 0 && N > 0 && (!codes || !sz || !Y || !ws)) return MOBI_ERR_INVALID_ARG;
+  if ((X && !aligned16(X)) || (Wr && !aligned16(Wr)) || (bias && !aligned4(bias)) || (k_t && !aligned4(k_t)) ||
+      (perm && !aligned4(perm)) || !aligned4(offsets) || (codes && !aligned16(codes)) || (sz && !aligned16(sz)) ||
+      (Y && !aligned16(Y)) || (ws && !aligned16(ws)))
+    return MOBI_ERR_MISALIGNED;
+  const size_t route_ws = align256(route_ws_bytes(T, K, S));
+  const bool decode = T <= 16;
+  const size_t need = route_ws + (T > 0 && N > 0 ? (decode ? decode_ws_bytes(N, K) : prefill_ws_bytes(T, N, K)) : 0);
+  if (need > 0 && (!ws || ws_bytes < need)) return MOBI_ERR_WORKSPACE;
+  cudaError_t e;
+  DeviceStatus* dst = device_status(&e);
+  if (!dst) return cuda_status(e);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  e = launch_route(X, T, K, Wr, bias, S, k_t, perm, offsets, ws, s);
+  if (e != cudaSuccess || T == 0 || N == 0) return cuda_status(e);
+  void* gws = static_cast<uint8_t*>(ws) + route_ws;
+  // For up to 16 tokens the kernel just launched is the routing kernel, which
+  // writes only k_t, perm and offsets: the decode kernel may fetch X and the
+  // weights before it waits on it.
+  if (decode) return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, gws, s, dst, true));
+  return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, gws, s, dst));
 }
 
 mobi_status mobi_gemm(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,

@@ -45,16 +45,20 @@ constexpr int kDecGW = 2;                    // groups per warp (64 bytes of a c
 constexpr int kDecQ = 4;                     // warps per team (one team per 32-row block)
 constexpr int kDecChunk = kDecQ * kDecGW;    // groups per CTA chunk
 constexpr int kDecRows = 32;                 // rows per stage: two 16-row MMA tiles
-constexpr uint32_t kDecRowBytes = kDecGW * 32;               // code bytes of one row in a stage
-constexpr uint32_t kDecSlotCodes = kDecRows * kDecRowBytes;  // one stage: 32 rows x 64 bytes of codes
-constexpr uint32_t kDecSlotSz = kDecGW * kDecRows * 4;       // and [2 groups][32 rows] scale/zero words
+// A stage belongs to a team: 32 rows x the chunk's 8 groups, as two
+// 128-byte-swizzled halves of 32 rows x 128 bytes, then [8 groups][32 rows]
+// scale/zero words.
+constexpr uint32_t kDecHalfBytes = kDecRows * 128;
+constexpr uint32_t kDecSlotCodes = 2 * kDecHalfBytes;
+constexpr uint32_t kDecSlotSz = kDecChunk * kDecRows * 4;
+constexpr uint32_t kDecSlot = kDecSlotCodes + kDecSlotSz;  // 9 KB, a multiple of 1 KB
 
 template <int NB>
 struct DecCfg;
 template <>
 struct DecCfg<1> {  // T <= 8: 16 B-fragment registers per group
-  static constexpr int kTeams = 4;
-  static constexpr int kDepth = 4;
+  static constexpr int kTeams = 3;
+  static constexpr int kDepth = 6;
 };
 template <>
 struct DecCfg<2> {  // T <= 16: 32 per group
@@ -72,11 +76,11 @@ struct DecLayout {
                                       ? 248
                                       : (16384 / (32 * ((kWarps + 4) / 4))) / 8 * 8;
   static constexpr int kDepth = DecCfg<NB>::kDepth;
-  static constexpr uint32_t kCodes = 0;                                      // [warp][slot] 2 KB, 1 KB aligned
-  static constexpr uint32_t kSz = kCodes + kWarps * kDepth * kDecSlotCodes;  // [warp][slot][2][32]
-  static constexpr uint32_t kXchg = kSz + kWarps * kDepth * kDecSlotSz;      // [team][2][kDecQ-1][32][8 NB] floats
+  static constexpr int kTeams = DecCfg<NB>::kTeams;
+  static constexpr uint32_t kSlots = 0;                                      // [team][slot] 9 KB, 1 KB aligned
+  static constexpr uint32_t kXchg = kSlots + kTeams * kDepth * kDecSlot;     // [team][2][kDecQ-1][32][8 NB] floats
   static constexpr uint32_t kBar = kXchg + DecCfg<NB>::kTeams * 2 * (kDecQ - 1) * 32 * 8 * NB * 4;  // full, empty
-  static constexpr uint32_t kReady = kBar + 2 * kWarps * kDepth * 8;  // consumers' fragments built
+  static constexpr uint32_t kReady = kBar + 2 * kTeams * kDepth * 8;  // consumers' fragments built
   static constexpr uint32_t kAbort = kReady + 8;
   static constexpr uint32_t kBytes = kAbort + 8;
   static constexpr size_t kDynamic = kBytes + 1024;  // + manual 1 KB alignment
@@ -108,16 +112,18 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// Issue one stage of a warp into ring slot `slot`: the warp's 64-byte slice
-// of 32 code rows (x = word column, y = s*N + row; 64-byte swizzle) and the
-// matching [2 groups][32 rows] scale/zero words.
-// Weights are read once per call, so they go in with L2 evict-first.
-__device__ __forceinline__ void dec_issue(const CUtensorMap* tm_codes, const CUtensorMap* tm_sz, uint8_t* codes_slot,
-                                          uint32_t* sz_slot, uint64_t* bar, int block, int s, int N, int ngroups,
-                                          int gbase, uint64_t policy) {
-  mbar_arrive_expect_tx(bar, kDecSlotCodes + kDecSlotSz);
-  tma_load_2d_hint(codes_slot, tm_codes, gbase * 8, s * N + block * kDecRows, bar, policy);
-  tma_load_2d_hint(sz_slot, tm_sz, block * kDecRows, s * ngroups + gbase, bar, policy);
+// Issue one team stage into `slot`: the chunk's 256 bytes of 32 code rows as
+// two 128-byte halves (x = word column, y = s*N + row) and the matching
+// [8 groups][32 rows] scale/zero words. Weights are read once per call, so
+// they go in with L2 evict-first.
+__device__ __forceinline__ void dec_issue(const CUtensorMap* tm_codes, const CUtensorMap* tm_sz, uint8_t* slot,
+                                          uint64_t* bar, int block, int s, int N, int ngroups, int chunk,
+                                          uint64_t policy) {
+  mbar_arrive_expect_tx(bar, kDecSlot);
+  const int y = s * N + block * kDecRows;
+  tma_load_2d_hint(slot, tm_codes, chunk * kDecChunk * 8, y, bar, policy);
+  tma_load_2d_hint(slot + kDecHalfBytes, tm_codes, chunk * kDecChunk * 8 + 32, y, bar, policy);
+  tma_load_2d_hint(slot + kDecSlotCodes, tm_sz, block * kDecRows, s * ngroups + chunk * kDecChunk, bar, policy);
 }
 
 // Groups g0, g0 + 1 of one stage for TT tiles: four MMA chains in flight.
@@ -132,8 +138,8 @@ __device__ __forceinline__ void dec_group_pair(int g0, const uint8_t* cs, const 
   for (int gg = 0; gg < 2; ++gg)
 #pragma unroll
     for (int tt = 0; tt < TT; ++tt) {
-      wa[gg][tt] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + tt * 16 * kDecRowBytes);
-      wb[gg][tt] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + tt * 16 * kDecRowBytes + 8 * kDecRowBytes);
+      wa[gg][tt] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + tt * 16 * 128);
+      wb[gg][tt] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + tt * 16 * 128 + 8 * 128);
     }
   float d[2][TT][NB][4];
 #pragma unroll
@@ -218,7 +224,7 @@ template <int NB>
 __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLayout<NB>::kMaxRegs) decode_kernel(
     const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_sz,
     const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ k_t, int T, int N, int K, int ngroups, int S,
-    int nblocks, float* __restrict__ out, DeviceStatus* st, uint64_t limit) {
+    int nblocks, float* __restrict__ out, DeviceStatus* st, uint64_t limit, int early) {
   using L = DecLayout<NB>;
   constexpr int kTeams = DecCfg<NB>::kTeams;
   constexpr int kW = L::kWarps;
@@ -236,38 +242,53 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLay
   // of them, starting with block b_begin + t.
   const int b_begin = (int)((int64_t)blockIdx.x * nblocks / gridDim.x);
   const int b_end = (int)((int64_t)(blockIdx.x + 1) * nblocks / gridDim.x);
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::kBar);  // [warp][slot]
-  uint64_t* empty = full + kW * D;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::kBar);  // [team][slot]
+  uint64_t* empty = full + kTeams * D;
   uint64_t* ready = reinterpret_cast<uint64_t*>(sm + L::kReady);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(sm + L::kAbort);
 
-  // One barrier per thread (about 130 in all), then one fence per warp.
-  for (int i = threadIdx.x; i < 2 * kW * D + 1; i += blockDim.x) {
-    if (i < kW * D) mbar_init(&full[i], 1);
-    else if (i < 2 * kW * D) mbar_init(&empty[i - kW * D], 1);
+  // One barrier per thread, then one fence per warp. A stage is freed by the
+  // four warps of its team.
+  for (int i = threadIdx.x; i < 2 * kTeams * D + 1; i += blockDim.x) {
+    if (i < kTeams * D) mbar_init(&full[i], 1);
+    else if (i < 2 * kTeams * D) mbar_init(&empty[i - kTeams * D], kDecQ);
     else mbar_init(ready, kW);
   }
   if (threadIdx.x == 0) *abort_flag = 0;
   if (lane == 0) fence_barrier_init();
   __syncthreads();
+  // Launched as a programmatic dependent of the previous kernel in the
+  // stream. By default nothing in global memory is read before this wait.
+  // With `early` set the caller guarantees that the previous kernel writes
+  // none of X, codes and sz (it is this library's routing kernel), so the
+  // activations and the first weight stages are fetched before the wait and
+  // only k_t is read after it.
+  if (!early) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == kW) {
-    // ---------------- producer: lane w feeds consumer warp w's ring ----------------
+    // ---------------- producer: lane w feeds team w's ring ----------------
     // All lanes poll their ring's empty barrier in one non-blocking test and
-    // issue their copies together, so one poll serves every consumer warp.
+    // issue their copies together, so one poll serves every team.
     named_bar_sync(15, 32 * (kW + 1));  // the consumers' activation loads go out first
     if (lane == 0) {
       prefetch_tmap(&tm_codes);
       prefetch_tmap(&tm_sz);
     }
     const uint64_t policy = l2_evict_first_policy();
+    const int w = lane, team = lane;
+    const int myb = (w < kTeams && b_end - b_begin > team) ? (b_end - b_begin - team + kTeams - 1) / kTeams : 0;
+    int r = 0, bo = 0, s = 0;  // next stage of team w: its index, block offset and slice
+    // Slice 0 of the team's first block does not depend on k_t.
+    if (early && myb > 0) {
+      dec_issue(&tm_codes, &tm_sz, sm + L::kSlots + (uint32_t)(w * D) * kDecSlot, &full[w * D], b_begin + team, 0, N,
+                ngroups, ch, policy);
+      r = 1;
+    }
+    if (early) asm volatile("griddepcontrol.wait;" ::: "memory");
     int kmax = __reduce_max_sync(0xffffffffu, lane < T ? (int)__ldg(k_t + lane) : 1);
     kmax = kmax < 1 ? 1 : (kmax > S ? S : kmax);
-    const int w = lane;
-    const int team = w / kDecQ, gb = ch * kDecChunk + (w % kDecQ) * kDecGW;
-    const int myb = (w < kW && b_end - b_begin > team) ? (b_end - b_begin - team + kTeams - 1) / kTeams : 0;
-    const int nit = (w < kW && gb < ngroups) ? myb * kmax : 0;  // items of warp w: blocks x slices
-    int r = 0, bo = 0, s = 0;  // next item of warp w: its index, block offset and slice
+    const int nit = myb * kmax;  // stages of team w: its blocks x slices
+    if (r == 1 && ++s == kmax) { s = 0; ++bo; }
     bool gate = false;         // every consumer has built its activations
     bool ok = true;
     uint64_t idle = 0;         // polls in a row without a copy issued
@@ -279,9 +300,8 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLay
       if (ok && r < nit && (r < 2 || gate)) {
         const int slot = r % D;
         if (r < D || mbar_test_wait(&empty[w * D + slot], (uint32_t)(((r / D) & 1) ^ 1))) {
-          dec_issue(&tm_codes, &tm_sz, sm + L::kCodes + (uint32_t)(w * D + slot) * kDecSlotCodes,
-                    reinterpret_cast<uint32_t*>(sm + L::kSz + (uint32_t)(w * D + slot) * kDecSlotSz),
-                    &full[w * D + slot], b_begin + team + bo * kTeams, s, N, ngroups, gb, policy);
+          dec_issue(&tm_codes, &tm_sz, sm + L::kSlots + (uint32_t)(w * D + slot) * kDecSlot, &full[w * D + slot],
+                    b_begin + team + bo * kTeams, s, N, ngroups, ch, policy);
           ++r;
           if (++s == kmax) { s = 0; ++bo; }
           issued = true;
@@ -318,11 +338,10 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLay
   const int gbase = ch * kDecChunk + q * kDecGW;  // first group of this warp
   const int ngv = ngroups - gbase < 0 ? 0 : (ngroups - gbase > kDecGW ? kDecGW : ngroups - gbase);
   const int my_blocks = b_end - b_begin > team ? (b_end - b_begin - team + kTeams - 1) / kTeams : 0;
-  const uint8_t* codes_w = sm + L::kCodes + (uint32_t)warp * D * kDecSlotCodes;
-  const uint32_t* sz_w = reinterpret_cast<const uint32_t*>(sm + L::kSz + (uint32_t)warp * D * kDecSlotSz);
+  const uint8_t* slots_t = sm + L::kSlots + (uint32_t)team * D * kDecSlot;  // the team's ring
   float* xchg = reinterpret_cast<float*>(sm + L::kXchg) + team * 2 * (kDecQ - 1) * 32 * 8 * NB;
-  uint64_t* full_w = full + warp * D;
-  uint64_t* empty_w = empty + warp * D;
+  uint64_t* full_w = full + team * D;
+  uint64_t* empty_w = empty + team * D;
 
   // This lane's activations (token gid + 8 nb, columns 32 t4 .. +31 of each
   // group) and k_t[lane].
@@ -341,10 +360,7 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLay
         for (int v = 0; v < 4; ++v) raw[g][nb][v] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
-  const int my_kt = lane < T ? k_t[lane] : 0;
   asm volatile("bar.arrive 15, %0;" ::"r"(32 * (kW + 1)) : "memory");
-  int kmax = __reduce_max_sync(0xffffffffu, my_kt);
-  kmax = kmax < 1 ? 1 : (kmax > S ? S : kmax);
 
   // Activation fragments of the warp's groups, in registers for the whole
   // kernel. B[g][j][2 nb + ih] is the B fragment of k16 step j = 4h + f for
@@ -401,6 +417,10 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLay
     if (__any_sync(0xffffffffu, bad) && lane == 0) report_error(st, kErrInputRange, 0x100);
   }
   if (lane == 0) mbar_arrive(ready);
+  if (early) asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int my_kt = lane < T ? k_t[lane] : 0;
+  int kmax = __reduce_max_sync(0xffffffffu, my_kt);
+  kmax = kmax < 1 ? 1 : (kmax > S ? S : kmax);
 
   // k_t of the two tokens whose D columns this lane holds.
   int ktl[NB][2];
@@ -410,14 +430,15 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLay
     ktl[nb][1] = __shfl_sync(0xffffffffu, my_kt, 2 * t4 + 1 + 8 * nb);
   }
 
-  // Code words 2 t4, 2 t4 + 1 of group g of row gid in the 64-byte-swizzled
-  // stage (16-byte chunk c of row r sits at c ^ ((r >> 1) & 3)); rows gid + 8,
-  // +16, +24 share the swizzle and sit 512 bytes apart.
+  // Code words 2 t4, 2 t4 + 1 of the warp's group g (chunk group 2q + g) of
+  // row gid: in half q / 2 of the stage, 128-byte-swizzled (16-byte chunk c of
+  // row r sits at c ^ (r & 7)); rows gid + 8, +16, +24 share the swizzle and
+  // sit 1, 2, 3 KB further on.
   uint32_t coff[kDecGW];
 #pragma unroll
   for (int g = 0; g < kDecGW; ++g)
-    coff[g] = (uint32_t)gid * kDecRowBytes + (uint32_t)(((2 * g + (t4 >> 1)) ^ ((gid >> 1) & 3)) * 16) +
-              (t4 & 1) * 8u;
+    coff[g] = (uint32_t)(q >> 1) * kDecHalfBytes + (uint32_t)gid * 128u +
+              (uint32_t)(((((q & 1) * kDecGW + g) * 2 + (t4 >> 1)) ^ gid) * 16) + (t4 & 1) * 8u;
 
   // y[tt][nb]: tile tt of the block, rows gid (A) and gid + 8 (B) of it,
   // tokens (2 t4, 2 t4 + 1) + 8 nb.
@@ -434,13 +455,13 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLay
   const int total_iters = my_blocks * kmax;  // both warps of a team walk the same sequence
   for (int it = 0; it < total_iters; ++it) {
     const bool two = blk * kDecRows + 16 < N;  // the block's second tile exists (N % 16 == 0)
-    if (ok && ngv > 0) {
+    if (ok) {  // every warp of the team frees each stage, also one past the last group
       const bool got = __all_sync(0xffffffffu, dec_wait(&full_w[slot], parity, limit, st, 0x200 + s, abort_flag));
       if (!got) {
         ok = false;
       } else {
-        const uint8_t* cs = codes_w + (uint32_t)slot * kDecSlotCodes;
-        const uint32_t* ss = sz_w + (uint32_t)slot * (kDecSlotSz / 4);
+        const uint8_t* cs = slots_t + (uint32_t)slot * kDecSlot;
+        const uint32_t* ss = reinterpret_cast<const uint32_t*>(cs + kDecSlotCodes) + q * kDecGW * kDecRows;
         float2 m37[NB], m1[NB];
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
@@ -511,14 +532,24 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLay
 }
 
 // Y[t][n] = sum over chunks c (in order) of partial[c][t][n]; n4 = T*N/4.
+// Up to 8 chunk loads are in flight at a time; the adds keep chunk order.
 __global__ void __launch_bounds__(256) decode_reduce_kernel(const float4* __restrict__ partial, int64_t n4, int nch,
                                                             float4* __restrict__ Y) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
-    float4 a = partial[i];
-    for (int c = 1; c < nch; ++c) {
-      const float4 b = partial[(int64_t)c * n4 + i];
-      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+    float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int c0 = 0; c0 < nch; c0 += 8) {
+      float4 b[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if (c0 + c < nch) b[c] = __ldcg(partial + (int64_t)(c0 + c) * n4 + i);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if (c0 + c < nch) {
+          if (c0 + c == 0) a = b[c];
+          else { a.x += b[c].x; a.y += b[c].y; a.z += b[c].z; a.w += b[c].w; }
+        }
     }
     Y[i] = a;
   }
@@ -547,19 +578,30 @@ void decode_grid(int64_t N, int64_t K, int sms, int64_t* cpc, int64_t* nch) {
 template <int NB>
 static cudaError_t launch_decode_nb(const CUtensorMap& tm_codes, const CUtensorMap& tm_sz, const void* X, int T,
                                     int64_t K, const int32_t* k_t, int64_t N, int S, float* out, int64_t cpc,
-                                    int64_t nch, cudaStream_t stream, DeviceStatus* st) {
+                                    int64_t nch, cudaStream_t stream, DeviceStatus* st, bool early) {
   using L = DecLayout<NB>;
   cudaError_t e = set_smem((const void*)decode_kernel<NB>, (int)L::kDynamic);
   if (e != cudaSuccess) return e;
-  decode_kernel<NB><<<dim3((unsigned)cpc, (unsigned)nch), L::kThreads, L::kDynamic, stream>>>(
-      tm_codes, tm_sz, static_cast<const __nv_bfloat16*>(X), k_t, T, (int)N, (int)K, (int)(K / 128), S,
-      (int)((N + kDecRows - 1) / kDecRows), out, st, wait_limit());
-  return note_error("decode launch", cudaGetLastError());
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)cpc, (unsigned)nch);
+  cfg.blockDim = dim3(L::kThreads);
+  cfg.dynamicSmemBytes = L::kDynamic;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // set-up overlaps the previous kernel
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<NB>, tm_codes, tm_sz, static_cast<const __nv_bfloat16*>(X), k_t, T,
+                         (int)N, (int)K, (int)(K / 128), S, (int)((N + kDecRows - 1) / kDecRows), out, st,
+                         wait_limit(), early ? 1 : 0);
+  if (e != cudaSuccess) return note_error("decode launch", e);
+  return note_error("kernel launch", cudaGetLastError());
 }
 
 cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
                           const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
-                          DeviceStatus* st) {
+                          DeviceStatus* st, bool early) {
   const int64_t ngroups = K / 128;
   int64_t cpc, nch;
   decode_grid(N, K, num_sms(), &cpc, &nch);
@@ -567,14 +609,14 @@ cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, c
   float* out = nch > 1 ? partial : Y;
 
   CUtensorMap tm_codes, tm_sz;
-  if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4,
-                    kDecGW * 8, kDecRows, 64))
+  if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4, 32,
+                    kDecRows, 128))
     return note_error("decode tensor map (codes)", cudaErrorInvalidValue);
-  if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, kDecRows, kDecGW, 0))
+  if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, kDecRows, kDecChunk, 0))
     return note_error("decode tensor map (scale/zero)", cudaErrorInvalidValue);
 
-  cudaError_t e = T > 8 ? launch_decode_nb<2>(tm_codes, tm_sz, X, T, K, k_t, N, S, out, cpc, nch, stream, st)
-                        : launch_decode_nb<1>(tm_codes, tm_sz, X, T, K, k_t, N, S, out, cpc, nch, stream, st);
+  cudaError_t e = T > 8 ? launch_decode_nb<2>(tm_codes, tm_sz, X, T, K, k_t, N, S, out, cpc, nch, stream, st, early)
+                        : launch_decode_nb<1>(tm_codes, tm_sz, X, T, K, k_t, N, S, out, cpc, nch, stream, st, early);
   if (e != cudaSuccess || nch <= 1) return e;
 
   // Chunk reduction, launched as a programmatic dependent of the decode kernel.
@@ -665,7 +707,7 @@ extern "C" mobi_status mobi_gemm_decode_noalloc(const void* X, int64_t T, int64_
   if (!st) return MOBI_ERR_CUDA;
   void* scratch = noalloc_scratch(&e);
   if (!scratch) return MOBI_ERR_CUDA;
-  e = launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, scratch, static_cast<cudaStream_t>(stream), st);
+  e = launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, scratch, static_cast<cudaStream_t>(stream), st, false);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     return MOBI_ERR_CUDA;

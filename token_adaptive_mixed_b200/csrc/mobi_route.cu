@@ -201,11 +201,13 @@ __global__ void __launch_bounds__(kBucketThreads) bucket_kernel(int64_t T, int k
 //
 // CTA r of the cluster sums the logits of every token over its share of the
 // 8-column octets of K (fp32 within a thread, fp32 xor tree within a warp,
-// fp64 across warps), keeps them in its shared memory, and after a cluster
-// barrier CTA 0 adds the eight partials in rank order through distributed
-// shared memory (fp64), takes the argmax and writes the stable bucketing
-// (warp ballots over the at most 16 tokens). A second cluster barrier keeps
-// the other CTAs alive until CTA 0 has read their partials.
+// fp64 across warps) and stores them into CTA 0's shared memory (distributed
+// shared memory); after one cluster barrier CTA 0 adds the eight partials in
+// rank order (fp64), takes the argmax and writes the stable bucketing (warp
+// ballots over the at most 16 tokens).
+// Launched as a programmatic dependent of whatever precedes it: it reads no
+// global memory before griddepcontrol.wait, and lets its own dependent (the
+// decode GEMM) start its set-up early.
 constexpr int kRouteSmallT = 16;
 constexpr int kRouteCluster = 8;
 
@@ -220,10 +222,8 @@ __device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
   return r;
 }
 
-__device__ __forceinline__ double ld_dsmem_f64(uint32_t addr) {
-  double v;
-  asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(addr) : "memory");
-  return v;
+__device__ __forceinline__ void st_dsmem_f64(uint32_t addr, double v) {
+  asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(addr), "d"(v) : "memory");
 }
 
 template <int S>
@@ -232,8 +232,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
     const float* __restrict__ bias, int32_t* __restrict__ k_t, int32_t* __restrict__ perm,
     int32_t* __restrict__ offsets) {
   __shared__ float red[kRouteThreads / 32][kRouteSmallT * S];
-  __shared__ double part[kRouteSmallT * S];
+  __shared__ double part[kRouteCluster][kRouteSmallT * S];  // used in CTA 0: [rank][token * S + j]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
   uint32_t rank;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
   const int64_t noct = K / 8;
@@ -279,9 +281,9 @@ __global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
   if (tid < kRouteSmallT * S) {
     double s = 0.0;
     for (int w8 = 0; w8 < kRouteThreads / 32; ++w8) s += (double)red[w8][tid];
-    part[tid] = s;
+    st_dsmem_f64(dsmem_addr(&part[rank][tid], 0), s);
   }
-  cluster_sync_all();  // every CTA's partial logits are in its shared memory
+  cluster_sync_all();  // every CTA's partial logits are in CTA 0's shared memory
 
   if (rank == 0 && warp == 0) {
     // Lane t < T: the logits of token t, partials added in rank order.
@@ -291,7 +293,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
 #pragma unroll
       for (int j = 0; j < S; ++j) {
         double s = 0.0;
-        for (uint32_t r = 0; r < kRouteCluster; ++r) s += ld_dsmem_f64(dsmem_addr(&part[lane * S + j], r));
+        for (int r = 0; r < kRouteCluster; ++r) s += part[r][lane * S + j];
         l[j] = s + (bias ? (double)__ldg(bias + j) : 0.0);
       }
       k = 1 + argmax_lowest(l, S);
@@ -308,7 +310,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
     }
     if (lane == 0) offsets[S] = run;
   }
-  cluster_sync_all();  // CTA 0 is done reading the others' shared memory
 }
 
 template <int S>
@@ -319,13 +320,15 @@ static cudaError_t launch_route_small(const void* X, int64_t T, int64_t K, const
   cfg.blockDim = dim3(kRouteThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = kRouteCluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the launch with the previous kernel
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, route_small_kernel<S>, static_cast<const __nv_bfloat16*>(X), (int)T, K,
                                            Wr, bias, k_t, perm, offsets);
   if (e != cudaSuccess) return note_error("route launch", e);
