@@ -52,6 +52,15 @@ def decode_bytes(N, K, T, kmax):
     return kmax * (N * K // 4 + N * (K // 128) * 4) + T * K * 2
 
 
+# DRAM bytes / algorithmic bytes of the decode kernel, from one ncu capture of
+# the 11008 x 4096, T=4, k_max=3 launch (dram__bytes_read.sum 38105600 +
+# dram__bytes_write.sum 256 against 38076416 algorithmic; see
+# profiles/decode_kernel_llama7b_decode.md). Traffic grows in proportion to
+# the bytes streamed, so the step's traffic is the step's algorithmic bytes
+# times this ratio. Valid for the decode kernel as captured.
+DECODE_DRAM_RATIO = (38105600 + 256) / 38076416
+
+
 class ClockSampler:
     """NVML samples of SM clock and throttle reasons while the timed region runs."""
 
@@ -379,7 +388,9 @@ def run_gpu(args, world, rank):
         "roofline": {"bound": "hbm", "kernel": "decode GEMM (staging + mma.sync decode kernels)",
                      "achieved": round(achieved, 2), "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "frac_of_8TBs_nominal": round(achieved / 8000.0, 4),
-                     "traffic": None, "per_call_us": [round(1e3 * x, 2) for x in per_case_ms]},
+                     "traffic": round(bytes_step * DECODE_DRAM_RATIO),
+                     "traffic_unit": "bytes per step (ncu DRAM bytes / algorithmic bytes x algorithmic bytes)",
+                     "per_call_us": [round(1e3 * x, 2) for x in per_case_ms]},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": launches_per_step * args.steps,
