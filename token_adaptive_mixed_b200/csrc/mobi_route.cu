@@ -34,6 +34,21 @@ __device__ __forceinline__ int argmax_lowest(const double* l, int S) {
   return best;
 }
 
+// The same with a compile-time S, so that l stays in registers.
+template <int S>
+__device__ __forceinline__ int argmax_lowest_t(const double (&l)[S]) {
+  int best = 0;
+  double m = l[0];
+#pragma unroll
+  for (int j = 1; j < S; ++j)
+    if (l[j] > m) { m = l[j]; best = j; }
+  return best;
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem)), "l"(gmem) : "memory");
+}
+
 // partial[ks][t][j] (fp64) when ksplit > 1, otherwise k_t directly.
 template <int S>
 __global__ void __launch_bounds__(kRouteThreads) route_partial_kernel(
@@ -204,12 +219,21 @@ __global__ void __launch_bounds__(kBucketThreads) bucket_kernel(int64_t T, int k
 // fp64 across warps) and stores them into CTA 0's shared memory (distributed
 // shared memory); after one cluster barrier CTA 0 adds the eight partials in
 // rank order (fp64), takes the argmax and writes the stable bucketing (warp
-// ballots over the at most 16 tokens).
+// ballots over the at most 16 tokens). The CTA's slices of X and Wr are first
+// staged into shared memory with cp.async (no registers held per load, so
+// every load of a pass is in flight at once), in passes of 256 octets.
 // Launched as a programmatic dependent of whatever precedes it: it reads no
 // global memory before griddepcontrol.wait, and lets its own dependent (the
 // decode GEMM) start its set-up early.
 constexpr int kRouteSmallT = 16;
 constexpr int kRouteCluster = 8;
+constexpr int kRoutePassOct = kRouteThreads;  // octets staged per pass: one per thread
+
+// Dynamic shared memory of route_small_kernel<S>: X [16 tokens][pass] 16-byte
+// octets, then Wr [pass][8 S] floats.
+__host__ __device__ constexpr size_t route_small_smem(int S) {
+  return (size_t)kRouteSmallT * kRoutePassOct * 16 + (size_t)kRoutePassOct * 8 * S * 4;
+}
 
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -241,32 +265,46 @@ __global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
   const int64_t noct = K / 8;
   const int64_t o_beg = rank * noct / kRouteCluster, o_end = (rank + 1) * noct / kRouteCluster;
 
+  extern __shared__ __align__(16) uint8_t rsm[];
+  uint4* xs = reinterpret_cast<uint4*>(rsm);                                   // [token][octet]
+  float* wsm = reinterpret_cast<float*>(rsm + kRouteSmallT * kRoutePassOct * 16);  // [octet][8 S]
   float acc[kRouteSmallT][S];
 #pragma unroll
   for (int i = 0; i < kRouteSmallT; ++i)
 #pragma unroll
     for (int j = 0; j < S; ++j) acc[i][j] = 0.0f;
-  for (int64_t o = o_beg + tid; o < o_end; o += kRouteThreads) {
-    const int64_t k = 8 * o;
-    float w[8][S];
+  for (int64_t p0 = o_beg; p0 < o_end; p0 += kRoutePassOct) {
+    const int np = (int)(o_end - p0 < kRoutePassOct ? o_end - p0 : kRoutePassOct);
+    for (int i = 0; i < T; ++i)
+      for (int o = tid; o < np; o += kRouteThreads)
+        cp_async16(&xs[i * kRoutePassOct + o], X + (int64_t)i * K + 8 * (p0 + o));
+    for (int e = tid; e < np * 2 * S; e += kRouteThreads)  // 8 S floats = 2 S pieces of 16 bytes per octet
+      cp_async16(&wsm[4 * e], Wr + p0 * 8 * S + 4 * e);
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    if (tid < np) {
+      const int o = tid;
+      float w[8][S];
 #pragma unroll
-    for (int e = 0; e < 8 * S; ++e) w[e / S][e % S] = __ldg(Wr + k * S + e);
+      for (int e = 0; e < 8 * S; ++e) w[e / S][e % S] = wsm[o * 8 * S + e];
 #pragma unroll
-    for (int i = 0; i < kRouteSmallT; ++i) {
-      if (i < T) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(X + (int64_t)i * K + k));
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+      for (int i = 0; i < kRouteSmallT; ++i) {
+        if (i < T) {
+          const uint4 v = xs[i * kRoutePassOct + o];
+          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const float x0 = bf16lo(u[p]), x1 = bf16hi(u[p]);
+          for (int p = 0; p < 4; ++p) {
+            const float x0 = bf16lo(u[p]), x1 = bf16hi(u[p]);
 #pragma unroll
-          for (int j = 0; j < S; ++j) {
-            acc[i][j] = fmaf(x0, w[2 * p][j], acc[i][j]);
-            acc[i][j] = fmaf(x1, w[2 * p + 1][j], acc[i][j]);
+            for (int j = 0; j < S; ++j) {
+              acc[i][j] = fmaf(x0, w[2 * p][j], acc[i][j]);
+              acc[i][j] = fmaf(x1, w[2 * p + 1][j], acc[i][j]);
+            }
           }
         }
       }
     }
+    __syncthreads();  // the next pass overwrites the staged slices
   }
 #pragma unroll
   for (int i = 0; i < kRouteSmallT; ++i)
@@ -296,7 +334,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
         for (int r = 0; r < kRouteCluster; ++r) s += part[r][lane * S + j];
         l[j] = s + (bias ? (double)__ldg(bias + j) : 0.0);
       }
-      k = 1 + argmax_lowest(l, S);
+      k = 1 + argmax_lowest_t<S>(l);
       k_t[lane] = k;
     }
     // Stable bucketing: tokens of value v keep their index order.
@@ -315,10 +353,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
 template <int S>
 static cudaError_t launch_route_small(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
                                       int32_t* k_t, int32_t* perm, int32_t* offsets, cudaStream_t stream) {
+  const size_t smem = route_small_smem(S);
+  cudaError_t e = set_smem((const void*)route_small_kernel<S>, (int)smem);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kRouteCluster);
   cfg.blockDim = dim3(kRouteThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -329,8 +370,8 @@ static cudaError_t launch_route_small(const void* X, int64_t T, int64_t K, const
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, route_small_kernel<S>, static_cast<const __nv_bfloat16*>(X), (int)T, K,
-                                           Wr, bias, k_t, perm, offsets);
+  e = cudaLaunchKernelEx(&cfg, route_small_kernel<S>, static_cast<const __nv_bfloat16*>(X), (int)T, K, Wr, bias, k_t,
+                         perm, offsets);
   if (e != cudaSuccess) return note_error("route launch", e);
   return note_error("kernel launch", cudaGetLastError());
 }
