@@ -93,9 +93,25 @@ int num_sms() {
   return g_sms[d];
 }
 
+// The attribute is set once per (kernel, device, size): later calls only look
+// it up, which keeps a driver call out of every launch.
 cudaError_t set_smem(const void* func, int bytes) {
-  return note_error("cudaFuncSetAttribute(max dynamic shared memory)",
-                    cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  struct Entry { const void* func; int device; int bytes; };
+  static Entry done[64];
+  static int ndone = 0;
+  const int d = current_device();
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (int i = 0; i < ndone; ++i)
+      if (done[i].func == func && done[i].device == d && done[i].bytes >= bytes) return cudaSuccess;
+  }
+  const cudaError_t e = note_error("cudaFuncSetAttribute(max dynamic shared memory)",
+                                   cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  if (e == cudaSuccess) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (ndone < 64) done[ndone++] = Entry{func, d, bytes};
+  }
+  return e;
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -112,8 +128,34 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// Encoded maps are a pure function of their arguments: a small cache keeps
+// the driver's encoder out of repeated calls on the same buffers.
+struct TmapKey {
+  const void* base;
+  uint64_t cols, rows, stride;
+  uint32_t box_cols, box_rows;
+  int elem_bytes, swizzle;
+  bool operator==(const TmapKey& o) const {
+    return base == o.base && cols == o.cols && rows == o.rows && stride == o.stride && box_cols == o.box_cols &&
+           box_rows == o.box_rows && elem_bytes == o.elem_bytes && swizzle == o.swizzle;
+  }
+};
+static constexpr int kTmapCache = 64;
+static TmapKey g_tmap_key[kTmapCache];
+static CUtensorMap g_tmap_val[kTmapCache];
+static int g_tmap_n = 0, g_tmap_next = 0;
+
 bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t cols, uint64_t rows,
                   uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes) {
+  const TmapKey key{base, cols, rows, row_stride_bytes, box_cols, box_rows, elem_bytes, swizzle_bytes};
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (int i = 0; i < g_tmap_n; ++i)
+      if (g_tmap_key[i] == key) {
+        *map = g_tmap_val[i];
+        return true;
+      }
+  }
   auto fn = encode_fn();
   if (!fn) return false;
   CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32;
@@ -132,6 +174,13 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t c
              "cuTensorMapEncodeTiled: CUresult %d (dims %llu x %llu, stride %llu, box %u x %u, swizzle %d)", (int)r,
              (unsigned long long)cols, (unsigned long long)rows, (unsigned long long)row_stride_bytes, box_cols,
              box_rows, swizzle_bytes);
+  if (r == CUDA_SUCCESS) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    g_tmap_key[g_tmap_next] = key;
+    g_tmap_val[g_tmap_next] = *map;
+    g_tmap_next = (g_tmap_next + 1) % kTmapCache;
+    if (g_tmap_n < kTmapCache) ++g_tmap_n;
+  }
   return r == CUDA_SUCCESS;
 }
 
