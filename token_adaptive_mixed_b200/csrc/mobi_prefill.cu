@@ -189,6 +189,19 @@ __device__ __forceinline__ TileInfo tile_info(int64_t tile, int64_t n_tt, int64_
   return ti;
 }
 
+// The i-th tile of this CTA, or -1 past the last. Tiles are dealt largest
+// first: token tiles in descending order (in bucket order a later token tile
+// needs as many slices or more) and, within one, the weight tiles in order;
+// pass i deals one tile to every CTA, in CTA order on even passes and in
+// reverse on odd ones, so heavy and light tiles even out across CTAs.
+__device__ __forceinline__ int64_t pf_tile(int64_t i, int64_t ntiles, int64_t n_wt, int64_t n_tt) {
+  const int64_t G = gridDim.x, c = blockIdx.x;
+  const int64_t idx = i * G + ((i & 1) ? G - 1 - c : c);
+  if (idx >= ntiles) return -1;
+  const int64_t tt = n_tt - 1 - idx / n_wt, wt = idx % n_wt;
+  return wt * n_tt + tt;
+}
+
 // Bounded wait that also gives up when another role has aborted.
 __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, uint64_t limit, DeviceStatus* st,
                                         uint32_t where, volatile int32_t* abort_flag) {
@@ -247,7 +260,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
       prefetch_tmap(&tm_codes); prefetch_tmap(&tm_sz);
       uint32_t xi = 0, ci = 0;  // running stage counters
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int64_t i = 0, tile; (tile = pf_tile(i, ntiles, n_wt, n_tt)) >= 0 && ok; ++i) {
         const TileInfo ti = tile_info(tile, n_tt, T, off, S);
         for (int64_t g = 0; g < ngroups && ok; ++g) {
           const uint32_t xs = xi % pf::XST, xph = (xi / pf::XST) & 1;
@@ -287,7 +300,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
       const uint32_t idesc = idesc_bf16(pf::BM, pf::BN);
       uint32_t xi = 0, u = 0;  // x stages, units (all units are counted by both threads)
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int64_t i = 0, tile; (tile = pf_tile(i, ntiles, n_wt, n_tt)) >= 0 && ok; ++i) {
         const TileInfo ti = tile_info(tile, n_tt, T, off, S);
         for (int64_t g = 0; g < ngroups && ok; ++g) {
           const uint32_t xs = xi % pf::XST, xph = (xi / pf::XST) & 1;
@@ -337,7 +350,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     uint32_t u = 0, hh = 0;
     bool ok = true;
-    for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+    for (int64_t i = 0, tile; (tile = pf_tile(i, ntiles, n_wt, n_tt)) >= 0 && ok; ++i) {
       const TileInfo ti = tile_info(tile, n_tt, T, off, S);
       for (int64_t g = 0; g < ngroups && ok; ++g) {
         for (int s = 0; s < ti.kmax && ok; ++s, ++u) {
@@ -398,7 +411,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     uint32_t u = 0;
     bool ok = true;
-    for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+    for (int64_t i = 0, tile; (tile = pf_tile(i, ntiles, n_wt, n_tt)) >= 0 && ok; ++i) {
       const TileInfo ti = tile_info(tile, n_tt, T, off, S);
       const int64_t n = ti.n0 + 32 * q + lane;
       float2 acc[pf::kColsPerEpi / 2];
