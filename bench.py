@@ -223,6 +223,84 @@ def l2_flush_buffer(dev):
     return torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
 
+def time_full_model(mobi, wl, dev, steps, hbm_peak):
+    """Full-model workload: pack the 7 projections x 32 layers of the Llama-2-7B-
+    shaped stack (6.5e9 fp16 parameters drawn on the device), then time batch-8
+    decode through every projection (224 mobi_linear calls per step, one CUDA
+    graph). Returns pack and decode throughput."""
+    projs = [(layer, p) for layer in range(wl.LLAMA7B_LAYERS) for p in range(len(wl.LLAMA7B_PROJECTIONS))]
+    layers = [wl.full_model_projection(layer, p, T=8, device=dev) for layer, p in projs]
+    packed = [(torch.empty((3, L.N, L.K // 16), dtype=torch.int32, device=dev),
+               torch.empty((3, L.K // 128, L.N), dtype=torch.int32, device=dev)) for L in layers]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for L, (c, z) in zip(layers[:7], packed[:7]):  # warm-up
+        mobi.mobi_pack(L.W, 3, codes=c, sz=z)
+    torch.cuda.synchronize()
+    e0.record()
+    for L, (c, z) in zip(layers, packed):
+        mobi.mobi_pack(L.W, 3, codes=c, sz=z)
+    e1.record()
+    torch.cuda.synchronize()
+    pack_ms = e0.elapsed_time(e1)
+    params = sum(L.N * L.K for L in layers)
+    pack_bytes = sum(L.N * L.K * 2 + c.numel() * 4 + z.numel() * 4 for L, (c, z) in zip(layers, packed))
+    dims = [(L.N, L.K) for L in layers]
+    for L in layers:
+        L.W = None  # free the fp16 stack (13 GB)
+    torch.cuda.empty_cache()
+
+    class Call:
+        pass
+    calls = []
+    for L, (c, z), (N, K) in zip(layers, packed, dims):
+        k = Call()
+        k.X, k.Wr = L.X.to(dev), torch.from_numpy(L.Wr).to(dev)
+        k.codes, k.sz, k.N, k.K = c, z, N, K
+        k.Y = torch.empty((8, N), dtype=torch.float32, device=dev)
+        k.k_t = torch.empty(8, dtype=torch.int32, device=dev)
+        k.perm = torch.empty(8, dtype=torch.int32, device=dev)
+        k.off = torch.empty(4, dtype=torch.int32, device=dev)
+        k.ws = torch.empty(max(mobi.mobi_linear_workspace_bytes(8, N, K, 3), 16), dtype=torch.uint8, device=dev)
+        calls.append(k)
+
+    def step():
+        for k in calls:
+            mobi.mobi_linear(k.X, k.Wr, None, k.codes, k.sz, k.N, Y=k.Y, k_t=k.k_t, perm=k.perm, offsets=k.off,
+                             ws=k.ws)
+    step()
+    torch.cuda.synchronize()
+    kmax = [int(k.k_t.max().item()) for k in calls]
+    bytes_step = sum(decode_bytes(k.N, k.K, 8, km) for k, km in zip(calls, kmax))
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(steps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    mobi.mobi_sync_check()
+    out = {"workload": "full model: 7 projections x 32 layers (Llama-2-7B shapes), batch 8, random router per "
+                       "projection; pack all, then decode through every projection (224 mobi_linear calls, one "
+                       "CUDA graph)",
+           "params": params, "pack_ms": round(pack_ms, 3), "pack_GB/s": round(pack_bytes / pack_ms / 1e6, 1),
+           "decode_ms_per_step": round(ms, 4), "decode_bytes_per_step": bytes_step,
+           "decode_GB/s": round(bytes_step / ms / 1e6, 1), "decode_frac_of_hbm": round(bytes_step / ms / 1e6 / hbm_peak, 4),
+           "kmax_histogram": [kmax.count(v) for v in (1, 2, 3)], "steps": steps}
+    del graph, calls, packed, layers
+    torch.cuda.empty_cache()
+    return out
+
+
 def time_prefill(mobi, L, dev, reps, tf_peak, flush):
     """Route + bucket + tcgen05 prefill GEMM on one prefill workload; CUDA events
     per repetition with the L2 flushed (256 MB write) before each one."""
@@ -412,8 +490,11 @@ def run_gpu(args, world, rank):
     }
     if rank == 0:
         out["pack"] = time_pack(mobi, wl, dev)
+    del cases, graph
+    torch.cuda.empty_cache()
+    if args.only == "all" and not args.skip_full_model:
+        out["full_model"] = time_full_model(mobi, wl, dev, 20, hbm_peak)
     if args.only != "decode":
-        del cases, graph
         torch.cuda.empty_cache()
         flush = l2_flush_buffer(dev)
         out["prefill"] = time_prefill(mobi, wl.prefill(), dev, args.prefill_reps, tf_peak, flush)
@@ -514,6 +595,7 @@ def main():
                     help="run a subset (profiling); the default runs everything")
     ap.add_argument("--prefill-reps", type=int, default=10)
     ap.add_argument("--skip-skewed", action="store_true")
+    ap.add_argument("--skip-full-model", action="store_true")
     args = ap.parse_args()
 
     if args.impl == "reference":
