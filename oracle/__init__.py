@@ -56,6 +56,9 @@ def _load():
             lib.oracle_reconstruct.restype = None
             lib.oracle_route.argtypes = [p, i64, i64, p, p, ci, p, p, p, ci]
             lib.oracle_route.restype = None
+            lib.oracle_route_mlp.argtypes = [p, i64, i64, p, p, i64, p, p, ci, ctypes.c_double, ctypes.c_double,
+                                             p, p, p, ci]
+            lib.oracle_route_mlp.restype = ci
             lib.oracle_bucket.argtypes = [p, i64, ci, p, p]
             lib.oracle_bucket.restype = ci
             lib.oracle_gemm.argtypes = [p, i64, i64, p, p, p, i64, ci, ci, p, i64, p, ci]
@@ -128,6 +131,28 @@ def route(X_bf16: np.ndarray, Wr: np.ndarray, bias: np.ndarray | None = None, nt
     logits = np.zeros((T, S), np.float64)
     lib.oracle_route(_ptr(X), T, K, _ptr(Wr), _ptr(b), S, _ptr(k), _ptr(gap), _ptr(logits), nthreads)
     return k, gap, logits
+
+
+def route_mlp(X_bf16: np.ndarray, W1: np.ndarray, b1: np.ndarray, W2: np.ndarray, b2: np.ndarray, tau: float,
+              delta: float, nthreads: int = 0):
+    """Threshold routing with a 2-layer MLP scorer (S = W2.shape[1] + 1).
+    Returns (k_t int32 [T], margin fp64 [T], scores fp64 [T, S-1])."""
+    lib = _load()
+    X = _u16(X_bf16)
+    T, K = X.shape
+    W1 = np.ascontiguousarray(W1, np.float32)
+    H = W1.shape[1]
+    b1 = np.ascontiguousarray(b1, np.float32)
+    W2 = np.ascontiguousarray(W2, np.float32).reshape(H, -1)
+    b2 = np.ascontiguousarray(b2, np.float32).reshape(-1)
+    S = W2.shape[1] + 1
+    k = np.zeros(T, np.int32)
+    margin = np.zeros(T, np.float64)
+    scores = np.zeros((T, max(S - 1, 1)), np.float64)
+    if lib.oracle_route_mlp(_ptr(X), T, K, _ptr(W1), _ptr(b1), H, _ptr(W2), _ptr(b2), S, float(tau), float(delta),
+                            _ptr(k), _ptr(margin), _ptr(scores), nthreads) != 0:
+        raise ValueError("oracle_route_mlp: tau must be > 0 and delta in (0, 1)")
+    return k, margin, scores[:, : S - 1]
 
 
 def bucket(k_t: np.ndarray, S: int = 3):

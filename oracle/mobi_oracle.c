@@ -27,12 +27,17 @@
  *   floored at 2^-14 and rounded to fp16 BEFORE it is used, deq = (q - z) * s,
  *   and the reconstruction W^(k) = sum_{s<k} deq_s kept exact (no rounding to
  *   a 16-bit type). Routing: a linear router, k_t = 1 + argmax (lowest index on
- *   an exact tie). Bucketing: stable ascending sort by k_t.
+ *   an exact tie). Bucketing: stable ascending sort by k_t. Threshold routing
+ *   (oracle_route_mlp): a ReLU two-layer MLP gives one score per residual
+ *   slice, a slice is active iff sigmoid(score / tau) > delta, and
+ *   k_t = 1 + the number of active residual slices.
  *
  * Parity pins: every function here is pinned by tests/test_oracle.py against
  * closed-form groups, hand-derived packed words, invariants (non-increasing
- * reconstruction error, half-step rounding bound), brute force (numpy fp64
- * matmul on tiny shapes, one-hot inputs) and special cases; see that file.
+ * reconstruction error, half-step rounding bound, fewer slices for a larger
+ * threshold), brute force (numpy fp64 matmul and Python loops on tiny shapes,
+ * one-hot inputs), library routines (torch's fp64 linear layers) and special
+ * cases; see that file.
  * Whether the quantiser reading matches the MoBiQuant authors' own Q cannot be
  * pinned from the pages ("parity unpinned" for that reading, not for the code).
  */
@@ -226,6 +231,56 @@ void oracle_route(const uint16_t* X, int64_t T, int64_t K, const float* Wr, cons
     if (logits)
       for (int j = 0; j < S; ++j) logits[t * S + j] = l[j];
   }
+}
+
+/*
+ * oracle_route_mlp: threshold routing with a two-layer MLP scorer
+ * ([ja] §2.2: a 2-layer MLP scores each token; a threshold turns the gate
+ * into a binary mask and moving it sets how many slices are active;
+ * [en] §2.B "Differentiable Gating" (temperature-scaled sigmoid, a binary
+ * mask at inference) and "Dynamic Adjustment" (raising delta activates fewer
+ * slices)). Readings where the pages are silent: ReLU hidden layer, one score
+ * per residual slice (S - 1 of them), slice j+1 active iff
+ * sigmoid(score_j / tau) > delta, and k_t = 1 + the number of active residual
+ * slices (the leading k_t slices are the ones summed).
+ *   h_i    = max(0, sum_k x[t,k] W1[k,i] + b1[i])          i < H   (fp64)
+ *   s_j    = sum_i h_i W2[i,j] + b2[j]                     j < S-1 (fp64)
+ *   active = 1 / (1 + exp(-s_j / tau)) > delta
+ * margin[t] = min_j |s_j - tau * log(delta / (1 - delta))| (the score's
+ * distance from the threshold; +inf when S == 1), scores (fp64 [T][S-1]) may
+ * be NULL. Returns -1 for tau <= 0 or delta outside (0, 1).
+ */
+int oracle_route_mlp(const uint16_t* X, int64_t T, int64_t K, const float* W1, const float* b1, int64_t H,
+                     const float* W2, const float* b2, int S, double tau, double delta, int32_t* k_out,
+                     double* margin, double* scores, int nthreads) {
+  if (!(tau > 0.0) || !(delta > 0.0 && delta < 1.0) || S < 1 || S > 8 || H < 1) return -1;
+  const double thr = tau * log(delta / (1.0 - delta));
+  set_threads(nthreads);
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    double* h = (double*)malloc((size_t)H * sizeof(double));
+    for (int64_t i = 0; i < H; ++i) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += bf16_bits_to_double(X[t * K + k]) * (double)W1[k * H + i];
+      acc += (double)b1[i];
+      h[i] = acc > 0.0 ? acc : 0.0;
+    }
+    int active = 0;
+    double m = INFINITY;
+    for (int j = 0; j < S - 1; ++j) {
+      double s = 0.0;
+      for (int64_t i = 0; i < H; ++i) s += h[i] * (double)W2[i * (S - 1) + j];
+      s += (double)b2[j];
+      if (1.0 / (1.0 + exp(-s / tau)) > delta) ++active;
+      const double d = fabs(s - thr);
+      if (d < m) m = d;
+      if (scores) scores[t * (S - 1) + j] = s;
+    }
+    free(h);
+    k_out[t] = 1 + active;
+    if (margin) margin[t] = m;
+  }
+  return 0;
 }
 
 /*

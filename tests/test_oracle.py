@@ -305,3 +305,87 @@ def test_workload_mixes(oracle):
     k, _, _ = oracle.route(L.X, L.Wr, L.bias)
     frac = np.bincount(k, minlength=4)[1:] / L.T
     assert np.all(np.abs(frac - np.array([0.7, 0.2, 0.1])) < 0.04), frac
+
+
+# ---- threshold routing with an MLP scorer ([ja] §2.2, [en] §2.B) ---------------------
+
+def _mlp_case(T=6, K=256, H=32, S=3, seed=11):
+    rng = np.random.default_rng(seed)
+    X = wl.to_bf16(rng.standard_normal((T, K), dtype=np.float32))
+    W1 = (rng.standard_normal((K, H)) / np.sqrt(K)).astype(np.float32)
+    b1 = (rng.standard_normal(H) * 0.1).astype(np.float32)
+    W2 = (rng.standard_normal((H, S - 1)) / np.sqrt(H)).astype(np.float32)
+    b2 = (rng.standard_normal(S - 1) * 0.1).astype(np.float32)
+    return X, W1, b1, W2, b2
+
+
+def test_route_mlp_scores_match_torch(oracle):
+    """Library pin: torch's fp64 linear layers with ReLU give the same scores."""
+    X, W1, b1, W2, b2 = _mlp_case()
+    _, _, scores = oracle.route_mlp(X, W1, b1, W2, b2, tau=1.0, delta=0.5)
+    x = X.to(torch.float64)
+    h = torch.nn.functional.relu(torch.nn.functional.linear(x, torch.from_numpy(W1).double().T,
+                                                            torch.from_numpy(b1).double()))
+    s = torch.nn.functional.linear(h, torch.from_numpy(W2).double().T, torch.from_numpy(b2).double())
+    assert np.allclose(scores, s.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_route_mlp_constant_score_closed_form(oracle):
+    """W2 = 0: the score is b2 for every token, so sigmoid(b2 / tau) > delta
+    decides every token alike (closed form)."""
+    X, W1, b1, _, _ = _mlp_case(T=5, S=3)
+    W2 = np.zeros((W1.shape[1], 2), np.float32)
+    # sigmoid(0.5) = 0.6225 and sigmoid(-0.5) = 0.3775
+    k, _, _ = oracle.route_mlp(X, W1, b1, W2, np.array([0.5, -0.5], np.float32), tau=1.0, delta=0.5)
+    assert k.tolist() == [2] * 5                 # first residual slice on, second off
+    k, _, _ = oracle.route_mlp(X, W1, b1, W2, np.array([0.5, 0.5], np.float32), tau=1.0, delta=0.6)
+    assert k.tolist() == [3] * 5                 # 0.6225 > 0.6 for both
+    k, _, _ = oracle.route_mlp(X, W1, b1, W2, np.array([0.5, 0.5], np.float32), tau=1.0, delta=0.7)
+    assert k.tolist() == [1] * 5                 # 0.6225 < 0.7
+    k, _, _ = oracle.route_mlp(X, W1, b1, W2, np.array([0.5, 0.5], np.float32), tau=4.0, delta=0.55)
+    assert k.tolist() == [1] * 5                 # sigmoid(0.5 / 4) = 0.5312 < 0.55: temperature matters
+
+def test_route_mlp_delta_half_is_sign(oracle):
+    """delta = 0.5: sigmoid(s / tau) > 1/2 exactly when s > 0, for any tau > 0."""
+    X, W1, b1, W2, b2 = _mlp_case(T=40, S=3, seed=12)
+    for tau in (0.3, 1.0, 7.0):
+        k, _, scores = oracle.route_mlp(X, W1, b1, W2, b2, tau=tau, delta=0.5)
+        assert np.array_equal(k, 1 + (scores > 0).sum(axis=1))
+
+
+def test_route_mlp_monotone_in_delta(oracle):
+    """[en] §2.B: raising delta activates fewer slices, never more."""
+    X, W1, b1, W2, b2 = _mlp_case(T=64, S=3, seed=13)
+    prev = None
+    for delta in (0.05, 0.2, 0.4, 0.5, 0.6, 0.8, 0.95):
+        k, _, _ = oracle.route_mlp(X, W1, b1, W2, b2, tau=0.5, delta=delta)
+        if prev is not None:
+            assert np.all(k <= prev)
+        prev = k
+    assert prev.min() >= 1
+
+
+def test_route_mlp_brute_force_tiny(oracle):
+    """Pure-Python loops on a tiny case."""
+    import math
+    X, W1, b1, W2, b2 = _mlp_case(T=3, K=8, H=3, S=3, seed=14)
+    x = X.float().numpy().astype(np.float64)
+    tau, delta = 0.7, 0.45
+    k, _, _ = oracle.route_mlp(X, W1, b1, W2, b2, tau=tau, delta=delta)
+    for t in range(3):
+        h = [max(0.0, sum(x[t, kk] * float(W1[kk, i]) for kk in range(8)) + float(b1[i])) for i in range(3)]
+        active = 0
+        for j in range(2):
+            sj = sum(h[i] * float(W2[i, j]) for i in range(3)) + float(b2[j])
+            active += 1.0 / (1.0 + math.exp(-sj / tau)) > delta
+        assert k[t] == 1 + active
+
+
+def test_route_mlp_one_slice_and_bad_args(oracle):
+    X, W1, b1, _, _ = _mlp_case(T=4, S=3)
+    k, margin, _ = oracle.route_mlp(X, W1, b1, np.zeros((W1.shape[1], 0), np.float32), np.zeros(0, np.float32),
+                                    tau=1.0, delta=0.5)
+    assert k.tolist() == [1] * 4 and np.all(np.isinf(margin))
+    with pytest.raises(ValueError):
+        oracle.route_mlp(X, W1, b1, np.zeros((W1.shape[1], 2), np.float32), np.zeros(2, np.float32),
+                         tau=0.0, delta=0.5)
