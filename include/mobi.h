@@ -147,6 +147,45 @@ MOBI_API mobi_status mobi_route(const void* X, int64_t T, int64_t K, const float
                        const float* bias, int S, int32_t* k_t, int32_t* perm,
                        int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
 
+/* Scratch bytes that mobi_route_mlp needs on the current device: the fp32
+ * hidden pre-activations of every K split, splits * T * H * 4 rounded up to
+ * 256 (the split count depends on T, K, H and the device's SM count; 0 for
+ * invalid sizes). */
+MOBI_API size_t mobi_route_mlp_workspace_bytes(int64_t T, int64_t K, int64_t H);
+
+/*
+ * mobi_route_mlp — threshold routing with a two-layer MLP scorer.
+ *   [ja] §2.2: a small MLP scores each token and, at inference, a threshold
+ *   turns the gate into a binary mask; moving the threshold trades accuracy
+ *   for speed. [en] §2.B "Differentiable Gating" (temperature-scaled sigmoid
+ *   gate) and "Dynamic Adjustment" (a larger delta activates fewer slices).
+ *   Readings where the pages are silent: a ReLU hidden layer, one score per
+ *   residual slice, k_t = 1 + the number of active residual slices:
+ *     h_i = max(0, sum_k x[t,k] W1[k,i] + b1[i])       (fp32 accumulation)
+ *     s_j = sum_i h_i W2[i,j] + b2[j],   j < S-1       (fp32 accumulation)
+ *     slice j+1 active  iff  sigmoid(s_j / tau) > delta,
+ *   evaluated as s_j > tau * log(delta / (1 - delta)) in fp64 (the same test,
+ *   the sigmoid being increasing).
+ *   X        bf16 [T][K] row-major; K % 128 == 0.
+ *   W1       fp32 [K][H] row-major.  b1  fp32 [H], or NULL for zeros.
+ *   W2       fp32 [H][S-1] row-major. b2  fp32 [S-1], or NULL for zeros.
+ *            (W1, W2 may be NULL when S == 1: every k_t is then 1.)
+ *   H        hidden width, 1..65536.
+ *   tau      temperature, > 0 and finite.  delta  threshold in (0, 1).
+ *   k_t, perm, offsets  out, exactly as for mobi_route.
+ *   ws       scratch of mobi_route_mlp_workspace_bytes(T, K, H) bytes (may
+ *            be NULL for S == 1 or T == 0).
+ * Errors: MOBI_ERR_INVALID_ARG for a bad tau, delta, S, H or missing pointer,
+ * MOBI_ERR_UNSUPPORTED_SHAPE for K not a multiple of 128 or sizes above the
+ * limits, MOBI_ERR_MISALIGNED (X and ws 16-byte, the rest 4-byte aligned),
+ * MOBI_ERR_WORKSPACE for a short ws; nothing is launched then.
+ */
+MOBI_API mobi_status mobi_route_mlp(const void* X, int64_t T, int64_t K, const float* W1,
+                                    const float* b1, int64_t H, const float* W2,
+                                    const float* b2, int S, double tau, double delta,
+                                    int32_t* k_t, int32_t* perm, int32_t* offsets, void* ws,
+                                    size_t ws_bytes, void* stream);
+
 /*
  * mobi_gemm — token-routed mixed-bit GEMM.
  *   y[t,n] = sum_k x[t,k] * W^(k_t)[n,k],  W^(k) = sum_{s<k} deq_s,

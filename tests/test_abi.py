@@ -116,3 +116,38 @@ def test_workspace_sizes_edge_cases(L):
     assert mobi.mobi_route_workspace_bytes(0, 256, 3) == 0
     assert mobi.mobi_route_workspace_bytes(2048, 4096, 3) == 0   # many token tiles: no split
     assert mobi.mobi_gemm_workspace_bytes(0, 0, 0, 3) >= 0
+
+
+def test_route_mlp_validation(L):
+    """Every rejection happens on the host, before a launch (no GPU needed)."""
+    p = ctypes.c_void_p
+
+    def call(T=16, K=256, H=128, S=3, tau=1.0, delta=0.5, X=p(FAKE), W1=p(FAKE), W2=p(FAKE), ws=p(FAKE),
+             wsb=1 << 30, perm=p(FAKE)):
+        return L.mobi_route_mlp(X, T, K, W1, None, H, W2, None, S, tau, delta, p(FAKE), perm, p(FAKE), ws, wsb,
+                                None)
+    assert call(tau=0.0) == 1
+    assert call(tau=-1.0) == 1
+    assert call(tau=float("inf")) == 1
+    assert call(tau=float("nan")) == 1
+    assert call(delta=0.0) == 1
+    assert call(delta=1.0) == 1
+    assert call(delta=float("nan")) == 1
+    assert call(S=0) == 1 and call(S=4) == 1
+    assert call(H=0) == 1
+    assert call(T=-1) == 1
+    assert call(K=200) == 2
+    assert call(H=65537) == 2
+    assert call(X=None) == 1 and call(perm=None) == 1
+    assert call(W1=None) == 1 and call(W2=None) == 1
+    assert call(X=p(FAKE + 8)) == 3
+    assert call(ws=p(FAKE + 8)) == 3
+    assert call(W1=p(FAKE + 2)) == 3
+    assert call(wsb=16) == 4
+    assert call(ws=None, wsb=0) == 4
+    for T, K, H in ((16, 4096, 128), (3, 128, 7), (2048, 4096, 128), (1, 128, 65536)):
+        b = mobi.mobi_route_mlp_workspace_bytes(T, K, H)
+        assert b >= T * H * 4 and b % 256 == 0, (T, K, H, b)
+        assert b <= max(K // 64, 1) * T * H * 4 + 255  # at most one split per 64 rows of K
+    assert mobi.mobi_route_mlp_workspace_bytes(0, 4096, 128) == 0
+    assert mobi.mobi_route_mlp_workspace_bytes(16, 4096, 0) == 0

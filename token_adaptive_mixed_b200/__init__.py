@@ -9,6 +9,7 @@ or a tensor is not on a CUDA device, the call raises.
 Entry points (same names as the C ABI):
   mobi_pack(W)                      MoBiSlice packing   -> (codes, sz)
   mobi_route(X, Wr, bias)           MoBiRoute routing   -> (k_t, perm, offsets)
+  mobi_route_mlp(X, W1, b1, W2, b2, tau, delta)  threshold routing, MLP scorer -> (k_t, perm, offsets)
   mobi_gemm(X, k_t, perm, offsets, codes, sz, N)         -> Y  (fp32)
   mobi_gemm_path(..., path)         the same with a forced kernel
   mobi_linear(X, Wr, bias, codes, sz, N)  route + GEMM in one call -> (Y, k_t, perm, offsets)
@@ -25,7 +26,7 @@ __all__ = [
     "MobiError", "lib", "mobi_version", "mobi_status_string", "mobi_codes_bytes", "mobi_sz_bytes",
     "mobi_route_workspace_bytes", "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm", "mobi_last_error",
     "mobi_gemm_path", "mobi_sync_check", "mobi_debug_set_wait_limit", "mobi_gemm_decode_noalloc", "mobi_linear",
-    "mobi_linear_workspace_bytes", "PATH_AUTO",
+    "mobi_linear_workspace_bytes", "mobi_route_mlp", "mobi_route_mlp_workspace_bytes", "PATH_AUTO",
     "PATH_DECODE",
     "PATH_PREFILL", "EXPORTED_SYMBOLS",
 ]
@@ -42,6 +43,7 @@ EXPORTED_SYMBOLS = (
     "mobi_status_string", "mobi_last_error", "mobi_version", "mobi_codes_bytes", "mobi_sz_bytes", "mobi_route_workspace_bytes",
     "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm", "mobi_gemm_path", "mobi_sync_check",
     "mobi_debug_set_wait_limit", "mobi_gemm_decode_noalloc", "mobi_linear", "mobi_linear_workspace_bytes",
+    "mobi_route_mlp", "mobi_route_mlp_workspace_bytes",
 )
 
 
@@ -92,6 +94,11 @@ def lib() -> ctypes.CDLL:
         L.mobi_linear_workspace_bytes.restype = sz_t
         L.mobi_linear.argtypes = [p, i64, i64, p, p, p, p, i64, ci, ci, p, p, p, p, p, sz_t, p]
         L.mobi_linear.restype = ci
+        L.mobi_route_mlp_workspace_bytes.argtypes = [i64, i64, i64]
+        L.mobi_route_mlp_workspace_bytes.restype = sz_t
+        L.mobi_route_mlp.argtypes = [p, i64, i64, p, p, i64, p, p, ci, ctypes.c_double, ctypes.c_double, p, p, p,
+                                     p, sz_t, p]
+        L.mobi_route_mlp.restype = ci
         L.mobi_sync_check.argtypes = [p]
         L.mobi_sync_check.restype = ci
         L.mobi_debug_set_wait_limit.argtypes = [i64]
@@ -185,6 +192,33 @@ def mobi_route(X: torch.Tensor, Wr: torch.Tensor, bias: torch.Tensor | None = No
     _check("mobi_route", lib().mobi_route(_ptr(X), T, K, _ptr(Wr), _ptr(bias), S, _ptr(k_t), _ptr(perm),
                                           _ptr(offsets), _ptr(ws), 0 if ws is None else ws.numel(),
                                           _stream(stream)))
+    return k_t, perm, offsets
+
+
+def mobi_route_mlp_workspace_bytes(T: int, K: int, H: int) -> int:
+    return lib().mobi_route_mlp_workspace_bytes(T, K, H)
+
+
+def mobi_route_mlp(X: torch.Tensor, W1: torch.Tensor, b1: torch.Tensor | None, W2: torch.Tensor,
+                   b2: torch.Tensor | None, tau: float = 1.0, delta: float = 0.5, S: int | None = None, k_t=None,
+                   perm=None, offsets=None, ws: torch.Tensor | None = None, stream=None):
+    """Threshold routing with a two-layer MLP scorer: k_t = 1 + #{j : sigmoid(s_j / tau) > delta},
+    s = ReLU(x.W1 + b1).W2 + b2, then the stable bucketing -> (k_t, perm, offsets).
+    S defaults to W2.shape[1] + 1."""
+    if X.dtype != torch.bfloat16 or W1.dtype != torch.float32 or W2.dtype != torch.float32:
+        raise ValueError("X must be bf16, W1 and W2 fp32")
+    T, K = X.shape
+    H = W1.shape[1]
+    S = W2.shape[1] + 1 if S is None else S
+    dev = X.device
+    k_t = torch.empty(T, dtype=torch.int32, device=dev) if k_t is None else k_t
+    perm = torch.empty(T, dtype=torch.int32, device=dev) if perm is None else perm
+    offsets = torch.empty(S + 1, dtype=torch.int32, device=dev) if offsets is None else offsets
+    need = mobi_route_mlp_workspace_bytes(T, K, H) if S > 1 else 0
+    ws = _workspace(need, dev, ws) if need > 0 else ws
+    _check("mobi_route_mlp", lib().mobi_route_mlp(_ptr(X), T, K, _ptr(W1), _ptr(b1), H, _ptr(W2), _ptr(b2), S,
+                                                  float(tau), float(delta), _ptr(k_t), _ptr(perm), _ptr(offsets),
+                                                  _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
     return k_t, perm, offsets
 
 

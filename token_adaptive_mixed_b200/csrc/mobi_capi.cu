@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -22,6 +23,10 @@ cudaError_t launch_pack(const void* W, int64_t N, int64_t K, int S, uint32_t* co
 cudaError_t launch_route(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias, int S,
                          int32_t* k_t, int32_t* perm, int32_t* offsets, void* ws, cudaStream_t stream);
 size_t route_ws_bytes(int64_t T, int64_t K, int S);
+cudaError_t launch_route_mlp(const void* X, int64_t T, int64_t K, const float* W1, const float* b1, int64_t H,
+                             const float* W2, const float* b2, int S, double thr, int32_t* k_t, int32_t* perm,
+                             int32_t* offsets, void* ws, cudaStream_t stream, int sms);
+size_t route_mlp_ws_bytes(int64_t T, int64_t K, int64_t H, int sms);
 cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
                           const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
                           DeviceStatus* st, bool early);
@@ -191,6 +196,7 @@ using namespace mobi;
 namespace {
 
 constexpr int64_t kMaxDim = int64_t(1) << 28;
+constexpr int64_t kMaxMlpHidden = 65536;  // scorer hidden width: grid.y of the hidden-layer kernel stays small
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -281,6 +287,34 @@ mobi_status mobi_route(const void* X, int64_t T, int64_t K, const float* Wr, con
   if (ws && !aligned16(ws)) return MOBI_ERR_MISALIGNED;
   return cuda_status(
       launch_route(X, T, K, Wr, bias, S, k_t, perm, offsets, ws, static_cast<cudaStream_t>(stream)));
+}
+
+size_t mobi_route_mlp_workspace_bytes(int64_t T, int64_t K, int64_t H) {
+  if (T < 0 || K < 0 || H < 1) return 0;
+  return route_mlp_ws_bytes(T, K, H, num_sms());
+}
+
+mobi_status mobi_route_mlp(const void* X, int64_t T, int64_t K, const float* W1, const float* b1, int64_t H,
+                           const float* W2, const float* b2, int S, double tau, double delta, int32_t* k_t,
+                           int32_t* perm, int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  if (T < 0 || K < 0 || H < 1 || S < 1 || S > 3) return MOBI_ERR_INVALID_ARG;
+  if (!(tau > 0.0) || !std::isfinite(tau) || !(delta > 0.0 && delta < 1.0)) return MOBI_ERR_INVALID_ARG;
+  if (K % 128 != 0 || K > kMaxDim || T > kMaxDim || H > kMaxMlpHidden) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  if (!offsets || (T > 0 && (!X || !k_t || !perm))) return MOBI_ERR_INVALID_ARG;
+  if (T > 0 && S > 1 && (!W1 || !W2)) return MOBI_ERR_INVALID_ARG;
+  if (T > 0 && K == 0) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  if ((X && !aligned16(X)) || (W1 && !aligned4(W1)) || (b1 && !aligned4(b1)) || (W2 && !aligned4(W2)) ||
+      (b2 && !aligned4(b2)) || (k_t && !aligned4(k_t)) || (perm && !aligned4(perm)) || !aligned4(offsets) ||
+      (ws && !aligned16(ws)))
+    return MOBI_ERR_MISALIGNED;
+  const int sms = num_sms();
+  const size_t need = S > 1 ? route_mlp_ws_bytes(T, K, H, sms) : 0;
+  if (need > 0 && (!ws || ws_bytes < need)) return MOBI_ERR_WORKSPACE;
+  // sigmoid(s / tau) > delta  <=>  s > tau * log(delta / (1 - delta))  (the sigmoid is increasing)
+  const double thr = tau * std::log(delta / (1.0 - delta));
+  return cuda_status(launch_route_mlp(X, T, K, W1, b1, H, W2, b2, S, thr, k_t, perm, offsets, ws,
+                                      static_cast<cudaStream_t>(stream), sms));
 }
 
 mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,

@@ -376,6 +376,228 @@ static cudaError_t launch_route_small(const void* X, int64_t T, int64_t K, const
   return note_error("kernel launch", cudaGetLastError());
 }
 
+// ---- threshold routing with a two-layer MLP scorer -----------------------------------
+//
+// MoBiQuant explainer [ja] §2.2 (a 2-layer MLP scores each token; at inference
+// a threshold turns the gate into a binary mask, and moving the threshold sets
+// how many slices are active) and [en] §2.B ("Differentiable Gating",
+// "Dynamic Adjustment": a larger delta activates fewer slices). Readings: ReLU
+// hidden layer, one score per residual slice, slice j+1 active iff
+// sigmoid(score_j / tau) > delta (i.e. score_j > tau * log(delta / (1 - delta))),
+// k_t = 1 + the number of active residual slices.
+//
+// route_mlp_hidden_kernel<TT>: the first layer's pre-activations, split along
+//   K: P[s][t][i] = sum_{k in split s} x[t,k] W1[k,i] (fp32 FMAs in k order).
+//   CTA = 16 TT tokens x 128 hidden units, 256 threads, each TT tokens x 8
+//   units (columns 4 tx .. 4 tx + 3 and 64 + 4 tx .. 64 + 4 tx + 3, so the
+//   128-bit shared loads of a quarter-warp hit distinct banks); K runs in
+//   32-row chunks staged in shared memory (x converted to fp32 and stored
+//   k-major, the [32][128] slice of W1). TT = 4 for prefill (ALU-bound: T K H
+//   FMAs), TT = 1 for up to 16 tokens (bound by the W1 read, K H 4 bytes).
+// route_mlp_score_kernel<S>: one CTA of 128 threads per token: h_i =
+//   max(0, sum_s P[s][t][i] + b1[i]) (splits in order), the thread's products
+//   h_i W2[i][j] accumulated over i = tid, tid + 128, ..., an xor tree per warp
+//   and the four warps in order, + b2[j], compared with the threshold in fp64.
+// The bucketing is bucket_kernel (no split logits).
+constexpr int kMlpHidTile = 128, kMlpKc = 32, kMlpThreads = 256, kMlpScoreThreads = 128;
+constexpr int kMlpMinSplitK = 64;
+
+template <int TT>
+__global__ void __launch_bounds__(kMlpThreads) route_mlp_hidden_kernel(const __nv_bfloat16* __restrict__ X,
+                                                                      int64_t T, int64_t K,
+                                                                      const float* __restrict__ W1, int64_t H,
+                                                                      int64_t k_per_split,
+                                                                      float* __restrict__ P) {
+  constexpr int kTok = 16 * TT;
+  __shared__ __align__(16) float xs[kMlpKc][kTok + 4];
+  __shared__ __align__(16) float wsm[kMlpKc][kMlpHidTile];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int64_t t0 = (int64_t)blockIdx.x * kTok, h0 = (int64_t)blockIdx.y * kMlpHidTile;
+  const int64_t split = blockIdx.z, kb = split * k_per_split;
+  const int64_t ke = kb + k_per_split < K ? kb + k_per_split : K;
+  const bool vec = (H & 3) == 0 && (reinterpret_cast<uintptr_t>(W1) & 15) == 0;
+  float acc[TT][8];
+#pragma unroll
+  for (int i = 0; i < TT; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+
+  for (int64_t k0 = kb; k0 < ke; k0 += kMlpKc) {  // K and every split are multiples of 32
+#pragma unroll
+    for (int m = 0; m < kTok * kMlpKc / kMlpThreads; ++m) {
+      const int e = tid + m * kMlpThreads, r = e >> 5, c = e & 31;
+      const int64_t t = t0 + r;
+      xs[c][r] = t < T ? __bfloat162float(X[t * K + k0 + c]) : 0.0f;
+    }
+#pragma unroll
+    for (int m = 0; m < kMlpKc * kMlpHidTile / 4 / kMlpThreads; ++m) {
+      const int e = tid + m * kMlpThreads, r = e >> 5, c4 = (e & 31) * 4;
+      const int64_t h = h0 + c4;
+      const float* src = W1 + (k0 + r) * H + h;
+      float4 v;
+      if (vec && h + 3 < H) {
+        v = __ldg(reinterpret_cast<const float4*>(src));
+      } else {
+        v.x = h < H ? __ldg(src) : 0.0f;
+        v.y = h + 1 < H ? __ldg(src + 1) : 0.0f;
+        v.z = h + 2 < H ? __ldg(src + 2) : 0.0f;
+        v.w = h + 3 < H ? __ldg(src + 3) : 0.0f;
+      }
+      *reinterpret_cast<float4*>(&wsm[r][c4]) = v;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int c = 0; c < kMlpKc; ++c) {
+      float xv[TT];
+      if constexpr (TT == 4) {
+        const float4 q = *reinterpret_cast<const float4*>(&xs[c][ty * 4]);
+        xv[0] = q.x; xv[1] = q.y; xv[2] = q.z; xv[3] = q.w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < TT; ++i) xv[i] = xs[c][ty * TT + i];
+      }
+      const float4 wa = *reinterpret_cast<const float4*>(&wsm[c][tx * 4]);
+      const float4 wb = *reinterpret_cast<const float4*>(&wsm[c][64 + tx * 4]);
+      const float w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+      for (int i = 0; i < TT; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(xv[i], w[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  asm volatile("griddepcontrol.launch_dependents;");
+#pragma unroll
+  for (int i = 0; i < TT; ++i) {
+    const int64_t t = t0 + ty * TT + i;
+    if (t >= T) continue;
+    float* row = P + (split * T + t) * H;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t h = h0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
+      if (h < H) row[h] = acc[i][j];
+    }
+  }
+}
+
+template <int S>
+__global__ void __launch_bounds__(kMlpScoreThreads) route_mlp_score_kernel(const float* __restrict__ P, int64_t T,
+                                                                          int64_t H, int ksplit,
+                                                                          const float* __restrict__ b1,
+                                                                          const float* __restrict__ W2,
+                                                                          const float* __restrict__ b2,
+                                                                          double thr, int32_t* __restrict__ k_t) {
+  constexpr int J = S - 1;
+  __shared__ float red[kMlpScoreThreads / 32][J];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t t = blockIdx.x;
+  float acc[J];
+#pragma unroll
+  for (int j = 0; j < J; ++j) acc[j] = 0.0f;
+  for (int64_t i = tid; i < H; i += kMlpScoreThreads) {
+    float pre = 0.0f;
+    for (int sp = 0; sp < ksplit; ++sp) pre += P[((int64_t)sp * T + t) * H + i];
+    const float hv = fmaxf(pre + (b1 ? __ldg(b1 + i) : 0.0f), 0.0f);
+#pragma unroll
+    for (int j = 0; j < J; ++j) acc[j] = fmaf(hv, __ldg(W2 + i * J + j), acc[j]);
+  }
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    float v = acc[j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[warp][j] = v;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int active = 0;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      float v = red[0][j];
+#pragma unroll
+      for (int w = 1; w < kMlpScoreThreads / 32; ++w) v += red[w][j];
+      if (b2) v += __ldg(b2 + j);
+      active += ((double)v > thr) ? 1 : 0;
+    }
+    k_t[t] = 1 + active;
+  }
+}
+
+__global__ void route_mlp_base_only_kernel(int64_t T, int32_t* __restrict__ k_t) {
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < T) k_t[t] = 1;
+}
+
+// Splits of K for the hidden layer: about four CTAs per SM in all, each split
+// a multiple of 32 rows and at least 64.
+static int64_t mlp_k_per_split(int64_t T, int64_t K, int64_t H, int sms) {
+  const int64_t tok = T <= 16 ? 16 : 64;
+  int64_t base = ((T + tok - 1) / tok) * ((H + kMlpHidTile - 1) / kMlpHidTile);
+  if (base < 1) base = 1;
+  int64_t ks = (4 * (int64_t)sms + base - 1) / base;
+  const int64_t kmax = K / kMlpMinSplitK > 0 ? K / kMlpMinSplitK : 1;
+  if (ks > kmax) ks = kmax;
+  if (ks < 1) ks = 1;
+  int64_t kps = (K + ks - 1) / ks;
+  kps = (kps + kMlpKc - 1) / kMlpKc * kMlpKc;
+  return kps > 0 ? kps : kMlpKc;
+}
+
+size_t route_mlp_ws_bytes(int64_t T, int64_t K, int64_t H, int sms) {
+  if (T <= 0 || H <= 0) return 0;
+  const int64_t kps = mlp_k_per_split(T, K, H, sms);
+  const int64_t ks = K > 0 ? (K + kps - 1) / kps : 1;
+  return ((size_t)ks * (size_t)T * (size_t)H * sizeof(float) + 255) / 256 * 256;
+}
+
+template <int S>
+static void launch_mlp_score(const float* P, int64_t T, int64_t H, int ks, const float* b1, const float* W2,
+                             const float* b2, double thr, int32_t* k_t, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)T);
+  cfg.blockDim = dim3(kMlpScoreThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, route_mlp_score_kernel<S>, P, T, H, ks, b1, W2, b2, thr, k_t);
+}
+
+cudaError_t launch_route_mlp(const void* X, int64_t T, int64_t K, const float* W1, const float* b1, int64_t H,
+                             const float* W2, const float* b2, int S, double thr, int32_t* k_t, int32_t* perm,
+                             int32_t* offsets, void* ws, cudaStream_t stream, int sms) {
+  if (T > 0 && S == 1) {  // no residual slice to score: every token keeps the base slice only
+    route_mlp_base_only_kernel<<<(unsigned)((T + 255) / 256), 256, 0, stream>>>(T, k_t);
+  } else if (T > 0) {
+    float* P = static_cast<float*>(ws);
+    const int64_t kps = mlp_k_per_split(T, K, H, sms);
+    const int ks = (int)((K + kps - 1) / kps);
+    const bool small = T <= 16;
+    const int64_t tok = small ? 16 : 64;
+    dim3 grid((unsigned)((T + tok - 1) / tok), (unsigned)((H + kMlpHidTile - 1) / kMlpHidTile), (unsigned)ks);
+    if (small)
+      route_mlp_hidden_kernel<1><<<grid, kMlpThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T, K, W1, H,
+                                                                   kps, P);
+    else
+      route_mlp_hidden_kernel<4><<<grid, kMlpThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T, K, W1, H,
+                                                                   kps, P);
+    if (S == 2)
+      launch_mlp_score<2>(P, T, H, ks, b1, W2, b2, thr, k_t, stream);
+    else
+      launch_mlp_score<3>(P, T, H, ks, b1, W2, b2, thr, k_t, stream);
+  }
+  switch (S) {
+    case 1: bucket_kernel<1><<<1, kBucketThreads, 0, stream>>>(T, 1, nullptr, nullptr, k_t, perm, offsets); break;
+    case 2: bucket_kernel<2><<<1, kBucketThreads, 0, stream>>>(T, 1, nullptr, nullptr, k_t, perm, offsets); break;
+    default: bucket_kernel<3><<<1, kBucketThreads, 0, stream>>>(T, 1, nullptr, nullptr, k_t, perm, offsets); break;
+  }
+  return note_error("kernel launch", cudaGetLastError());
+}
+
 int route_ksplit(int64_t T, int64_t K) {
   const int64_t tiles = (T + kRouteTB - 1) / kRouteTB;
   if (tiles == 0 || tiles >= 64) return 1;

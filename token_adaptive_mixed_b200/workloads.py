@@ -18,6 +18,10 @@ then rounded to its storage type with round-to-nearest-even):
     Gaussian model of the logits, l ~ N(0, Wr^T Wr) (times the token factor for
     the scaled tokens), by bisection on a fixed Monte-Carlo sample, so that
     P(argmax = j) matches the target fractions. It depends on Wr only, never on X.
+  * two-layer MLP scorer (threshold routing): W1[K,H] ~ N(0, 1/K), b1[H] ~
+    N(0, 0.1^2), W2[H,S-1] ~ N(0, 2/H) (He scale after the ReLU), b2[S-1] =
+    the given offsets (0 by default), all fp32; with tau = 1 and delta = 0.5
+    each residual slice is then active for about half of the tokens.
 """
 from __future__ import annotations
 
@@ -184,3 +188,54 @@ def full_model_projection(layer_idx: int, proj_idx: int, T: int = 8, device: str
     X = draw_activations(rng, T, K)
     Wr = draw_router(rng, K, S_DEFAULT)
     return Layer(f"L{layer_idx}.{name}", W, X, Wr, None)
+
+
+# ---- MLP scorer for threshold routing -----------------------------------------
+
+@dataclasses.dataclass
+class MlpRouter:
+    """Inputs of threshold routing with a two-layer MLP scorer."""
+    name: str
+    X: torch.Tensor        # bf16 [T, K] (CPU)
+    W1: np.ndarray         # fp32 [K, H]
+    b1: np.ndarray         # fp32 [H]
+    W2: np.ndarray         # fp32 [H, S-1]
+    b2: np.ndarray         # fp32 [S-1]
+
+    @property
+    def T(self) -> int:
+        return self.X.shape[0]
+
+    @property
+    def K(self) -> int:
+        return self.X.shape[1]
+
+    @property
+    def H(self) -> int:
+        return self.W1.shape[1]
+
+    @property
+    def S(self) -> int:
+        return self.W2.shape[1] + 1
+
+
+def mlp_router(name: str, T: int, K: int, H: int, seed: int, S: int = S_DEFAULT,
+               b2: Sequence[float] | None = None, token_scaled_frac: float = 0.0,
+               token_scale: float = 1.0) -> MlpRouter:
+    rng = np.random.default_rng(seed)
+    X = draw_activations(rng, T, K, token_scaled_frac, token_scale)
+    W1 = (rng.standard_normal((K, H), dtype=np.float32) / np.float32(np.sqrt(K))).astype(np.float32)
+    b1 = (rng.standard_normal(H, dtype=np.float32) * np.float32(0.1)).astype(np.float32)
+    W2 = (rng.standard_normal((H, S - 1), dtype=np.float32) * np.float32(np.sqrt(2.0 / H))).astype(np.float32)
+    b2a = np.zeros(S - 1, np.float32) if b2 is None else np.asarray(b2, np.float32).reshape(S - 1)
+    return MlpRouter(name, X, W1, b1, W2, b2a)
+
+
+def mlp_route_decode(T: int = 16) -> MlpRouter:
+    """Threshold routing at decode: T tokens of a K=4096 hidden state, H=128 scorer, S=3, seed 7."""
+    return mlp_router(f"mlp_route_K4096_H128_T{T}", T, 4096, 128, seed=7)
+
+
+def mlp_route_prefill(T: int = 2048) -> MlpRouter:
+    """Threshold routing at prefill: T=2048 tokens, K=4096, H=128, S=3, seed 8."""
+    return mlp_router(f"mlp_route_K4096_H128_T{T}", T, 4096, 128, seed=8)
