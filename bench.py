@@ -186,6 +186,62 @@ def launches_per_call(T, K):
     return 1 + 1 + (1 if K > 1024 else 0)
 
 
+def grouped_launches(group_T, group_K):
+    """Library kernels of one mobi_linear_grouped call: one routing launch, one
+    decode launch per fragment class present (T <= 8, T > 8) and one
+    chunk-reduce launch when any problem's K spans more than one chunk."""
+    classes = len({1 if T <= 8 else 2 for T in group_T})
+    return 1 + classes + (1 if any(K > 1024 for K in group_K) else 0)
+
+
+def time_graph(step, steps, warmup=3):
+    """Capture step() in a CUDA graph and return the mean ms of `steps` replays."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()
+        step()
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del graph
+    return e0.elapsed_time(e1) / steps
+
+
+def time_decode_grouped(mobi, cases, bytes_step, steps, hbm_peak):
+    """The headline decode step through mobi_linear_grouped: the six calls with
+    T <= 8 as one group and the three with T = 16 as another, so one step is two
+    grouped calls instead of nine mobi_linear calls (same inputs, same outputs)."""
+    groups = [[c for c in cases if c.T <= 8], [c for c in cases if c.T > 8]]
+    probs = [[{"X": c.X, "Wr": c.Wr, "bias": None, "codes": c.codes, "sz": c.sz, "N": c.N, "Y": c.Y,
+               "k_t": c.k_t, "perm": c.perm, "offsets": c.off} for c in g] for g in groups]
+    ws = [torch.empty(max(mobi.mobi_linear_grouped_workspace_bytes(pr), 16), dtype=torch.uint8,
+                      device=cases[0].X.device) for pr in probs]
+
+    def step():
+        for pr, w in zip(probs, ws):
+            mobi.mobi_linear_grouped(pr, ws=w)
+    step()
+    mobi.mobi_sync_check()
+    ms = time_graph(step, steps)
+    mobi.mobi_sync_check()
+    launches = sum(grouped_launches([c.T for c in g], [c.K for c in g]) for g in groups)
+    return {"workload": "the same nine decode calls as two mobi_linear_grouped calls (T <= 8: six problems; "
+                        "T = 16: three)", "ms_per_step": round(ms, 5),
+            "GB/s": round(bytes_step / ms / 1e6, 1), "frac_of_hbm": round(bytes_step / ms / 1e6 / hbm_peak, 4),
+            "launches_per_step": launches, "steps": steps}
+
+
 def build_decode_cases(mobi, wl, dev):
     cases = []
     for (N, K) in wl.DECODE_SHAPES:
@@ -289,14 +345,37 @@ def time_full_model(mobi, wl, dev, steps, hbm_peak):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     mobi.mobi_sync_check()
+    del graph
+
+    # The same step with the seven projections of each layer in one
+    # mobi_linear_grouped call (32 calls per step).
+    per_layer = len(wl.LLAMA7B_PROJECTIONS)
+    layer_probs = []
+    for li in range(0, len(calls), per_layer):
+        pr = [{"X": k.X, "Wr": k.Wr, "bias": None, "codes": k.codes, "sz": k.sz, "N": k.N, "Y": k.Y, "k_t": k.k_t,
+               "perm": k.perm, "offsets": k.off} for k in calls[li:li + per_layer]]
+        layer_probs.append(pr)
+    gws = torch.empty(max(mobi.mobi_linear_grouped_workspace_bytes(layer_probs[0]), 16), dtype=torch.uint8,
+                      device=dev)
+
+    def gstep():
+        for pr in layer_probs:  # the layers run one after another on one stream, so they share the scratch
+            mobi.mobi_linear_grouped(pr, ws=gws)
+    gstep()
+    mobi.mobi_sync_check()
+    gms = time_graph(gstep, steps)
+    mobi.mobi_sync_check()
     out = {"workload": "full model: 7 projections x 32 layers (Llama-2-7B shapes), batch 8, random router per "
                        "projection; pack all, then decode through every projection (224 mobi_linear calls, one "
                        "CUDA graph)",
            "params": params, "pack_ms": round(pack_ms, 3), "pack_GB/s": round(pack_bytes / pack_ms / 1e6, 1),
            "decode_ms_per_step": round(ms, 4), "decode_bytes_per_step": bytes_step,
            "decode_GB/s": round(bytes_step / ms / 1e6, 1), "decode_frac_of_hbm": round(bytes_step / ms / 1e6 / hbm_peak, 4),
-           "kmax_histogram": [kmax.count(v) for v in (1, 2, 3)], "steps": steps}
-    del graph, calls, packed, layers
+           "kmax_histogram": [kmax.count(v) for v in (1, 2, 3)], "steps": steps,
+           "grouped_per_layer": {"calls_per_step": len(layer_probs), "decode_ms_per_step": round(gms, 4),
+                                 "decode_GB/s": round(bytes_step / gms / 1e6, 1),
+                                 "decode_frac_of_hbm": round(bytes_step / gms / 1e6 / hbm_peak, 4)}}
+    del calls, packed, layers, layer_probs
     torch.cuda.empty_cache()
     return out
 
@@ -356,6 +435,73 @@ def time_prefill(mobi, L, dev, reps, tf_peak, flush):
             "reps": reps, "l2": "256 MB flush before each repetition"}
 
 
+# fp32 FMA peak of the SIMT pipes: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz
+# (the maximum SM clock), the bound of the MLP scorer's hidden layer at prefill.
+FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def time_route_mlp(mobi, wl, dev, hbm_peak, flush, reps=20):
+    """Threshold routing with the MLP scorer (hidden layer, scores, bucketing),
+    K=4096, H=128, S=3, at decode (T=16: bound by the W1 read) and prefill
+    (T=2048: bound by the fp32 FMAs of the hidden layer). CUDA events around
+    each call with the L2 flushed before it; the linear router of the same
+    tokens is timed the same way for comparison."""
+    out = {}
+    for R in (wl.mlp_route_decode(16), wl.mlp_route_prefill()):
+        T, K, H = R.T, R.K, R.H
+        X = R.X.to(dev)
+        W1, b1 = torch.from_numpy(R.W1).to(dev), torch.from_numpy(R.b1).to(dev)
+        W2, b2 = torch.from_numpy(R.W2).to(dev), torch.from_numpy(R.b2).to(dev)
+        k_t = torch.empty(T, dtype=torch.int32, device=dev)
+        perm = torch.empty(T, dtype=torch.int32, device=dev)
+        off = torch.empty(4, dtype=torch.int32, device=dev)
+        ws = torch.empty(max(mobi.mobi_route_mlp_workspace_bytes(T, K, H), 16), dtype=torch.uint8, device=dev)
+        Wr = torch.from_numpy(wl.draw_router(np.random.default_rng(1), K, 3)).to(dev)
+        ws_r = torch.empty(max(mobi.mobi_route_workspace_bytes(T, K, 3), 16), dtype=torch.uint8, device=dev)
+
+        def mlp():
+            mobi.mobi_route_mlp(X, W1, b1, W2, b2, 1.0, 0.5, k_t=k_t, perm=perm, offsets=off, ws=ws)
+
+        def lin():
+            mobi.mobi_route(X, Wr, None, k_t, perm, off, ws_r)
+        times = {}
+        for name, fn in (("mlp", mlp), ("linear", lin)):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(reps):
+                flush.sum()  # a read sweep: evicts the inputs without leaving dirty lines to write back
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            times[name] = statistics.median(ts)
+        mlp()
+        mobi.mobi_sync_check()
+        counts = torch.bincount(k_t, minlength=4)[1:].tolist()
+        ms = times["mlp"]
+        nbytes = T * K * 2 + K * H * 4 + H * 2 * 4 + T * 4 * 3
+        flops = 2.0 * T * K * H + 2.0 * T * H * 2
+        r = {"T": T, "K": K, "H": H, "S": 3, "tau": 1.0, "delta": 0.5, "k_counts": counts,
+             "us_per_call": round(1e3 * ms, 2), "linear_router_us_per_call": round(1e3 * times["linear"], 2),
+             "algorithmic_bytes": nbytes, "flops": flops}
+        if T <= 16:
+            r["roofline"] = {"bound": "hbm", "achieved": round(nbytes / ms / 1e6, 1), "peak": hbm_peak, "unit": "GB/s",
+                             "frac": round(nbytes / ms / 1e6 / hbm_peak, 4), "traffic": None}
+        else:
+            tf = flops / ms / 1e9
+            r["roofline"] = {"bound": "alu", "achieved": round(tf, 2), "peak": round(FP32_SIMT_PEAK_TFLOPS, 1),
+                             "unit": "TFLOP/s", "peak_kind": "fp32 FMA: 148 SMs x 128 lanes x 2 x 1965 MHz",
+                             "frac": round(tf / FP32_SIMT_PEAK_TFLOPS, 4), "traffic": None}
+        out[R.name] = r
+        del ws, ws_r
+    out["timing"] = f"median of {reps} calls, CUDA events, L2 flushed (256 MB read) before each"
+    return out
+
+
 def run_gpu(args, world, rank):
     import token_adaptive_mixed_b200 as mobi
     from token_adaptive_mixed_b200 import build as mobi_build
@@ -368,6 +514,8 @@ def run_gpu(args, world, rank):
     dev = torch.device("cuda", torch.cuda.current_device())
     hbm_peak, tf_peak, tf_sust, peak_kind = peaks()
 
+    if args.only == "route_mlp":
+        return {"route_mlp": time_route_mlp(mobi, wl, dev, hbm_peak, l2_flush_buffer(dev))}
     if args.only == "prefill":
         flush = l2_flush_buffer(dev)
         out = {"prefill": time_prefill(mobi, wl.prefill(), dev, args.prefill_reps, tf_peak, flush)}
@@ -435,6 +583,8 @@ def run_gpu(args, world, rank):
     gemm_ms = sum(per_case_ms)
     achieved = bytes_step / (gemm_ms * 1e-3) / 1e9
 
+    grouped = time_decode_grouped(mobi, cases, bytes_step, min(args.steps, 500), hbm_peak)
+
     # End to end through the public API with host buffers (pinned), copies inside:
     # the step's nine activation matrices live in one pinned host buffer and one
     # device buffer (one host-to-device copy), the nine outputs likewise (one
@@ -487,6 +637,7 @@ def run_gpu(args, world, rank):
                 "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
+        "decode_grouped": grouped,
     }
     if rank == 0:
         out["pack"] = time_pack(mobi, wl, dev)
@@ -500,6 +651,8 @@ def run_gpu(args, world, rank):
         out["prefill"] = time_prefill(mobi, wl.prefill(), dev, args.prefill_reps, tf_peak, flush)
         if not args.skip_skewed:
             out["skewed_prefill"] = time_prefill(mobi, wl.skewed_prefill(), dev, args.prefill_reps, tf_peak, flush)
+    if args.only == "all" and rank == 0:
+        out["route_mlp"] = time_route_mlp(mobi, wl, dev, hbm_peak, l2_flush_buffer(dev))
     return out
 
 
@@ -591,7 +744,7 @@ def main():
     ap.add_argument("--impl", default="mobi", choices=["mobi", "reference"])
     ap.add_argument("--cpu-baseline-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill"],
+    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill", "route_mlp"],
                     help="run a subset (profiling); the default runs everything")
     ap.add_argument("--prefill-reps", type=int, default=10)
     ap.add_argument("--skip-skewed", action="store_true")

@@ -246,6 +246,51 @@ MOBI_API mobi_status mobi_linear(const void* X, int64_t T, int64_t K, const floa
                                  int32_t* offsets, float* Y, void* ws, size_t ws_bytes,
                                  void* stream);
 
+/* One problem of mobi_linear_grouped: the arguments of one mobi_linear call. */
+typedef struct mobi_linear_problem {
+  const void* X;          /* bf16 [T][K] */
+  const float* Wr;        /* fp32 [K][S] */
+  const float* bias;      /* fp32 [S], or NULL for zeros */
+  const uint32_t* codes;  /* as produced by mobi_pack for N, K */
+  const uint32_t* sz;
+  float* Y;               /* out, fp32 [T][N] */
+  int32_t* k_t;           /* out, int32 [T] */
+  int32_t* perm;          /* out, int32 [T] */
+  int32_t* offsets;       /* out, int32 [S+1] */
+  int64_t T, N, K;
+} mobi_linear_problem;
+
+/* Largest problem count of one mobi_linear_grouped call. */
+#define MOBI_MAX_GROUP 8
+
+/* Scratch bytes of mobi_linear_grouped for these problems (0 for invalid
+ * arguments or when none is needed). */
+MOBI_API size_t mobi_linear_grouped_workspace_bytes(const mobi_linear_problem* problems, int count,
+                                                    int S);
+
+/*
+ * mobi_linear_grouped — up to MOBI_MAX_GROUP independent decode-sized
+ *   mobi_linear problems (every T <= 16) in one step: the projections of a
+ *   layer that read their weights in the same decode step ([en] §3: only the
+ *   slices needed are fetched, so the step is bound by weight bytes; the
+ *   explainer pages' deployment discussion of one model serving many
+ *   precisions). Each problem's results are exactly those of mobi_linear on
+ *   it alone (same kernels, same summation order).
+ *   problems  host array of `count` descriptors (1..MOBI_MAX_GROUP); the
+ *             library reads it during the call only.
+ *   G, S      group size (128) and slice count, shared by all problems.
+ *   ws        scratch of mobi_linear_grouped_workspace_bytes bytes.
+ * Launches: one routing launch (an 8-CTA cluster per problem), one decode
+ * launch per fragment class present (T <= 8 and 9..16 tokens; the SMs are
+ * shared among that class's problems in proportion to their weight counts),
+ * and one chunk-reduction launch, so per-launch ramp-up and drain are paid
+ * once per step instead of once per problem. Outputs must not overlap any
+ * problem's inputs or each other. Errors as for mobi_linear, checked for every
+ * problem before anything is launched; T > 16 gives MOBI_ERR_UNSUPPORTED_SHAPE.
+ */
+MOBI_API mobi_status mobi_linear_grouped(const mobi_linear_problem* problems, int count, int G,
+                                         int S, void* ws, size_t ws_bytes, void* stream);
+
 /*
  * mobi_gemm_decode_noalloc — the decode GEMM (T <= 16) without a workspace.
  *   Not part of the method: the MoBiQuant pages have no counterpart of this

@@ -151,3 +151,31 @@ def test_route_mlp_validation(L):
         assert b <= max(K // 64, 1) * T * H * 4 + 255  # at most one split per 64 rows of K
     assert mobi.mobi_route_mlp_workspace_bytes(0, 4096, 128) == 0
     assert mobi.mobi_route_mlp_workspace_bytes(16, 4096, 0) == 0
+
+
+def test_linear_grouped_validation(L):
+    P = mobi.LinearProblem
+
+    def prob(T=8, N=4096, K=4096, X=FAKE, Y=FAKE, codes=FAKE):
+        return P(X, FAKE, None, codes, FAKE, Y, FAKE, FAKE, FAKE, T, N, K)
+
+    def call(probs, S=3, G=128, ws=FAKE, wsb=1 << 30):
+        arr = (P * max(len(probs), 1))(*probs)
+        return L.mobi_linear_grouped(arr if probs else None, len(probs), G, S, ws, wsb, None)
+    assert call([]) == 1
+    assert call([prob()] * 9) == 1                  # more than MOBI_MAX_GROUP
+    assert call([prob(), prob(T=17)]) == 2          # decode-sized problems only
+    assert call([prob(), prob(K=200)]) == 2
+    assert call([prob(), prob(N=24)]) == 2
+    assert call([prob()], G=64) == 2
+    assert call([prob()], S=4) == 1
+    assert call([prob(), prob(X=None)]) == 1
+    assert call([prob(), prob(codes=None)]) == 1
+    assert call([prob(), prob(Y=FAKE + 4)]) == 3
+    assert call([prob()], ws=FAKE + 8) == 3
+    assert call([prob()], wsb=16) == 4
+    arr = (P * 2)(prob(T=4, N=4096, K=4096), prob(T=16, N=11008, K=4096))
+    need = L.mobi_linear_grouped_workspace_bytes(arr, 2, 3)
+    per = [L.mobi_linear_grouped_workspace_bytes((P * 1)(arr[i]), 1, 3) for i in range(2)]
+    assert need == sum(per) and all(b % 256 == 0 and b > 0 for b in per)
+    assert L.mobi_linear_grouped_workspace_bytes(arr, 2, 4) == 0

@@ -13,6 +13,7 @@ Entry points (same names as the C ABI):
   mobi_gemm(X, k_t, perm, offsets, codes, sz, N)         -> Y  (fp32)
   mobi_gemm_path(..., path)         the same with a forced kernel
   mobi_linear(X, Wr, bias, codes, sz, N)  route + GEMM in one call -> (Y, k_t, perm, offsets)
+  mobi_linear_grouped(problems)     up to 8 decode-sized mobi_linear problems in one step
   mobi_sync_check()                 sync + device-side error word
 """
 from __future__ import annotations
@@ -26,7 +27,8 @@ __all__ = [
     "MobiError", "lib", "mobi_version", "mobi_status_string", "mobi_codes_bytes", "mobi_sz_bytes",
     "mobi_route_workspace_bytes", "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm", "mobi_last_error",
     "mobi_gemm_path", "mobi_sync_check", "mobi_debug_set_wait_limit", "mobi_gemm_decode_noalloc", "mobi_linear",
-    "mobi_linear_workspace_bytes", "mobi_route_mlp", "mobi_route_mlp_workspace_bytes", "PATH_AUTO",
+    "mobi_linear_workspace_bytes", "mobi_route_mlp", "mobi_route_mlp_workspace_bytes", "mobi_linear_grouped",
+    "mobi_linear_grouped_workspace_bytes", "MAX_GROUP", "PATH_AUTO",
     "PATH_DECODE",
     "PATH_PREFILL", "EXPORTED_SYMBOLS",
 ]
@@ -35,6 +37,15 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("MOBI_LIB", os.path.join(_HERE, "libmobi.so"))
 
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
+MAX_GROUP = 8  # MOBI_MAX_GROUP
+
+
+class LinearProblem(ctypes.Structure):
+    """mobi_linear_problem (include/mobi.h): pointers and sizes of one problem."""
+    _fields_ = [("X", ctypes.c_void_p), ("Wr", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+                ("codes", ctypes.c_void_p), ("sz", ctypes.c_void_p), ("Y", ctypes.c_void_p),
+                ("k_t", ctypes.c_void_p), ("perm", ctypes.c_void_p), ("offsets", ctypes.c_void_p),
+                ("T", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
 STATUS_NAMES = ["MOBI_OK", "MOBI_ERR_INVALID_ARG", "MOBI_ERR_UNSUPPORTED_SHAPE", "MOBI_ERR_MISALIGNED",
                 "MOBI_ERR_WORKSPACE", "MOBI_ERR_CUDA", "MOBI_ERR_TIMEOUT"]
 
@@ -43,7 +54,7 @@ EXPORTED_SYMBOLS = (
     "mobi_status_string", "mobi_last_error", "mobi_version", "mobi_codes_bytes", "mobi_sz_bytes", "mobi_route_workspace_bytes",
     "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm", "mobi_gemm_path", "mobi_sync_check",
     "mobi_debug_set_wait_limit", "mobi_gemm_decode_noalloc", "mobi_linear", "mobi_linear_workspace_bytes",
-    "mobi_route_mlp", "mobi_route_mlp_workspace_bytes",
+    "mobi_route_mlp", "mobi_route_mlp_workspace_bytes", "mobi_linear_grouped", "mobi_linear_grouped_workspace_bytes",
 )
 
 
@@ -99,6 +110,10 @@ def lib() -> ctypes.CDLL:
         L.mobi_route_mlp.argtypes = [p, i64, i64, p, p, i64, p, p, ci, ctypes.c_double, ctypes.c_double, p, p, p,
                                      p, sz_t, p]
         L.mobi_route_mlp.restype = ci
+        L.mobi_linear_grouped_workspace_bytes.argtypes = [p, ci, ci]
+        L.mobi_linear_grouped_workspace_bytes.restype = sz_t
+        L.mobi_linear_grouped.argtypes = [p, ci, ci, ci, p, sz_t, p]
+        L.mobi_linear_grouped.restype = ci
         L.mobi_sync_check.argtypes = [p]
         L.mobi_sync_check.restype = ci
         L.mobi_debug_set_wait_limit.argtypes = [i64]
@@ -220,6 +235,51 @@ def mobi_route_mlp(X: torch.Tensor, W1: torch.Tensor, b1: torch.Tensor | None, W
                                                   float(tau), float(delta), _ptr(k_t), _ptr(perm), _ptr(offsets),
                                                   _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
     return k_t, perm, offsets
+
+
+def _problem_array(problems, S: int):
+    """problems: sequence of dicts with X, Wr, codes, sz, N and optionally bias, Y, k_t, perm,
+    offsets (allocated here when absent). Returns the ctypes array and the filled dicts."""
+    arr = (LinearProblem * len(problems))()
+    filled = []
+    for i, pr in enumerate(problems):
+        X = pr["X"]
+        T, K = X.shape
+        N = pr["N"]
+        dev = X.device
+        d = dict(pr)
+        d.setdefault("bias", None)
+        if d.get("Y") is None:
+            d["Y"] = torch.empty((T, N), dtype=torch.float32, device=dev)
+        if d.get("k_t") is None:
+            d["k_t"] = torch.empty(T, dtype=torch.int32, device=dev)
+        if d.get("perm") is None:
+            d["perm"] = torch.empty(T, dtype=torch.int32, device=dev)
+        if d.get("offsets") is None:
+            d["offsets"] = torch.empty(S + 1, dtype=torch.int32, device=dev)
+        arr[i] = LinearProblem(_ptr(X), _ptr(d["Wr"]), _ptr(d["bias"]), _ptr(d["codes"]), _ptr(d["sz"]),
+                               _ptr(d["Y"]), _ptr(d["k_t"]), _ptr(d["perm"]), _ptr(d["offsets"]), T, N, K)
+        filled.append(d)
+    return arr, filled
+
+
+def mobi_linear_grouped_workspace_bytes(problems, S: int = 3) -> int:
+    arr, _ = _problem_array(problems, S)
+    return lib().mobi_linear_grouped_workspace_bytes(arr, len(problems), S)
+
+
+def mobi_linear_grouped(problems, S: int = 3, G: int = 128, ws: torch.Tensor | None = None, stream=None):
+    """Up to MAX_GROUP independent decode-sized (T <= 16) mobi_linear problems in one step.
+    Each problem is a dict with X, Wr, codes, sz, N (and optionally bias, Y, k_t, perm, offsets).
+    Returns [(Y, k_t, perm, offsets)] in problem order."""
+    arr, filled = _problem_array(problems, S)
+    if len(filled) == 0:
+        raise ValueError("mobi_linear_grouped needs at least one problem")
+    need = lib().mobi_linear_grouped_workspace_bytes(arr, len(filled), S)
+    ws = _workspace(need, filled[0]["X"].device, ws) if need > 0 else ws
+    _check("mobi_linear_grouped", lib().mobi_linear_grouped(arr, len(filled), G, S, _ptr(ws),
+                                                            0 if ws is None else ws.numel(), _stream(stream)))
+    return [(d["Y"], d["k_t"], d["perm"], d["offsets"]) for d in filled]
 
 
 def mobi_gemm_path(X: torch.Tensor, k_t: torch.Tensor, perm: torch.Tensor, offsets: torch.Tensor,

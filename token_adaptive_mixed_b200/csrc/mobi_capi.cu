@@ -382,6 +382,69 @@ mobi_status mobi_linear(const void* X, int64_t T, int64_t K, const float* Wr, co
   return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, gws, s, dst));
 }
 
+static_assert(MOBI_MAX_GROUP == kMaxGroup, "group size of the header and the kernels");
+
+static mobi_status check_grouped(const mobi_linear_problem* problems, int count, int G, int S, size_t* need) {
+  *need = 0;
+  if (!problems || count < 1 || count > MOBI_MAX_GROUP) return MOBI_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    const mobi_linear_problem& p = problems[i];
+    mobi_status st = check_matrix(p.N, p.K, G, S);
+    if (st != MOBI_OK) return st;
+    if (p.T < 0) return MOBI_ERR_INVALID_ARG;
+    if (p.T > 16) return MOBI_ERR_UNSUPPORTED_SHAPE;
+    if (!p.offsets || (p.T > 0 && (!p.X || !p.Wr || !p.k_t || !p.perm))) return MOBI_ERR_INVALID_ARG;
+    if (p.T > 0 && p.K == 0) return MOBI_ERR_UNSUPPORTED_SHAPE;
+    if (p.T > 0 && p.N > 0 && (!p.codes || !p.sz || !p.Y)) return MOBI_ERR_INVALID_ARG;
+    if ((p.X && !aligned16(p.X)) || (p.Wr && !aligned16(p.Wr)) || (p.bias && !aligned4(p.bias)) ||
+        (p.k_t && !aligned4(p.k_t)) || (p.perm && !aligned4(p.perm)) || !aligned4(p.offsets) ||
+        (p.codes && !aligned16(p.codes)) || (p.sz && !aligned16(p.sz)) || (p.Y && !aligned16(p.Y)))
+      return MOBI_ERR_MISALIGNED;
+    if (p.T > 0 && p.N > 0) *need += align256(decode_ws_bytes(p.N, p.K));
+  }
+  return MOBI_OK;
+}
+
+size_t mobi_linear_grouped_workspace_bytes(const mobi_linear_problem* problems, int count, int S) {
+  size_t need = 0;
+  if (check_grouped(problems, count, 128, S, &need) != MOBI_OK) return 0;
+  return need;
+}
+
+mobi_status mobi_linear_grouped(const mobi_linear_problem* problems, int count, int G, int S, void* ws,
+                                size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  size_t need = 0;
+  mobi_status st = check_grouped(problems, count, G, S, &need);
+  if (st != MOBI_OK) return st;
+  if (ws && !aligned16(ws)) return MOBI_ERR_MISALIGNED;
+  if (need > 0 && (!ws || ws_bytes < need)) return MOBI_ERR_WORKSPACE;
+  cudaError_t e;
+  DeviceStatus* dst = device_status(&e);
+  if (!dst) return cuda_status(e);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  RouteSmallGroup rg = {};
+  rg.G = count;
+  DecodeJob jobs[MOBI_MAX_GROUP];
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  for (int i = 0; i < count; ++i) {
+    const mobi_linear_problem& p = problems[i];
+    rg.p[i] = RouteSmallProblem{static_cast<const __nv_bfloat16*>(p.X), p.Wr, p.bias, p.k_t, p.perm, p.offsets, p.K,
+                                (int)p.T};
+    jobs[i] = DecodeJob{p.X, p.k_t, p.codes, p.sz, p.Y, nullptr, p.N, p.K, (int)p.T};
+    if (p.T > 0 && p.N > 0) {
+      jobs[i].partial = reinterpret_cast<float*>(w);
+      w += align256(decode_ws_bytes(p.N, p.K));
+    }
+  }
+  e = launch_route_small_grouped(rg, S, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  // As in mobi_linear: the kernel just launched is the routing kernel, which
+  // writes only k_t, perm and offsets, so the decode kernels may fetch X and
+  // the weights before they wait on it.
+  return cuda_status(launch_decode_grouped(jobs, count, S, s, dst, true));
+}
+
 mobi_status mobi_gemm(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
                       const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S,
                       float* Y, void* ws, size_t ws_bytes, void* stream) {

@@ -32,6 +32,7 @@
 // programmatically dependent kernel that adds the per-chunk partials in chunk
 // order (deterministic).
 #include <cstdint>
+#include <cstring>
 #include <cstdio>
 #include <mutex>
 
@@ -216,15 +217,31 @@ __device__ __forceinline__ bool dec_wait(uint64_t* bar, uint32_t parity, uint64_
   return false;
 }
 
-// grid = (CTAs per chunk, chunks). out = Y when there is one chunk, else the
-// per-chunk partials [chunk][T][N]. All loop bookkeeping is incremental
-// 32-bit arithmetic (sizes are validated to N, K < 2^28).
-// Warps 0 .. kWarps-1 consume (teams of four), warp kWarps issues the copies.
-template <int NB>
+// A group of independent problems in one launch: problem i owns the CTAs
+// [cta0, cta0 + cpc * nch) of the 1-D grid, cpc CTAs per K chunk. out = Y when
+// the problem has one chunk, else its per-chunk partials [chunk][T][N].
+struct DecProblem {
+  const __nv_bfloat16* X;
+  const int32_t* k_t;
+  float* out;
+  int T, N, K, ngroups, nblocks, cpc, cta0;
+};
+// MG = table capacity: 1 for a single call (a small parameter block to copy
+// per launch), kMaxGroup for a group.
+template <int MG>
+struct DecGroup {
+  CUtensorMap tm_codes[MG];
+  CUtensorMap tm_sz[MG];
+  DecProblem p[MG];
+  int G, S;
+};
+
+// All loop bookkeeping is incremental 32-bit arithmetic (sizes are validated
+// to N, K < 2^28). Warps 0 .. kWarps-1 consume (teams of four), warp kWarps
+// issues the copies.
+template <int NB, int MG>
 __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLayout<NB>::kMaxRegs) decode_kernel(
-    const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_sz,
-    const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ k_t, int T, int N, int K, int ngroups, int S,
-    int nblocks, float* __restrict__ out, DeviceStatus* st, uint64_t limit, int early) {
+    const __grid_constant__ DecGroup<MG> grp, DeviceStatus* st, uint64_t limit, int early) {
   using L = DecLayout<NB>;
   constexpr int kTeams = DecCfg<NB>::kTeams;
   constexpr int kW = L::kWarps;
@@ -237,11 +254,23 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLay
   asm volatile("griddepcontrol.launch_dependents;");
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int ch = blockIdx.y;
+  int pi = 0;  // this CTA's problem
+#pragma unroll 1
+  for (int i = 1; i < (MG > 1 ? grp.G : 1); ++i)
+    if ((int)blockIdx.x >= grp.p[i].cta0) pi = i;
+  const DecProblem& prob = grp.p[pi];
+  const CUtensorMap* tm_codes = &grp.tm_codes[pi];
+  const CUtensorMap* tm_sz = &grp.tm_sz[pi];
+  const __nv_bfloat16* __restrict__ X = prob.X;
+  const int32_t* __restrict__ k_t = prob.k_t;
+  float* __restrict__ out = prob.out;
+  const int T = prob.T, N = prob.N, K = prob.K, ngroups = prob.ngroups, nblocks = prob.nblocks, S = grp.S;
+  const int local = (int)blockIdx.x - prob.cta0, cpc = prob.cpc;
+  const int ch = local / cpc, cx = local - ch * cpc;
   // This CTA's 32-row blocks [b_begin, b_end); team t takes every kTeams-th
   // of them, starting with block b_begin + t.
-  const int b_begin = (int)((int64_t)blockIdx.x * nblocks / gridDim.x);
-  const int b_end = (int)((int64_t)(blockIdx.x + 1) * nblocks / gridDim.x);
+  const int b_begin = (int)((int64_t)cx * nblocks / cpc);
+  const int b_end = (int)((int64_t)(cx + 1) * nblocks / cpc);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::kBar);  // [team][slot]
   uint64_t* empty = full + kTeams * D;
   uint64_t* ready = reinterpret_cast<uint64_t*>(sm + L::kReady);
@@ -271,8 +300,8 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLay
     // issue their copies together, so one poll serves every team.
     named_bar_sync(15, 32 * (kW + 1));  // the consumers' activation loads go out first
     if (lane == 0) {
-      prefetch_tmap(&tm_codes);
-      prefetch_tmap(&tm_sz);
+      prefetch_tmap(tm_codes);
+      prefetch_tmap(tm_sz);
     }
     const uint64_t policy = l2_evict_first_policy();
     const int w = lane, team = lane;
@@ -280,7 +309,7 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLay
     int r = 0, bo = 0, s = 0;  // next stage of team w: its index, block offset and slice
     // Slice 0 of the team's first block does not depend on k_t.
     if (early && myb > 0) {
-      dec_issue(&tm_codes, &tm_sz, sm + L::kSlots + (uint32_t)(w * D) * kDecSlot, &full[w * D], b_begin + team, 0, N,
+      dec_issue(tm_codes, tm_sz, sm + L::kSlots + (uint32_t)(w * D) * kDecSlot, &full[w * D], b_begin + team, 0, N,
                 ngroups, ch, policy);
       r = 1;
     }
@@ -300,7 +329,7 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLay
       if (ok && r < nit && (r < 2 || gate)) {
         const int slot = r % D;
         if (r < D || mbar_test_wait(&empty[w * D + slot], (uint32_t)(((r / D) & 1) ^ 1))) {
-          dec_issue(&tm_codes, &tm_sz, sm + L::kSlots + (uint32_t)(w * D + slot) * kDecSlot, &full[w * D + slot],
+          dec_issue(tm_codes, tm_sz, sm + L::kSlots + (uint32_t)(w * D + slot) * kDecSlot, &full[w * D + slot],
                     b_begin + team + bo * kTeams, s, N, ngroups, ch, policy);
           ++r;
           if (++s == kmax) { s = 0; ++bo; }
@@ -531,13 +560,32 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLay
   __syncthreads();
 }
 
-// Y[t][n] = sum over chunks c (in order) of partial[c][t][n]; n4 = T*N/4.
+// Y[t][n] = sum over chunks c (in order) of partial[c][t][n], for every problem
+// of a group with more than one chunk; problem i covers the float4 indices
+// [off[i], off[i + 1]) of the grid-stride range, n4 = T*N/4 of them.
 // Up to 8 chunk loads are in flight at a time; the adds keep chunk order.
-__global__ void __launch_bounds__(256) decode_reduce_kernel(const float4* __restrict__ partial, int64_t n4, int nch,
-                                                            float4* __restrict__ Y) {
+struct DecReduceGroup {
+  const float4* partial[kMaxGroup];
+  float4* Y[kMaxGroup];
+  int64_t off[kMaxGroup + 1];
+  int nch[kMaxGroup];
+  int G;
+};
+
+__global__ void __launch_bounds__(256) decode_reduce_kernel(const __grid_constant__ DecReduceGroup grp) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;");
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+  const int64_t total = grp.off[grp.G];
+  for (int64_t gi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; gi < total;
+       gi += (int64_t)gridDim.x * blockDim.x) {
+    int pi = 0;
+#pragma unroll 1
+    for (int j = 1; j < grp.G; ++j)
+      if (gi >= grp.off[j]) pi = j;
+    const int64_t i = gi - grp.off[pi], n4 = grp.off[pi + 1] - grp.off[pi];
+    const int nch = grp.nch[pi];
+    const float4* __restrict__ partial = grp.partial[pi];
+    float4* __restrict__ Y = grp.Y[pi];
     float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     for (int c0 = 0; c0 < nch; c0 += 8) {
       float4 b[8];
@@ -565,25 +613,14 @@ size_t decode_ws_bytes(int64_t N, int64_t K) {
   return ((size_t)nch * 16 * (size_t)N * sizeof(float) + 255) / 256 * 256;  // partials for up to 16 tokens
 }
 
-// Grid of the decode kernel: (CTAs per chunk, chunks), one CTA per SM.
-void decode_grid(int64_t N, int64_t K, int sms, int64_t* cpc, int64_t* nch) {
-  *nch = dec_chunks(K);
-  const int64_t nblocks = (N + kDecRows - 1) / kDecRows;
-  int64_t c = sms / *nch;
-  if (c < 1) c = 1;
-  if (c > nblocks) c = nblocks;
-  *cpc = c;
-}
-
-template <int NB>
-static cudaError_t launch_decode_nb(const CUtensorMap& tm_codes, const CUtensorMap& tm_sz, const void* X, int T,
-                                    int64_t K, const int32_t* k_t, int64_t N, int S, float* out, int64_t cpc,
-                                    int64_t nch, cudaStream_t stream, DeviceStatus* st, bool early) {
+template <int NB, int MG>
+static cudaError_t launch_decode_class(const DecGroup<MG>& grp, int ctas, cudaStream_t stream, DeviceStatus* st,
+                                       bool early) {
   using L = DecLayout<NB>;
-  cudaError_t e = set_smem((const void*)decode_kernel<NB>, (int)L::kDynamic);
+  cudaError_t e = set_smem((const void*)decode_kernel<NB, MG>, (int)L::kDynamic);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)cpc, (unsigned)nch);
+  cfg.gridDim = dim3((unsigned)ctas);
   cfg.blockDim = dim3(L::kThreads);
   cfg.dynamicSmemBytes = L::kDynamic;
   cfg.stream = stream;
@@ -592,37 +629,86 @@ static cudaError_t launch_decode_nb(const CUtensorMap& tm_codes, const CUtensorM
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, decode_kernel<NB>, tm_codes, tm_sz, static_cast<const __nv_bfloat16*>(X), k_t, T,
-                         (int)N, (int)K, (int)(K / 128), S, (int)((N + kDecRows - 1) / kDecRows), out, st,
-                         wait_limit(), early ? 1 : 0);
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<NB, MG>, grp, st, wait_limit(), early ? 1 : 0);
   if (e != cudaSuccess) return note_error("decode launch", e);
   return note_error("kernel launch", cudaGetLastError());
 }
 
-cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
-                          const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
-                          DeviceStatus* st, bool early) {
-  const int64_t ngroups = K / 128;
-  int64_t cpc, nch;
-  decode_grid(N, K, num_sms(), &cpc, &nch);
-  float* partial = static_cast<float*>(ws);
-  float* out = nch > 1 ? partial : Y;
+// One launch per fragment class present (T <= 8, then 9 <= T <= 16), each a
+// persistent grid of about one CTA per SM shared among that class's problems
+// in proportion to their weight counts N K (at least one CTA per K chunk, at
+// most one per 32-row block), then one chunk-reduction launch for every
+// problem with more than one chunk. Each launch is a programmatic dependent of
+// the one before; `early` as for the kernel (the launches that follow the
+// first class write none of the next class's inputs).
+// Fills a table of capacity MG with the problems `idx[0..n)` of one fragment
+// class and launches it; problems with several chunks are appended to `red`.
+template <int MG>
+static cudaError_t decode_class(const DecodeJob* jobs, const int* idx, int n, int cls, int S, int sms,
+                                DecReduceGroup* red, cudaStream_t stream, DeviceStatus* st, bool early) {
+  double wsum = 0.0;
+  for (int m = 0; m < n; ++m) wsum += (double)jobs[idx[m]].N * (double)jobs[idx[m]].K;
+  DecGroup<MG> grp;
+  memset(&grp, 0, sizeof grp);
+  grp.G = n;
+  grp.S = S;
+  int ctas = 0;
+  for (int m = 0; m < n; ++m) {
+    const DecodeJob& j = jobs[idx[m]];
+    const int64_t nch = dec_chunks(j.K), nblocks = (j.N + kDecRows - 1) / kDecRows;
+    int64_t cpc = (int64_t)((double)sms * ((double)j.N * (double)j.K / wsum) / (double)nch);
+    if (cpc > nblocks) cpc = nblocks;
+    if (cpc < 1) cpc = 1;
+    if (!make_tmap_2d(&grp.tm_codes[m], j.codes, 4, (uint64_t)(j.K / 16), (uint64_t)(S * j.N),
+                      (uint64_t)(j.K / 16) * 4, 32, kDecRows, 128))
+      return note_error("decode tensor map (codes)", cudaErrorInvalidValue);
+    if (!make_tmap_2d(&grp.tm_sz[m], j.sz, 4, (uint64_t)j.N, (uint64_t)(S * (j.K / 128)), (uint64_t)j.N * 4,
+                      kDecRows, kDecChunk, 0))
+      return note_error("decode tensor map (scale/zero)", cudaErrorInvalidValue);
+    grp.p[m] = DecProblem{static_cast<const __nv_bfloat16*>(j.X), j.k_t, nch > 1 ? j.partial : j.Y, j.T, (int)j.N,
+                          (int)j.K, (int)(j.K / 128), (int)nblocks, (int)cpc, ctas};
+    ctas += (int)(cpc * nch);
+    if (nch > 1) {
+      red->partial[red->G] = reinterpret_cast<const float4*>(j.partial);
+      red->Y[red->G] = reinterpret_cast<float4*>(j.Y);
+      red->nch[red->G] = (int)nch;
+      red->off[red->G + 1] = red->off[red->G] + (int64_t)j.T * j.N / 4;
+      ++red->G;
+    }
+  }
+  return cls == 1 ? launch_decode_class<1, MG>(grp, ctas, stream, st, early)
+                  : launch_decode_class<2, MG>(grp, ctas, stream, st, early);
+}
 
-  CUtensorMap tm_codes, tm_sz;
-  if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4, 32,
-                    kDecRows, 128))
-    return note_error("decode tensor map (codes)", cudaErrorInvalidValue);
-  if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, kDecRows, kDecChunk, 0))
-    return note_error("decode tensor map (scale/zero)", cudaErrorInvalidValue);
-
-  cudaError_t e = T > 8 ? launch_decode_nb<2>(tm_codes, tm_sz, X, T, K, k_t, N, S, out, cpc, nch, stream, st, early)
-                        : launch_decode_nb<1>(tm_codes, tm_sz, X, T, K, k_t, N, S, out, cpc, nch, stream, st, early);
-  if (e != cudaSuccess || nch <= 1) return e;
+// One launch per fragment class present (T <= 8, then 9 <= T <= 16), each a
+// persistent grid of about one CTA per SM shared among that class's problems
+// in proportion to their weight counts N K (at least one CTA per K chunk, at
+// most one per 32-row block), then one chunk-reduction launch for every
+// problem with more than one chunk. Each launch is a programmatic dependent of
+// the one before; `early` as for the kernel (the launches that follow the
+// first class write none of the next class's inputs).
+cudaError_t launch_decode_grouped(const DecodeJob* jobs, int G, int S, cudaStream_t stream, DeviceStatus* st,
+                                  bool early) {
+  const int sms = num_sms();
+  DecReduceGroup red = {};
+  red.off[0] = 0;
+  for (int cls = 1; cls <= 2; ++cls) {
+    int idx[kMaxGroup];
+    int n = 0;
+    for (int i = 0; i < G; ++i) {
+      const DecodeJob& j = jobs[i];
+      if (j.T > 0 && j.N > 0 && (j.T > 8 ? 2 : 1) == cls) idx[n++] = i;
+    }
+    if (n == 0) continue;
+    const cudaError_t e = n == 1 ? decode_class<1>(jobs, idx, n, cls, S, sms, &red, stream, st, early)
+                                 : decode_class<kMaxGroup>(jobs, idx, n, cls, S, sms, &red, stream, st, early);
+    if (e != cudaSuccess) return e;
+  }
+  if (red.G == 0) return cudaSuccess;
 
   // Chunk reduction, launched as a programmatic dependent of the decode kernel.
-  const int64_t n4 = (int64_t)T * N / 4;
-  int64_t blocks = (n4 + 255) / 256;
-  const int64_t cap = (int64_t)num_sms() * 4;
+  int64_t blocks = (red.off[red.G] + 255) / 256;
+  const int64_t cap = (int64_t)sms * 4;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   cudaLaunchConfig_t cfg = {};
@@ -635,10 +721,16 @@ cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, decode_reduce_kernel, (const float4*)partial, n4, (int)nch,
-                         reinterpret_cast<float4*>(Y));
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_reduce_kernel, red);
   if (e != cudaSuccess) return note_error("decode reduce launch", e);
   return note_error("kernel launch", cudaGetLastError());
+}
+
+cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
+                          const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
+                          DeviceStatus* st, bool early) {
+  const DecodeJob job{X, k_t, codes, sz, Y, static_cast<float*>(ws), N, K, T};
+  return launch_decode_grouped(&job, 1, S, stream, st, early);
 }
 
 }  // namespace mobi

@@ -5,6 +5,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cuda_bf16.h>
+
 #include <cstdint>
 
 #include "mobi_device.cuh"
@@ -27,5 +29,46 @@ cudaError_t set_smem(const void* func, int bytes);
 // 32, 64 or 128 (the shared-memory swizzle span of the copied tile).
 bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t cols, uint64_t rows,
                   uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes);
+
+// ---- groups of independent small problems (one launch each step) -------------------
+//
+// Problem tables travel as __grid_constant__ kernel parameters, so a CUDA graph
+// captures them by value and no device memory holds them.
+constexpr int kMaxGroup = 8;
+
+struct RouteSmallProblem {
+  const __nv_bfloat16* X;
+  const float* Wr;
+  const float* bias;
+  int32_t* k_t;
+  int32_t* perm;
+  int32_t* offsets;
+  int64_t K;
+  int T;
+};
+template <int MG>
+struct RouteSmallGroupT {
+  RouteSmallProblem p[MG];
+  int G;
+};
+using RouteSmallGroup = RouteSmallGroupT<kMaxGroup>;
+cudaError_t launch_route_small_grouped(const RouteSmallGroup& grp, int S, cudaStream_t stream);
+
+// One decode problem (T <= 16): inputs, k_t, and the output Y.
+struct DecodeJob {
+  const void* X;
+  const int32_t* k_t;
+  const uint32_t* codes;
+  const uint32_t* sz;
+  float* Y;
+  float* partial;  // scratch of decode_ws_bytes(N, K) bytes
+  int64_t N, K;
+  int T;
+};
+size_t decode_ws_bytes(int64_t N, int64_t K);
+// Decode GEMMs of up to kMaxGroup problems: one launch per fragment class
+// (T <= 8, T <= 16) plus one chunk-reduction launch.
+cudaError_t launch_decode_grouped(const DecodeJob* jobs, int G, int S, cudaStream_t stream, DeviceStatus* st,
+                                  bool early);
 
 }  // namespace mobi

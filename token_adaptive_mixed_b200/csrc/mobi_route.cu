@@ -250,14 +250,21 @@ __device__ __forceinline__ void st_dsmem_f64(uint32_t addr, double v) {
   asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(addr), "d"(v) : "memory");
 }
 
-template <int S>
-__global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
-    const __nv_bfloat16* __restrict__ X, int T, int64_t K, const float* __restrict__ Wr,
-    const float* __restrict__ bias, int32_t* __restrict__ k_t, int32_t* __restrict__ perm,
-    int32_t* __restrict__ offsets) {
+// Cluster c of the grid routes problem c of the group (one call is a group of one).
+template <int S, int MG>
+__global__ void __launch_bounds__(kRouteThreads) route_small_kernel(const __grid_constant__ RouteSmallGroupT<MG> grp) {
   __shared__ float red[kRouteThreads / 32][kRouteSmallT * S];
   __shared__ double part[kRouteCluster][kRouteSmallT * S];  // used in CTA 0: [rank][token * S + j]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const RouteSmallProblem& prob = grp.p[MG > 1 ? blockIdx.x / kRouteCluster : 0];
+  const __nv_bfloat16* __restrict__ X = prob.X;
+  const float* __restrict__ Wr = prob.Wr;
+  const float* __restrict__ bias = prob.bias;
+  int32_t* __restrict__ k_t = prob.k_t;
+  int32_t* __restrict__ perm = prob.perm;
+  int32_t* __restrict__ offsets = prob.offsets;
+  const int64_t K = prob.K;
+  const int T = prob.T;
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;");
   uint32_t rank;
@@ -350,14 +357,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_small_kernel(
   }
 }
 
-template <int S>
-static cudaError_t launch_route_small(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
-                                      int32_t* k_t, int32_t* perm, int32_t* offsets, cudaStream_t stream) {
+template <int S, int MG>
+static cudaError_t launch_route_small_group(const RouteSmallGroupT<MG>& grp, cudaStream_t stream) {
   const size_t smem = route_small_smem(S);
-  cudaError_t e = set_smem((const void*)route_small_kernel<S>, (int)smem);
+  cudaError_t e = set_smem((const void*)route_small_kernel<S, MG>, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kRouteCluster);
+  cfg.gridDim = dim3(kRouteCluster * grp.G);
   cfg.blockDim = dim3(kRouteThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -370,10 +376,27 @@ static cudaError_t launch_route_small(const void* X, int64_t T, int64_t K, const
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  e = cudaLaunchKernelEx(&cfg, route_small_kernel<S>, static_cast<const __nv_bfloat16*>(X), (int)T, K, Wr, bias, k_t,
-                         perm, offsets);
+  e = cudaLaunchKernelEx(&cfg, route_small_kernel<S, MG>, grp);
   if (e != cudaSuccess) return note_error("route launch", e);
   return note_error("kernel launch", cudaGetLastError());
+}
+
+template <int S>
+static cudaError_t launch_route_small(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
+                                      int32_t* k_t, int32_t* perm, int32_t* offsets, cudaStream_t stream) {
+  RouteSmallGroupT<1> grp = {};
+  grp.G = 1;
+  grp.p[0] = RouteSmallProblem{static_cast<const __nv_bfloat16*>(X), Wr, bias, k_t, perm, offsets, K, (int)T};
+  return launch_route_small_group<S, 1>(grp, stream);
+}
+
+// Routing of a group of small batches (every T <= 16, same S), one cluster each.
+cudaError_t launch_route_small_grouped(const RouteSmallGroup& grp, int S, cudaStream_t stream) {
+  switch (S) {
+    case 1: return launch_route_small_group<1, kMaxGroup>(grp, stream);
+    case 2: return launch_route_small_group<2, kMaxGroup>(grp, stream);
+    default: return launch_route_small_group<3, kMaxGroup>(grp, stream);
+  }
 }
 
 // ---- threshold routing with a two-layer MLP scorer -----------------------------------
@@ -403,48 +426,78 @@ constexpr int kMlpHidTile = 128, kMlpKc = 32, kMlpThreads = 256, kMlpScoreThread
 constexpr int kMlpMinSplitK = 64;
 
 template <int TT>
-__global__ void __launch_bounds__(kMlpThreads) route_mlp_hidden_kernel(const __nv_bfloat16* __restrict__ X,
-                                                                      int64_t T, int64_t K,
-                                                                      const float* __restrict__ W1, int64_t H,
-                                                                      int64_t k_per_split,
-                                                                      float* __restrict__ P) {
+__global__ void __launch_bounds__(kMlpThreads, 2) route_mlp_hidden_kernel(const __nv_bfloat16* __restrict__ X,
+                                                                         int64_t T, int64_t K,
+                                                                         const float* __restrict__ W1, int64_t H,
+                                                                         int64_t k_per_split,
+                                                                         float* __restrict__ P) {
   constexpr int kTok = 16 * TT;
-  __shared__ __align__(16) float xs[kMlpKc][kTok + 4];
-  __shared__ __align__(16) float wsm[kMlpKc][kMlpHidTile];
+  constexpr int kXThreads = kTok * kMlpKc / 8;  // threads that load 8 bf16 of x per chunk
+  __shared__ __align__(16) float xs[kMlpKc][kTok + 4];           // k-major fp32 copy of the x chunk
+  __shared__ __align__(16) float wsm[2][kMlpKc][kMlpHidTile];    // W1 chunks, double-buffered
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const int64_t t0 = (int64_t)blockIdx.x * kTok, h0 = (int64_t)blockIdx.y * kMlpHidTile;
   const int64_t split = blockIdx.z, kb = split * k_per_split;
   const int64_t ke = kb + k_per_split < K ? kb + k_per_split : K;
   const bool vec = (H & 3) == 0 && (reinterpret_cast<uintptr_t>(W1) & 15) == 0;
+  const int xr = tid >> 2, xc = (tid & 3) * 8;  // this thread's x row and first column in a chunk
+  const bool x_loader = tid < kXThreads && t0 + xr < T;
+
+  // W1 rows [k0, k0 + 32) x columns [h0, h0 + 128) into wsm[buf]: cp.async when
+  // every 16-byte piece is aligned, else plain loads; columns >= H read as 0.
+  auto stage_w = [&](int buf, int64_t k0) {
+#pragma unroll
+    for (int m = 0; m < kMlpKc * kMlpHidTile / 4 / kMlpThreads; ++m) {
+      const int e = tid + m * kMlpThreads, r = e >> 5, c4 = (e & 31) * 4;
+      const int64_t h = h0 + c4;
+      const float* src = W1 + (k0 + r) * H + h;
+      float* dst = &wsm[buf][r][c4];
+      if (vec && h < H) {  // H % 4 == 0, so h + 3 < H
+        cp_async16(dst, src);
+      } else {
+        dst[0] = h < H ? __ldg(src) : 0.0f;
+        dst[1] = h + 1 < H ? __ldg(src + 1) : 0.0f;
+        dst[2] = h + 2 < H ? __ldg(src + 2) : 0.0f;
+        dst[3] = h + 3 < H ? __ldg(src + 3) : 0.0f;
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  auto load_x = [&](int64_t k0) {
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (x_loader) v = __ldg(reinterpret_cast<const uint4*>(X + (t0 + xr) * K + k0 + xc));
+    return v;
+  };
+  auto store_x = [&](uint4 v) {
+    if (tid < kXThreads) {
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {  // bf16 -> fp32 is a 16-bit shift
+        xs[xc + 2 * q][xr] = __uint_as_float(w[q] << 16);
+        xs[xc + 2 * q + 1][xr] = __uint_as_float(w[q] & 0xffff0000u);
+      }
+    }
+  };
+
   float acc[TT][8];
 #pragma unroll
   for (int i = 0; i < TT; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
 
-  for (int64_t k0 = kb; k0 < ke; k0 += kMlpKc) {  // K and every split are multiples of 32
-#pragma unroll
-    for (int m = 0; m < kTok * kMlpKc / kMlpThreads; ++m) {
-      const int e = tid + m * kMlpThreads, r = e >> 5, c = e & 31;
-      const int64_t t = t0 + r;
-      xs[c][r] = t < T ? __bfloat162float(X[t * K + k0 + c]) : 0.0f;
-    }
-#pragma unroll
-    for (int m = 0; m < kMlpKc * kMlpHidTile / 4 / kMlpThreads; ++m) {
-      const int e = tid + m * kMlpThreads, r = e >> 5, c4 = (e & 31) * 4;
-      const int64_t h = h0 + c4;
-      const float* src = W1 + (k0 + r) * H + h;
-      float4 v;
-      if (vec && h + 3 < H) {
-        v = __ldg(reinterpret_cast<const float4*>(src));
-      } else {
-        v.x = h < H ? __ldg(src) : 0.0f;
-        v.y = h + 1 < H ? __ldg(src + 1) : 0.0f;
-        v.z = h + 2 < H ? __ldg(src + 2) : 0.0f;
-        v.w = h + 3 < H ? __ldg(src + 3) : 0.0f;
-      }
-      *reinterpret_cast<float4*>(&wsm[r][c4]) = v;
+  // K and every split are multiples of 32, so each split is a whole number of chunks.
+  uint4 xv_next = load_x(kb);
+  stage_w(0, kb);
+  int buf = 0;
+  for (int64_t k0 = kb; k0 < ke; k0 += kMlpKc, buf ^= 1) {
+    store_x(xv_next);  // xs is free: the previous chunk ended with a barrier
+    if (k0 + kMlpKc < ke) {
+      xv_next = load_x(k0 + kMlpKc);
+      stage_w(buf ^ 1, k0 + kMlpKc);  // wsm[buf ^ 1] is free for the same reason
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
     __syncthreads();
 #pragma unroll 8
@@ -457,8 +510,8 @@ __global__ void __launch_bounds__(kMlpThreads) route_mlp_hidden_kernel(const __n
 #pragma unroll
         for (int i = 0; i < TT; ++i) xv[i] = xs[c][ty * TT + i];
       }
-      const float4 wa = *reinterpret_cast<const float4*>(&wsm[c][tx * 4]);
-      const float4 wb = *reinterpret_cast<const float4*>(&wsm[c][64 + tx * 4]);
+      const float4 wa = *reinterpret_cast<const float4*>(&wsm[buf][c][tx * 4]);
+      const float4 wb = *reinterpret_cast<const float4*>(&wsm[buf][c][64 + tx * 4]);
       const float w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
       for (int i = 0; i < TT; ++i)
@@ -498,7 +551,17 @@ __global__ void __launch_bounds__(kMlpScoreThreads) route_mlp_score_kernel(const
   for (int j = 0; j < J; ++j) acc[j] = 0.0f;
   for (int64_t i = tid; i < H; i += kMlpScoreThreads) {
     float pre = 0.0f;
-    for (int sp = 0; sp < ksplit; ++sp) pre += P[((int64_t)sp * T + t) * H + i];
+    const float* p = P + t * H + i;
+    const int64_t stride = T * H;
+    int sp = 0;
+    for (; sp + 8 <= ksplit; sp += 8) {  // eight loads in flight, then the adds in split order
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = p[(int64_t)(sp + u) * stride];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) pre += v[u];
+    }
+    for (; sp < ksplit; ++sp) pre += p[(int64_t)sp * stride];
     const float hv = fmaxf(pre + (b1 ? __ldg(b1 + i) : 0.0f), 0.0f);
 #pragma unroll
     for (int j = 0; j < J; ++j) acc[j] = fmaf(hv, __ldg(W2 + i * J + j), acc[j]);
@@ -530,13 +593,13 @@ __global__ void route_mlp_base_only_kernel(int64_t T, int32_t* __restrict__ k_t)
   if (t < T) k_t[t] = 1;
 }
 
-// Splits of K for the hidden layer: about four CTAs per SM in all, each split
-// a multiple of 32 rows and at least 64.
+// Splits of K for the hidden layer: as many as fit one wave of two CTAs per SM
+// (no partial second wave), each split a multiple of 32 rows and at least 64.
 static int64_t mlp_k_per_split(int64_t T, int64_t K, int64_t H, int sms) {
   const int64_t tok = T <= 16 ? 16 : 64;
   int64_t base = ((T + tok - 1) / tok) * ((H + kMlpHidTile - 1) / kMlpHidTile);
   if (base < 1) base = 1;
-  int64_t ks = (4 * (int64_t)sms + base - 1) / base;
+  int64_t ks = 2 * (int64_t)sms / base;
   const int64_t kmax = K / kMlpMinSplitK > 0 ? K / kMlpMinSplitK : 1;
   if (ks > kmax) ks = kmax;
   if (ks < 1) ks = 1;
