@@ -37,7 +37,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "mixed-bit GEMM: decode HBM GB/s & prefill TFLOP/s, % of B200 roofline"
 WORKLOAD = ("decode GEMV, Llama-7B projections (N,K) in {(4096,4096),(11008,4096),(4096,11008)} "
-            "x T in {1,4,16}, 3x2-bit slices, group 128, route+bucket+GEMM per call (mobi_linear)")
+            "x T in {1,4,16}, 3x2-bit slices, group 128, route+bucket+GEMM per problem; the nine problems "
+            "of a step as two mobi_linear_grouped calls (T <= 8, T = 16)")
 
 
 def peaks():
@@ -179,13 +180,6 @@ class DecodeCase:
         return int(self.k_t.max().item())
 
 
-def launches_per_call(T, K):
-    """Library kernels one route + GEMM call launches (T <= 16): the one-cluster
-    route kernel, the decode kernel and, when K spans more than one 1024-column
-    chunk, the chunk-reduce kernel."""
-    return 1 + 1 + (1 if K > 1024 else 0)
-
-
 def grouped_launches(group_T, group_K):
     """Library kernels of one mobi_linear_grouped call: one routing launch, one
     decode launch per fragment class present (T <= 8, T > 8) and one
@@ -216,30 +210,6 @@ def time_graph(step, steps, warmup=3):
     torch.cuda.synchronize()
     del graph
     return e0.elapsed_time(e1) / steps
-
-
-def time_decode_grouped(mobi, cases, bytes_step, steps, hbm_peak):
-    """The headline decode step through mobi_linear_grouped: the six calls with
-    T <= 8 as one group and the three with T = 16 as another, so one step is two
-    grouped calls instead of nine mobi_linear calls (same inputs, same outputs)."""
-    groups = [[c for c in cases if c.T <= 8], [c for c in cases if c.T > 8]]
-    probs = [[{"X": c.X, "Wr": c.Wr, "bias": None, "codes": c.codes, "sz": c.sz, "N": c.N, "Y": c.Y,
-               "k_t": c.k_t, "perm": c.perm, "offsets": c.off} for c in g] for g in groups]
-    ws = [torch.empty(max(mobi.mobi_linear_grouped_workspace_bytes(pr), 16), dtype=torch.uint8,
-                      device=cases[0].X.device) for pr in probs]
-
-    def step():
-        for pr, w in zip(probs, ws):
-            mobi.mobi_linear_grouped(pr, ws=w)
-    step()
-    mobi.mobi_sync_check()
-    ms = time_graph(step, steps)
-    mobi.mobi_sync_check()
-    launches = sum(grouped_launches([c.T for c in g], [c.K for c in g]) for g in groups)
-    return {"workload": "the same nine decode calls as two mobi_linear_grouped calls (T <= 8: six problems; "
-                        "T = 16: three)", "ms_per_step": round(ms, 5),
-            "GB/s": round(bytes_step / ms / 1e6, 1), "frac_of_hbm": round(bytes_step / ms / 1e6 / hbm_peak, 4),
-            "launches_per_step": launches, "steps": steps}
 
 
 def build_decode_cases(mobi, wl, dev):
@@ -502,6 +472,56 @@ def time_route_mlp(mobi, wl, dev, hbm_peak, flush, reps=20):
     return out
 
 
+def time_ckpt(mobi, wl, dev, reps=3):
+    """Many-in-one checkpoint I/O: the seven packed projections of one
+    Llama-2-7B-shaped layer saved from HBM to one file, then loaded back into
+    HBM at 1, 2 and 3 slices (2, 4, 6 bits; each load reads only its slices).
+    Host wall time of the calls (each returns once the data is on the device);
+    the file was just written, so reads come from the OS page cache."""
+    import tempfile
+    import time
+    tensors = []
+    for p in range(len(wl.LLAMA7B_PROJECTIONS)):
+        L = wl.full_model_projection(0, p, T=1, device=dev)
+        codes, sz = mobi.mobi_pack(L.W, S=3)
+        tensors.append((f"layers.0.{wl.LLAMA7B_PROJECTIONS[p][0]}", codes, sz))
+        del L
+    torch.cuda.synchronize()
+    total = sum(c.numel() * 4 + z.numel() * 4 for _, c, z in tensors)
+    d = tempfile.mkdtemp(prefix="mobi_ckpt_")
+    path = os.path.join(d, "layer0.mobi")
+    out = {"workload": "7 packed projections of one Llama-2-7B layer (3 slices) in one checkpoint file",
+           "file_bytes_3_slices": total}
+    try:
+        t_save = []
+        for _ in range(reps):
+            t0 = time.perf_counter()
+            mobi.mobi_ckpt_save(path, tensors)
+            t_save.append(time.perf_counter() - t0)
+        out["save_GB/s"] = round(total / statistics.median(t_save) / 1e9, 2)
+        bufs = [(torch.empty_like(c), torch.empty_like(z)) for _, c, z in tensors]
+        with mobi.MobiCheckpoint(path) as ck:
+            for k in (1, 2, 3):
+                times = []
+                for _ in range(reps):
+                    r0 = ck.bytes_read
+                    t0 = time.perf_counter()
+                    for (name, c, z), (bc, bz) in zip(tensors, bufs):
+                        ck.load(name, k, device=dev, codes=bc[:k], sz=bz[:k])
+                    times.append(time.perf_counter() - t0)
+                    nread = ck.bytes_read - r0
+                for (name, c, z), (bc, bz) in zip(tensors, bufs):
+                    assert torch.equal(bc[:k], c[:k]) and torch.equal(bz[:k], z[:k])
+                out[f"load_{2 * k}bit"] = {"bytes_read": nread, "ms": round(1e3 * statistics.median(times), 2),
+                                           "GB/s": round(nread / statistics.median(times) / 1e9, 2)}
+    finally:
+        if os.path.exists(path):
+            os.remove(path)
+        os.rmdir(d)
+    out["timing"] = f"median of {reps}, host wall clock, CRC-32C verified on load"
+    return out
+
+
 def run_gpu(args, world, rank):
     import token_adaptive_mixed_b200 as mobi
     from token_adaptive_mixed_b200 import build as mobi_build
@@ -516,6 +536,8 @@ def run_gpu(args, world, rank):
 
     if args.only == "route_mlp":
         return {"route_mlp": time_route_mlp(mobi, wl, dev, hbm_peak, l2_flush_buffer(dev))}
+    if args.only == "ckpt":
+        return {"ckpt": time_ckpt(mobi, wl, dev)}
     if args.only == "prefill":
         flush = l2_flush_buffer(dev)
         out = {"prefill": time_prefill(mobi, wl.prefill(), dev, args.prefill_reps, tf_peak, flush)}
@@ -529,19 +551,31 @@ def run_gpu(args, world, rank):
     kmax = [c.kmax() for c in cases]
     bytes_step = sum(decode_bytes(c.N, c.K, c.T, km) for c, km in zip(cases, kmax))
 
-    # Capture one step (9 x (route + GEMM), 27 kernel launches) in a CUDA graph.
+    # One step = the nine decode problems through the public API as two
+    # mobi_linear_grouped calls (the six with T <= 8, the three with T = 16),
+    # captured in one CUDA graph.
+    groups = [[c for c in cases if c.T <= 8], [c for c in cases if c.T > 8]]
+    probs = [[{"X": c.X, "Wr": c.Wr, "bias": None, "codes": c.codes, "sz": c.sz, "N": c.N, "Y": c.Y,
+               "k_t": c.k_t, "perm": c.perm, "offsets": c.off} for c in g] for g in groups]
+    gws = [torch.empty(max(mobi.mobi_linear_grouped_workspace_bytes(pr), 16), dtype=torch.uint8, device=dev)
+           for pr in probs]
+
+    def grouped_step():
+        for pr, w in zip(probs, gws):
+            mobi.mobi_linear_grouped(pr, ws=w)
+    grouped_step()
+    mobi.mobi_sync_check()
+    launches_per_step = sum(grouped_launches([c.T for c in g], [c.K for c in g]) for g in groups)
+
     stream = torch.cuda.Stream()
     stream.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(stream):
         for _ in range(2):
-            for c in cases:
-                c.step()
+            grouped_step()
     torch.cuda.current_stream().wait_stream(stream)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        for c in cases:
-            c.step()
-    launches_per_step = sum(launches_per_call(c.T, c.K) for c in cases)
+        grouped_step()
 
     for _ in range(max(args.warmup, 3)):
         graph.replay()
@@ -560,35 +594,39 @@ def run_gpu(args, world, rank):
     ms_local = e0.elapsed_time(e1) / args.steps
     ms = max_over_ranks(ms_local, world)
     value = world * bytes_step / (ms * 1e-3) / 1e9
+    mobi.mobi_sync_check()
+    del graph
 
-    # Roofline of the dominant kernel pair (staging + decode GEMM kernels): events
-    # around each mobi_gemm on the launching stream, rotating through the cases.
-    per_case_ms = []
-    reps = 20
-    for c in cases:
-        c.gemm()
-    torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps * len(cases))]
-    i = 0
-    for r in range(reps):
+    # The same nine problems as nine mobi_linear calls (one per problem).
+    steps_cmp = min(args.steps, 500)
+
+    def linear_step():
         for c in cases:
-            ev[i][0].record()
-            c.gemm()
-            ev[i][1].record()
-            i += 1
-    torch.cuda.synchronize()
-    for ci, c in enumerate(cases):
-        per_case_ms.append(statistics.mean(ev[r * len(cases) + ci][0].elapsed_time(ev[r * len(cases) + ci][1])
-                                           for r in range(reps)))
-    gemm_ms = sum(per_case_ms)
-    achieved = bytes_step / (gemm_ms * 1e-3) / 1e9
+            c.step()
+    ms_linear = time_graph(linear_step, steps_cmp)
 
-    grouped = time_decode_grouped(mobi, cases, bytes_step, min(args.steps, 500), hbm_peak)
+    # Roofline of the dominant kernels (decode GEMM + chunk reduction): the
+    # step's two grouped GEMMs alone (mobi_gemm_grouped, k_t from the routing
+    # above), as one CUDA graph.
+    gprobs = [[{"X": c.X, "k_t": c.k_t, "codes": c.codes, "sz": c.sz, "N": c.N, "Y": c.Y} for c in g]
+              for g in groups]
+
+    def gemm_step():
+        for pr, w in zip(gprobs, gws):
+            mobi.mobi_gemm_grouped(pr, ws=w)
+    ms_gemm = time_graph(gemm_step, steps_cmp)
+    mobi.mobi_sync_check()
+    achieved = bytes_step / (ms_gemm * 1e-3) / 1e9
+
+    def gemm_calls_step():
+        for c in cases:
+            c.gemm()
+    ms_gemm_calls = time_graph(gemm_calls_step, steps_cmp)
 
     # End to end through the public API with host buffers (pinned), copies inside:
     # the step's nine activation matrices live in one pinned host buffer and one
     # device buffer (one host-to-device copy), the nine outputs likewise (one
-    # device-to-host copy), and the nine mobi_linear calls run in between.
+    # device-to-host copy), and the two grouped calls run in between.
     h2d = sum(c.T * c.K * 2 for c in cases)
     d2h = sum(c.T * c.N * 4 for c in cases)
     e2e_steps = max(3, min(args.steps, 50))
@@ -603,11 +641,12 @@ def run_gpu(args, world, rank):
         c.Y = Y_dev[yo:yo + c.T * c.N].view(c.T, c.N)
         xo += c.T * c.K
         yo += c.T * c.N
+    e2e_probs = [[dict(pr, X=c.X, Y=c.Y) for pr, c in zip(prs, g)] for prs, g in zip(probs, groups)]
 
     def e2e_step():
         X_dev.copy_(X_host, non_blocking=True)
-        for c in cases:
-            c.step()
+        for pr, w in zip(e2e_probs, gws):
+            mobi.mobi_linear_grouped(pr, ws=w)
         Y_host.copy_(Y_dev, non_blocking=True)
     for _ in range(3):
         e2e_step()
@@ -627,21 +666,25 @@ def run_gpu(args, world, rank):
         "config": {"workload": WORKLOAD, "bytes_per_step": bytes_step, "kmax_per_call": kmax,
                    "l2": "rotating packed copies, ~270 MB between reuses (> 2x L2)",
                    "timing": "CUDA graph of one step, CUDA events, max over ranks", "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": "decode GEMM (staging + mma.sync decode kernels)",
+        "roofline": {"bound": "hbm", "kernel": "decode GEMM (mma.sync decode kernels + chunk reduction): the "
+                                              "step's two mobi_gemm_grouped calls as one CUDA graph",
                      "achieved": round(achieved, 2), "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "frac_of_8TBs_nominal": round(achieved / 8000.0, 4),
                      "traffic": round(bytes_step * DECODE_DRAM_RATIO),
                      "traffic_unit": "bytes per step (ncu DRAM bytes / algorithmic bytes x algorithmic bytes)",
-                     "per_call_us": [round(1e3 * x, 2) for x in per_case_ms]},
+                     "gemm_ms_per_step": round(ms_gemm, 5),
+                     "gemm_ms_per_step_nine_calls": round(ms_gemm_calls, 5)},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
-        "decode_grouped": grouped,
+        "per_problem_calls": {"workload": "the same step as nine mobi_linear calls, one per problem (27 launches)",
+                              "ms_per_step": round(ms_linear, 5), "GB/s": round(bytes_step / ms_linear / 1e6, 1),
+                              "frac_of_hbm": round(bytes_step / ms_linear / 1e6 / hbm_peak, 4)},
     }
     if rank == 0:
         out["pack"] = time_pack(mobi, wl, dev)
-    del cases, graph
+    del cases
     torch.cuda.empty_cache()
     if args.only == "all" and not args.skip_full_model:
         out["full_model"] = time_full_model(mobi, wl, dev, 20, hbm_peak)
@@ -653,6 +696,7 @@ def run_gpu(args, world, rank):
             out["skewed_prefill"] = time_prefill(mobi, wl.skewed_prefill(), dev, args.prefill_reps, tf_peak, flush)
     if args.only == "all" and rank == 0:
         out["route_mlp"] = time_route_mlp(mobi, wl, dev, hbm_peak, l2_flush_buffer(dev))
+        out["ckpt"] = time_ckpt(mobi, wl, dev)
     return out
 
 
@@ -744,7 +788,7 @@ def main():
     ap.add_argument("--impl", default="mobi", choices=["mobi", "reference"])
     ap.add_argument("--cpu-baseline-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill", "route_mlp"],
+    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill", "route_mlp", "ckpt"],
                     help="run a subset (profiling); the default runs everything")
     ap.add_argument("--prefill-reps", type=int, default=10)
     ap.add_argument("--skip-skewed", action="store_true")

@@ -84,7 +84,9 @@ typedef enum {
   MOBI_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
   MOBI_ERR_WORKSPACE = 4,         /* ws == NULL or ws_bytes below the required size */
   MOBI_ERR_CUDA = 5,              /* a CUDA launch or query failed (error cleared) */
-  MOBI_ERR_TIMEOUT = 6            /* a device-side bounded wait ran out */
+  MOBI_ERR_TIMEOUT = 6,           /* a device-side bounded wait ran out */
+  MOBI_ERR_IO = 7                 /* a checkpoint file could not be read or written,
+                                     is not one, or failed a checksum */
 } mobi_status;
 
 /* Human-readable name of a status (static storage, never NULL). */
@@ -268,6 +270,29 @@ typedef struct mobi_linear_problem {
 MOBI_API size_t mobi_linear_grouped_workspace_bytes(const mobi_linear_problem* problems, int count,
                                                     int S);
 
+/* One problem of mobi_gemm_grouped: the arguments of one decode-sized mobi_gemm. */
+typedef struct mobi_gemm_problem {
+  const void* X;          /* bf16 [T][K] */
+  const int32_t* k_t;     /* int32 [T], values 1..S */
+  const uint32_t* codes;  /* as produced by mobi_pack for N, K */
+  const uint32_t* sz;
+  float* Y;               /* out, fp32 [T][N] */
+  int64_t T, N, K;
+} mobi_gemm_problem;
+
+/* Scratch bytes of mobi_gemm_grouped (0 for invalid arguments or none needed). */
+MOBI_API size_t mobi_gemm_grouped_workspace_bytes(const mobi_gemm_problem* problems, int count, int S);
+
+/*
+ * mobi_gemm_grouped — the GEMM half of mobi_linear_grouped: up to
+ *   MOBI_MAX_GROUP decode-sized (T <= 16) mobi_gemm problems whose k_t are
+ *   already known, one decode launch per fragment class plus one chunk
+ *   reduction. Results equal one mobi_gemm call per problem bit for bit.
+ *   Errors as for mobi_gemm, checked for every problem before any launch.
+ */
+MOBI_API mobi_status mobi_gemm_grouped(const mobi_gemm_problem* problems, int count, int G, int S,
+                                       void* ws, size_t ws_bytes, void* stream);
+
 /*
  * mobi_linear_grouped — up to MOBI_MAX_GROUP independent decode-sized
  *   mobi_linear problems (every T <= 16) in one step: the projections of a
@@ -290,6 +315,68 @@ MOBI_API size_t mobi_linear_grouped_workspace_bytes(const mobi_linear_problem* p
  */
 MOBI_API mobi_status mobi_linear_grouped(const mobi_linear_problem* problems, int count, int G,
                                          int S, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- many-in-one checkpoints of packed layers -------------------------------
+ *
+ * One file holds the packed slices of any number of layers ([ja] §2.1: a single
+ * decomposition serves every precision; [en] §3: "many-in-one" storage, only
+ * the slices needed are fetched). Because codes and scale/zero words are
+ * slice-major, loading a layer at k slices (2k bits) reads only the first k
+ * slices of each block: a prefix of the file's codes block and of its sz block.
+ *
+ * File format (little-endian; version 1):
+ *   [0, 64)  header: "MOBICKPT", u32 version, u32 count, u64 table offset,
+ *            u64 table bytes, u32 CRC-32C of the table, 28 reserved bytes.
+ *   table    count entries of 192 bytes: name (96 bytes, NUL-terminated),
+ *            i64 N, i64 K, i32 G, i32 S, u64 codes offset, u64 codes bytes per
+ *            slice (N K / 4), u64 sz offset, u64 sz bytes per slice (K/G N 4),
+ *            u32 CRC-32C of each slice's codes [3] and sz [3], zero padding.
+ *   data     per tensor its codes block [S][N][K/16] u32 and its sz block
+ *            [S][K/G][N] u32, each starting on a 4096-byte boundary.
+ * CRC-32C is the Castagnoli CRC (reflected polynomial 0x82F63B78, initial
+ * value and final xor 0xFFFFFFFF).
+ *
+ * host_ptrs = 1: codes and sz are host memory; 0: device memory (copied
+ * through pinned staging buffers on `stream`; the call returns once the data
+ * has arrived). Errors: MOBI_ERR_INVALID_ARG (bad argument, duplicate or
+ * over-long name, index or slice count out of range), MOBI_ERR_IO (file
+ * errors, bad magic or version, truncated file, checksum mismatch),
+ * MOBI_ERR_CUDA (a copy failed). A failed save leaves no file at `path`.
+ */
+typedef struct mobi_ckpt_tensor {
+  const char* name;       /* at most 95 bytes, unique in the file */
+  const uint32_t* codes;  /* [S][N][K/16], as produced by mobi_pack */
+  const uint32_t* sz;     /* [S][K/G][N] */
+  int64_t N, K;
+  int G, S;
+} mobi_ckpt_tensor;
+
+typedef struct mobi_ckpt mobi_ckpt; /* an open checkpoint (not thread-safe) */
+
+/* Write `count` packed tensors to `path` (written to a temporary name, then
+ * renamed). */
+MOBI_API mobi_status mobi_ckpt_save(const char* path, const mobi_ckpt_tensor* tensors, int count,
+                                    int host_ptrs, void* stream);
+/* Open a checkpoint: reads and checks the header and the table. */
+MOBI_API mobi_status mobi_ckpt_open(const char* path, mobi_ckpt** out);
+/* Number of tensors; -1 for NULL. */
+MOBI_API int mobi_ckpt_count(const mobi_ckpt* ckpt);
+/* Index of the tensor called `name`, or -1. */
+MOBI_API int mobi_ckpt_find(const mobi_ckpt* ckpt, const char* name);
+/* Shape of tensor `index`; *name points into the reader (valid until close). */
+MOBI_API mobi_status mobi_ckpt_info(const mobi_ckpt* ckpt, int index, const char** name, int64_t* N,
+                                    int64_t* K, int* G, int* S);
+/* Load the first `slices` slices (1..S) of tensor `index` into codes
+ * [slices][N][K/16] and sz [slices][K/G][N]: a packed array with S = slices.
+ * verify = 1 checks the CRC of every slice read. */
+MOBI_API mobi_status mobi_ckpt_load(mobi_ckpt* ckpt, int index, int slices, uint32_t* codes,
+                                    uint32_t* sz, int host_ptrs, int verify, void* stream);
+/* Bytes read from the file by this reader so far (data blocks only). */
+MOBI_API int64_t mobi_ckpt_bytes_read(const mobi_ckpt* ckpt);
+/* Close the reader (NULL is a no-op). */
+MOBI_API void mobi_ckpt_close(mobi_ckpt* ckpt);
+/* CRC-32C of n bytes of host memory, continuing from `crc` (0 to start). */
+MOBI_API uint32_t mobi_crc32c(uint32_t crc, const void* data, size_t n);
 
 /*
  * mobi_gemm_decode_noalloc — the decode GEMM (T <= 16) without a workspace.

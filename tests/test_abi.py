@@ -179,3 +179,25 @@ def test_linear_grouped_validation(L):
     per = [L.mobi_linear_grouped_workspace_bytes((P * 1)(arr[i]), 1, 3) for i in range(2)]
     assert need == sum(per) and all(b % 256 == 0 and b > 0 for b in per)
     assert L.mobi_linear_grouped_workspace_bytes(arr, 2, 4) == 0
+
+
+def test_gemm_grouped_validation(L):
+    P = mobi.GemmProblem
+
+    def prob(T=8, N=4096, K=4096, X=FAKE, Y=FAKE, k_t=FAKE):
+        return P(X, k_t, FAKE, FAKE, Y, T, N, K)
+
+    def call(probs, S=3, G=128, ws=FAKE, wsb=1 << 30):
+        arr = (P * max(len(probs), 1))(*probs)
+        return L.mobi_gemm_grouped(arr if probs else None, len(probs), G, S, ws, wsb, None)
+    assert call([]) == 1
+    assert call([prob()] * 9) == 1
+    assert call([prob(T=17)]) == 2
+    assert call([prob(K=200)]) == 2
+    assert call([prob(k_t=None)]) == 1
+    assert call([prob(Y=FAKE + 4)]) == 3
+    assert call([prob(k_t=FAKE + 2)]) == 3
+    assert call([prob()], wsb=16) == 4
+    arr = (P * 2)(prob(T=4), prob(T=16, N=11008))
+    assert L.mobi_gemm_grouped_workspace_bytes(arr, 2, 3) == sum(
+        L.mobi_gemm_grouped_workspace_bytes((P * 1)(arr[i]), 1, 3) for i in range(2))

@@ -122,3 +122,20 @@ def test_grouped_repeated_in_a_graph(mobi, oracle):
     mobi.mobi_sync_check()
     check_against_oracle(oracle, layers, probs, outs)
     del graph
+
+
+def test_gemm_grouped_equals_gemm_calls(mobi):
+    """mobi_gemm_grouped (k_t given) equals one mobi_gemm call per problem bit for bit."""
+    layers, probs = make_problems(mobi, [(256, 512, 2), (1024, 4096, 16), (512, 11008, 7), (64, 1024, 12)],
+                                  seed0=1800)
+    gprobs = []
+    for pr in probs:
+        k_t, perm, off = mobi.mobi_route(pr["X"], pr["Wr"], pr["bias"])
+        gprobs.append({"X": pr["X"], "k_t": k_t, "perm": perm, "off": off, "codes": pr["codes"], "sz": pr["sz"],
+                       "N": pr["N"]})
+    Ys = mobi.mobi_gemm_grouped(gprobs)
+    mobi.mobi_sync_check()
+    for g, Y in zip(gprobs, Ys):
+        Y1 = mobi.mobi_gemm(g["X"], g["k_t"], g["perm"], g["off"], g["codes"], g["sz"], g["N"])
+        mobi.mobi_sync_check()
+        assert torch.equal(Y, Y1)

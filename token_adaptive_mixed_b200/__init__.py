@@ -14,6 +14,7 @@ Entry points (same names as the C ABI):
   mobi_gemm_path(..., path)         the same with a forced kernel
   mobi_linear(X, Wr, bias, codes, sz, N)  route + GEMM in one call -> (Y, k_t, perm, offsets)
   mobi_linear_grouped(problems)     up to 8 decode-sized mobi_linear problems in one step
+  mobi_ckpt_save / MobiCheckpoint   many-in-one checkpoint of packed layers (load any slice count)
   mobi_sync_check()                 sync + device-side error word
 """
 from __future__ import annotations
@@ -28,7 +29,9 @@ __all__ = [
     "mobi_route_workspace_bytes", "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm", "mobi_last_error",
     "mobi_gemm_path", "mobi_sync_check", "mobi_debug_set_wait_limit", "mobi_gemm_decode_noalloc", "mobi_linear",
     "mobi_linear_workspace_bytes", "mobi_route_mlp", "mobi_route_mlp_workspace_bytes", "mobi_linear_grouped",
-    "mobi_linear_grouped_workspace_bytes", "MAX_GROUP", "PATH_AUTO",
+    "mobi_linear_grouped_workspace_bytes", "mobi_gemm_grouped", "mobi_gemm_grouped_workspace_bytes", "MAX_GROUP",
+    "mobi_ckpt_save", "MobiCheckpoint", "mobi_crc32c",
+    "PATH_AUTO",
     "PATH_DECODE",
     "PATH_PREFILL", "EXPORTED_SYMBOLS",
 ]
@@ -40,6 +43,19 @@ PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
 MAX_GROUP = 8  # MOBI_MAX_GROUP
 
 
+class CkptTensor(ctypes.Structure):
+    """mobi_ckpt_tensor (include/mobi.h)."""
+    _fields_ = [("name", ctypes.c_char_p), ("codes", ctypes.c_void_p), ("sz", ctypes.c_void_p),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("G", ctypes.c_int), ("S", ctypes.c_int)]
+
+
+class GemmProblem(ctypes.Structure):
+    """mobi_gemm_problem (include/mobi.h)."""
+    _fields_ = [("X", ctypes.c_void_p), ("k_t", ctypes.c_void_p), ("codes", ctypes.c_void_p),
+                ("sz", ctypes.c_void_p), ("Y", ctypes.c_void_p), ("T", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64)]
+
+
 class LinearProblem(ctypes.Structure):
     """mobi_linear_problem (include/mobi.h): pointers and sizes of one problem."""
     _fields_ = [("X", ctypes.c_void_p), ("Wr", ctypes.c_void_p), ("bias", ctypes.c_void_p),
@@ -47,7 +63,7 @@ class LinearProblem(ctypes.Structure):
                 ("k_t", ctypes.c_void_p), ("perm", ctypes.c_void_p), ("offsets", ctypes.c_void_p),
                 ("T", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
 STATUS_NAMES = ["MOBI_OK", "MOBI_ERR_INVALID_ARG", "MOBI_ERR_UNSUPPORTED_SHAPE", "MOBI_ERR_MISALIGNED",
-                "MOBI_ERR_WORKSPACE", "MOBI_ERR_CUDA", "MOBI_ERR_TIMEOUT"]
+                "MOBI_ERR_WORKSPACE", "MOBI_ERR_CUDA", "MOBI_ERR_TIMEOUT", "MOBI_ERR_IO"]
 
 # Every symbol include/mobi.h declares.
 EXPORTED_SYMBOLS = (
@@ -55,6 +71,9 @@ EXPORTED_SYMBOLS = (
     "mobi_gemm_workspace_bytes", "mobi_pack", "mobi_route", "mobi_gemm", "mobi_gemm_path", "mobi_sync_check",
     "mobi_debug_set_wait_limit", "mobi_gemm_decode_noalloc", "mobi_linear", "mobi_linear_workspace_bytes",
     "mobi_route_mlp", "mobi_route_mlp_workspace_bytes", "mobi_linear_grouped", "mobi_linear_grouped_workspace_bytes",
+    "mobi_gemm_grouped", "mobi_gemm_grouped_workspace_bytes",
+    "mobi_ckpt_save", "mobi_ckpt_open", "mobi_ckpt_count", "mobi_ckpt_find", "mobi_ckpt_info", "mobi_ckpt_load",
+    "mobi_ckpt_bytes_read", "mobi_ckpt_close", "mobi_crc32c",
 )
 
 
@@ -114,6 +133,29 @@ def lib() -> ctypes.CDLL:
         L.mobi_linear_grouped_workspace_bytes.restype = sz_t
         L.mobi_linear_grouped.argtypes = [p, ci, ci, ci, p, sz_t, p]
         L.mobi_linear_grouped.restype = ci
+        L.mobi_gemm_grouped_workspace_bytes.argtypes = [p, ci, ci]
+        L.mobi_gemm_grouped_workspace_bytes.restype = sz_t
+        L.mobi_gemm_grouped.argtypes = [p, ci, ci, ci, p, sz_t, p]
+        L.mobi_gemm_grouped.restype = ci
+        L.mobi_ckpt_save.argtypes = [ctypes.c_char_p, p, ci, ci, p]
+        L.mobi_ckpt_save.restype = ci
+        L.mobi_ckpt_open.argtypes = [ctypes.c_char_p, ctypes.POINTER(p)]
+        L.mobi_ckpt_open.restype = ci
+        L.mobi_ckpt_count.argtypes = [p]
+        L.mobi_ckpt_count.restype = ci
+        L.mobi_ckpt_find.argtypes = [p, ctypes.c_char_p]
+        L.mobi_ckpt_find.restype = ci
+        L.mobi_ckpt_info.argtypes = [p, ci, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(i64),
+                                     ctypes.POINTER(i64), ctypes.POINTER(ci), ctypes.POINTER(ci)]
+        L.mobi_ckpt_info.restype = ci
+        L.mobi_ckpt_load.argtypes = [p, ci, ci, p, p, ci, ci, p]
+        L.mobi_ckpt_load.restype = ci
+        L.mobi_ckpt_bytes_read.argtypes = [p]
+        L.mobi_ckpt_bytes_read.restype = i64
+        L.mobi_ckpt_close.argtypes = [p]
+        L.mobi_ckpt_close.restype = None
+        L.mobi_crc32c.argtypes = [ctypes.c_uint32, p, sz_t]
+        L.mobi_crc32c.restype = ctypes.c_uint32
         L.mobi_sync_check.argtypes = [p]
         L.mobi_sync_check.restype = ci
         L.mobi_debug_set_wait_limit.argtypes = [i64]
@@ -280,6 +322,148 @@ def mobi_linear_grouped(problems, S: int = 3, G: int = 128, ws: torch.Tensor | N
     _check("mobi_linear_grouped", lib().mobi_linear_grouped(arr, len(filled), G, S, _ptr(ws),
                                                             0 if ws is None else ws.numel(), _stream(stream)))
     return [(d["Y"], d["k_t"], d["perm"], d["offsets"]) for d in filled]
+
+
+def _gemm_problem_array(problems):
+    arr = (GemmProblem * len(problems))()
+    filled = []
+    for i, pr in enumerate(problems):
+        X = pr["X"]
+        T, K = X.shape
+        d = dict(pr)
+        if d.get("Y") is None:
+            d["Y"] = torch.empty((T, d["N"]), dtype=torch.float32, device=X.device)
+        arr[i] = GemmProblem(_ptr(X), _ptr(d["k_t"]), _ptr(d["codes"]), _ptr(d["sz"]), _ptr(d["Y"]), T, d["N"], K)
+        filled.append(d)
+    return arr, filled
+
+
+def mobi_gemm_grouped_workspace_bytes(problems, S: int = 3) -> int:
+    arr, _ = _gemm_problem_array(problems)
+    return lib().mobi_gemm_grouped_workspace_bytes(arr, len(problems), S)
+
+
+def mobi_gemm_grouped(problems, S: int = 3, G: int = 128, ws: torch.Tensor | None = None, stream=None):
+    """Up to MAX_GROUP decode-sized mobi_gemm problems (dicts with X, k_t, codes, sz, N and
+    optionally Y) in one launch per fragment class. Returns [Y] in problem order."""
+    arr, filled = _gemm_problem_array(problems)
+    if len(filled) == 0:
+        raise ValueError("mobi_gemm_grouped needs at least one problem")
+    need = lib().mobi_gemm_grouped_workspace_bytes(arr, len(filled), S)
+    ws = _workspace(need, filled[0]["X"].device, ws) if need > 0 else ws
+    _check("mobi_gemm_grouped", lib().mobi_gemm_grouped(arr, len(filled), G, S, _ptr(ws),
+                                                        0 if ws is None else ws.numel(), _stream(stream)))
+    return [d["Y"] for d in filled]
+
+
+def _any_ptr(t):
+    """(pointer, is_host) of a contiguous tensor or numpy array."""
+    if isinstance(t, torch.Tensor):
+        if not t.is_contiguous():
+            raise ValueError("checkpoint tensors must be contiguous")
+        return ctypes.c_void_p(t.data_ptr()), not t.is_cuda
+    import numpy as np
+    a = np.ascontiguousarray(t)
+    return ctypes.c_void_p(a.ctypes.data), True
+
+
+def mobi_crc32c(data, crc: int = 0) -> int:
+    """CRC-32C of a bytes-like object or a CPU tensor / numpy array."""
+    if isinstance(data, (bytes, bytearray)):
+        buf = (ctypes.c_char * len(data)).from_buffer_copy(bytes(data))
+        return lib().mobi_crc32c(crc, ctypes.cast(buf, ctypes.c_void_p), len(data))
+    ptr, host = _any_ptr(data)
+    if not host:
+        raise ValueError("mobi_crc32c takes host memory")
+    nbytes = data.numel() * data.element_size() if isinstance(data, torch.Tensor) else data.nbytes
+    return lib().mobi_crc32c(crc, ptr, nbytes)
+
+
+def mobi_ckpt_save(path: str, tensors, G: int = 128, stream=None) -> None:
+    """Write packed layers to one checkpoint. tensors: sequence of (name, codes, sz) with
+    codes int32/uint32 [S, N, K/16] and sz [S, K/G, N], all on the device or all on the host."""
+    arr = (CkptTensor * len(tensors))()
+    keep = []
+    host_flags = set()
+    for i, (name, codes, sz) in enumerate(tensors):
+        S, N, K16 = codes.shape
+        cp, ch = _any_ptr(codes)
+        zp, zh = _any_ptr(sz)
+        host_flags.update((ch, zh))
+        nb = name.encode()
+        keep.append(nb)
+        arr[i] = CkptTensor(nb, cp, zp, N, K16 * 16, G, S)
+    if len(host_flags) != 1:
+        raise ValueError("checkpoint tensors must be all on the host or all on the device")
+    host = host_flags.pop()
+    _check("mobi_ckpt_save", lib().mobi_ckpt_save(str(path).encode(), arr, len(tensors), int(host),
+                                                  None if host else _stream(stream)))
+
+
+class MobiCheckpoint:
+    """A checkpoint opened for reading; load(name, slices) returns packed (codes, sz) with S = slices."""
+
+    def __init__(self, path: str):
+        h = ctypes.c_void_p()
+        _check("mobi_ckpt_open", lib().mobi_ckpt_open(str(path).encode(), ctypes.byref(h)))
+        self._h = h
+
+    def close(self) -> None:
+        if self._h:
+            lib().mobi_ckpt_close(self._h)
+            self._h = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __len__(self) -> int:
+        return lib().mobi_ckpt_count(self._h)
+
+    def names(self) -> list[str]:
+        return [self.info(i)[0] for i in range(len(self))]
+
+    def find(self, name: str) -> int:
+        return lib().mobi_ckpt_find(self._h, name.encode())
+
+    def info(self, index: int):
+        """(name, N, K, G, S) of tensor `index`."""
+        nm = ctypes.c_char_p()
+        N, K = ctypes.c_int64(), ctypes.c_int64()
+        G, S = ctypes.c_int(), ctypes.c_int()
+        _check("mobi_ckpt_info", lib().mobi_ckpt_info(self._h, index, ctypes.byref(nm), ctypes.byref(N),
+                                                      ctypes.byref(K), ctypes.byref(G), ctypes.byref(S)))
+        return nm.value.decode(), N.value, K.value, G.value, S.value
+
+    @property
+    def bytes_read(self) -> int:
+        return lib().mobi_ckpt_bytes_read(self._h)
+
+    def load(self, name_or_index, slices: int | None = None, device=None, verify: bool = True, codes=None,
+             sz=None, stream=None):
+        idx = self.find(name_or_index) if isinstance(name_or_index, str) else int(name_or_index)
+        if idx < 0:
+            raise KeyError(name_or_index)
+        _, N, K, G, S = self.info(idx)
+        k = S if slices is None else slices
+        dev = torch.device("cpu") if device is None else torch.device(device)
+        if codes is None:
+            codes = torch.empty((k, N, K // 16), dtype=torch.int32, device=dev)
+        if sz is None:
+            sz = torch.empty((k, K // G, N), dtype=torch.int32, device=dev)
+        host = dev.type == "cpu"
+        _check("mobi_ckpt_load", lib().mobi_ckpt_load(self._h, idx, k, ctypes.c_void_p(codes.data_ptr()),
+                                                      ctypes.c_void_p(sz.data_ptr()), int(host), int(verify),
+                                                      None if host else _stream(stream)))
+        return codes, sz
 
 
 def mobi_gemm_path(X: torch.Tensor, k_t: torch.Tensor, perm: torch.Tensor, offsets: torch.Tensor,

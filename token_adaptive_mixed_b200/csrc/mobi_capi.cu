@@ -44,6 +44,8 @@ cudaError_t note_error(const char* where, cudaError_t e) {
   return e;
 }
 
+void note_message(const char* msg) { snprintf(g_last_error, sizeof g_last_error, "%s", msg); }
+
 // One status block per device, in the module's device memory.
 __device__ DeviceStatus g_device_status;
 
@@ -230,6 +232,7 @@ const char* mobi_status_string(mobi_status st) {
     case MOBI_ERR_WORKSPACE: return "MOBI_ERR_WORKSPACE";
     case MOBI_ERR_CUDA: return "MOBI_ERR_CUDA";
     case MOBI_ERR_TIMEOUT: return "MOBI_ERR_TIMEOUT";
+    case MOBI_ERR_IO: return "MOBI_ERR_IO";
   }
   return "MOBI_ERR_UNKNOWN";
 }
@@ -443,6 +446,55 @@ mobi_status mobi_linear_grouped(const mobi_linear_problem* problems, int count, 
   // writes only k_t, perm and offsets, so the decode kernels may fetch X and
   // the weights before they wait on it.
   return cuda_status(launch_decode_grouped(jobs, count, S, s, dst, true));
+}
+
+static mobi_status check_gemm_grouped(const mobi_gemm_problem* problems, int count, int G, int S, size_t* need) {
+  *need = 0;
+  if (!problems || count < 1 || count > MOBI_MAX_GROUP) return MOBI_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    const mobi_gemm_problem& p = problems[i];
+    mobi_status st = check_matrix(p.N, p.K, G, S);
+    if (st != MOBI_OK) return st;
+    if (p.T < 0) return MOBI_ERR_INVALID_ARG;
+    if (p.T > 16) return MOBI_ERR_UNSUPPORTED_SHAPE;
+    if (p.T == 0 || p.N == 0) continue;
+    if (p.K == 0) return MOBI_ERR_UNSUPPORTED_SHAPE;
+    if (!p.X || !p.k_t || !p.codes || !p.sz || !p.Y) return MOBI_ERR_INVALID_ARG;
+    if (!aligned16(p.X) || !aligned16(p.codes) || !aligned16(p.sz) || !aligned16(p.Y) || !aligned4(p.k_t))
+      return MOBI_ERR_MISALIGNED;
+    *need += align256(decode_ws_bytes(p.N, p.K));
+  }
+  return MOBI_OK;
+}
+
+size_t mobi_gemm_grouped_workspace_bytes(const mobi_gemm_problem* problems, int count, int S) {
+  size_t need = 0;
+  if (check_gemm_grouped(problems, count, 128, S, &need) != MOBI_OK) return 0;
+  return need;
+}
+
+mobi_status mobi_gemm_grouped(const mobi_gemm_problem* problems, int count, int G, int S, void* ws,
+                              size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  size_t need = 0;
+  mobi_status st = check_gemm_grouped(problems, count, G, S, &need);
+  if (st != MOBI_OK) return st;
+  if (ws && !aligned16(ws)) return MOBI_ERR_MISALIGNED;
+  if (need > 0 && (!ws || ws_bytes < need)) return MOBI_ERR_WORKSPACE;
+  cudaError_t e;
+  DeviceStatus* dst = device_status(&e);
+  if (!dst) return cuda_status(e);
+  DecodeJob jobs[MOBI_MAX_GROUP];
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  for (int i = 0; i < count; ++i) {
+    const mobi_gemm_problem& p = problems[i];
+    jobs[i] = DecodeJob{p.X, p.k_t, p.codes, p.sz, p.Y, nullptr, p.N, p.K, (int)p.T};
+    if (p.T > 0 && p.N > 0) {
+      jobs[i].partial = reinterpret_cast<float*>(w);
+      w += align256(decode_ws_bytes(p.N, p.K));
+    }
+  }
+  return cuda_status(launch_decode_grouped(jobs, count, S, static_cast<cudaStream_t>(stream), dst, false));
 }
 
 mobi_status mobi_gemm(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,

@@ -652,13 +652,38 @@ static cudaError_t decode_class(const DecodeJob* jobs, const int* idx, int n, in
   memset(&grp, 0, sizeof grp);
   grp.G = n;
   grp.S = S;
-  int ctas = 0;
+  // CTAs per chunk: each problem's share of the SMs by weight count, rounded
+  // down (at least 1, at most one per 32-row block); then the SMs left over go,
+  // one chunk-width at a time, to the problem with the most weights per CTA.
+  int64_t cpcs[kMaxGroup], used = 0;
   for (int m = 0; m < n; ++m) {
     const DecodeJob& j = jobs[idx[m]];
     const int64_t nch = dec_chunks(j.K), nblocks = (j.N + kDecRows - 1) / kDecRows;
     int64_t cpc = (int64_t)((double)sms * ((double)j.N * (double)j.K / wsum) / (double)nch);
     if (cpc > nblocks) cpc = nblocks;
     if (cpc < 1) cpc = 1;
+    cpcs[m] = cpc;
+    used += cpc * nch;
+  }
+  while (true) {
+    int best = -1;
+    double best_load = 0.0;
+    for (int m = 0; m < n; ++m) {
+      const DecodeJob& j = jobs[idx[m]];
+      const int64_t nch = dec_chunks(j.K), nblocks = (j.N + kDecRows - 1) / kDecRows;
+      if (cpcs[m] >= nblocks || used + nch > sms) continue;
+      const double load = (double)j.N * (double)j.K / (double)(cpcs[m] * nch);
+      if (load > best_load) { best_load = load; best = m; }
+    }
+    if (best < 0) break;
+    ++cpcs[best];
+    used += dec_chunks(jobs[idx[best]].K);
+  }
+  int ctas = 0;
+  for (int m = 0; m < n; ++m) {
+    const DecodeJob& j = jobs[idx[m]];
+    const int64_t nch = dec_chunks(j.K), nblocks = (j.N + kDecRows - 1) / kDecRows;
+    const int64_t cpc = cpcs[m];
     if (!make_tmap_2d(&grp.tm_codes[m], j.codes, 4, (uint64_t)(j.K / 16), (uint64_t)(S * j.N),
                       (uint64_t)(j.K / 16) * 4, 32, kDecRows, 128))
       return note_error("decode tensor map (codes)", cudaErrorInvalidValue);

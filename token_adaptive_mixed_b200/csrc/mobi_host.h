@@ -19,6 +19,8 @@ DeviceStatus* device_status(cudaError_t* err);
 uint64_t wait_limit();
 // Record a failure description for mobi_last_error (thread-local) and return e.
 cudaError_t note_error(const char* where, cudaError_t e);
+// Record a plain message for mobi_last_error.
+void note_message(const char* msg);
 // Multiprocessor count of the current device (cached).
 int num_sms();
 // Opt a kernel into `bytes` of dynamic shared memory (idempotent).
