@@ -56,6 +56,8 @@ def _load():
             lib.oracle_reconstruct.restype = None
             lib.oracle_route.argtypes = [p, i64, i64, p, p, ci, p, p, p, ci]
             lib.oracle_route.restype = None
+            lib.oracle_pack_bits.argtypes = [p, i64, i64, ci, ci, ci, p, p, p, ci]
+            lib.oracle_pack_bits.restype = ci
             lib.oracle_route_mlp.argtypes = [p, i64, i64, p, p, i64, p, p, ci, ctypes.c_double, ctypes.c_double,
                                              p, p, p, ci]
             lib.oracle_route_mlp.restype = ci
@@ -97,6 +99,21 @@ def pack(W_f16: np.ndarray, G: int = 128, S: int = 3, nthreads: int = 0):
     rc = lib.oracle_pack(_ptr(W), N, K, G, S, _ptr(codes), _ptr(sz), _ptr(q), nthreads)
     if rc != 0:
         raise ValueError("oracle_pack: unsupported arguments")
+    return codes, sz, q
+
+
+def pack_bits(W_f16: np.ndarray, G: int = 128, S: int = 3, bits: int = 2, nthreads: int = 0):
+    """MoBiSlice packing with `bits`-bit slices (1 or 2) over G-wide groups.
+    Returns (codes uint32 [S,N,K/16], sz uint32 [S,K/G,N], q uint8 [S,N,K])."""
+    lib = _load()
+    W = _u16(W_f16)
+    N, K = W.shape
+    codes = np.zeros((S, N, K // 16), np.uint32)
+    sz = np.zeros((S, K // G, N), np.uint32)
+    q = np.zeros((S, N, K), np.uint8)
+    rc = lib.oracle_pack_bits(_ptr(W), N, K, G, S, bits, _ptr(codes), _ptr(sz), _ptr(q), nthreads)
+    if rc != 0:
+        raise ValueError("oracle_pack_bits: unsupported arguments")
     return codes, sz, q
 
 

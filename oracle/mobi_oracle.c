@@ -30,7 +30,11 @@
  *   an exact tie). Bucketing: stable ascending sort by k_t. Threshold routing
  *   (oracle_route_mlp): a ReLU two-layer MLP gives one score per residual
  *   slice, a slice is active iff sigmoid(score / tau) > delta, and
- *   k_t = 1 + the number of active residual slices.
+ *   k_t = 1 + the number of active residual slices. Generic slicing
+ *   (oracle_pack_bits): the same quantiser with b-bit codes, L = 2^b - 1 steps
+ *   (s = (max-min)/L, z and q clamped to [0, L]) over G-wide groups; 1-bit
+ *   slices give 1..S bits per weight ([en] §2.A lists 3-bit precision, which
+ *   2-bit slices cannot reach).
  *
  * Parity pins: every function here is pinned by tests/test_oracle.py against
  * closed-form groups, hand-derived packed words, invariants (non-increasing
@@ -91,13 +95,16 @@ int oracle_max_threads(void) {
 
 /*
  * One group of G weights of one row through S rounds of the recursion
- * R_1 = W, W_s = Q(R_s), R_{s+1} = R_s - W_s   ([ja] §2.1, [en] §2.A).
+ * R_1 = W, W_s = Q(R_s), R_{s+1} = R_s - W_s   ([ja] §2.1, [en] §2.A), with Q
+ * the asymmetric min-max round-to-nearest of `bits`-bit codes: L = 2^bits - 1
+ * steps between the group's minimum and maximum.
  * q_out[s*G + i] receives the code of element i in slice s; scale_out[s] and
  * zero_out[s] the fp16 bit patterns of that slice's scale and zero.
  */
-static void quantise_group(const uint16_t* w, int G, int S, uint8_t* q_out,
+static void quantise_group(const uint16_t* w, int G, int S, int bits, uint8_t* q_out,
                            uint16_t* scale_out, uint16_t* zero_out) {
   float R[1024];
+  const float L = (float)((1 << bits) - 1); /* 2 bits: 4 levels, 3 steps; 1 bit: 1 step */
   for (int i = 0; i < G; ++i) R[i] = half_bits_to_float(w[i]);
   for (int s = 0; s < S; ++s) {
     float mn = R[0], mx = R[0];
@@ -105,18 +112,18 @@ static void quantise_group(const uint16_t* w, int G, int S, uint8_t* q_out,
       if (R[i] < mn) mn = R[i];
       if (R[i] > mx) mx = R[i];
     }
-    float sc = (mx - mn) / 3.0f;           /* 2 bits: 4 levels, 3 steps */
+    float sc = (mx - mn) / L;
     if (sc < 0x1p-14f) sc = 0x1p-14f;      /* degenerate group: smallest normal fp16 */
     uint16_t scale_bits = float_to_half_bits(sc);
     float step = half_bits_to_float(scale_bits); /* the stored scale is the one used */
     float zf = rintf(-mn / step);
     if (zf < 0.0f) zf = 0.0f;
-    if (zf > 3.0f) zf = 3.0f;
+    if (zf > L) zf = L;
     int z = (int)zf;
     for (int i = 0; i < G; ++i) {
       float qf = rintf(R[i] / step) + (float)z;
       if (qf < 0.0f) qf = 0.0f;
-      if (qf > 3.0f) qf = 3.0f;
+      if (qf > L) qf = L;
       int q = (int)qf;
       q_out[s * G + i] = (uint8_t)q;
       float deq = (float)(q - z) * step; /* exact: |q-z| <= 3 times an fp16 */
@@ -128,15 +135,17 @@ static void quantise_group(const uint16_t* w, int G, int S, uint8_t* q_out,
 }
 
 /*
- * oracle_pack: W fp16 [N][K] -> codes (the documented 2-bit word layout:
- * word (s, n, w) holds q(s, n, 16w + i) in bits [2i+1:2i]) and sz [S][K/G][N]
- * (fp16 scale in bits [15:0], fp16 zero in bits [31:16]), plus, if q_out is
- * not NULL, the unpacked codes uint8 [S][N][K].
+ * oracle_pack_bits: W fp16 [N][K] -> codes and sz for S slices of `bits`-bit
+ * codes (bits 1 or 2) over G-wide groups. Codes of either width sit in the
+ * documented 2-bit word layout (word (s, n, w) holds q(s, n, 16w + i) in bits
+ * [2i+1:2i]; a 1-bit code only uses values 0 and 1). sz is [S][K/G][N] (fp16
+ * scale in bits [15:0], fp16 zero in bits [31:16]). If q_out is not NULL it
+ * receives the unpacked codes uint8 [S][N][K].
  * Returns 0, or -1 on an unsupported argument.
  */
-int oracle_pack(const uint16_t* W, int64_t N, int64_t K, int G, int S,
-                uint32_t* codes, uint32_t* sz, uint8_t* q_out, int nthreads) {
-  if (G <= 0 || G > 1024 || K % G != 0 || K % 16 != 0 || S < 1 || S > 8) return -1;
+int oracle_pack_bits(const uint16_t* W, int64_t N, int64_t K, int G, int S, int bits,
+                     uint32_t* codes, uint32_t* sz, uint8_t* q_out, int nthreads) {
+  if (G <= 0 || G > 1024 || K % G != 0 || K % 16 != 0 || S < 1 || S > 8 || bits < 1 || bits > 2) return -1;
   set_threads(nthreads);
   const int64_t ngroups = K / G;
   const int64_t nwords = K / 16;
@@ -146,7 +155,7 @@ int oracle_pack(const uint16_t* W, int64_t N, int64_t K, int G, int S,
     uint16_t sc[8], zr[8];
     uint8_t* row_codes = (uint8_t*)malloc((size_t)S * (size_t)K);
     for (int64_t g = 0; g < ngroups; ++g) {
-      quantise_group(W + n * K + g * G, G, S, q, sc, zr);
+      quantise_group(W + n * K + g * G, G, S, bits, q, sc, zr);
       for (int s = 0; s < S; ++s) {
         sz[((int64_t)s * ngroups + g) * N + n] = (uint32_t)sc[s] | ((uint32_t)zr[s] << 16);
         for (int i = 0; i < G; ++i) row_codes[(int64_t)s * K + g * G + i] = q[s * G + i];
@@ -165,6 +174,15 @@ int oracle_pack(const uint16_t* W, int64_t N, int64_t K, int G, int S,
     free(row_codes);
   }
   return 0;
+}
+
+/*
+ * oracle_pack: the 2-bit slicing (the method's configuration): oracle_pack_bits
+ * with bits = 2.
+ */
+int oracle_pack(const uint16_t* W, int64_t N, int64_t K, int G, int S,
+                uint32_t* codes, uint32_t* sz, uint8_t* q_out, int nthreads) {
+  return oracle_pack_bits(W, N, K, G, S, 2, codes, sz, q_out, nthreads);
 }
 
 /* oracle_unpack: the documented word layout back to codes uint8 [S][N][K]. */

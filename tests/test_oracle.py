@@ -389,3 +389,92 @@ def test_route_mlp_one_slice_and_bad_args(oracle):
     with pytest.raises(ValueError):
         oracle.route_mlp(X, W1, b1, np.zeros((W1.shape[1], 2), np.float32), np.zeros(2, np.float32),
                          tau=0.0, delta=0.5)
+
+
+# ---- generic slicings: b-bit slices over G-wide groups ------------------------
+
+def test_pack_bits_two_is_the_method_packer(oracle):
+    """The generic packer with 2-bit slices and G = 128 is the method's packer."""
+    W = _random_W(32, 512, 21)
+    c0, s0, q0 = oracle.pack(W, S=3)
+    c1, s1, q1 = oracle.pack_bits(W, G=128, S=3, bits=2)
+    assert np.array_equal(c0, c1) and np.array_equal(s0, s1) and np.array_equal(q0, q1)
+
+
+@pytest.mark.parametrize("bits,G", [(1, 128), (1, 256), (2, 256), (2, 512), (1, 64)])
+def test_generic_slice1_matches_torch_fake_quantize(oracle, bits, G):
+    """Slice 1 of b-bit slicing over G-wide groups is one round of asymmetric
+    min-max RTN with 2^b - 1 steps: torch's fake quantiser (quant range
+    [0, 2^b - 1], round half to even) with the oracle's scale and zero gives the
+    oracle's dequantised slice bit for bit."""
+    N, K = 32, 1024
+    W = _random_W(N, K, 22 + bits + G)
+    codes, sz, q = oracle.pack_bits(W, G=G, S=1, bits=bits)
+    assert q.max() <= (1 << bits) - 1
+    scale = (sz[0].T & 0xFFFF).astype(np.uint16).view(F16).astype(np.float32).ravel()
+    zero = (sz[0].T >> 16).astype(np.uint16).view(F16).astype(np.float32).ravel().astype(np.int32)
+    x = torch.from_numpy(W.astype(np.float32).reshape(N * K // G, G))
+    fq = torch.fake_quantize_per_channel_affine(x, torch.from_numpy(scale), torch.from_numpy(zero), 0, 0,
+                                                (1 << bits) - 1)
+    W1 = oracle.reconstruct(codes, sz, N, K, k=1, G=G, S=1)
+    assert np.array_equal(fq.numpy().astype(np.float64).reshape(N, K), W1)
+
+
+@pytest.mark.parametrize("bits", [1, 2])
+def test_generic_scale_matches_torch_minmax_observer(oracle, bits):
+    """torch's MinMax observer with quant range [0, 2^b - 1] computes the step
+    (max - min) / (2^b - 1) in fp32; rounded to fp16 it is the stored scale, here
+    over 256-wide groups."""
+    from torch.ao.quantization.observer import MinMaxObserver
+    N, K, G = 4, 512, 256
+    W = _random_W(N, K, 30 + bits)
+    codes, sz, _ = oracle.pack_bits(W, G=G, S=1, bits=bits)
+    for n in range(N):
+        for g in range(K // G):
+            grp = torch.from_numpy(W[n, g * G:(g + 1) * G].astype(np.float32))
+            obs = MinMaxObserver(dtype=torch.quint8, quant_min=0, quant_max=(1 << bits) - 1)
+            obs(grp)
+            sc, _ = obs.calculate_qparams()
+            assert f16_bits(float(sc.to(torch.float16))) == int(sz[0, g, n] & 0xFFFF)
+
+
+def test_one_bit_hand_group(oracle):
+    """Derived by hand: a 128-group of -1 and 2 (alternating). Slice 1: step
+    (2 - (-1)) / 1 = 3, zero rint(1/3) = 0, codes 0 for -1 and 1 for 2 (2/3 rounds
+    to 1), residual -1 everywhere. Slice 2: a constant group, step floored at
+    2^-14, zero clamped to 1, codes rint(-2^14) + 1 -> clamped to 0, so each
+    residual moves by one step: -1 + 2^-14."""
+    W = group_row([-1.0, 2.0])
+    codes, sz, q = oracle.pack_bits(W, G=128, S=2, bits=1)
+    assert int(sz[0, 0, 0]) == f16_bits(3.0) | (f16_bits(0.0) << 16)
+    assert np.array_equal(q[0, 0], np.tile([0, 1], 64))
+    assert int(codes[0, 0, 0]) == sum(1 << (2 * i) for i in range(1, 16, 2))  # odd fields hold 1
+    assert int(sz[1, 0, 0]) == 0x0400 | (f16_bits(1.0) << 16)  # 2^-14, zero 1
+    assert np.all(q[1, 0] == 0)
+    W2 = oracle.reconstruct(codes, sz, 1, 128, k=2, G=128, S=2)
+    assert np.all(W2[0] == np.tile([0.0 - 2.0 ** -14, 3.0 - 2.0 ** -14], 64))
+
+
+@pytest.mark.parametrize("bits,G", [(1, 128), (1, 256), (2, 256)])
+def test_generic_residual_never_grows(oracle, bits, G):
+    """0 is on the grid for any b (integer zero in [0, 2^b - 1]) and clamping
+    moves toward it, so the residual never grows element by element and the
+    Frobenius error falls with every slice (four 1-bit slices: 1 to 4 bits)."""
+    N, K, S = 64, 1024, 4
+    W = _random_W(N, K, 40 + bits + G, outliers=4)
+    codes, sz, _ = oracle.pack_bits(W, G=G, S=S, bits=bits)
+    Wd = W.astype(np.float64)
+    prev, fro = np.abs(Wd), [np.linalg.norm(Wd)]
+    for k in range(1, S + 1):
+        e = np.abs(Wd - oracle.reconstruct(codes, sz, N, K, k=k, G=G, S=S))
+        assert np.all(e <= prev + 1e-6 * np.abs(Wd) + 1e-9)
+        prev = e
+        fro.append(np.linalg.norm(e))
+    assert all(b < a for a, b in zip(fro[:-1], fro[1:]))
+
+
+def test_pack_bits_rejects_bad_arguments(oracle):
+    W = _random_W(4, 256, 50)
+    for kw in ({"bits": 0}, {"bits": 3}, {"G": 96}):
+        with pytest.raises(ValueError):
+            oracle.pack_bits(W, **{"G": 128, "S": 2, "bits": 2, **kw})
