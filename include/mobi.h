@@ -28,8 +28,9 @@
  *     Calls enqueue work and return without synchronising.
  *   - Arguments are validated on the host before anything is launched; on an
  *     error nothing is enqueued and the status says why.
- *   - Supported shapes: S in {1,2,3} slices of b = 2 bits, group G = 128 along
- *     K, K % 128 == 0, N % 16 == 0, T >= 0. K, N, T up to 2^30 elements per
+ *   - Supported shapes: S in {1,2,3,4} slices of b = 2 bits (or b = 1 bit
+ *     through mobi_pack_bits), group G = 128 along K (256 or 512 through
+ *     mobi_pack_bits), K % 128 == 0, N % 16 == 0, T >= 0. K, N, T up to 2^30 elements per
  *     dimension and N*K, T*K, T*N below 2^40.
  *   - A device-side bounded wait that runs out sets a per-device error word;
  *     the next call on that device (or mobi_sync_check) reports
@@ -45,7 +46,7 @@
  *          k = 16w .. 16w+15; code q(s,n,16w+i) sits in bits [2i+1 : 2i]
  *          (little-endian 2-bit fields). mobi_codes_bytes() gives the size.
  *   sz     uint32 [S][K/G][N]    element (s,g,n): bits [15:0] = fp16 scale,
- *          bits [31:16] = fp16 zero (an integer 0..3). mobi_sz_bytes().
+ *          bits [31:16] = fp16 zero (an integer 0..2^b - 1). mobi_sz_bytes().
  *          Group-major so that the scales of one group for consecutive rows
  *          are contiguous (N*4-byte rows, which tensor copies can stage).
  *   The dequantised slice is deq_s[n,k] = (q(s,n,k) - zero(s,n,k/G)) *
@@ -60,6 +61,8 @@
  *     z  = clamp(rint(-mn / s), 0, 3)
  *     q  = clamp(rint(R / s) + z, 0, 3)          (per element)
  *     R  = R - (q - z) * s                      (the product is exact)
+ * Generic slicing (mobi_pack_bits): the same with b-bit codes, L = 2^b - 1
+ * steps: sc = max((mx - mn) / L, 2^-14), z and q clamped to [0, L].
  */
 #ifndef MOBI_H_
 #define MOBI_H_
@@ -120,13 +123,36 @@ MOBI_API size_t mobi_gemm_workspace_bytes(int64_t T, int64_t N, int64_t K, int S
  *   W        fp16 [N][K] row-major (device). Values must be finite.
  *   N, K     rows and columns; K % G == 0, N % 16 == 0.
  *   G        group size along K; must be 128.
- *   S        number of slices, 1..3.
+ *   S        number of slices, 1..4.
  *   codes    out, uint32 [S][N][K/16] (layout above).
  *   sz       out, uint32 [S][K/G][N]  (fp16 scale | fp16 zero << 16).
  * Bit-exact with the quantiser above (IEEE division, RNE, no flush-to-zero).
  */
 MOBI_API mobi_status mobi_pack(const void* W, int64_t N, int64_t K, int G, int S,
                       uint32_t* codes, uint32_t* sz, void* stream);
+
+/*
+ * mobi_pack_bits — MoBiSlice with generic slicing: S slices of `bits`-bit
+ *   codes over G-wide groups ([en] §2.A lists 2, 3, 4 or 6-bit precisions;
+ *   four 1-bit slices give every width from 1 to 4 bits, three-slice 2-bit
+ *   packing only 2, 4 and 6). The quantiser is the one stated at the top of
+ *   this header with L = 2^bits - 1 steps.
+ *   W, N, K, S, codes  as for mobi_pack (S 1..4; K % G == 0).
+ *   G        128, 256 or 512.
+ *   bits     1 or 2. Codes of either width sit in the 2-bit fields of the
+ *            documented layout (a 1-bit code uses only the values 0 and 1), so
+ *            every GEMM entry point reads them unchanged; a 1-bit slice costs
+ *            the bytes of a 2-bit one.
+ *   sz       out, uint32 [S][K/128][N] whatever G is: the scale/zero word of
+ *            a G-wide group is repeated in each of its G/128 128-column
+ *            sub-groups (size: mobi_sz_bytes(N, K, S, 128)), which is the
+ *            form the GEMM kernels read.
+ * Bit-exact with the quantiser (IEEE division, RNE, no flush-to-zero).
+ * Errors: MOBI_ERR_INVALID_ARG for bits outside 1..2, S outside 1..4 or a
+ * missing pointer; MOBI_ERR_UNSUPPORTED_SHAPE for other G or K % G != 0.
+ */
+MOBI_API mobi_status mobi_pack_bits(const void* W, int64_t N, int64_t K, int G, int S, int bits,
+                                    uint32_t* codes, uint32_t* sz, void* stream);
 
 /*
  * mobi_route — MoBiRoute slice count per token and token bucketing.
@@ -330,7 +356,7 @@ MOBI_API mobi_status mobi_linear_grouped(const mobi_linear_problem* problems, in
  *   table    count entries of 192 bytes: name (96 bytes, NUL-terminated),
  *            i64 N, i64 K, i32 G, i32 S, u64 codes offset, u64 codes bytes per
  *            slice (N K / 4), u64 sz offset, u64 sz bytes per slice (K/G N 4),
- *            u32 CRC-32C of each slice's codes [3] and sz [3], zero padding.
+ *            u32 CRC-32C of each slice's codes [4] and sz [4], zero padding.
  *   data     per tensor its codes block [S][N][K/16] u32 and its sz block
  *            [S][K/G][N] u32, each starting on a 4096-byte boundary.
  * CRC-32C is the Castagnoli CRC (reflected polynomial 0x82F63B78, initial

@@ -54,7 +54,7 @@ def test_pack_validation(L):
     assert L.mobi_pack(p(FAKE), 16, 100, 128, 3, p(FAKE), p(FAKE), None) == 2   # K % 128
     assert L.mobi_pack(p(FAKE), 24, 128, 128, 3, p(FAKE), p(FAKE), None) == 2   # N % 16
     assert L.mobi_pack(p(FAKE), 16, 128, 64, 3, p(FAKE), p(FAKE), None) == 2    # G != 128
-    assert L.mobi_pack(p(FAKE), 16, 128, 128, 4, p(FAKE), p(FAKE), None) == 1   # S > 3
+    assert L.mobi_pack(p(FAKE), 16, 128, 128, 5, p(FAKE), p(FAKE), None) == 1   # S > 4
     assert L.mobi_pack(None, 16, 128, 128, 3, p(FAKE), p(FAKE), None) == 1      # null W
     assert L.mobi_pack(p(FAKE + 2), 16, 128, 128, 3, p(FAKE), p(FAKE), None) == 3  # misaligned
     assert L.mobi_pack(p(FAKE), 0, 128, 128, 3, p(FAKE), p(FAKE), None) == 0    # empty: no-op
@@ -101,7 +101,7 @@ def test_linear_validation(L):
     assert call(K=200) == 2
     assert call(N=24) == 2
     assert call(G=64) == 2
-    assert call(S=4) == 1
+    assert call(S=5) == 1
     assert call(X=None) == 1
     assert call(codes=None) == 1
     assert call(Y=p(FAKE + 4)) == 3
@@ -133,7 +133,7 @@ def test_route_mlp_validation(L):
     assert call(delta=0.0) == 1
     assert call(delta=1.0) == 1
     assert call(delta=float("nan")) == 1
-    assert call(S=0) == 1 and call(S=4) == 1
+    assert call(S=0) == 1 and call(S=5) == 1
     assert call(H=0) == 1
     assert call(T=-1) == 1
     assert call(K=200) == 2
@@ -168,7 +168,7 @@ def test_linear_grouped_validation(L):
     assert call([prob(), prob(K=200)]) == 2
     assert call([prob(), prob(N=24)]) == 2
     assert call([prob()], G=64) == 2
-    assert call([prob()], S=4) == 1
+    assert call([prob()], S=5) == 1
     assert call([prob(), prob(X=None)]) == 1
     assert call([prob(), prob(codes=None)]) == 1
     assert call([prob(), prob(Y=FAKE + 4)]) == 3
@@ -178,7 +178,7 @@ def test_linear_grouped_validation(L):
     need = L.mobi_linear_grouped_workspace_bytes(arr, 2, 3)
     per = [L.mobi_linear_grouped_workspace_bytes((P * 1)(arr[i]), 1, 3) for i in range(2)]
     assert need == sum(per) and all(b % 256 == 0 and b > 0 for b in per)
-    assert L.mobi_linear_grouped_workspace_bytes(arr, 2, 4) == 0
+    assert L.mobi_linear_grouped_workspace_bytes(arr, 2, 5) == 0
 
 
 def test_gemm_grouped_validation(L):
@@ -201,3 +201,18 @@ def test_gemm_grouped_validation(L):
     arr = (P * 2)(prob(T=4), prob(T=16, N=11008))
     assert L.mobi_gemm_grouped_workspace_bytes(arr, 2, 3) == sum(
         L.mobi_gemm_grouped_workspace_bytes((P * 1)(arr[i]), 1, 3) for i in range(2))
+
+
+def test_pack_bits_validation(L):
+    p = ctypes.c_void_p
+
+    def call(N=16, K=512, G=256, S=4, bits=1, W=p(FAKE), codes=p(FAKE)):
+        return L.mobi_pack_bits(W, N, K, G, S, bits, codes, p(FAKE), None)
+    assert call(bits=0) == 1 and call(bits=3) == 1
+    assert call(S=5) == 1 and call(S=0) == 1
+    assert call(G=64) == 2 and call(G=384) == 2
+    assert call(K=384, G=256) == 2          # K % G
+    assert call(N=24) == 2
+    assert call(W=None) == 1 and call(codes=None) == 1
+    assert call(W=p(FAKE + 2)) == 3
+    assert call(N=0) == 0                   # empty: no-op

@@ -73,7 +73,7 @@ def test_format_as_documented(ckpt_file):
         e = raw[toff + 192 * i: toff + 192 * (i + 1)]
         assert e[:96].split(b"\0")[0].decode() == name
         n, k, g, s, coff, cslice, zoff, zslice = struct.unpack_from("<qqiiQQQQ", e, 96)
-        crcs = struct.unpack_from("<6I", e, 96 + 56)
+        crcs = struct.unpack_from("<8I", e, 96 + 56)
         assert (n, k, g, s) == (N, K, 128, S)
         assert cslice == N * K // 4 and zslice == (K // 128) * N * 4
         assert coff % 4096 == 0 and zoff % 4096 == 0
@@ -82,8 +82,8 @@ def test_format_as_documented(ckpt_file):
             cb = raw[coff + sl * cslice: coff + (sl + 1) * cslice]
             zb = raw[zoff + sl * zslice: zoff + (sl + 1) * zslice]
             assert cb == codes[sl].tobytes() and zb == sz[sl].tobytes()
-            assert crcs[sl] == crc32c_bitwise(cb) and crcs[3 + sl] == crc32c_bitwise(zb)
-        assert all(c == 0 for c in crcs[S:3]) and all(c == 0 for c in crcs[3 + S:])
+            assert crcs[sl] == crc32c_bitwise(cb) and crcs[4 + sl] == crc32c_bitwise(zb)
+        assert all(c == 0 for c in crcs[S:4]) and all(c == 0 for c in crcs[4 + S:])
 
 
 def test_load_every_slice_count(ckpt_file):

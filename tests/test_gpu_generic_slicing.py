@@ -1,0 +1,127 @@
+"""Generic slicing on the GPU: b-bit slices (b = 1, 2) over G-wide groups
+(G = 128, 256, 512) and up to four slices, against the CPU oracle.
+
+Pack: codes bit-exact; the scale/zero words bit-exact after repeating each
+G-wide group's word over its G/128 sub-groups (the layout the GEMM kernels
+read). GEMMs, routing and bucketing: the bars of the other parity tests, with
+the oracle computing at the native group width.
+"""
+import numpy as np
+import pytest
+import torch
+
+from parity import check_gemm, check_route
+from token_adaptive_mixed_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def mobi():
+    import token_adaptive_mixed_b200 as m
+    from token_adaptive_mixed_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+    m.lib()
+    return m
+
+
+def expand_sz(sz, G):
+    """Oracle sz [S][K/G][N] -> the GPU layout [S][K/128][N]."""
+    return np.repeat(sz, G // 128, axis=1)
+
+
+@pytest.mark.parametrize("bits,G,S,N,K", [(1, 128, 4, 256, 1024), (1, 256, 4, 80, 2304), (2, 256, 3, 128, 4096),
+                                          (2, 512, 2, 48, 1024), (1, 512, 3, 64, 11264), (2, 128, 4, 32, 384)])
+def test_pack_generic_bit_exact(mobi, oracle, bits, G, S, N, K):
+    L = wl.layer("gp", N, K, 1, seed=2000 + bits + G + S, outlier_frac_cols=0.01)
+    codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(DEV), S=S, G=G, bits=bits)
+    torch.cuda.synchronize()
+    c_ref, s_ref, q_ref = oracle.pack_bits(L.W, G=G, S=S, bits=bits)
+    assert np.array_equal(codes.cpu().numpy().view(np.uint32), c_ref)
+    assert np.array_equal(sz.cpu().numpy().view(np.uint32), expand_sz(s_ref, G))
+    assert q_ref.max() <= (1 << bits) - 1
+
+
+def _layer_s(name, N, K, T, S, seed, mix=None):
+    return wl.layer(name, N, K, T, seed=seed, outlier_frac_cols=0.005, S=S,
+                    mix=mix if mix is not None else tuple([1.0 / S] * S))
+
+
+@pytest.mark.parametrize("T", [1, 4, 16, 300])
+@pytest.mark.parametrize("bits,G", [(1, 128), (1, 256)])
+def test_four_slice_linear(mobi, oracle, T, bits, G):
+    """Four b-bit slices (1..4 bits for b = 1) through route + GEMM (decode for
+    T <= 16, tcgen05 prefill for T = 300)."""
+    N, K, S = 512, 2048, 4
+    L = _layer_s("l4", N, K, T, S, seed=2100 + T + bits + G)
+    codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(DEV), S=S, G=G, bits=bits)
+    Wr = torch.from_numpy(L.Wr).to(DEV)
+    b = torch.from_numpy(L.bias).to(DEV)
+    Y, k_t, perm, off = mobi.mobi_linear(L.X.to(DEV), Wr, b, codes, sz, N)
+    mobi.mobi_sync_check()
+    tag = f"S=4 b={bits} G={G} T={T}"
+    k_gpu = k_t.cpu().numpy()
+    k_ref, gap, _ = oracle.route(L.X, L.Wr, L.bias)
+    check_route(k_gpu, k_ref, gap, tag)
+    perm_ref, off_ref = oracle.bucket(k_gpu, S)
+    assert np.array_equal(perm.cpu().numpy(), perm_ref) and np.array_equal(off.cpu().numpy(), off_ref)
+    c_ref, s_ref, _ = oracle.pack_bits(L.W, G=G, S=S, bits=bits)
+    check_gemm(Y.cpu().numpy(), oracle.gemm(L.X, k_gpu, c_ref, s_ref, N, G=G, S=S), tag)
+    if T > 1:
+        assert len(set(k_gpu.tolist())) > 1, "the mix should use several precisions"
+
+
+def test_four_slice_grouped_and_checkpoint(mobi, oracle, tmp_path):
+    """Grouped decode step and a checkpoint of 4-slice layers: the grouped
+    results equal single calls, and a checkpoint loaded at 2 slices serves
+    tokens routed to at most 2 slices exactly like the full pack."""
+    S = 4
+    specs = [(256, 1024, 3), (512, 2048, 16), (128, 512, 8)]
+    probs, layers = [], []
+    for i, (N, K, T) in enumerate(specs):
+        L = _layer_s("g4", N, K, T, S, seed=2200 + i)
+        codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(DEV), S=S, bits=1)
+        layers.append(L)
+        probs.append({"X": L.X.to(DEV), "Wr": torch.from_numpy(L.Wr).to(DEV), "bias": torch.from_numpy(L.bias).to(DEV),
+                      "codes": codes, "sz": sz, "N": N})
+    outs = mobi.mobi_linear_grouped(probs, S=S)
+    mobi.mobi_sync_check()
+    for pr, (Y, k_t, perm, off) in zip(probs, outs):
+        Ys, ks, _, _ = mobi.mobi_linear(pr["X"], pr["Wr"], pr["bias"], pr["codes"], pr["sz"], pr["N"])
+        assert torch.equal(Y, Ys) and torch.equal(k_t, ks)
+    path = tmp_path / "four.mobi"
+    mobi.mobi_ckpt_save(path, [(f"p{i}", pr["codes"], pr["sz"]) for i, pr in enumerate(probs)])
+    with mobi.MobiCheckpoint(path) as ck:
+        for i, (pr, L) in enumerate(zip(probs, layers)):
+            c2, z2 = ck.load(f"p{i}", 2, device=DEV)
+            assert torch.equal(c2, pr["codes"][:2]) and torch.equal(z2, pr["sz"][:2])
+            k_np = np.random.default_rng(i).integers(1, 3, L.T).astype(np.int32)
+            perm_np, off2 = oracle.bucket(k_np, 2)
+            _, off4 = oracle.bucket(k_np, 4)
+            k_t = torch.from_numpy(k_np).to(DEV)
+            perm = torch.from_numpy(perm_np).to(DEV)
+            Y2 = mobi.mobi_gemm(pr["X"], k_t, perm, torch.from_numpy(off2).to(DEV), c2, z2, pr["N"])
+            Y4 = mobi.mobi_gemm(pr["X"], k_t, perm, torch.from_numpy(off4).to(DEV), pr["codes"], pr["sz"], pr["N"])
+            mobi.mobi_sync_check()
+            assert torch.equal(Y2, Y4)
+
+
+def test_four_slice_threshold_routing(mobi, oracle):
+    """Threshold routing with three residual slices (S = 4)."""
+    from parity import check_route_mlp, mlp_score_bound
+    R = wl.mlp_router("mlp4", 200, 1024, 64, seed=2300, S=4)
+    W1 = torch.from_numpy(R.W1).to(DEV)
+    W2 = torch.from_numpy(np.ascontiguousarray(R.W2)).to(DEV)
+    k_t, perm, off = mobi.mobi_route_mlp(R.X.to(DEV), W1, torch.from_numpy(R.b1).to(DEV), W2,
+                                         torch.from_numpy(R.b2).to(DEV), 1.0, 0.5)
+    mobi.mobi_sync_check()
+    k_gpu = k_t.cpu().numpy()
+    k_ref, _, scores = oracle.route_mlp(R.X, R.W1, R.b1, R.W2, R.b2, 1.0, 0.5)
+    check_route_mlp(k_gpu, scores, mlp_score_bound(R.X.float().numpy(), R.W1, R.b1, R.W2, R.b2, 0.0), 0.0,
+                    "mlp S=4")
+    perm_ref, off_ref = oracle.bucket(k_gpu, 4)
+    assert np.array_equal(perm.cpu().numpy(), perm_ref) and np.array_equal(off.cpu().numpy(), off_ref)
+    assert k_gpu.max() == 4 and len(set(k_gpu.tolist())) >= 3

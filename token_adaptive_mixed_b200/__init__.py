@@ -7,7 +7,7 @@ library's sm_100a kernels. There is no CPU fallback: if the library is missing
 or a tensor is not on a CUDA device, the call raises.
 
 Entry points (same names as the C ABI):
-  mobi_pack(W)                      MoBiSlice packing   -> (codes, sz)
+  mobi_pack(W, S, G, bits)          MoBiSlice packing   -> (codes, sz)
   mobi_route(X, Wr, bias)           MoBiRoute routing   -> (k_t, perm, offsets)
   mobi_route_mlp(X, W1, b1, W2, b2, tau, delta)  threshold routing, MLP scorer -> (k_t, perm, offsets)
   mobi_gemm(X, k_t, perm, offsets, codes, sz, N)         -> Y  (fp32)
@@ -73,7 +73,7 @@ EXPORTED_SYMBOLS = (
     "mobi_route_mlp", "mobi_route_mlp_workspace_bytes", "mobi_linear_grouped", "mobi_linear_grouped_workspace_bytes",
     "mobi_gemm_grouped", "mobi_gemm_grouped_workspace_bytes",
     "mobi_ckpt_save", "mobi_ckpt_open", "mobi_ckpt_count", "mobi_ckpt_find", "mobi_ckpt_info", "mobi_ckpt_load",
-    "mobi_ckpt_bytes_read", "mobi_ckpt_close", "mobi_crc32c",
+    "mobi_ckpt_bytes_read", "mobi_ckpt_close", "mobi_crc32c", "mobi_pack_bits",
 )
 
 
@@ -112,6 +112,8 @@ def lib() -> ctypes.CDLL:
         L.mobi_gemm_workspace_bytes.restype = sz_t
         L.mobi_pack.argtypes = [p, i64, i64, ci, ci, p, p, p]
         L.mobi_pack.restype = ci
+        L.mobi_pack_bits.argtypes = [p, i64, i64, ci, ci, ci, p, p, p]
+        L.mobi_pack_bits.restype = ci
         L.mobi_route.argtypes = [p, i64, i64, p, p, ci, p, p, p, p, sz_t, p]
         L.mobi_route.restype = ci
         L.mobi_gemm.argtypes = [p, i64, i64, p, p, p, p, p, i64, ci, ci, p, p, sz_t, p]
@@ -220,16 +222,22 @@ def _workspace(nbytes: int, device, ws: torch.Tensor | None) -> torch.Tensor:
 
 
 def mobi_pack(W: torch.Tensor, S: int = 3, G: int = 128, codes: torch.Tensor | None = None,
-              sz: torch.Tensor | None = None, stream=None):
-    """MoBiSlice packing of fp16 W[N,K] -> (codes int32 [S,N,K/16], sz int32 [S,K/G,N])."""
+              sz: torch.Tensor | None = None, stream=None, bits: int = 2):
+    """MoBiSlice packing of fp16 W[N,K] -> (codes int32 [S,N,K/16], sz int32 [S,K/128,N]).
+    bits = 2 and G = 128 is the method's slicing (mobi_pack); other values go
+    through mobi_pack_bits (bits 1 or 2, G 128/256/512, S up to 4)."""
     if W.dtype != torch.float16 or W.dim() != 2:
         raise ValueError("W must be a 2-D fp16 tensor")
     N, K = W.shape
     if codes is None:
         codes = torch.empty((S, N, K // 16), dtype=torch.int32, device=W.device)
     if sz is None:
-        sz = torch.empty((S, K // G, N), dtype=torch.int32, device=W.device)
-    _check("mobi_pack", lib().mobi_pack(_ptr(W), N, K, G, S, _ptr(codes), _ptr(sz), _stream(stream)))
+        sz = torch.empty((S, K // 128, N), dtype=torch.int32, device=W.device)
+    if bits == 2 and G == 128:
+        _check("mobi_pack", lib().mobi_pack(_ptr(W), N, K, G, S, _ptr(codes), _ptr(sz), _stream(stream)))
+    else:
+        _check("mobi_pack_bits", lib().mobi_pack_bits(_ptr(W), N, K, G, S, bits, _ptr(codes), _ptr(sz),
+                                                      _stream(stream)))
     return codes, sz
 
 

@@ -19,7 +19,7 @@ namespace mobi {
 
 // Launchers defined in the kernel files.
 cudaError_t launch_pack(const void* W, int64_t N, int64_t K, int S, uint32_t* codes, uint32_t* sz,
-                        cudaStream_t stream, int num_sms);
+                        cudaStream_t stream, int num_sms, int bits, int G);
 cudaError_t launch_route(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias, int S,
                          int32_t* k_t, int32_t* perm, int32_t* offsets, void* ws, cudaStream_t stream);
 size_t route_ws_bytes(int64_t T, int64_t K, int S);
@@ -211,7 +211,7 @@ mobi_status cuda_status(cudaError_t e) {
 }
 
 mobi_status check_matrix(int64_t N, int64_t K, int G, int S) {
-  if (N < 0 || K < 0 || S < 1 || S > 3) return MOBI_ERR_INVALID_ARG;
+  if (N < 0 || K < 0 || S < 1 || S > kMaxSlices) return MOBI_ERR_INVALID_ARG;
   if (G != 128) return MOBI_ERR_UNSUPPORTED_SHAPE;
   if (K % 128 != 0 || N % 16 != 0 || N > kMaxDim || K > kMaxDim) return MOBI_ERR_UNSUPPORTED_SHAPE;
   return MOBI_OK;
@@ -242,22 +242,22 @@ const char* mobi_last_error(void) { return g_last_error; }
 int mobi_version(void) { return 100; }
 
 size_t mobi_codes_bytes(int64_t N, int64_t K, int S) {
-  if (N < 0 || K < 0 || K % 16 != 0 || S < 1 || S > 3) return 0;
+  if (N < 0 || K < 0 || K % 16 != 0 || S < 1 || S > kMaxSlices) return 0;
   return (size_t)S * (size_t)N * (size_t)(K / 16) * 4;
 }
 
 size_t mobi_sz_bytes(int64_t N, int64_t K, int S, int G) {
-  if (N < 0 || K < 0 || G <= 0 || K % G != 0 || S < 1 || S > 3) return 0;
+  if (N < 0 || K < 0 || G <= 0 || K % G != 0 || S < 1 || S > kMaxSlices) return 0;
   return (size_t)S * (size_t)N * (size_t)(K / G) * 4;
 }
 
 size_t mobi_route_workspace_bytes(int64_t T, int64_t K, int S) {
-  if (T < 0 || K < 0 || S < 1 || S > 3) return 0;
+  if (T < 0 || K < 0 || S < 1 || S > kMaxSlices) return 0;
   return route_ws_bytes(T, K, S);
 }
 
 size_t mobi_gemm_workspace_bytes(int64_t T, int64_t N, int64_t K, int S) {
-  if (T < 0 || N < 0 || K < 0 || S < 1 || S > 3) return 0;
+  if (T < 0 || N < 0 || K < 0 || S < 1 || S > kMaxSlices) return 0;
   size_t b = decode_ws_bytes(N, K);
   const size_t p = prefill_ws_bytes(T, N, K);  // either kernel may be chosen (mobi_gemm_path)
   if (p > b) b = p;
@@ -272,13 +272,27 @@ mobi_status mobi_pack(const void* W, int64_t N, int64_t K, int G, int S, uint32_
   if (N == 0 || K == 0) return MOBI_OK;
   if (!W || !codes || !sz) return MOBI_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(codes) || !aligned16(sz)) return MOBI_ERR_MISALIGNED;
-  return cuda_status(launch_pack(W, N, K, S, codes, sz, static_cast<cudaStream_t>(stream), num_sms()));
+  return cuda_status(launch_pack(W, N, K, S, codes, sz, static_cast<cudaStream_t>(stream), num_sms(), 2, 128));
+}
+
+mobi_status mobi_pack_bits(const void* W, int64_t N, int64_t K, int G, int S, int bits, uint32_t* codes,
+                           uint32_t* sz, void* stream) {
+  g_last_error[0] = 0;
+  if (bits < 1 || bits > 2) return MOBI_ERR_INVALID_ARG;
+  if (G != 128 && G != 256 && G != 512) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  mobi_status st = check_matrix(N, K, 128, S);
+  if (st != MOBI_OK) return st;
+  if (K % G != 0) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  if (N == 0 || K == 0) return MOBI_OK;
+  if (!W || !codes || !sz) return MOBI_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(codes) || !aligned16(sz)) return MOBI_ERR_MISALIGNED;
+  return cuda_status(launch_pack(W, N, K, S, codes, sz, static_cast<cudaStream_t>(stream), num_sms(), bits, G));
 }
 
 mobi_status mobi_route(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias, int S,
                        int32_t* k_t, int32_t* perm, int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
   g_last_error[0] = 0;
-  if (T < 0 || K < 0 || S < 1 || S > 3) return MOBI_ERR_INVALID_ARG;
+  if (T < 0 || K < 0 || S < 1 || S > kMaxSlices) return MOBI_ERR_INVALID_ARG;
   if (K % 128 != 0 || K > kMaxDim || T > kMaxDim) return MOBI_ERR_UNSUPPORTED_SHAPE;
   if (!offsets || (T > 0 && (!X || !Wr || !k_t || !perm))) return MOBI_ERR_INVALID_ARG;
   if (T > 0 && K == 0) return MOBI_ERR_UNSUPPORTED_SHAPE;
@@ -301,7 +315,7 @@ mobi_status mobi_route_mlp(const void* X, int64_t T, int64_t K, const float* W1,
                            const float* W2, const float* b2, int S, double tau, double delta, int32_t* k_t,
                            int32_t* perm, int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
   g_last_error[0] = 0;
-  if (T < 0 || K < 0 || H < 1 || S < 1 || S > 3) return MOBI_ERR_INVALID_ARG;
+  if (T < 0 || K < 0 || H < 1 || S < 1 || S > kMaxSlices) return MOBI_ERR_INVALID_ARG;
   if (!(tau > 0.0) || !std::isfinite(tau) || !(delta > 0.0 && delta < 1.0)) return MOBI_ERR_INVALID_ARG;
   if (K % 128 != 0 || K > kMaxDim || T > kMaxDim || H > kMaxMlpHidden) return MOBI_ERR_UNSUPPORTED_SHAPE;
   if (!offsets || (T > 0 && (!X || !k_t || !perm))) return MOBI_ERR_INVALID_ARG;
@@ -348,7 +362,7 @@ mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const int32_t* k
 }
 
 size_t mobi_linear_workspace_bytes(int64_t T, int64_t N, int64_t K, int S) {
-  if (T < 0 || N < 0 || K < 0 || S < 1 || S > 3) return 0;
+  if (T < 0 || N < 0 || K < 0 || S < 1 || S > kMaxSlices) return 0;
   return align256(route_ws_bytes(T, K, S)) + mobi_gemm_workspace_bytes(T, N, K, S);
 }
 

@@ -35,7 +35,6 @@ constexpr size_t kEntryBytes = 192;
 constexpr size_t kNameBytes = 96;
 constexpr uint64_t kAlign = 4096;
 constexpr size_t kStageBytes = size_t(16) << 20;  // per pinned staging buffer
-constexpr int kMaxSlices = 3;
 
 struct Entry {
   char name[kNameBytes];

@@ -803,7 +803,7 @@ extern "C" mobi_status mobi_gemm_decode_noalloc(const void* X, int64_t T, int64_
                                                 int S, float* Y, void* stream) {
   using namespace mobi;
   auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-  if (N < 0 || K < 0 || T < 0 || S < 1 || S > 3) return MOBI_ERR_INVALID_ARG;
+  if (N < 0 || K < 0 || T < 0 || S < 1 || S > kMaxSlices) return MOBI_ERR_INVALID_ARG;
   if (G != 128 || K % 128 != 0 || N % 16 != 0 || T > 16 || N > (int64_t(1) << 28) || K > (int64_t(1) << 28))
     return MOBI_ERR_UNSUPPORTED_SHAPE;
   if (T == 0 || N == 0) return MOBI_OK;

@@ -2,13 +2,18 @@
 //
 // MoBiQuant explainer [ja] §2.1 / [en] §2.A: R_1 = W, W_s = Q(R_s),
 // R_{s+1} = R_s - W_s, with Q the asymmetric min-max round-to-nearest of each
-// 128-wide group (the quantiser written out in include/mobi.h).
+// G-wide group (the quantiser written out in include/mobi.h): b-bit codes,
+// L = 2^b - 1 steps (b = 2 for the method's slices, b = 1 for generic ones),
+// G = 128, 256 or 512.
 //
-// Work split: one warp per (row n, chunk of 4 groups = 512 columns); lane l
-// owns the 16 consecutive weights k = 512c + 16l .. +15, i.e. exactly one
-// packed word per slice. The 8 lanes of a group reduce min/max with three xor
-// shuffles. Codes leave as 128-bit stores (4 lanes' words gathered into one
-// lane), so each slice's 128 bytes per warp are one coalesced transaction.
+// Work split: one warp per (row n, chunk of 512 columns); lane l owns the 16
+// consecutive weights k = 512c + 16l .. +15, i.e. exactly one packed word per
+// slice. The G/16 lanes of a group reduce min/max with xor shuffles. Codes of
+// either width sit in 2-bit fields and leave as 128-bit stores (4 lanes' words
+// gathered into one lane), so each slice's 128 bytes per warp are one
+// coalesced transaction. Scale/zero words are written per 128-column
+// sub-group, so a wider group's word appears once per sub-group (the layout
+// the GEMM kernels read).
 //
 // Bit-exactness: IEEE division (__fdiv_rn), round-to-nearest-even (rintf,
 // __float2half_rn), explicit _rn multiply/subtract so that nothing is
@@ -21,8 +26,9 @@
 namespace mobi {
 
 __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W, int64_t N, int64_t K,
-                                                   int S, uint32_t* __restrict__ codes,
+                                                   int S, int bits, int glanes, uint32_t* __restrict__ codes,
                                                    uint32_t* __restrict__ sz) {
+  const float L = (float)((1 << bits) - 1);  // steps between min and max
   const int lane = threadIdx.x & 31;
   const int64_t ngroups = K / 128;
   const int64_t nchunks = (ngroups + 3) / 4;
@@ -61,24 +67,23 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
         mn = fminf(mn, R[i]);
         mx = fmaxf(mx, R[i]);
       }
-#pragma unroll
-      for (int o = 1; o < 8; o <<= 1) {
+      for (int o = 1; o < glanes; o <<= 1) {  // the G / 16 lanes of this group
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       }
-      float sc = __fdiv_rn(__fsub_rn(mx, mn), 3.0f);
+      float sc = __fdiv_rn(__fsub_rn(mx, mn), L);
       sc = fmaxf(sc, 0x1p-14f);
       const __half scale_h = __float2half_rn(sc);
       const float step = __half2float(scale_h);
       float zf = rintf(__fdiv_rn(-mn, step));
-      zf = fminf(fmaxf(zf, 0.0f), 3.0f);
+      zf = fminf(fmaxf(zf, 0.0f), L);
       const int z = (int)zf;
 
       uint32_t word = 0;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         float qf = rintf(__fdiv_rn(R[i], step)) + (float)z;
-        qf = fminf(fmaxf(qf, 0.0f), 3.0f);
+        qf = fminf(fmaxf(qf, 0.0f), L);
         const int q = (int)qf;
         word |= (uint32_t)q << (2 * i);
         R[i] = __fsub_rn(R[i], __fmul_rn((float)(q - z), step));
@@ -101,7 +106,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
 }
 
 cudaError_t launch_pack(const void* W, int64_t N, int64_t K, int S, uint32_t* codes, uint32_t* sz,
-                        cudaStream_t stream, int num_sms) {
+                        cudaStream_t stream, int num_sms, int bits, int G) {
   const int64_t nchunks = (K / 128 + 3) / 4;
   const int64_t units = N * nchunks;
   const int warps_per_block = 8;
@@ -110,7 +115,7 @@ cudaError_t launch_pack(const void* W, int64_t N, int64_t K, int S, uint32_t* co
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   pack_kernel<<<(unsigned)blocks, 32 * warps_per_block, 0, stream>>>(
-      static_cast<const __half*>(W), N, K, S, codes, sz);
+      static_cast<const __half*>(W), N, K, S, bits, G / 16, codes, sz);
   return note_error("kernel launch", cudaGetLastError());
 }
 

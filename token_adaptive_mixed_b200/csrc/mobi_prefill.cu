@@ -165,7 +165,7 @@ struct TileInfo {
   int64_t t0;      // first bucket-ordered token
   int nvalid;      // tokens in the tile
   int kmax;        // slices needed by the tile (k of its last token)
-  int lo[3];       // first tile column whose token takes slice s
+  int lo[kMaxSlices];  // first tile column whose token takes slice s
 };
 
 __device__ __forceinline__ TileInfo tile_info(int64_t tile, int64_t n_tt, int64_t T, const int32_t* off, int S) {
@@ -177,11 +177,11 @@ __device__ __forceinline__ TileInfo tile_info(int64_t tile, int64_t n_tt, int64_
   const int64_t last = ti.t0 + ti.nvalid - 1;
   int km = 1;
 #pragma unroll
-  for (int j = 1; j < 3; ++j)
+  for (int j = 1; j < kMaxSlices; ++j)
     if (j < S && (int64_t)off[j] <= last) km = j + 1;
   ti.kmax = km;
 #pragma unroll
-  for (int s = 0; s < 3; ++s) {
+  for (int s = 0; s < kMaxSlices; ++s) {
     int64_t l = s < S ? (int64_t)off[s] - ti.t0 : 0;
     l = l < 0 ? 0 : (l > ti.nvalid ? ti.nvalid : l);
     ti.lo[s] = (int)l;
@@ -229,9 +229,9 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
   const int64_t n_wt = (N + pf::BM - 1) / pf::BM;
   const int64_t n_tt = (T + pf::BN - 1) / pf::BN;
   const int64_t ntiles = n_wt * n_tt;
-  int32_t off[4];
+  int32_t off[kMaxSlices + 1];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) off[j] = j <= S ? __ldg(offsets + j) : 0;
+  for (int j = 0; j <= kMaxSlices; ++j) off[j] = j <= S ? __ldg(offsets + j) : 0;
 
   if (threadIdx.x == 0) {
     // An x stage is released by both MMA issuers (each commits after its own MMAs).
@@ -431,7 +431,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
           if (!(ok = pf_wait(&sm.d_full[db], dph, limit, st, 0x331, abort_flag))) break;
           tc_fence_after();
           const uint32_t d_tmem = tmem + lane_addr + pf::kTmemD + db * pf::BN + cbase;
-          const int lo = (s == 0 ? ti.lo[0] : (s == 1 ? ti.lo[1] : ti.lo[2])) - cbase;  // first active column
+          const int lo = (s == 0 ? ti.lo[0] : s == 1 ? ti.lo[1] : s == 2 ? ti.lo[2] : ti.lo[3]) - cbase;  // first active column
 #pragma unroll
           for (int cp = 0; cp < pf::kColsPerEpi / 48; ++cp) {  // three 16-column loads per wait
             if (48 * cp + 48 <= lo) continue;  // all three chunks inactive (warp-uniform)

@@ -395,7 +395,8 @@ cudaError_t launch_route_small_grouped(const RouteSmallGroup& grp, int S, cudaSt
   switch (S) {
     case 1: return launch_route_small_group<1, kMaxGroup>(grp, stream);
     case 2: return launch_route_small_group<2, kMaxGroup>(grp, stream);
-    default: return launch_route_small_group<3, kMaxGroup>(grp, stream);
+    case 3: return launch_route_small_group<3, kMaxGroup>(grp, stream);
+    default: return launch_route_small_group<4, kMaxGroup>(grp, stream);
   }
 }
 
@@ -650,13 +651,16 @@ cudaError_t launch_route_mlp(const void* X, int64_t T, int64_t K, const float* W
                                                                    kps, P);
     if (S == 2)
       launch_mlp_score<2>(P, T, H, ks, b1, W2, b2, thr, k_t, stream);
-    else
+    else if (S == 3)
       launch_mlp_score<3>(P, T, H, ks, b1, W2, b2, thr, k_t, stream);
+    else
+      launch_mlp_score<4>(P, T, H, ks, b1, W2, b2, thr, k_t, stream);
   }
   switch (S) {
     case 1: bucket_kernel<1><<<1, kBucketThreads, 0, stream>>>(T, 1, nullptr, nullptr, k_t, perm, offsets); break;
     case 2: bucket_kernel<2><<<1, kBucketThreads, 0, stream>>>(T, 1, nullptr, nullptr, k_t, perm, offsets); break;
-    default: bucket_kernel<3><<<1, kBucketThreads, 0, stream>>>(T, 1, nullptr, nullptr, k_t, perm, offsets); break;
+    case 3: bucket_kernel<3><<<1, kBucketThreads, 0, stream>>>(T, 1, nullptr, nullptr, k_t, perm, offsets); break;
+    default: bucket_kernel<4><<<1, kBucketThreads, 0, stream>>>(T, 1, nullptr, nullptr, k_t, perm, offsets); break;
   }
   return note_error("kernel launch", cudaGetLastError());
 }
@@ -700,7 +704,8 @@ cudaError_t launch_route(const void* X, int64_t T, int64_t K, const float* Wr, c
   switch (S) {
     case 1: return launch_route_s<1>(X, T, K, Wr, bias, k_t, perm, offsets, ws, stream);
     case 2: return launch_route_s<2>(X, T, K, Wr, bias, k_t, perm, offsets, ws, stream);
-    default: return launch_route_s<3>(X, T, K, Wr, bias, k_t, perm, offsets, ws, stream);
+    case 3: return launch_route_s<3>(X, T, K, Wr, bias, k_t, perm, offsets, ws, stream);
+    default: return launch_route_s<4>(X, T, K, Wr, bias, k_t, perm, offsets, ws, stream);
   }
 }
 
