@@ -54,12 +54,11 @@ def decode_bytes(N, K, T, kmax):
 
 
 # DRAM bytes / algorithmic bytes of the decode kernel, from one ncu capture of
-# the 11008 x 4096, T=4, k_max=3 launch (dram__bytes_read.sum 38105600 +
-# dram__bytes_write.sum 256 against 38076416 algorithmic; see
-# profiles/decode_kernel_llama7b_decode.md). Traffic grows in proportion to
-# the bytes streamed, so the step's traffic is the step's algorithmic bytes
-# times this ratio. Valid for the decode kernel as captured.
-DECODE_DRAM_RATIO = (38105600 + 256) / 38076416
+# a single 11008 x 4096, T=4, k_max=3 launch (dram__bytes_read.sum 38124288 +
+# dram__bytes_write.sum 0 against 38076416 algorithmic bytes). Traffic grows
+# in proportion to the bytes streamed, so the step's traffic is the step's
+# algorithmic bytes times this ratio. Valid for the decode kernel as captured.
+DECODE_DRAM_RATIO = 38124288 / 38076416
 
 
 class ClockSampler:
@@ -531,6 +530,75 @@ def time_ckpt(mobi, wl, dev, reps=3):
     return out
 
 
+def time_generic(mobi, wl, dev, hbm_peak, tf_peak, flush, steps=200):
+    """Generic slicing: four 1-bit slices (1..4 bits per weight), G = 128.
+    (a) the decode step of the three Llama-7B shapes at T = 4 as one
+    mobi_linear_grouped call, router mix 1/4 each; (b) the prefill workload's
+    shape (T = 2048, 11008 x 4096) through route + prefill GEMM. 1-bit codes
+    sit in 2-bit fields, so the bytes read are those of 2-bit slices."""
+    S = 4
+    out = {"slicing": "4 x 1-bit slices, G = 128 (codes stored in 2-bit fields)"}
+    probs = []
+    for i, (N, K) in enumerate(wl.DECODE_SHAPES):
+        L = wl.layer(f"gen_{N}x{K}", N, K, 4, seed=3000 + i, outlier_frac_cols=0.005, S=S, mix=(0.25,) * S)
+        codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(dev), S=S, bits=1)
+        probs.append({"X": L.X.to(dev), "Wr": torch.from_numpy(L.Wr).to(dev), "bias": torch.from_numpy(L.bias).to(dev),
+                      "codes": codes, "sz": sz, "N": N,
+                      "Y": torch.empty((4, N), dtype=torch.float32, device=dev),
+                      "k_t": torch.empty(4, dtype=torch.int32, device=dev),
+                      "perm": torch.empty(4, dtype=torch.int32, device=dev),
+                      "offsets": torch.empty(S + 1, dtype=torch.int32, device=dev)})
+    ws = torch.empty(max(mobi.mobi_linear_grouped_workspace_bytes(probs, S=S), 16), dtype=torch.uint8, device=dev)
+
+    def step():
+        mobi.mobi_linear_grouped(probs, S=S, ws=ws)
+    step()
+    mobi.mobi_sync_check()
+    kmax = [int(p["k_t"].max().item()) for p in probs]
+    nbytes = sum(decode_bytes(p["N"], p["X"].shape[1], 4, km) for p, km in zip(probs, kmax))
+    ms = time_graph(step, steps)
+    out["decode_T4_grouped"] = {"kmax_per_problem": kmax, "bytes_per_step": nbytes, "ms_per_step": round(ms, 5),
+                                "GB/s": round(nbytes / ms / 1e6, 1), "frac_of_hbm": round(nbytes / ms / 1e6 / hbm_peak, 4),
+                                "bits_per_weight_read": kmax}
+    del probs, ws
+    L = wl.layer("gen_prefill_11008x4096_T2048", 11008, 4096, 2048, seed=3010, n_outlier_cols=20, S=S,
+                 mix=(0.25,) * S)
+    W = torch.from_numpy(L.W).to(dev)
+    codes, sz = mobi.mobi_pack(W, S=S, bits=1)
+    del W
+    X = L.X.to(dev)
+    Wr = torch.from_numpy(L.Wr).to(dev)
+    b = torch.from_numpy(L.bias).to(dev)
+    T, N, K = L.T, L.N, L.K
+    k_t = torch.empty(T, dtype=torch.int32, device=dev)
+    perm = torch.empty(T, dtype=torch.int32, device=dev)
+    off = torch.empty(S + 1, dtype=torch.int32, device=dev)
+    Y = torch.empty((T, N), dtype=torch.float32, device=dev)
+    ws_r = torch.empty(max(mobi.mobi_route_workspace_bytes(T, K, S), 16), dtype=torch.uint8, device=dev)
+    ws_g = torch.empty(mobi.mobi_gemm_workspace_bytes(T, N, K, S), dtype=torch.uint8, device=dev)
+    mobi.mobi_route(X, Wr, b, k_t, perm, off, ws_r)
+    for _ in range(3):
+        mobi.mobi_gemm(X, k_t, perm, off, codes, sz, N, Y=Y, ws=ws_g)
+    mobi.mobi_sync_check()
+    sumk = int(k_t.sum().item())
+    ts = []
+    for _ in range(10):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mobi.mobi_gemm(X, k_t, perm, off, codes, sz, N, Y=Y, ws=ws_g)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ms = statistics.median(ts)
+    issued = 2.0 * N * K * sumk
+    out["prefill_T2048"] = {"k_counts": torch.bincount(k_t, minlength=S + 1)[1:].tolist(), "sum_k": sumk,
+                            "ms_gemm": round(ms, 4), "tflops_issued": round(issued / ms / 1e9, 2),
+                            "frac_of_bf16_peak": round(issued / ms / 1e9 / tf_peak, 4),
+                            "tflops_effective": round(2.0 * T * N * K / ms / 1e9, 2)}
+    return out
+
+
 def run_gpu(args, world, rank):
     import token_adaptive_mixed_b200 as mobi
     from token_adaptive_mixed_b200 import build as mobi_build
@@ -547,6 +615,8 @@ def run_gpu(args, world, rank):
         return {"route_mlp": time_route_mlp(mobi, wl, dev, hbm_peak, l2_flush_buffer(dev))}
     if args.only == "ckpt":
         return {"ckpt": time_ckpt(mobi, wl, dev)}
+    if args.only == "generic":
+        return {"generic_slicing": time_generic(mobi, wl, dev, hbm_peak, tf_peak, l2_flush_buffer(dev))}
     if args.only == "prefill":
         flush = l2_flush_buffer(dev)
         out = {"prefill": time_prefill(mobi, wl.prefill(), dev, args.prefill_reps, tf_peak, flush)}
@@ -706,6 +776,7 @@ def run_gpu(args, world, rank):
     if args.only == "all" and rank == 0:
         out["route_mlp"] = time_route_mlp(mobi, wl, dev, hbm_peak, l2_flush_buffer(dev))
         out["ckpt"] = time_ckpt(mobi, wl, dev)
+        out["generic_slicing"] = time_generic(mobi, wl, dev, hbm_peak, tf_peak, l2_flush_buffer(dev))
     return out
 
 
@@ -797,7 +868,7 @@ def main():
     ap.add_argument("--impl", default="mobi", choices=["mobi", "reference"])
     ap.add_argument("--cpu-baseline-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill", "route_mlp", "ckpt"],
+    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill", "route_mlp", "ckpt", "generic"],
                     help="run a subset (profiling); the default runs everything")
     ap.add_argument("--prefill-reps", type=int, default=10)
     ap.add_argument("--skip-skewed", action="store_true")
