@@ -62,7 +62,7 @@ def check(mobi, oracle, R, tau, delta, tag, null_bias=False):
 
 
 @pytest.mark.parametrize("T,K,H", [(1, 128, 1), (5, 1024, 7), (16, 4096, 128), (37, 512, 100), (300, 1024, 32),
-                                   (129, 256, 33)])
+                                   (129, 256, 33), (700, 1024, 128), (513, 512, 200)])
 def test_route_mlp_parity(mobi, oracle, T, K, H):
     R = wl.mlp_router("mlp", T, K, H, seed=900 + T + H)
     k_gpu, k_ref = check(mobi, oracle, R, 1.0, 0.5, f"mlp T={T} K={K} H={H}")

@@ -415,9 +415,11 @@ cudaError_t launch_route_small_grouped(const RouteSmallGroup& grp, int S, cudaSt
 //   CTA = 16 TT tokens x 128 hidden units, 256 threads, each TT tokens x 8
 //   units (columns 4 tx .. 4 tx + 3 and 64 + 4 tx .. 64 + 4 tx + 3, so the
 //   128-bit shared loads of a quarter-warp hit distinct banks); K runs in
-//   32-row chunks staged in shared memory (x converted to fp32 and stored
-//   k-major, the [32][128] slice of W1). TT = 4 for prefill (ALU-bound: T K H
-//   FMAs), TT = 1 for up to 16 tokens (bound by the W1 read, K H 4 bytes).
+//   32-row chunks: W1 double-buffered through cp.async, the x chunk prefetched
+//   in registers and stored k-major as fp32. TT = 8 (an 8 x 8 register tile,
+//   64 FMAs per 4 shared loads) from 512 tokens on, where the layer is
+//   ALU-bound (T K H FMAs); TT = 4 below; TT = 1 up to 16 tokens, where it is
+//   bound by the W1 read (K H 4 bytes).
 // route_mlp_score_kernel<S>: one CTA of 128 threads per token: h_i =
 //   max(0, sum_s P[s][t][i] + b1[i]) (splits in order), the thread's products
 //   h_i W2[i][j] accumulated over i = tid, tid + 128, ..., an xor tree per warp
@@ -433,8 +435,10 @@ __global__ void __launch_bounds__(kMlpThreads, 2) route_mlp_hidden_kernel(const 
                                                                          int64_t k_per_split,
                                                                          float* __restrict__ P) {
   constexpr int kTok = 16 * TT;
-  constexpr int kXThreads = kTok * kMlpKc / 8;  // threads that load 8 bf16 of x per chunk
-  __shared__ __align__(16) float xs[kMlpKc][kTok + 4];           // k-major fp32 copy of the x chunk
+  constexpr int kXPieces = kTok * kMlpKc / 8;  // 8-bf16 pieces of x per chunk
+  constexpr int kXPer = (kXPieces + kMlpThreads - 1) / kMlpThreads;  // per thread
+  constexpr int kXPad = TT == 8 ? 0 : 4;       // row padding (none at TT = 8: 48 KB of static shared memory)
+  __shared__ __align__(16) float xs[kMlpKc][kTok + kXPad];       // k-major fp32 copy of the x chunk
   __shared__ __align__(16) float wsm[2][kMlpKc][kMlpHidTile];    // W1 chunks, double-buffered
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
@@ -442,8 +446,6 @@ __global__ void __launch_bounds__(kMlpThreads, 2) route_mlp_hidden_kernel(const 
   const int64_t split = blockIdx.z, kb = split * k_per_split;
   const int64_t ke = kb + k_per_split < K ? kb + k_per_split : K;
   const bool vec = (H & 3) == 0 && (reinterpret_cast<uintptr_t>(W1) & 15) == 0;
-  const int xr = tid >> 2, xc = (tid & 3) * 8;  // this thread's x row and first column in a chunk
-  const bool x_loader = tid < kXThreads && t0 + xr < T;
 
   // W1 rows [k0, k0 + 32) x columns [h0, h0 + 128) into wsm[buf]: cp.async when
   // every 16-byte piece is aligned, else plain loads; columns >= H read as 0.
@@ -465,18 +467,26 @@ __global__ void __launch_bounds__(kMlpThreads, 2) route_mlp_hidden_kernel(const 
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
-  auto load_x = [&](int64_t k0) {
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (x_loader) v = __ldg(reinterpret_cast<const uint4*>(X + (t0 + xr) * K + k0 + xc));
-    return v;
-  };
-  auto store_x = [&](uint4 v) {
-    if (tid < kXThreads) {
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  // Piece e of a chunk: token row e / 4, columns 8 (e % 4) .. +7.
+  auto load_x = [&](int64_t k0, uint4 (&v)[kXPer]) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {  // bf16 -> fp32 is a 16-bit shift
-        xs[xc + 2 * q][xr] = __uint_as_float(w[q] << 16);
-        xs[xc + 2 * q + 1][xr] = __uint_as_float(w[q] & 0xffff0000u);
+    for (int m = 0; m < kXPer; ++m) {
+      const int e = tid + m * kMlpThreads, xr = e >> 2, xc = (e & 3) * 8;
+      v[m] = make_uint4(0u, 0u, 0u, 0u);
+      if (e < kXPieces && t0 + xr < T) v[m] = __ldg(reinterpret_cast<const uint4*>(X + (t0 + xr) * K + k0 + xc));
+    }
+  };
+  auto store_x = [&](const uint4 (&v)[kXPer]) {
+#pragma unroll
+    for (int m = 0; m < kXPer; ++m) {
+      const int e = tid + m * kMlpThreads, xr = e >> 2, xc = (e & 3) * 8;
+      if (e < kXPieces) {
+        const uint32_t w[4] = {v[m].x, v[m].y, v[m].z, v[m].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // bf16 -> fp32 is a 16-bit shift
+          xs[xc + 2 * q][xr] = __uint_as_float(w[q] << 16);
+          xs[xc + 2 * q + 1][xr] = __uint_as_float(w[q] & 0xffff0000u);
+        }
       }
     }
   };
@@ -488,13 +498,14 @@ __global__ void __launch_bounds__(kMlpThreads, 2) route_mlp_hidden_kernel(const 
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
 
   // K and every split are multiples of 32, so each split is a whole number of chunks.
-  uint4 xv_next = load_x(kb);
+  uint4 xv_next[kXPer];
+  load_x(kb, xv_next);
   stage_w(0, kb);
   int buf = 0;
   for (int64_t k0 = kb; k0 < ke; k0 += kMlpKc, buf ^= 1) {
     store_x(xv_next);  // xs is free: the previous chunk ended with a barrier
     if (k0 + kMlpKc < ke) {
-      xv_next = load_x(k0 + kMlpKc);
+      load_x(k0 + kMlpKc, xv_next);
       stage_w(buf ^ 1, k0 + kMlpKc);  // wsm[buf ^ 1] is free for the same reason
       asm volatile("cp.async.wait_group 1;" ::: "memory");
     } else {
@@ -507,6 +518,11 @@ __global__ void __launch_bounds__(kMlpThreads, 2) route_mlp_hidden_kernel(const 
       if constexpr (TT == 4) {
         const float4 q = *reinterpret_cast<const float4*>(&xs[c][ty * 4]);
         xv[0] = q.x; xv[1] = q.y; xv[2] = q.z; xv[3] = q.w;
+      } else if constexpr (TT == 8) {
+        const float4 q0 = *reinterpret_cast<const float4*>(&xs[c][ty * 8]);
+        const float4 q1 = *reinterpret_cast<const float4*>(&xs[c][ty * 8 + 4]);
+        xv[0] = q0.x; xv[1] = q0.y; xv[2] = q0.z; xv[3] = q0.w;
+        xv[4] = q1.x; xv[5] = q1.y; xv[6] = q1.z; xv[7] = q1.w;
       } else {
 #pragma unroll
         for (int i = 0; i < TT; ++i) xv[i] = xs[c][ty * TT + i];
@@ -596,8 +612,12 @@ __global__ void route_mlp_base_only_kernel(int64_t T, int32_t* __restrict__ k_t)
 
 // Splits of K for the hidden layer: as many as fit one wave of two CTAs per SM
 // (no partial second wave), each split a multiple of 32 rows and at least 64.
+// Tokens per CTA tile: 16 (one per thread row) up to 16 tokens, 64 below 512,
+// 128 (an 8 x 8 register tile per thread) from there on.
+static int mlp_tt(int64_t T) { return T <= 16 ? 1 : (T < 512 ? 4 : 8); }
+
 static int64_t mlp_k_per_split(int64_t T, int64_t K, int64_t H, int sms) {
-  const int64_t tok = T <= 16 ? 16 : 64;
+  const int64_t tok = 16 * mlp_tt(T);
   int64_t base = ((T + tok - 1) / tok) * ((H + kMlpHidTile - 1) / kMlpHidTile);
   if (base < 1) base = 1;
   int64_t ks = 2 * (int64_t)sms / base;
@@ -640,15 +660,16 @@ cudaError_t launch_route_mlp(const void* X, int64_t T, int64_t K, const float* W
     float* P = static_cast<float*>(ws);
     const int64_t kps = mlp_k_per_split(T, K, H, sms);
     const int ks = (int)((K + kps - 1) / kps);
-    const bool small = T <= 16;
-    const int64_t tok = small ? 16 : 64;
+    const int tt = mlp_tt(T);
+    const int64_t tok = 16 * tt;
     dim3 grid((unsigned)((T + tok - 1) / tok), (unsigned)((H + kMlpHidTile - 1) / kMlpHidTile), (unsigned)ks);
-    if (small)
-      route_mlp_hidden_kernel<1><<<grid, kMlpThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T, K, W1, H,
-                                                                   kps, P);
+    const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
+    if (tt == 1)
+      route_mlp_hidden_kernel<1><<<grid, kMlpThreads, 0, stream>>>(Xb, T, K, W1, H, kps, P);
+    else if (tt == 4)
+      route_mlp_hidden_kernel<4><<<grid, kMlpThreads, 0, stream>>>(Xb, T, K, W1, H, kps, P);
     else
-      route_mlp_hidden_kernel<4><<<grid, kMlpThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T, K, W1, H,
-                                                                   kps, P);
+      route_mlp_hidden_kernel<8><<<grid, kMlpThreads, 0, stream>>>(Xb, T, K, W1, H, kps, P);
     if (S == 2)
       launch_mlp_score<2>(P, T, H, ks, b1, W2, b2, thr, k_t, stream);
     else if (S == 3)
