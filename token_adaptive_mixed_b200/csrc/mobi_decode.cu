@@ -751,6 +751,32 @@ cudaError_t launch_decode_grouped(const DecodeJob* jobs, int G, int S, cudaStrea
   return note_error("kernel launch", cudaGetLastError());
 }
 
+cudaError_t launch_chunk_reduce(const float* partial, float* Y, int64_t T, int64_t N, int nch, cudaStream_t stream) {
+  DecReduceGroup red = {};
+  red.G = 1;
+  red.partial[0] = reinterpret_cast<const float4*>(partial);
+  red.Y[0] = reinterpret_cast<float4*>(Y);
+  red.nch[0] = nch;
+  red.off[0] = 0;
+  red.off[1] = T * N / 4;
+  int64_t blocks = (red.off[1] + 255) / 256;
+  const int64_t cap = (int64_t)num_sms() * 4;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_reduce_kernel, red);
+  if (e != cudaSuccess) return note_error("chunk reduce launch", e);
+  return note_error("kernel launch", cudaGetLastError());
+}
+
 cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
                           const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
                           DeviceStatus* st, bool early) {

@@ -70,6 +70,9 @@ struct DecodeJob {
   int T;
 };
 size_t decode_ws_bytes(int64_t N, int64_t K);
+// Y[t][n] = sum over chunks c (in order) of partial[c][t][n] (T N % 4 == 0),
+// launched as a programmatic dependent of the kernel before it.
+cudaError_t launch_chunk_reduce(const float* partial, float* Y, int64_t T, int64_t N, int nch, cudaStream_t stream);
 // Decode GEMMs of up to kMaxGroup problems: one launch per fragment class
 // (T <= 8, T <= 16) plus one chunk-reduction launch.
 cudaError_t launch_decode_grouped(const DecodeJob* jobs, int G, int S, cudaStream_t stream, DeviceStatus* st,

@@ -48,7 +48,6 @@ namespace mobi {
 
 namespace pf {
 constexpr int BM = 128;          // weight rows per tile (tcgen05 M)
-constexpr int BN = 192;          // tokens per tile (tcgen05 N)
 constexpr int GK = 128;          // group width along K
 constexpr int XST = 3;           // x-tile stages (one group each)
 constexpr int CST = 6;           // code/scale stages (one unit each)
@@ -61,19 +60,29 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kDeqWarp0 = 4;
 constexpr int kEpiWarp0 = 8;
 constexpr int kEpiWarps = 8;                   // two per TMEM lane quadrant
-constexpr int kColsPerEpi = BN / 2;            // 96 token columns per epilogue warp
-constexpr uint32_t kXHalfBytes = BN * 128;     // 192 rows x 64 bf16 = 24576
-constexpr uint32_t kXStageBytes = 2 * kXHalfBytes;
 constexpr uint32_t kCodeBytes = BM * 32;       // 128 rows x 8 words
 constexpr uint32_t kSzBytes = BM * 4;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemD = 0;                 // D slot j at columns j * BN
-constexpr uint32_t kTmemA = DST * BN;          // A slot j at columns kTmemA + 32 j
-static_assert(DST * BN + AST * 32 <= kTmemCols, "TMEM budget");
+
+// Token-tile width BN (tcgen05 N): 192 for prefill, 64 for small batches
+// (up to 64 tokens, where a 192-wide tile would be mostly padding).
+template <int BN_>
+struct Tile {
+  static constexpr int BN = BN_;
+  static constexpr int kColsPerEpi = BN / 2;                // token columns per epilogue warp
+  static constexpr int kChunkCols = BN == 192 ? 48 : 32;    // columns per TMEM wait in the epilogue
+  static constexpr uint32_t kXHalfBytes = BN * 128;         // BN rows x 64 bf16
+  static constexpr uint32_t kXStageBytes = 2 * kXHalfBytes;
+  static constexpr uint32_t kTmemD = 0;                     // D slot j at columns j * BN
+  static constexpr uint32_t kTmemA = DST * BN;              // A slot j at columns kTmemA + 32 j
+  static_assert(DST * BN + AST * 32 <= (int)kTmemCols, "TMEM budget");
+  static_assert(kColsPerEpi % kChunkCols == 0 && kChunkCols % 16 == 0, "epilogue chunks");
+};
 }  // namespace pf
 
+template <int BN>
 struct PfSmem {
-  uint8_t x[pf::XST][pf::kXStageBytes];     // 1024-byte aligned (offset 0)
+  uint8_t x[pf::XST][pf::Tile<BN>::kXStageBytes];     // 1024-byte aligned (offset 0)
   uint32_t codes[pf::CST][pf::BM * 8];      // [row][word]
   uint32_t sz[pf::CST][pf::BM];
   uint64_t x_full[pf::XST], x_empty[pf::XST];
@@ -163,17 +172,31 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
 struct TileInfo {
   int64_t n0;      // first weight row
   int64_t t0;      // first bucket-ordered token
+  int64_t g0, g1;  // the tile's groups [g0, g1) along K
+  int kc;          // its K chunk
   int nvalid;      // tokens in the tile
   int kmax;        // slices needed by the tile (k of its last token)
   int lo[kMaxSlices];  // first tile column whose token takes slice s
 };
 
-__device__ __forceinline__ TileInfo tile_info(int64_t tile, int64_t n_tt, int64_t T, const int32_t* off, int S) {
+// Tile index = (weight tile * n_tt + token tile) * nkc + K chunk; a chunk is
+// gpc consecutive groups.
+template <int BN, bool KSPLIT>
+__device__ __forceinline__ TileInfo tile_info(int64_t tile, int64_t n_tt, int nkc, int64_t gpc, int64_t ngroups,
+                                              int64_t T, const int32_t* off, int S) {
   TileInfo ti;
-  const int64_t wt = tile / n_tt, tt = tile % n_tt;
+  if constexpr (!KSPLIT) {  // one K chunk: the whole K
+    nkc = 1;
+    gpc = ngroups;
+  }
+  const int64_t kc = tile % nkc, rest = tile / nkc;
+  const int64_t wt = rest / n_tt, tt = rest % n_tt;
+  ti.kc = (int)kc;
+  ti.g0 = kc * gpc;
+  ti.g1 = ti.g0 + gpc < ngroups ? ti.g0 + gpc : ngroups;
   ti.n0 = wt * pf::BM;
-  ti.t0 = tt * pf::BN;
-  ti.nvalid = (int)(T - ti.t0 < pf::BN ? T - ti.t0 : pf::BN);
+  ti.t0 = tt * BN;
+  ti.nvalid = (int)(T - ti.t0 < BN ? T - ti.t0 : BN);
   const int64_t last = ti.t0 + ti.nvalid - 1;
   int km = 1;
 #pragma unroll
@@ -194,12 +217,14 @@ __device__ __forceinline__ TileInfo tile_info(int64_t tile, int64_t n_tt, int64_
 // needs as many slices or more) and, within one, the weight tiles in order;
 // pass i deals one tile to every CTA, in CTA order on even passes and in
 // reverse on odd ones, so heavy and light tiles even out across CTAs.
-__device__ __forceinline__ int64_t pf_tile(int64_t i, int64_t ntiles, int64_t n_wt, int64_t n_tt) {
+__device__ __forceinline__ int64_t pf_tile(int64_t i, int64_t ntiles, int64_t n_wt, int64_t n_tt, int nkc) {
   const int64_t G = gridDim.x, c = blockIdx.x;
   const int64_t idx = i * G + ((i & 1) ? G - 1 - c : c);
   if (idx >= ntiles) return -1;
-  const int64_t tt = n_tt - 1 - idx / n_wt, wt = idx % n_wt;
-  return wt * n_tt + tt;
+  const int64_t per_tt = n_wt * nkc;
+  const int64_t tt = n_tt - 1 - idx / per_tt, r = idx % per_tt;
+  const int64_t wt = r / nkc, kc = r % nkc;
+  return (wt * n_tt + tt) * nkc + kc;
 }
 
 // Bounded wait that also gives up when another role has aborted.
@@ -214,21 +239,29 @@ __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, uint64_t
   return false;
 }
 
+// Y: the output [T][N] when nkc == 1, else the per-chunk partials [nkc][T][N]
+// (added in chunk order by a separate reduction). KSPLIT = false compiles the
+// single-chunk kernel (nkc ignored), which keeps the K-chunk bookkeeping out
+// of its registers.
+template <int BN, bool KSPLIT>
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
     const uint8_t* __restrict__ Xt, const __grid_constant__ CUtensorMap tm_codes,
     const __grid_constant__ CUtensorMap tm_sz, const uint32_t* __restrict__ sz, const int32_t* __restrict__ perm,
-    const int32_t* __restrict__ offsets, int64_t T, int64_t N, int64_t ngroups, int S, float* __restrict__ Y,
-    DeviceStatus* st, uint64_t limit) {
+    const int32_t* __restrict__ offsets, int64_t T, int64_t N, int64_t ngroups, int S, int nkc,
+    float* __restrict__ Y, DeviceStatus* st, uint64_t limit) {
+  using TL = pf::Tile<BN>;
+  if constexpr (!KSPLIT) nkc = 1;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // Dynamic shared memory is rounded up to a 1024-byte boundary for the swizzled tiles.
-  PfSmem& sm = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  PfSmem<BN>& sm = *reinterpret_cast<PfSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int32_t* abort_flag = &sm.abort_flag;
   (void)sz;
 
   const int64_t n_wt = (N + pf::BM - 1) / pf::BM;
-  const int64_t n_tt = (T + pf::BN - 1) / pf::BN;
-  const int64_t ntiles = n_wt * n_tt;
+  const int64_t n_tt = (T + BN - 1) / BN;
+  const int64_t ntiles = n_wt * n_tt * nkc;
+  const int64_t gpc = (ngroups + nkc - 1) / nkc;  // groups per K chunk
   int32_t off[kMaxSlices + 1];
 #pragma unroll
   for (int j = 0; j <= kMaxSlices; ++j) off[j] = j <= S ? __ldg(offsets + j) : 0;
@@ -260,15 +293,15 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
       prefetch_tmap(&tm_codes); prefetch_tmap(&tm_sz);
       uint32_t xi = 0, ci = 0;  // running stage counters
       bool ok = true;
-      for (int64_t i = 0, tile; (tile = pf_tile(i, ntiles, n_wt, n_tt)) >= 0 && ok; ++i) {
-        const TileInfo ti = tile_info(tile, n_tt, T, off, S);
-        for (int64_t g = 0; g < ngroups && ok; ++g) {
+      for (int64_t i = 0, tile; (tile = pf_tile(i, ntiles, n_wt, n_tt, nkc)) >= 0 && ok; ++i) {
+        const TileInfo ti = tile_info<BN, KSPLIT>(tile, n_tt, nkc, gpc, ngroups, T, off, S);
+        for (int64_t g = ti.g0; g < ti.g1 && ok; ++g) {
           const uint32_t xs = xi % pf::XST, xph = (xi / pf::XST) & 1;
           if (!(ok = pf_wait(&sm.x_empty[xs], xph ^ 1, limit, st, 0x301, abort_flag))) break;
-          mbar_arrive_expect_tx(&sm.x_full[xs], pf::kXStageBytes);
+          mbar_arrive_expect_tx(&sm.x_full[xs], TL::kXStageBytes);
           // Pre-swizzled tile (token tile, group g): one contiguous bulk copy.
-          const int64_t tt = ti.t0 / pf::BN;
-          bulk_g2s(&sm.x[xs][0], Xt + (tt * ngroups + g) * (int64_t)pf::kXStageBytes, pf::kXStageBytes,
+          const int64_t tt = ti.t0 / BN;
+          bulk_g2s(&sm.x[xs][0], Xt + (tt * ngroups + g) * (int64_t)TL::kXStageBytes, TL::kXStageBytes,
                    &sm.x_full[xs]);
           ++xi;
           for (int s = 0; s < ti.kmax; ++s) {
@@ -297,12 +330,12 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
     // both threads release every x stage (count 2).
     if (lane == 0) {
       const uint32_t par = (uint32_t)(warp - 1);
-      const uint32_t idesc = idesc_bf16(pf::BM, pf::BN);
+      const uint32_t idesc = idesc_bf16(pf::BM, BN);
       uint32_t xi = 0, u = 0;  // x stages, units (all units are counted by both threads)
       bool ok = true;
-      for (int64_t i = 0, tile; (tile = pf_tile(i, ntiles, n_wt, n_tt)) >= 0 && ok; ++i) {
-        const TileInfo ti = tile_info(tile, n_tt, T, off, S);
-        for (int64_t g = 0; g < ngroups && ok; ++g) {
+      for (int64_t i = 0, tile; (tile = pf_tile(i, ntiles, n_wt, n_tt, nkc)) >= 0 && ok; ++i) {
+        const TileInfo ti = tile_info<BN, KSPLIT>(tile, n_tt, nkc, gpc, ngroups, T, off, S);
+        for (int64_t g = ti.g0; g < ti.g1 && ok; ++g) {
           const uint32_t xs = xi % pf::XST, xph = (xi / pf::XST) & 1;
           const uint32_t xbase = smem_addr(&sm.x[xs][0]);
           bool have_x = false;
@@ -319,13 +352,13 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
             const uint32_t hh1 = 2 * u + 1;
             if (!(ok = pf_wait(&sm.a_full[hh1 % pf::AST], (hh1 / pf::AST) & 1, limit, st, 0x312, abort_flag))) break;
             tc_fence_after();
-            const uint32_t d_tmem = tmem + pf::kTmemD + db * pf::BN;
+            const uint32_t d_tmem = tmem + TL::kTmemD + db * BN;
             for (int half = 0; half < 2; ++half) {
               const uint32_t ab = (2 * u + half) % pf::AST;
-              const uint32_t a_tmem = tmem + pf::kTmemA + ab * 32;
+              const uint32_t a_tmem = tmem + TL::kTmemA + ab * 32;
 #pragma unroll
               for (int i = 0; i < 4; ++i) {  // k16 steps 4*half .. 4*half+3: one x half tile
-                const uint32_t saddr = xbase + half * pf::kXHalfBytes + i * 32;
+                const uint32_t saddr = xbase + half * TL::kXHalfBytes + i * 32;
                 mma_ts(d_tmem, a_tmem + 8 * i, desc_sw128(saddr), idesc, (half > 0 || i > 0) ? 1u : 0u);
               }
               mma_commit(&sm.a_empty[ab]);
@@ -350,9 +383,9 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     uint32_t u = 0, hh = 0;
     bool ok = true;
-    for (int64_t i = 0, tile; (tile = pf_tile(i, ntiles, n_wt, n_tt)) >= 0 && ok; ++i) {
-      const TileInfo ti = tile_info(tile, n_tt, T, off, S);
-      for (int64_t g = 0; g < ngroups && ok; ++g) {
+    for (int64_t i = 0, tile; (tile = pf_tile(i, ntiles, n_wt, n_tt, nkc)) >= 0 && ok; ++i) {
+      const TileInfo ti = tile_info<BN, KSPLIT>(tile, n_tt, nkc, gpc, ngroups, T, off, S);
+      for (int64_t g = ti.g0; g < ti.g1 && ok; ++g) {
         for (int s = 0; s < ti.kmax && ok; ++s, ++u) {
           const uint32_t cs = u % pf::CST, cph = (u / pf::CST) & 1;
           if (!(ok = pf_wait(&sm.c_full[cs], cph, limit, st, 0x321, abort_flag))) break;
@@ -376,7 +409,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
             const uint32_t ab = hh % pf::AST, aph = (hh / pf::AST) & 1;
             if (!(ok = pf_wait(&sm.a_empty[ab], aph ^ 1, limit, st, 0x322, abort_flag))) break;
             tc_fence_after();
-            const uint32_t a_tmem = tmem + lane_addr + pf::kTmemA + ab * 32;
+            const uint32_t a_tmem = tmem + lane_addr + TL::kTmemA + ab * 32;
 #pragma unroll
             for (int wp = 0; wp < 2; ++wp) {  // 16 columns (two words) per store
               uint32_t regs[16];
@@ -407,17 +440,17 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
     // ---------------- epilogue: per-group fp32 scale promotion ----------------
     const int e = warp - pf::kEpiWarp0;   // 0..7
     const int q = warp & 3;               // TMEM lane quadrant
-    const int cbase = (e >> 2) * pf::kColsPerEpi;  // 0 or 64
+    const int cbase = (e >> 2) * TL::kColsPerEpi;  // 0 or BN / 2
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     uint32_t u = 0;
     bool ok = true;
-    for (int64_t i = 0, tile; (tile = pf_tile(i, ntiles, n_wt, n_tt)) >= 0 && ok; ++i) {
-      const TileInfo ti = tile_info(tile, n_tt, T, off, S);
+    for (int64_t i = 0, tile; (tile = pf_tile(i, ntiles, n_wt, n_tt, nkc)) >= 0 && ok; ++i) {
+      const TileInfo ti = tile_info<BN, KSPLIT>(tile, n_tt, nkc, gpc, ngroups, T, off, S);
       const int64_t n = ti.n0 + 32 * q + lane;
-      float2 acc[pf::kColsPerEpi / 2];
+      float2 acc[TL::kColsPerEpi / 2];
 #pragma unroll
-      for (int c = 0; c < pf::kColsPerEpi / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
-      for (int64_t g = 0; g < ngroups && ok; ++g) {
+      for (int c = 0; c < TL::kColsPerEpi / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
+      for (int64_t g = ti.g0; g < ti.g1 && ok; ++g) {
         for (int s = 0; s < ti.kmax; ++s, ++u) {
           // Scale of (slice s, group g, row r) from the staged copy of this unit.
           const uint32_t cs = u % pf::CST, cph = (u / pf::CST) & 1;
@@ -430,27 +463,30 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
           const uint32_t db = u % pf::DST, dph = (u / pf::DST) & 1;
           if (!(ok = pf_wait(&sm.d_full[db], dph, limit, st, 0x331, abort_flag))) break;
           tc_fence_after();
-          const uint32_t d_tmem = tmem + lane_addr + pf::kTmemD + db * pf::BN + cbase;
+          const uint32_t d_tmem = tmem + lane_addr + TL::kTmemD + db * BN + cbase;
           const int lo = (s == 0 ? ti.lo[0] : s == 1 ? ti.lo[1] : s == 2 ? ti.lo[2] : ti.lo[3]) - cbase;  // first active column
+          constexpr int CC = TL::kChunkCols;  // columns per wait: CC / 16 loads of 16
 #pragma unroll
-          for (int cp = 0; cp < pf::kColsPerEpi / 48; ++cp) {  // three 16-column loads per wait
-            if (48 * cp + 48 <= lo) continue;  // all three chunks inactive (warp-uniform)
-            uint32_t r[48];
-            tmem_ld16(d_tmem + 48 * cp, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-            tmem_ld16(d_tmem + 48 * cp + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
-            tmem_ld16(d_tmem + 48 * cp + 32, *reinterpret_cast<uint32_t(*)[16]>(&r[32]));
+          for (int cp = 0; cp < TL::kColsPerEpi / CC; ++cp) {
+            if (CC * cp + CC <= lo) continue;  // the whole chunk inactive (warp-uniform)
+            uint32_t r[CC];
+#pragma unroll
+            for (int l = 0; l < CC / 16; ++l)
+              tmem_ld16(d_tmem + CC * cp + 16 * l, *reinterpret_cast<uint32_t(*)[16]>(&r[16 * l]));
             tmem_ld_wait();
-            if (48 * cp >= lo) {  // all 48 columns active: packed fp32x2 FMAs
+            if (CC * cp >= lo) {  // every column active: packed fp32x2 FMAs
 #pragma unroll
-              for (int j = 0; j < 24; ++j)
-                acc[24 * cp + j] = __ffma2_rn(sc2, make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])),
-                                              acc[24 * cp + j]);
+              for (int j = 0; j < CC / 2; ++j)
+                acc[CC / 2 * cp + j] = __ffma2_rn(sc2, make_float2(__uint_as_float(r[2 * j]),
+                                                                   __uint_as_float(r[2 * j + 1])),
+                                                  acc[CC / 2 * cp + j]);
             } else {
 #pragma unroll
-              for (int j = 0; j < 24; ++j) {
-                const int c = 48 * cp + 2 * j;
-                if (c >= lo) acc[24 * cp + j].x = fmaf(sc, __uint_as_float(r[2 * j]), acc[24 * cp + j].x);
-                if (c + 1 >= lo) acc[24 * cp + j].y = fmaf(sc, __uint_as_float(r[2 * j + 1]), acc[24 * cp + j].y);
+              for (int j = 0; j < CC / 2; ++j) {
+                const int c = CC * cp + 2 * j;
+                if (c >= lo) acc[CC / 2 * cp + j].x = fmaf(sc, __uint_as_float(r[2 * j]), acc[CC / 2 * cp + j].x);
+                if (c + 1 >= lo)
+                  acc[CC / 2 * cp + j].y = fmaf(sc, __uint_as_float(r[2 * j + 1]), acc[CC / 2 * cp + j].y);
               }
             }
           }
@@ -461,12 +497,13 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
       }
       if (!ok) break;
       if (n < N) {
+        float* out = Y + (int64_t)ti.kc * T * N;  // chunk kc's partials (the output itself when nkc == 1)
 #pragma unroll
-        for (int c = 0; c < pf::kColsPerEpi; ++c) {
+        for (int c = 0; c < TL::kColsPerEpi; ++c) {
           const int col = cbase + c;
           if (col < ti.nvalid) {
             const int32_t t = __ldg(perm + ti.t0 + col);
-            if (t >= 0 && t < T) Y[(int64_t)t * N + n] = (c & 1) ? acc[c >> 1].y : acc[c >> 1].x;
+            if (t >= 0 && t < T) out[(int64_t)t * N + n] = (c & 1) ? acc[c >> 1].y : acc[c >> 1].x;
           }
         }
       }
@@ -490,6 +527,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
 // swizzle). Row r of tile tt is the token perm[192 tt + r] (zeros beyond T);
 // its permuted column 16w + 2c + e holds x[16w + c + 8e], matching the pair
 // order (c, c+8) of a packed word. One thread per 16-column block of a row.
+template <int BN>
 __global__ void __launch_bounds__(256) prefill_gather_kernel(const __nv_bfloat16* __restrict__ X, int64_t T,
                                                              int64_t K, const int32_t* __restrict__ perm,
                                                              int64_t T_pad, uint8_t* __restrict__ Xt) {
@@ -515,58 +553,115 @@ __global__ void __launch_bounds__(256) prefill_gather_kernel(const __nv_bfloat16
     out[c] = lo | (hi << 16);
   }
   const int64_t ngroups = K / 128;
-  const int64_t tt = i / pf::BN, r = i % pf::BN;
+  const int64_t tt = i / BN, r = i % BN;
   const int64_t g = w / 8, h = (w % 8) / 4, j0 = 2 * (w % 4);  // chunks j0, j0+1 of half h
-  uint8_t* tile = Xt + ((tt * ngroups + g) * 2 + h) * (int64_t)pf::kXHalfBytes + r * 128;
+  uint8_t* tile = Xt + ((tt * ngroups + g) * 2 + h) * (int64_t)pf::Tile<BN>::kXHalfBytes + r * 128;
   *reinterpret_cast<uint4*>(tile + 16 * ((j0) ^ (r & 7))) = make_uint4(out[0], out[1], out[2], out[3]);
   *reinterpret_cast<uint4*>(tile + 16 * ((j0 + 1) ^ (r & 7))) = make_uint4(out[4], out[5], out[6], out[7]);
 }
 
 // ---- host side -------------------------------------------------------------------------
 
-size_t prefill_ws_bytes(int64_t T, int64_t N, int64_t K) {
-  (void)N;
-  const int64_t T_pad = (T + pf::BN - 1) / pf::BN * pf::BN;
-  return ((size_t)T_pad * (size_t)K * 2 + 255) / 256 * 256;
+// Tile width and K chunks of a launch: 64-token tiles up to 64 tokens,
+// 192-token tiles beyond. K is cut into nkc chunks of equal group counts (none
+// empty) when that shortens the launch; the chunk partials are then added by a
+// separate reduction. The count minimises a simple cost fitted to
+// measurements: the busiest CTA's tiles x (groups per chunk x 3 slices + 4),
+// about 1 us per group and slice of a tile plus ~4 us to start and finish a
+// tile, plus each chunk's partials written and read back (8 T N bytes at
+// 6 TB/s).
+struct PfPlan {
+  int bn, nkc;
+  int64_t T_pad;
+  size_t xt_bytes, part_bytes;
+};
+
+static PfPlan pf_plan(int64_t T, int64_t N, int64_t K, int sms) {
+  PfPlan p;
+  const int64_t ngroups = K / 128;
+  p.bn = T <= 64 ? 64 : 192;
+  p.T_pad = (T + p.bn - 1) / p.bn * p.bn;
+  int64_t nkc = 1;
+  const int64_t base = ((N + pf::BM - 1) / pf::BM) * ((T + p.bn - 1) / p.bn);
+  if (ngroups > 1 && base > 0 && sms > 0) {
+    double best = 1e300;
+    const int64_t cmax = ngroups < 64 ? ngroups : 64;
+    for (int64_t c = 1; c <= cmax; ++c) {
+      const int64_t gpc = (ngroups + c - 1) / c, used = (ngroups + gpc - 1) / gpc;
+      const int64_t per_cta = (base * used + sms - 1) / sms;
+      const double cost = (double)per_cta * ((double)gpc * 3.0 + 4.0) +
+                          (used > 1 ? (double)used * 8.0 * (double)T * (double)N / 6.0e6 : 0.0);
+      if (cost < best - 1e-9) {
+        best = cost;
+        nkc = used;
+      }
+    }
+  }
+  p.nkc = (int)nkc;
+  p.xt_bytes = ((size_t)p.T_pad * (size_t)K * 2 + 255) / 256 * 256;
+  p.part_bytes = nkc > 1 ? ((size_t)nkc * (size_t)T * (size_t)N * 4 + 255) / 256 * 256 : 0;
+  return p;
 }
 
-static size_t pf_smem_bytes() { return sizeof(PfSmem) + 1024; }
+size_t prefill_ws_bytes(int64_t T, int64_t N, int64_t K) {
+  if (T <= 0 || K <= 0) return 256;
+  const PfPlan p = pf_plan(T, N, K, num_sms());
+  return p.xt_bytes + p.part_bytes;
+}
 
-cudaError_t launch_prefill(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
-                           const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int S,
-                           float* Y, void* ws, cudaStream_t stream, DeviceStatus* st) {
-  (void)k_t;
+template <int BN, bool KSPLIT>
+static cudaError_t launch_prefill_bn(const PfPlan& plan, const void* X, int64_t T, int64_t K, const int32_t* perm,
+                                     const int32_t* offsets, const CUtensorMap& tm_codes, const CUtensorMap& tm_sz,
+                                     const uint32_t* sz, int64_t N, int S, float* out, uint8_t* Xt,
+                                     cudaStream_t stream, DeviceStatus* st) {
   const int64_t ngroups = K / 128;
-  const int64_t T_pad = (T + pf::BN - 1) / pf::BN * pf::BN;
-  uint8_t* Xt = static_cast<uint8_t*>(ws);
-  CUtensorMap tm_codes, tm_sz;
-  if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4, 8, pf::BM,
-                    0))
-    return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, pf::BM, 1, 0))
-    return cudaErrorInvalidValue;
-
-  const int64_t blocks_g = (T_pad * (K / 16) + 255) / 256;
-  prefill_gather_kernel<<<(unsigned)blocks_g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T, K, perm,
-                                                               T_pad, Xt);
-
-  const int64_t ntiles = ((N + pf::BM - 1) / pf::BM) * ((T + pf::BN - 1) / pf::BN);
+  const int64_t blocks_g = (plan.T_pad * (K / 16) + 255) / 256;
+  prefill_gather_kernel<BN><<<(unsigned)blocks_g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), T, K,
+                                                                   perm, plan.T_pad, Xt);
+  auto kernel = prefill_kernel<BN, KSPLIT>;
+  const int64_t ntiles = ((N + pf::BM - 1) / pf::BM) * ((T + BN - 1) / BN) * plan.nkc;
   const int grid = (int)(ntiles < num_sms() ? ntiles : num_sms());
-  const size_t smem = pf_smem_bytes();
-  cudaError_t e = set_smem((const void*)prefill_kernel, (int)smem);
+  const size_t smem = sizeof(PfSmem<BN>) + 1024;
+  cudaError_t e = set_smem((const void*)kernel, (int)smem);
   if (e != cudaSuccess) return e;
-  prefill_kernel<<<grid, pf::kThreads, smem, stream>>>(Xt, tm_codes, tm_sz, sz, perm, offsets, T, N, ngroups, S, Y,
-                                                       st, wait_limit());
+  kernel<<<grid, pf::kThreads, smem, stream>>>(Xt, tm_codes, tm_sz, sz, perm, offsets, T, N, ngroups, S, plan.nkc,
+                                               out, st, wait_limit());
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     cudaFuncAttributes fa{};
-    cudaFuncGetAttributes(&fa, (const void*)prefill_kernel);
+    cudaFuncGetAttributes(&fa, (const void*)kernel);
     char where[160];
     snprintf(where, sizeof where, "prefill launch (%d threads, %d regs/thread, max %d threads, %zu B smem)",
              pf::kThreads, fa.numRegs, fa.maxThreadsPerBlock, smem);
     return note_error(where, e);
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_prefill(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
+                           const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int S,
+                           float* Y, void* ws, cudaStream_t stream, DeviceStatus* st) {
+  (void)k_t;
+  const int64_t ngroups = K / 128;
+  const PfPlan plan = pf_plan(T, N, K, num_sms());
+  uint8_t* Xt = static_cast<uint8_t*>(ws);
+  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + plan.xt_bytes);
+  float* out = plan.nkc > 1 ? partial : Y;
+  CUtensorMap tm_codes, tm_sz;
+  if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4, 8, pf::BM,
+                    0))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, pf::BM, 1, 0))
+    return cudaErrorInvalidValue;
+  cudaError_t e;
+  if (plan.bn == 64)
+    e = launch_prefill_bn<64, true>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, out, Xt, stream, st);
+  else if (plan.nkc > 1)
+    e = launch_prefill_bn<192, true>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, out, Xt, stream, st);
+  else
+    e = launch_prefill_bn<192, false>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, out, Xt, stream, st);
+  if (e != cudaSuccess || plan.nkc <= 1) return e;
+  return launch_chunk_reduce(partial, Y, T, N, plan.nkc, stream);
 }
 
 }  // namespace mobi
