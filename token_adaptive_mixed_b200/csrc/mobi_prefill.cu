@@ -405,10 +405,15 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
             const float a = -(128.0f * m + zf);  // exact in bf16: 128 + z, 32 + z or 8 + z
             add[f] = __floats2bfloat162_rn(a, a);
           }
-          for (int half = 0; half < 2 && ok; ++half, ++hh) {
-            const uint32_t ab = hh % pf::AST, aph = (hh / pf::AST) & 1;
-            if (!(ok = pf_wait(&sm.a_empty[ab], aph ^ 1, limit, st, 0x322, abort_flag))) break;
-            tc_fence_after();
+          // Both halves' slots first, then both halves stored, one store wait and
+          // both arrivals (the MMA issuer waits for the second half only).
+          const uint32_t ab0 = hh % pf::AST, ab1 = (hh + 1) % pf::AST;
+          if (!(ok = pf_wait(&sm.a_empty[ab0], ((hh / pf::AST) & 1) ^ 1, limit, st, 0x322, abort_flag))) break;
+          if (!(ok = pf_wait(&sm.a_empty[ab1], (((hh + 1) / pf::AST) & 1) ^ 1, limit, st, 0x322, abort_flag))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t ab = half ? ab1 : ab0;
             const uint32_t a_tmem = tmem + lane_addr + TL::kTmemA + ab * 32;
 #pragma unroll
             for (int wp = 0; wp < 2; ++wp) {  // 16 columns (two words) per store
@@ -427,11 +432,15 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
               }
               tmem_st16(a_tmem + 16 * wp, regs);
             }
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.a_full[ab]);
           }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&sm.a_full[ab0]);
+            mbar_arrive(&sm.a_full[ab1]);
+          }
+          hh += 2;
         }
       }
     }
