@@ -18,6 +18,16 @@
  *               [ja] §2.2; [en] §2.B "Routing Mechanism", "Dynamic Adjustment".
  *   mobi_gemm   y_t = x_t . (sum_{s <= k_t} deq(slice_s))^T, fp32 accumulation.
  *               [ja] §2.1 (W^(b) = sum W_e); [en] §2.A "Elasticity".
+ * and, built on them:
+ *   mobi_linear          routing + GEMM in one call.
+ *   mobi_linear_grouped  up to MOBI_MAX_GROUP decode-sized mobi_linear problems
+ *                        in one step (mobi_gemm_grouped: the GEMM half).
+ *   mobi_route_mlp       threshold routing with a two-layer MLP scorer
+ *                        ([ja] §2.2; [en] §2.B "Differentiable Gating").
+ *   mobi_pack_bits       generic slicing: 1- or 2-bit slices, wider groups.
+ *   mobi_ckpt_*          many-in-one checkpoints of packed layers.
+ *   mobi_gemm_path, mobi_gemm_decode_noalloc, mobi_sync_check and the size
+ *   and status helpers.
  *
  * Conventions shared by every entry point
  *   - Every pointer argument is a DEVICE pointer (allocated by the caller, e.g.
