@@ -168,13 +168,9 @@ class DecodeCase:
         self.off = torch.empty(4, dtype=torch.int32, device=dev)
         self.Y = torch.empty((T, N), dtype=torch.float32, device=dev)
         self.Y_host = torch.empty((T, N), dtype=torch.float32).pin_memory()
-        self.ws_r = torch.empty(max(mobi.mobi_route_workspace_bytes(T, K, 3), 16), dtype=torch.uint8, device=dev)
         self.ws_g = torch.empty(mobi.mobi_gemm_workspace_bytes(T, N, K, 3), dtype=torch.uint8, device=dev)
         self.ws_l = torch.empty(max(mobi.mobi_linear_workspace_bytes(T, N, K, 3), 16), dtype=torch.uint8, device=dev)
         self.mobi = mobi
-
-    def route(self):
-        self.mobi.mobi_route(self.X, self.Wr, None, self.k_t, self.perm, self.off, self.ws_r)
 
     def gemm(self):
         self.mobi.mobi_gemm(self.X, self.k_t, self.perm, self.off, self.codes, self.sz, self.N, Y=self.Y, ws=self.ws_g)
