@@ -123,8 +123,12 @@ MOBI_API size_t mobi_sz_bytes(int64_t N, int64_t K, int S, int G);
 /* Scratch bytes that mobi_route needs for T tokens (may be 0). */
 MOBI_API size_t mobi_route_workspace_bytes(int64_t T, int64_t K, int S);
 
-/* Scratch bytes that mobi_gemm needs (covers both the decode and the prefill
- * kernels, so one buffer serves every T up to the given one). */
+/* Scratch bytes that mobi_gemm needs for exactly this T on the current device
+ * (covers both the decode and the prefill kernels, so mobi_gemm_path may pick
+ * either). The prefill kernel splits K into chunks when that shortens the
+ * launch, and the split depends on T, N, K and the SM count, so the size is
+ * not monotone in T: query it for each T used. A smaller buffer is refused
+ * with MOBI_ERR_WORKSPACE. */
 MOBI_API size_t mobi_gemm_workspace_bytes(int64_t T, int64_t N, int64_t K, int S);
 
 /*
