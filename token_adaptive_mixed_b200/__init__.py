@@ -4,7 +4,8 @@ A thin ctypes binding over ``libmobi.so`` (the C ABI declared in
 ``include/mobi.h``). Every function here only marshals torch tensors into
 pointers, sizes and the current CUDA stream; all arithmetic runs in the
 library's sm_100a kernels. There is no CPU fallback: if the library is missing
-or a tensor is not on a CUDA device, the call raises.
+or a tensor is not on a CUDA device, the call raises (the checkpoint calls,
+which move bytes between a file and memory, also take host tensors).
 
 Entry points (same names as the C ABI):
   mobi_pack(W, S, G, bits)          MoBiSlice packing   -> (codes, sz)
@@ -14,6 +15,7 @@ Entry points (same names as the C ABI):
   mobi_gemm_path(..., path)         the same with a forced kernel
   mobi_linear(X, Wr, bias, codes, sz, N)  route + GEMM in one call -> (Y, k_t, perm, offsets)
   mobi_linear_grouped(problems)     up to 8 decode-sized mobi_linear problems in one step
+  mobi_gemm_grouped(problems)       the GEMM half of it (k_t given)
   mobi_ckpt_save / MobiCheckpoint   many-in-one checkpoint of packed layers (load any slice count)
   mobi_sync_check()                 sync + device-side error word
 """
