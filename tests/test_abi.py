@@ -39,6 +39,10 @@ def test_every_declared_symbol_is_exported(L):
 def test_status_strings_and_sizes(L):
     assert mobi.mobi_status_string(0) == "MOBI_OK"
     assert mobi.mobi_status_string(6) == "MOBI_ERR_TIMEOUT"
+    assert mobi.mobi_status_string(7) == "MOBI_ERR_IO"
+    assert [mobi.mobi_status_string(i) for i in range(8)] == mobi.STATUS_NAMES
+    assert mobi.mobi_codes_bytes(4096, 4096, 4) == 4 * 4096 * 256 * 4  # four slices (generic slicing)
+    assert mobi.mobi_codes_bytes(4096, 4096, 5) == 0
     assert mobi.mobi_version() >= 100
     assert mobi.mobi_codes_bytes(4096, 4096, 3) == 3 * 4096 * 256 * 4
     assert mobi.mobi_sz_bytes(4096, 4096, 3, 128) == 3 * 4096 * 32 * 4
