@@ -149,6 +149,36 @@ def test_damaged_table_and_foreign_files(ckpt_file, tmp_path):
         mobi.MobiCheckpoint(tmp_path / "missing.mobi")
 
 
+def rewrite_entry(path, i, fields):
+    """Overwrite entry i's size and offset fields and re-seal the table with a
+    correct CRC-32C, so only the reader's bounds checks stand between a crafted
+    file and out-of-range reads."""
+    raw = bytearray(path.read_bytes())
+    struct.pack_into("<qqiiQQQQ", raw, 64 + 192 * i + 96, *fields)
+    count, toff, tbytes = struct.unpack_from("<IQQ", raw, 12)
+    struct.pack_into("<I", raw, 32, crc32c_bitwise(bytes(raw[toff:toff + tbytes])))
+    path.write_bytes(bytes(raw))
+
+
+@pytest.mark.parametrize("case", ["huge_N", "wrapping_codes_offset", "wrapping_sz_offset", "slices_past_end"])
+def test_crafted_table_with_valid_crc_is_rejected(ckpt_file, case):
+    path, _ = ckpt_file
+    N, K, G, S, coff, cslice, zoff, zslice = entry_fields(path, 0)
+    if case == "huge_N":  # N * K / 4 no longer fits the bound (and would wrap the slice arithmetic)
+        N2 = 1 << 61
+        f = (N2, K, G, S, coff, (N2 * K // 4) % (1 << 64), zoff, ((K // G) * N2 * 4) % (1 << 64))
+    elif case == "wrapping_codes_offset":  # offset + S * slice wraps past 2^64 to a small number
+        f = (N, K, G, S, (1 << 64) - cslice, cslice, zoff, zslice)
+    elif case == "wrapping_sz_offset":
+        f = (N, K, G, S, coff, cslice, (1 << 64) - zslice, zslice)
+    else:  # a valid-looking entry whose last slice runs past the end of the file
+        f = (N, K, G, S, path.stat().st_size - cslice, cslice, zoff, zslice)
+    rewrite_entry(path, 0, f)
+    with pytest.raises(mobi.MobiError, match="IO"):
+        mobi.MobiCheckpoint(path)
+    assert "corrupt table entry" in mobi.mobi_last_error()
+
+
 def test_truncated_file(ckpt_file, tmp_path):
     path, _ = ckpt_file
     raw = path.read_bytes()

@@ -139,22 +139,31 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // the driver's encoder out of repeated calls on the same buffers.
 struct TmapKey {
   const void* base;
-  uint64_t cols, rows, stride;
-  uint32_t box_cols, box_rows;
-  int elem_bytes, swizzle;
-  bool operator==(const TmapKey& o) const {
-    return base == o.base && cols == o.cols && rows == o.rows && stride == o.stride && box_cols == o.box_cols &&
-           box_rows == o.box_rows && elem_bytes == o.elem_bytes && swizzle == o.swizzle;
-  }
+  uint64_t dims[3], strides[2];
+  uint32_t box[3];
+  int rank, elem_bytes, swizzle;
+  bool operator==(const TmapKey& o) const { return memcmp(this, &o, sizeof *this) == 0; }
 };
 static constexpr int kTmapCache = 64;
 static TmapKey g_tmap_key[kTmapCache];
 static CUtensorMap g_tmap_val[kTmapCache];
 static int g_tmap_n = 0, g_tmap_next = 0;
 
-bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t cols, uint64_t rows,
-                  uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes) {
-  const TmapKey key{base, cols, rows, row_stride_bytes, box_cols, box_rows, elem_bytes, swizzle_bytes};
+// Tiled tensor map of rank 2 or 3: dims[0] innermost (elements), strides[i] the
+// byte stride of dimension i + 1, box in elements.
+static bool make_tmap(CUtensorMap* map, const void* base, int elem_bytes, int rank, const uint64_t* dims,
+                      const uint64_t* strides, const uint32_t* box, int swizzle_bytes) {
+  TmapKey key;
+  memset(&key, 0, sizeof key);  // padding included, so memcmp compares only what is set
+  key.base = base;
+  key.rank = rank;
+  key.elem_bytes = elem_bytes;
+  key.swizzle = swizzle_bytes;
+  for (int i = 0; i < rank; ++i) {
+    key.dims[i] = dims[i];
+    key.box[i] = box[i];
+    if (i + 1 < rank) key.strides[i] = strides[i];
+  }
   {
     std::lock_guard<std::mutex> lock(g_mu);
     for (int i = 0; i < g_tmap_n; ++i)
@@ -166,11 +175,15 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t c
   auto fn = encode_fn();
   if (!fn) return false;
   CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {row_stride_bytes};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  cuuint64_t cdims[3], cstr[2];
+  cuuint32_t cbox[3], estr[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    cdims[i] = dims[i];
+    cbox[i] = box[i];
+    if (i + 1 < rank) cstr[i] = strides[i];
+  }
+  CUresult r = fn(map, dt, (cuuint32_t)rank, const_cast<void*>(base), cdims, cstr, cbox, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
                   : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                   : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
@@ -178,9 +191,9 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t c
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     snprintf(g_last_error, sizeof g_last_error,
-             "cuTensorMapEncodeTiled: CUresult %d (dims %llu x %llu, stride %llu, box %u x %u, swizzle %d)", (int)r,
-             (unsigned long long)cols, (unsigned long long)rows, (unsigned long long)row_stride_bytes, box_cols,
-             box_rows, swizzle_bytes);
+             "cuTensorMapEncodeTiled: CUresult %d (rank %d, dims %llu x %llu x %llu, box %u x %u x %u, swizzle %d)",
+             (int)r, rank, (unsigned long long)dims[0], (unsigned long long)dims[1],
+             (unsigned long long)(rank > 2 ? dims[2] : 1), box[0], box[1], rank > 2 ? box[2] : 1, swizzle_bytes);
   if (r == CUDA_SUCCESS) {
     std::lock_guard<std::mutex> lock(g_mu);
     g_tmap_key[g_tmap_next] = key;
@@ -189,6 +202,13 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t c
     if (g_tmap_n < kTmapCache) ++g_tmap_n;
   }
   return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t cols, uint64_t rows,
+                  uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes) {
+  const uint64_t dims[2] = {cols, rows}, strides[1] = {row_stride_bytes};
+  const uint32_t box[2] = {box_cols, box_rows};
+  return make_tmap(map, base, elem_bytes, 2, dims, strides, box, swizzle_bytes);
 }
 
 }  // namespace mobi
@@ -220,6 +240,11 @@ mobi_status check_matrix(int64_t N, int64_t K, int G, int S) {
 size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
 }  // namespace
+
+namespace mobi {
+mobi_status status_of(cudaError_t e) { return cuda_status(e); }
+void clear_message() { g_last_error[0] = 0; }
+}  // namespace mobi
 
 extern "C" {
 
@@ -519,6 +544,7 @@ mobi_status mobi_gemm(const void* X, int64_t T, int64_t K, const int32_t* k_t, c
 }
 
 mobi_status mobi_sync_check(void* stream) {
+  g_last_error[0] = 0;
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_status(e);
   DeviceStatus* dst = device_status(&e);
@@ -530,8 +556,12 @@ mobi_status mobi_sync_check(void* stream) {
   const DeviceStatus zero = {};
   e = cudaMemcpy(dst, &zero, sizeof zero, cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return cuda_status(e);
-  if (h.error & kErrTimeout) return MOBI_ERR_TIMEOUT;
-  return MOBI_ERR_INVALID_ARG;  // kErrInputRange: an activation outside the supported range
+  if (h.error & kErrTimeout) {
+    snprintf(g_last_error, sizeof g_last_error, "a bounded wait ran out in a kernel (wait site 0x%x)", h.where);
+    return MOBI_ERR_TIMEOUT;
+  }
+  note_message("an activation of a decode call (T <= 16) had |x| >= 2^31");
+  return MOBI_ERR_INVALID_ARG;  // kErrInputRange
 }
 
 mobi_status mobi_debug_set_wait_limit(int64_t limit) {

@@ -36,6 +36,8 @@ constexpr size_t kNameBytes = 96;
 constexpr uint64_t kAlign = 4096;
 constexpr size_t kStageBytes = size_t(16) << 20;  // per pinned staging buffer
 
+constexpr int64_t kMaxCkptDim = int64_t(1) << 28;  // largest N or K of a stored tensor (as the GEMM)
+
 struct Entry {
   char name[kNameBytes];
   int64_t N, K;
@@ -299,7 +301,7 @@ mobi_status mobi_ckpt_open(const char* path, mobi_ckpt** out) {
   memcpy(&tcrc, hdr + 32, 4);
   if (ver != kVersion) return fail("unsupported checkpoint version");
   if (cnt == 0 || cnt > (1u << 20) || tbytes != (uint64_t)cnt * kEntryBytes || toff < kHeaderBytes ||
-      toff + tbytes > fsize)
+      toff > fsize || tbytes > fsize - toff)
     return fail("corrupt table header");
   std::vector<uint8_t> table((size_t)tbytes);
   if (!pread_all(fd, table.data(), table.size(), toff)) return fail("truncated table");
@@ -312,11 +314,14 @@ mobi_status mobi_ckpt_open(const char* path, mobi_ckpt** out) {
     Entry& e = c->entries[i];
     memcpy(&e, table.data() + (size_t)i * kEntryBytes, sizeof(Entry));
     e.name[kNameBytes - 1] = 0;
-    const bool ok = e.N > 0 && e.K > 0 && e.G > 0 && e.K % e.G == 0 && e.S >= 1 && e.S <= kMaxSlices &&
-                    e.codes_slice == (uint64_t)e.N * (uint64_t)e.K / 4 &&
-                    e.sz_slice == (uint64_t)(e.K / e.G) * (uint64_t)e.N * 4 &&
-                    e.codes_off + e.codes_slice * (uint64_t)e.S <= fsize &&
-                    e.sz_off + e.sz_slice * (uint64_t)e.S <= fsize;
+    // Sizes bounded as for the GEMM (N, K <= 2^28), so the products below stay
+    // under 2^59; offsets are compared by subtraction, so nothing can wrap.
+    const bool dims_ok = e.N > 0 && e.K > 0 && e.N <= kMaxCkptDim && e.K <= kMaxCkptDim && e.G > 0 &&
+                         e.K % e.G == 0 && e.S >= 1 && e.S <= kMaxSlices;
+    const bool ok = dims_ok && e.codes_slice == (uint64_t)e.N * (uint64_t)e.K / 4 &&
+                    e.sz_slice == (uint64_t)(e.K / e.G) * (uint64_t)e.N * 4 && e.codes_off <= fsize &&
+                    e.codes_slice * (uint64_t)e.S <= fsize - e.codes_off && e.sz_off <= fsize &&
+                    e.sz_slice * (uint64_t)e.S <= fsize - e.sz_off;
     if (!ok) {
       delete c;
       return fail("corrupt table entry");

@@ -788,10 +788,11 @@ cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, c
 
 // ---- the decode GEMM with static scratch (mobi_gemm_decode_noalloc) -------------------
 //
-// For callers that cannot allocate: the decode scratch (staged activations,
-// group sums, split-K tickets and partials) lives in one file-scope array of
-// static device memory instead of a caller workspace. The kernels are the ones
-// above; only the scratch pointer differs.
+// For callers that cannot allocate: the decode scratch (the per-chunk fp32
+// partial sums [chunk][T][N] for up to 16 tokens, used when K spans more than
+// one 1024-column chunk) lives in one file-scope array of static device memory
+// instead of a caller workspace. The kernels are the ones above; only the
+// scratch pointer differs.
 
 namespace mobi {
 
@@ -828,6 +829,7 @@ extern "C" mobi_status mobi_gemm_decode_noalloc(const void* X, int64_t T, int64_
                                                 const uint32_t* codes, const uint32_t* sz, int64_t N, int G,
                                                 int S, float* Y, void* stream) {
   using namespace mobi;
+  clear_message();
   auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   if (N < 0 || K < 0 || T < 0 || S < 1 || S > kMaxSlices) return MOBI_ERR_INVALID_ARG;
   if (G != 128 || K % 128 != 0 || N % 16 != 0 || T > 16 || N > (int64_t(1) << 28) || K > (int64_t(1) << 28))
@@ -842,18 +844,14 @@ extern "C" mobi_status mobi_gemm_decode_noalloc(const void* X, int64_t T, int64_
     char msg[128];
     snprintf(msg, sizeof msg, "decode scratch of %zu bytes exceeds the %zu-byte static array", need,
              kNoAllocScratchBytes);
-    note_error(msg, cudaErrorInvalidValue);
+    note_message(msg);
     return MOBI_ERR_WORKSPACE;
   }
   cudaError_t e;
   DeviceStatus* st = device_status(&e);
-  if (!st) return MOBI_ERR_CUDA;
+  if (!st) return status_of(e);
   void* scratch = noalloc_scratch(&e);
-  if (!scratch) return MOBI_ERR_CUDA;
-  e = launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, scratch, static_cast<cudaStream_t>(stream), st, false);
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    return MOBI_ERR_CUDA;
-  }
-  return MOBI_OK;
+  if (!scratch) return status_of(e);
+  return status_of(
+      launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, scratch, static_cast<cudaStream_t>(stream), st, false));
 }

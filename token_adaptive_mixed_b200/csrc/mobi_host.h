@@ -9,6 +9,7 @@
 
 #include <cstdint>
 
+#include "../../include/mobi.h"
 #include "mobi_device.cuh"
 
 namespace mobi {
@@ -21,6 +22,11 @@ uint64_t wait_limit();
 cudaError_t note_error(const char* where, cudaError_t e);
 // Record a plain message for mobi_last_error.
 void note_message(const char* msg);
+// Clear the message mobi_last_error returns (each entry point starts with this).
+void clear_message();
+// C-ABI status of a CUDA error: MOBI_OK, or MOBI_ERR_CUDA with the error kept
+// for mobi_last_error and a sticky launch error cleared.
+mobi_status status_of(cudaError_t e);
 // Multiprocessor count of the current device (cached).
 int num_sms();
 // Opt a kernel into `bytes` of dynamic shared memory (idempotent).
@@ -69,6 +75,8 @@ struct DecodeJob {
   int64_t N, K;
   int T;
 };
+// Decode scratch of one problem: the per-chunk partial sums when K spans more
+// than one 1024-column chunk.
 size_t decode_ws_bytes(int64_t N, int64_t K);
 // Y[t][n] = sum over chunks c (in order) of partial[c][t][n] (T N % 4 == 0),
 // launched as a programmatic dependent of the kernel before it.
