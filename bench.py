@@ -339,6 +339,21 @@ def time_full_model(mobi, wl, dev, steps, hbm_peak):
     mobi.mobi_sync_check()
     gms = time_graph(gstep, steps)
     mobi.mobi_sync_check()
+
+    # The grouping a real layer allows: q, k, v read the same attention input
+    # and gate, up the same MLP input, while o reads the attention output and
+    # down the activated MLP product, so a layer is four grouped calls
+    # ({q,k,v}, {o}, {gate,up}, {down}; 128 calls per step).
+    dep_groups = [(0, 1, 2), (3,), (4, 5), (6,)]
+    dep_probs = [[pr[j] for j in g] for pr in layer_probs for g in dep_groups]
+
+    def dstep():
+        for pr in dep_probs:
+            mobi.mobi_linear_grouped(pr, ws=gws)
+    dstep()
+    mobi.mobi_sync_check()
+    dms = time_graph(dstep, steps)
+    mobi.mobi_sync_check()
     out = {"workload": "full model: 7 projections x 32 layers (Llama-2-7B shapes), batch 8, random router per "
                        "projection; pack all, then decode through every projection (224 mobi_linear calls, one "
                        "CUDA graph)",
@@ -348,8 +363,14 @@ def time_full_model(mobi, wl, dev, steps, hbm_peak):
            "kmax_histogram": [kmax.count(v) for v in (1, 2, 3)], "steps": steps,
            "grouped_per_layer": {"calls_per_step": len(layer_probs), "decode_ms_per_step": round(gms, 4),
                                  "decode_GB/s": round(bytes_step / gms / 1e6, 1),
-                                 "decode_frac_of_hbm": round(bytes_step / gms / 1e6 / hbm_peak, 4)}}
-    del calls, packed, layers, layer_probs
+                                 "decode_frac_of_hbm": round(bytes_step / gms / 1e6 / hbm_peak, 4),
+                                 "note": "all seven projections of a layer in one call: an upper bound, since "
+                                         "o and down depend on the others' outputs in a real layer"},
+           "grouped_by_dependency": {"groups_per_layer": "{q,k,v}, {o}, {gate,up}, {down}",
+                                     "calls_per_step": len(dep_probs), "decode_ms_per_step": round(dms, 4),
+                                     "decode_GB/s": round(bytes_step / dms / 1e6, 1),
+                                     "decode_frac_of_hbm": round(bytes_step / dms / 1e6 / hbm_peak, 4)}}
+    del calls, packed, layers, layer_probs, dep_probs
     torch.cuda.empty_cache()
     return out
 
@@ -405,8 +426,18 @@ def time_prefill(mobi, L, dev, reps, tf_peak, flush):
             "tflops_issued_step": round(issued / ms_step / 1e9, 2),
             "roofline": {"bound": "tensor", "kernel": "prefill GEMM (gather + tcgen05 prefill kernels)",
                          "achieved": round(issued / ms_gemm / 1e9, 2), "peak": tf_peak, "unit": "TFLOP/s",
-                         "frac": round(issued / ms_gemm / 1e9 / tf_peak, 4), "traffic": None},
+                         "frac": round(issued / ms_gemm / 1e9 / tf_peak, 4),
+                         "traffic": PREFILL_DRAM_BYTES.get(L.name),
+                         "traffic_unit": "bytes per prefill_kernel launch (ncu DRAM read + write)"},
             "reps": reps, "l2": "256 MB flush before each repetition"}
+
+
+# DRAM bytes (read + write) of one prefill_kernel launch, from one ncu capture
+# per workload (dram__bytes_read.sum + dram__bytes_write.sum; the summary and
+# command are in profiles/small_kernels_prefill_11008x4096.md). Valid while the
+# prefill kernel is unchanged.
+PREFILL_DRAM_BYTES = {"prefill_11008x4096_T2048": 62713344 + 46622464,
+                      "skewed_prefill_28672x8192_T4096": 1596453376 + 446456320}
 
 
 # fp32 FMA peak of the SIMT pipes: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz
@@ -529,34 +560,46 @@ def time_ckpt(mobi, wl, dev, reps=3):
 def time_generic(mobi, wl, dev, hbm_peak, tf_peak, flush, steps=200):
     """Generic slicing: four 1-bit slices (1..4 bits per weight), G = 128.
     (a) the decode step of the three Llama-7B shapes at T = 4 as one
-    mobi_linear_grouped call, router mix 1/4 each; (b) the prefill workload's
-    shape (T = 2048, 11008 x 4096) through route + prefill GEMM. 1-bit codes
-    sit in 2-bit fields, so the bytes read are those of 2-bit slices."""
+    mobi_linear_grouped call, router mix 1/4 each (three packed copies in
+    rotation, so no copy is L2-resident when it is read again); (b) the prefill
+    workload's shape (T = 2048, 11008 x 4096) through route + prefill GEMM.
+    1-bit codes sit in 2-bit fields, so the bytes read are those of 2-bit
+    slices: k slices give k bits of precision and cost 2k bits of codes."""
     S = 4
     out = {"slicing": "4 x 1-bit slices, G = 128 (codes stored in 2-bit fields)"}
-    probs = []
-    for i, (N, K) in enumerate(wl.DECODE_SHAPES):
-        L = wl.layer(f"gen_{N}x{K}", N, K, 4, seed=3000 + i, outlier_frac_cols=0.005, S=S, mix=(0.25,) * S)
-        codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(dev), S=S, bits=1)
-        probs.append({"X": L.X.to(dev), "Wr": torch.from_numpy(L.Wr).to(dev), "bias": torch.from_numpy(L.bias).to(dev),
-                      "codes": codes, "sz": sz, "N": N,
-                      "Y": torch.empty((4, N), dtype=torch.float32, device=dev),
-                      "k_t": torch.empty(4, dtype=torch.int32, device=dev),
-                      "perm": torch.empty(4, dtype=torch.int32, device=dev),
-                      "offsets": torch.empty(S + 1, dtype=torch.int32, device=dev)})
-    ws = torch.empty(max(mobi.mobi_linear_grouped_workspace_bytes(probs, S=S), 16), dtype=torch.uint8, device=dev)
+    # Three packed copies of the three problems, run one after another in each
+    # step, so a copy is read again only after ~240 MB of other weights (> 2x L2).
+    copies = 3
+    groups = []
+    for r in range(copies):
+        probs = []
+        for i, (N, K) in enumerate(wl.DECODE_SHAPES):
+            L = wl.layer(f"gen_{N}x{K}", N, K, 4, seed=3000 + i, outlier_frac_cols=0.005, S=S, mix=(0.25,) * S)
+            codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(dev), S=S, bits=1)
+            probs.append({"X": L.X.to(dev), "Wr": torch.from_numpy(L.Wr).to(dev),
+                          "bias": torch.from_numpy(L.bias).to(dev), "codes": codes, "sz": sz, "N": N,
+                          "Y": torch.empty((4, N), dtype=torch.float32, device=dev),
+                          "k_t": torch.empty(4, dtype=torch.int32, device=dev),
+                          "perm": torch.empty(4, dtype=torch.int32, device=dev),
+                          "offsets": torch.empty(S + 1, dtype=torch.int32, device=dev)})
+        groups.append(probs)
+    ws = torch.empty(max(mobi.mobi_linear_grouped_workspace_bytes(groups[0], S=S), 16), dtype=torch.uint8,
+                     device=dev)
 
     def step():
-        mobi.mobi_linear_grouped(probs, S=S, ws=ws)
+        for probs in groups:
+            mobi.mobi_linear_grouped(probs, S=S, ws=ws)
     step()
     mobi.mobi_sync_check()
-    kmax = [int(p["k_t"].max().item()) for p in probs]
-    nbytes = sum(decode_bytes(p["N"], p["X"].shape[1], 4, km) for p, km in zip(probs, kmax))
-    ms = time_graph(step, steps)
-    out["decode_T4_grouped"] = {"kmax_per_problem": kmax, "bytes_per_step": nbytes, "ms_per_step": round(ms, 5),
+    kmax = [int(p["k_t"].max().item()) for p in groups[0]]
+    nbytes = sum(decode_bytes(p["N"], p["X"].shape[1], 4, km) for p, km in zip(groups[0], kmax))
+    ms = time_graph(step, steps) / copies
+    out["decode_T4_grouped"] = {"kmax_per_problem": kmax, "bytes_per_call": nbytes, "ms_per_call": round(ms, 5),
                                 "GB/s": round(nbytes / ms / 1e6, 1), "frac_of_hbm": round(nbytes / ms / 1e6 / hbm_peak, 4),
-                                "bits_per_weight_read": kmax}
-    del probs, ws
+                                "precision_bits_per_weight": kmax,
+                                "code_bits_read_per_weight": [2 * km for km in kmax],
+                                "l2": f"{copies} packed copies in rotation, each read again after ~{2 * nbytes / 1e6:.0f} MB"}
+    del groups, ws
     L = wl.layer("gen_prefill_11008x4096_T2048", 11008, 4096, 2048, seed=3010, n_outlier_cols=20, S=S,
                  mix=(0.25,) * S)
     W = torch.from_numpy(L.W).to(dev)
@@ -839,12 +882,13 @@ def _oracle_case(N, K, T, rows):
     return _ORACLE_CASES[key]
 
 
-def oracle_decode_sample(budget_s: float, cases_spec, rows_cap=None):
+def oracle_decode_sample(budget_s: float, cases_spec, rows_cap=None, nthreads=0):
     """Time the CPU oracle (route + GEMM) on a bounded sample of the decode workload:
     every listed case once, then further passes until `budget_s` of CPU time.
     Returns (bytes credited, seconds, threads, description)."""
     import oracle
-    threads = oracle.max_threads()
+    nthreads = nthreads or len(os.sched_getaffinity(0))
+    threads = nthreads
     credited, spent, done = 0, 0.0, []
     i = 0
     while i < len(cases_spec) or spent < budget_s:
@@ -853,8 +897,8 @@ def oracle_decode_sample(budget_s: float, cases_spec, rows_cap=None):
         rows = N if rows_cap is None else min(N, rows_cap)
         X, Wr, c_sub, s_sub = _oracle_case(N, K, T, rows)
         t0 = time.perf_counter()
-        k, _, _ = oracle.route(X, Wr)
-        oracle.gemm(X, k, c_sub, s_sub, rows)
+        k, _, _ = oracle.route(X, Wr, nthreads=nthreads)
+        oracle.gemm(X, k, c_sub, s_sub, rows, nthreads=nthreads)
         dt = time.perf_counter() - t0
         km = int(k.max())
         credited += km * (rows * K // 4 + rows * (K // 128) * 4) + T * K * 2
@@ -863,13 +907,107 @@ def oracle_decode_sample(budget_s: float, cases_spec, rows_cap=None):
     return credited, spent, threads, "; ".join(done)
 
 
+def _timed(fn):
+    t0 = time.perf_counter()
+    r = fn()
+    return r, time.perf_counter() - t0
+
+
 def cpu_baseline(budget_s=20.0):
+    """The oracle on the host cores, following the measurement protocol: all
+    threads (OpenMP over output rows; each output's reduction order unchanged)
+    on configs 1-3 in full, config 4 on one layer of the stack (pack + batch-8
+    decode of its seven projections, extrapolated x32), config 5 packed in full
+    with its GEMM on a stated token subset (extrapolated to T = 4096); then one
+    thread on a bounded sample. `value` is the decode workload's rate (config 2,
+    all threads) in the headline unit."""
+    import oracle
     from token_adaptive_mixed_b200 import workloads as wl
-    spec = [(N, K, T) for (N, K) in wl.DECODE_SHAPES for T in wl.DECODE_TOKENS]
-    credited, spent, threads, desc = oracle_decode_sample(budget_s, spec, rows_cap=4096)
-    return {"value": round(credited / spent / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"oracle route + fp64 GEMM on the first 4096 rows of the decode cases, cycling through the "
-                      f"nine cases until ~{budget_s:.0f}s of CPU time ({len(desc.split(';'))} GEMVs, {spent:.1f}s)"}
+    oracle.build()
+    cores = len(os.sched_getaffinity(0))
+    nt = cores
+    proto = {"threads_all": cores}
+
+    def gemm_rate(macs, sec):
+        return round(2.0 * macs / sec / 1e9, 3)  # GFLOP/s (fp64)
+
+    # config 1: pack + route + GEMM, T = 16
+    L = wl.tiny()
+    (c, z, _), tp = _timed(lambda: oracle.pack(L.W, S=3, nthreads=nt))
+    (k, _, _), tr = _timed(lambda: oracle.route(L.X, L.Wr, nthreads=nt))
+    _, tg = _timed(lambda: oracle.gemm(L.X, k, c, z, L.N, nthreads=nt))
+    proto["config1_tiny"] = {"s": round(tp + tr + tg, 4), "pack_s": round(tp, 4), "route_s": round(tr, 4),
+                             "gemm_s": round(tg, 4)}
+    # config 2: the nine decode problems (route + GEMM), packs timed apart
+    dec_bytes, dec_s, pack_s = 0, 0.0, 0.0
+    for (N, K) in wl.DECODE_SHAPES:
+        L1 = wl.decode(N, K, 1)
+        (c, z, _), tp = _timed(lambda: oracle.pack(L1.W, S=3, nthreads=nt))
+        pack_s += tp
+        for T in wl.DECODE_TOKENS:
+            L = wl.decode(N, K, T)
+            def run():
+                k, _, _ = oracle.route(L.X, L.Wr, nthreads=nt)
+                oracle.gemm(L.X, k, c, z, N, nthreads=nt)
+                return k
+            k, dt = _timed(run)
+            dec_bytes += decode_bytes(N, K, T, int(k.max()))
+            dec_s += dt
+    proto["config2_decode"] = {"s": round(dec_s, 3), "bytes": dec_bytes, "GB/s": round(dec_bytes / dec_s / 1e9, 4),
+                               "pack_s_three_shapes": round(pack_s, 3)}
+    # config 3: the whole prefill workload
+    L = wl.prefill()
+    (c, z, _), tp = _timed(lambda: oracle.pack(L.W, S=3, nthreads=nt))
+    (k, _, _), tr = _timed(lambda: oracle.route(L.X, L.Wr, L.bias, nthreads=nt))
+    _, tg = _timed(lambda: oracle.gemm(L.X, k, c, z, L.N, nthreads=nt))
+    macs = L.T * L.N * L.K
+    proto["config3_prefill"] = {"s": round(tp + tr + tg, 3), "pack_s": round(tp, 3), "route_s": round(tr, 3),
+                                "gemm_s": round(tg, 3), "gemm_GFLOP/s_effective": gemm_rate(macs, tg)}
+    # config 4: one layer (7 projections) of the 32-layer stack, extrapolated x32
+    lay_pack, lay_dec, params = 0.0, 0.0, 0
+    for pi in range(len(wl.LLAMA7B_PROJECTIONS)):
+        Lp = wl.full_model_projection(0, pi, T=8, device="cpu")
+        W = Lp.W.numpy()
+        (c, z, _), tp = _timed(lambda: oracle.pack(W, S=3, nthreads=nt))
+        def run():
+            k, _, _ = oracle.route(Lp.X, Lp.Wr, nthreads=nt)
+            oracle.gemm(Lp.X, k, c, z, Lp.N, nthreads=nt)
+        _, td = _timed(run)
+        lay_pack += tp
+        lay_dec += td
+        params += Lp.N * Lp.K
+    layers = wl.LLAMA7B_LAYERS
+    proto["config4_full_model"] = {"measured": "layer 0 (7 projections), extrapolated x32", "params_layer": params,
+                                   "pack_s_layer": round(lay_pack, 3), "decode_s_layer": round(lay_dec, 3),
+                                   "pack_s_model": round(lay_pack * layers, 2),
+                                   "decode_s_per_step_model": round(lay_dec * layers, 2)}
+    # config 5: pack in full, GEMM on a token subset (every bucket), extrapolated to all tokens
+    L = wl.skewed_prefill()
+    (c, z, _), tp = _timed(lambda: oracle.pack(L.W, S=3, nthreads=nt))
+    (k, _, _), tr = _timed(lambda: oracle.route(L.X, L.Wr, L.bias, nthreads=nt))
+    sub = np.arange(0, L.T, L.T // 128, dtype=np.int32)
+    _, tg = _timed(lambda: oracle.gemm(L.X, k, c, z, L.N, tokens=sub, nthreads=nt))
+    proto["config5_skewed_prefill"] = {"pack_s": round(tp, 3), "route_s": round(tr, 3),
+                                       "gemm_tokens": int(sub.size), "gemm_s_subset": round(tg, 3),
+                                       "gemm_s_all_tokens_extrapolated": round(tg * L.T / sub.size, 2),
+                                       "gemm_GFLOP/s_effective": gemm_rate(sub.size * L.N * L.K, tg)}
+    # one thread: the decode sample (first 4096 rows of every case) and a 32-token prefill subset
+    credited, spent, _, desc = oracle_decode_sample(0.0, [(N, K, T) for (N, K) in wl.DECODE_SHAPES
+                                                          for T in wl.DECODE_TOKENS], rows_cap=1024, nthreads=1)
+    L = wl.prefill()
+    c, z, _ = oracle.pack(L.W[:1024], S=3, nthreads=1)
+    k, _, _ = oracle.route(L.X, L.Wr, L.bias, nthreads=1)
+    sub = np.arange(0, L.T, L.T // 32, dtype=np.int32)
+    _, tg1 = _timed(lambda: oracle.gemm(L.X, k, c, z, 1024, tokens=sub, nthreads=1))
+    proto["single_thread"] = {"decode_GB/s": round(credited / spent / 1e9, 4),
+                              "decode_sample": "first 1024 rows of each of the nine decode cases",
+                              "prefill_gemm_GFLOP/s_effective": gemm_rate(sub.size * 1024 * L.K, tg1),
+                              "prefill_sample": "32 tokens x first 1024 rows of config 3"}
+    value = dec_bytes / dec_s / 1e9
+    return {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": "config 2 in full (nine decode problems, oracle route + fp64 GEMM, all threads); the "
+                      "protocol below covers configs 1-5 and one thread",
+            "protocol": proto}
 
 
 def run_reference(args, world, rank):
@@ -895,7 +1033,7 @@ def run_reference(args, world, rank):
             "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": WORKLOAD, "parallelism": "host cores"},
-            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.max_threads(),
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": len(os.sched_getaffinity(0)),
                              "kind": "oracle",
                              "sample": f"per step: oracle route + fp64 GEMM on the first {rows} rows of one decode case, "
                                        f"cycling through the nine cases"},

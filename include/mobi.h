@@ -43,8 +43,15 @@
  *     mobi_pack_bits), K % 128 == 0, N % 16 == 0, T >= 0. K, N, T up to 2^30 elements per
  *     dimension and N*K, T*K, T*N below 2^40.
  *   - A device-side bounded wait that runs out sets a per-device error word;
- *     the next call on that device (or mobi_sync_check) reports
- *     MOBI_ERR_TIMEOUT and clears it.
+ *     mobi_sync_check reports it as MOBI_ERR_TIMEOUT (naming the wait site in
+ *     mobi_last_error) and clears it.
+ *   - Activation range of the decode kernel (every GEMM with T <= 16, and
+ *     every grouped or no-alloc call): |x| < 2^31. The kernel feeds x * 2^(96 - 2f)
+ *     to the tensor cores as bf16 (so that subnormal code operands stay exact),
+ *     which overflows from 2^31 on. A larger |x| (or a NaN/Inf) is not checked
+ *     on the host; the kernel flags it and mobi_sync_check returns
+ *     MOBI_ERR_INVALID_ARG for that call (its outputs are then unspecified).
+ *     The prefill kernel (T > 16) takes any finite bf16.
  *   - The library keeps no per-call host state and is reentrant.
  *
  * Packed format (one checkpoint serves every precision: [ja] §3 "Many-in-One";
@@ -445,16 +452,20 @@ MOBI_API mobi_status mobi_gemm_decode_noalloc(const void* X, int64_t T, int64_t 
 /*
  * mobi_sync_check — synchronise `stream`, then report and clear the
  * device-side error word of the current device. Returns MOBI_ERR_TIMEOUT if a
- * bounded wait ran out since the last check, MOBI_ERR_CUDA on a CUDA error.
+ * bounded wait ran out since the last check (mobi_last_error names the wait
+ * site), MOBI_ERR_INVALID_ARG if a decode call met an activation with
+ * |x| >= 2^31 (see the activation range above), MOBI_ERR_CUDA on a CUDA error,
+ * MOBI_OK otherwise.
  */
 MOBI_API mobi_status mobi_sync_check(void* stream);
 
 /*
  * mobi_debug_set_wait_limit — set the iteration limit of the device-side
  * bounded waits of the current device (0 restores the default). A tiny limit
- * makes the prefill kernel's waits run out, which exercises the timeout path
- * without faulting anything: the kernel records the error, drains its own
- * copies in flight, frees its tensor memory and returns. Test use only.
+ * makes the decode and prefill kernels' waits run out, which exercises the
+ * timeout path without faulting anything: the kernel records the error, drains
+ * its own copies (and MMAs) in flight, frees its tensor memory and returns.
+ * Test use only.
  */
 MOBI_API mobi_status mobi_debug_set_wait_limit(int64_t limit);
 

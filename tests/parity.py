@@ -24,6 +24,25 @@ def check_gemm(y_gpu: np.ndarray, y_ref: np.ndarray, what: str = "") -> dict:
     return stats
 
 
+CANARY_BITS = 0x7FC0DEAD  # a quiet-NaN pattern no kernel writes
+
+
+def guarded_output(T: int, N: int, device: str = "cuda:0", pad: int = 64):
+    """Y [T, N] fp32 inside a buffer with `pad` canary words on each side (pad a
+    multiple of 4 keeps Y 16-byte aligned). Returns (Y, check) where check()
+    asserts every canary word is unchanged: nothing was written outside Y."""
+    import torch
+    buf = torch.full((pad + T * N + pad,), CANARY_BITS, dtype=torch.int32, device=device)
+    Y = buf[pad:pad + T * N].view(torch.float32).view(T, N)
+
+    def check(what: str = ""):
+        b = buf.cpu().numpy().view(np.uint32)
+        head, tail = b[:pad], b[pad + T * N:]
+        assert np.all(head == CANARY_BITS) and np.all(tail == CANARY_BITS), \
+            f"{what}: writes outside Y (head {np.count_nonzero(head != CANARY_BITS)}, tail {np.count_nonzero(tail != CANARY_BITS)})"
+    return Y, check
+
+
 def check_route(k_gpu: np.ndarray, k_ref: np.ndarray, gap_ref: np.ndarray, what: str = "") -> int:
     diff = np.nonzero(np.asarray(k_gpu) != np.asarray(k_ref))[0]
     near = gap_ref[diff] < TIE_BAND

@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from parity import check_gemm, check_route
+from parity import check_gemm, check_route, guarded_output
 from token_adaptive_mixed_b200 import workloads as wl
 
 pytestmark = pytest.mark.gpu
@@ -128,13 +128,17 @@ def test_route_ties_lowest_index(mobi):
 
 # ---- decode GEMM ---------------------------------------------------------------------
 
-def run_gemm(mobi, L, codes, sz, k, path=0):
-    X = L.X.to(DEV)
+def run_gemm(mobi, L, codes, sz, k, path=0, X=None):
+    """The GEMM on the GPU with canary words around Y (checked: nothing written
+    outside the output)."""
+    X = (L.X if X is None else X).to(DEV)
     k_t = torch.from_numpy(k.astype(np.int32)).to(DEV)
     perm = torch.from_numpy(np.argsort(k, kind="stable").astype(np.int32)).to(DEV)
     off = torch.from_numpy(np.concatenate([[0], np.cumsum(np.bincount(k, minlength=4)[1:])]).astype(np.int32)).to(DEV)
-    Y = mobi.mobi_gemm_path(X, k_t, perm, off, to_dev_u32(codes), to_dev_u32(sz), L.N, path=path)
+    Y, guards = guarded_output(X.shape[0], L.N)
+    mobi.mobi_gemm_path(X, k_t, perm, off, to_dev_u32(codes), to_dev_u32(sz), L.N, path=path, Y=Y)
     mobi.mobi_sync_check()
+    guards(f"N={L.N} K={L.K} T={X.shape[0]}")
     return Y.cpu().numpy()
 
 
@@ -192,3 +196,37 @@ def test_decode_llama_shapes_full(mobi, oracle, N, K):
     Y = mobi.mobi_gemm(X, k_t, perm, off, codes_t, sz_t, N)
     mobi.mobi_sync_check()
     check_gemm(Y.cpu().numpy(), oracle.gemm(L.X, k, codes, sz, N), f"decode {N}x{K}")
+
+
+def test_decode_activation_range(mobi, oracle):
+    """The decode kernel takes |x| < 2^31 (it scales x by up to 2^96 in bf16).
+    One x = 2^31 is reported by mobi_sync_check as MOBI_ERR_INVALID_ARG; the
+    largest bf16 below 2^31 is accepted (within the bars and the fp32
+    cancellation bound of the folded zero point); the prefill kernel (any T)
+    has no such limit; the context stays usable."""
+    L = wl.tiny(4)
+    codes, sz, _ = oracle.pack(L.W, S=3)
+    k = np.array([3, 1, 2, 3], np.int32)
+    big = L.X.clone()
+    big[1, 5] = 2.0 ** 31
+    with pytest.raises(mobi.MobiError) as ei:
+        run_gemm(mobi, L, codes, sz, k, path=1, X=big)
+    assert ei.value.status == 1 and "2^31" in mobi.mobi_last_error()
+    check_gemm(run_gemm(mobi, L, codes, sz, k, path=2, X=big), oracle.gemm(big, k, codes, sz, L.N), "prefill, x=2^31")
+    edge = L.X.clone()
+    edge[1, 5] = 2.0 ** 31 - 2.0 ** 23  # bf16 0x4EFF, the largest bf16 below 2^31
+    assert float(edge[1, 5]) == 2.0 ** 31 - 2.0 ** 23
+    # Accepted and finite; the zero point is folded as sum x q - z sum x in fp32,
+    # so the absolute error grows with |x|: per (slice, group) both terms are at
+    # most 3 sum|x| and the fp32 sums (tensor core, then one fma each) round at
+    # most ~32 times by u = 2^-24, i.e. |err| <= 2^-18 sum_s sum_g scale * 3 sum_g |x|
+    # on top of the element bar. The relative Frobenius bar holds as usual.
+    y = run_gemm(mobi, L, codes, sz, k, path=1, X=edge)
+    y_ref = oracle.gemm(edge, k, codes, sz, L.N)
+    assert np.isfinite(y).all()
+    xs = np.abs(edge.float().numpy().astype(np.float64)).reshape(edge.shape[0], -1, 128).sum(2)  # [T][K/128]
+    scale = (sz & 0xFFFF).astype(np.uint16).view(np.float16).astype(np.float64)  # [S][K/128][N]
+    allow = np.stack([2.0 ** -18 * 3 * np.einsum("sgn,g->n", scale[:k[t]], xs[t]) for t in range(len(k))])
+    assert np.all(np.abs(y - y_ref) <= 1e-2 * (np.abs(y_ref) + 1e-3) + allow)
+    assert np.linalg.norm(y - y_ref) <= 2e-3 * np.linalg.norm(y_ref)
+    check_gemm(run_gemm(mobi, L, codes, sz, k, path=1), oracle.gemm(L.X, k, codes, sz, L.N), "decode after the error")

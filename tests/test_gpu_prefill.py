@@ -2,7 +2,9 @@
 
 Sizes span several weight tiles (128 rows) and token tiles (192 tokens) with
 ragged tails, every mix of slice counts, tokens unsorted (the routing order is
-applied inside), and the full prefill workloads on sampled tokens. The bar is
+applied inside), and the full prefill workloads: every token of the 2048-token
+one; for the 4096-token skewed one every x8-scaled token and whole 192-token
+tiles of every bucket. The bar is
 max |y - y_ref| <= 1e-2 (|y_ref| + 1e-3) element-wise and a relative
 Frobenius error <= 2e-3.
 """
@@ -10,7 +12,7 @@ import numpy as np
 import pytest
 import torch
 
-from parity import check_gemm, check_route
+from parity import check_gemm, check_route, guarded_output
 from token_adaptive_mixed_b200 import workloads as wl
 
 pytestmark = pytest.mark.gpu
@@ -37,10 +39,14 @@ def bucket_host(k):
 
 
 def gemm(mobi, X, k, codes, sz, N, path):
+    """The GEMM on the GPU with canary words around Y (checked: nothing written
+    outside the output, ragged token and row tails included)."""
     perm, off = bucket_host(k)
-    Y = mobi.mobi_gemm_path(X.to(DEV), torch.from_numpy(k).to(DEV), torch.from_numpy(perm).to(DEV),
-                            torch.from_numpy(off).to(DEV), u32(codes), u32(sz), N, path=path)
+    Y, guards = guarded_output(X.shape[0], N)
+    mobi.mobi_gemm_path(X.to(DEV), torch.from_numpy(k).to(DEV), torch.from_numpy(perm).to(DEV),
+                        torch.from_numpy(off).to(DEV), u32(codes), u32(sz), N, path=path, Y=Y)
     mobi.mobi_sync_check()
+    guards(f"N={N} T={X.shape[0]} path={path}")
     return Y.cpu().numpy()
 
 
@@ -104,7 +110,11 @@ def test_prefill_one_slice(mobi, oracle):
     check_gemm(Y.cpu().numpy(), oracle.gemm(L.X, k, codes, sz, N, S=1), "S=1")
 
 
-def _full_workload(mobi, oracle, L, n_sample):
+def _full_workload(mobi, oracle, L, pick_tokens):
+    """Pack, route and GEMM the whole workload on the GPU (as the benchmark's
+    prefill does); then pack bit-exact on sampled rows, routing on every token,
+    and every output row n < N of the tokens pick_tokens(k) selects against the
+    oracle."""
     W = torch.from_numpy(L.W).to(DEV)
     codes_t, sz_t = mobi.mobi_pack(W, S=3)
     X = L.X.to(DEV)
@@ -120,25 +130,48 @@ def _full_workload(mobi, oracle, L, n_sample):
     k_ref, gap, _ = oracle.route(L.X, L.Wr, L.bias)
     k_gpu = k_t.cpu().numpy()
     check_route(k_gpu, k_ref, gap)
-    # sampled tokens: some from every bucket, plus the first and last
-    rng = np.random.default_rng(2)
-    toks = [0, L.T - 1]
-    for j in (1, 2, 3):
-        idx = np.nonzero(k_gpu == j)[0]
-        if idx.size:
-            toks += list(rng.choice(idx, min(n_sample // 3, idx.size), replace=False))
-    toks = np.array(sorted(set(int(t) for t in toks)), np.int32)
+    assert np.array_equal(perm.cpu().numpy(), np.argsort(k_gpu, kind="stable"))
+    toks = np.asarray(sorted(set(int(t) for t in pick_tokens(k_gpu))), np.int32)
     ref = oracle.gemm(L.X, k_gpu, codes, sz, L.N, tokens=toks)
-    return check_gemm(Y.cpu().numpy()[toks], ref, L.name)
+    check_gemm(Y.cpu().numpy()[toks], ref, L.name)
+    return toks
+
+
+def bucket_tiles(k, tile=192, per_bucket=2):
+    """Tokens of whole 192-token tiles in bucket order (the prefill kernel's token
+    tiles): the first and last tile, and `per_bucket` tiles lying wholly inside
+    each slice-count bucket (the first ones of the bucket and the last)."""
+    perm = np.argsort(k, kind="stable")
+    T = len(k)
+    starts = {0, (T - 1) // tile * tile}
+    for j in (1, 2, 3):
+        idx = np.nonzero(k[perm] == j)[0]
+        if idx.size == 0:
+            continue
+        lo = (idx[0] + tile - 1) // tile * tile        # first tile starting inside the bucket
+        hi = (idx[-1] + 1) // tile * tile - tile        # last tile ending inside it
+        inside = list(range(lo, hi + 1, tile)) if hi >= lo else [idx[0] // tile * tile]
+        starts.update(inside[:per_bucket - 1] + inside[-1:])
+    return np.concatenate([perm[s:s + tile] for s in sorted(starts)])
 
 
 @pytest.mark.slow
 def test_prefill_workload_full_size(mobi, oracle):
-    """T=2048, N=11008, K=4096, thirds: sampled tokens against the oracle (all N)."""
-    _full_workload(mobi, oracle, wl.prefill(), 24)
+    """T=2048, N=11008, K=4096, thirds: every token and every output row against the oracle."""
+    L = wl.prefill()
+    toks = _full_workload(mobi, oracle, L, lambda k: range(len(k)))
+    assert len(toks) == L.T
 
 
 @pytest.mark.slow
 def test_skewed_prefill_workload_full_size(mobi, oracle):
-    """T=4096, N=28672, K=8192, 70/20/10 with 2% tokens x8: sampled tokens."""
-    _full_workload(mobi, oracle, wl.skewed_prefill(), 12)
+    """T=4096, N=28672, K=8192, 70/20/10 with 2% of tokens x8: every x8 token,
+    two whole 192-token tiles inside each bucket plus the first and last tile of
+    the bucket order, all output rows, against the oracle."""
+    L = wl.skewed_prefill()
+    assert len(L.scaled_tokens) == 82
+
+    def pick(k):
+        return np.concatenate([L.scaled_tokens, bucket_tiles(k)])
+    toks = _full_workload(mobi, oracle, L, pick)
+    assert set(L.scaled_tokens.tolist()) <= set(toks.tolist())

@@ -1,9 +1,11 @@
 """Failure detection without a GPU fault: the bounded device waits.
 
-A tiny wait limit makes the prefill kernel's first mbarrier wait run out (as a
-flag that is never set would). The kernel must record MOBI_ERR_TIMEOUT, drain
-its copies and MMAs, free tensor memory and return, leaving the context usable:
-the next call with the default limit must be correct again.
+A tiny wait limit makes a kernel's first mbarrier wait (or the decode
+producer's first poll of a full ring) run out, as a flag that is never set
+would. The kernel must record MOBI_ERR_TIMEOUT, drain its copies (and, in the
+prefill kernel, its MMAs and tensor memory) and return, leaving the context
+usable: the next call with the default limit must be correct again. Covered
+for the prefill kernel and the decode kernel (both fragment classes).
 """
 import numpy as np
 import pytest
@@ -39,3 +41,34 @@ def test_timeout_is_reported_and_context_survives(oracle):
     Y = mobi.mobi_gemm_path(*args, path=2)
     mobi.mobi_sync_check()
     check_gemm(Y.cpu().numpy(), oracle.gemm(L.X, k, codes, sz, N), "after timeout")
+
+
+@pytest.mark.parametrize("T", [4, 16])
+def test_decode_timeout_is_reported_and_context_survives(oracle, T):
+    import token_adaptive_mixed_b200 as mobi
+    # Enough 32-row blocks per CTA (~24 stages per team against rings of 6 or 8)
+    # that the producer fills its rings and has to poll for a free slot (its
+    # first idle poll then runs out); four K chunks, so the chunk-reduction
+    # kernel runs behind the decode kernel.
+    N, K = 28672, 4096
+    L = wl.layer("tod", N, K, T, seed=19 + T)
+    codes, sz, _ = oracle.pack(L.W, S=3)
+    k = np.random.default_rng(T).integers(1, 4, T).astype(np.int32)
+    perm = np.argsort(k, kind="stable").astype(np.int32)
+    off = np.concatenate([[0], np.cumsum(np.bincount(k, minlength=4)[1:])]).astype(np.int32)
+    args = [L.X.to(DEV), torch.from_numpy(k).to(DEV), torch.from_numpy(perm).to(DEV), torch.from_numpy(off).to(DEV),
+            torch.from_numpy(codes.view(np.int32)).to(DEV), torch.from_numpy(sz.view(np.int32)).to(DEV), N]
+    mobi.mobi_sync_check()
+    mobi.mobi_debug_set_wait_limit(1)
+    try:
+        mobi.mobi_gemm_path(*args, path=1)
+        with pytest.raises(mobi.MobiError) as ei:
+            mobi.mobi_sync_check()
+        assert ei.value.status == 6  # MOBI_ERR_TIMEOUT
+        assert "wait site" in mobi.mobi_last_error()
+    finally:
+        mobi.mobi_debug_set_wait_limit(0)
+    mobi.mobi_sync_check()  # error word cleared, context healthy
+    Y = mobi.mobi_gemm_path(*args, path=1)
+    mobi.mobi_sync_check()
+    check_gemm(Y.cpu().numpy(), oracle.gemm(L.X, k, codes, sz, N), f"decode after timeout, T={T}")

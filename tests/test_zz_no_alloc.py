@@ -5,10 +5,10 @@ engine plugin that must not allocate while it enqueues work, or a host whose
 device memory belongs to another runtime): its scratch is a fixed 8 MiB array
 of static device memory. This test calls it through the C ABI twice in a row
 (the array keeps the first call's contents) and checks both outputs against
-mobi_gemm, the entry point that takes a workspace, within the GEMM tolerance
-of the other tests; it also checks that a shape needing more scratch than the
-array holds is refused before anything runs. It passes alone in a fresh
-process and after the rest of the suite.
+mobi_gemm, the entry point that takes a workspace, and against the CPU oracle,
+within the GEMM tolerance of the other tests; it also checks that a shape
+needing more scratch than the array holds is refused before anything runs. It
+passes alone in a fresh process and after the rest of the suite.
 """
 import ctypes
 
@@ -37,7 +37,7 @@ def _p(t):
 
 
 @pytest.mark.parametrize("N,K,T", [(4096, 4096, 16), (11008, 4096, 5), (512, 11008, 1)])
-def test_noalloc_matches_workspace_entry_point(mobi, N, K, T):
+def test_noalloc_matches_workspace_entry_point(mobi, oracle, N, K, T):
     L = wl.layer("na", N, K, T, seed=N + K + T, outlier_frac_cols=0.005)
     W = torch.from_numpy(L.W).to(DEV)
     codes, sz = mobi.mobi_pack(W, S=3)
@@ -46,13 +46,18 @@ def test_noalloc_matches_workspace_entry_point(mobi, N, K, T):
     y_ws = mobi.mobi_gemm(X, k_t, perm, off, codes, sz, N)
     mobi.mobi_sync_check()
     ref = y_ws.cpu().numpy().astype(np.float64)
+    k = k_t.cpu().numpy()
+    y_oracle = oracle.gemm(L.X, k, codes.cpu().numpy().view(np.uint32), sz.cpu().numpy().view(np.uint32), N)
+    check_gemm(ref, y_oracle, f"workspace entry point, N={N} K={K} T={T}")
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     for call in range(2):
         Y = torch.full((T, N), float("nan"), dtype=torch.float32, device=DEV)
         st = mobi.lib().mobi_gemm_decode_noalloc(_p(X), T, K, _p(k_t), _p(codes), _p(sz), N, 128, 3, _p(Y), stream)
         assert st == 0, mobi.mobi_last_error()
         mobi.mobi_sync_check()
-        check_gemm(Y.cpu().numpy(), ref, f"no-alloc call {call + 1}, N={N} K={K} T={T}")
+        y = Y.cpu().numpy()
+        check_gemm(y, ref, f"no-alloc call {call + 1} vs mobi_gemm, N={N} K={K} T={T}")
+        check_gemm(y, y_oracle, f"no-alloc call {call + 1} vs the oracle, N={N} K={K} T={T}")
 
 
 def test_noalloc_refuses_oversized_scratch(mobi):

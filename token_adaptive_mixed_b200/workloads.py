@@ -54,13 +54,14 @@ def draw_weights(rng: np.random.Generator, N: int, K: int, sigma: float, n_outli
 
 
 def draw_activations(rng: np.random.Generator, T: int, K: int, scaled_frac: float = 0.0,
-                     scale: float = 1.0) -> torch.Tensor:
+                     scale: float = 1.0, return_rows: bool = False):
     X = rng.standard_normal((T, K), dtype=np.float32)
+    rows = np.zeros(0, np.int64)
     if scaled_frac > 0.0 and T > 0:
         m = int(round(scaled_frac * T))
         rows = rng.choice(T, m, replace=False)
         X[rows] *= np.float32(scale)
-    return to_bf16(X)
+    return (to_bf16(X), np.sort(rows)) if return_rows else to_bf16(X)
 
 
 def draw_router(rng: np.random.Generator, K: int, S: int) -> np.ndarray:
@@ -112,6 +113,7 @@ class Layer:
     X: torch.Tensor        # bf16 [T, K] (CPU)
     Wr: np.ndarray         # fp32 [K, S]
     bias: np.ndarray | None  # fp32 [S] or None
+    scaled_tokens: np.ndarray = dataclasses.field(default_factory=lambda: np.zeros(0, np.int64))  # rows of X scaled
 
     @property
     def N(self) -> int:
@@ -132,10 +134,10 @@ def layer(name: str, N: int, K: int, T: int, seed: int, sigma: float = 0.02, out
     rng = np.random.default_rng(seed)
     m = n_outlier_cols if n_outlier_cols is not None else int(round(outlier_frac_cols * K))
     W = draw_weights(rng, N, K, sigma, m)
-    X = draw_activations(rng, T, K, token_scaled_frac, token_scale)
+    X, scaled = draw_activations(rng, T, K, token_scaled_frac, token_scale, return_rows=True)
     Wr = draw_router(rng, K, S)
     bias = None if mix is None else bias_for_mix(Wr, mix, token_scaled_frac, token_scale)
-    return Layer(name, W, X, Wr, bias)
+    return Layer(name, W, X, Wr, bias, scaled)
 
 
 # ---- the five workloads -----------------------------------------------------
