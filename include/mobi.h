@@ -462,9 +462,11 @@ MOBI_API mobi_status mobi_sync_check(void* stream);
 /*
  * mobi_debug_set_wait_limit — set the iteration limit of the device-side
  * bounded waits of the current device (0 restores the default). A tiny limit
- * makes the decode and prefill kernels' waits run out, which exercises the
- * timeout path without faulting anything: the kernel records the error, drains
- * its own copies (and MMAs) in flight, frees its tensor memory and returns.
+ * makes the kernels' waits run out, which exercises the timeout path without
+ * faulting anything: the kernel records the error, drains its own copies (and
+ * MMAs) in flight, frees its tensor memory and returns. Below 64 the decode
+ * kernel's waits poll without suspending and each of its warps first waits on
+ * a barrier that nothing completes, so its timeout path always runs.
  * Test use only.
  */
 MOBI_API mobi_status mobi_debug_set_wait_limit(int64_t limit);

@@ -1,11 +1,12 @@
 """Failure detection without a GPU fault: the bounded device waits.
 
-A tiny wait limit makes a kernel's first mbarrier wait (or the decode
-producer's first poll of a full ring) run out, as a flag that is never set
-would. The kernel must record MOBI_ERR_TIMEOUT, drain its copies (and, in the
-prefill kernel, its MMAs and tensor memory) and return, leaving the context
-usable: the next call with the default limit must be correct again. Covered
-for the prefill kernel and the decode kernel (both fragment classes).
+A tiny wait limit makes a kernel's first mbarrier wait run out, as a flag
+that is never set would (below 64 the decode kernel's warps first wait on a
+barrier that nothing completes, so its timeout path runs on every call). The
+kernel must record MOBI_ERR_TIMEOUT, drain its copies (and, in the prefill
+kernel, its MMAs and tensor memory) and return, leaving the context usable:
+the next call with the default limit must be correct again. Covered for the
+prefill kernel and the decode kernel (both fragment classes).
 """
 import numpy as np
 import pytest
@@ -46,10 +47,8 @@ def test_timeout_is_reported_and_context_survives(oracle):
 @pytest.mark.parametrize("T", [4, 16])
 def test_decode_timeout_is_reported_and_context_survives(oracle, T):
     import token_adaptive_mixed_b200 as mobi
-    # Enough 32-row blocks per CTA (~24 stages per team against rings of 6 or 8)
-    # that the producer fills its rings and has to poll for a free slot (its
-    # first idle poll then runs out); four K chunks, so the chunk-reduction
-    # kernel runs behind the decode kernel.
+    # A large layer, so every CTA has work when the limit runs out; four K
+    # chunks, so the chunk-reduction kernel runs behind the decode kernel.
     N, K = 28672, 4096
     L = wl.layer("tod", N, K, T, seed=19 + T)
     codes, sz, _ = oracle.pack(L.W, S=3)

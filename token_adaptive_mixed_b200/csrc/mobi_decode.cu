@@ -19,18 +19,22 @@
 // (mma.sync m16n8k16) and in the per-group promotion
 // y += scale * 2^37 * acc - scale * z * xsum.
 //
-// Work split (persistent, one CTA per SM). K is cut into chunks of 8 groups
-// (1024 columns); a CTA owns one chunk and a contiguous range of 32-row
-// blocks (two 16-row MMA tiles each). Its consumer warps form teams of four:
-// the warps of a team work on the same block, each on 2 of the chunk's 8
-// groups, and hand their sums to the team's first warp through shared
-// memory. A warp keeps the activation fragments of its 2 groups in registers
-// for the whole kernel (built once from X), which keeps its unrolled stage
-// code small enough for the instruction cache. One producer warp feeds a
-// TMA ring per consumer warp with (block, slice) stages, so code bytes stream
-// in while earlier stages are multiplied. Chunks are combined by a second,
-// programmatically dependent kernel that adds the per-chunk partials in chunk
-// order (deterministic).
+// Work split (persistent, one CTA per SM, stream-K style). K is cut into
+// chunks of 8 groups (1024 columns). Once k_t is known (the slices each
+// problem reads), the 16-row tiles of all (problem, chunk) pairs are laid out
+// in one sequence, each costing its slices x (groups + a per-stage overhead),
+// and every CTA takes the tiles whose start falls in its equal share of the
+// total cost. A CTA's range is one or a few segments (runs of tiles in one
+// chunk). For each segment the CTA builds the chunk's B operand image in
+// shared memory (read with ldmatrix), then its twelve warps split the
+// segment's (tile, slice) stages evenly, one contiguous run each; every warp
+// streams its stages' codes and scale/zero words through its own three-stage
+// TMA ring (it issues its own copies and waits on its own barriers). A tile
+// is cut between two warps only before its last slice: the second warp leaves
+// that slice's sums in shared memory and the first adds them after the
+// segment's barrier, which rounds exactly as the uncut order does. Chunks
+// are combined by a second, programmatically dependent kernel that adds the
+// per-chunk partials in chunk order (deterministic).
 #include <cstdint>
 #include <cstring>
 #include <cstdio>
@@ -42,49 +46,35 @@
 
 namespace mobi {
 
-constexpr int kDecGW = 2;                    // groups per warp (64 bytes of a code row)
-constexpr int kDecQ = 4;                     // warps per team (one team per 32-row block)
-constexpr int kDecChunk = kDecQ * kDecGW;    // groups per CTA chunk
-constexpr int kDecRows = 32;                 // rows per stage: two 16-row MMA tiles
-// A stage belongs to a team: 32 rows x the chunk's 8 groups, as two
-// 128-byte-swizzled halves of 32 rows x 128 bytes, then [8 groups][32 rows]
-// scale/zero words.
-constexpr uint32_t kDecHalfBytes = kDecRows * 128;
-constexpr uint32_t kDecSlotCodes = 2 * kDecHalfBytes;
-constexpr uint32_t kDecSlotSz = kDecChunk * kDecRows * 4;
-constexpr uint32_t kDecSlot = kDecSlotCodes + kDecSlotSz;  // 9 KB, a multiple of 1 KB
+constexpr int kDecChunk = 8;       // groups per K chunk (1024 columns)
+constexpr int kDecRows = 16;       // rows per tile (one m16n8k16 A tile)
+constexpr int kDecWarps = 12;      // warps per CTA
+constexpr int kDecDepth = 3;       // stages per warp ring
+constexpr int kDecStageOv = 3;     // fixed cost of a stage, in groups (work split cost model)
+constexpr int kDecSegCost = 28 * (kDecChunk + kDecStageOv);  // set-up of a segment: about 28 full stages
+// A stage is one (tile, slice): the chunk's 8 groups of 16 code rows as two
+// 128-byte-swizzled halves of 16 rows x 128 bytes (4 KB, 1 KB aligned), and
+// the [8 groups][16 rows] scale/zero words (512 bytes, in a ring of their own).
+constexpr uint32_t kDecHalf = kDecRows * 128;
+constexpr uint32_t kDecCodes = 2 * kDecHalf;
+constexpr uint32_t kDecSz = kDecChunk * kDecRows * 4;
 
-template <int NB>
-struct DecCfg;
-template <>
-struct DecCfg<1> {  // T <= 8: 16 B-fragment registers per group
-  static constexpr int kTeams = 3;
-  static constexpr int kDepth = 6;
-};
-template <>
-struct DecCfg<2> {  // T <= 16: 32 per group
-  static constexpr int kTeams = 2;
-  static constexpr int kDepth = 8;
-};
-
+// Shared memory of the decode kernel for NB 8-token column blocks (T <= 8 NB).
 template <int NB>
 struct DecLayout {
-  static constexpr int kWarps = kDecQ * DecCfg<NB>::kTeams;  // consumer warps; one producer warp follows
-  static constexpr int kThreads = 32 * (kWarps + 1);
-  // Registers per thread for one CTA: the warps are spread over the SM's four
-  // 16K-register sub-partitions, so the fullest one decides.
-  static constexpr int kMaxRegs = (16384 / (32 * ((kWarps + 4) / 4))) / 8 * 8 > 248
-                                      ? 248
-                                      : (16384 / (32 * ((kWarps + 4) / 4))) / 8 * 8;
-  static constexpr int kDepth = DecCfg<NB>::kDepth;
-  static constexpr int kTeams = DecCfg<NB>::kTeams;
-  static constexpr uint32_t kSlots = 0;                                      // [team][slot] 9 KB, 1 KB aligned
-  static constexpr uint32_t kXchg = kSlots + kTeams * kDepth * kDecSlot;     // [team][2][kDecQ-1][32][8 NB] floats
-  static constexpr uint32_t kBar = kXchg + DecCfg<NB>::kTeams * 2 * (kDecQ - 1) * 32 * 8 * NB * 4;  // full, empty
-  static constexpr uint32_t kReady = kBar + 2 * kTeams * kDepth * 8;  // consumers' fragments built
-  static constexpr uint32_t kAbort = kReady + 8;
-  static constexpr uint32_t kBytes = kAbort + 8;
+  static constexpr int kThreads = 32 * kDecWarps;
+  static constexpr uint32_t kCodes = 0;                                          // [warp][depth] code stages
+  static constexpr uint32_t kSzs = kCodes + kDecWarps * kDecDepth * kDecCodes;   // [warp][depth] scale/zero stages
+  static constexpr uint32_t kBimg = kSzs + kDecWarps * kDecDepth * kDecSz;       // B image, 16 KB per NB
+  static constexpr uint32_t kBimgBytes = kDecChunk * NB * 8 * 256;
+  static constexpr uint32_t kXs = kBimg + kBimgBytes;                            // sum_k x [group][16 tokens]
+  static constexpr uint32_t kSc = kXs + kDecChunk * 16 * 4;                      // [warp][group][row] float2
+  static constexpr uint32_t kHead = kSc + kDecWarps * kDecChunk * kDecRows * 8;  // [warp][nb][A/B][lane] float2
+  static constexpr uint32_t kBar = kHead + kDecWarps * NB * 2 * 32 * 8;          // [warp][depth] full barriers
+  static constexpr uint32_t kNever = kBar + kDecWarps * kDecDepth * 8;           // a barrier nothing completes
+  static constexpr uint32_t kBytes = kNever + 8;
   static constexpr size_t kDynamic = kBytes + 1024;  // + manual 1 KB alignment
+  static_assert(kDynamic <= 232448, "fits the opt-in shared memory of one CTA");
 };
 
 constexpr float kTwo37 = 137438953472.0f;  // 2^37
@@ -98,133 +88,58 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Exact for a power-of-two multiplier as long as nothing overflows.
-__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
+// The same with a zero accumulator: d = A B.
+__device__ __forceinline__ void mma_bf16_16816_z(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                 uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};\n"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+// Four 8x8 b16 matrices: lane l gives the address of row l % 8 of matrix l / 8.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+// Issue one stage: the codes of 16-row tile `tile`, slice s, chunk `chunk`
+// (x = word column, y = s N + row) and its scale/zero words.
+__device__ __forceinline__ void dec_issue(const CUtensorMap* tm_codes, const CUtensorMap* tm_sz, uint8_t* codes,
+                                          uint8_t* sz, uint64_t* bar, int tile, int s, int N, int ngroups,
+                                          int chunk, uint64_t policy) {
+  mbar_arrive_expect_tx(bar, kDecCodes + kDecSz);
+  const int y = s * N + tile * kDecRows;
+  tma_load_2d_hint(codes, tm_codes, chunk * kDecChunk * 8, y, bar, policy);
+  tma_load_2d_hint(codes + kDecHalf, tm_codes, chunk * kDecChunk * 8 + 32, y, bar, policy);
+  tma_load_2d_hint(sz, tm_sz, tile * kDecRows, s * ngroups + chunk * kDecChunk, bar, policy);
 }
 
-// Issue one team stage into `slot`: the chunk's 256 bytes of 32 code rows as
-// two 128-byte halves (x = word column, y = s*N + row) and the matching
-// [8 groups][32 rows] scale/zero words. Weights are read once per call, so
-// they go in with L2 evict-first.
-__device__ __forceinline__ void dec_issue(const CUtensorMap* tm_codes, const CUtensorMap* tm_sz, uint8_t* slot,
-                                          uint64_t* bar, int block, int s, int N, int ngroups, int chunk,
-                                          uint64_t policy) {
-  mbar_arrive_expect_tx(bar, kDecSlot);
-  const int y = s * N + block * kDecRows;
-  tma_load_2d_hint(slot, tm_codes, chunk * kDecChunk * 8, y, bar, policy);
-  tma_load_2d_hint(slot + kDecHalfBytes, tm_codes, chunk * kDecChunk * 8 + 32, y, bar, policy);
-  tma_load_2d_hint(slot + kDecSlotCodes, tm_sz, block * kDecRows, s * ngroups + chunk * kDecChunk, bar, policy);
-}
-
-// Groups g0, g0 + 1 of one stage for TT tiles: four MMA chains in flight.
-template <int NB, int TT>
-__device__ __forceinline__ void dec_group_pair(int g0, const uint8_t* cs, const uint32_t* ss,
-                                               const uint32_t (&coff)[kDecGW], const uint32_t (&B)[kDecGW][8][2 * NB],
-                                               const float2 (&xs)[kDecGW][NB], const float2 (&m37)[NB],
-                                               const float2 (&m1)[NB], int gid, float2 (&yA)[2][NB],
-                                               float2 (&yB)[2][NB]) {
-  uint2 wa[2][TT], wb[2][TT];
-#pragma unroll
-  for (int gg = 0; gg < 2; ++gg)
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt) {
-      wa[gg][tt] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + tt * 16 * 128);
-      wb[gg][tt] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + tt * 16 * 128 + 8 * 128);
-    }
-  float d[2][TT][NB][4];
-#pragma unroll
-  for (int gg = 0; gg < 2; ++gg)
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) d[gg][tt][nb][0] = d[gg][tt][nb][1] = d[gg][tt][nb][2] = d[gg][tt][nb][3] = 0.0f;
-#pragma unroll
-  for (int h = 0; h < 2; ++h)
-#pragma unroll
-    for (int f = 0; f < 4; ++f) {
-      const uint32_t m = 0x00030003u << (2 * f);
-#pragma unroll
-      for (int gg = 0; gg < 2; ++gg)
-#pragma unroll
-        for (int tt = 0; tt < TT; ++tt) {
-          const uint32_t a0 = (wa[gg][tt].x >> (8 * h)) & m, a2 = (wa[gg][tt].y >> (8 * h)) & m;
-          const uint32_t a1 = (wb[gg][tt].x >> (8 * h)) & m, a3 = (wb[gg][tt].y >> (8 * h)) & m;
-#pragma unroll
-          for (int nb = 0; nb < NB; ++nb)
-            mma_bf16_16816(d[gg][tt][nb], a0, a1, a2, a3, B[g0 + gg][4 * h + f][2 * nb],
-                           B[g0 + gg][4 * h + f][2 * nb + 1]);
-        }
-    }
-#pragma unroll
-  for (int gg = 0; gg < 2; ++gg) {
-    const int g = g0 + gg;
-    float2 xm[NB];
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) xm[nb] = __fmul2_rn(xs[g][nb], m1[nb]);
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt) {
-      const uint32_t szA = ss[g * kDecRows + tt * 16 + gid], szB = ss[g * kDecRows + tt * 16 + gid + 8];
-      const float scA = __half2float(__ushort_as_half((unsigned short)(szA & 0xffffu)));
-      const float zA = __half2float(__ushort_as_half((unsigned short)(szA >> 16)));
-      const float scB = __half2float(__ushort_as_half((unsigned short)(szB & 0xffffu)));
-      const float zB = __half2float(__ushort_as_half((unsigned short)(szB >> 16)));
-      const float cA = -scA * zA, cB = -scB * zB;
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        // y += m * (scale 2^37 acc - scale z xsum), as packed fp32x2 FMAs.
-        yA[tt][nb] = __ffma2_rn(make_float2(cA, cA), xm[nb],
-                                __ffma2_rn(__fmul2_rn(make_float2(scA, scA), m37[nb]),
-                                           make_float2(d[gg][tt][nb][0], d[gg][tt][nb][1]), yA[tt][nb]));
-        yB[tt][nb] = __ffma2_rn(make_float2(cB, cB), xm[nb],
-                                __ffma2_rn(__fmul2_rn(make_float2(scB, scB), m37[nb]),
-                                           make_float2(d[gg][tt][nb][2], d[gg][tt][nb][3]), yB[tt][nb]));
-      }
-    }
-  }
-}
-
-// One stage: the warp's groups for TT tiles.
-template <int NB, int TT>
-__device__ __forceinline__ void dec_stage(int ngv, const uint8_t* cs, const uint32_t* ss,
-                                          const uint32_t (&coff)[kDecGW], const uint32_t (&B)[kDecGW][8][2 * NB],
-                                          const float2 (&xs)[kDecGW][NB], const float2 (&m37)[NB],
-                                          const float2 (&m1)[NB], int gid, float2 (&yA)[2][NB], float2 (&yB)[2][NB]) {
-  // A group beyond K has zero activations and zero-filled codes: it adds 0.
-  (void)ngv;
-  dec_group_pair<NB, TT>(0, cs, ss, coff, B, xs, m37, m1, gid, yA, yB);
-}
-
-// Bounded wait that also gives up once another warp has aborted.
+// Bounded wait; records the site and returns false when the limit runs out.
+// A test-sized limit (mobi_debug_set_wait_limit below 64) polls without the
+// hardware suspension of try_wait, so that a stage still in flight runs it out.
 __device__ __forceinline__ bool dec_wait(uint64_t* bar, uint32_t parity, uint64_t limit, DeviceStatus* st,
-                                         uint32_t where, volatile int32_t* abort_flag) {
-  for (uint64_t i = 0; i < limit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255) == 255 && *abort_flag) return false;
+                                         uint32_t where) {
+  if (limit < 64) {
+    for (uint64_t i = 0; i < limit; ++i)
+      if (mbar_test_wait(bar, parity)) return true;
+  } else {
+    for (uint64_t i = 0; i < limit; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
   }
   report_error(st, kErrTimeout, where);
-  *abort_flag = 1;
   return false;
 }
 
-// A group of independent problems in one launch: problem i owns the CTAs
-// [cta0, cta0 + cpc * nch) of the 1-D grid, cpc CTAs per K chunk. out = Y when
+// One problem of a launch: nblocks 16-row tiles, nch K chunks. out = Y when
 // the problem has one chunk, else its per-chunk partials [chunk][T][N].
 struct DecProblem {
   const __nv_bfloat16* X;
   const int32_t* k_t;
   float* out;
-  int T, N, K, ngroups, nblocks, cpc, cta0;
+  int T, N, K, ngroups, nblocks, nch;
 };
 // MG = table capacity: 1 for a single call (a small parameter block to copy
 // per launch), kMaxGroup for a group.
@@ -236,328 +151,468 @@ struct DecGroup {
   int G, S;
 };
 
-// All loop bookkeeping is incremental 32-bit arithmetic (sizes are validated
-// to N, K < 2^28). Warps 0 .. kWarps-1 consume (teams of four), warp kWarps
-// issues the copies.
+// The cost terms of the work split, per problem: a tile of a full chunk costs
+// u_full = k_max (8 + ov), a tile of the last chunk u_last = k_max (g_last +
+// ov) (the stages it reads, each its groups plus a fixed overhead), and every
+// chunk starts with the set-up cost Z of a segment (its B image), paid by the
+// CTA whose range crosses into it; problem m starts at pre[m] of the sequence,
+// pre[G] is the total.
+template <int MG>
+struct DecSplit {
+  long long pre[MG + 1];
+  long long chunk[MG];  // cost of one full chunk: Z + tiles x u_full
+  int u_full[MG], u_last[MG], km[MG];
+};
+
+// Warp 0, one lane per problem. Every CTA computes the same terms (the same
+// integer operations on the same k_t), so no CTA waits for another.
+template <int MG>
+__device__ __forceinline__ void dec_split(const DecGroup<MG>& grp, int lane, DecSplit<MG>* sp) {
+  const int G = MG > 1 ? grp.G : 1;
+  long long w = 0;
+  if (lane < G) {
+    const DecProblem& pr = grp.p[lane];
+    int km = 1;
+    for (int t = 0; t < pr.T && t < 16; ++t) km = max(km, (int)pr.k_t[t]);
+    km = km > grp.S ? grp.S : km;  // at least 1, at most S, as the stages clamp it
+    const int g_last = pr.ngroups - (pr.nch - 1) * kDecChunk;
+    const int uf = km * (kDecChunk + kDecStageOv), ul = km * (g_last + kDecStageOv);
+    const long long cf = kDecSegCost + (long long)pr.nblocks * uf;
+    w = cf * (pr.nch - 1) + kDecSegCost + (long long)pr.nblocks * ul;
+    sp->km[lane] = km;
+    sp->u_full[lane] = uf;
+    sp->u_last[lane] = ul;
+    sp->chunk[lane] = cf;
+  }
+  long long pre = w;  // inclusive prefix over the problems
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long v = __shfl_up_sync(0xffffffffu, pre, o);
+    if (lane >= o) pre += v;
+  }
+  if (lane < G) sp->pre[lane] = pre - w;
+  if (lane == G - 1) sp->pre[G] = pre;
+}
+
+// The B image of the chunk: for group g, k16 step j = 4h + f, column block nb
+// (tokens 8 nb .. 8 nb + 7) and half m, an 8 x 8 b16 matrix whose row n holds,
+// at column c = 2 t4 + e, x[8 nb + n][128 g + 32 t4 + 16 m + 4h + f + 8e]
+// scaled by 2^(96 - 2f) (exact in bf16 for |x| < 2^31). ldmatrix of (j, m = 0)
+// and (j, m = 1) gives exactly the B fragment that pairs with the A fragment
+// `(word >> 8h) & (0x00030003 << 2f)` of words 2 t4, 2 t4 + 1. Matrices are
+// 128 bytes each, [g][nb][j][m] in order, so one ldmatrix.x4 reads two steps.
+__device__ __forceinline__ uint32_t bimg_off(int g, int nb, int j, int m, int NB) {
+  return ((((uint32_t)g * NB + nb) * 8 + j) * 2 + m) * 128u;
+}
+
+// A warp boundary in a segment's stage sequence (stage x = tile x / km, slice
+// x % km), moved to the nearest place where a tile is either not cut or cut
+// just before its last slice. The warp that holds the tile's other slices then
+// finishes it with one add of the last slice's masked sums, the same rounding
+// as the uncut sequence: results do not depend on the split. Runs of at least
+// km stages stay non-empty (a boundary moves by at most one stage).
+__device__ __forceinline__ int dec_cut(int x, int km) {
+  const int o = x % km;
+  if (o == 0 || o == km - 1) return x;
+  return 2 * o <= km - 1 ? x - o : x - o + km - 1;
+}
+
+// Tile sums of one warp for 16 rows (gid, gid + 8) and the lane's tokens
+// 8 nb + 2 t4 + {0, 1}, written to o[t N + row] for tokens < T.
+template <int NB>
+__device__ __forceinline__ void dec_write_tile(float* o, int T, int N, int gid, int t4, const float2* yA,
+                                               const float2* yB) {
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    const int t0 = 8 * nb + 2 * t4;
+    if (t0 < T) {
+      o[(int64_t)t0 * N + gid] = yA[nb].x;
+      o[(int64_t)t0 * N + gid + 8] = yB[nb].x;
+    }
+    if (t0 + 1 < T) {
+      o[(int64_t)(t0 + 1) * N + gid] = yA[nb].y;
+      o[(int64_t)(t0 + 1) * N + gid + 8] = yB[nb].y;
+    }
+  }
+}
+
+// All loop bookkeeping is 32-bit arithmetic (sizes are validated to N, K <
+// 2^28); positions in the cost sequence are 64-bit.
 template <int NB, int MG>
-__global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) __maxnreg__(DecLayout<NB>::kMaxRegs) decode_kernel(
-    const __grid_constant__ DecGroup<MG> grp, DeviceStatus* st, uint64_t limit, int early) {
+__global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
+    const __grid_constant__ DecGroup<MG> grp, DeviceStatus* st, uint64_t limit) {
   using L = DecLayout<NB>;
-  constexpr int kTeams = DecCfg<NB>::kTeams;
-  constexpr int kW = L::kWarps;
-  constexpr int D = L::kDepth;
+  constexpr int D = kDecDepth;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ DecSplit<MG> sp;
+  __shared__ int s_abort;
+  __shared__ float* s_tail_o[kDecWarps];  // where each warp's unfinished tile goes, and its T, N
+  __shared__ int2 s_tail_tn[kDecWarps];
 
   // The reduction kernel behind this one may be scheduled now; it waits for
   // this grid's completion before reading anything.
   asm volatile("griddepcontrol.launch_dependents;");
+  // Launched as a programmatic dependent of the previous kernel: nothing in
+  // global memory is read before this wait (the split needs k_t).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int pi = 0;  // this CTA's problem
-#pragma unroll 1
-  for (int i = 1; i < (MG > 1 ? grp.G : 1); ++i)
-    if ((int)blockIdx.x >= grp.p[i].cta0) pi = i;
-  const DecProblem& prob = grp.p[pi];
-  const CUtensorMap* tm_codes = &grp.tm_codes[pi];
-  const CUtensorMap* tm_sz = &grp.tm_sz[pi];
-  const __nv_bfloat16* __restrict__ X = prob.X;
-  const int32_t* __restrict__ k_t = prob.k_t;
-  float* __restrict__ out = prob.out;
-  const int T = prob.T, N = prob.N, K = prob.K, ngroups = prob.ngroups, nblocks = prob.nblocks, S = grp.S;
-  const int local = (int)blockIdx.x - prob.cta0, cpc = prob.cpc;
-  const int ch = local / cpc, cx = local - ch * cpc;
-  // This CTA's 32-row blocks [b_begin, b_end); team t takes every kTeams-th
-  // of them, starting with block b_begin + t.
-  const int b_begin = (int)((int64_t)cx * nblocks / cpc);
-  const int b_end = (int)((int64_t)(cx + 1) * nblocks / cpc);
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::kBar);  // [team][slot]
-  uint64_t* empty = full + kTeams * D;
-  uint64_t* ready = reinterpret_cast<uint64_t*>(sm + L::kReady);
-  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(sm + L::kAbort);
-
-  // One barrier per thread, then one fence per warp. A stage is freed by the
-  // four warps of its team.
-  for (int i = threadIdx.x; i < 2 * kTeams * D + 1; i += blockDim.x) {
-    if (i < kTeams * D) mbar_init(&full[i], 1);
-    else if (i < 2 * kTeams * D) mbar_init(&empty[i - kTeams * D], kDecQ);
-    else mbar_init(ready, kW);
-  }
-  if (threadIdx.x == 0) *abort_flag = 0;
-  if (lane == 0) fence_barrier_init();
-  __syncthreads();
-  // Launched as a programmatic dependent of the previous kernel in the
-  // stream. By default nothing in global memory is read before this wait.
-  // With `early` set the caller guarantees that the previous kernel writes
-  // none of X, codes and sz (it is this library's routing kernel), so the
-  // activations and the first weight stages are fetched before the wait and
-  // only k_t is read after it.
-  if (!early) asm volatile("griddepcontrol.wait;" ::: "memory");
-
-  if (warp == kW) {
-    // ---------------- producer: lane w feeds team w's ring ----------------
-    // All lanes poll their ring's empty barrier in one non-blocking test and
-    // issue their copies together, so one poll serves every team.
-    named_bar_sync(15, 32 * (kW + 1));  // the consumers' activation loads go out first
-    if (lane == 0) {
-      prefetch_tmap(tm_codes);
-      prefetch_tmap(tm_sz);
-    }
-    const uint64_t policy = l2_evict_first_policy();
-    const int w = lane, team = lane;
-    const int myb = (w < kTeams && b_end - b_begin > team) ? (b_end - b_begin - team + kTeams - 1) / kTeams : 0;
-    int r = 0, bo = 0, s = 0;  // next stage of team w: its index, block offset and slice
-    // Slice 0 of the team's first block does not depend on k_t.
-    if (early && myb > 0) {
-      dec_issue(tm_codes, tm_sz, sm + L::kSlots + (uint32_t)(w * D) * kDecSlot, &full[w * D], b_begin + team, 0, N,
-                ngroups, ch, policy);
-      r = 1;
-    }
-    if (early) asm volatile("griddepcontrol.wait;" ::: "memory");
-    int kmax = __reduce_max_sync(0xffffffffu, lane < T ? (int)__ldg(k_t + lane) : 1);
-    kmax = kmax < 1 ? 1 : (kmax > S ? S : kmax);
-    const int nit = myb * kmax;  // stages of team w: its blocks x slices
-    if (r == 1 && ++s == kmax) { s = 0; ++bo; }
-    bool gate = false;         // every consumer has built its activations
-    bool ok = true;
-    uint64_t idle = 0;         // polls in a row without a copy issued
-    while (true) {
-      // Two stages per consumer first; the rest once every consumer has its
-      // activations, so that those small loads do not queue behind the rings.
-      if (!gate) gate = __shfl_sync(0xffffffffu, lane == 0 ? (int)mbar_test_wait(ready, 0) : 0, 0) != 0;
-      bool issued = false;
-      if (ok && r < nit && (r < 2 || gate)) {
-        const int slot = r % D;
-        if (r < D || mbar_test_wait(&empty[w * D + slot], (uint32_t)(((r / D) & 1) ^ 1))) {
-          dec_issue(tm_codes, tm_sz, sm + L::kSlots + (uint32_t)(w * D + slot) * kDecSlot, &full[w * D + slot],
-                    b_begin + team + bo * kTeams, s, N, ngroups, ch, policy);
-          ++r;
-          if (++s == kmax) { s = 0; ++bo; }
-          issued = true;
-        }
-      }
-      if (!__any_sync(0xffffffffu, ok && r < nit)) break;
-      if (__any_sync(0xffffffffu, issued)) {
-        idle = 0;
-      } else if (++idle >= limit || ((idle & 255) == 0 && *abort_flag)) {
-        if (idle >= limit && lane == 0) {
-          report_error(st, kErrTimeout, 0x2e0);
-          *abort_flag = 1;
-        }
-        ok = false;
-      }
-    }
-    // Normally the consumers have waited for every copy. If any warp gave up,
-    // every copy issued must still land before the CTA can exit (the last
-    // copy into a slot completes after the earlier ones).
-    __syncwarp();
-    __syncthreads();  // all consumers are done
-    if (*abort_flag) {
-      for (int sl = 0; sl < D && sl < r; ++sl) {
-        const int last = sl + (r - 1 - sl) / D * D;
-        mbar_wait(&full[w * D + sl], (uint32_t)((last / D) & 1), kDefaultWaitLimit, st, 0x2f0);
-      }
-    }
-    return;
-  }
-
-  // ---------------- consumers ----------------
   const int gid = lane >> 2, t4 = lane & 3;
-  const int team = warp / kDecQ, q = warp % kDecQ;
-  const int gbase = ch * kDecChunk + q * kDecGW;  // first group of this warp
-  const int ngv = ngroups - gbase < 0 ? 0 : (ngroups - gbase > kDecGW ? kDecGW : ngroups - gbase);
-  const int my_blocks = b_end - b_begin > team ? (b_end - b_begin - team + kTeams - 1) / kTeams : 0;
-  const uint8_t* slots_t = sm + L::kSlots + (uint32_t)team * D * kDecSlot;  // the team's ring
-  float* xchg = reinterpret_cast<float*>(sm + L::kXchg) + team * 2 * (kDecQ - 1) * 32 * 8 * NB;
-  uint64_t* full_w = full + team * D;
-  uint64_t* empty_w = empty + team * D;
+  const int G = MG > 1 ? grp.G : 1;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::kBar) + warp * D;
+  uint64_t* never = reinterpret_cast<uint64_t*>(sm + L::kNever);
+  if (warp == 0) dec_split(grp, lane, &sp);
+  if (threadIdx.x == 32) s_abort = 0;
+  if (lane == 0) {
+    for (int d = 0; d < D; ++d) mbar_init(&full[d], 1);
+    if (warp == 0) mbar_init(never, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
 
-  // This lane's activations (token gid + 8 nb, columns 32 t4 .. +31 of each
-  // group) and k_t[lane].
-  uint4 raw[kDecGW][NB][4];
-#pragma unroll
-  for (int g = 0; g < kDecGW; ++g)
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      const int tok = gid + 8 * nb;
-      if (g < ngv && tok < T) {
-        const uint4* src = reinterpret_cast<const uint4*>(X + (int64_t)tok * K + (gbase + g) * 128 + 32 * t4);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) raw[g][nb][v] = __ldg(src + v);
-      } else {
-#pragma unroll
-        for (int v = 0; v < 4; ++v) raw[g][nb][v] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-  asm volatile("bar.arrive 15, %0;" ::"r"(32 * (kW + 1)) : "memory");
+  // This CTA's share of the cost sequence: the tiles starting in [X0, X1).
+  const long long Wt = sp.pre[G], C = gridDim.x, bi = blockIdx.x;
+  const long long q = Wt / C, r = Wt % C;
+  const long long X0 = q * bi + (r * bi + C - 1) / C, X1 = q * (bi + 1) + (r * (bi + 1) + C - 1) / C;
+  if (X0 >= X1) return;  // the whole CTA, before any copy is issued
 
-  // Activation fragments of the warp's groups, in registers for the whole
-  // kernel. B[g][j][2 nb + ih] is the B fragment of k16 step j = 4h + f for
-  // token gid + 8 nb: register ih holds columns 32 t4 + 16 ih + 4h + f + 8e
-  // (e = 0 low half, 1 high half) of group g, scaled by 2^(96 - 2f). The
-  // matching A fragment of the codes is (word 2 t4 + ih >> 8h) & (3 << 2f).
-  uint32_t B[kDecGW][8][2 * NB];
-  float2 xs[kDecGW][NB];  // sum_k x of tokens (2 t4, 2 t4 + 1) + 8 nb, group g
+  // A test-sized wait limit (mobi_debug_set_wait_limit below 64) first waits
+  // on a barrier that nothing completes, so the timeout path runs
+  // deterministically; every warp runs it out, so every warp stops here.
+  if (limit < 64 && !__all_sync(0xffffffffu, dec_wait(never, 0, limit, st, 0x2ff))) return;
+
+  // The first tile starting at or after X0: problem p, chunk c, tile b (b may
+  // be one past the chunk's last tile; the loop moves on to the next chunk).
+  int p = 0;
+#pragma unroll 1
+  for (int j = 1; j < G; ++j)
+    if (sp.pre[j] <= X0) p = j;
+  int c, b;
   {
-    bool bad = false;
-#pragma unroll
-    for (int g = 0; g < kDecGW; ++g) {
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        const uint32_t u[16] = {raw[g][nb][0].x, raw[g][nb][0].y, raw[g][nb][0].z, raw[g][nb][0].w,
-                                raw[g][nb][1].x, raw[g][nb][1].y, raw[g][nb][1].z, raw[g][nb][1].w,
-                                raw[g][nb][2].x, raw[g][nb][2].y, raw[g][nb][2].z, raw[g][nb][2].w,
-                                raw[g][nb][3].x, raw[g][nb][3].y, raw[g][nb][3].z, raw[g][nb][3].w};
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          bad |= ((u[i] & 0x7F80u) >= (158u << 7)) || ((u[i] & 0x7F800000u) >= (158u << 23));
-#pragma unroll
-        for (int ih = 0; ih < 2; ++ih)
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int f = 0; f < 4; ++f) {
-              const int w0 = 8 * ih + 2 * h + (f >> 1);
-              const uint32_t pair = __byte_perm(u[w0], u[w0 + 4], (f & 1) ? 0x7632u : 0x5410u);
-              const uint32_t e = (uint32_t)(223 - 2 * f) << 7;  // bf16 bits of 2^(96 - 2f)
-              B[g][4 * h + f][2 * nb + ih] = bf16x2_mul(pair, e | (e << 16));
-            }
-      }
-    }
-    // Group sums on the tensor core: codes all 1 -> every D row is sum_k x * 2^-37.
-    float d[kDecGW][NB][4];
-#pragma unroll
-    for (int g = 0; g < kDecGW; ++g)
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) d[g][nb][0] = d[g][nb][1] = d[g][nb][2] = d[g][nb][3] = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t one = 0x00010001u << (2 * (j & 3));
-#pragma unroll
-      for (int g = 0; g < kDecGW; ++g)
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb)
-          mma_bf16_16816(d[g][nb], one, one, one, one, B[g][j][2 * nb], B[g][j][2 * nb + 1]);
-    }
-#pragma unroll
-    for (int g = 0; g < kDecGW; ++g)
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) xs[g][nb] = make_float2(d[g][nb][0] * kTwo37, d[g][nb][1] * kTwo37);
-    if (__any_sync(0xffffffffu, bad) && lane == 0) report_error(st, kErrInputRange, 0x100);
-  }
-  if (lane == 0) mbar_arrive(ready);
-  if (early) asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int my_kt = lane < T ? k_t[lane] : 0;
-  int kmax = __reduce_max_sync(0xffffffffu, my_kt);
-  kmax = kmax < 1 ? 1 : (kmax > S ? S : kmax);
-
-  // k_t of the two tokens whose D columns this lane holds.
-  int ktl[NB][2];
-#pragma unroll
-  for (int nb = 0; nb < NB; ++nb) {
-    ktl[nb][0] = __shfl_sync(0xffffffffu, my_kt, 2 * t4 + 8 * nb);
-    ktl[nb][1] = __shfl_sync(0xffffffffu, my_kt, 2 * t4 + 1 + 8 * nb);
+    const long long x = X0 - sp.pre[p];
+    const int nch = grp.p[p].nch;
+    const long long cc = x / sp.chunk[p];
+    c = (int)(cc < nch - 1 ? cc : nch - 1);
+    const long long rem = x - (long long)c * sp.chunk[p] - kDecSegCost;
+    const int u = c < nch - 1 ? sp.u_full[p] : sp.u_last[p];
+    b = rem <= 0 ? 0 : (int)((rem + u - 1) / u);
   }
 
-  // Code words 2 t4, 2 t4 + 1 of the warp's group g (chunk group 2q + g) of
-  // row gid: in half q / 2 of the stage, 128-byte-swizzled (16-byte chunk c of
-  // row r sits at c ^ (r & 7)); rows gid + 8, +16, +24 share the swizzle and
-  // sit 1, 2, 3 KB further on.
-  uint32_t coff[kDecGW];
-#pragma unroll
-  for (int g = 0; g < kDecGW; ++g)
-    coff[g] = (uint32_t)(q >> 1) * kDecHalfBytes + (uint32_t)gid * 128u +
-              (uint32_t)(((((q & 1) * kDecGW + g) * 2 + (t4 >> 1)) ^ gid) * 16) + (t4 & 1) * 8u;
+  const uint64_t policy = l2_evict_first_policy();
+  uint8_t* const codes_ring = sm + L::kCodes + (uint32_t)warp * D * kDecCodes;
+  uint8_t* const sz_ring = sm + L::kSzs + (uint32_t)warp * D * kDecSz;
+  float2* const scw = reinterpret_cast<float2*>(sm + L::kSc) + warp * kDecChunk * kDecRows;
+  float2* const head_mine = reinterpret_cast<float2*>(sm + L::kHead) + warp * NB * 2 * 32;
+  const float2* const head_next = head_mine + NB * 2 * 32;
+  const float* const xs_sm = reinterpret_cast<const float*>(sm + L::kXs);
+  const uint32_t bimg = smem_addr(sm + L::kBimg) + (uint32_t)lane * 16;
 
-  // y[tt][nb]: tile tt of the block, rows gid (A) and gid + 8 (B) of it,
-  // tokens (2 t4, 2 t4 + 1) + 8 nb.
-  float2 yA[2][NB], yB[2][NB];
+  // Code words 2 t4, 2 t4 + 1 of group g for row r of the tile: half g / 4,
+  // 16-byte chunk 2 (g % 4) + t4 / 2 stored at chunk ^ (r % 8), rows 128 bytes.
+  uint32_t coff[kDecChunk];
 #pragma unroll
-  for (int tt = 0; tt < 2; ++tt)
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) yA[tt][nb] = yB[tt][nb] = make_float2(0.0f, 0.0f);
+  for (int g = 0; g < kDecChunk; ++g)
+    coff[g] = (uint32_t)(g >> 2) * kDecHalf + (uint32_t)gid * 128u +
+              (uint32_t)((((g & 3) * 2 + (t4 >> 1)) ^ gid) * 16) + (t4 & 1) * 8u;
 
   bool ok = true;
-  int slot = 0;
-  uint32_t parity = 0;
-  int s = 0, blk = b_begin + team, blk_i = 0;
-  const int total_iters = my_blocks * kmax;  // both warps of a team walk the same sequence
-  for (int it = 0; it < total_iters; ++it) {
-    const bool two = blk * kDecRows + 16 < N;  // the block's second tile exists (N % 16 == 0)
-    if (ok) {  // every warp of the team frees each stage, also one past the last group
-      const bool got = __all_sync(0xffffffffu, dec_wait(&full_w[slot], parity, limit, st, 0x200 + s, abort_flag));
-      if (!got) {
-        ok = false;
-      } else {
-        const uint8_t* cs = slots_t + (uint32_t)slot * kDecSlot;
-        const uint32_t* ss = reinterpret_cast<const uint32_t*>(cs + kDecSlotCodes) + q * kDecGW * kDecRows;
-        float2 m37[NB], m1[NB];
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-          m37[nb] = make_float2(ktl[nb][0] > s ? kTwo37 : 0.0f, ktl[nb][1] > s ? kTwo37 : 0.0f);
-          m1[nb] = make_float2(ktl[nb][0] > s ? 1.0f : 0.0f, ktl[nb][1] > s ? 1.0f : 0.0f);
-        }
-        // Past N the second tile holds zero-filled or neighbouring rows; its
-        // sums are computed like the first tile's and never written.
-        dec_stage<NB, 2>(ngv, cs, ss, coff, B, xs, m37, m1, gid, yA, yB);
-        // Slot free again for the producer.
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_w[slot]);
+  uint32_t issued = 0, done = 0;  // stages this warp has issued / consumed (ring slot = count % D)
+  // A tile this warp left unfinished at the end of the previous segment (its
+  // first slices, parked in the warp's scale/zero scratch); the next warp
+  // holds the rest in its head slot.
+  bool tail = false;
+
+#pragma unroll 1
+  for (;;) {
+    // ---- the next segment: tiles b .. b_end - 1 of chunk c of problem p ----
+    if (p < G && b >= grp.p[p].nblocks) {
+      b = 0;
+      if (++c == grp.p[p].nch) {
+        c = 0;
+        ++p;
       }
     }
-    if (++slot == D) { slot = 0; parity ^= 1u; }
-    if (s == kmax - 1) {
-      // Team hand-off: warps 1..3 of the team pass their groups' sums to
-      // warp 0, which adds them in warp order.
-      float* xb = xchg + (blk_i & 1) * (kDecQ - 1) * 32 * 8 * NB;
-      if (q > 0) {
-        float* mine = xb + ((q - 1) * 32 + lane) * 8 * NB;
+    bool more = p < G;
+    int km = 1, b_end = 0, a = 0, a1 = 0;
+    // The chunk of X (for the B image) and k_t are loaded before this
+    // segment's first stages are requested, so they return ahead of them.
+    constexpr int kMaxVec = (8 * NB * kDecChunk * 16 + L::kThreads - 1) / L::kThreads;
+    uint4 raw[kMaxVec];
+    int my_kt = 0, g_valid = 0, nvec = 0;
+    if (more) {
+      const int nch = grp.p[p].nch, tiles = grp.p[p].nblocks;
+      const int u = c < nch - 1 ? sp.u_full[p] : sp.u_last[p];
+      const long long base = sp.pre[p] + (long long)c * sp.chunk[p] + kDecSegCost;  // start of tile 0
+      more = base + (long long)b * u < X1;
+      if (more) {
+        km = sp.km[p];
+        const long long be = (X1 - base + u - 1) / u;  // tiles starting before X1
+        b_end = be < tiles ? (int)be : tiles;
+        const int nt = b_end - b, ns = nt * km;
+        if (ns >= kDecWarps * km) {  // even runs of stages, cut only before a tile's last slice
+          a = dec_cut(warp * ns / kDecWarps, km);
+          a1 = dec_cut((warp + 1) * ns / kDecWarps, km);
+        } else {  // whole tiles, one per warp
+          a = (warp < nt ? warp : nt) * km;
+          a1 = (warp + 1 < nt ? warp + 1 : nt) * km;
+        }
+        const DecProblem& pr = grp.p[p];
+        g_valid = pr.ngroups - c * kDecChunk < kDecChunk ? pr.ngroups - c * kDecChunk : kDecChunk;
+        nvec = pr.T * g_valid * 16;  // 8-element vectors of X in this chunk
+        my_kt = lane < pr.T ? pr.k_t[lane] : 0;
 #pragma unroll
-        for (int tt = 0; tt < 2; ++tt)
-#pragma unroll
-          for (int nb = 0; nb < NB; ++nb)
-            *reinterpret_cast<float4*>(mine + 8 * nb + 4 * tt) =
-                make_float4(yA[tt][nb].x, yA[tt][nb].y, yB[tt][nb].x, yB[tt][nb].y);
+        for (int i = 0; i < kMaxVec; ++i) {
+          const int v = threadIdx.x + i * L::kThreads;
+          if (v < nvec) {
+            const int t = v / (g_valid * 16), rr = v - t * (g_valid * 16);
+            raw[i] = __ldg(reinterpret_cast<const uint4*>(pr.X + (int64_t)t * pr.K +
+                                                          (int64_t)(c * kDecChunk + (rr >> 4)) * 128 + (rr & 15) * 8));
+          }
+        }
+        // The first D - 1 stages go out before the segment's set-up.
+        const int nramp = a1 - a < D - 1 ? a1 - a : D - 1;
+        if (lane == 0 && ok) {
+          for (int k = 0; k < nramp; ++k) {
+            const uint32_t slot = (issued + k) % D;
+            const int jj = a + k;
+            dec_issue(&grp.tm_codes[p], &grp.tm_sz[p], codes_ring + slot * kDecCodes, sz_ring + slot * kDecSz,
+                      &full[slot], b + jj / km, jj % km, pr.N, pr.ngroups, c, policy);
+          }
+        }
+        if (ok) issued += nramp;
       }
-      named_bar_sync(1 + team, 32 * kDecQ);
-      if (q == 0) {
-        float* o = out + (int64_t)ch * T * N + blk * kDecRows;
+    }
+    __syncthreads();  // every warp is done with the previous segment (image, head slots)
+    ok = *reinterpret_cast<volatile int*>(&s_abort) == 0;
+    if (tail) {  // finish the tile left by this warp: its slices so far plus the next warp's last slice
+      if (ok) {
+        float2 tA[NB], tB[NB];
 #pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          if (tt == 1 && !two) break;
+        for (int nb = 0; nb < NB; ++nb) {
+          const float2 hA = head_next[(nb * 2 + 0) * 32 + lane], hB = head_next[(nb * 2 + 1) * 32 + lane];
+          const float2 mA = scw[(nb * 2 + 0) * 32 + lane], mB = scw[(nb * 2 + 1) * 32 + lane];
+          tA[nb] = make_float2(mA.x + hA.x, mA.y + hA.y);
+          tB[nb] = make_float2(mB.x + hB.x, mB.y + hB.y);
+        }
+        dec_write_tile<NB>(s_tail_o[warp], s_tail_tn[warp].x, s_tail_tn[warp].y, gid, t4, tA, tB);
+      }
+      tail = false;
+    }
+    if (!more || !ok) break;
+
+    const DecProblem& prob = grp.p[p];
+    const int T = prob.T, N = prob.N, ngroups = prob.ngroups;
+
+    // ---- the chunk's B image (zero beyond T tokens and beyond the last group) ----
+    {
+      uint4* img = reinterpret_cast<uint4*>(sm + L::kBimg);
+      for (uint32_t i = threadIdx.x; i < L::kBimgBytes / 16; i += blockDim.x) img[i] = make_uint4(0u, 0u, 0u, 0u);
+      __syncthreads();
+      uint16_t* img16 = reinterpret_cast<uint16_t*>(sm + L::kBimg);
+      bool bad = false;
 #pragma unroll
-          for (int nb = 0; nb < NB; ++nb) {
-            float v[4] = {yA[tt][nb].x, yA[tt][nb].y, yB[tt][nb].x, yB[tt][nb].y};
+      for (int i = 0; i < kMaxVec; ++i) {
+        const int v = threadIdx.x + i * L::kThreads;
+        if (v < nvec) {
+          const int t = v / (g_valid * 16), rr = v - t * (g_valid * 16);
+          const int g = rr >> 4, k0 = (rr & 15) * 8;  // k0 = 32 t4 + 16 m + 8 e
+          const uint32_t uu[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+          const int tt4 = k0 >> 5, m = (k0 >> 4) & 1, e = (k0 >> 3) & 1;
+          const int nb = t >> 3, n = t & 7, cc = 2 * tt4 + e;
 #pragma unroll
-            for (int w = 0; w < kDecQ - 1; ++w) {
-              const float4 p = *reinterpret_cast<const float4*>(xb + (w * 32 + lane) * 8 * NB + 8 * nb + 4 * tt);
-              v[0] += p.x; v[1] += p.y; v[2] += p.z; v[3] += p.w;
-            }
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int tk = 2 * t4 + 8 * nb + e;
-              if (tk < T) {
-                o[(int64_t)tk * N + tt * 16 + gid] = v[e];
-                o[(int64_t)tk * N + tt * 16 + gid + 8] = v[2 + e];
-              }
-            }
+          for (int qq = 0; qq < 8; ++qq) {  // element k0 + qq: h = qq >> 2, f = qq & 3
+            const uint32_t bits = (uu[qq >> 1] >> (16 * (qq & 1))) & 0xffffu;
+            bad |= (bits & 0x7F80u) >= (158u << 7);
+            const int h = qq >> 2, f = qq & 3, j = 4 * h + f;
+            const float v32 = __uint_as_float(bits << 16) * __uint_as_float((uint32_t)(127 + 96 - 2 * f) << 23);
+            img16[(bimg_off(g, nb, j, m, NB) + (uint32_t)n * 16 + (uint32_t)cc * 2) >> 1] =
+                (uint16_t)(__float_as_uint(v32) >> 16);  // exact: a power-of-two scaling of a bf16
           }
         }
       }
-#pragma unroll
-      for (int tt = 0; tt < 2; ++tt)
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) yA[tt][nb] = yB[tt][nb] = make_float2(0.0f, 0.0f);
-      s = 0;
-      blk += kTeams;
-      ++blk_i;
-    } else {
-      ++s;
+      if (__any_sync(0xffffffffu, bad) && lane == 0) report_error(st, kErrInputRange, 0x100);
+      __syncthreads();
     }
+    // ---- group sums on the tensor core: codes all 1 -> every D row is sum_k x * 2^-37 ----
+    if (warp < kDecChunk) {
+      const int g = warp;
+      const uint32_t base = smem_addr(sm + L::kBimg);
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int jp = 0; jp < 4; ++jp) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(base + bimg_off(g, nb, 2 * jp, 0, NB) + (uint32_t)lane * 16, b0, b1, b2, b3);
+          const uint32_t one0 = 0x00010001u << (2 * ((2 * jp) & 3)), one1 = 0x00010001u << (2 * ((2 * jp + 1) & 3));
+          mma_bf16_16816(d, one0, one0, one0, one0, b0, b1);
+          mma_bf16_16816(d, one1, one1, one1, one1, b2, b3);
+        }
+        if (gid == 0) {
+          float* xs = reinterpret_cast<float*>(sm + L::kXs) + g * 16 + 8 * nb + 2 * t4;
+          xs[0] = d[0] * kTwo37;
+          xs[1] = d[1] * kTwo37;
+        }
+      }
+    }
+    __syncthreads();
+
+    float2 yA[NB], yB[NB];  // rows gid (A) and gid + 8 (B), tokens 8 nb + 2 t4 + {0, 1}
+    // k_t of the tokens whose columns this lane holds: 8 nb + 2 t4 + e.
+    int ktl[NB][2];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      ktl[nb][0] = __shfl_sync(0xffffffffu, my_kt, 8 * nb + 2 * t4);
+      ktl[nb][1] = __shfl_sync(0xffffffffu, my_kt, 8 * nb + 2 * t4 + 1);
+    }
+    // sum_k x of the lane's two tokens, per group and column block.
+    float2 xs[kDecChunk][NB];
+#pragma unroll
+    for (int g = 0; g < kDecChunk; ++g)
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+        xs[g][nb] = *reinterpret_cast<const float2*>(xs_sm + g * 16 + 8 * nb + 2 * t4);
+
+    float* const out = prob.out + (int64_t)c * T * N;
+    const CUtensorMap* tm_codes = &grp.tm_codes[p];
+    const CUtensorMap* tm_sz = &grp.tm_sz[p];
+    int s = a % km, tile = b + a / km;  // consumer cursor
+    bool head = s != 0;                 // the first tile's other slices are the previous warp's
+    int pj = a + (a1 - a < D - 1 ? a1 - a : D - 1);
+    int ps = pj % km, ptile = b + pj / km;  // producer cursor
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) yA[nb] = yB[nb] = make_float2(0.0f, 0.0f);
+
+#pragma unroll 1
+    for (int j = a; j < a1; ++j) {
+      const uint32_t slot = done % D;
+      // Refill the slot read in the previous iteration (every lane is done with it).
+      __syncwarp();
+      if (pj < a1) {
+        const uint32_t ns = issued % D;
+        if (lane == 0)
+          dec_issue(tm_codes, tm_sz, codes_ring + ns * kDecCodes, sz_ring + ns * kDecSz, &full[ns], ptile, ps, N,
+                    ngroups, c, policy);
+        ++issued;
+        ++pj;
+        if (++ps == km) {
+          ps = 0;
+          ++ptile;
+        }
+      }
+      if (!(ok = __all_sync(0xffffffffu, dec_wait(&full[slot], (done / D) & 1u, limit, st, 0x200 + s)))) {
+        if (lane == 0) *reinterpret_cast<volatile int*>(&s_abort) = 1;
+        break;
+      }
+      ++done;
+      const uint8_t* cs = codes_ring + slot * kDecCodes;
+      // Scale/zero words of the stage as fp32 pairs (scale 2^37, -scale zero),
+      // one conversion per word for the whole warp.
+      {
+        const uint32_t* szw = reinterpret_cast<const uint32_t*>(sz_ring + slot * kDecSz);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t w = szw[lane + 32 * i];
+          const float sc = __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
+          const float zf = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+          scw[lane + 32 * i] = make_float2(sc * kTwo37, -sc * zf);
+        }
+        __syncwarp();
+      }
+      float2 ysA[NB], ysB[NB];
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) ysA[nb] = ysB[nb] = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int g0 = 0; g0 < kDecChunk; g0 += 2) {
+        if (g0 >= g_valid) break;  // the last chunk's missing groups (their B image is zero)
+        uint2 wa[2], wb[2];
+        uint32_t bf[2][NB][8][2];
+#pragma unroll
+        for (int gg = 0; gg < 2; ++gg) {
+          wa[gg] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg]);
+          wb[gg] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + 8 * 128);
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+            for (int jp = 0; jp < 4; ++jp)
+              ldsm_x4(bimg + bimg_off(g0 + gg, nb, 2 * jp, 0, NB), bf[gg][nb][2 * jp][0], bf[gg][nb][2 * jp][1],
+                      bf[gg][nb][2 * jp + 1][0], bf[gg][nb][2 * jp + 1][1]);
+        }
+        float d[2][NB][4];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int h = jj >> 2, f = jj & 3;
+          const uint32_t mk = 0x00030003u << (2 * f);
+#pragma unroll
+          for (int gg = 0; gg < 2; ++gg) {
+            const uint32_t a0 = (wa[gg].x >> (8 * h)) & mk, a2 = (wa[gg].y >> (8 * h)) & mk;
+            const uint32_t a1r = (wb[gg].x >> (8 * h)) & mk, a3 = (wb[gg].y >> (8 * h)) & mk;
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+              if (jj == 0) mma_bf16_16816_z(d[gg][nb], a0, a1r, a2, a3, bf[gg][nb][jj][0], bf[gg][nb][jj][1]);
+              else mma_bf16_16816(d[gg][nb], a0, a1r, a2, a3, bf[gg][nb][jj][0], bf[gg][nb][jj][1]);
+            }
+          }
+        }
+        // Per-group promotion: ys += scale 2^37 acc - scale z sum_k x.
+#pragma unroll
+        for (int gg = 0; gg < 2; ++gg) {
+          const int g = g0 + gg;
+          const float2 pA = scw[g * kDecRows + gid], pB = scw[g * kDecRows + gid + 8];
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            ysA[nb] = __ffma2_rn(make_float2(pA.x, pA.x), make_float2(d[gg][nb][0], d[gg][nb][1]),
+                                 __ffma2_rn(make_float2(pA.y, pA.y), xs[g][nb], ysA[nb]));
+            ysB[nb] = __ffma2_rn(make_float2(pB.x, pB.x), make_float2(d[gg][nb][2], d[gg][nb][3]),
+                                 __ffma2_rn(make_float2(pB.y, pB.y), xs[g][nb], ysB[nb]));
+          }
+        }
+      }
+      // The slice counts only for the tokens that take it (k_t > s).
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        const float2 m = make_float2(ktl[nb][0] > s ? 1.0f : 0.0f, ktl[nb][1] > s ? 1.0f : 0.0f);
+        yA[nb] = __ffma2_rn(m, ysA[nb], yA[nb]);
+        yB[nb] = __ffma2_rn(m, ysB[nb], yB[nb]);
+      }
+      if (++s == km) {
+        if (head) {  // the last slice of a tile the previous warp started: it adds this after the barrier
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            head_mine[(nb * 2 + 0) * 32 + lane] = yA[nb];
+            head_mine[(nb * 2 + 1) * 32 + lane] = yB[nb];
+          }
+          head = false;
+        } else {
+          dec_write_tile<NB>(out + tile * kDecRows, T, N, gid, t4, yA, yB);
+        }
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) yA[nb] = yB[nb] = make_float2(0.0f, 0.0f);
+        s = 0;
+        ++tile;
+      }
+    }
+    if (ok && s != 0) {  // this warp's run ended inside a tile: finished after the next barrier
+      tail = true;
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        scw[(nb * 2 + 0) * 32 + lane] = yA[nb];
+        scw[(nb * 2 + 1) * 32 + lane] = yB[nb];
+      }
+      if (lane == 0) {
+        s_tail_o[warp] = out + tile * kDecRows;
+        s_tail_tn[warp] = make_int2(T, N);
+      }
+    }
+    b = b_end;
   }
-  // Final CTA barrier: the producer then drains its copies if a warp gave up.
+  // Every copy this warp issued lands before the CTA may exit: normally all
+  // have been waited for; after a timeout the stages still in flight are
+  // drained here.
   __syncwarp();
-  __syncthreads();
+  if (lane == 0)
+    for (uint32_t i = done; i < issued; ++i) mbar_wait(&full[i % D], (i / D) & 1u, kDefaultWaitLimit, st, 0x2f0);
 }
 
 // Y[t][n] = sum over chunks c (in order) of partial[c][t][n], for every problem
@@ -614,8 +669,7 @@ size_t decode_ws_bytes(int64_t N, int64_t K) {
 }
 
 template <int NB, int MG>
-static cudaError_t launch_decode_class(const DecGroup<MG>& grp, int ctas, cudaStream_t stream, DeviceStatus* st,
-                                       bool early) {
+static cudaError_t launch_decode_class(const DecGroup<MG>& grp, int ctas, cudaStream_t stream, DeviceStatus* st) {
   using L = DecLayout<NB>;
   cudaError_t e = set_smem((const void*)decode_kernel<NB, MG>, (int)L::kDynamic);
   if (e != cudaSuccess) return e;
@@ -629,61 +683,25 @@ static cudaError_t launch_decode_class(const DecGroup<MG>& grp, int ctas, cudaSt
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, decode_kernel<NB, MG>, grp, st, wait_limit(), early ? 1 : 0);
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<NB, MG>, grp, st, wait_limit());
   if (e != cudaSuccess) return note_error("decode launch", e);
   return note_error("kernel launch", cudaGetLastError());
 }
 
-// One launch per fragment class present (T <= 8, then 9 <= T <= 16), each a
-// persistent grid of about one CTA per SM shared among that class's problems
-// in proportion to their weight counts N K (at least one CTA per K chunk, at
-// most one per 32-row block), then one chunk-reduction launch for every
-// problem with more than one chunk. Each launch is a programmatic dependent of
-// the one before; `early` as for the kernel (the launches that follow the
-// first class write none of the next class's inputs).
 // Fills a table of capacity MG with the problems `idx[0..n)` of one fragment
-// class and launches it; problems with several chunks are appended to `red`.
+// class and launches it on one CTA per SM; the kernel itself shares the CTAs
+// among the problems once it knows their k_t. Problems with several chunks are
+// appended to `red`.
 template <int MG>
 static cudaError_t decode_class(const DecodeJob* jobs, const int* idx, int n, int cls, int S, int sms,
-                                DecReduceGroup* red, cudaStream_t stream, DeviceStatus* st, bool early) {
-  double wsum = 0.0;
-  for (int m = 0; m < n; ++m) wsum += (double)jobs[idx[m]].N * (double)jobs[idx[m]].K;
+                                DecReduceGroup* red, cudaStream_t stream, DeviceStatus* st) {
   DecGroup<MG> grp;
   memset(&grp, 0, sizeof grp);
   grp.G = n;
   grp.S = S;
-  // CTAs per chunk: each problem's share of the SMs by weight count, rounded
-  // down (at least 1, at most one per 32-row block); then the SMs left over go,
-  // one chunk-width at a time, to the problem with the most weights per CTA.
-  int64_t cpcs[kMaxGroup], used = 0;
   for (int m = 0; m < n; ++m) {
     const DecodeJob& j = jobs[idx[m]];
     const int64_t nch = dec_chunks(j.K), nblocks = (j.N + kDecRows - 1) / kDecRows;
-    int64_t cpc = (int64_t)((double)sms * ((double)j.N * (double)j.K / wsum) / (double)nch);
-    if (cpc > nblocks) cpc = nblocks;
-    if (cpc < 1) cpc = 1;
-    cpcs[m] = cpc;
-    used += cpc * nch;
-  }
-  while (true) {
-    int best = -1;
-    double best_load = 0.0;
-    for (int m = 0; m < n; ++m) {
-      const DecodeJob& j = jobs[idx[m]];
-      const int64_t nch = dec_chunks(j.K), nblocks = (j.N + kDecRows - 1) / kDecRows;
-      if (cpcs[m] >= nblocks || used + nch > sms) continue;
-      const double load = (double)j.N * (double)j.K / (double)(cpcs[m] * nch);
-      if (load > best_load) { best_load = load; best = m; }
-    }
-    if (best < 0) break;
-    ++cpcs[best];
-    used += dec_chunks(jobs[idx[best]].K);
-  }
-  int ctas = 0;
-  for (int m = 0; m < n; ++m) {
-    const DecodeJob& j = jobs[idx[m]];
-    const int64_t nch = dec_chunks(j.K), nblocks = (j.N + kDecRows - 1) / kDecRows;
-    const int64_t cpc = cpcs[m];
     if (!make_tmap_2d(&grp.tm_codes[m], j.codes, 4, (uint64_t)(j.K / 16), (uint64_t)(S * j.N),
                       (uint64_t)(j.K / 16) * 4, 32, kDecRows, 128))
       return note_error("decode tensor map (codes)", cudaErrorInvalidValue);
@@ -691,8 +709,7 @@ static cudaError_t decode_class(const DecodeJob* jobs, const int* idx, int n, in
                       kDecRows, kDecChunk, 0))
       return note_error("decode tensor map (scale/zero)", cudaErrorInvalidValue);
     grp.p[m] = DecProblem{static_cast<const __nv_bfloat16*>(j.X), j.k_t, nch > 1 ? j.partial : j.Y, j.T, (int)j.N,
-                          (int)j.K, (int)(j.K / 128), (int)nblocks, (int)cpc, ctas};
-    ctas += (int)(cpc * nch);
+                          (int)j.K, (int)(j.K / 128), (int)nblocks, (int)nch};
     if (nch > 1) {
       red->partial[red->G] = reinterpret_cast<const float4*>(j.partial);
       red->Y[red->G] = reinterpret_cast<float4*>(j.Y);
@@ -701,19 +718,20 @@ static cudaError_t decode_class(const DecodeJob* jobs, const int* idx, int n, in
       ++red->G;
     }
   }
-  return cls == 1 ? launch_decode_class<1, MG>(grp, ctas, stream, st, early)
-                  : launch_decode_class<2, MG>(grp, ctas, stream, st, early);
+  return cls == 1 ? launch_decode_class<1, MG>(grp, sms, stream, st)
+                  : launch_decode_class<2, MG>(grp, sms, stream, st);
 }
 
 // One launch per fragment class present (T <= 8, then 9 <= T <= 16), each a
-// persistent grid of about one CTA per SM shared among that class's problems
-// in proportion to their weight counts N K (at least one CTA per K chunk, at
-// most one per 32-row block), then one chunk-reduction launch for every
-// problem with more than one chunk. Each launch is a programmatic dependent of
-// the one before; `early` as for the kernel (the launches that follow the
-// first class write none of the next class's inputs).
+// persistent grid of one CTA per SM that the kernel shares among that class's
+// problems in equal parts of the slices they read, then one chunk-reduction launch for
+// every problem with more than one chunk. Each launch is a programmatic
+// dependent of the one before. `early` (the kernel before is this library's
+// routing kernel) no longer changes anything: the decode kernel needs k_t
+// before it can choose its work, so it always waits first.
 cudaError_t launch_decode_grouped(const DecodeJob* jobs, int G, int S, cudaStream_t stream, DeviceStatus* st,
                                   bool early) {
+  (void)early;
   const int sms = num_sms();
   DecReduceGroup red = {};
   red.off[0] = 0;
@@ -725,8 +743,8 @@ cudaError_t launch_decode_grouped(const DecodeJob* jobs, int G, int S, cudaStrea
       if (j.T > 0 && j.N > 0 && (j.T > 8 ? 2 : 1) == cls) idx[n++] = i;
     }
     if (n == 0) continue;
-    const cudaError_t e = n == 1 ? decode_class<1>(jobs, idx, n, cls, S, sms, &red, stream, st, early)
-                                 : decode_class<kMaxGroup>(jobs, idx, n, cls, S, sms, &red, stream, st, early);
+    const cudaError_t e = n == 1 ? decode_class<1>(jobs, idx, n, cls, S, sms, &red, stream, st)
+                                 : decode_class<kMaxGroup>(jobs, idx, n, cls, S, sms, &red, stream, st);
     if (e != cudaSuccess) return e;
   }
   if (red.G == 0) return cudaSuccess;
