@@ -65,6 +65,12 @@ def _load():
             lib.oracle_bucket.restype = ci
             lib.oracle_gemm.argtypes = [p, i64, i64, p, p, p, i64, ci, ci, p, i64, p, ci]
             lib.oracle_gemm.restype = None
+            lib.oracle_gemm_bits.argtypes = [p, i64, i64, p, p, p, i64, ci, ci, ci, p, i64, p, ci]
+            lib.oracle_gemm_bits.restype = None
+            lib.oracle_unpack_bits.argtypes = [p, i64, i64, ci, ci, p]
+            lib.oracle_unpack_bits.restype = None
+            lib.oracle_reconstruct_bits.argtypes = [p, p, i64, i64, ci, ci, ci, ci, p]
+            lib.oracle_reconstruct_bits.restype = None
             lib.oracle_max_threads.argtypes = []
             lib.oracle_max_threads.restype = ci
             _lib = lib
@@ -104,11 +110,12 @@ def pack(W_f16: np.ndarray, G: int = 128, S: int = 3, nthreads: int = 0):
 
 def pack_bits(W_f16: np.ndarray, G: int = 128, S: int = 3, bits: int = 2, nthreads: int = 0):
     """MoBiSlice packing with `bits`-bit slices (1 or 2) over G-wide groups.
-    Returns (codes uint32 [S,N,K/16], sz uint32 [S,K/G,N], q uint8 [S,N,K])."""
+    Returns (codes uint32 [S,N,K*bits/32], sz uint32 [S,K/G,N], q uint8 [S,N,K]):
+    2-bit codes 16 per word, 1-bit codes 32 per word (documented layouts)."""
     lib = _load()
     W = _u16(W_f16)
     N, K = W.shape
-    codes = np.zeros((S, N, K // 16), np.uint32)
+    codes = np.zeros((S, N, K * bits // 32), np.uint32)
     sz = np.zeros((S, K // G, N), np.uint32)
     q = np.zeros((S, N, K), np.uint8)
     rc = lib.oracle_pack_bits(_ptr(W), N, K, G, S, bits, _ptr(codes), _ptr(sz), _ptr(q), nthreads)
@@ -117,21 +124,22 @@ def pack_bits(W_f16: np.ndarray, G: int = 128, S: int = 3, bits: int = 2, nthrea
     return codes, sz, q
 
 
-def unpack(codes: np.ndarray, N: int, K: int, S: int) -> np.ndarray:
-    """Packed words -> codes uint8 [S,N,K] by the documented layout."""
+def unpack(codes: np.ndarray, N: int, K: int, S: int, bits: int = 2) -> np.ndarray:
+    """Packed words -> codes uint8 [S,N,K] by the documented layout of `bits`-bit codes."""
     lib = _load()
     codes = np.ascontiguousarray(codes, np.uint32)
     q = np.zeros((S, N, K), np.uint8)
-    lib.oracle_unpack(_ptr(codes), N, K, S, _ptr(q))
+    lib.oracle_unpack_bits(_ptr(codes), N, K, S, bits, _ptr(q))
     return q
 
 
-def reconstruct(codes: np.ndarray, sz: np.ndarray, N: int, K: int, k: int, G: int = 128, S: int = 3) -> np.ndarray:
+def reconstruct(codes: np.ndarray, sz: np.ndarray, N: int, K: int, k: int, G: int = 128, S: int = 3,
+                bits: int = 2) -> np.ndarray:
     """W^(k) = sum of the first k dequantised slices, fp64 [N,K]."""
     lib = _load()
     out = np.zeros((N, K), np.float64)
-    lib.oracle_reconstruct(_ptr(np.ascontiguousarray(codes, np.uint32)), _ptr(np.ascontiguousarray(sz, np.uint32)),
-                           N, K, G, S, k, _ptr(out))
+    lib.oracle_reconstruct_bits(_ptr(np.ascontiguousarray(codes, np.uint32)),
+                                _ptr(np.ascontiguousarray(sz, np.uint32)), N, K, G, S, bits, k, _ptr(out))
     return out
 
 
@@ -185,8 +193,8 @@ def bucket(k_t: np.ndarray, S: int = 3):
 
 
 def gemm(X_bf16: np.ndarray, k_t: np.ndarray, codes: np.ndarray, sz: np.ndarray, N: int,
-         G: int = 128, S: int = 3, tokens: np.ndarray | None = None, nthreads: int = 0) -> np.ndarray:
-    """Y fp64 [len(tokens) or T, N] = x_t . W^(k_t)^T for the listed tokens."""
+         G: int = 128, S: int = 3, tokens: np.ndarray | None = None, nthreads: int = 0, bits: int = 2) -> np.ndarray:
+    """Y fp64 [len(tokens) or T, N] = x_t . W^(k_t)^T for the listed tokens (`bits`-bit codes)."""
     lib = _load()
     X = _u16(X_bf16)
     T, K = X.shape
@@ -194,6 +202,7 @@ def gemm(X_bf16: np.ndarray, k_t: np.ndarray, codes: np.ndarray, sz: np.ndarray,
     tok = None if tokens is None else np.ascontiguousarray(tokens, np.int32)
     n_tok = T if tok is None else tok.shape[0]
     Y = np.zeros((n_tok, N), np.float64)
-    lib.oracle_gemm(_ptr(X), T, K, _ptr(k_t), _ptr(np.ascontiguousarray(codes, np.uint32)),
-                    _ptr(np.ascontiguousarray(sz, np.uint32)), N, G, S, _ptr(tok), n_tok, _ptr(Y), nthreads)
+    lib.oracle_gemm_bits(_ptr(X), T, K, _ptr(k_t), _ptr(np.ascontiguousarray(codes, np.uint32)),
+                         _ptr(np.ascontiguousarray(sz, np.uint32)), N, G, S, bits, _ptr(tok), n_tok, _ptr(Y),
+                         nthreads)
     return Y

@@ -34,7 +34,9 @@
  *   (oracle_pack_bits): the same quantiser with b-bit codes, L = 2^b - 1 steps
  *   (s = (max-min)/L, z and q clamped to [0, L]) over G-wide groups; 1-bit
  *   slices give 1..S bits per weight ([en] §2.A lists 3-bit precision, which
- *   2-bit slices cannot reach).
+ *   2-bit slices cannot reach) and are stored at 1 bit per weight ([en] §3,
+ *   "Specialized Kernel Implementation": the bytes fetched follow the bits
+ *   used), 32 codes per word in the library's documented bit order.
  *
  * Parity pins: every function here is pinned by tests/test_oracle.py against
  * closed-form groups, hand-derived packed words, invariants (non-increasing
@@ -135,20 +137,38 @@ static void quantise_group(const uint16_t* w, int G, int S, int bits, uint8_t* q
 }
 
 /*
+ * The documented word layouts. 2-bit codes: words [S][N][K/16]; word (s, n, w)
+ * holds q(s, n, 16w + i) in bits [2i+1 : 2i]. 1-bit codes: words [S][N][K/32];
+ * word (s, n, w) holds q(s, n, 32w + i) in bit 2i for i < 16 and
+ * q(s, n, 32w + 16 + i) in bit 2i + 1 (the first 16 codes on the even bits,
+ * the next 16 on the odd bits).
+ */
+static int64_t words_per_row(int64_t K, int bits) { return bits == 1 ? K / 32 : K / 16; }
+
+static int code_of(const uint32_t* codes, int64_t N, int64_t K, int bits, int64_t s, int64_t n, int64_t k) {
+  const uint32_t word = codes[(s * N + n) * words_per_row(K, bits) + (bits == 1 ? k / 32 : k / 16)];
+  if (bits == 1) {
+    const int i = (int)(k % 32);
+    return (int)((word >> (i < 16 ? 2 * i : 2 * (i - 16) + 1)) & 1u);
+  }
+  return (int)((word >> (2 * (k % 16))) & 3u);
+}
+
+/*
  * oracle_pack_bits: W fp16 [N][K] -> codes and sz for S slices of `bits`-bit
- * codes (bits 1 or 2) over G-wide groups. Codes of either width sit in the
- * documented 2-bit word layout (word (s, n, w) holds q(s, n, 16w + i) in bits
- * [2i+1:2i]; a 1-bit code only uses values 0 and 1). sz is [S][K/G][N] (fp16
- * scale in bits [15:0], fp16 zero in bits [31:16]). If q_out is not NULL it
- * receives the unpacked codes uint8 [S][N][K].
+ * codes (bits 1 or 2) over G-wide groups, codes in the word layout of their
+ * width (above). sz is [S][K/G][N] (fp16 scale in bits [15:0], fp16 zero in
+ * bits [31:16]). If q_out is not NULL it receives the unpacked codes uint8
+ * [S][N][K].
  * Returns 0, or -1 on an unsupported argument.
  */
 int oracle_pack_bits(const uint16_t* W, int64_t N, int64_t K, int G, int S, int bits,
                      uint32_t* codes, uint32_t* sz, uint8_t* q_out, int nthreads) {
   if (G <= 0 || G > 1024 || K % G != 0 || K % 16 != 0 || S < 1 || S > 8 || bits < 1 || bits > 2) return -1;
+  if (bits == 1 && K % 32 != 0) return -1;
   set_threads(nthreads);
   const int64_t ngroups = K / G;
-  const int64_t nwords = K / 16;
+  const int64_t nwords = words_per_row(K, bits);
 #pragma omp parallel for schedule(dynamic, 4)
   for (int64_t n = 0; n < N; ++n) {
     uint8_t q[8 * 1024];
@@ -164,8 +184,15 @@ int oracle_pack_bits(const uint16_t* W, int64_t N, int64_t K, int G, int S, int 
     for (int s = 0; s < S; ++s) {
       for (int64_t w = 0; w < nwords; ++w) {
         uint32_t word = 0;
-        for (int i = 0; i < 16; ++i)
-          word |= (uint32_t)row_codes[(int64_t)s * K + 16 * w + i] << (2 * i);
+        if (bits == 1) {
+          for (int i = 0; i < 16; ++i) {
+            word |= (uint32_t)row_codes[(int64_t)s * K + 32 * w + i] << (2 * i);
+            word |= (uint32_t)row_codes[(int64_t)s * K + 32 * w + 16 + i] << (2 * i + 1);
+          }
+        } else {
+          for (int i = 0; i < 16; ++i)
+            word |= (uint32_t)row_codes[(int64_t)s * K + 16 * w + i] << (2 * i);
+        }
         codes[((int64_t)s * N + n) * nwords + w] = word;
       }
       if (q_out)
@@ -185,15 +212,16 @@ int oracle_pack(const uint16_t* W, int64_t N, int64_t K, int G, int S,
   return oracle_pack_bits(W, N, K, G, S, 2, codes, sz, q_out, nthreads);
 }
 
-/* oracle_unpack: the documented word layout back to codes uint8 [S][N][K]. */
-void oracle_unpack(const uint32_t* codes, int64_t N, int64_t K, int S, uint8_t* q_out) {
-  const int64_t nwords = K / 16;
+/* oracle_unpack_bits: the documented word layout of `bits`-bit codes back to
+ * codes uint8 [S][N][K]; oracle_unpack is the 2-bit case. */
+void oracle_unpack_bits(const uint32_t* codes, int64_t N, int64_t K, int S, int bits, uint8_t* q_out) {
   for (int64_t s = 0; s < S; ++s)
     for (int64_t n = 0; n < N; ++n)
-      for (int64_t k = 0; k < K; ++k) {
-        uint32_t word = codes[(s * N + n) * nwords + k / 16];
-        q_out[(s * N + n) * K + k] = (uint8_t)((word >> (2 * (k % 16))) & 3u);
-      }
+      for (int64_t k = 0; k < K; ++k) q_out[(s * N + n) * K + k] = (uint8_t)code_of(codes, N, K, bits, s, n, k);
+}
+
+void oracle_unpack(const uint32_t* codes, int64_t N, int64_t K, int S, uint8_t* q_out) {
+  oracle_unpack_bits(codes, N, K, S, 2, q_out);
 }
 
 /*
@@ -201,15 +229,14 @@ void oracle_unpack(const uint32_t* codes, int64_t N, int64_t K, int S, uint8_t* 
  * in fp64 (exact: every term is a small integer times an fp16 value)
  * ([ja] §2.1 W^(b) = sum W_e; [en] §2.A "Elasticity").
  */
-void oracle_reconstruct(const uint32_t* codes, const uint32_t* sz, int64_t N, int64_t K,
-                        int G, int S, int k, double* W_hat) {
-  const int64_t nwords = K / 16, ngroups = K / G;
+void oracle_reconstruct_bits(const uint32_t* codes, const uint32_t* sz, int64_t N, int64_t K, int G, int S,
+                             int bits, int k, double* W_hat) {
+  const int64_t ngroups = K / G;
   for (int64_t n = 0; n < N; ++n)
     for (int64_t j = 0; j < K; ++j) {
       double acc = 0.0;
       for (int s = 0; s < k && s < S; ++s) {
-        uint32_t word = codes[((int64_t)s * N + n) * nwords + j / 16];
-        int q = (int)((word >> (2 * (j % 16))) & 3u);
+        int q = code_of(codes, N, K, bits, s, n, j);
         uint32_t e = sz[((int64_t)s * ngroups + j / G) * N + n];
         double scale = (double)half_bits_to_float((uint16_t)(e & 0xffffu));
         double zero = (double)half_bits_to_float((uint16_t)(e >> 16));
@@ -217,6 +244,11 @@ void oracle_reconstruct(const uint32_t* codes, const uint32_t* sz, int64_t N, in
       }
       W_hat[n * K + j] = acc;
     }
+}
+
+void oracle_reconstruct(const uint32_t* codes, const uint32_t* sz, int64_t N, int64_t K,
+                        int G, int S, int k, double* W_hat) {
+  oracle_reconstruct_bits(codes, sz, N, K, G, S, 2, k, W_hat);
 }
 
 /* ---- MoBiRoute ---------------------------------------------------------- */
@@ -325,17 +357,18 @@ int oracle_bucket(const int32_t* k_t, int64_t T, int S, int32_t* perm, int32_t* 
 /* ---- mixed-bit GEMM ----------------------------------------------------- */
 
 /*
- * oracle_gemm: for each listed token t = tokens[i] (all tokens when tokens is
- * NULL, i = t), Y[i][n] = sum_k x[t,k] * W^(k_t)[n,k] in fp64, with
- * W^(k) = sum_{s<k} (q - z) * scale built exactly ([ja] §2.1; [en] §2.A).
- * Y is fp64 [n_tokens][N]. The sum over k runs in index order.
+ * oracle_gemm_bits: for each listed token t = tokens[i] (all tokens when
+ * tokens is NULL, i = t), Y[i][n] = sum_k x[t,k] * W^(k_t)[n,k] in fp64, with
+ * W^(k) = sum_{s<k} (q - z) * scale built exactly ([ja] §2.1; [en] §2.A) from
+ * `bits`-bit codes. Y is fp64 [n_tokens][N]. The sum over k runs in index
+ * order. oracle_gemm is the 2-bit case.
  */
-void oracle_gemm(const uint16_t* X, int64_t T, int64_t K, const int32_t* k_t,
-                 const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S,
-                 const int32_t* tokens, int64_t n_tokens, double* Y, int nthreads) {
+void oracle_gemm_bits(const uint16_t* X, int64_t T, int64_t K, const int32_t* k_t,
+                      const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S, int bits,
+                      const int32_t* tokens, int64_t n_tokens, double* Y, int nthreads) {
   (void)T;
   set_threads(nthreads);
-  const int64_t nwords = K / 16, ngroups = K / G;
+  const int64_t ngroups = K / G;
   if (!tokens) n_tokens = T;
 #pragma omp parallel for schedule(dynamic, 8)
   for (int64_t n = 0; n < N; ++n) {
@@ -344,8 +377,7 @@ void oracle_gemm(const uint16_t* X, int64_t T, int64_t K, const int32_t* k_t,
     for (int64_t j = 0; j < K; ++j) {
       double acc = 0.0;
       for (int s = 0; s < S; ++s) {
-        uint32_t word = codes[((int64_t)s * N + n) * nwords + j / 16];
-        int q = (int)((word >> (2 * (j % 16))) & 3u);
+        int q = code_of(codes, N, K, bits, s, n, j);
         uint32_t e = sz[((int64_t)s * ngroups + j / G) * N + n];
         double scale = (double)half_bits_to_float((uint16_t)(e & 0xffffu));
         double zero = (double)half_bits_to_float((uint16_t)(e >> 16));
@@ -362,4 +394,10 @@ void oracle_gemm(const uint16_t* X, int64_t T, int64_t K, const int32_t* k_t,
     }
     free(wk);
   }
+}
+
+void oracle_gemm(const uint16_t* X, int64_t T, int64_t K, const int32_t* k_t,
+                 const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S,
+                 const int32_t* tokens, int64_t n_tokens, double* Y, int nthreads) {
+  oracle_gemm_bits(X, T, K, k_t, codes, sz, N, G, S, 2, tokens, n_tokens, Y, nthreads);
 }

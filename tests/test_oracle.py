@@ -416,7 +416,7 @@ def test_generic_slice1_matches_torch_fake_quantize(oracle, bits, G):
     x = torch.from_numpy(W.astype(np.float32).reshape(N * K // G, G))
     fq = torch.fake_quantize_per_channel_affine(x, torch.from_numpy(scale), torch.from_numpy(zero), 0, 0,
                                                 (1 << bits) - 1)
-    W1 = oracle.reconstruct(codes, sz, N, K, k=1, G=G, S=1)
+    W1 = oracle.reconstruct(codes, sz, N, K, k=1, G=G, S=1, bits=bits)
     assert np.array_equal(fq.numpy().astype(np.float64).reshape(N, K), W1)
 
 
@@ -448,10 +448,13 @@ def test_one_bit_hand_group(oracle):
     codes, sz, q = oracle.pack_bits(W, G=128, S=2, bits=1)
     assert int(sz[0, 0, 0]) == f16_bits(3.0) | (f16_bits(0.0) << 16)
     assert np.array_equal(q[0, 0], np.tile([0, 1], 64))
-    assert int(codes[0, 0, 0]) == sum(1 << (2 * i) for i in range(1, 16, 2))  # odd fields hold 1
+    # 1 bit per weight: 4 words per 128-group; word 0 holds k = 0..15 on the
+    # even bits and k = 16..31 on the odd bits, and every odd k is 1.
+    assert codes.shape == (2, 1, 4)
+    assert int(codes[0, 0, 0]) == 0xCCCCCCCC
     assert int(sz[1, 0, 0]) == 0x0400 | (f16_bits(1.0) << 16)  # 2^-14, zero 1
     assert np.all(q[1, 0] == 0)
-    W2 = oracle.reconstruct(codes, sz, 1, 128, k=2, G=128, S=2)
+    W2 = oracle.reconstruct(codes, sz, 1, 128, k=2, G=128, S=2, bits=1)
     assert np.all(W2[0] == np.tile([0.0 - 2.0 ** -14, 3.0 - 2.0 ** -14], 64))
 
 
@@ -466,11 +469,47 @@ def test_generic_residual_never_grows(oracle, bits, G):
     Wd = W.astype(np.float64)
     prev, fro = np.abs(Wd), [np.linalg.norm(Wd)]
     for k in range(1, S + 1):
-        e = np.abs(Wd - oracle.reconstruct(codes, sz, N, K, k=k, G=G, S=S))
+        e = np.abs(Wd - oracle.reconstruct(codes, sz, N, K, k=k, G=G, S=S, bits=bits))
         assert np.all(e <= prev + 1e-6 * np.abs(Wd) + 1e-9)
         prev = e
         fro.append(np.linalg.norm(e))
     assert all(b < a for a, b in zip(fro[:-1], fro[1:]))
+
+
+def test_one_bit_words_hand_derived(oracle):
+    """Derived by hand from the documented 1-bit layout: a 0/1 row quantises to
+    itself in one 1-bit slice (step 1, zero 0), so ones at k = 0, 15, 16, 31,
+    32 and 127 give word 0 = bits 0, 30, 1, 31 = 0xC0000003, word 1 = bit 0,
+    word 2 = 0 and word 3 = bit 31 (k = 96 + 31)."""
+    row = np.zeros(128, np.float32)
+    row[[0, 15, 16, 31, 32, 127]] = 1.0
+    W = row.astype(np.float16)[None, :]
+    codes, sz, q = oracle.pack_bits(W, G=128, S=1, bits=1)
+    assert int(sz[0, 0, 0]) == f16_bits(1.0)  # scale 1, zero 0
+    assert [int(w) for w in codes[0, 0]] == [0xC0000003, 0x00000001, 0x00000000, 0x80000000]
+    assert np.array_equal(oracle.unpack(codes, 1, 128, 1, bits=1)[0, 0], row.astype(np.uint8))
+
+
+@pytest.mark.parametrize("S", [1, 4])
+def test_one_bit_gemm_equals_two_bit_storage(oracle, S):
+    """The same 1-bit codes stored in the 2-bit word layout (pinned above by
+    hand words) give the same reconstruction and GEMM, bit for bit: the 1-bit
+    reader only changes where a code is read from."""
+    N, K, T = 24, 512, 5
+    W = _random_W(N, K, 60 + S, outliers=3)
+    codes1, sz, q = oracle.pack_bits(W, G=128, S=S, bits=1)
+    assert codes1.shape == (S, N, K // 32)
+    assert np.array_equal(oracle.unpack(codes1, N, K, S, bits=1), q)
+    codes2 = np.zeros((S, N, K // 16), np.uint32)  # 2-bit layout: q(16w + i) in bits [2i+1 : 2i]
+    for i in range(16):
+        codes2 |= q[:, :, i::16].astype(np.uint32) << np.uint32(2 * i)
+    for k in range(1, S + 1):
+        assert np.array_equal(oracle.reconstruct(codes1, sz, N, K, k=k, S=S, bits=1),
+                              oracle.reconstruct(codes2, sz, N, K, k=k, S=S, bits=2))
+    rng = np.random.default_rng(S)
+    X = torch.from_numpy(rng.standard_normal((T, K), dtype=np.float32)).to(torch.bfloat16)
+    k_t = rng.integers(1, S + 1, T).astype(np.int32)
+    assert np.array_equal(oracle.gemm(X, k_t, codes1, sz, N, S=S, bits=1), oracle.gemm(X, k_t, codes2, sz, N, S=S))
 
 
 def test_pack_bits_rejects_bad_arguments(oracle):
