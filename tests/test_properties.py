@@ -44,11 +44,11 @@ def test_packer_invariants(oracle, case):
     assert np.all(sc >= 2.0 ** -14) and np.all(np.isfinite(sc))
     assert np.all((zr == np.round(zr)) & (zr >= 0) & (zr <= L))
     # the documented word layout holds the unpacked codes
-    assert np.array_equal(oracle.unpack(codes, N, K, S), q)
+    assert np.array_equal(oracle.unpack(codes, N, K, S, bits=bits), q)
     Wd = W.astype(np.float64)
     prev = np.abs(Wd)
     for k in range(1, S + 1):
-        err = np.abs(Wd - oracle.reconstruct(codes, sz, N, K, k=k, G=G, S=S))
+        err = np.abs(Wd - oracle.reconstruct(codes, sz, N, K, k=k, G=G, S=S, bits=bits))
         assert np.all(err <= prev + 1e-6 * np.abs(Wd) + 1e-12)
         prev = err
 
@@ -67,7 +67,7 @@ def test_on_grid_group_is_exact(oracle, seed, bits, zshift):
     W = ((c - z) * step).astype(F16).reshape(1, 128)
     codes, sz, q = oracle.pack_bits(W, G=128, S=2, bits=bits)
     assert np.array_equal(q[0, 0], c)
-    W1 = oracle.reconstruct(codes, sz, 1, 128, k=1, G=128, S=2)
+    W1 = oracle.reconstruct(codes, sz, 1, 128, k=1, G=128, S=2, bits=bits)
     assert np.array_equal(W1, W.astype(np.float64))
 
 
