@@ -49,8 +49,10 @@ def peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def decode_bytes(N, K, T, kmax):
-    return kmax * (N * K // 4 + N * (K // 128) * 4) + T * K * 2
+def decode_bytes(N, K, T, kmax, bits=2):
+    """Algorithmic bytes of one decode GEMM: k_max slices of codes (bits per
+    weight) and scale/zero words, plus X."""
+    return kmax * (N * K * bits // 8 + N * (K // 128) * 4) + T * K * 2
 
 
 # DRAM bytes / algorithmic bytes of the decode kernel, from one ncu capture of
@@ -558,53 +560,57 @@ def time_ckpt(mobi, wl, dev, reps=3):
 
 
 def time_generic(mobi, wl, dev, hbm_peak, tf_peak, flush, steps=200):
-    """Generic slicing: four 1-bit slices (1..4 bits per weight), G = 128.
-    (a) the decode step of the three Llama-7B shapes at T = 4 as one
-    mobi_linear_grouped call, router mix 1/4 each (three packed copies in
-    rotation, so no copy is L2-resident when it is read again); (b) the prefill
-    workload's shape (T = 2048, 11008 x 4096) through route + prefill GEMM.
-    1-bit codes sit in 2-bit fields, so the bytes read are those of 2-bit
-    slices: k slices give k bits of precision and cost 2k bits of codes."""
+    """Generic slicing: four 1-bit slices (1..4 bits per weight), G = 128, the
+    codes stored at 1 bit per weight. (a) the decode step of the three
+    Llama-7B shapes at T = 4 as one mobi_linear_grouped call, router mix 1/4
+    each (five packed copies in rotation, so no copy is L2-resident when it is
+    read again), beside the same step with four 2-bit slices (same k_max, twice
+    the code bytes); (b) the prefill workload's shape (T = 2048, 11008 x 4096)
+    through route + prefill GEMM."""
     S = 4
-    out = {"slicing": "4 x 1-bit slices, G = 128 (codes stored in 2-bit fields)"}
-    # Three packed copies of the three problems, run one after another in each
-    # step, so a copy is read again only after ~240 MB of other weights (> 2x L2).
-    copies = 3
-    groups = []
-    for r in range(copies):
-        probs = []
-        for i, (N, K) in enumerate(wl.DECODE_SHAPES):
-            L = wl.layer(f"gen_{N}x{K}", N, K, 4, seed=3000 + i, outlier_frac_cols=0.005, S=S, mix=(0.25,) * S)
-            codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(dev), S=S, bits=1)
-            probs.append({"X": L.X.to(dev), "Wr": torch.from_numpy(L.Wr).to(dev),
-                          "bias": torch.from_numpy(L.bias).to(dev), "codes": codes, "sz": sz, "N": N,
-                          "Y": torch.empty((4, N), dtype=torch.float32, device=dev),
-                          "k_t": torch.empty(4, dtype=torch.int32, device=dev),
-                          "perm": torch.empty(4, dtype=torch.int32, device=dev),
-                          "offsets": torch.empty(S + 1, dtype=torch.int32, device=dev)})
-        groups.append(probs)
-    ws = torch.empty(max(mobi.mobi_linear_grouped_workspace_bytes(groups[0], S=S), 16), dtype=torch.uint8,
-                     device=dev)
+    out = {"slicing": "4 x 1-bit slices, G = 128, codes at 1 bit per weight (32 per word)"}
+    # Five packed copies of the three problems, run one after another in each
+    # step, so a copy is read again only after 4 x its bytes of other weights
+    # (above 200 MB at 1 bit per weight, more than the 126 MB L2).
+    copies = 5
+    for bits in (1, 2):
+        groups = []
+        for r in range(copies):
+            probs = []
+            for i, (N, K) in enumerate(wl.DECODE_SHAPES):
+                L = wl.layer(f"gen_{N}x{K}", N, K, 4, seed=3000 + i, outlier_frac_cols=0.005, S=S, mix=(0.25,) * S)
+                codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(dev), S=S, bits=bits)
+                probs.append({"X": L.X.to(dev), "Wr": torch.from_numpy(L.Wr).to(dev),
+                              "bias": torch.from_numpy(L.bias).to(dev), "codes": codes, "sz": sz, "N": N,
+                              "Y": torch.empty((4, N), dtype=torch.float32, device=dev),
+                              "k_t": torch.empty(4, dtype=torch.int32, device=dev),
+                              "perm": torch.empty(4, dtype=torch.int32, device=dev),
+                              "offsets": torch.empty(S + 1, dtype=torch.int32, device=dev)})
+            groups.append(probs)
+        ws = torch.empty(max(mobi.mobi_linear_grouped_workspace_bytes(groups[0], S=S), 16), dtype=torch.uint8,
+                         device=dev)
 
-    def step():
-        for probs in groups:
-            mobi.mobi_linear_grouped(probs, S=S, ws=ws)
-    step()
-    mobi.mobi_sync_check()
-    kmax = [int(p["k_t"].max().item()) for p in groups[0]]
-    nbytes = sum(decode_bytes(p["N"], p["X"].shape[1], 4, km) for p, km in zip(groups[0], kmax))
-    ms = time_graph(step, steps) / copies
-    out["decode_T4_grouped"] = {"kmax_per_problem": kmax, "bytes_per_call": nbytes, "ms_per_call": round(ms, 5),
-                                "GB/s": round(nbytes / ms / 1e6, 1), "frac_of_hbm": round(nbytes / ms / 1e6 / hbm_peak, 4),
-                                "precision_bits_per_weight": kmax,
-                                "code_bits_read_per_weight": [2 * km for km in kmax],
-                                "l2": f"{copies} packed copies in rotation, each read again after ~{2 * nbytes / 1e6:.0f} MB"}
-    del groups, ws
+        def step():
+            for probs in groups:
+                mobi.mobi_linear_grouped(probs, S=S, ws=ws, bits=bits)
+        step()
+        mobi.mobi_sync_check()
+        kmax = [int(p["k_t"].max().item()) for p in groups[0]]
+        nbytes = sum(decode_bytes(p["N"], p["X"].shape[1], 4, km, bits) for p, km in zip(groups[0], kmax))
+        ms = time_graph(step, steps) / copies
+        key = "decode_T4_grouped" if bits == 1 else "decode_T4_grouped_2bit_slices"
+        out[key] = {"kmax_per_problem": kmax, "bytes_per_call": nbytes, "ms_per_call": round(ms, 5),
+                    "GB/s": round(nbytes / ms / 1e6, 1), "frac_of_hbm": round(nbytes / ms / 1e6 / hbm_peak, 4),
+                    "precision_bits_per_weight": [bits * km for km in kmax],
+                    "code_bits_read_per_weight": [bits * km for km in kmax],
+                    "l2": f"{copies} packed copies in rotation, each read again after ~{(copies - 1) * nbytes / 1e6:.0f} MB"}
+        del groups, ws
     L = wl.layer("gen_prefill_11008x4096_T2048", 11008, 4096, 2048, seed=3010, n_outlier_cols=20, S=S,
                  mix=(0.25,) * S)
     W = torch.from_numpy(L.W).to(dev)
     codes, sz = mobi.mobi_pack(W, S=S, bits=1)
     del W
+    assert codes.numel() * 4 == mobi.mobi_codes_bytes(11008, 4096, S, bits=1)
     X = L.X.to(dev)
     Wr = torch.from_numpy(L.Wr).to(dev)
     b = torch.from_numpy(L.bias).to(dev)
@@ -617,7 +623,7 @@ def time_generic(mobi, wl, dev, hbm_peak, tf_peak, flush, steps=200):
     ws_g = torch.empty(mobi.mobi_gemm_workspace_bytes(T, N, K, S), dtype=torch.uint8, device=dev)
     mobi.mobi_route(X, Wr, b, k_t, perm, off, ws_r)
     for _ in range(3):
-        mobi.mobi_gemm(X, k_t, perm, off, codes, sz, N, Y=Y, ws=ws_g)
+        mobi.mobi_gemm(X, k_t, perm, off, codes, sz, N, Y=Y, ws=ws_g, bits=1)
     mobi.mobi_sync_check()
     sumk = int(k_t.sum().item())
     ts = []
@@ -625,7 +631,7 @@ def time_generic(mobi, wl, dev, hbm_peak, tf_peak, flush, steps=200):
         flush.fill_(1.0)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        mobi.mobi_gemm(X, k_t, perm, off, codes, sz, N, Y=Y, ws=ws_g)
+        mobi.mobi_gemm(X, k_t, perm, off, codes, sz, N, Y=Y, ws=ws_g, bits=1)
         e1.record()
         torch.cuda.synchronize()
         ts.append(e0.elapsed_time(e1))

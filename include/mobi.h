@@ -62,6 +62,11 @@
  *   codes  uint32 [S][N][K/16]   word w of (slice s, row n) holds the codes of
  *          k = 16w .. 16w+15; code q(s,n,16w+i) sits in bits [2i+1 : 2i]
  *          (little-endian 2-bit fields). mobi_codes_bytes() gives the size.
+ *          1-bit codes (mobi_pack_bits with bits = 1) take 1 bit per weight:
+ *          uint32 [S][N][K/32], word w holds k = 32w .. 32w+31 with
+ *          q(s,n,32w+i) in bit 2i and q(s,n,32w+16+i) in bit 2i+1 (i < 16): its
+ *          even bits are the 2-bit layout's word 2w and its odd bits word
+ *          2w+1, each code a 0/1 field. mobi_codes_bytes_bits() gives the size.
  *   sz     uint32 [S][K/G][N]    element (s,g,n): bits [15:0] = fp16 scale,
  *          bits [31:16] = fp16 zero (an integer 0..2^b - 1). mobi_sz_bytes().
  *          Group-major so that the scales of one group for consecutive rows
@@ -123,6 +128,8 @@ MOBI_API int mobi_version(void);
 /* Bytes of the packed code array for S slices of an N x K matrix:
  * S * N * (K/16) * 4. Returns 0 for invalid sizes. */
 MOBI_API size_t mobi_codes_bytes(int64_t N, int64_t K, int S);
+/* Bytes of the codes of S slices of `bits`-bit codes (1 or 2; K % 32 == 0). */
+MOBI_API size_t mobi_codes_bytes_bits(int64_t N, int64_t K, int S, int bits);
 
 /* Bytes of the scale/zero array: S * N * (K/G) * 4. Returns 0 for invalid sizes. */
 MOBI_API size_t mobi_sz_bytes(int64_t N, int64_t K, int S, int G);
@@ -160,10 +167,11 @@ MOBI_API mobi_status mobi_pack(const void* W, int64_t N, int64_t K, int G, int S
  *   this header with L = 2^bits - 1 steps.
  *   W, N, K, S, codes  as for mobi_pack (S 1..4; K % G == 0).
  *   G        128, 256 or 512.
- *   bits     1 or 2. Codes of either width sit in the 2-bit fields of the
- *            documented layout (a 1-bit code uses only the values 0 and 1), so
- *            every GEMM entry point reads them unchanged; a 1-bit slice costs
- *            the bytes of a 2-bit one.
+ *   bits     1 or 2. 2-bit codes in the 2-bit layout; 1-bit codes at 1 bit per
+ *            weight in the 1-bit layout ([en] §3 "Specialized Kernel
+ *            Implementation": the bytes fetched follow the bits used), read by
+ *            mobi_gemm_bits / mobi_gemm_grouped_bits with bits = 1.
+ *   codes    out, mobi_codes_bytes_bits(N, K, S, bits) bytes.
  *   sz       out, uint32 [S][K/128][N] whatever G is: the scale/zero word of
  *            a G-wide group is repeated in each of its G/128 128-column
  *            sub-groups (size: mobi_sz_bytes(N, K, S, 128)), which is the
@@ -254,7 +262,7 @@ MOBI_API mobi_status mobi_gemm(const void* X, int64_t T, int64_t K, const int32_
                       const uint32_t* codes, const uint32_t* sz, int64_t N, int G,
                       int S, float* Y, void* ws, size_t ws_bytes, void* stream);
 
-/* Kernel selection for mobi_gemm_path. */
+/* Kernel selection for mobi_gemm_path and mobi_gemm_bits. */
 typedef enum {
   MOBI_PATH_AUTO = 0,    /* decode for T <= 16, prefill otherwise */
   MOBI_PATH_DECODE = 1,  /* decode kernel; requires T <= 16 */
@@ -267,6 +275,19 @@ MOBI_API mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const i
                            const uint32_t* codes, const uint32_t* sz, int64_t N,
                            int G, int S, float* Y, void* ws, size_t ws_bytes,
                            void* stream, int path);
+
+/*
+ * mobi_gemm_bits — mobi_gemm_path for slices of `bits`-bit codes (1 or 2, as
+ *   written by mobi_pack_bits; 2 is mobi_gemm_path). Same arguments, result
+ *   and workspace. Both kernels read each slice's codes in their own layout:
+ *   a 1-bit slice streams half the code bytes of a 2-bit one, and the
+ *   operands stay exact (a 1-bit code is a 0/1 field where a 2-bit code is a
+ *   0..3 field). MOBI_ERR_INVALID_ARG for other widths.
+ */
+MOBI_API mobi_status mobi_gemm_bits(const void* X, int64_t T, int64_t K, const int32_t* k_t,
+                                    const int32_t* perm, const int32_t* offsets, const uint32_t* codes,
+                                    const uint32_t* sz, int64_t N, int G, int S, int bits, float* Y, void* ws,
+                                    size_t ws_bytes, void* stream, int path);
 
 /* Scratch bytes of mobi_linear: the routing workspace (rounded up to 256
  * bytes) followed by the GEMM workspace. */
@@ -294,6 +315,13 @@ MOBI_API mobi_status mobi_linear(const void* X, int64_t T, int64_t K, const floa
                                  int64_t N, int G, int S, int32_t* k_t, int32_t* perm,
                                  int32_t* offsets, float* Y, void* ws, size_t ws_bytes,
                                  void* stream);
+
+/* mobi_linear for slices of `bits`-bit codes (1 or 2; 2 is mobi_linear), as
+ * mobi_gemm_bits is to mobi_gemm_path. */
+MOBI_API mobi_status mobi_linear_bits(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
+                                      const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S, int bits,
+                                      int32_t* k_t, int32_t* perm, int32_t* offsets, float* Y, void* ws,
+                                      size_t ws_bytes, void* stream);
 
 /* One problem of mobi_linear_grouped: the arguments of one mobi_linear call. */
 typedef struct mobi_linear_problem {
@@ -340,6 +368,11 @@ MOBI_API size_t mobi_gemm_grouped_workspace_bytes(const mobi_gemm_problem* probl
 MOBI_API mobi_status mobi_gemm_grouped(const mobi_gemm_problem* problems, int count, int G, int S,
                                        void* ws, size_t ws_bytes, void* stream);
 
+/* mobi_gemm_grouped for slices of `bits`-bit codes (1 or 2; every problem of
+ * the call has that width), as mobi_gemm_bits is to mobi_gemm_path. */
+MOBI_API mobi_status mobi_gemm_grouped_bits(const mobi_gemm_problem* problems, int count, int G, int S, int bits,
+                                            void* ws, size_t ws_bytes, void* stream);
+
 /*
  * mobi_linear_grouped — up to MOBI_MAX_GROUP independent decode-sized
  *   mobi_linear problems (every T <= 16) in one step: the projections of a
@@ -362,6 +395,11 @@ MOBI_API mobi_status mobi_gemm_grouped(const mobi_gemm_problem* problems, int co
  */
 MOBI_API mobi_status mobi_linear_grouped(const mobi_linear_problem* problems, int count, int G,
                                          int S, void* ws, size_t ws_bytes, void* stream);
+
+/* mobi_linear_grouped for slices of `bits`-bit codes (1 or 2; every problem of
+ * the call has that width). */
+MOBI_API mobi_status mobi_linear_grouped_bits(const mobi_linear_problem* problems, int count, int G, int S,
+                                              int bits, void* ws, size_t ws_bytes, void* stream);
 
 /* ---- many-in-one checkpoints of packed layers -------------------------------
  *
@@ -392,7 +430,7 @@ MOBI_API mobi_status mobi_linear_grouped(const mobi_linear_problem* problems, in
  */
 typedef struct mobi_ckpt_tensor {
   const char* name;       /* at most 95 bytes, unique in the file */
-  const uint32_t* codes;  /* [S][N][K/16], as produced by mobi_pack */
+  const uint32_t* codes;  /* [S][N][K/16], as produced by mobi_pack (2-bit codes only) */
   const uint32_t* sz;     /* [S][K/G][N] */
   int64_t N, K;
   int G, S;

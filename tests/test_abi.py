@@ -46,7 +46,9 @@ def test_status_strings_and_sizes(L):
     assert mobi.mobi_version() >= 100
     assert mobi.mobi_codes_bytes(4096, 4096, 3) == 3 * 4096 * 256 * 4
     assert mobi.mobi_sz_bytes(4096, 4096, 3, 128) == 3 * 4096 * 32 * 4
-    assert mobi.mobi_codes_bytes(16, 100, 3) == 0  # K % 16 != 0
+    assert mobi.mobi_codes_bytes(16, 100, 3) == 0  # K % 32 != 0
+    assert mobi.mobi_codes_bytes(4096, 4096, 4, bits=1) == 4 * 4096 * 128 * 4  # 1-bit codes: 32 per word
+    assert L.mobi_codes_bytes_bits(4096, 4096, 3, 3) == 0
     assert mobi.mobi_gemm_workspace_bytes(16, 4096, 4096, 3) > 0
 
 
@@ -94,6 +96,15 @@ def test_gemm_validation(L):
     assert call(Y=p(FAKE + 4)) == 3
     assert call(wsb=16) == 4
     assert call(T=0) == 0                 # nothing to do
+
+    def call_bits(bits, T=16, K=256, N=64, S=3, G=128):
+        return L.mobi_gemm_bits(p(FAKE), T, K, p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE), N, G, S, bits, p(FAKE),
+                                p(FAKE), 1 << 30, None, 0)
+    assert call_bits(0) == 1 and call_bits(3) == 1   # code width 1 or 2
+    assert call_bits(1, K=200) == 2
+    assert call_bits(1, T=0) == 0
+    prob = mobi.GemmProblem(p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE), 4, 64, 256)
+    assert L.mobi_gemm_grouped_bits(ctypes.byref(prob), 1, 128, 3, 4, p(FAKE), 1 << 30, None) == 1
 
 
 def test_linear_validation(L):

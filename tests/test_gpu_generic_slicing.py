@@ -1,10 +1,11 @@
 """Generic slicing on the GPU: b-bit slices (b = 1, 2) over G-wide groups
 (G = 128, 256, 512) and up to four slices, against the CPU oracle.
 
-Pack: codes bit-exact; the scale/zero words bit-exact after repeating each
-G-wide group's word over its G/128 sub-groups (the layout the GEMM kernels
-read). GEMMs, routing and bucketing: the bars of the other parity tests, with
-the oracle computing at the native group width.
+Pack: codes bit-exact (1-bit codes at 32 per word); the scale/zero words
+bit-exact after repeating each G-wide group's word over its G/128 sub-groups
+(the layout the GEMM kernels read). GEMMs (decode and prefill kernels reading
+1-bit codes in their own layout), routing and bucketing: the bars of the other
+parity tests, with the oracle computing at the native group width.
 """
 import numpy as np
 import pytest
@@ -40,6 +41,7 @@ def test_pack_generic_bit_exact(mobi, oracle, bits, G, S, N, K):
     codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(DEV), S=S, G=G, bits=bits)
     torch.cuda.synchronize()
     c_ref, s_ref, q_ref = oracle.pack_bits(L.W, G=G, S=S, bits=bits)
+    assert codes.numel() * 4 == mobi.mobi_codes_bytes(N, K, S, bits=bits) == S * N * K * bits // 8
     assert np.array_equal(codes.cpu().numpy().view(np.uint32), c_ref)
     assert np.array_equal(sz.cpu().numpy().view(np.uint32), expand_sz(s_ref, G))
     assert q_ref.max() <= (1 << bits) - 1
@@ -60,7 +62,7 @@ def test_four_slice_linear(mobi, oracle, T, bits, G):
     codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(DEV), S=S, G=G, bits=bits)
     Wr = torch.from_numpy(L.Wr).to(DEV)
     b = torch.from_numpy(L.bias).to(DEV)
-    Y, k_t, perm, off = mobi.mobi_linear(L.X.to(DEV), Wr, b, codes, sz, N)
+    Y, k_t, perm, off = mobi.mobi_linear(L.X.to(DEV), Wr, b, codes, sz, N, bits=bits)
     mobi.mobi_sync_check()
     tag = f"S=4 b={bits} G={G} T={T}"
     k_gpu = k_t.cpu().numpy()
@@ -69,21 +71,66 @@ def test_four_slice_linear(mobi, oracle, T, bits, G):
     perm_ref, off_ref = oracle.bucket(k_gpu, S)
     assert np.array_equal(perm.cpu().numpy(), perm_ref) and np.array_equal(off.cpu().numpy(), off_ref)
     c_ref, s_ref, _ = oracle.pack_bits(L.W, G=G, S=S, bits=bits)
-    check_gemm(Y.cpu().numpy(), oracle.gemm(L.X, k_gpu, c_ref, s_ref, N, G=G, S=S), tag)
+    check_gemm(Y.cpu().numpy(), oracle.gemm(L.X, k_gpu, c_ref, s_ref, N, G=G, S=S, bits=bits), tag)
     if T > 1:
         assert len(set(k_gpu.tolist())) > 1, "the mix should use several precisions"
 
 
+@pytest.mark.parametrize("T", [1, 5, 8, 9, 16, 17, 130])
+@pytest.mark.parametrize("S", [1, 3])
+def test_one_bit_gemm_both_kernels(mobi, oracle, T, S):
+    """1-bit slices through both kernels with an explicit path: K = 1152 ends in
+    a ragged 1024-column chunk (decode) and N = 208 in a partial 128-row tile
+    (prefill); k_t drawn over 1..S."""
+    N, K = 208, 1152
+    L = wl.layer("b1", N, K, T, seed=2400 + T + 10 * S, outlier_frac_cols=0.01)
+    codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(DEV), S=S, bits=1)
+    c_ref, s_ref, _ = oracle.pack_bits(L.W, G=128, S=S, bits=1)
+    assert np.array_equal(codes.cpu().numpy().view(np.uint32), c_ref)
+    k = np.random.default_rng(T + S).integers(1, S + 1, T).astype(np.int32)
+    perm_np, off_np = oracle.bucket(k, S)
+    ref = oracle.gemm(L.X, k, c_ref, s_ref, N, S=S, bits=1)
+    paths = [1, 2] if T <= 16 else [2]
+    for path in paths:
+        Y = mobi.mobi_gemm_path(L.X.to(DEV), torch.from_numpy(k).to(DEV), torch.from_numpy(perm_np).to(DEV),
+                                torch.from_numpy(off_np).to(DEV), codes, sz, N, path=path, bits=1)
+        mobi.mobi_sync_check()
+        check_gemm(Y.cpu().numpy(), ref, f"1-bit S={S} T={T} path={path}")
+
+
+def test_one_bit_grouped_decode(mobi, oracle):
+    """A grouped decode step of 4-slice 1-bit layers (both fragment classes):
+    the grouped results equal single calls bit for bit and meet the oracle."""
+    S = 4
+    specs = [(256, 1024, 3), (512, 2048, 16), (128, 512, 8), (4096, 4096, 4)]
+    probs, layers = [], []
+    for i, (N, K, T) in enumerate(specs):
+        L = _layer_s("g1", N, K, T, S, seed=2250 + i)
+        codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(DEV), S=S, bits=1)
+        layers.append(L)
+        probs.append({"X": L.X.to(DEV), "Wr": torch.from_numpy(L.Wr).to(DEV), "bias": torch.from_numpy(L.bias).to(DEV),
+                      "codes": codes, "sz": sz, "N": N})
+    outs = mobi.mobi_linear_grouped(probs, S=S, bits=1)
+    mobi.mobi_sync_check()
+    for pr, L, (Y, k_t, perm, off) in zip(probs, layers, outs):
+        Ys, ks, _, _ = mobi.mobi_linear(pr["X"], pr["Wr"], pr["bias"], pr["codes"], pr["sz"], pr["N"], bits=1)
+        mobi.mobi_sync_check()
+        assert torch.equal(Y, Ys) and torch.equal(k_t, ks)
+        c_ref, s_ref, _ = oracle.pack_bits(L.W, G=128, S=S, bits=1)
+        check_gemm(Y.cpu().numpy(), oracle.gemm(L.X, k_t.cpu().numpy(), c_ref, s_ref, pr["N"], S=S, bits=1),
+                   f"grouped 1-bit N={pr['N']} T={L.T}")
+
+
 def test_four_slice_grouped_and_checkpoint(mobi, oracle, tmp_path):
-    """Grouped decode step and a checkpoint of 4-slice layers: the grouped
-    results equal single calls, and a checkpoint loaded at 2 slices serves
-    tokens routed to at most 2 slices exactly like the full pack."""
+    """Grouped decode step and a checkpoint of 4-slice (2-bit) layers: the
+    grouped results equal single calls, and a checkpoint loaded at 2 slices
+    serves tokens routed to at most 2 slices exactly like the full pack."""
     S = 4
     specs = [(256, 1024, 3), (512, 2048, 16), (128, 512, 8)]
     probs, layers = [], []
     for i, (N, K, T) in enumerate(specs):
         L = _layer_s("g4", N, K, T, S, seed=2200 + i)
-        codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(DEV), S=S, bits=1)
+        codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(DEV), S=S, bits=2)
         layers.append(L)
         probs.append({"X": L.X.to(DEV), "Wr": torch.from_numpy(L.Wr).to(DEV), "bias": torch.from_numpy(L.bias).to(DEV),
                       "codes": codes, "sz": sz, "N": N})

@@ -75,7 +75,8 @@ EXPORTED_SYMBOLS = (
     "mobi_route_mlp", "mobi_route_mlp_workspace_bytes", "mobi_linear_grouped", "mobi_linear_grouped_workspace_bytes",
     "mobi_gemm_grouped", "mobi_gemm_grouped_workspace_bytes",
     "mobi_ckpt_save", "mobi_ckpt_open", "mobi_ckpt_count", "mobi_ckpt_find", "mobi_ckpt_info", "mobi_ckpt_load",
-    "mobi_ckpt_bytes_read", "mobi_ckpt_close", "mobi_crc32c", "mobi_pack_bits",
+    "mobi_ckpt_bytes_read", "mobi_ckpt_close", "mobi_crc32c", "mobi_pack_bits", "mobi_codes_bytes_bits",
+    "mobi_gemm_bits", "mobi_gemm_grouped_bits", "mobi_linear_bits", "mobi_linear_grouped_bits",
 )
 
 
@@ -106,6 +107,8 @@ def lib() -> ctypes.CDLL:
         L.mobi_version.restype = ci
         L.mobi_codes_bytes.argtypes = [i64, i64, ci]
         L.mobi_codes_bytes.restype = sz_t
+        L.mobi_codes_bytes_bits.argtypes = [i64, i64, ci, ci]
+        L.mobi_codes_bytes_bits.restype = sz_t
         L.mobi_sz_bytes.argtypes = [i64, i64, ci, ci]
         L.mobi_sz_bytes.restype = sz_t
         L.mobi_route_workspace_bytes.argtypes = [i64, i64, ci]
@@ -122,12 +125,16 @@ def lib() -> ctypes.CDLL:
         L.mobi_gemm.restype = ci
         L.mobi_gemm_path.argtypes = [p, i64, i64, p, p, p, p, p, i64, ci, ci, p, p, sz_t, p, ci]
         L.mobi_gemm_path.restype = ci
+        L.mobi_gemm_bits.argtypes = [p, i64, i64, p, p, p, p, p, i64, ci, ci, ci, p, p, sz_t, p, ci]
+        L.mobi_gemm_bits.restype = ci
         L.mobi_gemm_decode_noalloc.argtypes = [p, i64, i64, p, p, p, i64, ci, ci, p, p]
         L.mobi_gemm_decode_noalloc.restype = ci
         L.mobi_linear_workspace_bytes.argtypes = [i64, i64, i64, ci]
         L.mobi_linear_workspace_bytes.restype = sz_t
         L.mobi_linear.argtypes = [p, i64, i64, p, p, p, p, i64, ci, ci, p, p, p, p, p, sz_t, p]
         L.mobi_linear.restype = ci
+        L.mobi_linear_bits.argtypes = [p, i64, i64, p, p, p, p, i64, ci, ci, ci, p, p, p, p, p, sz_t, p]
+        L.mobi_linear_bits.restype = ci
         L.mobi_route_mlp_workspace_bytes.argtypes = [i64, i64, i64]
         L.mobi_route_mlp_workspace_bytes.restype = sz_t
         L.mobi_route_mlp.argtypes = [p, i64, i64, p, p, i64, p, p, ci, ctypes.c_double, ctypes.c_double, p, p, p,
@@ -137,10 +144,14 @@ def lib() -> ctypes.CDLL:
         L.mobi_linear_grouped_workspace_bytes.restype = sz_t
         L.mobi_linear_grouped.argtypes = [p, ci, ci, ci, p, sz_t, p]
         L.mobi_linear_grouped.restype = ci
+        L.mobi_linear_grouped_bits.argtypes = [p, ci, ci, ci, ci, p, sz_t, p]
+        L.mobi_linear_grouped_bits.restype = ci
         L.mobi_gemm_grouped_workspace_bytes.argtypes = [p, ci, ci]
         L.mobi_gemm_grouped_workspace_bytes.restype = sz_t
         L.mobi_gemm_grouped.argtypes = [p, ci, ci, ci, p, sz_t, p]
         L.mobi_gemm_grouped.restype = ci
+        L.mobi_gemm_grouped_bits.argtypes = [p, ci, ci, ci, ci, p, sz_t, p]
+        L.mobi_gemm_grouped_bits.restype = ci
         L.mobi_ckpt_save.argtypes = [ctypes.c_char_p, p, ci, ci, p]
         L.mobi_ckpt_save.restype = ci
         L.mobi_ckpt_open.argtypes = [ctypes.c_char_p, ctypes.POINTER(p)]
@@ -201,8 +212,8 @@ def mobi_last_error() -> str:
     return lib().mobi_last_error().decode(errors="replace")
 
 
-def mobi_codes_bytes(N: int, K: int, S: int = 3) -> int:
-    return lib().mobi_codes_bytes(N, K, S)
+def mobi_codes_bytes(N: int, K: int, S: int = 3, bits: int = 2) -> int:
+    return lib().mobi_codes_bytes_bits(N, K, S, bits)
 
 
 def mobi_sz_bytes(N: int, K: int, S: int = 3, G: int = 128) -> int:
@@ -225,14 +236,15 @@ def _workspace(nbytes: int, device, ws: torch.Tensor | None) -> torch.Tensor:
 
 def mobi_pack(W: torch.Tensor, S: int = 3, G: int = 128, codes: torch.Tensor | None = None,
               sz: torch.Tensor | None = None, stream=None, bits: int = 2):
-    """MoBiSlice packing of fp16 W[N,K] -> (codes int32 [S,N,K/16], sz int32 [S,K/128,N]).
+    """MoBiSlice packing of fp16 W[N,K] -> (codes int32 [S,N,K*bits/32], sz int32 [S,K/128,N]).
     bits = 2 and G = 128 is the method's slicing (mobi_pack); other values go
-    through mobi_pack_bits (bits 1 or 2, G 128/256/512, S up to 4)."""
+    through mobi_pack_bits (bits 1 or 2, G 128/256/512, S up to 4; 1-bit codes
+    at 32 per word)."""
     if W.dtype != torch.float16 or W.dim() != 2:
         raise ValueError("W must be a 2-D fp16 tensor")
     N, K = W.shape
     if codes is None:
-        codes = torch.empty((S, N, K // 16), dtype=torch.int32, device=W.device)
+        codes = torch.empty((S, N, K * bits // 32), dtype=torch.int32, device=W.device)
     if sz is None:
         sz = torch.empty((S, K // 128, N), dtype=torch.int32, device=W.device)
     if bits == 2 and G == 128:
@@ -320,17 +332,18 @@ def mobi_linear_grouped_workspace_bytes(problems, S: int = 3) -> int:
     return lib().mobi_linear_grouped_workspace_bytes(arr, len(problems), S)
 
 
-def mobi_linear_grouped(problems, S: int = 3, G: int = 128, ws: torch.Tensor | None = None, stream=None):
+def mobi_linear_grouped(problems, S: int = 3, G: int = 128, ws: torch.Tensor | None = None, stream=None,
+                        bits: int = 2):
     """Up to MAX_GROUP independent decode-sized (T <= 16) mobi_linear problems in one step.
-    Each problem is a dict with X, Wr, codes, sz, N (and optionally bias, Y, k_t, perm, offsets).
-    Returns [(Y, k_t, perm, offsets)] in problem order."""
+    Each problem is a dict with X, Wr, codes, sz, N (and optionally bias, Y, k_t, perm, offsets);
+    `bits` is the code width of every slice. Returns [(Y, k_t, perm, offsets)] in problem order."""
     arr, filled = _problem_array(problems, S)
     if len(filled) == 0:
         raise ValueError("mobi_linear_grouped needs at least one problem")
     need = lib().mobi_linear_grouped_workspace_bytes(arr, len(filled), S)
     ws = _workspace(need, filled[0]["X"].device, ws) if need > 0 else ws
-    _check("mobi_linear_grouped", lib().mobi_linear_grouped(arr, len(filled), G, S, _ptr(ws),
-                                                            0 if ws is None else ws.numel(), _stream(stream)))
+    _check("mobi_linear_grouped", lib().mobi_linear_grouped_bits(arr, len(filled), G, S, bits, _ptr(ws),
+                                                                 0 if ws is None else ws.numel(), _stream(stream)))
     return [(d["Y"], d["k_t"], d["perm"], d["offsets"]) for d in filled]
 
 
@@ -353,16 +366,18 @@ def mobi_gemm_grouped_workspace_bytes(problems, S: int = 3) -> int:
     return lib().mobi_gemm_grouped_workspace_bytes(arr, len(problems), S)
 
 
-def mobi_gemm_grouped(problems, S: int = 3, G: int = 128, ws: torch.Tensor | None = None, stream=None):
+def mobi_gemm_grouped(problems, S: int = 3, G: int = 128, ws: torch.Tensor | None = None, stream=None,
+                      bits: int = 2):
     """Up to MAX_GROUP decode-sized mobi_gemm problems (dicts with X, k_t, codes, sz, N and
-    optionally Y) in one launch per fragment class. Returns [Y] in problem order."""
+    optionally Y) in one launch per fragment class; `bits` is the code width of every
+    slice (mobi_gemm_grouped_bits). Returns [Y] in problem order."""
     arr, filled = _gemm_problem_array(problems)
     if len(filled) == 0:
         raise ValueError("mobi_gemm_grouped needs at least one problem")
     need = lib().mobi_gemm_grouped_workspace_bytes(arr, len(filled), S)
     ws = _workspace(need, filled[0]["X"].device, ws) if need > 0 else ws
-    _check("mobi_gemm_grouped", lib().mobi_gemm_grouped(arr, len(filled), G, S, _ptr(ws),
-                                                        0 if ws is None else ws.numel(), _stream(stream)))
+    _check("mobi_gemm_grouped", lib().mobi_gemm_grouped_bits(arr, len(filled), G, S, bits, _ptr(ws),
+                                                             0 if ws is None else ws.numel(), _stream(stream)))
     return [d["Y"] for d in filled]
 
 
@@ -478,21 +493,23 @@ class MobiCheckpoint:
 
 def mobi_gemm_path(X: torch.Tensor, k_t: torch.Tensor, perm: torch.Tensor, offsets: torch.Tensor,
                    codes: torch.Tensor, sz: torch.Tensor, N: int, path: int = PATH_AUTO, S: int | None = None,
-                   G: int = 128, Y: torch.Tensor | None = None, ws: torch.Tensor | None = None, stream=None):
-    """Token-routed mixed-bit GEMM y_t = x_t . W^(k_t)^T (fp32) with an explicit kernel choice."""
+                   G: int = 128, Y: torch.Tensor | None = None, ws: torch.Tensor | None = None, stream=None,
+                   bits: int = 2):
+    """Token-routed mixed-bit GEMM y_t = x_t . W^(k_t)^T (fp32) with an explicit kernel choice
+    and the code width of the slices (mobi_gemm_bits)."""
     T, K = X.shape
     S = codes.shape[0] if S is None else S
     Y = torch.empty((T, N), dtype=torch.float32, device=X.device) if Y is None else Y
     ws = _workspace(mobi_gemm_workspace_bytes(T, N, K, S), X.device, ws)
-    _check("mobi_gemm", lib().mobi_gemm_path(_ptr(X), T, K, _ptr(k_t), _ptr(perm), _ptr(offsets), _ptr(codes),
-                                             _ptr(sz), N, G, S, _ptr(Y), _ptr(ws), ws.numel(), _stream(stream),
-                                             path))
+    _check("mobi_gemm", lib().mobi_gemm_bits(_ptr(X), T, K, _ptr(k_t), _ptr(perm), _ptr(offsets), _ptr(codes),
+                                             _ptr(sz), N, G, S, bits, _ptr(Y), _ptr(ws), ws.numel(),
+                                             _stream(stream), path))
     return Y
 
 
-def mobi_gemm(X, k_t, perm, offsets, codes, sz, N, S=None, G=128, Y=None, ws=None, stream=None):
+def mobi_gemm(X, k_t, perm, offsets, codes, sz, N, S=None, G=128, Y=None, ws=None, stream=None, bits=2):
     """Token-routed mixed-bit GEMM (decode kernel for T <= 16, tcgen05 prefill kernel above)."""
-    return mobi_gemm_path(X, k_t, perm, offsets, codes, sz, N, PATH_AUTO, S, G, Y, ws, stream)
+    return mobi_gemm_path(X, k_t, perm, offsets, codes, sz, N, PATH_AUTO, S, G, Y, ws, stream, bits)
 
 
 def mobi_gemm_decode_noalloc(X, k_t, codes, sz, N, S=None, G=128, Y=None, stream=None):
@@ -509,8 +526,10 @@ def mobi_linear_workspace_bytes(T: int, N: int, K: int, S: int = 3) -> int:
     return lib().mobi_linear_workspace_bytes(T, N, K, S)
 
 
-def mobi_linear(X, Wr, bias, codes, sz, N, G=128, Y=None, k_t=None, perm=None, offsets=None, ws=None, stream=None):
-    """Route + mixed-bit GEMM in one call (S = Wr.shape[1]) -> (Y fp32 [T,N], k_t, perm, offsets)."""
+def mobi_linear(X, Wr, bias, codes, sz, N, G=128, Y=None, k_t=None, perm=None, offsets=None, ws=None, stream=None,
+                bits=2):
+    """Route + mixed-bit GEMM in one call (S = Wr.shape[1], slices of `bits`-bit codes)
+    -> (Y fp32 [T,N], k_t, perm, offsets)."""
     if X.dtype != torch.bfloat16 or Wr.dtype != torch.float32:
         raise ValueError("X must be bf16 and Wr fp32")
     T, K = X.shape
@@ -521,9 +540,9 @@ def mobi_linear(X, Wr, bias, codes, sz, N, G=128, Y=None, k_t=None, perm=None, o
     perm = torch.empty(T, dtype=torch.int32, device=dev) if perm is None else perm
     offsets = torch.empty(S + 1, dtype=torch.int32, device=dev) if offsets is None else offsets
     ws = _workspace(mobi_linear_workspace_bytes(T, N, K, S), dev, ws)
-    _check("mobi_linear", lib().mobi_linear(_ptr(X), T, K, _ptr(Wr), _ptr(bias), _ptr(codes), _ptr(sz), N, G, S,
-                                            _ptr(k_t), _ptr(perm), _ptr(offsets), _ptr(Y), _ptr(ws), ws.numel(),
-                                            _stream(stream)))
+    _check("mobi_linear", lib().mobi_linear_bits(_ptr(X), T, K, _ptr(Wr), _ptr(bias), _ptr(codes), _ptr(sz), N, G,
+                                                 S, bits, _ptr(k_t), _ptr(perm), _ptr(offsets), _ptr(Y), _ptr(ws),
+                                                 ws.numel(), _stream(stream)))
     return Y, k_t, perm, offsets
 
 

@@ -29,11 +29,11 @@ cudaError_t launch_route_mlp(const void* X, int64_t T, int64_t K, const float* W
 size_t route_mlp_ws_bytes(int64_t T, int64_t K, int64_t H, int sms);
 cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
                           const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
-                          DeviceStatus* st, bool early);
+                          DeviceStatus* st, bool early, int bits);
 size_t decode_ws_bytes(int64_t N, int64_t K);
 cudaError_t launch_prefill(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
                            const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int S,
-                           float* Y, void* ws, cudaStream_t stream, DeviceStatus* st);
+                           float* Y, void* ws, cudaStream_t stream, DeviceStatus* st, int bits);
 size_t prefill_ws_bytes(int64_t T, int64_t N, int64_t K);
 
 static thread_local char g_last_error[256];
@@ -266,9 +266,11 @@ const char* mobi_last_error(void) { return g_last_error; }
 
 int mobi_version(void) { return 100; }
 
-size_t mobi_codes_bytes(int64_t N, int64_t K, int S) {
-  if (N < 0 || K < 0 || K % 16 != 0 || S < 1 || S > kMaxSlices) return 0;
-  return (size_t)S * (size_t)N * (size_t)(K / 16) * 4;
+size_t mobi_codes_bytes(int64_t N, int64_t K, int S) { return mobi_codes_bytes_bits(N, K, S, 2); }
+
+size_t mobi_codes_bytes_bits(int64_t N, int64_t K, int S, int bits) {
+  if (N < 0 || K < 0 || K % 32 != 0 || S < 1 || S > kMaxSlices || bits < 1 || bits > 2) return 0;
+  return (size_t)S * (size_t)N * (size_t)(K / 32 * bits) * 4;
 }
 
 size_t mobi_sz_bytes(int64_t N, int64_t K, int S, int G) {
@@ -362,7 +364,14 @@ mobi_status mobi_route_mlp(const void* X, int64_t T, int64_t K, const float* W1,
 mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
                            const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int G,
                            int S, float* Y, void* ws, size_t ws_bytes, void* stream, int path) {
+  return mobi_gemm_bits(X, T, K, k_t, perm, offsets, codes, sz, N, G, S, 2, Y, ws, ws_bytes, stream, path);
+}
+
+mobi_status mobi_gemm_bits(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
+                           const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int G,
+                           int S, int bits, float* Y, void* ws, size_t ws_bytes, void* stream, int path) {
   g_last_error[0] = 0;
+  if (bits < 1 || bits > 2) return MOBI_ERR_INVALID_ARG;
   mobi_status st = check_matrix(N, K, G, S);
   if (st != MOBI_OK) return st;
   if (T < 0) return MOBI_ERR_INVALID_ARG;
@@ -382,8 +391,8 @@ mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const int32_t* k
   DeviceStatus* dst = device_status(&e);
   if (!dst) return cuda_status(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (decode) return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, ws, s, dst, false));
-  return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, ws, s, dst));
+  if (decode) return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, ws, s, dst, false, bits));
+  return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, ws, s, dst, bits));
 }
 
 size_t mobi_linear_workspace_bytes(int64_t T, int64_t N, int64_t K, int S) {
@@ -394,7 +403,15 @@ size_t mobi_linear_workspace_bytes(int64_t T, int64_t N, int64_t K, int S) {
 mobi_status mobi_linear(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
                         const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S, int32_t* k_t,
                         int32_t* perm, int32_t* offsets, float* Y, void* ws, size_t ws_bytes, void* stream) {
+  return mobi_linear_bits(X, T, K, Wr, bias, codes, sz, N, G, S, 2, k_t, perm, offsets, Y, ws, ws_bytes, stream);
+}
+
+mobi_status mobi_linear_bits(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
+                             const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S, int bits,
+                             int32_t* k_t, int32_t* perm, int32_t* offsets, float* Y, void* ws, size_t ws_bytes,
+                             void* stream) {
   g_last_error[0] = 0;
+  if (bits < 1 || bits > 2) return MOBI_ERR_INVALID_ARG;
   mobi_status st = check_matrix(N, K, G, S);
   if (st != MOBI_OK) return st;
   if (T < 0) return MOBI_ERR_INVALID_ARG;
@@ -420,8 +437,8 @@ mobi_status mobi_linear(const void* X, int64_t T, int64_t K, const float* Wr, co
   // For up to 16 tokens the kernel just launched is the routing kernel, which
   // writes only k_t, perm and offsets: the decode kernel may fetch X and the
   // weights before it waits on it.
-  if (decode) return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, gws, s, dst, true));
-  return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, gws, s, dst));
+  if (decode) return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, gws, s, dst, true, bits));
+  return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, gws, s, dst, bits));
 }
 
 static_assert(MOBI_MAX_GROUP == kMaxGroup, "group size of the header and the kernels");
@@ -455,7 +472,13 @@ size_t mobi_linear_grouped_workspace_bytes(const mobi_linear_problem* problems, 
 
 mobi_status mobi_linear_grouped(const mobi_linear_problem* problems, int count, int G, int S, void* ws,
                                 size_t ws_bytes, void* stream) {
+  return mobi_linear_grouped_bits(problems, count, G, S, 2, ws, ws_bytes, stream);
+}
+
+mobi_status mobi_linear_grouped_bits(const mobi_linear_problem* problems, int count, int G, int S, int bits,
+                                     void* ws, size_t ws_bytes, void* stream) {
   g_last_error[0] = 0;
+  if (bits < 1 || bits > 2) return MOBI_ERR_INVALID_ARG;
   size_t need = 0;
   mobi_status st = check_grouped(problems, count, G, S, &need);
   if (st != MOBI_OK) return st;
@@ -473,7 +496,7 @@ mobi_status mobi_linear_grouped(const mobi_linear_problem* problems, int count, 
     const mobi_linear_problem& p = problems[i];
     rg.p[i] = RouteSmallProblem{static_cast<const __nv_bfloat16*>(p.X), p.Wr, p.bias, p.k_t, p.perm, p.offsets, p.K,
                                 (int)p.T};
-    jobs[i] = DecodeJob{p.X, p.k_t, p.codes, p.sz, p.Y, nullptr, p.N, p.K, (int)p.T};
+    jobs[i] = DecodeJob{p.X, p.k_t, p.codes, p.sz, p.Y, nullptr, p.N, p.K, (int)p.T, bits};
     if (p.T > 0 && p.N > 0) {
       jobs[i].partial = reinterpret_cast<float*>(w);
       w += align256(decode_ws_bytes(p.N, p.K));
@@ -514,7 +537,13 @@ size_t mobi_gemm_grouped_workspace_bytes(const mobi_gemm_problem* problems, int 
 
 mobi_status mobi_gemm_grouped(const mobi_gemm_problem* problems, int count, int G, int S, void* ws,
                               size_t ws_bytes, void* stream) {
+  return mobi_gemm_grouped_bits(problems, count, G, S, 2, ws, ws_bytes, stream);
+}
+
+mobi_status mobi_gemm_grouped_bits(const mobi_gemm_problem* problems, int count, int G, int S, int bits, void* ws,
+                                   size_t ws_bytes, void* stream) {
   g_last_error[0] = 0;
+  if (bits < 1 || bits > 2) return MOBI_ERR_INVALID_ARG;
   size_t need = 0;
   mobi_status st = check_gemm_grouped(problems, count, G, S, &need);
   if (st != MOBI_OK) return st;
@@ -527,7 +556,7 @@ mobi_status mobi_gemm_grouped(const mobi_gemm_problem* problems, int count, int 
   uint8_t* w = static_cast<uint8_t*>(ws);
   for (int i = 0; i < count; ++i) {
     const mobi_gemm_problem& p = problems[i];
-    jobs[i] = DecodeJob{p.X, p.k_t, p.codes, p.sz, p.Y, nullptr, p.N, p.K, (int)p.T};
+    jobs[i] = DecodeJob{p.X, p.k_t, p.codes, p.sz, p.Y, nullptr, p.N, p.K, (int)p.T, bits};
     if (p.T > 0 && p.N > 0) {
       jobs[i].partial = reinterpret_cast<float*>(w);
       w += align256(decode_ws_bytes(p.N, p.K));

@@ -106,14 +106,16 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r
 }
 
 // Issue one stage: the codes of 16-row tile `tile`, slice s, chunk `chunk`
-// (x = word column, y = s N + row) and its scale/zero words.
+// (x = word column, y = s N + row) and its scale/zero words. 2-bit codes fill
+// two 2 KB halves (64 words per row and chunk), 1-bit codes one (32 words).
+template <int BITS>
 __device__ __forceinline__ void dec_issue(const CUtensorMap* tm_codes, const CUtensorMap* tm_sz, uint8_t* codes,
                                           uint8_t* sz, uint64_t* bar, int tile, int s, int N, int ngroups,
                                           int chunk, uint64_t policy) {
-  mbar_arrive_expect_tx(bar, kDecCodes + kDecSz);
+  mbar_arrive_expect_tx(bar, kDecHalf * BITS + kDecSz);
   const int y = s * N + tile * kDecRows;
-  tma_load_2d_hint(codes, tm_codes, chunk * kDecChunk * 8, y, bar, policy);
-  tma_load_2d_hint(codes + kDecHalf, tm_codes, chunk * kDecChunk * 8 + 32, y, bar, policy);
+  tma_load_2d_hint(codes, tm_codes, chunk * kDecChunk * 4 * BITS, y, bar, policy);
+  if (BITS == 2) tma_load_2d_hint(codes + kDecHalf, tm_codes, chunk * kDecChunk * 8 + 32, y, bar, policy);
   tma_load_2d_hint(sz, tm_sz, tile * kDecRows, s * ngroups + chunk * kDecChunk, bar, policy);
 }
 
@@ -238,7 +240,7 @@ __device__ __forceinline__ void dec_write_tile(float* o, int T, int N, int gid, 
 
 // All loop bookkeeping is 32-bit arithmetic (sizes are validated to N, K <
 // 2^28); positions in the cost sequence are 64-bit.
-template <int NB, int MG>
+template <int NB, int MG, int BITS>
 __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
     const __grid_constant__ DecGroup<MG> grp, DeviceStatus* st, uint64_t limit) {
   using L = DecLayout<NB>;
@@ -308,13 +310,18 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
   const float* const xs_sm = reinterpret_cast<const float*>(sm + L::kXs);
   const uint32_t bimg = smem_addr(sm + L::kBimg) + (uint32_t)lane * 16;
 
-  // Code words 2 t4, 2 t4 + 1 of group g for row r of the tile: half g / 4,
-  // 16-byte chunk 2 (g % 4) + t4 / 2 stored at chunk ^ (r % 8), rows 128 bytes.
+  // 2-bit codes: words 2 t4, 2 t4 + 1 of group g for row r of the tile: half
+  // g / 4, 16-byte chunk 2 (g % 4) + t4 / 2 stored at chunk ^ (r % 8), rows
+  // 128 bytes. 1-bit codes: word t4 of group g, 16-byte chunk g stored at
+  // g ^ (r % 8); its even bits are the codes of 2-bit word 2 t4 and its odd
+  // bits those of word 2 t4 + 1, so (w, w >> 1) take the place of that pair.
   uint32_t coff[kDecChunk];
 #pragma unroll
   for (int g = 0; g < kDecChunk; ++g)
-    coff[g] = (uint32_t)(g >> 2) * kDecHalf + (uint32_t)gid * 128u +
-              (uint32_t)((((g & 3) * 2 + (t4 >> 1)) ^ gid) * 16) + (t4 & 1) * 8u;
+    coff[g] = BITS == 2 ? (uint32_t)(g >> 2) * kDecHalf + (uint32_t)gid * 128u +
+                              (uint32_t)((((g & 3) * 2 + (t4 >> 1)) ^ gid) * 16) + (t4 & 1) * 8u
+                        : (uint32_t)gid * 128u + (uint32_t)((g ^ gid) * 16) + (uint32_t)t4 * 4u;
+  constexpr uint32_t kFieldMask = BITS == 2 ? 0x00030003u : 0x00010001u;
 
   bool ok = true;
   uint32_t issued = 0, done = 0;  // stages this warp has issued / consumed (ring slot = count % D)
@@ -376,7 +383,7 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
           for (int k = 0; k < nramp; ++k) {
             const uint32_t slot = (issued + k) % D;
             const int jj = a + k;
-            dec_issue(&grp.tm_codes[p], &grp.tm_sz[p], codes_ring + slot * kDecCodes, sz_ring + slot * kDecSz,
+            dec_issue<BITS>(&grp.tm_codes[p], &grp.tm_sz[p], codes_ring + slot * kDecCodes, sz_ring + slot * kDecSz,
                       &full[slot], b + jj / km, jj % km, pr.N, pr.ngroups, c, policy);
           }
         }
@@ -492,8 +499,8 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
       if (pj < a1) {
         const uint32_t ns = issued % D;
         if (lane == 0)
-          dec_issue(tm_codes, tm_sz, codes_ring + ns * kDecCodes, sz_ring + ns * kDecSz, &full[ns], ptile, ps, N,
-                    ngroups, c, policy);
+          dec_issue<BITS>(tm_codes, tm_sz, codes_ring + ns * kDecCodes, sz_ring + ns * kDecSz, &full[ns], ptile,
+                          ps, N, ngroups, c, policy);
         ++issued;
         ++pj;
         if (++ps == km) {
@@ -530,8 +537,15 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
         uint32_t bf[2][NB][8][2];
 #pragma unroll
         for (int gg = 0; gg < 2; ++gg) {
-          wa[gg] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg]);
-          wb[gg] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + 8 * 128);
+          if (BITS == 2) {
+            wa[gg] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg]);
+            wb[gg] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + 8 * 128);
+          } else {
+            const uint32_t x = *reinterpret_cast<const uint32_t*>(cs + coff[g0 + gg]);
+            const uint32_t y = *reinterpret_cast<const uint32_t*>(cs + coff[g0 + gg] + 8 * 128);
+            wa[gg] = make_uint2(x, x >> 1);
+            wb[gg] = make_uint2(y, y >> 1);
+          }
 #pragma unroll
           for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
@@ -543,7 +557,7 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           const int h = jj >> 2, f = jj & 3;
-          const uint32_t mk = 0x00030003u << (2 * f);
+          const uint32_t mk = kFieldMask << (2 * f);
 #pragma unroll
           for (int gg = 0; gg < 2; ++gg) {
             const uint32_t a0 = (wa[gg].x >> (8 * h)) & mk, a2 = (wa[gg].y >> (8 * h)) & mk;
@@ -668,10 +682,10 @@ size_t decode_ws_bytes(int64_t N, int64_t K) {
   return ((size_t)nch * 16 * (size_t)N * sizeof(float) + 255) / 256 * 256;  // partials for up to 16 tokens
 }
 
-template <int NB, int MG>
+template <int NB, int MG, int BITS>
 static cudaError_t launch_decode_class(const DecGroup<MG>& grp, int ctas, cudaStream_t stream, DeviceStatus* st) {
   using L = DecLayout<NB>;
-  cudaError_t e = set_smem((const void*)decode_kernel<NB, MG>, (int)L::kDynamic);
+  cudaError_t e = set_smem((const void*)decode_kernel<NB, MG, BITS>, (int)L::kDynamic);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)ctas);
@@ -683,7 +697,7 @@ static cudaError_t launch_decode_class(const DecGroup<MG>& grp, int ctas, cudaSt
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, decode_kernel<NB, MG>, grp, st, wait_limit());
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<NB, MG, BITS>, grp, st, wait_limit());
   if (e != cudaSuccess) return note_error("decode launch", e);
   return note_error("kernel launch", cudaGetLastError());
 }
@@ -692,7 +706,7 @@ static cudaError_t launch_decode_class(const DecGroup<MG>& grp, int ctas, cudaSt
 // class and launches it on one CTA per SM; the kernel itself shares the CTAs
 // among the problems once it knows their k_t. Problems with several chunks are
 // appended to `red`.
-template <int MG>
+template <int MG, int BITS>
 static cudaError_t decode_class(const DecodeJob* jobs, const int* idx, int n, int cls, int S, int sms,
                                 DecReduceGroup* red, cudaStream_t stream, DeviceStatus* st) {
   DecGroup<MG> grp;
@@ -702,8 +716,8 @@ static cudaError_t decode_class(const DecodeJob* jobs, const int* idx, int n, in
   for (int m = 0; m < n; ++m) {
     const DecodeJob& j = jobs[idx[m]];
     const int64_t nch = dec_chunks(j.K), nblocks = (j.N + kDecRows - 1) / kDecRows;
-    if (!make_tmap_2d(&grp.tm_codes[m], j.codes, 4, (uint64_t)(j.K / 16), (uint64_t)(S * j.N),
-                      (uint64_t)(j.K / 16) * 4, 32, kDecRows, 128))
+    const uint64_t words = (uint64_t)(j.K / 32 * BITS);  // per row and slice
+    if (!make_tmap_2d(&grp.tm_codes[m], j.codes, 4, words, (uint64_t)(S * j.N), words * 4, 32, kDecRows, 128))
       return note_error("decode tensor map (codes)", cudaErrorInvalidValue);
     if (!make_tmap_2d(&grp.tm_sz[m], j.sz, 4, (uint64_t)j.N, (uint64_t)(S * (j.K / 128)), (uint64_t)j.N * 4,
                       kDecRows, kDecChunk, 0))
@@ -718,8 +732,8 @@ static cudaError_t decode_class(const DecodeJob* jobs, const int* idx, int n, in
       ++red->G;
     }
   }
-  return cls == 1 ? launch_decode_class<1, MG>(grp, sms, stream, st)
-                  : launch_decode_class<2, MG>(grp, sms, stream, st);
+  return cls == 1 ? launch_decode_class<1, MG, BITS>(grp, sms, stream, st)
+                  : launch_decode_class<2, MG, BITS>(grp, sms, stream, st);
 }
 
 // One launch per fragment class present (T <= 8, then 9 <= T <= 16), each a
@@ -735,18 +749,24 @@ cudaError_t launch_decode_grouped(const DecodeJob* jobs, int G, int S, cudaStrea
   const int sms = num_sms();
   DecReduceGroup red = {};
   red.off[0] = 0;
-  for (int cls = 1; cls <= 2; ++cls) {
-    int idx[kMaxGroup];
-    int n = 0;
-    for (int i = 0; i < G; ++i) {
-      const DecodeJob& j = jobs[i];
-      if (j.T > 0 && j.N > 0 && (j.T > 8 ? 2 : 1) == cls) idx[n++] = i;
+  for (int cls = 1; cls <= 2; ++cls)
+    for (int bits = 2; bits >= 1; --bits) {
+      int idx[kMaxGroup];
+      int n = 0;
+      for (int i = 0; i < G; ++i) {
+        const DecodeJob& j = jobs[i];
+        if (j.T > 0 && j.N > 0 && (j.T > 8 ? 2 : 1) == cls && j.bits == bits) idx[n++] = i;
+      }
+      if (n == 0) continue;
+      cudaError_t e;
+      if (bits == 2)
+        e = n == 1 ? decode_class<1, 2>(jobs, idx, n, cls, S, sms, &red, stream, st)
+                   : decode_class<kMaxGroup, 2>(jobs, idx, n, cls, S, sms, &red, stream, st);
+      else
+        e = n == 1 ? decode_class<1, 1>(jobs, idx, n, cls, S, sms, &red, stream, st)
+                   : decode_class<kMaxGroup, 1>(jobs, idx, n, cls, S, sms, &red, stream, st);
+      if (e != cudaSuccess) return e;
     }
-    if (n == 0) continue;
-    const cudaError_t e = n == 1 ? decode_class<1>(jobs, idx, n, cls, S, sms, &red, stream, st)
-                                 : decode_class<kMaxGroup>(jobs, idx, n, cls, S, sms, &red, stream, st);
-    if (e != cudaSuccess) return e;
-  }
   if (red.G == 0) return cudaSuccess;
 
   // Chunk reduction, launched as a programmatic dependent of the decode kernel.
@@ -797,8 +817,8 @@ cudaError_t launch_chunk_reduce(const float* partial, float* Y, int64_t T, int64
 
 cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
                           const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
-                          DeviceStatus* st, bool early) {
-  const DecodeJob job{X, k_t, codes, sz, Y, static_cast<float*>(ws), N, K, T};
+                          DeviceStatus* st, bool early, int bits) {
+  const DecodeJob job{X, k_t, codes, sz, Y, static_cast<float*>(ws), N, K, T, bits};
   return launch_decode_grouped(&job, 1, S, stream, st, early);
 }
 
@@ -871,5 +891,5 @@ extern "C" mobi_status mobi_gemm_decode_noalloc(const void* X, int64_t T, int64_
   void* scratch = noalloc_scratch(&e);
   if (!scratch) return status_of(e);
   return status_of(
-      launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, scratch, static_cast<cudaStream_t>(stream), st, false));
+      launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, scratch, static_cast<cudaStream_t>(stream), st, false, 2));
 }

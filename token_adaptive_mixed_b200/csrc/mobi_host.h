@@ -74,6 +74,7 @@ struct DecodeJob {
   float* partial;  // scratch of decode_ws_bytes(N, K) bytes
   int64_t N, K;
   int T;
+  int bits;  // code width of every slice: 2 (16 codes per word) or 1 (32 per word)
 };
 // Decode scratch of one problem: the per-chunk partial sums when K spans more
 // than one 1024-column chunk.
@@ -82,7 +83,7 @@ size_t decode_ws_bytes(int64_t N, int64_t K);
 // launched as a programmatic dependent of the kernel before it.
 cudaError_t launch_chunk_reduce(const float* partial, float* Y, int64_t T, int64_t N, int nch, cudaStream_t stream);
 // Decode GEMMs of up to kMaxGroup problems: one launch per fragment class
-// (T <= 8, T <= 16) plus one chunk-reduction launch.
+// (T <= 8, T <= 16) and code width present, plus one chunk-reduction launch.
 cudaError_t launch_decode_grouped(const DecodeJob* jobs, int G, int S, cudaStream_t stream, DeviceStatus* st,
                                   bool early);
 

@@ -7,13 +7,15 @@
 // G = 128, 256 or 512.
 //
 // Work split: one warp per (row n, chunk of 512 columns); lane l owns the 16
-// consecutive weights k = 512c + 16l .. +15, i.e. exactly one packed word per
-// slice. The G/16 lanes of a group reduce min/max with xor shuffles. Codes of
-// either width sit in 2-bit fields and leave as 128-bit stores (4 lanes' words
-// gathered into one lane), so each slice's 128 bytes per warp are one
-// coalesced transaction. Scale/zero words are written per 128-column
-// sub-group, so a wider group's word appears once per sub-group (the layout
-// the GEMM kernels read).
+// consecutive weights k = 512c + 16l .. +15, i.e. exactly one 2-bit-field
+// word per slice. The G/16 lanes of a group reduce min/max with xor shuffles.
+// 2-bit codes leave as 128-bit stores (4 lanes' words gathered into one lane),
+// so each slice's 128 bytes per warp are one coalesced transaction. 1-bit
+// codes are stored at 1 bit per weight: lanes 2m and 2m + 1 merge their words
+// (the odd lane's codes on the odd bits) into one 32-code word, and four such
+// words leave as one 128-bit store (64 bytes per warp and slice). Scale/zero
+// words are written per 128-column sub-group, so a wider group's word appears
+// once per sub-group (the layout the GEMM kernels read).
 //
 // Bit-exactness: IEEE division (__fdiv_rn), round-to-nearest-even (rintf,
 // __float2half_rn), explicit _rn multiply/subtract so that nothing is
@@ -89,13 +91,27 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
         R[i] = __fsub_rn(R[i], __fmul_rn((float)(q - z), step));
       }
 
-      // Gather 4 consecutive lanes' words into the first of them: one uint4.
-      const uint32_t w1 = __shfl_down_sync(0xffffffffu, word, 1);
-      const uint32_t w2 = __shfl_down_sync(0xffffffffu, word, 2);
-      const uint32_t w3 = __shfl_down_sync(0xffffffffu, word, 3);
-      if (valid && (lane & 3) == 0) {
-        uint4* dst = reinterpret_cast<uint4*>(codes + ((int64_t)s * N + n) * nwords + 32 * c + lane);
-        *dst = make_uint4(word, w1, w2, w3);
+      if (bits == 1) {
+        // 32 codes per word: this lane's 16 on the even bits, the next lane's on
+        // the odd bits (valid in even lanes); lanes 8j, 8j + 2, 8j + 4, 8j + 6
+        // hold one group's four words, gathered into lane 8j: one uint4.
+        const uint32_t dense = word | (__shfl_down_sync(0xffffffffu, word, 1) << 1);
+        const uint32_t d1 = __shfl_down_sync(0xffffffffu, dense, 2);
+        const uint32_t d2 = __shfl_down_sync(0xffffffffu, dense, 4);
+        const uint32_t d3 = __shfl_down_sync(0xffffffffu, dense, 6);
+        if (valid && (lane & 7) == 0) {
+          uint4* dst = reinterpret_cast<uint4*>(codes + ((int64_t)s * N + n) * (K / 32) + 16 * c + (lane >> 1));
+          *dst = make_uint4(dense, d1, d2, d3);
+        }
+      } else {
+        // Gather 4 consecutive lanes' words into the first of them: one uint4.
+        const uint32_t w1 = __shfl_down_sync(0xffffffffu, word, 1);
+        const uint32_t w2 = __shfl_down_sync(0xffffffffu, word, 2);
+        const uint32_t w3 = __shfl_down_sync(0xffffffffu, word, 3);
+        if (valid && (lane & 3) == 0) {
+          uint4* dst = reinterpret_cast<uint4*>(codes + ((int64_t)s * N + n) * nwords + 32 * c + lane);
+          *dst = make_uint4(word, w1, w2, w3);
+        }
       }
       if (valid && (lane & 7) == 0) {
         const uint32_t zbits = (uint32_t)__half_as_ushort(__int2half_rn(z));

@@ -48,7 +48,6 @@ namespace mobi {
 
 namespace pf {
 constexpr int BM = 128;          // weight rows per tile (tcgen05 M)
-constexpr int GK = 128;          // group width along K
 constexpr int XST = 3;           // x-tile stages (one group each)
 constexpr int CST = 6;           // code/scale stages (one unit each)
 constexpr int DST = 2;           // accumulator buffers in TMEM (one unit each)
@@ -60,7 +59,7 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kDeqWarp0 = 4;
 constexpr int kEpiWarp0 = 8;
 constexpr int kEpiWarps = 8;                   // two per TMEM lane quadrant
-constexpr uint32_t kCodeBytes = BM * 32;       // 128 rows x 8 words
+constexpr uint32_t kCodeBytes = BM * 32;       // 128 rows x 8 words (2-bit codes; 4 words for 1-bit)
 constexpr uint32_t kSzBytes = BM * 4;
 constexpr uint32_t kTmemCols = 512;
 
@@ -174,7 +173,7 @@ template <int BN, bool KSPLIT>
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
     const uint8_t* __restrict__ Xt, const __grid_constant__ CUtensorMap tm_codes,
     const __grid_constant__ CUtensorMap tm_sz, const uint32_t* __restrict__ sz, const int32_t* __restrict__ perm,
-    const int32_t* __restrict__ offsets, int64_t T, int64_t N, int64_t ngroups, int S, int nkc,
+    const int32_t* __restrict__ offsets, int64_t T, int64_t N, int64_t ngroups, int S, int nkc, int bits,
     float* __restrict__ Y, DeviceStatus* st, uint64_t limit) {
   using TL = pf::Tile<BN>;
   if constexpr (!KSPLIT) nkc = 1;
@@ -234,8 +233,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
           for (int s = 0; s < ti.kmax; ++s) {
             const uint32_t cs = ci % pf::CST, cph = (ci / pf::CST) & 1;
             if (!(ok = pf_wait(&sm.c_empty[cs], cph ^ 1, limit, st, 0x302, abort_flag))) break;
-            mbar_arrive_expect_tx(&sm.c_full[cs], pf::kCodeBytes + pf::kSzBytes);
-            tma_load_2d(&sm.codes[cs][0], &tm_codes, (int)(g * 8), (int)(s * N + ti.n0), &sm.c_full[cs]);
+            mbar_arrive_expect_tx(&sm.c_full[cs], pf::kCodeBytes / 2 * bits + pf::kSzBytes);
+            tma_load_2d(&sm.codes[cs][0], &tm_codes, (int)(g * 4 * bits), (int)(s * N + ti.n0), &sm.c_full[cs]);
             tma_load_2d(&sm.sz[cs][0], &tm_sz, (int)ti.n0, (int)(s * ngroups + g), &sm.c_full[cs]);
             ++ci;
           }
@@ -316,12 +315,24 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
         for (int s = 0; s < ti.kmax && ok; ++s, ++u) {
           const uint32_t cs = u % pf::CST, cph = (u / pf::CST) & 1;
           if (!(ok = pf_wait(&sm.c_full[cs], cph, limit, st, 0x321, abort_flag))) break;
-          const uint4 w0 = *reinterpret_cast<const uint4*>(&sm.codes[cs][r * 8]);
-          const uint4 w1 = *reinterpret_cast<const uint4*>(&sm.codes[cs][r * 8 + 4]);
+          // The group's 128 codes of row r as eight 2-bit-field words: 2-bit
+          // codes as stored; 1-bit codes (4 words) as (w, w >> 1) pairs, whose
+          // even bits are the codes of the 2-bit words 2i and 2i + 1.
+          uint32_t words[8];
+          if (bits == 2) {
+            const uint4 w0 = *reinterpret_cast<const uint4*>(&sm.codes[cs][r * 8]);
+            const uint4 w1 = *reinterpret_cast<const uint4*>(&sm.codes[cs][r * 8 + 4]);
+            words[0] = w0.x; words[1] = w0.y; words[2] = w0.z; words[3] = w0.w;
+            words[4] = w1.x; words[5] = w1.y; words[6] = w1.z; words[7] = w1.w;
+          } else {
+            const uint4 w0 = *reinterpret_cast<const uint4*>(&sm.codes[cs][r * 4]);
+            words[0] = w0.x; words[1] = w0.x >> 1; words[2] = w0.y; words[3] = w0.y >> 1;
+            words[4] = w0.z; words[5] = w0.z >> 1; words[6] = w0.w; words[7] = w0.w >> 1;
+          }
+          const uint32_t fmask = bits == 2 ? 0x00030003u : 0x00010001u;
           const uint32_t zsz = sm.sz[cs][r];
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.c_empty[cs]);
-          const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
           // FMA constants: v * 4^-f - (128 / 4^f + z) = q - z for the field at bit 2f.
           const float zf = __half2float(__ushort_as_half((unsigned short)(zsz >> 16)));
           __nv_bfloat162 mul[3], add[3];
@@ -352,7 +363,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
                 for (int c = 0; c < 8; ++c) {
                   // pair (c, c+8): field f = c % 3 of the word shifted by 6 * (c / 3)
                   const int f = c % 3, sh = 6 * (c / 3);
-                  const uint32_t v = ((w >> sh) & (0x00030003u << (2 * f))) | 0x43004300u;
+                  const uint32_t v = ((w >> sh) & (fmask << (2 * f))) | 0x43004300u;
                   __nv_bfloat162 p = __hfma2(*reinterpret_cast<const __nv_bfloat162*>(&v), mul[f], add[f]);
                   regs[8 * ww + c] = *reinterpret_cast<uint32_t*>(&p);
                 }
@@ -548,7 +559,7 @@ size_t prefill_ws_bytes(int64_t T, int64_t N, int64_t K) {
 template <int BN, bool KSPLIT>
 static cudaError_t launch_prefill_bn(const PfPlan& plan, const void* X, int64_t T, int64_t K, const int32_t* perm,
                                      const int32_t* offsets, const CUtensorMap& tm_codes, const CUtensorMap& tm_sz,
-                                     const uint32_t* sz, int64_t N, int S, float* out, uint8_t* Xt,
+                                     const uint32_t* sz, int64_t N, int S, int bits, float* out, uint8_t* Xt,
                                      cudaStream_t stream, DeviceStatus* st) {
   const int64_t ngroups = K / 128;
   const int64_t blocks_g = (plan.T_pad * (K / 16) + 255) / 256;
@@ -561,7 +572,7 @@ static cudaError_t launch_prefill_bn(const PfPlan& plan, const void* X, int64_t 
   cudaError_t e = set_smem((const void*)kernel, (int)smem);
   if (e != cudaSuccess) return e;
   kernel<<<grid, pf::kThreads, smem, stream>>>(Xt, tm_codes, tm_sz, sz, perm, offsets, T, N, ngroups, S, plan.nkc,
-                                               out, st, wait_limit());
+                                               bits, out, st, wait_limit());
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     cudaFuncAttributes fa{};
@@ -576,7 +587,7 @@ static cudaError_t launch_prefill_bn(const PfPlan& plan, const void* X, int64_t 
 
 cudaError_t launch_prefill(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
                            const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int S,
-                           float* Y, void* ws, cudaStream_t stream, DeviceStatus* st) {
+                           float* Y, void* ws, cudaStream_t stream, DeviceStatus* st, int bits) {
   (void)k_t;
   const int64_t ngroups = K / 128;
   const PfPlan plan = pf_plan(T, N, K, num_sms());
@@ -584,18 +595,18 @@ cudaError_t launch_prefill(const void* X, int64_t T, int64_t K, const int32_t* k
   float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + plan.xt_bytes);
   float* out = plan.nkc > 1 ? partial : Y;
   CUtensorMap tm_codes, tm_sz;
-  if (!make_tmap_2d(&tm_codes, codes, 4, (uint64_t)(K / 16), (uint64_t)(S * N), (uint64_t)(K / 16) * 4, 8, pf::BM,
-                    0))
+  const uint64_t words = (uint64_t)(K / 32 * bits);  // per row and slice
+  if (!make_tmap_2d(&tm_codes, codes, 4, words, (uint64_t)(S * N), words * 4, (uint32_t)(4 * bits), pf::BM, 0))
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, pf::BM, 1, 0))
     return cudaErrorInvalidValue;
   cudaError_t e;
   if (plan.bn == 64)
-    e = launch_prefill_bn<64, true>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, out, Xt, stream, st);
+    e = launch_prefill_bn<64, true>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, bits, out, Xt, stream, st);
   else if (plan.nkc > 1)
-    e = launch_prefill_bn<192, true>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, out, Xt, stream, st);
+    e = launch_prefill_bn<192, true>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, bits, out, Xt, stream, st);
   else
-    e = launch_prefill_bn<192, false>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, out, Xt, stream, st);
+    e = launch_prefill_bn<192, false>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, bits, out, Xt, stream, st);
   if (e != cudaSuccess || plan.nkc <= 1) return e;
   return launch_chunk_reduce(partial, Y, T, N, plan.nkc, stream);
 }
