@@ -303,11 +303,10 @@ MOBI_API size_t mobi_linear_workspace_bytes(int64_t T, int64_t N, int64_t K, int
  *            NULL when that size is 0); the first
  *            align256(mobi_route_workspace_bytes) bytes serve the routing step.
  * What the single call adds: for T <= 16 the decode kernel is launched as a
- * programmatic dependent of the routing kernel and, knowing that kernel
- * writes only k_t, perm and offsets, loads X and its first weight stages
- * before waiting on it, so the routing time is hidden behind the GEMM's
- * start. Nothing in X, Wr, bias, codes or sz may be written by other work
- * while the call runs. Errors as for mobi_route and mobi_gemm; nothing is
+ * programmatic dependent of the routing kernel, so its launch and set-up
+ * overlap the routing (it reads k_t, which decides its work split, only after
+ * the routing kernel has finished). Nothing in X, Wr, bias, codes or sz may be
+ * written by other work while the call runs. Errors as for mobi_route and mobi_gemm; nothing is
  * launched when an argument is rejected.
  */
 MOBI_API mobi_status mobi_linear(const void* X, int64_t T, int64_t K, const float* Wr,
@@ -338,7 +337,7 @@ typedef struct mobi_linear_problem {
 } mobi_linear_problem;
 
 /* Largest problem count of one mobi_linear_grouped call. */
-#define MOBI_MAX_GROUP 8
+#define MOBI_MAX_GROUP 16
 
 /* Scratch bytes of mobi_linear_grouped for these problems (0 for invalid
  * arguments or when none is needed). */
@@ -387,9 +386,9 @@ MOBI_API mobi_status mobi_gemm_grouped_bits(const mobi_gemm_problem* problems, i
  *   ws        scratch of mobi_linear_grouped_workspace_bytes bytes.
  * Launches: one routing launch (an 8-CTA cluster per problem), one decode
  * launch per fragment class present (T <= 8 and 9..16 tokens; the SMs are
- * shared among that class's problems in proportion to their weight counts),
- * and one chunk-reduction launch, so per-launch ramp-up and drain are paid
- * once per step instead of once per problem. Outputs must not overlap any
+ * shared among that class's problems in equal parts of the slice bytes they
+ * read, once k_t is known), and one chunk-reduction launch, so per-launch
+ * ramp-up and drain are paid once per step instead of once per problem. Outputs must not overlap any
  * problem's inputs or each other. Errors as for mobi_linear, checked for every
  * problem before anything is launched; T > 16 gives MOBI_ERR_UNSUPPORTED_SHAPE.
  */

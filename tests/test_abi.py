@@ -178,7 +178,7 @@ def test_linear_grouped_validation(L):
         arr = (P * max(len(probs), 1))(*probs)
         return L.mobi_linear_grouped(arr if probs else None, len(probs), G, S, ws, wsb, None)
     assert call([]) == 1
-    assert call([prob()] * 9) == 1                  # more than MOBI_MAX_GROUP
+    assert call([prob()] * 17) == 1                 # more than MOBI_MAX_GROUP
     assert call([prob(), prob(T=17)]) == 2          # decode-sized problems only
     assert call([prob(), prob(K=200)]) == 2
     assert call([prob(), prob(N=24)]) == 2
@@ -206,7 +206,7 @@ def test_gemm_grouped_validation(L):
         arr = (P * max(len(probs), 1))(*probs)
         return L.mobi_gemm_grouped(arr if probs else None, len(probs), G, S, ws, wsb, None)
     assert call([]) == 1
-    assert call([prob()] * 9) == 1
+    assert call([prob()] * 17) == 1
     assert call([prob(T=17)]) == 2
     assert call([prob(K=200)]) == 2
     assert call([prob(k_t=None)]) == 1

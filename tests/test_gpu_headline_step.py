@@ -1,7 +1,8 @@
 """The decode workload in the launch configuration the benchmark times: the
 nine Llama-7B-shaped problems ((N,K) in {(4096,4096), (11008,4096),
-(4096,11008)} x T in {1,4,16}), each with its own packed copy, as two
-mobi_linear_grouped calls (the six with T <= 8, the three with T = 16).
+(4096,11008)} x T in {1,4,16}), each with its own packed copy, as one
+mobi_linear_grouped call (one routing launch, a decode launch per fragment
+class, one chunk reduction).
 
 Every output is checked against the oracle (routing exact outside the 1e-5
 near-tie band, GEMM bars of the other tests), and the grouped results must
@@ -43,11 +44,7 @@ def test_headline_decode_step(mobi, oracle):
             probs.append({"X": L.X.to(DEV), "Wr": torch.from_numpy(L.Wr).to(DEV), "bias": None, "codes": codes,
                           "sz": sz, "N": N})
         del W
-    groups = [[i for i, L in enumerate(layers) if L.T <= 8], [i for i, L in enumerate(layers) if L.T > 8]]
-    outs = [None] * len(layers)
-    for g in groups:
-        for i, o in zip(g, mobi.mobi_linear_grouped([probs[i] for i in g])):
-            outs[i] = o
+    outs = mobi.mobi_linear_grouped(probs)
     mobi.mobi_sync_check()
     for L, pr, (c_ref, s_ref), (Y, k_t, perm, off) in zip(layers, probs, packs_ref, outs):
         tag = f"headline {L.N}x{L.K} T={L.T}"

@@ -42,7 +42,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("MOBI_LIB", os.path.join(_HERE, "libmobi.so"))
 
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
-MAX_GROUP = 8  # MOBI_MAX_GROUP
+MAX_GROUP = 16  # MOBI_MAX_GROUP
 
 
 class CkptTensor(ctypes.Structure):

@@ -434,9 +434,8 @@ mobi_status mobi_linear_bits(const void* X, int64_t T, int64_t K, const float* W
   e = launch_route(X, T, K, Wr, bias, S, k_t, perm, offsets, ws, s);
   if (e != cudaSuccess || T == 0 || N == 0) return cuda_status(e);
   void* gws = static_cast<uint8_t*>(ws) + route_ws;
-  // For up to 16 tokens the kernel just launched is the routing kernel, which
-  // writes only k_t, perm and offsets: the decode kernel may fetch X and the
-  // weights before it waits on it.
+  // For up to 16 tokens the decode kernel is a programmatic dependent of the
+  // routing kernel just launched: its launch and set-up overlap the routing.
   if (decode) return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, gws, s, dst, true, bits));
   return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, gws, s, dst, bits));
 }
@@ -504,9 +503,8 @@ mobi_status mobi_linear_grouped_bits(const mobi_linear_problem* problems, int co
   }
   e = launch_route_small_grouped(rg, S, s);
   if (e != cudaSuccess) return cuda_status(e);
-  // As in mobi_linear: the kernel just launched is the routing kernel, which
-  // writes only k_t, perm and offsets, so the decode kernels may fetch X and
-  // the weights before they wait on it.
+  // As in mobi_linear: the decode launches are programmatic dependents of the
+  // routing launch.
   return cuda_status(launch_decode_grouped(jobs, count, S, s, dst, true));
 }
 

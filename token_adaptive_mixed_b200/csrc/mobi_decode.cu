@@ -26,10 +26,10 @@
 // and every CTA takes the tiles whose start falls in its equal share of the
 // total cost. A CTA's range is one or a few segments (runs of tiles in one
 // chunk). For each segment the CTA builds the chunk's B operand image in
-// shared memory (read with ldmatrix), then its twelve warps split the
-// segment's (tile, slice) stages evenly, one contiguous run each; every warp
-// streams its stages' codes and scale/zero words through its own three-stage
-// TMA ring (it issues its own copies and waits on its own barriers). A tile
+// shared memory (read with ldmatrix), then its warps split the segment's
+// (tile, slice) stages evenly, one contiguous run each; every warp streams its
+// stages' codes and scale/zero words through its own TMA ring (it issues its
+// own copies and waits on its own barriers). A tile
 // is cut between two warps only before its last slice: the second warp leaves
 // that slice's sums in shared memory and the first adds them after the
 // segment's barrier, which rounds exactly as the uncut order does. Chunks
@@ -48,8 +48,18 @@ namespace mobi {
 
 constexpr int kDecChunk = 8;       // groups per K chunk (1024 columns)
 constexpr int kDecRows = 16;       // rows per tile (one m16n8k16 A tile)
-constexpr int kDecWarps = 12;      // warps per CTA
-constexpr int kDecDepth = 3;       // stages per warp ring
+// Warps per CTA and stages per warp ring, per fragment class. T <= 8 runs 16
+// warps (128 registers each) with two-stage rings; T <= 16 needs more
+// registers per warp and runs 12 with three-stage rings. Both load the B
+// fragments two k16 steps at a time, just before their MMAs; T <= 16 also
+// reads the group sums from shared memory at each promotion.
+template <int NB>
+struct DecCfg {
+  static constexpr int kWarps = NB == 1 ? 16 : 12;
+  static constexpr int kDepth = NB == 1 ? 2 : 3;
+  static constexpr bool kJitB = true;
+  static constexpr bool kXsSmem = NB != 1;
+};
 constexpr int kDecStageOv = 3;     // fixed cost of a stage, in groups (work split cost model)
 constexpr int kDecSegCost = 28 * (kDecChunk + kDecStageOv);  // set-up of a segment: about 28 full stages
 // A stage is one (tile, slice): the chunk's 8 groups of 16 code rows as two
@@ -62,16 +72,18 @@ constexpr uint32_t kDecSz = kDecChunk * kDecRows * 4;
 // Shared memory of the decode kernel for NB 8-token column blocks (T <= 8 NB).
 template <int NB>
 struct DecLayout {
-  static constexpr int kThreads = 32 * kDecWarps;
+  static constexpr int kWarps = DecCfg<NB>::kWarps;
+  static constexpr int kDepth = DecCfg<NB>::kDepth;
+  static constexpr int kThreads = 32 * kWarps;
   static constexpr uint32_t kCodes = 0;                                          // [warp][depth] code stages
-  static constexpr uint32_t kSzs = kCodes + kDecWarps * kDecDepth * kDecCodes;   // [warp][depth] scale/zero stages
-  static constexpr uint32_t kBimg = kSzs + kDecWarps * kDecDepth * kDecSz;       // B image, 16 KB per NB
+  static constexpr uint32_t kSzs = kCodes + kWarps * kDepth * kDecCodes;         // [warp][depth] scale/zero stages
+  static constexpr uint32_t kBimg = kSzs + kWarps * kDepth * kDecSz;             // B image, 16 KB per NB
   static constexpr uint32_t kBimgBytes = kDecChunk * NB * 8 * 256;
   static constexpr uint32_t kXs = kBimg + kBimgBytes;                            // sum_k x [group][16 tokens]
   static constexpr uint32_t kSc = kXs + kDecChunk * 16 * 4;                      // [warp][group][row] float2
-  static constexpr uint32_t kHead = kSc + kDecWarps * kDecChunk * kDecRows * 8;  // [warp][nb][A/B][lane] float2
-  static constexpr uint32_t kBar = kHead + kDecWarps * NB * 2 * 32 * 8;          // [warp][depth] full barriers
-  static constexpr uint32_t kNever = kBar + kDecWarps * kDecDepth * 8;           // a barrier nothing completes
+  static constexpr uint32_t kHead = kSc + kWarps * kDecChunk * kDecRows * 8;     // [warp][nb][A/B][lane] float2
+  static constexpr uint32_t kBar = kHead + kWarps * NB * 2 * 32 * 8;             // [warp][depth] full barriers
+  static constexpr uint32_t kNever = kBar + kWarps * kDepth * 8;                 // a barrier nothing completes
   static constexpr uint32_t kBytes = kNever + 8;
   static constexpr size_t kDynamic = kBytes + 1024;  // + manual 1 KB alignment
   static_assert(kDynamic <= 232448, "fits the opt-in shared memory of one CTA");
@@ -244,7 +256,8 @@ template <int NB, int MG, int BITS>
 __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
     const __grid_constant__ DecGroup<MG> grp, DeviceStatus* st, uint64_t limit) {
   using L = DecLayout<NB>;
-  constexpr int D = kDecDepth;
+  constexpr int D = L::kDepth;
+  constexpr int kDecWarps = L::kWarps;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ DecSplit<MG> sp;
@@ -474,12 +487,15 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
       ktl[nb][1] = __shfl_sync(0xffffffffu, my_kt, 8 * nb + 2 * t4 + 1);
     }
     // sum_k x of the lane's two tokens, per group and column block.
-    float2 xs[kDecChunk][NB];
+    constexpr bool kJitB = DecCfg<NB>::kJitB, kXsSmem = DecCfg<NB>::kXsSmem;
+    float2 xs[kXsSmem ? 1 : kDecChunk][NB];
+    if constexpr (!kXsSmem) {
 #pragma unroll
-    for (int g = 0; g < kDecChunk; ++g)
+      for (int g = 0; g < kDecChunk; ++g)
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb)
-        xs[g][nb] = *reinterpret_cast<const float2*>(xs_sm + g * 16 + 8 * nb + 2 * t4);
+        for (int nb = 0; nb < NB; ++nb)
+          xs[g][nb] = *reinterpret_cast<const float2*>(xs_sm + g * 16 + 8 * nb + 2 * t4);
+    }
 
     float* const out = prob.out + (int64_t)c * T * N;
     const CUtensorMap* tm_codes = &grp.tm_codes[p];
@@ -534,7 +550,9 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
       for (int g0 = 0; g0 < kDecChunk; g0 += 2) {
         if (g0 >= g_valid) break;  // the last chunk's missing groups (their B image is zero)
         uint2 wa[2], wb[2];
-        uint32_t bf[2][NB][8][2];
+        // B fragments: all eight k16 steps of both groups up front, or (kJitB)
+        // two steps at a time just before their MMAs.
+        uint32_t bf[2][NB][kJitB ? 2 : 8][2];
 #pragma unroll
         for (int gg = 0; gg < 2; ++gg) {
           if (BITS == 2) {
@@ -546,26 +564,39 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
             wa[gg] = make_uint2(x, x >> 1);
             wb[gg] = make_uint2(y, y >> 1);
           }
+          if constexpr (!kJitB) {
 #pragma unroll
-          for (int nb = 0; nb < NB; ++nb)
+            for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-            for (int jp = 0; jp < 4; ++jp)
-              ldsm_x4(bimg + bimg_off(g0 + gg, nb, 2 * jp, 0, NB), bf[gg][nb][2 * jp][0], bf[gg][nb][2 * jp][1],
-                      bf[gg][nb][2 * jp + 1][0], bf[gg][nb][2 * jp + 1][1]);
+              for (int jp = 0; jp < 4; ++jp)
+                ldsm_x4(bimg + bimg_off(g0 + gg, nb, 2 * jp, 0, NB), bf[gg][nb][2 * jp][0], bf[gg][nb][2 * jp][1],
+                        bf[gg][nb][2 * jp + 1][0], bf[gg][nb][2 * jp + 1][1]);
+          }
         }
         float d[2][NB][4];
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           const int h = jj >> 2, f = jj & 3;
           const uint32_t mk = kFieldMask << (2 * f);
+          const int jb = kJitB ? (jj & 1) : jj;  // the step's slot in bf
+          if constexpr (kJitB) {
+            if ((jj & 1) == 0) {
+#pragma unroll
+              for (int gg = 0; gg < 2; ++gg)
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb)
+                  ldsm_x4(bimg + bimg_off(g0 + gg, nb, jj, 0, NB), bf[gg][nb][0][0], bf[gg][nb][0][1],
+                          bf[gg][nb][1][0], bf[gg][nb][1][1]);
+            }
+          }
 #pragma unroll
           for (int gg = 0; gg < 2; ++gg) {
             const uint32_t a0 = (wa[gg].x >> (8 * h)) & mk, a2 = (wa[gg].y >> (8 * h)) & mk;
             const uint32_t a1r = (wb[gg].x >> (8 * h)) & mk, a3 = (wb[gg].y >> (8 * h)) & mk;
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {
-              if (jj == 0) mma_bf16_16816_z(d[gg][nb], a0, a1r, a2, a3, bf[gg][nb][jj][0], bf[gg][nb][jj][1]);
-              else mma_bf16_16816(d[gg][nb], a0, a1r, a2, a3, bf[gg][nb][jj][0], bf[gg][nb][jj][1]);
+              if (jj == 0) mma_bf16_16816_z(d[gg][nb], a0, a1r, a2, a3, bf[gg][nb][jb][0], bf[gg][nb][jb][1]);
+              else mma_bf16_16816(d[gg][nb], a0, a1r, a2, a3, bf[gg][nb][jb][0], bf[gg][nb][jb][1]);
             }
           }
         }
@@ -576,10 +607,12 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
           const float2 pA = scw[g * kDecRows + gid], pB = scw[g * kDecRows + gid + 8];
 #pragma unroll
           for (int nb = 0; nb < NB; ++nb) {
+            const float2 xg =
+                kXsSmem ? *reinterpret_cast<const float2*>(xs_sm + g * 16 + 8 * nb + 2 * t4) : xs[kXsSmem ? 0 : g][nb];
             ysA[nb] = __ffma2_rn(make_float2(pA.x, pA.x), make_float2(d[gg][nb][0], d[gg][nb][1]),
-                                 __ffma2_rn(make_float2(pA.y, pA.y), xs[g][nb], ysA[nb]));
+                                 __ffma2_rn(make_float2(pA.y, pA.y), xg, ysA[nb]));
             ysB[nb] = __ffma2_rn(make_float2(pB.x, pB.x), make_float2(d[gg][nb][2], d[gg][nb][3]),
-                                 __ffma2_rn(make_float2(pB.y, pB.y), xs[g][nb], ysB[nb]));
+                                 __ffma2_rn(make_float2(pB.y, pB.y), xg, ysB[nb]));
           }
         }
       }

@@ -42,7 +42,7 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t c
 //
 // Problem tables travel as __grid_constant__ kernel parameters, so a CUDA graph
 // captures them by value and no device memory holds them.
-constexpr int kMaxGroup = 8;
+constexpr int kMaxGroup = 16;
 // Slices per packed layer: up to four (e.g. four 1-bit slices for 1..4 bits).
 constexpr int kMaxSlices = 4;
 
