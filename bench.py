@@ -55,12 +55,13 @@ def decode_bytes(N, K, T, kmax, bits=2):
     return kmax * (N * K * bits // 8 + N * (K // 128) * 4) + T * K * 2
 
 
-# DRAM bytes / algorithmic bytes of the decode kernel, from one ncu capture of
-# a single 11008 x 4096, T=4, k_max=3 launch (dram__bytes_read.sum 38124288 +
-# dram__bytes_write.sum 0 against 38076416 algorithmic bytes). Traffic grows
-# in proportion to the bytes streamed, so the step's traffic is the step's
-# algorithmic bytes times this ratio. Valid for the decode kernel as captured.
-DECODE_DRAM_RATIO = 38124288 / 38076416
+# DRAM bytes / algorithmic bytes of the decode step, from one ncu capture of
+# each of the step's two decode launches (T <= 8 class: 147277056 read +
+# 3972608 written; T = 16 class: 92629760 read + 3942912 written) against the
+# step's 228773376 algorithmic bytes. Traffic grows in proportion to the bytes
+# streamed, so the step's traffic is its algorithmic bytes times this ratio.
+# Valid for the decode kernel as captured.
+DECODE_DRAM_RATIO = (147277056 + 3972608 + 92629760 + 3942912) / 228773376
 
 
 class ClockSampler:
@@ -435,11 +436,10 @@ def time_prefill(mobi, L, dev, reps, tf_peak, flush):
 
 
 # DRAM bytes (read + write) of one prefill_kernel launch, from one ncu capture
-# per workload (dram__bytes_read.sum + dram__bytes_write.sum; the summary and
-# command are in profiles/small_kernels_prefill_11008x4096.md). Valid while the
-# prefill kernel is unchanged.
-PREFILL_DRAM_BYTES = {"prefill_11008x4096_T2048": 62713344 + 46622464,
-                      "skewed_prefill_28672x8192_T4096": 1596453376 + 446456320}
+# (dram__bytes_read.sum + dram__bytes_write.sum) of the 11008 x 4096, T = 2048
+# workload. The 28672 x 8192 workload has no capture of the current kernel
+# (its traffic is reported as null). Valid while the prefill kernel is unchanged.
+PREFILL_DRAM_BYTES = {"prefill_11008x4096_T2048": 60248576 + 45078784}
 
 
 # fp32 FMA peak of the SIMT pipes: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz
