@@ -71,6 +71,14 @@ def _load():
             lib.oracle_unpack_bits.restype = None
             lib.oracle_reconstruct_bits.argtypes = [p, p, i64, i64, ci, ci, ci, ci, p]
             lib.oracle_reconstruct_bits.restype = None
+            lib.oracle_pack_slices.argtypes = [p, i64, i64, ci, ci, p, p, p, p, ci]
+            lib.oracle_pack_slices.restype = ci
+            lib.oracle_unpack_slices.argtypes = [p, i64, i64, ci, p, p]
+            lib.oracle_unpack_slices.restype = None
+            lib.oracle_reconstruct_slices.argtypes = [p, p, i64, i64, ci, ci, p, ci, p]
+            lib.oracle_reconstruct_slices.restype = None
+            lib.oracle_gemm_slices.argtypes = [p, i64, i64, p, p, p, i64, ci, ci, p, p, i64, p, ci]
+            lib.oracle_gemm_slices.restype = None
             lib.oracle_max_threads.argtypes = []
             lib.oracle_max_threads.restype = ci
             _lib = lib
@@ -124,22 +132,58 @@ def pack_bits(W_f16: np.ndarray, G: int = 128, S: int = 3, bits: int = 2, nthrea
     return codes, sz, q
 
 
-def unpack(codes: np.ndarray, N: int, K: int, S: int, bits: int = 2) -> np.ndarray:
-    """Packed words -> codes uint8 [S,N,K] by the documented layout of `bits`-bit codes."""
+def _widths(S: int, widths) -> np.ndarray:
+    w = np.ascontiguousarray(widths, np.int32).reshape(-1)
+    if w.shape[0] != S:
+        raise ValueError("one width per slice")
+    return w
+
+
+def codes_words(N: int, K: int, widths) -> int:
+    """32-bit words of the codes of slices of the given widths, stored one after another."""
+    return sum(N * K * int(b) // 32 for b in widths)
+
+
+def pack_slices(W_f16: np.ndarray, widths, G: int = 128, nthreads: int = 0):
+    """MoBiSlice packing with slice s of widths[s]-bit codes (1 or 2), G-wide groups.
+    Returns (codes uint32 flat [sum_s N*K*w_s/32], sz uint32 [S,K/G,N], q uint8 [S,N,K])."""
+    lib = _load()
+    W = _u16(W_f16)
+    N, K = W.shape
+    S = len(widths)
+    w = _widths(S, widths)
+    codes = np.zeros(codes_words(N, K, w), np.uint32)
+    sz = np.zeros((S, K // G, N), np.uint32)
+    q = np.zeros((S, N, K), np.uint8)
+    if lib.oracle_pack_slices(_ptr(W), N, K, G, S, _ptr(w), _ptr(codes), _ptr(sz), _ptr(q), nthreads) != 0:
+        raise ValueError("oracle_pack_slices: unsupported arguments")
+    return codes, sz, q
+
+
+def unpack(codes: np.ndarray, N: int, K: int, S: int, bits: int = 2, widths=None) -> np.ndarray:
+    """Packed words -> codes uint8 [S,N,K] by the documented layout of `bits`-bit codes
+    (or of slices of the given widths)."""
     lib = _load()
     codes = np.ascontiguousarray(codes, np.uint32)
     q = np.zeros((S, N, K), np.uint8)
-    lib.oracle_unpack_bits(_ptr(codes), N, K, S, bits, _ptr(q))
+    if widths is not None:
+        lib.oracle_unpack_slices(_ptr(codes), N, K, S, _ptr(_widths(S, widths)), _ptr(q))
+    else:
+        lib.oracle_unpack_bits(_ptr(codes), N, K, S, bits, _ptr(q))
     return q
 
 
 def reconstruct(codes: np.ndarray, sz: np.ndarray, N: int, K: int, k: int, G: int = 128, S: int = 3,
-                bits: int = 2) -> np.ndarray:
+                bits: int = 2, widths=None) -> np.ndarray:
     """W^(k) = sum of the first k dequantised slices, fp64 [N,K]."""
     lib = _load()
     out = np.zeros((N, K), np.float64)
-    lib.oracle_reconstruct_bits(_ptr(np.ascontiguousarray(codes, np.uint32)),
-                                _ptr(np.ascontiguousarray(sz, np.uint32)), N, K, G, S, bits, k, _ptr(out))
+    c = _ptr(np.ascontiguousarray(codes, np.uint32))
+    z = _ptr(np.ascontiguousarray(sz, np.uint32))
+    if widths is not None:
+        lib.oracle_reconstruct_slices(c, z, N, K, G, S, _ptr(_widths(S, widths)), k, _ptr(out))
+    else:
+        lib.oracle_reconstruct_bits(c, z, N, K, G, S, bits, k, _ptr(out))
     return out
 
 
@@ -193,8 +237,10 @@ def bucket(k_t: np.ndarray, S: int = 3):
 
 
 def gemm(X_bf16: np.ndarray, k_t: np.ndarray, codes: np.ndarray, sz: np.ndarray, N: int,
-         G: int = 128, S: int = 3, tokens: np.ndarray | None = None, nthreads: int = 0, bits: int = 2) -> np.ndarray:
-    """Y fp64 [len(tokens) or T, N] = x_t . W^(k_t)^T for the listed tokens (`bits`-bit codes)."""
+         G: int = 128, S: int = 3, tokens: np.ndarray | None = None, nthreads: int = 0, bits: int = 2,
+         widths=None) -> np.ndarray:
+    """Y fp64 [len(tokens) or T, N] = x_t . W^(k_t)^T for the listed tokens (`bits`-bit codes,
+    or slices of the given widths)."""
     lib = _load()
     X = _u16(X_bf16)
     T, K = X.shape
@@ -202,7 +248,11 @@ def gemm(X_bf16: np.ndarray, k_t: np.ndarray, codes: np.ndarray, sz: np.ndarray,
     tok = None if tokens is None else np.ascontiguousarray(tokens, np.int32)
     n_tok = T if tok is None else tok.shape[0]
     Y = np.zeros((n_tok, N), np.float64)
-    lib.oracle_gemm_bits(_ptr(X), T, K, _ptr(k_t), _ptr(np.ascontiguousarray(codes, np.uint32)),
-                         _ptr(np.ascontiguousarray(sz, np.uint32)), N, G, S, bits, _ptr(tok), n_tok, _ptr(Y),
-                         nthreads)
+    c = _ptr(np.ascontiguousarray(codes, np.uint32))
+    z = _ptr(np.ascontiguousarray(sz, np.uint32))
+    if widths is not None:
+        lib.oracle_gemm_slices(_ptr(X), T, K, _ptr(k_t), c, z, N, G, S, _ptr(_widths(S, widths)), _ptr(tok), n_tok,
+                               _ptr(Y), nthreads)
+    else:
+        lib.oracle_gemm_bits(_ptr(X), T, K, _ptr(k_t), c, z, N, G, S, bits, _ptr(tok), n_tok, _ptr(Y), nthreads)
     return Y

@@ -36,7 +36,11 @@
  *   slices give 1..S bits per weight ([en] §2.A lists 3-bit precision, which
  *   2-bit slices cannot reach) and are stored at 1 bit per weight ([en] §3,
  *   "Specialized Kernel Implementation": the bytes fetched follow the bits
- *   used), 32 codes per word in the library's documented bit order.
+ *   used), 32 codes per word in the library's documented bit order. Slices of
+ *   different widths in one layer (oracle_pack_slices): round s quantises the
+ *   residual with its own width, and the slices are stored one after another,
+ *   each in the layout of its width; widths (2, 1, 1, 2) give 2, 3, 4 and 6
+ *   bits, the precisions [en] §2.A lists.
  *
  * Parity pins: every function here is pinned by tests/test_oracle.py against
  * closed-form groups, hand-derived packed words, invariants (non-increasing
@@ -98,17 +102,17 @@ int oracle_max_threads(void) {
 /*
  * One group of G weights of one row through S rounds of the recursion
  * R_1 = W, W_s = Q(R_s), R_{s+1} = R_s - W_s   ([ja] §2.1, [en] §2.A), with Q
- * the asymmetric min-max round-to-nearest of `bits`-bit codes: L = 2^bits - 1
- * steps between the group's minimum and maximum.
+ * the asymmetric min-max round-to-nearest of widths[s]-bit codes in round s:
+ * L = 2^widths[s] - 1 steps between the group's minimum and maximum.
  * q_out[s*G + i] receives the code of element i in slice s; scale_out[s] and
  * zero_out[s] the fp16 bit patterns of that slice's scale and zero.
  */
-static void quantise_group(const uint16_t* w, int G, int S, int bits, uint8_t* q_out,
+static void quantise_group(const uint16_t* w, int G, int S, const int* widths, uint8_t* q_out,
                            uint16_t* scale_out, uint16_t* zero_out) {
   float R[1024];
-  const float L = (float)((1 << bits) - 1); /* 2 bits: 4 levels, 3 steps; 1 bit: 1 step */
   for (int i = 0; i < G; ++i) R[i] = half_bits_to_float(w[i]);
   for (int s = 0; s < S; ++s) {
+    const float L = (float)((1 << widths[s]) - 1); /* 2 bits: 4 levels, 3 steps; 1 bit: 1 step */
     float mn = R[0], mx = R[0];
     for (int i = 1; i < G; ++i) {
       if (R[i] < mn) mn = R[i];
@@ -145,8 +149,19 @@ static void quantise_group(const uint16_t* w, int G, int S, int bits, uint8_t* q
  */
 static int64_t words_per_row(int64_t K, int bits) { return bits == 1 ? K / 32 : K / 16; }
 
-static int code_of(const uint32_t* codes, int64_t N, int64_t K, int bits, int64_t s, int64_t n, int64_t k) {
-  const uint32_t word = codes[(s * N + n) * words_per_row(K, bits) + (bits == 1 ? k / 32 : k / 16)];
+/* Word offset of slice s when the slices (widths[0..s-1]) are stored one after
+ * another, each [N][K * width / 32]. */
+static int64_t slice_offset(const int* widths, int64_t N, int64_t K, int64_t s) {
+  int64_t off = 0;
+  for (int64_t j = 0; j < s; ++j) off += N * words_per_row(K, widths[j]);
+  return off;
+}
+
+static int code_of(const uint32_t* codes, int64_t N, int64_t K, const int* widths, int64_t s, int64_t n,
+                   int64_t k) {
+  const int bits = widths[s];
+  const uint32_t word =
+      codes[slice_offset(widths, N, K, s) + n * words_per_row(K, bits) + (bits == 1 ? k / 32 : k / 16)];
   if (bits == 1) {
     const int i = (int)(k % 32);
     return (int)((word >> (i < 16 ? 2 * i : 2 * (i - 16) + 1)) & 1u);
@@ -154,34 +169,45 @@ static int code_of(const uint32_t* codes, int64_t N, int64_t K, int bits, int64_
   return (int)((word >> (2 * (k % 16))) & 3u);
 }
 
+static int uniform_widths(int* widths, int S, int bits) {
+  if (S < 1 || S > 8) return -1;
+  for (int j = 0; j < S; ++j) widths[j] = bits;
+  return 0;
+}
+
 /*
- * oracle_pack_bits: W fp16 [N][K] -> codes and sz for S slices of `bits`-bit
- * codes (bits 1 or 2) over G-wide groups, codes in the word layout of their
- * width (above). sz is [S][K/G][N] (fp16 scale in bits [15:0], fp16 zero in
- * bits [31:16]). If q_out is not NULL it receives the unpacked codes uint8
- * [S][N][K].
+ * oracle_pack_slices: W fp16 [N][K] -> codes and sz for S slices over G-wide
+ * groups, slice s of widths[s]-bit codes (1 or 2) in the word layout of its
+ * width (above), the slices one after another. sz is [S][K/G][N] (fp16 scale
+ * in bits [15:0], fp16 zero in bits [31:16]). If q_out is not NULL it
+ * receives the unpacked codes uint8 [S][N][K].
  * Returns 0, or -1 on an unsupported argument.
  */
-int oracle_pack_bits(const uint16_t* W, int64_t N, int64_t K, int G, int S, int bits,
-                     uint32_t* codes, uint32_t* sz, uint8_t* q_out, int nthreads) {
-  if (G <= 0 || G > 1024 || K % G != 0 || K % 16 != 0 || S < 1 || S > 8 || bits < 1 || bits > 2) return -1;
-  if (bits == 1 && K % 32 != 0) return -1;
+int oracle_pack_slices(const uint16_t* W, int64_t N, int64_t K, int G, int S, const int* widths,
+                       uint32_t* codes, uint32_t* sz, uint8_t* q_out, int nthreads) {
+  if (G <= 0 || G > 1024 || K % G != 0 || K % 16 != 0 || S < 1 || S > 8) return -1;
+  for (int j = 0; j < S; ++j) {
+    if (widths[j] < 1 || widths[j] > 2) return -1;
+    if (widths[j] == 1 && K % 32 != 0) return -1;
+  }
   set_threads(nthreads);
   const int64_t ngroups = K / G;
-  const int64_t nwords = words_per_row(K, bits);
 #pragma omp parallel for schedule(dynamic, 4)
   for (int64_t n = 0; n < N; ++n) {
     uint8_t q[8 * 1024];
     uint16_t sc[8], zr[8];
     uint8_t* row_codes = (uint8_t*)malloc((size_t)S * (size_t)K);
     for (int64_t g = 0; g < ngroups; ++g) {
-      quantise_group(W + n * K + g * G, G, S, bits, q, sc, zr);
+      quantise_group(W + n * K + g * G, G, S, widths, q, sc, zr);
       for (int s = 0; s < S; ++s) {
         sz[((int64_t)s * ngroups + g) * N + n] = (uint32_t)sc[s] | ((uint32_t)zr[s] << 16);
         for (int i = 0; i < G; ++i) row_codes[(int64_t)s * K + g * G + i] = q[s * G + i];
       }
     }
     for (int s = 0; s < S; ++s) {
+      const int bits = widths[s];
+      const int64_t nwords = words_per_row(K, bits);
+      uint32_t* slice = codes + slice_offset(widths, N, K, s);
       for (int64_t w = 0; w < nwords; ++w) {
         uint32_t word = 0;
         if (bits == 1) {
@@ -193,7 +219,7 @@ int oracle_pack_bits(const uint16_t* W, int64_t N, int64_t K, int G, int S, int 
           for (int i = 0; i < 16; ++i)
             word |= (uint32_t)row_codes[(int64_t)s * K + 16 * w + i] << (2 * i);
         }
-        codes[((int64_t)s * N + n) * nwords + w] = word;
+        slice[n * nwords + w] = word;
       }
       if (q_out)
         memcpy(q_out + ((int64_t)s * N + n) * K, row_codes + (int64_t)s * K, (size_t)K);
@@ -201,6 +227,14 @@ int oracle_pack_bits(const uint16_t* W, int64_t N, int64_t K, int G, int S, int 
     free(row_codes);
   }
   return 0;
+}
+
+/* oracle_pack_bits: every slice `bits`-bit (1 or 2). */
+int oracle_pack_bits(const uint16_t* W, int64_t N, int64_t K, int G, int S, int bits,
+                     uint32_t* codes, uint32_t* sz, uint8_t* q_out, int nthreads) {
+  int widths[8];
+  if (uniform_widths(widths, S, bits) != 0) return -1;
+  return oracle_pack_slices(W, N, K, G, S, widths, codes, sz, q_out, nthreads);
 }
 
 /*
@@ -212,12 +246,18 @@ int oracle_pack(const uint16_t* W, int64_t N, int64_t K, int G, int S,
   return oracle_pack_bits(W, N, K, G, S, 2, codes, sz, q_out, nthreads);
 }
 
-/* oracle_unpack_bits: the documented word layout of `bits`-bit codes back to
- * codes uint8 [S][N][K]; oracle_unpack is the 2-bit case. */
-void oracle_unpack_bits(const uint32_t* codes, int64_t N, int64_t K, int S, int bits, uint8_t* q_out) {
+/* oracle_unpack_slices: the documented word layouts (slice s of widths[s]-bit
+ * codes) back to codes uint8 [S][N][K]; oracle_unpack_bits has one width for
+ * every slice and oracle_unpack is the 2-bit case. */
+void oracle_unpack_slices(const uint32_t* codes, int64_t N, int64_t K, int S, const int* widths, uint8_t* q_out) {
   for (int64_t s = 0; s < S; ++s)
     for (int64_t n = 0; n < N; ++n)
-      for (int64_t k = 0; k < K; ++k) q_out[(s * N + n) * K + k] = (uint8_t)code_of(codes, N, K, bits, s, n, k);
+      for (int64_t k = 0; k < K; ++k) q_out[(s * N + n) * K + k] = (uint8_t)code_of(codes, N, K, widths, s, n, k);
+}
+
+void oracle_unpack_bits(const uint32_t* codes, int64_t N, int64_t K, int S, int bits, uint8_t* q_out) {
+  int widths[8];
+  if (uniform_widths(widths, S, bits) == 0) oracle_unpack_slices(codes, N, K, S, widths, q_out);
 }
 
 void oracle_unpack(const uint32_t* codes, int64_t N, int64_t K, int S, uint8_t* q_out) {
@@ -229,14 +269,14 @@ void oracle_unpack(const uint32_t* codes, int64_t N, int64_t K, int S, uint8_t* 
  * in fp64 (exact: every term is a small integer times an fp16 value)
  * ([ja] §2.1 W^(b) = sum W_e; [en] §2.A "Elasticity").
  */
-void oracle_reconstruct_bits(const uint32_t* codes, const uint32_t* sz, int64_t N, int64_t K, int G, int S,
-                             int bits, int k, double* W_hat) {
+void oracle_reconstruct_slices(const uint32_t* codes, const uint32_t* sz, int64_t N, int64_t K, int G, int S,
+                               const int* widths, int k, double* W_hat) {
   const int64_t ngroups = K / G;
   for (int64_t n = 0; n < N; ++n)
     for (int64_t j = 0; j < K; ++j) {
       double acc = 0.0;
       for (int s = 0; s < k && s < S; ++s) {
-        int q = code_of(codes, N, K, bits, s, n, j);
+        int q = code_of(codes, N, K, widths, s, n, j);
         uint32_t e = sz[((int64_t)s * ngroups + j / G) * N + n];
         double scale = (double)half_bits_to_float((uint16_t)(e & 0xffffu));
         double zero = (double)half_bits_to_float((uint16_t)(e >> 16));
@@ -244,6 +284,12 @@ void oracle_reconstruct_bits(const uint32_t* codes, const uint32_t* sz, int64_t 
       }
       W_hat[n * K + j] = acc;
     }
+}
+
+void oracle_reconstruct_bits(const uint32_t* codes, const uint32_t* sz, int64_t N, int64_t K, int G, int S,
+                             int bits, int k, double* W_hat) {
+  int widths[8];
+  if (uniform_widths(widths, S, bits) == 0) oracle_reconstruct_slices(codes, sz, N, K, G, S, widths, k, W_hat);
 }
 
 void oracle_reconstruct(const uint32_t* codes, const uint32_t* sz, int64_t N, int64_t K,
@@ -357,15 +403,16 @@ int oracle_bucket(const int32_t* k_t, int64_t T, int S, int32_t* perm, int32_t* 
 /* ---- mixed-bit GEMM ----------------------------------------------------- */
 
 /*
- * oracle_gemm_bits: for each listed token t = tokens[i] (all tokens when
+ * oracle_gemm_slices: for each listed token t = tokens[i] (all tokens when
  * tokens is NULL, i = t), Y[i][n] = sum_k x[t,k] * W^(k_t)[n,k] in fp64, with
  * W^(k) = sum_{s<k} (q - z) * scale built exactly ([ja] §2.1; [en] §2.A) from
- * `bits`-bit codes. Y is fp64 [n_tokens][N]. The sum over k runs in index
- * order. oracle_gemm is the 2-bit case.
+ * slices of widths[s]-bit codes. Y is fp64 [n_tokens][N]. The sum over k runs
+ * in index order. oracle_gemm_bits has one width for every slice, and
+ * oracle_gemm is the 2-bit case.
  */
-void oracle_gemm_bits(const uint16_t* X, int64_t T, int64_t K, const int32_t* k_t,
-                      const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S, int bits,
-                      const int32_t* tokens, int64_t n_tokens, double* Y, int nthreads) {
+void oracle_gemm_slices(const uint16_t* X, int64_t T, int64_t K, const int32_t* k_t,
+                        const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S, const int* widths,
+                        const int32_t* tokens, int64_t n_tokens, double* Y, int nthreads) {
   (void)T;
   set_threads(nthreads);
   const int64_t ngroups = K / G;
@@ -377,7 +424,7 @@ void oracle_gemm_bits(const uint16_t* X, int64_t T, int64_t K, const int32_t* k_
     for (int64_t j = 0; j < K; ++j) {
       double acc = 0.0;
       for (int s = 0; s < S; ++s) {
-        int q = code_of(codes, N, K, bits, s, n, j);
+        int q = code_of(codes, N, K, widths, s, n, j);
         uint32_t e = sz[((int64_t)s * ngroups + j / G) * N + n];
         double scale = (double)half_bits_to_float((uint16_t)(e & 0xffffu));
         double zero = (double)half_bits_to_float((uint16_t)(e >> 16));
@@ -394,6 +441,14 @@ void oracle_gemm_bits(const uint16_t* X, int64_t T, int64_t K, const int32_t* k_
     }
     free(wk);
   }
+}
+
+void oracle_gemm_bits(const uint16_t* X, int64_t T, int64_t K, const int32_t* k_t,
+                      const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S, int bits,
+                      const int32_t* tokens, int64_t n_tokens, double* Y, int nthreads) {
+  int widths[8];
+  if (uniform_widths(widths, S, bits) == 0)
+    oracle_gemm_slices(X, T, K, k_t, codes, sz, N, G, S, widths, tokens, n_tokens, Y, nthreads);
 }
 
 void oracle_gemm(const uint16_t* X, int64_t T, int64_t K, const int32_t* k_t,

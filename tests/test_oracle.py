@@ -517,3 +517,81 @@ def test_pack_bits_rejects_bad_arguments(oracle):
     for kw in ({"bits": 0}, {"bits": 3}, {"G": 96}):
         with pytest.raises(ValueError):
             oracle.pack_bits(W, **{"G": 128, "S": 2, "bits": 2, **kw})
+
+
+# ---- slices of mixed widths in one layer ---------------------------------------
+
+def test_mixed_uniform_widths_are_pack_bits(oracle):
+    """One width for every slice is the uniform packer, bit for bit."""
+    W = _random_W(32, 512, 70, outliers=2)
+    for b in (1, 2):
+        c1, s1, q1 = oracle.pack_bits(W, G=128, S=3, bits=b)
+        c2, s2, q2 = oracle.pack_slices(W, (b, b, b), G=128)
+        assert np.array_equal(c1.ravel(), c2) and np.array_equal(s1, s2) and np.array_equal(q1, q2)
+
+
+def test_mixed_each_round_quantises_its_residual(oracle):
+    """Widths (2, 1, 1, 2): round s is one asymmetric min-max RTN of the fp32
+    residual left by rounds < s with 2^w_s - 1 steps. The residual is rebuilt
+    here in fp32 from the oracle's own earlier codes, scales and zeros, then
+    torch's fake quantiser (range [0, 2^w_s - 1], the oracle's scale and zero)
+    and MinMax observer (its step, rounded to fp16) must give round s's
+    dequantised slice and stored scale."""
+    from torch.ao.quantization.observer import MinMaxObserver
+    N, K, G, widths = 16, 512, 128, (2, 1, 1, 2)
+    W = _random_W(N, K, 71, outliers=3)
+    codes, sz, q = oracle.pack_slices(W, widths, G=G)
+    R = W.astype(np.float32)
+    for s, b in enumerate(widths):
+        L = (1 << b) - 1
+        scale = (sz[s].T & 0xFFFF).astype(np.uint16).view(F16).astype(np.float32)  # [N, K/G]
+        zero = (sz[s].T >> 16).astype(np.uint16).view(F16).astype(np.float32)
+        x = torch.from_numpy(R.reshape(N * K // G, G).copy())
+        fq = torch.fake_quantize_per_channel_affine(x, torch.from_numpy(scale.ravel()),
+                                                    torch.from_numpy(zero.ravel().astype(np.int32)), 0, 0, L)
+        deq = (q[s].astype(np.float32) - np.repeat(zero, G, axis=1)) * np.repeat(scale, G, axis=1)
+        assert np.array_equal(fq.numpy().reshape(N, K), deq), f"round {s}"
+        for n in range(0, N, 5):
+            for g in range(K // G):
+                obs = MinMaxObserver(dtype=torch.quint8, quant_min=0, quant_max=L)
+                obs(torch.from_numpy(R[n, g * G:(g + 1) * G].copy()))
+                sc, _ = obs.calculate_qparams()
+                assert f16_bits(float(sc.to(torch.float16))) == int(sz[s, g, n] & 0xFFFF)
+        R = (R - deq).astype(np.float32)
+
+
+def test_mixed_layout_is_slice_major(oracle):
+    """Slice 0 of widths (2, 1, 1, 2) is the first N*K/16 words and equals a
+    one-slice 2-bit pack; every slice unpacks to the codes of its round, and
+    the layer's code words total N*K*(2+1+1+2)/32."""
+    N, K, widths = 24, 1024, (2, 1, 1, 2)
+    W = _random_W(N, K, 72)
+    codes, sz, q = oracle.pack_slices(W, widths)
+    assert codes.shape == (N * K * 6 // 32,)
+    c0, s0, _ = oracle.pack_bits(W, G=128, S=1, bits=2)
+    assert np.array_equal(codes[:N * K // 16], c0.ravel()) and np.array_equal(sz[:1], s0)
+    assert np.array_equal(oracle.unpack(codes, N, K, 4, widths=widths), q)
+
+
+def test_mixed_gemm_equals_two_bit_storage(oracle):
+    """The same codes in the (hand-pinned) uniform 2-bit layout give the same
+    reconstruction and GEMM bit for bit, and the error falls with every slice
+    (2, 3, 4 and 6 bits)."""
+    N, K, T, widths = 24, 512, 6, (2, 1, 1, 2)
+    W = _random_W(N, K, 73, outliers=2)
+    codes, sz, q = oracle.pack_slices(W, widths)
+    codes2 = np.zeros((4, N, K // 16), np.uint32)
+    for i in range(16):
+        codes2 |= q[:, :, i::16].astype(np.uint32) << np.uint32(2 * i)
+    Wd = W.astype(np.float64)
+    fro = []
+    for k in range(1, 5):
+        Wk = oracle.reconstruct(codes, sz, N, K, k=k, S=4, widths=widths)
+        assert np.array_equal(Wk, oracle.reconstruct(codes2, sz, N, K, k=k, S=4, bits=2))
+        fro.append(np.linalg.norm(Wd - Wk))
+    assert all(b < a for a, b in zip(fro[:-1], fro[1:]))
+    rng = np.random.default_rng(9)
+    X = torch.from_numpy(rng.standard_normal((T, K), dtype=np.float32)).to(torch.bfloat16)
+    k_t = rng.integers(1, 5, T).astype(np.int32)
+    assert np.array_equal(oracle.gemm(X, k_t, codes, sz, N, S=4, widths=widths),
+                          oracle.gemm(X, k_t, codes2, sz, N, S=4, bits=2))
