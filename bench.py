@@ -49,9 +49,11 @@ def peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def decode_bytes(N, K, T, kmax, bits=2):
+def decode_bytes(N, K, T, kmax, bits=2, widths=None):
     """Algorithmic bytes of one decode GEMM: k_max slices of codes (bits per
-    weight) and scale/zero words, plus X."""
+    weight, or widths[s] for slice s) and scale/zero words, plus X."""
+    if widths is not None:
+        return sum(N * K * int(w) // 8 + N * (K // 128) * 4 for w in widths[:kmax]) + T * K * 2
     return kmax * (N * K * bits // 8 + N * (K // 128) * 4) + T * K * 2
 
 
@@ -565,21 +567,24 @@ def time_generic(mobi, wl, dev, hbm_peak, tf_peak, flush, steps=200):
     Llama-7B shapes at T = 4 as one mobi_linear_grouped call, router mix 1/4
     each (five packed copies in rotation, so no copy is L2-resident when it is
     read again), beside the same step with four 2-bit slices (same k_max, twice
-    the code bytes); (b) the prefill workload's shape (T = 2048, 11008 x 4096)
-    through route + prefill GEMM."""
+    the code bytes) and with slices of widths (2, 1, 1, 2) (2, 3, 4, 6 bits);
+    (b) the prefill workload's shape (T = 2048, 11008 x 4096) through route +
+    prefill GEMM."""
     S = 4
     out = {"slicing": "4 x 1-bit slices, G = 128, codes at 1 bit per weight (32 per word)"}
     # Five packed copies of the three problems, run one after another in each
     # step, so a copy is read again only after 4 x its bytes of other weights
     # (above 200 MB at 1 bit per weight, more than the 126 MB L2).
     copies = 5
-    for bits in (1, 2):
+    for bits in (1, 2, "mixed"):
+        widths = (2, 1, 1, 2) if bits == "mixed" else None
         groups = []
         for r in range(copies):
             probs = []
             for i, (N, K) in enumerate(wl.DECODE_SHAPES):
                 L = wl.layer(f"gen_{N}x{K}", N, K, 4, seed=3000 + i, outlier_frac_cols=0.005, S=S, mix=(0.25,) * S)
-                codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(dev), S=S, bits=bits)
+                codes, sz = (mobi.mobi_pack(torch.from_numpy(L.W).to(dev), widths=widths) if widths else
+                             mobi.mobi_pack(torch.from_numpy(L.W).to(dev), S=S, bits=bits))
                 probs.append({"X": L.X.to(dev), "Wr": torch.from_numpy(L.Wr).to(dev),
                               "bias": torch.from_numpy(L.bias).to(dev), "codes": codes, "sz": sz, "N": N,
                               "Y": torch.empty((4, N), dtype=torch.float32, device=dev),
@@ -592,17 +597,22 @@ def time_generic(mobi, wl, dev, hbm_peak, tf_peak, flush, steps=200):
 
         def step():
             for probs in groups:
-                mobi.mobi_linear_grouped(probs, S=S, ws=ws, bits=bits)
+                if widths:
+                    mobi.mobi_linear_grouped(probs, S=S, ws=ws, widths=widths)
+                else:
+                    mobi.mobi_linear_grouped(probs, S=S, ws=ws, bits=bits)
         step()
         mobi.mobi_sync_check()
         kmax = [int(p["k_t"].max().item()) for p in groups[0]]
-        nbytes = sum(decode_bytes(p["N"], p["X"].shape[1], 4, km, bits) for p, km in zip(groups[0], kmax))
+        nbytes = sum(decode_bytes(p["N"], p["X"].shape[1], 4, km, 2 if widths else bits, widths)
+                     for p, km in zip(groups[0], kmax))
         ms = time_graph(step, steps) / copies
-        key = "decode_T4_grouped" if bits == 1 else "decode_T4_grouped_2bit_slices"
+        key = {1: "decode_T4_grouped", 2: "decode_T4_grouped_2bit_slices"}.get(bits, "decode_T4_grouped_widths_2_1_1_2")
+        prec = [sum(widths[:km]) if widths else bits * km for km in kmax]
         out[key] = {"kmax_per_problem": kmax, "bytes_per_call": nbytes, "ms_per_call": round(ms, 5),
                     "GB/s": round(nbytes / ms / 1e6, 1), "frac_of_hbm": round(nbytes / ms / 1e6 / hbm_peak, 4),
-                    "precision_bits_per_weight": [bits * km for km in kmax],
-                    "code_bits_read_per_weight": [bits * km for km in kmax],
+                    "precision_bits_per_weight": prec,
+                    "code_bits_read_per_weight": prec,
                     "l2": f"{copies} packed copies in rotation, each read again after ~{(copies - 1) * nbytes / 1e6:.0f} MB"}
         del groups, ws
     L = wl.layer("gen_prefill_11008x4096_T2048", 11008, 4096, 2048, seed=3010, n_outlier_cols=20, S=S,

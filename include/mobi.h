@@ -67,6 +67,10 @@
  *          q(s,n,32w+i) in bit 2i and q(s,n,32w+16+i) in bit 2i+1 (i < 16): its
  *          even bits are the 2-bit layout's word 2w and its odd bits word
  *          2w+1, each code a 0/1 field. mobi_codes_bytes_bits() gives the size.
+ *          Slices of mixed widths (mobi_pack_slices): slice s in the layout of
+ *          its width, [N][K*width_s/32] words, the slices one after another
+ *          (slice s starts after the words of slices 0..s-1);
+ *          mobi_codes_bytes_slices() gives the size.
  *   sz     uint32 [S][K/G][N]    element (s,g,n): bits [15:0] = fp16 scale,
  *          bits [31:16] = fp16 zero (an integer 0..2^b - 1). mobi_sz_bytes().
  *          Group-major so that the scales of one group for consecutive rows
@@ -130,6 +134,8 @@ MOBI_API int mobi_version(void);
 MOBI_API size_t mobi_codes_bytes(int64_t N, int64_t K, int S);
 /* Bytes of the codes of S slices of `bits`-bit codes (1 or 2; K % 32 == 0). */
 MOBI_API size_t mobi_codes_bytes_bits(int64_t N, int64_t K, int S, int bits);
+/* Bytes of the codes of S slices of widths[s]-bit codes (each 1 or 2). */
+MOBI_API size_t mobi_codes_bytes_slices(int64_t N, int64_t K, int S, const int* widths);
 
 /* Bytes of the scale/zero array: S * N * (K/G) * 4. Returns 0 for invalid sizes. */
 MOBI_API size_t mobi_sz_bytes(int64_t N, int64_t K, int S, int G);
@@ -182,6 +188,20 @@ MOBI_API mobi_status mobi_pack(const void* W, int64_t N, int64_t K, int G, int S
  */
 MOBI_API mobi_status mobi_pack_bits(const void* W, int64_t N, int64_t K, int G, int S, int bits,
                                     uint32_t* codes, uint32_t* sz, void* stream);
+
+/*
+ * mobi_pack_slices — mobi_pack_bits with one width per slice: round s of the
+ *   recursion quantises the residual with widths[s]-bit codes (1 or 2,
+ *   L = 2^widths[s] - 1 steps), and each slice is stored in the layout of its
+ *   width, the slices one after another. Widths (2, 1, 1, 2) give 2, 3, 4 and
+ *   6 bits per weight from one packed layer, the precisions [en] §2.A lists.
+ *   widths   host array of S widths (read during the call only).
+ *   codes    out, mobi_codes_bytes_slices(N, K, S, widths) bytes.
+ *   Other arguments and errors as for mobi_pack_bits (an invalid width is
+ *   MOBI_ERR_INVALID_ARG).
+ */
+MOBI_API mobi_status mobi_pack_slices(const void* W, int64_t N, int64_t K, int G, int S, const int* widths,
+                                      uint32_t* codes, uint32_t* sz, void* stream);
 
 /*
  * mobi_route — MoBiRoute slice count per token and token bucketing.
@@ -289,6 +309,18 @@ MOBI_API mobi_status mobi_gemm_bits(const void* X, int64_t T, int64_t K, const i
                                     const uint32_t* sz, int64_t N, int G, int S, int bits, float* Y, void* ws,
                                     size_t ws_bytes, void* stream, int path);
 
+/*
+ * mobi_gemm_slices — mobi_gemm_bits for slices of mixed widths (widths[s]
+ *   for slice s, as written by mobi_pack_slices; a host array read during the
+ *   call). Every kernel reads each slice in the layout of its width. Same
+ *   arguments, result and workspace otherwise; MOBI_ERR_INVALID_ARG for a
+ *   width other than 1 or 2.
+ */
+MOBI_API mobi_status mobi_gemm_slices(const void* X, int64_t T, int64_t K, const int32_t* k_t,
+                                      const int32_t* perm, const int32_t* offsets, const uint32_t* codes,
+                                      const uint32_t* sz, int64_t N, int G, int S, const int* widths, float* Y,
+                                      void* ws, size_t ws_bytes, void* stream, int path);
+
 /* Scratch bytes of mobi_linear: the routing workspace (rounded up to 256
  * bytes) followed by the GEMM workspace. */
 MOBI_API size_t mobi_linear_workspace_bytes(int64_t T, int64_t N, int64_t K, int S);
@@ -321,6 +353,13 @@ MOBI_API mobi_status mobi_linear_bits(const void* X, int64_t T, int64_t K, const
                                       const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S, int bits,
                                       int32_t* k_t, int32_t* perm, int32_t* offsets, float* Y, void* ws,
                                       size_t ws_bytes, void* stream);
+
+/* mobi_linear for slices of mixed widths (widths[s] for slice s), as
+ * mobi_gemm_slices is to mobi_gemm_path. */
+MOBI_API mobi_status mobi_linear_slices(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
+                                        const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S,
+                                        const int* widths, int32_t* k_t, int32_t* perm, int32_t* offsets,
+                                        float* Y, void* ws, size_t ws_bytes, void* stream);
 
 /* One problem of mobi_linear_grouped: the arguments of one mobi_linear call. */
 typedef struct mobi_linear_problem {
@@ -372,6 +411,11 @@ MOBI_API mobi_status mobi_gemm_grouped(const mobi_gemm_problem* problems, int co
 MOBI_API mobi_status mobi_gemm_grouped_bits(const mobi_gemm_problem* problems, int count, int G, int S, int bits,
                                             void* ws, size_t ws_bytes, void* stream);
 
+/* mobi_gemm_grouped for slices of mixed widths (every problem of the call has
+ * the widths `widths`). */
+MOBI_API mobi_status mobi_gemm_grouped_slices(const mobi_gemm_problem* problems, int count, int G, int S,
+                                              const int* widths, void* ws, size_t ws_bytes, void* stream);
+
 /*
  * mobi_linear_grouped — up to MOBI_MAX_GROUP independent decode-sized
  *   mobi_linear problems (every T <= 16) in one step: the projections of a
@@ -399,6 +443,11 @@ MOBI_API mobi_status mobi_linear_grouped(const mobi_linear_problem* problems, in
  * the call has that width). */
 MOBI_API mobi_status mobi_linear_grouped_bits(const mobi_linear_problem* problems, int count, int G, int S,
                                               int bits, void* ws, size_t ws_bytes, void* stream);
+
+/* mobi_linear_grouped for slices of mixed widths (every problem of the call
+ * has the widths `widths`). */
+MOBI_API mobi_status mobi_linear_grouped_slices(const mobi_linear_problem* problems, int count, int G, int S,
+                                                const int* widths, void* ws, size_t ws_bytes, void* stream);
 
 /* ---- many-in-one checkpoints of packed layers -------------------------------
  *

@@ -49,6 +49,8 @@ def test_status_strings_and_sizes(L):
     assert mobi.mobi_codes_bytes(16, 100, 3) == 0  # K % 32 != 0
     assert mobi.mobi_codes_bytes(4096, 4096, 4, bits=1) == 4 * 4096 * 128 * 4  # 1-bit codes: 32 per word
     assert L.mobi_codes_bytes_bits(4096, 4096, 3, 3) == 0
+    assert mobi.mobi_codes_bytes(4096, 4096, widths=(2, 1, 1, 2)) == 4096 * 4096 * 6 // 8  # 2+1+1+2 bits
+    assert mobi.mobi_codes_bytes(4096, 4096, widths=(2, 3)) == 0
     assert mobi.mobi_gemm_workspace_bytes(16, 4096, 4096, 3) > 0
 
 
@@ -105,6 +107,18 @@ def test_gemm_validation(L):
     assert call_bits(1, T=0) == 0
     prob = mobi.GemmProblem(p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE), 4, 64, 256)
     assert L.mobi_gemm_grouped_bits(ctypes.byref(prob), 1, 128, 3, 4, p(FAKE), 1 << 30, None) == 1
+
+    def call_slices(widths, T=16, K=256, N=64, S=None):
+        w = mobi._int_array(widths)
+        S = len(widths) if S is None else S
+        return L.mobi_gemm_slices(p(FAKE), T, K, p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE), N, 128, S, w,
+                                  p(FAKE), p(FAKE), 1 << 30, None, 0)
+    assert call_slices((2, 0, 1)) == 1 and call_slices((2, 3)) == 1 and call_slices((2, 1), S=5) == 1
+    assert call_slices((2, 1), K=200) == 2
+    assert call_slices((2, 1, 1, 2), T=0) == 0
+    assert L.mobi_gemm_slices(p(FAKE), 16, 256, p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE), 64, 128, 2, None,
+                              p(FAKE), p(FAKE), 1 << 30, None, 0) == 1  # widths missing
+    assert L.mobi_pack_slices(p(FAKE), 16, 256, 128, 2, mobi._int_array((2, 4)), p(FAKE), p(FAKE), None) == 1
 
 
 def test_linear_validation(L):

@@ -172,3 +172,74 @@ def test_four_slice_threshold_routing(mobi, oracle):
     perm_ref, off_ref = oracle.bucket(k_gpu, 4)
     assert np.array_equal(perm.cpu().numpy(), perm_ref) and np.array_equal(off.cpu().numpy(), off_ref)
     assert k_gpu.max() == 4 and len(set(k_gpu.tolist())) >= 3
+
+
+# ---- slices of mixed widths in one layer ---------------------------------------
+
+MIXED = (2, 1, 1, 2)  # 2, 3, 4 and 6 bits per weight
+
+
+@pytest.mark.parametrize("widths,N,K", [(MIXED, 256, 1024), ((1, 2), 80, 1152), ((2, 1, 2), 208, 4096)])
+def test_pack_slices_bit_exact(mobi, oracle, widths, N, K):
+    L = wl.layer("ps", N, K, 1, seed=2500 + N + len(widths), outlier_frac_cols=0.01)
+    codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(DEV), widths=widths)
+    torch.cuda.synchronize()
+    c_ref, s_ref, _ = oracle.pack_slices(L.W, widths)
+    assert codes.numel() * 4 == mobi.mobi_codes_bytes(N, K, widths=widths) == c_ref.size * 4
+    assert np.array_equal(codes.cpu().numpy().view(np.uint32), c_ref)
+    assert np.array_equal(sz.cpu().numpy().view(np.uint32), s_ref)
+
+
+@pytest.mark.parametrize("T", [1, 6, 16, 130])
+@pytest.mark.parametrize("widths", [MIXED, (1, 2)])
+def test_mixed_gemm_both_kernels(mobi, oracle, T, widths):
+    """Mixed widths through both kernels with an explicit path: K = 1152 ends
+    in a ragged 1024-column chunk, N = 208 in a partial 128-row tile; k_t over
+    1..S, so every slice width is read."""
+    S = len(widths)
+    N, K = 208, 1152
+    L = wl.layer("mx", N, K, T, seed=2600 + T + 10 * S, outlier_frac_cols=0.01)
+    codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(DEV), widths=widths)
+    c_ref, s_ref, _ = oracle.pack_slices(L.W, widths)
+    assert np.array_equal(codes.cpu().numpy().view(np.uint32), c_ref)
+    k = np.random.default_rng(T + S).integers(1, S + 1, T).astype(np.int32)
+    perm_np, off_np = oracle.bucket(k, S)
+    ref = oracle.gemm(L.X, k, c_ref, s_ref, N, S=S, widths=widths)
+    for path in ([1, 2] if T <= 16 else [2]):
+        Y = mobi.mobi_gemm_path(L.X.to(DEV), torch.from_numpy(k).to(DEV), torch.from_numpy(perm_np).to(DEV),
+                                torch.from_numpy(off_np).to(DEV), codes, sz, N, path=path, widths=widths)
+        mobi.mobi_sync_check()
+        check_gemm(Y.cpu().numpy(), ref, f"widths={widths} T={T} path={path}")
+
+
+def test_mixed_linear_and_grouped(mobi, oracle):
+    """Route + GEMM with widths (2, 1, 1, 2) (2, 3, 4, 6 bits): single calls and
+    one grouped call over both fragment classes; grouped results equal single
+    calls bit for bit and meet the oracle."""
+    S = 4
+    specs = [(512, 2048, 4), (256, 1024, 16), (4096, 4096, 8)]
+    probs, layers = [], []
+    for i, (N, K, T) in enumerate(specs):
+        L = _layer_s("lm", N, K, T, S, seed=2700 + i)
+        codes, sz = mobi.mobi_pack(torch.from_numpy(L.W).to(DEV), widths=MIXED)
+        layers.append(L)
+        probs.append({"X": L.X.to(DEV), "Wr": torch.from_numpy(L.Wr).to(DEV), "bias": torch.from_numpy(L.bias).to(DEV),
+                      "codes": codes, "sz": sz, "N": N})
+    outs = mobi.mobi_linear_grouped(probs, S=S, widths=MIXED)
+    mobi.mobi_sync_check()
+    for pr, L, (Y, k_t, perm, off) in zip(probs, layers, outs):
+        Ys, ks, _, _ = mobi.mobi_linear(pr["X"], pr["Wr"], pr["bias"], pr["codes"], pr["sz"], pr["N"], widths=MIXED)
+        mobi.mobi_sync_check()
+        assert torch.equal(Y, Ys) and torch.equal(k_t, ks)
+        c_ref, s_ref, _ = oracle.pack_slices(L.W, MIXED)
+        k_gpu = k_t.cpu().numpy()
+        k_ref, gap, _ = oracle.route(L.X, L.Wr, L.bias)
+        check_route(k_gpu, k_ref, gap, f"mixed N={pr['N']}")
+        check_gemm(Y.cpu().numpy(), oracle.gemm(L.X, k_gpu, c_ref, s_ref, pr["N"], S=S, widths=MIXED),
+                   f"mixed linear N={pr['N']} T={L.T}")
+    # the GEMM half alone, k_t given
+    gp = [{"X": pr["X"], "k_t": o[1], "codes": pr["codes"], "sz": pr["sz"], "N": pr["N"]} for pr, o in zip(probs, outs)]
+    Yg = mobi.mobi_gemm_grouped(gp, S=S, widths=MIXED)
+    mobi.mobi_sync_check()
+    for y, o in zip(Yg, outs):
+        assert torch.equal(y, o[0])

@@ -77,6 +77,8 @@ EXPORTED_SYMBOLS = (
     "mobi_ckpt_save", "mobi_ckpt_open", "mobi_ckpt_count", "mobi_ckpt_find", "mobi_ckpt_info", "mobi_ckpt_load",
     "mobi_ckpt_bytes_read", "mobi_ckpt_close", "mobi_crc32c", "mobi_pack_bits", "mobi_codes_bytes_bits",
     "mobi_gemm_bits", "mobi_gemm_grouped_bits", "mobi_linear_bits", "mobi_linear_grouped_bits",
+    "mobi_codes_bytes_slices", "mobi_pack_slices", "mobi_gemm_slices", "mobi_linear_slices",
+    "mobi_gemm_grouped_slices", "mobi_linear_grouped_slices",
 )
 
 
@@ -109,6 +111,18 @@ def lib() -> ctypes.CDLL:
         L.mobi_codes_bytes.restype = sz_t
         L.mobi_codes_bytes_bits.argtypes = [i64, i64, ci, ci]
         L.mobi_codes_bytes_bits.restype = sz_t
+        L.mobi_codes_bytes_slices.argtypes = [i64, i64, ci, p]
+        L.mobi_codes_bytes_slices.restype = sz_t
+        L.mobi_pack_slices.argtypes = [p, i64, i64, ci, ci, p, p, p, p]
+        L.mobi_pack_slices.restype = ci
+        L.mobi_gemm_slices.argtypes = [p, i64, i64, p, p, p, p, p, i64, ci, ci, p, p, p, sz_t, p, ci]
+        L.mobi_gemm_slices.restype = ci
+        L.mobi_linear_slices.argtypes = [p, i64, i64, p, p, p, p, i64, ci, ci, p, p, p, p, p, p, sz_t, p]
+        L.mobi_linear_slices.restype = ci
+        L.mobi_gemm_grouped_slices.argtypes = [p, ci, ci, ci, p, p, sz_t, p]
+        L.mobi_gemm_grouped_slices.restype = ci
+        L.mobi_linear_grouped_slices.argtypes = [p, ci, ci, ci, p, p, sz_t, p]
+        L.mobi_linear_grouped_slices.restype = ci
         L.mobi_sz_bytes.argtypes = [i64, i64, ci, ci]
         L.mobi_sz_bytes.restype = sz_t
         L.mobi_route_workspace_bytes.argtypes = [i64, i64, ci]
@@ -212,7 +226,14 @@ def mobi_last_error() -> str:
     return lib().mobi_last_error().decode(errors="replace")
 
 
-def mobi_codes_bytes(N: int, K: int, S: int = 3, bits: int = 2) -> int:
+def _int_array(vals):
+    """A host int32 array for an `const int*` argument (kept alive by the caller)."""
+    return (ctypes.c_int * len(vals))(*[int(v) for v in vals])
+
+
+def mobi_codes_bytes(N: int, K: int, S: int = 3, bits: int = 2, widths=None) -> int:
+    if widths is not None:
+        return lib().mobi_codes_bytes_slices(N, K, len(widths), _int_array(widths))
     return lib().mobi_codes_bytes_bits(N, K, S, bits)
 
 
@@ -235,7 +256,7 @@ def _workspace(nbytes: int, device, ws: torch.Tensor | None) -> torch.Tensor:
 
 
 def mobi_pack(W: torch.Tensor, S: int = 3, G: int = 128, codes: torch.Tensor | None = None,
-              sz: torch.Tensor | None = None, stream=None, bits: int = 2):
+              sz: torch.Tensor | None = None, stream=None, bits: int = 2, widths=None):
     """MoBiSlice packing of fp16 W[N,K] -> (codes int32 [S,N,K*bits/32], sz int32 [S,K/128,N]).
     bits = 2 and G = 128 is the method's slicing (mobi_pack); other values go
     through mobi_pack_bits (bits 1 or 2, G 128/256/512, S up to 4; 1-bit codes
@@ -243,6 +264,17 @@ def mobi_pack(W: torch.Tensor, S: int = 3, G: int = 128, codes: torch.Tensor | N
     if W.dtype != torch.float16 or W.dim() != 2:
         raise ValueError("W must be a 2-D fp16 tensor")
     N, K = W.shape
+    if widths is not None:  # one width per slice: codes are one flat array of every slice's words
+        S = len(widths)
+        wa = _int_array(widths)
+        if codes is None:
+            codes = torch.empty(max(mobi_codes_bytes(N, K, widths=widths) // 4, 1), dtype=torch.int32,
+                                device=W.device)
+        if sz is None:
+            sz = torch.empty((S, K // 128, N), dtype=torch.int32, device=W.device)
+        _check("mobi_pack_slices", lib().mobi_pack_slices(_ptr(W), N, K, G, S, wa, _ptr(codes), _ptr(sz),
+                                                          _stream(stream)))
+        return codes, sz
     if codes is None:
         codes = torch.empty((S, N, K * bits // 32), dtype=torch.int32, device=W.device)
     if sz is None:
@@ -333,7 +365,7 @@ def mobi_linear_grouped_workspace_bytes(problems, S: int = 3) -> int:
 
 
 def mobi_linear_grouped(problems, S: int = 3, G: int = 128, ws: torch.Tensor | None = None, stream=None,
-                        bits: int = 2):
+                        bits: int = 2, widths=None):
     """Up to MAX_GROUP independent decode-sized (T <= 16) mobi_linear problems in one step.
     Each problem is a dict with X, Wr, codes, sz, N (and optionally bias, Y, k_t, perm, offsets);
     `bits` is the code width of every slice. Returns [(Y, k_t, perm, offsets)] in problem order."""
@@ -342,8 +374,15 @@ def mobi_linear_grouped(problems, S: int = 3, G: int = 128, ws: torch.Tensor | N
         raise ValueError("mobi_linear_grouped needs at least one problem")
     need = lib().mobi_linear_grouped_workspace_bytes(arr, len(filled), S)
     ws = _workspace(need, filled[0]["X"].device, ws) if need > 0 else ws
-    _check("mobi_linear_grouped", lib().mobi_linear_grouped_bits(arr, len(filled), G, S, bits, _ptr(ws),
-                                                                 0 if ws is None else ws.numel(), _stream(stream)))
+    if widths is not None:
+        _check("mobi_linear_grouped", lib().mobi_linear_grouped_slices(arr, len(filled), G, len(widths),
+                                                                       _int_array(widths), _ptr(ws),
+                                                                       0 if ws is None else ws.numel(),
+                                                                       _stream(stream)))
+    else:
+        _check("mobi_linear_grouped", lib().mobi_linear_grouped_bits(arr, len(filled), G, S, bits, _ptr(ws),
+                                                                     0 if ws is None else ws.numel(),
+                                                                     _stream(stream)))
     return [(d["Y"], d["k_t"], d["perm"], d["offsets"]) for d in filled]
 
 
@@ -367,7 +406,7 @@ def mobi_gemm_grouped_workspace_bytes(problems, S: int = 3) -> int:
 
 
 def mobi_gemm_grouped(problems, S: int = 3, G: int = 128, ws: torch.Tensor | None = None, stream=None,
-                      bits: int = 2):
+                      bits: int = 2, widths=None):
     """Up to MAX_GROUP decode-sized mobi_gemm problems (dicts with X, k_t, codes, sz, N and
     optionally Y) in one launch per fragment class; `bits` is the code width of every
     slice (mobi_gemm_grouped_bits). Returns [Y] in problem order."""
@@ -376,8 +415,13 @@ def mobi_gemm_grouped(problems, S: int = 3, G: int = 128, ws: torch.Tensor | Non
         raise ValueError("mobi_gemm_grouped needs at least one problem")
     need = lib().mobi_gemm_grouped_workspace_bytes(arr, len(filled), S)
     ws = _workspace(need, filled[0]["X"].device, ws) if need > 0 else ws
-    _check("mobi_gemm_grouped", lib().mobi_gemm_grouped_bits(arr, len(filled), G, S, bits, _ptr(ws),
-                                                             0 if ws is None else ws.numel(), _stream(stream)))
+    if widths is not None:
+        _check("mobi_gemm_grouped", lib().mobi_gemm_grouped_slices(arr, len(filled), G, len(widths),
+                                                                   _int_array(widths), _ptr(ws),
+                                                                   0 if ws is None else ws.numel(), _stream(stream)))
+    else:
+        _check("mobi_gemm_grouped", lib().mobi_gemm_grouped_bits(arr, len(filled), G, S, bits, _ptr(ws),
+                                                                 0 if ws is None else ws.numel(), _stream(stream)))
     return [d["Y"] for d in filled]
 
 
@@ -494,22 +538,28 @@ class MobiCheckpoint:
 def mobi_gemm_path(X: torch.Tensor, k_t: torch.Tensor, perm: torch.Tensor, offsets: torch.Tensor,
                    codes: torch.Tensor, sz: torch.Tensor, N: int, path: int = PATH_AUTO, S: int | None = None,
                    G: int = 128, Y: torch.Tensor | None = None, ws: torch.Tensor | None = None, stream=None,
-                   bits: int = 2):
+                   bits: int = 2, widths=None):
     """Token-routed mixed-bit GEMM y_t = x_t . W^(k_t)^T (fp32) with an explicit kernel choice
     and the code width of the slices (mobi_gemm_bits)."""
     T, K = X.shape
-    S = codes.shape[0] if S is None else S
+    S = (len(widths) if widths is not None else codes.shape[0]) if S is None else S
     Y = torch.empty((T, N), dtype=torch.float32, device=X.device) if Y is None else Y
     ws = _workspace(mobi_gemm_workspace_bytes(T, N, K, S), X.device, ws)
-    _check("mobi_gemm", lib().mobi_gemm_bits(_ptr(X), T, K, _ptr(k_t), _ptr(perm), _ptr(offsets), _ptr(codes),
-                                             _ptr(sz), N, G, S, bits, _ptr(Y), _ptr(ws), ws.numel(),
-                                             _stream(stream), path))
+    if widths is not None:
+        _check("mobi_gemm", lib().mobi_gemm_slices(_ptr(X), T, K, _ptr(k_t), _ptr(perm), _ptr(offsets), _ptr(codes),
+                                                   _ptr(sz), N, G, S, _int_array(widths), _ptr(Y), _ptr(ws),
+                                                   ws.numel(), _stream(stream), path))
+    else:
+        _check("mobi_gemm", lib().mobi_gemm_bits(_ptr(X), T, K, _ptr(k_t), _ptr(perm), _ptr(offsets), _ptr(codes),
+                                                 _ptr(sz), N, G, S, bits, _ptr(Y), _ptr(ws), ws.numel(),
+                                                 _stream(stream), path))
     return Y
 
 
-def mobi_gemm(X, k_t, perm, offsets, codes, sz, N, S=None, G=128, Y=None, ws=None, stream=None, bits=2):
+def mobi_gemm(X, k_t, perm, offsets, codes, sz, N, S=None, G=128, Y=None, ws=None, stream=None, bits=2,
+              widths=None):
     """Token-routed mixed-bit GEMM (decode kernel for T <= 16, tcgen05 prefill kernel above)."""
-    return mobi_gemm_path(X, k_t, perm, offsets, codes, sz, N, PATH_AUTO, S, G, Y, ws, stream, bits)
+    return mobi_gemm_path(X, k_t, perm, offsets, codes, sz, N, PATH_AUTO, S, G, Y, ws, stream, bits, widths)
 
 
 def mobi_gemm_decode_noalloc(X, k_t, codes, sz, N, S=None, G=128, Y=None, stream=None):
@@ -527,7 +577,7 @@ def mobi_linear_workspace_bytes(T: int, N: int, K: int, S: int = 3) -> int:
 
 
 def mobi_linear(X, Wr, bias, codes, sz, N, G=128, Y=None, k_t=None, perm=None, offsets=None, ws=None, stream=None,
-                bits=2):
+                bits=2, widths=None):
     """Route + mixed-bit GEMM in one call (S = Wr.shape[1], slices of `bits`-bit codes)
     -> (Y fp32 [T,N], k_t, perm, offsets)."""
     if X.dtype != torch.bfloat16 or Wr.dtype != torch.float32:
@@ -540,9 +590,17 @@ def mobi_linear(X, Wr, bias, codes, sz, N, G=128, Y=None, k_t=None, perm=None, o
     perm = torch.empty(T, dtype=torch.int32, device=dev) if perm is None else perm
     offsets = torch.empty(S + 1, dtype=torch.int32, device=dev) if offsets is None else offsets
     ws = _workspace(mobi_linear_workspace_bytes(T, N, K, S), dev, ws)
-    _check("mobi_linear", lib().mobi_linear_bits(_ptr(X), T, K, _ptr(Wr), _ptr(bias), _ptr(codes), _ptr(sz), N, G,
-                                                 S, bits, _ptr(k_t), _ptr(perm), _ptr(offsets), _ptr(Y), _ptr(ws),
-                                                 ws.numel(), _stream(stream)))
+    if widths is not None:
+        if len(widths) != S:
+            raise ValueError("one width per slice (the router's column count)")
+        _check("mobi_linear", lib().mobi_linear_slices(_ptr(X), T, K, _ptr(Wr), _ptr(bias), _ptr(codes), _ptr(sz),
+                                                       N, G, S, _int_array(widths), _ptr(k_t), _ptr(perm),
+                                                       _ptr(offsets), _ptr(Y), _ptr(ws), ws.numel(),
+                                                       _stream(stream)))
+    else:
+        _check("mobi_linear", lib().mobi_linear_bits(_ptr(X), T, K, _ptr(Wr), _ptr(bias), _ptr(codes), _ptr(sz), N,
+                                                     G, S, bits, _ptr(k_t), _ptr(perm), _ptr(offsets), _ptr(Y),
+                                                     _ptr(ws), ws.numel(), _stream(stream)))
     return Y, k_t, perm, offsets
 
 

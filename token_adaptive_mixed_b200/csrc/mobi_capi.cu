@@ -29,11 +29,11 @@ cudaError_t launch_route_mlp(const void* X, int64_t T, int64_t K, const float* W
 size_t route_mlp_ws_bytes(int64_t T, int64_t K, int64_t H, int sms);
 cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
                           const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
-                          DeviceStatus* st, bool early, int bits);
+                          DeviceStatus* st, bool early, int bits, int mask1);
 size_t decode_ws_bytes(int64_t N, int64_t K);
 cudaError_t launch_prefill(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
                            const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int S,
-                           float* Y, void* ws, cudaStream_t stream, DeviceStatus* st, int bits);
+                           float* Y, void* ws, cudaStream_t stream, DeviceStatus* st, int bits, int mask1);
 size_t prefill_ws_bytes(int64_t T, int64_t N, int64_t K);
 
 static thread_local char g_last_error[256];
@@ -266,11 +266,40 @@ const char* mobi_last_error(void) { return g_last_error; }
 
 int mobi_version(void) { return 100; }
 
+namespace {
+// Width mode of S slices: 2 or 1 when every slice has that width, 3 when they
+// differ; mask1 has bit s set when slice s is 1-bit. False for an invalid
+// width or S.
+bool width_mode(int S, const int* widths, int* mode, int* mask1) {
+  if (S < 1 || S > mobi::kMaxSlices || !widths) return false;
+  int m = 0, n1 = 0;
+  for (int j = 0; j < S; ++j) {
+    if (widths[j] != 1 && widths[j] != 2) return false;
+    if (widths[j] == 1) {
+      m |= 1 << j;
+      ++n1;
+    }
+  }
+  *mask1 = m;
+  *mode = n1 == 0 ? 2 : (n1 == S ? 1 : 3);
+  return true;
+}
+int uniform_mask(int bits, int S) { return bits == 1 ? (1 << S) - 1 : 0; }
+}  // namespace
+
 size_t mobi_codes_bytes(int64_t N, int64_t K, int S) { return mobi_codes_bytes_bits(N, K, S, 2); }
 
 size_t mobi_codes_bytes_bits(int64_t N, int64_t K, int S, int bits) {
   if (N < 0 || K < 0 || K % 32 != 0 || S < 1 || S > kMaxSlices || bits < 1 || bits > 2) return 0;
   return (size_t)S * (size_t)N * (size_t)(K / 32 * bits) * 4;
+}
+
+size_t mobi_codes_bytes_slices(int64_t N, int64_t K, int S, const int* widths) {
+  int mode = 0, mask1 = 0;
+  if (N < 0 || K < 0 || K % 32 != 0 || !width_mode(S, widths, &mode, &mask1)) return 0;
+  size_t words = 0;
+  for (int j = 0; j < S; ++j) words += (size_t)N * (size_t)(K / 32 * widths[j]);
+  return words * 4;
 }
 
 size_t mobi_sz_bytes(int64_t N, int64_t K, int S, int G) {
@@ -299,7 +328,7 @@ mobi_status mobi_pack(const void* W, int64_t N, int64_t K, int G, int S, uint32_
   if (N == 0 || K == 0) return MOBI_OK;
   if (!W || !codes || !sz) return MOBI_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(codes) || !aligned16(sz)) return MOBI_ERR_MISALIGNED;
-  return cuda_status(launch_pack(W, N, K, S, codes, sz, static_cast<cudaStream_t>(stream), num_sms(), 2, 128));
+  return cuda_status(launch_pack(W, N, K, S, codes, sz, static_cast<cudaStream_t>(stream), num_sms(), 0, 128));
 }
 
 mobi_status mobi_pack_bits(const void* W, int64_t N, int64_t K, int G, int S, int bits, uint32_t* codes,
@@ -313,7 +342,23 @@ mobi_status mobi_pack_bits(const void* W, int64_t N, int64_t K, int G, int S, in
   if (N == 0 || K == 0) return MOBI_OK;
   if (!W || !codes || !sz) return MOBI_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(codes) || !aligned16(sz)) return MOBI_ERR_MISALIGNED;
-  return cuda_status(launch_pack(W, N, K, S, codes, sz, static_cast<cudaStream_t>(stream), num_sms(), bits, G));
+  return cuda_status(
+      launch_pack(W, N, K, S, codes, sz, static_cast<cudaStream_t>(stream), num_sms(), uniform_mask(bits, S), G));
+}
+
+mobi_status mobi_pack_slices(const void* W, int64_t N, int64_t K, int G, int S, const int* widths, uint32_t* codes,
+                             uint32_t* sz, void* stream) {
+  g_last_error[0] = 0;
+  int mode = 0, mask1 = 0;
+  if (!width_mode(S, widths, &mode, &mask1)) return MOBI_ERR_INVALID_ARG;
+  if (G != 128 && G != 256 && G != 512) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  mobi_status st = check_matrix(N, K, 128, S);
+  if (st != MOBI_OK) return st;
+  if (K % G != 0) return MOBI_ERR_UNSUPPORTED_SHAPE;
+  if (N == 0 || K == 0) return MOBI_OK;
+  if (!W || !codes || !sz) return MOBI_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(codes) || !aligned16(sz)) return MOBI_ERR_MISALIGNED;
+  return cuda_status(launch_pack(W, N, K, S, codes, sz, static_cast<cudaStream_t>(stream), num_sms(), mask1, G));
 }
 
 mobi_status mobi_route(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias, int S,
@@ -367,11 +412,10 @@ mobi_status mobi_gemm_path(const void* X, int64_t T, int64_t K, const int32_t* k
   return mobi_gemm_bits(X, T, K, k_t, perm, offsets, codes, sz, N, G, S, 2, Y, ws, ws_bytes, stream, path);
 }
 
-mobi_status mobi_gemm_bits(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
-                           const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int G,
-                           int S, int bits, float* Y, void* ws, size_t ws_bytes, void* stream, int path) {
-  g_last_error[0] = 0;
-  if (bits < 1 || bits > 2) return MOBI_ERR_INVALID_ARG;
+static mobi_status gemm_impl(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
+                             const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int G,
+                             int S, int bits, int mask1, float* Y, void* ws, size_t ws_bytes, void* stream,
+                             int path) {
   mobi_status st = check_matrix(N, K, G, S);
   if (st != MOBI_OK) return st;
   if (T < 0) return MOBI_ERR_INVALID_ARG;
@@ -391,8 +435,28 @@ mobi_status mobi_gemm_bits(const void* X, int64_t T, int64_t K, const int32_t* k
   DeviceStatus* dst = device_status(&e);
   if (!dst) return cuda_status(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (decode) return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, ws, s, dst, false, bits));
-  return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, ws, s, dst, bits));
+  if (decode)
+    return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, ws, s, dst, false, bits, mask1));
+  return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, ws, s, dst, bits, mask1));
+}
+
+mobi_status mobi_gemm_bits(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
+                           const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int G,
+                           int S, int bits, float* Y, void* ws, size_t ws_bytes, void* stream, int path) {
+  g_last_error[0] = 0;
+  if (bits < 1 || bits > 2) return MOBI_ERR_INVALID_ARG;
+  return gemm_impl(X, T, K, k_t, perm, offsets, codes, sz, N, G, S, bits, uniform_mask(bits, S), Y, ws, ws_bytes,
+                   stream, path);
+}
+
+mobi_status mobi_gemm_slices(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
+                             const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int G,
+                             int S, const int* widths, float* Y, void* ws, size_t ws_bytes, void* stream,
+                             int path) {
+  g_last_error[0] = 0;
+  int mode = 0, mask1 = 0;
+  if (!width_mode(S, widths, &mode, &mask1)) return MOBI_ERR_INVALID_ARG;
+  return gemm_impl(X, T, K, k_t, perm, offsets, codes, sz, N, G, S, mode, mask1, Y, ws, ws_bytes, stream, path);
 }
 
 size_t mobi_linear_workspace_bytes(int64_t T, int64_t N, int64_t K, int S) {
@@ -406,12 +470,10 @@ mobi_status mobi_linear(const void* X, int64_t T, int64_t K, const float* Wr, co
   return mobi_linear_bits(X, T, K, Wr, bias, codes, sz, N, G, S, 2, k_t, perm, offsets, Y, ws, ws_bytes, stream);
 }
 
-mobi_status mobi_linear_bits(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
-                             const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S, int bits,
-                             int32_t* k_t, int32_t* perm, int32_t* offsets, float* Y, void* ws, size_t ws_bytes,
-                             void* stream) {
-  g_last_error[0] = 0;
-  if (bits < 1 || bits > 2) return MOBI_ERR_INVALID_ARG;
+static mobi_status linear_impl(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
+                               const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S, int bits,
+                               int mask1, int32_t* k_t, int32_t* perm, int32_t* offsets, float* Y, void* ws,
+                               size_t ws_bytes, void* stream) {
   mobi_status st = check_matrix(N, K, G, S);
   if (st != MOBI_OK) return st;
   if (T < 0) return MOBI_ERR_INVALID_ARG;
@@ -436,8 +498,30 @@ mobi_status mobi_linear_bits(const void* X, int64_t T, int64_t K, const float* W
   void* gws = static_cast<uint8_t*>(ws) + route_ws;
   // For up to 16 tokens the decode kernel is a programmatic dependent of the
   // routing kernel just launched: its launch and set-up overlap the routing.
-  if (decode) return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, gws, s, dst, true, bits));
-  return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, gws, s, dst, bits));
+  if (decode)
+    return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, gws, s, dst, true, bits, mask1));
+  return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, gws, s, dst, bits, mask1));
+}
+
+mobi_status mobi_linear_bits(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
+                             const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S, int bits,
+                             int32_t* k_t, int32_t* perm, int32_t* offsets, float* Y, void* ws, size_t ws_bytes,
+                             void* stream) {
+  g_last_error[0] = 0;
+  if (bits < 1 || bits > 2) return MOBI_ERR_INVALID_ARG;
+  return linear_impl(X, T, K, Wr, bias, codes, sz, N, G, S, bits, uniform_mask(bits, S), k_t, perm, offsets, Y, ws,
+                     ws_bytes, stream);
+}
+
+mobi_status mobi_linear_slices(const void* X, int64_t T, int64_t K, const float* Wr, const float* bias,
+                               const uint32_t* codes, const uint32_t* sz, int64_t N, int G, int S, const int* widths,
+                               int32_t* k_t, int32_t* perm, int32_t* offsets, float* Y, void* ws, size_t ws_bytes,
+                               void* stream) {
+  g_last_error[0] = 0;
+  int mode = 0, mask1 = 0;
+  if (!width_mode(S, widths, &mode, &mask1)) return MOBI_ERR_INVALID_ARG;
+  return linear_impl(X, T, K, Wr, bias, codes, sz, N, G, S, mode, mask1, k_t, perm, offsets, Y, ws, ws_bytes,
+                     stream);
 }
 
 static_assert(MOBI_MAX_GROUP == kMaxGroup, "group size of the header and the kernels");
@@ -474,10 +558,8 @@ mobi_status mobi_linear_grouped(const mobi_linear_problem* problems, int count, 
   return mobi_linear_grouped_bits(problems, count, G, S, 2, ws, ws_bytes, stream);
 }
 
-mobi_status mobi_linear_grouped_bits(const mobi_linear_problem* problems, int count, int G, int S, int bits,
-                                     void* ws, size_t ws_bytes, void* stream) {
-  g_last_error[0] = 0;
-  if (bits < 1 || bits > 2) return MOBI_ERR_INVALID_ARG;
+static mobi_status linear_grouped_impl(const mobi_linear_problem* problems, int count, int G, int S, int bits,
+                                       int mask1, void* ws, size_t ws_bytes, void* stream) {
   size_t need = 0;
   mobi_status st = check_grouped(problems, count, G, S, &need);
   if (st != MOBI_OK) return st;
@@ -495,7 +577,7 @@ mobi_status mobi_linear_grouped_bits(const mobi_linear_problem* problems, int co
     const mobi_linear_problem& p = problems[i];
     rg.p[i] = RouteSmallProblem{static_cast<const __nv_bfloat16*>(p.X), p.Wr, p.bias, p.k_t, p.perm, p.offsets, p.K,
                                 (int)p.T};
-    jobs[i] = DecodeJob{p.X, p.k_t, p.codes, p.sz, p.Y, nullptr, p.N, p.K, (int)p.T, bits};
+    jobs[i] = DecodeJob{p.X, p.k_t, p.codes, p.sz, p.Y, nullptr, p.N, p.K, (int)p.T, bits, mask1};
     if (p.T > 0 && p.N > 0) {
       jobs[i].partial = reinterpret_cast<float*>(w);
       w += align256(decode_ws_bytes(p.N, p.K));
@@ -506,6 +588,21 @@ mobi_status mobi_linear_grouped_bits(const mobi_linear_problem* problems, int co
   // As in mobi_linear: the decode launches are programmatic dependents of the
   // routing launch.
   return cuda_status(launch_decode_grouped(jobs, count, S, s, dst, true));
+}
+
+mobi_status mobi_linear_grouped_bits(const mobi_linear_problem* problems, int count, int G, int S, int bits,
+                                     void* ws, size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  if (bits < 1 || bits > 2) return MOBI_ERR_INVALID_ARG;
+  return linear_grouped_impl(problems, count, G, S, bits, uniform_mask(bits, S), ws, ws_bytes, stream);
+}
+
+mobi_status mobi_linear_grouped_slices(const mobi_linear_problem* problems, int count, int G, int S,
+                                       const int* widths, void* ws, size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  int mode = 0, mask1 = 0;
+  if (!width_mode(S, widths, &mode, &mask1)) return MOBI_ERR_INVALID_ARG;
+  return linear_grouped_impl(problems, count, G, S, mode, mask1, ws, ws_bytes, stream);
 }
 
 static mobi_status check_gemm_grouped(const mobi_gemm_problem* problems, int count, int G, int S, size_t* need) {
@@ -538,10 +635,8 @@ mobi_status mobi_gemm_grouped(const mobi_gemm_problem* problems, int count, int 
   return mobi_gemm_grouped_bits(problems, count, G, S, 2, ws, ws_bytes, stream);
 }
 
-mobi_status mobi_gemm_grouped_bits(const mobi_gemm_problem* problems, int count, int G, int S, int bits, void* ws,
-                                   size_t ws_bytes, void* stream) {
-  g_last_error[0] = 0;
-  if (bits < 1 || bits > 2) return MOBI_ERR_INVALID_ARG;
+static mobi_status gemm_grouped_impl(const mobi_gemm_problem* problems, int count, int G, int S, int bits,
+                                     int mask1, void* ws, size_t ws_bytes, void* stream) {
   size_t need = 0;
   mobi_status st = check_gemm_grouped(problems, count, G, S, &need);
   if (st != MOBI_OK) return st;
@@ -554,13 +649,28 @@ mobi_status mobi_gemm_grouped_bits(const mobi_gemm_problem* problems, int count,
   uint8_t* w = static_cast<uint8_t*>(ws);
   for (int i = 0; i < count; ++i) {
     const mobi_gemm_problem& p = problems[i];
-    jobs[i] = DecodeJob{p.X, p.k_t, p.codes, p.sz, p.Y, nullptr, p.N, p.K, (int)p.T, bits};
+    jobs[i] = DecodeJob{p.X, p.k_t, p.codes, p.sz, p.Y, nullptr, p.N, p.K, (int)p.T, bits, mask1};
     if (p.T > 0 && p.N > 0) {
       jobs[i].partial = reinterpret_cast<float*>(w);
       w += align256(decode_ws_bytes(p.N, p.K));
     }
   }
   return cuda_status(launch_decode_grouped(jobs, count, S, static_cast<cudaStream_t>(stream), dst, false));
+}
+
+mobi_status mobi_gemm_grouped_bits(const mobi_gemm_problem* problems, int count, int G, int S, int bits, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  if (bits < 1 || bits > 2) return MOBI_ERR_INVALID_ARG;
+  return gemm_grouped_impl(problems, count, G, S, bits, uniform_mask(bits, S), ws, ws_bytes, stream);
+}
+
+mobi_status mobi_gemm_grouped_slices(const mobi_gemm_problem* problems, int count, int G, int S, const int* widths,
+                                     void* ws, size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  int mode = 0, mask1 = 0;
+  if (!width_mode(S, widths, &mode, &mask1)) return MOBI_ERR_INVALID_ARG;
+  return gemm_grouped_impl(problems, count, G, S, mode, mask1, ws, ws_bytes, stream);
 }
 
 mobi_status mobi_gemm(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,

@@ -118,16 +118,16 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r
 }
 
 // Issue one stage: the codes of 16-row tile `tile`, slice s, chunk `chunk`
-// (x = word column, y = s N + row) and its scale/zero words. 2-bit codes fill
-// two 2 KB halves (64 words per row and chunk), 1-bit codes one (32 words).
-template <int BITS>
+// (x = word column, y = the code map's row: s N + row when one map covers
+// every slice, the row alone with one map per slice) and its scale/zero
+// words. 2-bit codes fill two 2 KB halves (64 words per row and chunk), 1-bit
+// codes one (32 words).
 __device__ __forceinline__ void dec_issue(const CUtensorMap* tm_codes, const CUtensorMap* tm_sz, uint8_t* codes,
-                                          uint8_t* sz, uint64_t* bar, int tile, int s, int N, int ngroups,
-                                          int chunk, uint64_t policy) {
-  mbar_arrive_expect_tx(bar, kDecHalf * BITS + kDecSz);
-  const int y = s * N + tile * kDecRows;
-  tma_load_2d_hint(codes, tm_codes, chunk * kDecChunk * 4 * BITS, y, bar, policy);
-  if (BITS == 2) tma_load_2d_hint(codes + kDecHalf, tm_codes, chunk * kDecChunk * 8 + 32, y, bar, policy);
+                                          uint8_t* sz, uint64_t* bar, int y, int bits, int tile, int s,
+                                          int ngroups, int chunk, uint64_t policy) {
+  mbar_arrive_expect_tx(bar, kDecHalf * bits + kDecSz);
+  tma_load_2d_hint(codes, tm_codes, chunk * kDecChunk * 4 * bits, y, bar, policy);
+  if (bits == 2) tma_load_2d_hint(codes + kDecHalf, tm_codes, chunk * kDecChunk * 8 + 32, y, bar, policy);
   tma_load_2d_hint(sz, tm_sz, tile * kDecRows, s * ngroups + chunk * kDecChunk, bar, policy);
 }
 
@@ -157,12 +157,17 @@ struct DecProblem {
 };
 // MG = table capacity: 1 for a single call (a small parameter block to copy
 // per launch), kMaxGroup for a group.
-template <int MG>
+// BITS: 2 or 1 (every slice that wide, one code map per problem over all
+// slices) or 3 (slice widths given by mask1: bit s set = slice s is 1-bit;
+// one code map per slice).
+template <int MG, int BITS = 2>
 struct DecGroup {
-  CUtensorMap tm_codes[MG];
+  static constexpr int kMaps = BITS == 3 ? kMaxSlices : 1;
+  CUtensorMap tm_codes[MG][kMaps];
   CUtensorMap tm_sz[MG];
   DecProblem p[MG];
   int G, S;
+  int mask1;
 };
 
 // The cost terms of the work split, per problem: a tile of a full chunk costs
@@ -180,8 +185,8 @@ struct DecSplit {
 
 // Warp 0, one lane per problem. Every CTA computes the same terms (the same
 // integer operations on the same k_t), so no CTA waits for another.
-template <int MG>
-__device__ __forceinline__ void dec_split(const DecGroup<MG>& grp, int lane, DecSplit<MG>* sp) {
+template <int MG, int BITS>
+__device__ __forceinline__ void dec_split(const DecGroup<MG, BITS>& grp, int lane, DecSplit<MG>* sp) {
   const int G = MG > 1 ? grp.G : 1;
   long long w = 0;
   if (lane < G) {
@@ -231,6 +236,12 @@ __device__ __forceinline__ int dec_cut(int x, int km) {
   return 2 * o <= km - 1 ? x - o : x - o + km - 1;
 }
 
+// Code width of slice s (2 or 1 bits) for a launch of width mode BITS.
+template <int BITS>
+__device__ __forceinline__ int dec_width(int mask1, int s) {
+  return BITS == 3 ? (((mask1 >> s) & 1) ? 1 : 2) : BITS;
+}
+
 // Tile sums of one warp for 16 rows (gid, gid + 8) and the lane's tokens
 // 8 nb + 2 t4 + {0, 1}, written to o[t N + row] for tokens < T.
 template <int NB>
@@ -254,7 +265,7 @@ __device__ __forceinline__ void dec_write_tile(float* o, int T, int N, int gid, 
 // 2^28); positions in the cost sequence are 64-bit.
 template <int NB, int MG, int BITS>
 __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
-    const __grid_constant__ DecGroup<MG> grp, DeviceStatus* st, uint64_t limit) {
+    const __grid_constant__ DecGroup<MG, BITS> grp, DeviceStatus* st, uint64_t limit) {
   using L = DecLayout<NB>;
   constexpr int D = L::kDepth;
   constexpr int kDecWarps = L::kWarps;
@@ -328,13 +339,14 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
   // 128 bytes. 1-bit codes: word t4 of group g, 16-byte chunk g stored at
   // g ^ (r % 8); its even bits are the codes of 2-bit word 2 t4 and its odd
   // bits those of word 2 t4 + 1, so (w, w >> 1) take the place of that pair.
+  // With per-slice widths (BITS 3) coff holds the 2-bit offsets and the 1-bit
+  // ones are formed when needed.
   uint32_t coff[kDecChunk];
 #pragma unroll
   for (int g = 0; g < kDecChunk; ++g)
-    coff[g] = BITS == 2 ? (uint32_t)(g >> 2) * kDecHalf + (uint32_t)gid * 128u +
+    coff[g] = BITS != 1 ? (uint32_t)(g >> 2) * kDecHalf + (uint32_t)gid * 128u +
                               (uint32_t)((((g & 3) * 2 + (t4 >> 1)) ^ gid) * 16) + (t4 & 1) * 8u
                         : (uint32_t)gid * 128u + (uint32_t)((g ^ gid) * 16) + (uint32_t)t4 * 4u;
-  constexpr uint32_t kFieldMask = BITS == 2 ? 0x00030003u : 0x00010001u;
 
   bool ok = true;
   uint32_t issued = 0, done = 0;  // stages this warp has issued / consumed (ring slot = count % D)
@@ -396,8 +408,11 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
           for (int k = 0; k < nramp; ++k) {
             const uint32_t slot = (issued + k) % D;
             const int jj = a + k;
-            dec_issue<BITS>(&grp.tm_codes[p], &grp.tm_sz[p], codes_ring + slot * kDecCodes, sz_ring + slot * kDecSz,
-                      &full[slot], b + jj / km, jj % km, pr.N, pr.ngroups, c, policy);
+            const int tt = b + jj / km, ss = jj % km;
+            const int bw = dec_width<BITS>(grp.mask1, ss);
+            dec_issue(&grp.tm_codes[p][BITS == 3 ? ss : 0], &grp.tm_sz[p], codes_ring + slot * kDecCodes,
+                      sz_ring + slot * kDecSz, &full[slot], (BITS == 3 ? 0 : ss * pr.N) + tt * kDecRows, bw, tt, ss,
+                      pr.ngroups, c, policy);
           }
         }
         if (ok) issued += nramp;
@@ -498,7 +513,6 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
     }
 
     float* const out = prob.out + (int64_t)c * T * N;
-    const CUtensorMap* tm_codes = &grp.tm_codes[p];
     const CUtensorMap* tm_sz = &grp.tm_sz[p];
     int s = a % km, tile = b + a / km;  // consumer cursor
     bool head = s != 0;                 // the first tile's other slices are the previous warp's
@@ -515,8 +529,9 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
       if (pj < a1) {
         const uint32_t ns = issued % D;
         if (lane == 0)
-          dec_issue<BITS>(tm_codes, tm_sz, codes_ring + ns * kDecCodes, sz_ring + ns * kDecSz, &full[ns], ptile,
-                          ps, N, ngroups, c, policy);
+          dec_issue(&grp.tm_codes[p][BITS == 3 ? ps : 0], tm_sz, codes_ring + ns * kDecCodes,
+                    sz_ring + ns * kDecSz, &full[ns], (BITS == 3 ? 0 : ps * N) + ptile * kDecRows,
+                    dec_width<BITS>(grp.mask1, ps), ptile, ps, ngroups, c, policy);
         ++issued;
         ++pj;
         if (++ps == km) {
@@ -530,6 +545,8 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
       }
       ++done;
       const uint8_t* cs = codes_ring + slot * kDecCodes;
+      const bool w1 = dec_width<BITS>(grp.mask1, s) == 1;  // this stage's codes are 1-bit
+      const uint32_t kFieldMask = w1 ? 0x00010001u : 0x00030003u;
       // Scale/zero words of the stage as fp32 pairs (scale 2^37, -scale zero),
       // one conversion per word for the whole warp.
       {
@@ -555,12 +572,14 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
         uint32_t bf[2][NB][kJitB ? 2 : 8][2];
 #pragma unroll
         for (int gg = 0; gg < 2; ++gg) {
-          if (BITS == 2) {
+          if (!w1) {
             wa[gg] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg]);
             wb[gg] = *reinterpret_cast<const uint2*>(cs + coff[g0 + gg] + 8 * 128);
           } else {
-            const uint32_t x = *reinterpret_cast<const uint32_t*>(cs + coff[g0 + gg]);
-            const uint32_t y = *reinterpret_cast<const uint32_t*>(cs + coff[g0 + gg] + 8 * 128);
+            const uint32_t o1 = BITS == 1 ? coff[g0 + gg]
+                                          : (uint32_t)gid * 128u + (uint32_t)(((g0 + gg) ^ gid) * 16) + (uint32_t)t4 * 4u;
+            const uint32_t x = *reinterpret_cast<const uint32_t*>(cs + o1);
+            const uint32_t y = *reinterpret_cast<const uint32_t*>(cs + o1 + 8 * 128);
             wa[gg] = make_uint2(x, x >> 1);
             wb[gg] = make_uint2(y, y >> 1);
           }
@@ -716,7 +735,8 @@ size_t decode_ws_bytes(int64_t N, int64_t K) {
 }
 
 template <int NB, int MG, int BITS>
-static cudaError_t launch_decode_class(const DecGroup<MG>& grp, int ctas, cudaStream_t stream, DeviceStatus* st) {
+static cudaError_t launch_decode_class(const DecGroup<MG, BITS>& grp, int ctas, cudaStream_t stream,
+                                       DeviceStatus* st) {
   using L = DecLayout<NB>;
   cudaError_t e = set_smem((const void*)decode_kernel<NB, MG, BITS>, (int)L::kDynamic);
   if (e != cudaSuccess) return e;
@@ -742,16 +762,28 @@ static cudaError_t launch_decode_class(const DecGroup<MG>& grp, int ctas, cudaSt
 template <int MG, int BITS>
 static cudaError_t decode_class(const DecodeJob* jobs, const int* idx, int n, int cls, int S, int sms,
                                 DecReduceGroup* red, cudaStream_t stream, DeviceStatus* st) {
-  DecGroup<MG> grp;
+  DecGroup<MG, BITS> grp;
   memset(&grp, 0, sizeof grp);
   grp.G = n;
   grp.S = S;
+  grp.mask1 = n > 0 ? jobs[idx[0]].mask1 : 0;
   for (int m = 0; m < n; ++m) {
     const DecodeJob& j = jobs[idx[m]];
     const int64_t nch = dec_chunks(j.K), nblocks = (j.N + kDecRows - 1) / kDecRows;
-    const uint64_t words = (uint64_t)(j.K / 32 * BITS);  // per row and slice
-    if (!make_tmap_2d(&grp.tm_codes[m], j.codes, 4, words, (uint64_t)(S * j.N), words * 4, 32, kDecRows, 128))
-      return note_error("decode tensor map (codes)", cudaErrorInvalidValue);
+    if (BITS != 3) {
+      const uint64_t words = (uint64_t)(j.K / 32 * BITS);  // per row and slice
+      if (!make_tmap_2d(&grp.tm_codes[m][0], j.codes, 4, words, (uint64_t)(S * j.N), words * 4, 32, kDecRows, 128))
+        return note_error("decode tensor map (codes)", cudaErrorInvalidValue);
+    } else {  // one map per slice: slice s starts after the words of slices 0 .. s-1
+      const uint32_t* base = j.codes;
+      for (int sl = 0; sl < S; ++sl) {
+        const int w = ((j.mask1 >> sl) & 1) ? 1 : 2;
+        const uint64_t words = (uint64_t)(j.K / 32 * w);
+        if (!make_tmap_2d(&grp.tm_codes[m][sl], base, 4, words, (uint64_t)j.N, words * 4, 32, kDecRows, 128))
+          return note_error("decode tensor map (codes of a slice)", cudaErrorInvalidValue);
+        base += (size_t)j.N * words;
+      }
+    }
     if (!make_tmap_2d(&grp.tm_sz[m], j.sz, 4, (uint64_t)j.N, (uint64_t)(S * (j.K / 128)), (uint64_t)j.N * 4,
                       kDecRows, kDecChunk, 0))
       return note_error("decode tensor map (scale/zero)", cudaErrorInvalidValue);
@@ -783,7 +815,7 @@ cudaError_t launch_decode_grouped(const DecodeJob* jobs, int G, int S, cudaStrea
   DecReduceGroup red = {};
   red.off[0] = 0;
   for (int cls = 1; cls <= 2; ++cls)
-    for (int bits = 2; bits >= 1; --bits) {
+    for (int bits = 3; bits >= 1; --bits) {
       int idx[kMaxGroup];
       int n = 0;
       for (int i = 0; i < G; ++i) {
@@ -795,9 +827,12 @@ cudaError_t launch_decode_grouped(const DecodeJob* jobs, int G, int S, cudaStrea
       if (bits == 2)
         e = n == 1 ? decode_class<1, 2>(jobs, idx, n, cls, S, sms, &red, stream, st)
                    : decode_class<kMaxGroup, 2>(jobs, idx, n, cls, S, sms, &red, stream, st);
-      else
+      else if (bits == 1)
         e = n == 1 ? decode_class<1, 1>(jobs, idx, n, cls, S, sms, &red, stream, st)
                    : decode_class<kMaxGroup, 1>(jobs, idx, n, cls, S, sms, &red, stream, st);
+      else
+        e = n == 1 ? decode_class<1, 3>(jobs, idx, n, cls, S, sms, &red, stream, st)
+                   : decode_class<kMaxGroup, 3>(jobs, idx, n, cls, S, sms, &red, stream, st);
       if (e != cudaSuccess) return e;
     }
   if (red.G == 0) return cudaSuccess;
@@ -850,8 +885,8 @@ cudaError_t launch_chunk_reduce(const float* partial, float* Y, int64_t T, int64
 
 cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
                           const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
-                          DeviceStatus* st, bool early, int bits) {
-  const DecodeJob job{X, k_t, codes, sz, Y, static_cast<float*>(ws), N, K, T, bits};
+                          DeviceStatus* st, bool early, int bits, int mask1) {
+  const DecodeJob job{X, k_t, codes, sz, Y, static_cast<float*>(ws), N, K, T, bits, mask1};
   return launch_decode_grouped(&job, 1, S, stream, st, early);
 }
 
@@ -924,5 +959,6 @@ extern "C" mobi_status mobi_gemm_decode_noalloc(const void* X, int64_t T, int64_
   void* scratch = noalloc_scratch(&e);
   if (!scratch) return status_of(e);
   return status_of(
-      launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, scratch, static_cast<cudaStream_t>(stream), st, false, 2));
+      launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, scratch, static_cast<cudaStream_t>(stream), st, false, 2,
+                    0));
 }

@@ -74,7 +74,8 @@ struct DecodeJob {
   float* partial;  // scratch of decode_ws_bytes(N, K) bytes
   int64_t N, K;
   int T;
-  int bits;  // code width of every slice: 2 (16 codes per word) or 1 (32 per word)
+  int bits;   // 2 or 1: every slice that wide (16 or 32 codes per word); 3: widths per slice (mask1)
+  int mask1;  // bits == 3: bit s set = slice s has 1-bit codes; the slices are stored one after another
 };
 // Decode scratch of one problem: the per-chunk partial sums when K spans more
 // than one 1024-column chunk.

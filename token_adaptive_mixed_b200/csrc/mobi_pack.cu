@@ -3,8 +3,8 @@
 // MoBiQuant explainer [ja] §2.1 / [en] §2.A: R_1 = W, W_s = Q(R_s),
 // R_{s+1} = R_s - W_s, with Q the asymmetric min-max round-to-nearest of each
 // G-wide group (the quantiser written out in include/mobi.h): b-bit codes,
-// L = 2^b - 1 steps (b = 2 for the method's slices, b = 1 for generic ones),
-// G = 128, 256 or 512.
+// L = 2^b - 1 steps (b = 2 for the method's slices, b = 1 for generic ones,
+// one width per slice), G = 128, 256 or 512.
 //
 // Work split: one warp per (row n, chunk of 512 columns); lane l owns the 16
 // consecutive weights k = 512c + 16l .. +15, i.e. exactly one 2-bit-field
@@ -27,10 +27,11 @@
 
 namespace mobi {
 
+// Slice s has 1-bit codes when bit s of mask1 is set, 2-bit codes otherwise;
+// the slices are stored one after another, each in the layout of its width.
 __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W, int64_t N, int64_t K,
-                                                   int S, int bits, int glanes, uint32_t* __restrict__ codes,
+                                                   int S, int mask1, int glanes, uint32_t* __restrict__ codes,
                                                    uint32_t* __restrict__ sz) {
-  const float L = (float)((1 << bits) - 1);  // steps between min and max
   const int lane = threadIdx.x & 31;
   const int64_t ngroups = K / 128;
   const int64_t nchunks = (ngroups + 3) / 4;
@@ -62,7 +63,10 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
       for (int i = 0; i < 16; ++i) R[i] = 0.0f;
     }
 
+    int64_t slice_base = 0;  // word offset of slice s
     for (int s = 0; s < S; ++s) {
+      const int bits = ((mask1 >> s) & 1) ? 1 : 2;
+      const float L = (float)((1 << bits) - 1);  // steps between min and max
       float mn = R[0], mx = R[0];
 #pragma unroll
       for (int i = 1; i < 16; ++i) {
@@ -100,7 +104,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
         const uint32_t d2 = __shfl_down_sync(0xffffffffu, dense, 4);
         const uint32_t d3 = __shfl_down_sync(0xffffffffu, dense, 6);
         if (valid && (lane & 7) == 0) {
-          uint4* dst = reinterpret_cast<uint4*>(codes + ((int64_t)s * N + n) * (K / 32) + 16 * c + (lane >> 1));
+          uint4* dst = reinterpret_cast<uint4*>(codes + slice_base + n * (K / 32) + 16 * c + (lane >> 1));
           *dst = make_uint4(dense, d1, d2, d3);
         }
       } else {
@@ -109,7 +113,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
         const uint32_t w2 = __shfl_down_sync(0xffffffffu, word, 2);
         const uint32_t w3 = __shfl_down_sync(0xffffffffu, word, 3);
         if (valid && (lane & 3) == 0) {
-          uint4* dst = reinterpret_cast<uint4*>(codes + ((int64_t)s * N + n) * nwords + 32 * c + lane);
+          uint4* dst = reinterpret_cast<uint4*>(codes + slice_base + n * nwords + 32 * c + lane);
           *dst = make_uint4(word, w1, w2, w3);
         }
       }
@@ -117,12 +121,13 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
         const uint32_t zbits = (uint32_t)__half_as_ushort(__int2half_rn(z));
         sz[((int64_t)s * ngroups + g) * N + n] = (uint32_t)__half_as_ushort(scale_h) | (zbits << 16);
       }
+      slice_base += N * (K / 32) * bits;
     }
   }
 }
 
 cudaError_t launch_pack(const void* W, int64_t N, int64_t K, int S, uint32_t* codes, uint32_t* sz,
-                        cudaStream_t stream, int num_sms, int bits, int G) {
+                        cudaStream_t stream, int num_sms, int mask1, int G) {
   const int64_t nchunks = (K / 128 + 3) / 4;
   const int64_t units = N * nchunks;
   const int warps_per_block = 8;
@@ -131,7 +136,7 @@ cudaError_t launch_pack(const void* W, int64_t N, int64_t K, int S, uint32_t* co
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   pack_kernel<<<(unsigned)blocks, 32 * warps_per_block, 0, stream>>>(
-      static_cast<const __half*>(W), N, K, S, bits, G / 16, codes, sz);
+      static_cast<const __half*>(W), N, K, S, mask1, G / 16, codes, sz);
   return note_error("kernel launch", cudaGetLastError());
 }
 

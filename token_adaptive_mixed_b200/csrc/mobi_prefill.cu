@@ -40,6 +40,7 @@
 // stops issuing, drains its copies and MMAs in flight, frees TMEM and returns.
 #include <cstdint>
 #include <cstdio>
+#include <cstring>
 
 #include "mobi_device.cuh"
 #include "mobi_host.h"
@@ -78,6 +79,15 @@ struct Tile {
   static_assert(kColsPerEpi % kChunkCols == 0 && kChunkCols % 16 == 0, "epilogue chunks");
 };
 }  // namespace pf
+
+// Code maps of the packed slices: one map over every slice (per_slice 0, row
+// s N + n) or one per slice (per_slice 1, row n); slice s has 1-bit codes when
+// bit s of mask1 is set, 2-bit codes otherwise.
+struct PfCodeMaps {
+  CUtensorMap m[kMaxSlices];
+  int per_slice;
+  int mask1;
+};
 
 template <int BN>
 struct PfSmem {
@@ -171,9 +181,9 @@ __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, uint64_t
 // of its registers.
 template <int BN, bool KSPLIT>
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
-    const uint8_t* __restrict__ Xt, const __grid_constant__ CUtensorMap tm_codes,
+    const uint8_t* __restrict__ Xt, const __grid_constant__ PfCodeMaps tm_codes,
     const __grid_constant__ CUtensorMap tm_sz, const uint32_t* __restrict__ sz, const int32_t* __restrict__ perm,
-    const int32_t* __restrict__ offsets, int64_t T, int64_t N, int64_t ngroups, int S, int nkc, int bits,
+    const int32_t* __restrict__ offsets, int64_t T, int64_t N, int64_t ngroups, int S, int nkc,
     float* __restrict__ Y, DeviceStatus* st, uint64_t limit) {
   using TL = pf::Tile<BN>;
   if constexpr (!KSPLIT) nkc = 1;
@@ -216,7 +226,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
    if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      prefetch_tmap(&tm_codes); prefetch_tmap(&tm_sz);
+      for (int j = 0; j < (tm_codes.per_slice ? S : 1); ++j) prefetch_tmap(&tm_codes.m[j]);
+      prefetch_tmap(&tm_sz);
       uint32_t xi = 0, ci = 0;  // running stage counters
       bool ok = true;
       for (int64_t i = 0, tile; (tile = pf_tile(i, ntiles, n_wt, n_tt, nkc)) >= 0 && ok; ++i) {
@@ -233,8 +244,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
           for (int s = 0; s < ti.kmax; ++s) {
             const uint32_t cs = ci % pf::CST, cph = (ci / pf::CST) & 1;
             if (!(ok = pf_wait(&sm.c_empty[cs], cph ^ 1, limit, st, 0x302, abort_flag))) break;
+            const int bits = ((tm_codes.mask1 >> s) & 1) ? 1 : 2;
             mbar_arrive_expect_tx(&sm.c_full[cs], pf::kCodeBytes / 2 * bits + pf::kSzBytes);
-            tma_load_2d(&sm.codes[cs][0], &tm_codes, (int)(g * 4 * bits), (int)(s * N + ti.n0), &sm.c_full[cs]);
+            tma_load_2d(&sm.codes[cs][0], &tm_codes.m[tm_codes.per_slice ? s : 0], (int)(g * 4 * bits),
+                        (int)((tm_codes.per_slice ? 0 : s * N) + ti.n0), &sm.c_full[cs]);
             tma_load_2d(&sm.sz[cs][0], &tm_sz, (int)ti.n0, (int)(s * ngroups + g), &sm.c_full[cs]);
             ++ci;
           }
@@ -318,6 +331,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(
           // The group's 128 codes of row r as eight 2-bit-field words: 2-bit
           // codes as stored; 1-bit codes (4 words) as (w, w >> 1) pairs, whose
           // even bits are the codes of the 2-bit words 2i and 2i + 1.
+          const int bits = ((tm_codes.mask1 >> s) & 1) ? 1 : 2;
           uint32_t words[8];
           if (bits == 2) {
             const uint4 w0 = *reinterpret_cast<const uint4*>(&sm.codes[cs][r * 8]);
@@ -558,8 +572,8 @@ size_t prefill_ws_bytes(int64_t T, int64_t N, int64_t K) {
 
 template <int BN, bool KSPLIT>
 static cudaError_t launch_prefill_bn(const PfPlan& plan, const void* X, int64_t T, int64_t K, const int32_t* perm,
-                                     const int32_t* offsets, const CUtensorMap& tm_codes, const CUtensorMap& tm_sz,
-                                     const uint32_t* sz, int64_t N, int S, int bits, float* out, uint8_t* Xt,
+                                     const int32_t* offsets, const PfCodeMaps& tm_codes, const CUtensorMap& tm_sz,
+                                     const uint32_t* sz, int64_t N, int S, float* out, uint8_t* Xt,
                                      cudaStream_t stream, DeviceStatus* st) {
   const int64_t ngroups = K / 128;
   const int64_t blocks_g = (plan.T_pad * (K / 16) + 255) / 256;
@@ -572,7 +586,7 @@ static cudaError_t launch_prefill_bn(const PfPlan& plan, const void* X, int64_t 
   cudaError_t e = set_smem((const void*)kernel, (int)smem);
   if (e != cudaSuccess) return e;
   kernel<<<grid, pf::kThreads, smem, stream>>>(Xt, tm_codes, tm_sz, sz, perm, offsets, T, N, ngroups, S, plan.nkc,
-                                               bits, out, st, wait_limit());
+                                               out, st, wait_limit());
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     cudaFuncAttributes fa{};
@@ -587,26 +601,44 @@ static cudaError_t launch_prefill_bn(const PfPlan& plan, const void* X, int64_t 
 
 cudaError_t launch_prefill(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
                            const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int S,
-                           float* Y, void* ws, cudaStream_t stream, DeviceStatus* st, int bits) {
+                           float* Y, void* ws, cudaStream_t stream, DeviceStatus* st, int bits, int mask1) {
   (void)k_t;
   const int64_t ngroups = K / 128;
   const PfPlan plan = pf_plan(T, N, K, num_sms());
   uint8_t* Xt = static_cast<uint8_t*>(ws);
   float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + plan.xt_bytes);
   float* out = plan.nkc > 1 ? partial : Y;
-  CUtensorMap tm_codes, tm_sz;
-  const uint64_t words = (uint64_t)(K / 32 * bits);  // per row and slice
-  if (!make_tmap_2d(&tm_codes, codes, 4, words, (uint64_t)(S * N), words * 4, (uint32_t)(4 * bits), pf::BM, 0))
-    return cudaErrorInvalidValue;
+  PfCodeMaps tm_codes;
+  memset(&tm_codes, 0, sizeof tm_codes);
+  CUtensorMap tm_sz;
+  if (bits != 3) {  // every slice the same width: one map over all slices
+    tm_codes.per_slice = 0;
+    tm_codes.mask1 = bits == 1 ? (1 << S) - 1 : 0;
+    const uint64_t words = (uint64_t)(K / 32 * bits);  // per row and slice
+    if (!make_tmap_2d(&tm_codes.m[0], codes, 4, words, (uint64_t)(S * N), words * 4, (uint32_t)(4 * bits), pf::BM,
+                      0))
+      return cudaErrorInvalidValue;
+  } else {  // one map per slice: slice s starts after the words of slices 0 .. s-1
+    tm_codes.per_slice = 1;
+    tm_codes.mask1 = mask1;
+    const uint32_t* base = codes;
+    for (int sl = 0; sl < S; ++sl) {
+      const int w = ((mask1 >> sl) & 1) ? 1 : 2;
+      const uint64_t words = (uint64_t)(K / 32 * w);
+      if (!make_tmap_2d(&tm_codes.m[sl], base, 4, words, (uint64_t)N, words * 4, (uint32_t)(4 * w), pf::BM, 0))
+        return cudaErrorInvalidValue;
+      base += (size_t)N * words;
+    }
+  }
   if (!make_tmap_2d(&tm_sz, sz, 4, (uint64_t)N, (uint64_t)(S * ngroups), (uint64_t)N * 4, pf::BM, 1, 0))
     return cudaErrorInvalidValue;
   cudaError_t e;
   if (plan.bn == 64)
-    e = launch_prefill_bn<64, true>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, bits, out, Xt, stream, st);
+    e = launch_prefill_bn<64, true>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, out, Xt, stream, st);
   else if (plan.nkc > 1)
-    e = launch_prefill_bn<192, true>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, bits, out, Xt, stream, st);
+    e = launch_prefill_bn<192, true>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, out, Xt, stream, st);
   else
-    e = launch_prefill_bn<192, false>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, bits, out, Xt, stream, st);
+    e = launch_prefill_bn<192, false>(plan, X, T, K, perm, offsets, tm_codes, tm_sz, sz, N, S, out, Xt, stream, st);
   if (e != cudaSuccess || plan.nkc <= 1) return e;
   return launch_chunk_reduce(partial, Y, T, N, plan.nkc, stream);
 }
