@@ -24,7 +24,9 @@
  *                        in one step (mobi_gemm_grouped: the GEMM half).
  *   mobi_route_mlp       threshold routing with a two-layer MLP scorer
  *                        ([ja] §2.2; [en] §2.B "Differentiable Gating").
- *   mobi_pack_bits       generic slicing: 1- or 2-bit slices, wider groups.
+ *   mobi_pack_bits       generic slicing: 1- or 2-bit slices, wider groups
+ *                        (mobi_pack_slices: one width per slice); the GEMM
+ *                        entry points' _bits / _slices forms read them.
  *   mobi_ckpt_*          many-in-one checkpoints of packed layers.
  *   mobi_gemm_path, mobi_gemm_decode_noalloc, mobi_sync_check and the size
  *   and status helpers.

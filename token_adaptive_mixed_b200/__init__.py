@@ -7,14 +7,15 @@ library's sm_100a kernels. There is no CPU fallback: if the library is missing
 or a tensor is not on a CUDA device, the call raises (the checkpoint calls,
 which move bytes between a file and memory, also take host tensors).
 
-Entry points (same names as the C ABI):
-  mobi_pack(W, S, G, bits)          MoBiSlice packing   -> (codes, sz)
+Entry points (same names as the C ABI; `bits=` selects the *_bits form and
+`widths=` the *_slices form of a call):
+  mobi_pack(W, S, G, bits, widths)  MoBiSlice packing   -> (codes, sz)
   mobi_route(X, Wr, bias)           MoBiRoute routing   -> (k_t, perm, offsets)
   mobi_route_mlp(X, W1, b1, W2, b2, tau, delta)  threshold routing, MLP scorer -> (k_t, perm, offsets)
   mobi_gemm(X, k_t, perm, offsets, codes, sz, N)         -> Y  (fp32)
   mobi_gemm_path(..., path)         the same with a forced kernel
   mobi_linear(X, Wr, bias, codes, sz, N)  route + GEMM in one call -> (Y, k_t, perm, offsets)
-  mobi_linear_grouped(problems)     up to 8 decode-sized mobi_linear problems in one step
+  mobi_linear_grouped(problems)     up to 16 decode-sized mobi_linear problems in one step
   mobi_gemm_grouped(problems)       the GEMM half of it (k_t given)
   mobi_ckpt_save / MobiCheckpoint   many-in-one checkpoint of packed layers (load any slice count)
   mobi_sync_check()                 sync + device-side error word
