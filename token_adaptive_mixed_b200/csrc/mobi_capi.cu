@@ -29,7 +29,7 @@ cudaError_t launch_route_mlp(const void* X, int64_t T, int64_t K, const float* W
 size_t route_mlp_ws_bytes(int64_t T, int64_t K, int64_t H, int sms);
 cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
                           const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
-                          DeviceStatus* st, bool early, int bits, int mask1);
+                          DeviceStatus* st, int bits, int mask1);
 size_t decode_ws_bytes(int64_t N, int64_t K);
 cudaError_t launch_prefill(const void* X, int64_t T, int64_t K, const int32_t* k_t, const int32_t* perm,
                            const int32_t* offsets, const uint32_t* codes, const uint32_t* sz, int64_t N, int S,
@@ -436,7 +436,7 @@ static mobi_status gemm_impl(const void* X, int64_t T, int64_t K, const int32_t*
   if (!dst) return cuda_status(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (decode)
-    return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, ws, s, dst, false, bits, mask1));
+    return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, ws, s, dst, bits, mask1));
   return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, ws, s, dst, bits, mask1));
 }
 
@@ -499,7 +499,7 @@ static mobi_status linear_impl(const void* X, int64_t T, int64_t K, const float*
   // For up to 16 tokens the decode kernel is a programmatic dependent of the
   // routing kernel just launched: its launch and set-up overlap the routing.
   if (decode)
-    return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, gws, s, dst, true, bits, mask1));
+    return cuda_status(launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, gws, s, dst, bits, mask1));
   return cuda_status(launch_prefill(X, T, K, k_t, perm, offsets, codes, sz, N, S, Y, gws, s, dst, bits, mask1));
 }
 
@@ -587,7 +587,7 @@ static mobi_status linear_grouped_impl(const mobi_linear_problem* problems, int 
   if (e != cudaSuccess) return cuda_status(e);
   // As in mobi_linear: the decode launches are programmatic dependents of the
   // routing launch.
-  return cuda_status(launch_decode_grouped(jobs, count, S, s, dst, true));
+  return cuda_status(launch_decode_grouped(jobs, count, S, s, dst));
 }
 
 mobi_status mobi_linear_grouped_bits(const mobi_linear_problem* problems, int count, int G, int S, int bits,
@@ -655,7 +655,7 @@ static mobi_status gemm_grouped_impl(const mobi_gemm_problem* problems, int coun
       w += align256(decode_ws_bytes(p.N, p.K));
     }
   }
-  return cuda_status(launch_decode_grouped(jobs, count, S, static_cast<cudaStream_t>(stream), dst, false));
+  return cuda_status(launch_decode_grouped(jobs, count, S, static_cast<cudaStream_t>(stream), dst));
 }
 
 mobi_status mobi_gemm_grouped_bits(const mobi_gemm_problem* problems, int count, int G, int S, int bits, void* ws,

@@ -805,12 +805,9 @@ static cudaError_t decode_class(const DecodeJob* jobs, const int* idx, int n, in
 // persistent grid of one CTA per SM that the kernel shares among that class's
 // problems in equal parts of the slices they read, then one chunk-reduction launch for
 // every problem with more than one chunk. Each launch is a programmatic
-// dependent of the one before. `early` (the kernel before is this library's
-// routing kernel) no longer changes anything: the decode kernel needs k_t
-// before it can choose its work, so it always waits first.
-cudaError_t launch_decode_grouped(const DecodeJob* jobs, int G, int S, cudaStream_t stream, DeviceStatus* st,
-                                  bool early) {
-  (void)early;
+// dependent of the one before (the decode kernel reads k_t, which decides its
+// work split, only after the kernel before has finished).
+cudaError_t launch_decode_grouped(const DecodeJob* jobs, int G, int S, cudaStream_t stream, DeviceStatus* st) {
   const int sms = num_sms();
   DecReduceGroup red = {};
   red.off[0] = 0;
@@ -885,9 +882,9 @@ cudaError_t launch_chunk_reduce(const float* partial, float* Y, int64_t T, int64
 
 cudaError_t launch_decode(const void* X, int T, int64_t K, const int32_t* k_t, const uint32_t* codes,
                           const uint32_t* sz, int64_t N, int S, float* Y, void* ws, cudaStream_t stream,
-                          DeviceStatus* st, bool early, int bits, int mask1) {
+                          DeviceStatus* st, int bits, int mask1) {
   const DecodeJob job{X, k_t, codes, sz, Y, static_cast<float*>(ws), N, K, T, bits, mask1};
-  return launch_decode_grouped(&job, 1, S, stream, st, early);
+  return launch_decode_grouped(&job, 1, S, stream, st);
 }
 
 }  // namespace mobi
@@ -959,6 +956,6 @@ extern "C" mobi_status mobi_gemm_decode_noalloc(const void* X, int64_t T, int64_
   void* scratch = noalloc_scratch(&e);
   if (!scratch) return status_of(e);
   return status_of(
-      launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, scratch, static_cast<cudaStream_t>(stream), st, false, 2,
+      launch_decode(X, (int)T, K, k_t, codes, sz, N, S, Y, scratch, static_cast<cudaStream_t>(stream), st, 2,
                     0));
 }

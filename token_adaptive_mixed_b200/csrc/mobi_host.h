@@ -85,7 +85,6 @@ size_t decode_ws_bytes(int64_t N, int64_t K);
 cudaError_t launch_chunk_reduce(const float* partial, float* Y, int64_t T, int64_t N, int nch, cudaStream_t stream);
 // Decode GEMMs of up to kMaxGroup problems: one launch per fragment class
 // (T <= 8, T <= 16) and code width present, plus one chunk-reduction launch.
-cudaError_t launch_decode_grouped(const DecodeJob* jobs, int G, int S, cudaStream_t stream, DeviceStatus* st,
-                                  bool early);
+cudaError_t launch_decode_grouped(const DecodeJob* jobs, int G, int S, cudaStream_t stream, DeviceStatus* st);
 
 }  // namespace mobi

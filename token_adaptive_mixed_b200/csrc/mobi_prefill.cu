@@ -21,7 +21,10 @@
 //     With w the packed word, ((w >> sh) & (0x00030003 << 2f)) | 0x43004300 is
 //     the bf16 pair (128 + 4^f q); one bf16x2 FMA by 4^-f minus (128 / 4^f + z)
 //     gives q - z exactly, so each pair costs one logic op and one FMA (plus a
-//     shift shared by three pairs).
+//     shift shared by three pairs). A 1-bit word w (32 codes) is read as the
+//     2-bit-field pair (w, w >> 1) with the masks 0x00010001 << 2f: its even
+//     bits are the codes of one 16-code block, its odd bits the next. Each
+//     slice may have its own width (one code map per slice).
 //   B (tokens) comes from shared memory: one bulk copy per group brings a
 //     192-token x tile that the gather kernel has already laid out as the
 //     128-byte-swizzled shared-memory image (rows in bucket order and, within
