@@ -546,7 +546,7 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
       ++done;
       const uint8_t* cs = codes_ring + slot * kDecCodes;
       const bool w1 = dec_width<BITS>(grp.mask1, s) == 1;  // this stage's codes are 1-bit
-      const uint32_t kFieldMask = w1 ? 0x00010001u : 0x00030003u;
+      const uint32_t field_mask = w1 ? 0x00010001u : 0x00030003u;
       // Scale/zero words of the stage as fp32 pairs (scale 2^37, -scale zero),
       // one conversion per word for the whole warp.
       {
@@ -596,7 +596,7 @@ __global__ void __launch_bounds__(DecLayout<NB>::kThreads, 1) decode_kernel(
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           const int h = jj >> 2, f = jj & 3;
-          const uint32_t mk = kFieldMask << (2 * f);
+          const uint32_t mk = field_mask << (2 * f);
           const int jb = kJitB ? (jj & 1) : jj;  // the step's slot in bf
           if constexpr (kJitB) {
             if ((jj & 1) == 0) {
